@@ -1,0 +1,515 @@
+"""Benchmark of the differentiable tile rasterizer (one JSON line on rank 0).
+
+Default workload: 1M-Gaussian 64-cluster mixture (SH degree 3) seen from a batch
+of 16 camera poses at 1920x1080; one step (iteration) = for every view
+project -> bin/sort -> raster forward -> L1 loss -> raster backward ->
+project backward (with the densification statistic), then one Adam update of
+all five parameter groups.  Metric: iterations/s (fwd+bwd), plus the step's
+algorithmic HBM bytes against the measured copy bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload multiview|mixture|box|city|tiny]
+
+--impl reference times the CPU oracle (the plain double-precision per-pixel
+renderer the tests use as ground truth) on a bounded sample of the same
+workload.  With N > 1 every rank runs an independent replica (the path has no
+exchange step); the reported value is the sum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "fwd+bwd iterations/s and HBM GB/s vs roofline at 1M Gaussians, 1920x1080"
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
+# FP32 lanes per SM and SMs of a B200; the ALU roofline uses the max SM clock
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+# float32 operations per (pixel, list entry) pair, counted from the kernels'
+# arithmetic with an FMA as two: alpha evaluation (dx, dy, quadratic form,
+# exponent, clamp, threshold tests) = 14; forward blend = 8; backward
+# transmittance recovery, colour/alpha gradients and the chain to
+# (u, v, A, B, C, o) = 46.
+FLOPS_ALPHA = 14
+FLOPS_FWD_BLEND = 8
+FLOPS_BWD_GRAD = 46
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(PEAK_FALLBACK)
+
+
+# --------------------------------------------------------------------- workloads
+
+def make_workload(name: str):
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    if name == "multiview":
+        return scenes.multiview1m(views=16)
+    if name == "mixture":
+        return scenes.mixture1m()
+    if name == "box":
+        wl = scenes.box100k(poses=16)
+        return wl
+    if name == "city":
+        return scenes.city3m(poses=4)
+    if name == "tiny":
+        wl = scenes.tiny()
+        wl.targets = [np.full((128, 128, 3), 0.5, np.float32)]
+        return wl
+    raise ValueError(name)
+
+
+def step_bytes(n, sh_degree, views_stats, tiles, pixels):
+    """Algorithmic HBM bytes of one step: per view, the sum of the stage terms,
+    then Adam over the 59 floats (SH degree 3) per Gaussian."""
+    pb = 4 * (11 + 3 * (sh_degree + 1) ** 2)
+    total = 0
+    for (K, V, passes) in views_stats:
+        total += n * (pb + 52)                 # project
+        total += n * 24 + K * 12               # count/scan + emit
+        total += K * (8 + 24 * passes)         # radix sort
+        total += K * 8 + tiles * 8             # tile ranges
+        total += K * 4 + V * 36 + pixels * 20  # raster forward
+        total += pixels * 36                   # L1 + dL/dimage
+        total += K * 4 + V * 108 + pixels * 20  # raster backward
+        total += n * (pb + 36 + 2 * pb + 8)    # project backward: params, grad2d, grads (+=), densify
+    total += n * pb // 4 * 28                  # Adam: param, m, v read+write, grad read
+    return total
+
+
+# ----------------------------------------------------------------- clock sampling
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-i", str(device_index), "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Largest value over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- reference arm
+
+def cpu_oracle_sample(wl, fraction: float, seed: int = 0):
+    """Time the oracle on a bounded sample of one view of the workload and scale
+    to one iteration.  Returns (seconds per iteration, threads, description)."""
+    import oracle
+    threads = oracle.set_threads(0)
+    rng = np.random.default_rng(seed)
+    scene, cam = wl.scene, wl.cameras[0]
+    n = scene.n
+    W, H = cam["width"], cam["height"]
+    tx, ty = (W + 15) // 16, (H + 15) // 16
+    ntiles = max(1, int(round(fraction * tx * ty)))
+    tiles = rng.choice(tx * ty, ntiles, replace=False)
+    pix = np.concatenate([[(t // tx) * 16 * W + (t % tx) * 16 + yy * W + xx for yy in range(16) for xx in range(16)
+                           if (t // tx) * 16 + yy < H and (t % tx) * 16 + xx < W] for t in tiles]).astype(np.int64)
+    gidx = np.sort(rng.choice(n, max(1, int(round(fraction * n))), replace=False))
+    t0 = time.perf_counter()
+    proj = oracle.project(scene, cam)                      # all Gaussians (needed by every pixel)
+    t_proj = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    keys, vals, ranges = oracle.keys(proj, cam)
+    t_keys = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    img, T, nc, amb = oracle.render(proj, cam, pix=pix)
+    tgt = wl.targets[0].reshape(-1, 3)[pix] if wl.targets else np.zeros((len(pix), 3), np.float32)
+    loss, g = oracle.l1(img.astype(np.float32), tgt)
+    g2, _, _ = oracle.render_bwd(proj, cam, g.astype(np.float64), pix=pix)
+    t_pix = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.project_bwd(scene, cam, g2[gidx], idx=gidx, densify=True)
+    t_pb = time.perf_counter() - t0
+    nv = len(wl.cameras)
+    per_view = t_proj + t_keys + t_pix * (tx * ty) / ntiles + t_pb * n / len(gidx)
+    t0 = time.perf_counter()
+    p = np.zeros(len(gidx) * 59, np.float32)
+    oracle.adam(p, p, p, p, 1e-3, 0.9, 0.99, 1e-15, 1)
+    t_adam = (time.perf_counter() - t0) * n / len(gidx)
+    per_iter = nv * per_view + t_adam
+    desc = (f"1 of {nv} views: projection+sort of all {n} Gaussians, forward+L1+backward on {ntiles} of {tx*ty} "
+            f"tiles, project_bwd on {len(gidx)} Gaussians, Adam on {len(gidx)*59} floats; scaled to "
+            f"{tx*ty} tiles, {n} Gaussians and {nv} views per iteration")
+    return per_iter, threads, desc
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    wl = make_workload(args.workload)
+    fraction = args.cpu_fraction
+    vals = []
+    per_iter = threads = desc = None
+    for i in range(args.warmup + args.steps):
+        per_iter, threads, desc = cpu_oracle_sample(wl, fraction, seed=i)
+        if i >= args.warmup:
+            vals.append(per_iter)
+    sec = statistics.mean(vals)
+    value = 1.0 / sec
+    line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "gaussians": wl.scene.n, "views_per_step": len(wl.cameras)},
+            "cpu_baseline": {"value": value, "unit": "iterations/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "iterations/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import oracle  # noqa: F401  (only for the cpu_baseline leg below)
+    from gaussian_splatting_differentiable_02_b200 import abi
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    abi.lib()
+    wl = make_workload(args.workload)
+    scene = wl.scene
+    nv = len(wl.cameras)
+    gauss = pl.Gaussians.from_scene(scene)
+    views = [pl.View(scene.n, cam) for cam in wl.cameras]
+    targets_host = torch.from_numpy(np.stack(wl.targets)).pin_memory() if wl.targets else None
+    targets = targets_host.cuda() if targets_host is not None else None
+    lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
+                                                  "opacity_logits": 5e-2, "sh": 2.5e-3}
+    tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also sizes every view's instance buffers)
+    for _ in range(args.warmup):
+        tr.step()
+    torch.cuda.synchronize()
+
+    # per-stage breakdown of one untimed step, to find the dominant kernel
+    stages = stage_breakdown(tr, pl, torch)
+    dominant = max(stages, key=lambda k: stages[k])
+
+    # ---- timed region: K steps on resident inputs
+    ev_dom = []
+    orig = {"raster_bwd": pl.raster_bwd, "raster_fwd": pl.raster_fwd, "project_bwd": pl.project_bwd,
+            "project": pl.project}
+
+    def wrap(fn):
+        def inner(*a, **k):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(*a, **k)
+            e1.record(stream)
+            ev_dom.append((e0, e1))
+        return inner
+
+    if dominant in orig:
+        setattr(pl, dominant, wrap(orig[dominant]))
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = abi.gs_kernel_launches()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        tr.step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = abi.gs_kernel_launches() - launches0
+    barrier(world)
+    clk = clocks.stop()
+    for k, f in orig.items():
+        setattr(pl, k, f)
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world)
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # ---- instance statistics for the byte / flop model
+    stats = []
+    pairs = 0
+    for v in views:
+        T = v.tiles_x * v.tiles_y
+        passes = (32 + max(1, math.ceil(math.log2(T))) + 7) // 8
+        stats.append((v.num_instances, int((tr.proj.radius > 0).sum().item()), passes))
+        pairs += int(v.n_contrib.sum().item())
+    cam0 = wl.cameras[0]
+    P = cam0["width"] * cam0["height"]
+    nbytes = step_bytes(scene.n, scene.sh_degree, stats, views[0].tiles_x * views[0].tiles_y, P)
+    peaks = measured_peaks()
+    hbm_peak = peaks["hbm_gbs"]
+    step_gbs = nbytes / (ms_per_step * 1e-3) / 1e9
+
+    dom_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev_dom) if ev_dom else stages[dominant]
+    roof = roofline_for(dominant, dom_ms, stats, pairs / nv, scene, P, clk, peaks)
+
+    line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv,
+                       "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
+                       "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2: each step streams %.2f GB of parameters, optimizer state, "
+                             "instances and images" % (nbytes / 1e9)},
+            "hbm": {"algorithmic_bytes_per_step": nbytes, "achieved_gbs": step_gbs, "peak_gbs": hbm_peak,
+                    "frac": step_gbs / hbm_peak, "peak_source": peaks["source"]},
+            "stages_ms_per_step": {k: round(v, 4) for k, v in stages.items()},
+            "roofline": roof,
+            "gpu_launches": int(launches),
+            "clocks": clk}
+    # e2e: the same step with the per-step inputs (16 target images) copied from
+    # pinned host memory and the loss read back, inside the timed region
+    line["e2e"] = run_e2e(tr, targets_host, targets, args, world, torch)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
+        line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def stage_breakdown(tr, pl, torch):
+    """Milliseconds per step of each stage, from CUDA events around every call of
+    one untimed step."""
+    stream = torch.cuda.current_stream()
+    acc = {}
+
+    def timed(name, fn, *a):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        r = fn(*a)
+        e1.record(stream)
+        acc.setdefault(name, []).append((e0, e1))
+        return r
+
+    tr.grads.zero_()
+    for view, tgt in zip(tr.views, tr.targets):
+        timed("project", pl.project, tr.gauss, view, tr.proj)
+        timed("bin_sort", pl.bin_sort, tr.proj, view)
+        timed("raster_fwd", pl.raster_fwd, tr.proj, view, tr.bg)
+        timed("l1", pl.l1_loss_grad, view, tgt, tr.loss)
+        tr.grad2d.zero_()
+        timed("raster_bwd", pl.raster_bwd, tr.proj, view, tr.grad2d, tr.bg)
+        timed("project_bwd", pl.project_bwd, tr.gauss, view, tr.proj, tr.grad2d, tr.grads, tr.densify_accum,
+              tr.densify_count)
+    tr.step_count += 1
+    timed("adam", pl.adam_step, tr.gauss, tr.grads, tr.m, tr.v, tr.lrs, tr.step_count)
+    torch.cuda.synchronize()
+    return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
+
+
+def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks):
+    """Roofline object of the dominant kernel: the raster kernels against the
+    float32 ALU peak (148 SMs x 128 lanes x 2 x max SM clock), the streaming
+    kernels against the measured HBM copy bandwidth."""
+    K = float(np.mean([s[0] for s in stats]))
+    V = float(np.mean([s[1] for s in stats]))
+    pb = 4 * (11 + 3 * (scene.sh_degree + 1) ** 2)
+    smax = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
+    if stage in ("raster_bwd", "raster_fwd"):
+        per_pair = FLOPS_ALPHA + (FLOPS_BWD_GRAD if stage == "raster_bwd" else FLOPS_FWD_BLEND)
+        flops = pairs_per_view * per_pair
+        achieved = flops / (ms * 1e-3) / 1e12
+        return {"kernel": stage, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": achieved / alu_peak, "traffic": None,
+                "work": f"{pairs_per_view:.4g} (pixel, entry) pairs x {per_pair} flops per launch",
+                "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"}
+    n = scene.n
+    per_launch = {"project_bwd": n * (pb + 36 + 2 * pb + 8), "project": n * (pb + 52),
+                  "bin_sort": n * 24 + K * 12 + K * (8 + 24 * stats[0][2]) + K * 8,
+                  "adam": n * pb // 4 * 28, "l1": P * 36}.get(stage, 0)
+    achieved = per_launch / (ms * 1e-3) / 1e9
+    return {"kernel": stage, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"]}
+
+
+def run_e2e(tr, targets_host, targets, args, world, torch):
+    """Steps whose target images arrive from pinned host memory (copied on a side
+    stream one view ahead, overlapping the previous view's kernels) and whose
+    loss is read back every step."""
+    if targets_host is None:
+        return None
+    stream = torch.cuda.current_stream()
+    copy_stream = torch.cuda.Stream()
+    nv = len(tr.views)
+    loss_host = torch.zeros(1, dtype=torch.float64).pin_memory()
+    bufs = [torch.empty_like(targets[0]) for _ in range(2)]
+
+    # the view loop mirrors Trainer.step with the target taken from the copy buffers
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    from gaussian_splatting_differentiable_02_b200 import abi
+
+    def step():
+        nonlocal done
+        done = [torch.cuda.Event() for _ in range(nv)]
+        s = stream.cuda_stream
+        tr.grads.zero_()
+        abi.gs_zero(tr.loss.data_ptr(), 8, s)
+        copy_events = []
+        with torch.cuda.stream(copy_stream):
+            for v in range(min(2, nv)):
+                bufs[v % 2].copy_(targets_host[v], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(copy_stream)
+                copy_events.append(e)
+        for v, view in enumerate(tr.views):
+            stream.wait_event(copy_events[v])
+            pl.project(tr.gauss, view, tr.proj)
+            pl.bin_sort(tr.proj, view)
+            pl.raster_fwd(tr.proj, view, tr.bg)
+            pl.l1_loss_grad(view, bufs[v % 2], tr.loss)
+            done[v].record(stream)
+            if v + 2 < nv:
+                with torch.cuda.stream(copy_stream):
+                    copy_stream.wait_event(done[v])
+                    bufs[v % 2].copy_(targets_host[v + 2], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(copy_stream)
+                    copy_events.append(e)
+            tr.grad2d.zero_()
+            pl.raster_bwd(tr.proj, view, tr.grad2d, tr.bg)
+            pl.project_bwd(tr.gauss, view, tr.proj, tr.grad2d, tr.grads, tr.densify_accum, tr.densify_count)
+        tr.step_count += 1
+        pl.adam_step(tr.gauss, tr.grads, tr.m, tr.v, tr.lrs, tr.step_count)
+        loss_host.copy_(tr.loss, non_blocking=True)
+
+    done = []
+    for _ in range(max(1, args.warmup // 2)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    h2d = int(targets_host.numel() * 4)
+    return {"value": world * args.steps / (ms / 1e3), "unit": "iterations/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": 8, "ms_per_step": ms / args.steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["multiview", "mixture", "box", "city", "tiny"], default="multiview")
+    ap.add_argument("--cpu-fraction", type=float, default=1.0 / 256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+"""ctypes binding of libgs.so: the C structures of include/gs.h and one Python
+function per C entry point, with the same name and argument order.
+
+Marshalling only.  Pointers are passed as integers (device addresses, e.g.
+``tensor.data_ptr()``), streams as the integer handle of a cudaStream_t.  A
+non-OK status raises ``GsError`` carrying gs_last_error_detail().  The library
+must have been built (``python -m gaussian_splatting_differentiable_02_b200.build``
+or ``__graft_entry__.build()``); a missing library is an error, never a fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgs.so")
+
+GS_OK = 0
+GS_ERR_INVALID_ARG = 1
+GS_ERR_UNSUPPORTED = 2
+GS_ERR_CAPACITY = 3
+GS_ERR_CUDA = 4
+GS_TILE = 16
+
+
+class GsError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"status {status}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+class gs_camera(C.Structure):
+    _fields_ = [("R", C.c_float * 9), ("t", C.c_float * 3), ("fx", C.c_float), ("fy", C.c_float),
+                ("cx", C.c_float), ("cy", C.c_float), ("width", C.c_int32), ("height", C.c_int32),
+                ("near_plane", C.c_float), ("eps2d", C.c_float)]
+
+
+class gs_params(C.Structure):
+    _fields_ = [("means", C.c_void_p), ("quats", C.c_void_p), ("log_scales", C.c_void_p),
+                ("opacity_logits", C.c_void_p), ("sh", C.c_void_p), ("sh_degree", C.c_int32), ("n", C.c_int64)]
+
+
+class gs_param_grads(C.Structure):
+    _fields_ = [("means", C.c_void_p), ("quats", C.c_void_p), ("log_scales", C.c_void_p),
+                ("opacity_logits", C.c_void_p), ("sh", C.c_void_p)]
+
+
+class gs_projected(C.Structure):
+    _fields_ = [("xy", C.c_void_p), ("depth", C.c_void_p), ("conic_opacity", C.c_void_p), ("rgb", C.c_void_p),
+                ("radius", C.c_void_p), ("rect", C.c_void_p), ("tiles_touched", C.c_void_p)]
+
+
+class gs_grad2d(C.Structure):
+    _fields_ = [("xy", C.c_void_p), ("conic_opacity", C.c_void_p), ("rgb", C.c_void_p)]
+
+
+# name -> (restype, argtypes), exactly the declarations of include/gs.h
+_P = C.c_void_p
+SIGNATURES = {
+    "gs_status_string": (C.c_char_p, [C.c_int32]),
+    "gs_last_error_detail": (C.c_char_p, []),
+    "gs_sh_planes": (C.c_int32, [C.c_int32]),
+    "gs_tile_grid": (C.c_int32, [C.POINTER(gs_camera), C.POINTER(C.c_int32), C.POINTER(C.c_int32)]),
+    "gs_project": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected), _P]),
+    "gs_bin_sort_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.POINTER(gs_camera)]),
+    "gs_bin_sort": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, C.c_size_t, _P, _P,
+                                C.c_int64, C.POINTER(C.c_int64), _P, _P]),
+    "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
+                                  _P, _P, _P]),
+    "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
+                                  _P, _P, C.POINTER(gs_grad2d), _P]),
+    "gs_project_bwd": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected),
+                                   C.POINTER(gs_grad2d), C.POINTER(gs_param_grads), _P, _P, _P]),
+    "gs_adam": (C.c_int32, [_P, _P, _P, _P, C.c_int64, C.c_float, C.c_float, C.c_float, C.c_float, C.c_int32, _P]),
+    "gs_l1_loss_grad": (C.c_int32, [_P, _P, C.c_int64, _P, _P, _P]),
+    "gs_zero": (C.c_int32, [_P, C.c_size_t, _P]),
+    "gs_kernel_launches": (C.c_uint64, []),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libgs.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgs.so not built ({LIB_PATH}); run the package's build.py")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != GS_OK:
+        raise GsError(status, lib().gs_last_error_detail().decode())
+    return status
+
+
+def make_camera(cam: dict) -> gs_camera:
+    """gs_camera from a scene camera dict (R 3x3 row-major, t, fx, fy, cx, cy, width, height, near, eps2d)."""
+    c = gs_camera()
+    R = [float(v) for v in __import__("numpy").asarray(cam["R"], "float32").reshape(9)]
+    t = [float(v) for v in __import__("numpy").asarray(cam["t"], "float32").reshape(3)]
+    for i in range(9):
+        c.R[i] = R[i]
+    for i in range(3):
+        c.t[i] = t[i]
+    c.fx, c.fy, c.cx, c.cy = cam["fx"], cam["fy"], cam["cx"], cam["cy"]
+    c.width, c.height = int(cam["width"]), int(cam["height"])
+    c.near_plane = cam.get("near", 0.2)
+    c.eps2d = cam.get("eps2d", 0.3)
+    return c
+
+
+# ------------------------------------------------------------ entry points
+
+def gs_status_string(status: int) -> str:
+    return lib().gs_status_string(status).decode()
+
+
+def gs_last_error_detail() -> str:
+    return lib().gs_last_error_detail().decode()
+
+
+def gs_sh_planes(sh_degree: int) -> int:
+    return lib().gs_sh_planes(sh_degree)
+
+
+def gs_tile_grid(cam: gs_camera):
+    tx, ty = C.c_int32(), C.c_int32()
+    _check(lib().gs_tile_grid(C.byref(cam), C.byref(tx), C.byref(ty)))
+    return tx.value, ty.value
+
+
+def gs_project(params: gs_params, cam: gs_camera, out: gs_projected, stream: int = 0):
+    return _check(lib().gs_project(C.byref(params), C.byref(cam), C.byref(out), stream))
+
+
+def gs_bin_sort_workspace_bytes(n: int, capacity: int, cam: gs_camera) -> int:
+    return lib().gs_bin_sort_workspace_bytes(n, capacity, C.byref(cam))
+
+
+def gs_bin_sort(proj: gs_projected, n: int, cam: gs_camera, workspace: int, workspace_bytes: int, keys: int,
+                vals: int, capacity: int, tile_ranges: int, stream: int = 0, check: bool = True):
+    """Returns (status, K).  With check=False a GS_ERR_CAPACITY status is returned, not raised."""
+    K = C.c_int64(0)
+    st = lib().gs_bin_sort(C.byref(proj), n, C.byref(cam), workspace, workspace_bytes, keys, vals, capacity,
+                           C.byref(K), tile_ranges, stream)
+    if check or st not in (GS_OK, GS_ERR_CAPACITY):
+        _check(st)
+    return st, K.value
+
+
+def gs_raster_fwd(proj: gs_projected, vals: int, tile_ranges: int, cam: gs_camera, bg, image: int, final_T: int,
+                  n_contrib: int, stream: int = 0):
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_fwd(C.byref(proj), vals, tile_ranges, C.byref(cam), b, image, final_T, n_contrib,
+                                      stream))
+
+
+def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, cam: gs_camera, bg, final_T: int, n_contrib: int,
+                  dL_dimage: int, grad2d: gs_grad2d, stream: int = 0):
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_bwd(C.byref(proj), vals, tile_ranges, C.byref(cam), b, final_T, n_contrib,
+                                      dL_dimage, C.byref(grad2d), stream))
+
+
+def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d: gs_grad2d, grads: gs_param_grads,
+                   densify_accum: int = 0, densify_count: int = 0, stream: int = 0):
+    return _check(lib().gs_project_bwd(C.byref(params), C.byref(cam), C.byref(proj), C.byref(grad2d),
+                                       C.byref(grads), densify_accum or None, densify_count or None, stream))
+
+
+def gs_adam(param: int, grad: int, m: int, v: int, count: int, lr: float, beta1: float, beta2: float, eps: float,
+            step: int, stream: int = 0):
+    return _check(lib().gs_adam(param, grad, m, v, count, lr, beta1, beta2, eps, step, stream))
+
+
+def gs_l1_loss_grad(image: int, target: int, count: int, dL_dimage: int, loss_dev: int, stream: int = 0):
+    return _check(lib().gs_l1_loss_grad(image, target, count, dL_dimage, loss_dev, stream))
+
+
+def gs_kernel_launches() -> int:
+    return lib().gs_kernel_launches()
+
+
+def gs_zero(ptr: int, nbytes: int, stream: int = 0):
+    return _check(lib().gs_zero(ptr, nbytes, stream))

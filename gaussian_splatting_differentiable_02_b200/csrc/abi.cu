@@ -1,0 +1,313 @@
+// C-ABI entry points of libgs.so (declared in gs.h): argument checks on the
+// host, then the kernel launches.  Nothing here allocates device memory.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.cuh"
+
+namespace gsk {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launches(int k) { g_launches.fetch_add(uint64_t(k), std::memory_order_relaxed); }
+
+CamArgs make_cam(const gs_camera& c) {
+    CamArgs k;
+    for (int i = 0; i < 9; ++i) k.R[i] = c.R[i];
+    for (int i = 0; i < 3; ++i) k.t[i] = c.t[i];
+    k.fx = c.fx;
+    k.fy = c.fy;
+    k.cx = c.cx;
+    k.cy = c.cy;
+    k.near_plane = c.near_plane;
+    k.eps2d = c.eps2d;
+    k.W = c.width;
+    k.H = c.height;
+    k.TX = (c.width + kTile - 1) / kTile;
+    k.TY = (c.height + kTile - 1) / kTile;
+    k.limx = 1.3 * (0.5 * double(c.width) / k.fx);
+    k.limy = 1.3 * (0.5 * double(c.height) / k.fy);
+    for (int j = 0; j < 3; ++j) k.cc[j] = -((k.R[0 + j] * k.t[0] + k.R[3 + j] * k.t[1]) + k.R[6 + j] * k.t[2]);
+    return k;
+}
+
+}  // namespace gsk
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+gs_status fail(gs_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+gs_status ok() {
+    g_detail[0] = '\0';
+    return GS_OK;
+}
+
+gs_status cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return ok();
+    return fail(GS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#define CHECK_PTR(p, align)                                                                      \
+    do {                                                                                         \
+        if ((p) == nullptr) return fail(GS_ERR_INVALID_ARG, "%s: %s is NULL", fn, #p);           \
+        if (!aligned((p), (align)))                                                              \
+            return fail(GS_ERR_INVALID_ARG, "%s: %s is not %d-byte aligned", fn, #p, int(align)); \
+    } while (0)
+
+gs_status check_camera(const char* fn, const gs_camera* cam) {
+    if (!cam) return fail(GS_ERR_INVALID_ARG, "%s: camera is NULL", fn);
+    if (cam->width <= 0 || cam->height <= 0 || cam->width > 16384 || cam->height > 16384)
+        return fail(GS_ERR_UNSUPPORTED, "%s: image %dx%d outside 1..16384", fn, cam->width, cam->height);
+    const float f[] = {cam->fx, cam->fy, cam->cx, cam->cy, cam->near_plane, cam->eps2d};
+    for (float v : f)
+        if (!std::isfinite(v)) return fail(GS_ERR_INVALID_ARG, "%s: non-finite camera intrinsics", fn);
+    for (int i = 0; i < 9; ++i)
+        if (!std::isfinite(cam->R[i])) return fail(GS_ERR_INVALID_ARG, "%s: non-finite camera rotation", fn);
+    for (int i = 0; i < 3; ++i)
+        if (!std::isfinite(cam->t[i])) return fail(GS_ERR_INVALID_ARG, "%s: non-finite camera translation", fn);
+    if (!(cam->fx > 0.f) || !(cam->fy > 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: focal lengths must be > 0", fn);
+    if (!(cam->near_plane > 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: near_plane must be > 0", fn);
+    if (!(cam->eps2d >= 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: eps2d must be >= 0", fn);
+    return GS_OK;
+}
+
+gs_status check_params(const char* fn, const gs_params* p) {
+    if (!p) return fail(GS_ERR_INVALID_ARG, "%s: params is NULL", fn);
+    if (p->n < 0 || p->n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n = %lld out of range", fn, (long long)p->n);
+    if (p->sh_degree < 0 || p->sh_degree > 3)
+        return fail(GS_ERR_UNSUPPORTED, "%s: SH degree %d (0..3 supported)", fn, int(p->sh_degree));
+    if (p->n == 0) return GS_OK;
+    CHECK_PTR(p->means, 16);
+    CHECK_PTR(p->quats, 16);
+    CHECK_PTR(p->log_scales, 16);
+    CHECK_PTR(p->opacity_logits, 4);
+    CHECK_PTR(p->sh, 16);
+    return GS_OK;
+}
+
+gs_status check_projected(const char* fn, const gs_projected* o, int64_t n, bool need_all) {
+    if (!o) return fail(GS_ERR_INVALID_ARG, "%s: projected is NULL", fn);
+    if (n == 0) return GS_OK;
+    CHECK_PTR(o->xy, 8);
+    CHECK_PTR(o->conic_opacity, 16);
+    CHECK_PTR(o->rgb, 16);
+    CHECK_PTR(o->radius, 4);
+    if (need_all) {
+        CHECK_PTR(o->depth, 4);
+        CHECK_PTR(o->rect, 8);
+        CHECK_PTR(o->tiles_touched, 4);
+    }
+    return GS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gs_status_string(gs_status s) {
+    switch (s) {
+        case GS_OK: return "GS_OK";
+        case GS_ERR_INVALID_ARG: return "GS_ERR_INVALID_ARG: invalid argument";
+        case GS_ERR_UNSUPPORTED: return "GS_ERR_UNSUPPORTED: unsupported configuration";
+        case GS_ERR_CAPACITY: return "GS_ERR_CAPACITY: instance buffer too small";
+        case GS_ERR_CUDA: return "GS_ERR_CUDA: CUDA error";
+        default: return "unknown gs_status";
+    }
+}
+
+const char* gs_last_error_detail(void) { return g_detail; }
+
+int32_t gs_sh_planes(int32_t sh_degree) { return gsk::sh_planes(sh_degree); }
+
+gs_status gs_tile_grid(const gs_camera* cam, int32_t* tiles_x_host, int32_t* tiles_y_host) {
+    const char* fn = "gs_tile_grid";
+    gs_status st = check_camera(fn, cam);
+    if (st != GS_OK) return st;
+    if (!tiles_x_host || !tiles_y_host) return fail(GS_ERR_INVALID_ARG, "%s: NULL output", fn);
+    *tiles_x_host = (cam->width + GS_TILE - 1) / GS_TILE;
+    *tiles_y_host = (cam->height + GS_TILE - 1) / GS_TILE;
+    return ok();
+}
+
+gs_status gs_project(const gs_params* params, const gs_camera* cam, gs_projected* out, void* stream) {
+    const char* fn = "gs_project";
+    gs_status st;
+    if ((st = check_params(fn, params)) != GS_OK) return st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, out, params->n, true)) != GS_OK) return st;
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_project_fwd(*params, c, *out, static_cast<cudaStream_t>(stream)), fn);
+}
+
+size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam) {
+    (void)cam;
+    if (n < 0) n = 0;
+    if (capacity < 0) capacity = 0;
+    return gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+}
+
+gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                      size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                      int64_t* num_instances_host, uint32_t* tile_ranges, void* stream) {
+    const char* fn = "gs_bin_sort";
+    gs_status st;
+    if (n < 0 || n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n out of range", fn);
+    if (capacity < 0 || capacity > 0xffffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: capacity out of range", fn);
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, proj, n, true)) != GS_OK) return st;
+    if (!num_instances_host) return fail(GS_ERR_INVALID_ARG, "%s: num_instances_host is NULL", fn);
+    CHECK_PTR(workspace, 16);
+    CHECK_PTR(tile_ranges, 8);
+    if (capacity > 0) {
+        CHECK_PTR(keys, 8);
+        CHECK_PTR(vals, 4);
+    }
+    const size_t need = gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+    if (workspace_bytes < need)
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
+    const int64_t tiles = int64_t((cam->width + GS_TILE - 1) / GS_TILE) * ((cam->height + GS_TILE - 1) / GS_TILE);
+    if (tiles > (int64_t(1) << 20)) return fail(GS_ERR_UNSUPPORTED, "%s: more than 2^20 tiles", fn);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    gsk::SortWorkspace ws;
+    gsk::sort_workspace_layout(n, capacity, workspace, &ws);
+    cudaError_t e = gsk::launch_count_instances(*proj, n, ws, s);
+    if (e != cudaSuccess) return cuda_status(e, fn);
+    unsigned long long K = 0;
+    e = cudaMemcpyAsync(&K, ws.total, sizeof K, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e, fn);
+    *num_instances_host = int64_t(K);
+    if (int64_t(K) > capacity)
+        return fail(GS_ERR_CAPACITY, "%s: %llu instances, capacity %lld", fn, K, (long long)capacity);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_emit_sort_ranges(*proj, n, c, ws, keys, vals, int64_t(K), tile_ranges, s), fn);
+}
+
+gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const gs_camera* cam, const float* bg_host, float* image, float* final_T,
+                        int32_t* n_contrib, void* stream) {
+    const char* fn = "gs_raster_fwd";
+    gs_status st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, proj, 1, false)) != GS_OK) return st;
+    if (!bg_host) return fail(GS_ERR_INVALID_ARG, "%s: bg_host is NULL", fn);
+    CHECK_PTR(vals, 4);
+    CHECK_PTR(tile_ranges, 8);
+    CHECK_PTR(image, 4);
+    CHECK_PTR(final_T, 4);
+    CHECK_PTR(n_contrib, 4);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_raster_fwd(*proj, vals, tile_ranges, c, bg_host, image, final_T, n_contrib,
+                                              static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const gs_camera* cam, const float* bg_host, const float* final_T,
+                        const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream) {
+    const char* fn = "gs_raster_bwd";
+    gs_status st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, proj, 1, false)) != GS_OK) return st;
+    if (!bg_host) return fail(GS_ERR_INVALID_ARG, "%s: bg_host is NULL", fn);
+    if (!grad2d) return fail(GS_ERR_INVALID_ARG, "%s: grad2d is NULL", fn);
+    CHECK_PTR(vals, 4);
+    CHECK_PTR(tile_ranges, 8);
+    CHECK_PTR(final_T, 4);
+    CHECK_PTR(n_contrib, 4);
+    CHECK_PTR(dL_dimage, 4);
+    CHECK_PTR(grad2d->xy, 8);
+    CHECK_PTR(grad2d->conic_opacity, 16);
+    CHECK_PTR(grad2d->rgb, 16);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_raster_bwd(*proj, vals, tile_ranges, c, bg_host, final_T, n_contrib, dL_dimage,
+                                              *grad2d, static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
+                         const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
+                         int32_t* densify_count, void* stream) {
+    const char* fn = "gs_project_bwd";
+    gs_status st;
+    if ((st = check_params(fn, params)) != GS_OK) return st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, proj, params->n, false)) != GS_OK) return st;
+    if (!grad2d || !grads) return fail(GS_ERR_INVALID_ARG, "%s: grad2d or grads is NULL", fn);
+    if ((densify_accum == nullptr) != (densify_count == nullptr))
+        return fail(GS_ERR_INVALID_ARG, "%s: densify_accum and densify_count must both be set or both NULL", fn);
+    if (params->n > 0) {
+        CHECK_PTR(grad2d->xy, 8);
+        CHECK_PTR(grad2d->conic_opacity, 16);
+        CHECK_PTR(grad2d->rgb, 16);
+        CHECK_PTR(grads->means, 16);
+        CHECK_PTR(grads->quats, 16);
+        CHECK_PTR(grads->log_scales, 16);
+        CHECK_PTR(grads->opacity_logits, 4);
+        CHECK_PTR(grads->sh, 16);
+        if (densify_accum) {
+            CHECK_PTR(densify_accum, 4);
+            CHECK_PTR(densify_count, 4);
+        }
+    }
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_project_bwd(*params, c, *proj, *grad2d, *grads, densify_accum, densify_count,
+                                               static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+gs_status gs_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
+                  float beta2, float eps, int32_t step, void* stream) {
+    const char* fn = "gs_adam";
+    if (count < 0) return fail(GS_ERR_INVALID_ARG, "%s: count < 0", fn);
+    if (step < 1) return fail(GS_ERR_INVALID_ARG, "%s: step must be >= 1", fn);
+    if (!std::isfinite(lr) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f))
+        return fail(GS_ERR_INVALID_ARG, "%s: invalid hyper-parameters", fn);
+    if (count == 0) return ok();
+    CHECK_PTR(param, 16);
+    CHECK_PTR(grad, 16);
+    CHECK_PTR(m, 16);
+    CHECK_PTR(v, 16);
+    return cuda_status(gsk::launch_adam(param, grad, m, v, count, lr, beta1, beta2, eps, step,
+                                        static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+gs_status gs_l1_loss_grad(const float* image, const float* target, int64_t count, float* dL_dimage,
+                          double* loss_dev, void* stream) {
+    const char* fn = "gs_l1_loss_grad";
+    if (count < 0) return fail(GS_ERR_INVALID_ARG, "%s: count < 0", fn);
+    if (count == 0) return ok();
+    CHECK_PTR(image, 16);
+    CHECK_PTR(target, 16);
+    CHECK_PTR(dL_dimage, 16);
+    CHECK_PTR(loss_dev, 8);
+    return cuda_status(gsk::launch_l1(image, target, count, dL_dimage, loss_dev, static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+uint64_t gs_kernel_launches(void) { return gsk::g_launches.load(std::memory_order_relaxed); }
+
+gs_status gs_zero(void* ptr, size_t bytes, void* stream) {
+    const char* fn = "gs_zero";
+    if (bytes == 0) return ok();
+    if (!ptr) return fail(GS_ERR_INVALID_ARG, "%s: ptr is NULL", fn);
+    return cuda_status(cudaMemsetAsync(ptr, 0, bytes, static_cast<cudaStream_t>(stream)), fn);
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libgs.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gs.h"
+
+namespace gsk {
+
+constexpr int kTile = GS_TILE;              // 16x16 pixel tiles
+constexpr int kTilePixels = kTile * kTile;  // 256
+constexpr int kNumSMs = 148;                // B200
+
+// Camera with the derived quantities every kernel needs, computed once on the
+// host in double precision from the float32 fields.
+struct CamArgs {
+    double R[9], t[3];
+    double fx, fy, cx, cy, near_plane, eps2d;
+    double limx, limy;  // 1.3 x half field of view, in x/z and y/z
+    double cc[3];       // camera centre -R^T t
+    int W, H, TX, TY;
+};
+
+CamArgs make_cam(const gs_camera& c);
+
+inline int sh_planes(int deg) {
+    switch (deg) {
+        case 0: return 1;
+        case 1: return 3;
+        case 2: return 7;
+        case 3: return 12;
+        default: return 0;
+    }
+}
+
+inline int tile_bits(int64_t tiles) {
+    int b = 0;
+    while ((int64_t(1) << b) < tiles) ++b;
+    return b;
+}
+
+// ------------------------------------------------------------------ launchers
+// Each returns the launch's cudaGetLastError().
+
+cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s);
+
+cudaError_t launch_project_bwd(const gs_params& p, const CamArgs& cam, const gs_projected& proj,
+                               const gs_grad2d& g2, const gs_param_grads& g, float* densify_accum,
+                               int32_t* densify_count, cudaStream_t s);
+
+struct SortWorkspace {
+    unsigned long long* block_sums;  // [nb_emit]
+    unsigned long long* total;       // [1]
+    uint64_t* keys_alt;              // [capacity]
+    uint32_t* vals_alt;              // [capacity]
+    uint32_t* hist;                  // [256][nb_sort]
+    uint32_t* digit_totals;          // [256]
+    int64_t nb_emit, nb_sort;
+};
+size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws);
+
+cudaError_t launch_count_instances(const gs_projected& proj, int64_t n, const SortWorkspace& ws, cudaStream_t s);
+cudaError_t launch_emit_sort_ranges(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
+                                    uint64_t* keys, uint32_t* vals, int64_t K, uint32_t* ranges, cudaStream_t s);
+
+cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
+                              const CamArgs& cam, const float bg[3], float* image, float* final_T,
+                              int32_t* n_contrib, cudaStream_t s);
+
+cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
+                              const CamArgs& cam, const float bg[3], const float* final_T, const int32_t* n_contrib,
+                              const float* dL_dimage, const gs_grad2d& g2, cudaStream_t s);
+
+cudaError_t launch_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
+                        float beta2, float eps, int32_t step, cudaStream_t s);
+
+cudaError_t launch_l1(const float* image, const float* target, int64_t count, float* dL, double* loss,
+                      cudaStream_t s);
+
+// host-side count of kernel launches (gs_kernel_launches)
+void count_launches(int k);
+
+// grid size: a multiple of the SM count, capped by the work
+inline unsigned grid_for(int64_t work, int block, int per_sm = 8) {
+    int64_t g = (work + block - 1) / block;
+    int64_t cap = int64_t(kNumSMs) * per_sm;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return unsigned(g);
+}
+
+}  // namespace gsk

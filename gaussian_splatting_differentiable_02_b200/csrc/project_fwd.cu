@@ -1,0 +1,236 @@
+// gs_project: per-Gaussian projection (stages 1-2 of the pipeline in the gsplat
+// guide, lmnt.cn/news/262699 §2.1) in double precision.
+//
+// This file is compiled with -fmad=false: every product and sum rounds as
+// written, so the integer decisions taken from floating point (culling, the
+// 3-sigma radius, the tile rectangle) and the float32 depth used in the sort key
+// come out the same on any IEEE double implementation that evaluates the same
+// expressions in the same order.  The projection is streaming work (about 290
+// bytes per Gaussian) and sits far below the device's double-precision rate, so
+// the wider arithmetic costs no time.
+#include "internal.cuh"
+
+namespace gsk {
+namespace {
+
+// Real spherical harmonics to degree 3 (orthonormal, Condon-Shortley phase),
+// index l^2 + l + m.
+constexpr double kY0 = 0.28209479177387814;
+constexpr double kY1 = 0.4886025119029199;
+__constant__ double kY2[5] = {1.0925484305920792, -1.0925484305920792, 0.31539156525252005, -1.0925484305920792,
+                           0.5462742152960396};
+__constant__ double kY3[7] = {-0.5900435899266435, 2.890611442640554, -0.4570457994644658, 0.3731763325901154,
+                           -0.4570457994644658, 1.445305721320277, -0.5900435899266435};
+
+struct FwdArgs {
+    const float4* means;
+    const float4* quats;
+    const float4* log_scales;
+    const float* logits;
+    const float4* sh;
+    int deg, planes;
+    int64_t n;
+    CamArgs cam;
+    float2* xy;
+    float* depth;
+    float4* conic_op;
+    float4* rgb;
+    int32_t* radius;
+    uint2* rect;
+    uint32_t* tiles_touched;
+};
+
+__device__ __forceinline__ bool finite(double x) { return isfinite(x); }
+
+__device__ void write_culled(const FwdArgs& a, int64_t i) {
+    a.xy[i] = make_float2(0.f, 0.f);
+    a.depth[i] = 0.f;
+    a.conic_op[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    a.rgb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    a.radius[i] = 0;
+    a.rect[i] = make_uint2(0u, 0u);
+    a.tiles_touched[i] = 0u;
+}
+
+__global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
+    const CamArgs& cam = a.cam;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < a.n; i += int64_t(gridDim.x) * blockDim.x) {
+        const float4 m4 = __ldg(a.means + i);
+        const float4 q4 = __ldg(a.quats + i);
+        const float4 s4 = __ldg(a.log_scales + i);
+        const float lg = __ldg(a.logits + i);
+        const double mu[3] = {m4.x, m4.y, m4.z};
+        const double q[4] = {q4.x, q4.y, q4.z, q4.w};
+        const double ls[3] = {s4.x, s4.y, s4.z};
+        const double logit = lg;
+        bool ok = finite(mu[0]) && finite(mu[1]) && finite(mu[2]) && finite(q[0]) && finite(q[1]) &&
+                  finite(q[2]) && finite(q[3]) && finite(ls[0]) && finite(ls[1]) && finite(ls[2]) && finite(logit);
+        if (!ok) { write_culled(a, i); continue; }
+
+        // camera space
+        double pc[3];
+#pragma unroll
+        for (int r = 0; r < 3; ++r)
+            pc[r] = ((cam.R[3 * r + 0] * mu[0] + cam.R[3 * r + 1] * mu[1]) + cam.R[3 * r + 2] * mu[2]) + cam.t[r];
+        if (!(pc[2] > cam.near_plane)) { write_culled(a, i); continue; }
+
+        // rotation of the normalised quaternion (w, x, y, z)
+        const double qn2 = ((q[0] * q[0] + q[1] * q[1]) + q[2] * q[2]) + q[3] * q[3];
+        if (!(qn2 > 0.0)) { write_culled(a, i); continue; }
+        const double qn = sqrt(qn2);
+        const double w = q[0] / qn, x = q[1] / qn, y = q[2] / qn, z = q[3] / qn;
+        double Rq[3][3];
+        Rq[0][0] = 1.0 - 2.0 * (y * y + z * z);
+        Rq[0][1] = 2.0 * (x * y - w * z);
+        Rq[0][2] = 2.0 * (x * z + w * y);
+        Rq[1][0] = 2.0 * (x * y + w * z);
+        Rq[1][1] = 1.0 - 2.0 * (x * x + z * z);
+        Rq[1][2] = 2.0 * (y * z - w * x);
+        Rq[2][0] = 2.0 * (x * z - w * y);
+        Rq[2][1] = 2.0 * (y * z + w * x);
+        Rq[2][2] = 1.0 - 2.0 * (x * x + y * y);
+
+        const double s[3] = {exp(ls[0]), exp(ls[1]), exp(ls[2])};
+        double M[3][3];
+#pragma unroll
+        for (int r = 0; r < 3; ++r)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) M[r][c] = Rq[r][c] * s[c];
+        double S[3][3];
+#pragma unroll
+        for (int r = 0; r < 3; ++r)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) S[r][c] = (M[r][0] * M[c][0] + M[r][1] * M[c][1]) + M[r][2] * M[c][2];
+
+        // perspective Jacobian with x/z, y/z clamped to 1.3 x the half field of view
+        double txz = pc[0] / pc[2], tyz = pc[1] / pc[2];
+        if (txz < -cam.limx) txz = -cam.limx;
+        if (txz > cam.limx) txz = cam.limx;
+        if (tyz < -cam.limy) tyz = -cam.limy;
+        if (tyz > cam.limy) tyz = cam.limy;
+        const double tx = txz * pc[2], ty = tyz * pc[2];
+        const double iz = 1.0 / pc[2];
+        const double J00 = cam.fx * iz, J02 = -(cam.fx * tx) * (iz * iz);
+        const double J11 = cam.fy * iz, J12 = -(cam.fy * ty) * (iz * iz);
+        double Tm[2][3];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            Tm[0][c] = J00 * cam.R[0 + c] + J02 * cam.R[6 + c];
+            Tm[1][c] = J11 * cam.R[3 + c] + J12 * cam.R[6 + c];
+        }
+        double X[2][3];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int c = 0; c < 3; ++c) X[r][c] = (Tm[r][0] * S[0][c] + Tm[r][1] * S[1][c]) + Tm[r][2] * S[2][c];
+        const double ca = ((X[0][0] * Tm[0][0] + X[0][1] * Tm[0][1]) + X[0][2] * Tm[0][2]) + cam.eps2d;
+        const double cb = (X[0][0] * Tm[1][0] + X[0][1] * Tm[1][1]) + X[0][2] * Tm[1][2];
+        const double cc = ((X[1][0] * Tm[1][0] + X[1][1] * Tm[1][1]) + X[1][2] * Tm[1][2]) + cam.eps2d;
+        const double det = ca * cc - cb * cb;
+        if (!(det > 0.0)) { write_culled(a, i); continue; }
+        const double idet = 1.0 / det;
+
+        const double mid = 0.5 * (ca + cc);
+        const double lmax = mid + sqrt(fmax(0.1, mid * mid - det));
+        const double r = ceil(3.0 * sqrt(lmax));
+
+        const double u = cam.fx * (pc[0] / pc[2]) + cam.cx;
+        const double v = cam.fy * (pc[1] / pc[2]) + cam.cy;
+        if (!finite(u) || !finite(v) || !finite(r)) { write_culled(a, i); continue; }
+
+        const double TXd = cam.TX, TYd = cam.TY;
+        const double xmin = fmin(fmax(floor((u - r) * 0.0625), 0.0), TXd);
+        const double xmax = fmin(fmax(floor((u + r) * 0.0625) + 1.0, 0.0), TXd);
+        const double ymin = fmin(fmax(floor((v - r) * 0.0625), 0.0), TYd);
+        const double ymax = fmin(fmax(floor((v + r) * 0.0625) + 1.0, 0.0), TYd);
+        if ((xmax - xmin) * (ymax - ymin) <= 0.0) { write_culled(a, i); continue; }
+
+        // colour from the SH of the unit viewing direction
+        const double dvx = mu[0] - cam.cc[0], dvy = mu[1] - cam.cc[1], dvz = mu[2] - cam.cc[2];
+        const double dn = sqrt((dvx * dvx + dvy * dvy) + dvz * dvz);
+        const double ux = dvx / dn, uy = dvy / dn, uz = dvz / dn;
+        double Y[16];
+        Y[0] = kY0;
+        if (a.deg >= 1) {
+            Y[1] = -kY1 * uy;
+            Y[2] = kY1 * uz;
+            Y[3] = -kY1 * ux;
+        }
+        if (a.deg >= 2) {
+            const double xx = ux * ux, yy = uy * uy, zz = uz * uz;
+            Y[4] = kY2[0] * (ux * uy);
+            Y[5] = kY2[1] * (uy * uz);
+            Y[6] = kY2[2] * (2.0 * zz - xx - yy);
+            Y[7] = kY2[3] * (ux * uz);
+            Y[8] = kY2[4] * (xx - yy);
+            if (a.deg >= 3) {
+                Y[9] = kY3[0] * uy * (3.0 * xx - yy);
+                Y[10] = kY3[1] * (ux * uy) * uz;
+                Y[11] = kY3[2] * uy * (4.0 * zz - xx - yy);
+                Y[12] = kY3[3] * uz * (2.0 * zz - 3.0 * xx - 3.0 * yy);
+                Y[13] = kY3[4] * ux * (4.0 * zz - xx - yy);
+                Y[14] = kY3[5] * uz * (xx - yy);
+                Y[15] = kY3[6] * ux * (xx - 3.0 * yy);
+            }
+        }
+        const int nc = (a.deg + 1) * (a.deg + 1);
+        double col[3] = {0.0, 0.0, 0.0};
+        for (int p = 0; p < a.planes; ++p) {
+            const float4 c4 = __ldg(a.sh + int64_t(p) * a.n + i);
+            const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int f = 4 * p + e;  // flat coefficient index = 3 k + channel
+                const int k = f / 3;
+                if (k < nc) col[f - 3 * k] += double(cv[e]) * Y[k];
+            }
+        }
+        float rgbf[3];
+        bool colour_ok = true;
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) {
+            const double c = col[ch] + 0.5;
+            colour_ok = colour_ok && finite(c);
+            rgbf[ch] = float(c < 0.0 ? 0.0 : c);
+        }
+        if (!colour_ok) { write_culled(a, i); continue; }
+
+        const double o = 1.0 / (1.0 + exp(-logit));
+        a.xy[i] = make_float2(float(u), float(v));
+        a.depth[i] = float(pc[2]);
+        a.conic_op[i] = make_float4(float(cc * idet), float(-cb * idet), float(ca * idet), float(o));
+        a.rgb[i] = make_float4(rgbf[0], rgbf[1], rgbf[2], 0.f);
+        a.radius[i] = int32_t(r);
+        const uint32_t x0 = uint32_t(xmin), y0 = uint32_t(ymin), x1 = uint32_t(xmax), y1 = uint32_t(ymax);
+        a.rect[i] = make_uint2(x0 | (y0 << 16), x1 | (y1 << 16));
+        a.tiles_touched[i] = (x1 - x0) * (y1 - y0);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s) {
+    FwdArgs a;
+    a.means = reinterpret_cast<const float4*>(p.means);
+    a.quats = reinterpret_cast<const float4*>(p.quats);
+    a.log_scales = reinterpret_cast<const float4*>(p.log_scales);
+    a.logits = p.opacity_logits;
+    a.sh = reinterpret_cast<const float4*>(p.sh);
+    a.deg = p.sh_degree;
+    a.planes = sh_planes(p.sh_degree);
+    a.n = p.n;
+    a.cam = cam;
+    a.xy = reinterpret_cast<float2*>(out.xy);
+    a.depth = out.depth;
+    a.conic_op = reinterpret_cast<float4*>(out.conic_opacity);
+    a.rgb = reinterpret_cast<float4*>(out.rgb);
+    a.radius = out.radius;
+    a.rect = reinterpret_cast<uint2*>(out.rect);
+    a.tiles_touched = out.tiles_touched;
+    if (p.n == 0) return cudaSuccess;
+    project_fwd_kernel<<<grid_for(p.n, 256, 16), 256, 0, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace gsk

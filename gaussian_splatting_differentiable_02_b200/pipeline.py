@@ -1,0 +1,263 @@
+"""Device buffers (torch) and the call sequence of one view / one training step.
+
+Argument marshalling only: every computation runs in libgs.so through the
+binding in ``abi``.  torch provides device memory and the current stream.
+
+Layouts follow include/gs.h: means/quats/log_scales are [n,4] float32,
+opacity logits [n], SH [P,n,4] with P = gs_sh_planes(degree).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import abi
+
+PARAM_NAMES = ("means", "quats", "log_scales", "opacity_logits", "sh")
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def sh_planes(deg: int) -> int:
+    return {0: 1, 1: 3, 2: 7, 3: 12}[deg]
+
+
+def sh_to_planes(sh: np.ndarray) -> np.ndarray:
+    """[n, nc, 3] coefficients -> [P, n, 4] float4 planes (coefficient-major, zero tail)."""
+    n, nc, _ = sh.shape
+    deg = int(round(math.sqrt(nc))) - 1
+    P = sh_planes(deg)
+    flat = np.zeros((n, 4 * P), np.float32)
+    flat[:, :3 * nc] = sh.reshape(n, 3 * nc)
+    return np.ascontiguousarray(flat.reshape(n, P, 4).transpose(1, 0, 2))
+
+
+def planes_to_sh(planes: np.ndarray, deg: int) -> np.ndarray:
+    P, n, _ = planes.shape
+    nc = (deg + 1) ** 2
+    flat = planes.transpose(1, 0, 2).reshape(n, 4 * P)
+    return flat[:, :3 * nc].reshape(n, nc, 3)
+
+
+class Gaussians:
+    """SoA device copy of a scene's parameters (or of gradients / Adam moments of the same shape)."""
+
+    def __init__(self, n: int, sh_degree: int, device="cuda"):
+        self.n = int(n)
+        self.sh_degree = int(sh_degree)
+        z = dict(device=device, dtype=torch.float32)
+        self.means = torch.zeros((n, 4), **z)
+        self.quats = torch.zeros((n, 4), **z)
+        self.log_scales = torch.zeros((n, 4), **z)
+        self.opacity_logits = torch.zeros((n,), **z)
+        self.sh = torch.zeros((sh_planes(sh_degree), n, 4), **z)
+
+    @classmethod
+    def from_scene(cls, scene, device="cuda") -> "Gaussians":
+        g = cls(scene.n, scene.sh_degree, device)
+        g.load_scene(scene)
+        return g
+
+    def load_scene(self, scene):
+        n = self.n
+        m = np.zeros((n, 4), np.float32)
+        m[:, :3] = scene.means
+        self.means.copy_(torch.from_numpy(m))
+        self.quats.copy_(torch.from_numpy(np.ascontiguousarray(scene.quats, np.float32)))
+        s = np.zeros((n, 4), np.float32)
+        s[:, :3] = scene.log_scales
+        self.log_scales.copy_(torch.from_numpy(s))
+        self.opacity_logits.copy_(torch.from_numpy(np.ascontiguousarray(scene.opacity_logits, np.float32)))
+        self.sh.copy_(torch.from_numpy(sh_to_planes(np.asarray(scene.sh, np.float32))))
+
+    def zeros_like(self) -> "Gaussians":
+        return Gaussians(self.n, self.sh_degree, self.means.device)
+
+    def tensors(self):
+        return {k: getattr(self, k) for k in PARAM_NAMES}
+
+    def params(self) -> abi.gs_params:
+        return abi.gs_params(_ptr(self.means), _ptr(self.quats), _ptr(self.log_scales), _ptr(self.opacity_logits),
+                             _ptr(self.sh), self.sh_degree, self.n)
+
+    def grads(self) -> abi.gs_param_grads:
+        return abi.gs_param_grads(_ptr(self.means), _ptr(self.quats), _ptr(self.log_scales),
+                                  _ptr(self.opacity_logits), _ptr(self.sh))
+
+    def zero_(self):
+        s = _stream()
+        for t in self.tensors().values():
+            abi.gs_zero(_ptr(t), t.numel() * 4, s)
+
+    def to_numpy(self) -> dict:
+        """Natural layout: means [n,3], quats [n,4], log_scales [n,3], opacity_logits [n], sh [n,nc,3]."""
+        return {"means": self.means[:, :3].cpu().numpy(), "quats": self.quats.cpu().numpy(),
+                "log_scales": self.log_scales[:, :3].cpu().numpy(),
+                "opacity_logits": self.opacity_logits.cpu().numpy(),
+                "sh": planes_to_sh(self.sh.cpu().numpy(), self.sh_degree)}
+
+
+class Projected:
+    def __init__(self, n: int, device="cuda"):
+        f = dict(device=device, dtype=torch.float32)
+        i = dict(device=device, dtype=torch.int32)
+        self.n = n
+        n = max(n, 1)   # the raster calls take non-NULL feature arrays even for an empty scene
+        self.xy = torch.zeros((n, 2), **f)
+        self.depth = torch.zeros((n,), **f)
+        self.conic_opacity = torch.zeros((n, 4), **f)
+        self.rgb = torch.zeros((n, 4), **f)
+        self.radius = torch.zeros((n,), **i)
+        self.rect = torch.zeros((n, 4), device=device, dtype=torch.int16)   # uint16 values < 2^15
+        self.tiles_touched = torch.zeros((n,), **i)                         # uint32 values < 2^31
+
+    def struct(self) -> abi.gs_projected:
+        return abi.gs_projected(_ptr(self.xy), _ptr(self.depth), _ptr(self.conic_opacity), _ptr(self.rgb),
+                                _ptr(self.radius), _ptr(self.rect), _ptr(self.tiles_touched))
+
+
+class Grad2D:
+    def __init__(self, n: int, device="cuda"):
+        f = dict(device=device, dtype=torch.float32)
+        n = max(n, 1)
+        self.xy = torch.zeros((n, 2), **f)
+        self.conic_opacity = torch.zeros((n, 4), **f)
+        self.rgb = torch.zeros((n, 4), **f)
+
+    def struct(self) -> abi.gs_grad2d:
+        return abi.gs_grad2d(_ptr(self.xy), _ptr(self.conic_opacity), _ptr(self.rgb))
+
+    def zero_(self):
+        s = _stream()
+        for t in (self.xy, self.conic_opacity, self.rgb):
+            abi.gs_zero(_ptr(t), t.numel() * 4, s)
+
+    def as_rows(self) -> np.ndarray:
+        """[n, 9]: u, v, A, B, C, o, r, g, b (the oracle's order)."""
+        return np.concatenate([self.xy.cpu().numpy(), self.conic_opacity.cpu().numpy(),
+                               self.rgb[:, :3].cpu().numpy()], axis=1)
+
+
+class View:
+    """Per-camera buffers: sorted instances, tile ranges, image and its gradient."""
+
+    def __init__(self, n: int, cam: dict, device="cuda", capacity: int = 0):
+        self.cam = cam
+        self.gcam = abi.make_camera(cam)
+        self.n = n
+        self.device = device
+        self.tiles_x, self.tiles_y = abi.gs_tile_grid(self.gcam)
+        T = self.tiles_x * self.tiles_y
+        H, W = cam["height"], cam["width"]
+        self.ranges = torch.zeros((T, 2), device=device, dtype=torch.int32)
+        self.image = torch.zeros((H, W, 3), device=device, dtype=torch.float32)
+        self.final_T = torch.zeros((H, W), device=device, dtype=torch.float32)
+        self.n_contrib = torch.zeros((H, W), device=device, dtype=torch.int32)
+        self.dL_dimage = torch.zeros((H, W, 3), device=device, dtype=torch.float32)
+        self.num_instances = 0
+        self.capacity = 0
+        self._alloc(max(capacity, 4 * n, 1024))
+
+    def _alloc(self, capacity: int):
+        self.capacity = int(capacity)
+        self.keys = torch.zeros((self.capacity,), device=self.device, dtype=torch.int64)
+        self.vals = torch.zeros((self.capacity,), device=self.device, dtype=torch.int32)
+        nbytes = abi.gs_bin_sort_workspace_bytes(self.n, self.capacity, self.gcam)
+        self.workspace = torch.zeros((nbytes,), device=self.device, dtype=torch.uint8)
+
+
+def project(g: Gaussians, view: View, proj: Projected):
+    abi.gs_project(g.params(), view.gcam, proj.struct(), _stream())
+
+
+def bin_sort(proj: Projected, view: View):
+    """Sort the instances; grows the view's buffers when they are too small.  Returns K."""
+    s = _stream()
+    while True:
+        st, K = abi.gs_bin_sort(proj.struct(), view.n, view.gcam, _ptr(view.workspace), view.workspace.numel(),
+                                _ptr(view.keys), _ptr(view.vals), view.capacity, _ptr(view.ranges), s, check=False)
+        if st == abi.GS_OK:
+            view.num_instances = K
+            return K
+        view._alloc(int(K * 1.25) + 1024)
+
+
+def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0)):
+    abi.gs_raster_fwd(proj.struct(), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.image),
+                      _ptr(view.final_T), _ptr(view.n_contrib), _stream())
+
+
+def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), dL_dimage: torch.Tensor = None):
+    d = view.dL_dimage if dL_dimage is None else dL_dimage
+    abi.gs_raster_bwd(proj.struct(), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.final_T),
+                      _ptr(view.n_contrib), _ptr(d), grad2d.struct(), _stream())
+
+
+def project_bwd(g: Gaussians, view: View, proj: Projected, grad2d: Grad2D, grads: Gaussians,
+                densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None):
+    abi.gs_project_bwd(g.params(), view.gcam, proj.struct(), grad2d.struct(), grads.grads(), _ptr(densify_accum),
+                       _ptr(densify_count), _stream())
+
+
+def l1_loss_grad(view: View, target: torch.Tensor, loss_dev: torch.Tensor):
+    abi.gs_l1_loss_grad(_ptr(view.image), _ptr(target), view.image.numel(), _ptr(view.dL_dimage), _ptr(loss_dev),
+                        _stream())
+
+
+def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: dict, step: int,
+              betas=(0.9, 0.99), eps=1e-15):
+    s = _stream()
+    for name in PARAM_NAMES:
+        p = getattr(g, name)
+        abi.gs_adam(_ptr(p), _ptr(getattr(grads, name)), _ptr(getattr(m, name)), _ptr(getattr(v, name)), p.numel(),
+                    lrs[name], betas[0], betas[1], eps, step, s)
+
+
+@dataclass
+class Trainer:
+    """One or several views of L1 training with Adam (the training loop of the gsplat guide §4.1-4.2),
+    optionally accumulating the densification statistic."""
+    gauss: Gaussians
+    views: list
+    targets: list
+    lrs: dict
+    bg: tuple = (0.0, 0.0, 0.0)
+    densify: bool = False
+
+    def __post_init__(self):
+        n = self.gauss.n
+        dev = self.gauss.means.device
+        self.proj = Projected(n, dev)
+        self.grad2d = Grad2D(n, dev)
+        self.grads = self.gauss.zeros_like()
+        self.m = self.gauss.zeros_like()
+        self.v = self.gauss.zeros_like()
+        self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
+        self.densify_accum = torch.zeros((n,), device=dev, dtype=torch.float32) if self.densify else None
+        self.densify_count = torch.zeros((n,), device=dev, dtype=torch.int32) if self.densify else None
+        self.step_count = 0
+
+    def step(self) -> None:
+        """forward + L1 + backward for every view, then one Adam step; loss stays on the device."""
+        s = _stream()
+        self.grads.zero_()
+        abi.gs_zero(_ptr(self.loss), 8, s)
+        for view, tgt in zip(self.views, self.targets):
+            project(self.gauss, view, self.proj)
+            bin_sort(self.proj, view)
+            raster_fwd(self.proj, view, self.bg)
+            l1_loss_grad(view, tgt, self.loss)
+            self.grad2d.zero_()
+            raster_bwd(self.proj, view, self.grad2d, self.bg)
+            project_bwd(self.gauss, view, self.proj, self.grad2d, self.grads, self.densify_accum, self.densify_count)
+        self.step_count += 1
+        adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)

@@ -1,0 +1,237 @@
+/*
+ * gs.h - C ABI of the B200 differentiable Gaussian-splatting tile rasterizer (libgs.so).
+ *
+ * The library is the data-parallel hot path of 3D Gaussian Splatting: per-Gaussian
+ * projection, tile binning with a (tile_id << 32 | depth) radix sort, front-to-back
+ * alpha compositing per 16x16 tile, its reverse pass, the chain back to the Gaussian
+ * parameters, and the Adam update.  The three stages are the ones named in the gsplat
+ * guide (lmnt.cn/news/262699) §2.1 -- "3D transform (R, t, scale, rot)", "depth and
+ * screen-space projection", "differentiable alpha-blending rasterization" -- and the
+ * split into a forward call and a standalone backward call follows the same guide
+ * §2.2 (rasterize_gaussians / rasterize_gaussians_backward).
+ *
+ * Conventions for every call
+ *   - Plain C.  Every call returns a gs_status; GS_OK is 0.  On failure,
+ *     gs_last_error_detail() returns a thread-local description.
+ *   - The library allocates nothing.  The caller owns every buffer.  Pointers are
+ *     device pointers unless the name ends in _host.  `stream` is a cudaStream_t
+ *     (NULL = the legacy default stream); calls enqueue work on it and return
+ *     without waiting, except gs_bin_sort, which reads the instance count back
+ *     to the host (one device-to-host copy and a stream synchronisation).
+ *   - Arguments are checked on the host before anything is launched: NULL
+ *     pointers, negative sizes and misaligned buffers (alignment as stated per
+ *     array) return GS_ERR_INVALID_ARG; an SH degree above 3 or an image side
+ *     outside 1..16384 returns GS_ERR_UNSUPPORTED.  A CUDA launch or copy error
+ *     returns GS_ERR_CUDA.  No kernel traps or asserts.
+ *   - Gradient outputs are accumulated (+=): callers zero them, and several views
+ *     can add into the same buffers.
+ *   - Arrays are structure-of-arrays, read with 128-bit loads: an array written
+ *     "[n][4]" is n consecutive float4 records (16-byte aligned).
+ *   - n (Gaussians) up to 2^31 - 1; instance counts up to 2^32 - 1; tiles up to 2^20.
+ */
+#ifndef GS_H
+#define GS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t gs_status;
+#define GS_OK 0
+#define GS_ERR_INVALID_ARG 1
+#define GS_ERR_UNSUPPORTED 2
+#define GS_ERR_CAPACITY 3
+#define GS_ERR_CUDA 4
+
+#define GS_TILE 16 /* tile side in pixels */
+
+/* Pinhole camera.  x_cam = R x_world + t (R row-major, world to camera), OpenCV
+ * axes (x right, y down, z forward).  Pixel (x, y) samples the image plane at
+ * (x + 0.5, y + 0.5).  Gaussians with camera depth <= near_plane are culled; eps2d
+ * is added to both diagonal entries of every projected 2D covariance (the
+ * screen-space low-pass of the original 3DGS rasterizer, 0.3). */
+typedef struct gs_camera {
+    float R[9];
+    float t[3];
+    float fx, fy, cx, cy;
+    int32_t width, height;
+    float near_plane;
+    float eps2d;
+} gs_camera;
+
+/* Gaussian parameters, stored pre-activation as the gsplat guide §3.3 sets
+ * them up: scale = exp(log_scale), opacity = sigmoid(logit), rotation = the
+ * normalised quaternion (w, x, y, z).
+ *   means          [n][4]  x, y, z, unused        (16-byte aligned)
+ *   quats          [n][4]  w, x, y, z             (16-byte aligned)
+ *   log_scales     [n][4]  x, y, z, unused        (16-byte aligned)
+ *   opacity_logits [n]                            (4-byte aligned)
+ *   sh             [P][n][4] with P = gs_sh_planes(sh_degree): the Gaussian's
+ *                  3*(d+1)^2 SH coefficients, coefficient-major and channel-minor
+ *                  (c0.r c0.g c0.b c1.r ...), cut into float4 planes; plane j of
+ *                  Gaussian i is sh[(j*n + i)*4 .. +3]; unused tail lanes are zero.
+ *                  (16-byte aligned) */
+typedef struct gs_params {
+    const float* means;
+    const float* quats;
+    const float* log_scales;
+    const float* opacity_logits;
+    const float* sh;
+    int32_t sh_degree;
+    int64_t n;
+} gs_params;
+
+/* Gradients of the same parameters, same layouts; written with +=. */
+typedef struct gs_param_grads {
+    float* means;
+    float* quats;
+    float* log_scales;
+    float* opacity_logits;
+    float* sh;
+} gs_param_grads;
+
+/* Per-Gaussian projection results (written by gs_project, read by the later
+ * calls).  A culled Gaussian has radius 0, tiles_touched 0 and zero features.
+ *   xy            [n][2]  pixel position (u, v) of the mean        (8-byte aligned)
+ *   depth         [n]     camera-space z                           (4-byte aligned)
+ *   conic_opacity [n][4]  A, B, C of the inverse 2D covariance, so that
+ *                         sigma = 1/2 (A dx^2 + C dy^2) + B dx dy, and the
+ *                         opacity o                                 (16-byte aligned)
+ *   rgb           [n][4]  colour r, g, b, 0                        (16-byte aligned)
+ *   radius        [n]     ceil(3 sqrt(largest eigenvalue)) in pixels
+ *   rect          [n][4]  tile rectangle xmin, ymin, xmax, ymax (max exclusive),
+ *                         uint16                                   (8-byte aligned)
+ *   tiles_touched [n]     (xmax - xmin) * (ymax - ymin)            (4-byte aligned) */
+typedef struct gs_projected {
+    float* xy;
+    float* depth;
+    float* conic_opacity;
+    float* rgb;
+    int32_t* radius;
+    uint16_t* rect;
+    uint32_t* tiles_touched;
+} gs_projected;
+
+/* Gradients with respect to the projected features, written by gs_raster_bwd (+=):
+ *   xy            [n][2]  dL/du, dL/dv                              (8-byte aligned)
+ *   conic_opacity [n][4]  dL/dA, dL/dB, dL/dC, dL/do                (16-byte aligned)
+ *   rgb           [n][4]  dL/dr, dL/dg, dL/db, 0                    (16-byte aligned) */
+typedef struct gs_grad2d {
+    float* xy;
+    float* conic_opacity;
+    float* rgb;
+} gs_grad2d;
+
+/* Text for a status code (static storage). */
+const char* gs_status_string(gs_status status);
+
+/* Description of the last failure on the calling thread ("" if none). */
+const char* gs_last_error_detail(void);
+
+/* Number of float4 planes of the SH array for a degree (1, 3, 7, 12 for 0..3;
+ * 0 for an unsupported degree). */
+int32_t gs_sh_planes(int32_t sh_degree);
+
+/* Tile grid of a camera: ceil(width / 16) x ceil(height / 16). */
+gs_status gs_tile_grid(const gs_camera* cam, int32_t* tiles_x_host, int32_t* tiles_y_host);
+
+/* gs_project -- stages 1 and 2 of the pipeline (gsplat guide §2.1) for every
+ * Gaussian: camera-space mean, 3D covariance R S S^T R^T from the normalised
+ * quaternion and exp(log_scale), EWA projection J W Sigma W^T J^T + eps2d I with
+ * the perspective Jacobian J (x/z and y/z clamped to 1.3 times the half field of
+ * view), its inverse (conic), the 3-sigma radius and tile rectangle, sigmoid
+ * opacity, and the colour from real spherical harmonics of the viewing direction
+ * (mean minus camera centre), offset by 0.5 and clamped at 0.  Culled: non-finite
+ * parameters, a zero quaternion, depth <= near_plane, a non-positive 2D
+ * determinant, an empty rectangle, a non-finite colour.
+ * Arithmetic is double precision; outputs are rounded to float32. */
+gs_status gs_project(const gs_params* params, const gs_camera* cam, gs_projected* out, void* stream);
+
+/* Bytes of device workspace gs_bin_sort needs for n Gaussians and up to `capacity`
+ * instances (16-byte aligned buffer, owned by the caller). */
+size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam);
+
+/* gs_bin_sort -- tile binning.  Every visible Gaussian emits one instance per tile
+ * of its rectangle, key = (ty * tiles_x + tx) << 32 | float32 bits of its depth,
+ * value = Gaussian index; the instances are sorted by key with a stable LSD radix
+ * sort over the low 32 + ceil(log2(tiles)) key bits (equal keys keep ascending
+ * Gaussian index), and tile_ranges[2t], [2t+1] receive the [begin, end) of tile t
+ * in the sorted list ([0, 0) when empty).
+ *   keys [capacity] (8-byte aligned), vals [capacity] (4-byte aligned),
+ *   tile_ranges [tiles][2] uint32 (8-byte aligned), workspace as sized above.
+ * *num_instances_host receives K, the instance count.  K > capacity returns
+ * GS_ERR_CAPACITY with nothing else written; call again with a larger buffer. */
+gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                      size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                      int64_t* num_instances_host, uint32_t* tile_ranges, void* stream);
+
+/* gs_raster_fwd -- stage 3 (gsplat guide §2.1), one CTA per 16x16 tile.  For each
+ * pixel, front to back over its tile's sorted list: sigma as above with
+ * d = (u, v) - pixel centre; entries with sigma < 0 are skipped;
+ * alpha = min(0.99, o exp(-sigma)); entries with alpha < 1/255 are skipped; if
+ * T (1 - alpha) < 1e-4 the pixel stops without blending that entry; otherwise
+ * C += rgb alpha T and T *= 1 - alpha.
+ *   image   [H][W][3] = C + T bg (bg_host: 3 floats read during the call)
+ *   final_T [H][W]    transmittance after the last blended entry
+ *   n_contrib [H][W]  1 + list position of the last blended entry (0 if none) */
+gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const gs_camera* cam, const float* bg_host, float* image, float* final_T,
+                        int32_t* n_contrib, void* stream);
+
+/* gs_raster_bwd -- the reverse of gs_raster_fwd for an upstream dL/dimage
+ * [H][W][3]: per pixel, back to front from n_contrib, the transmittance in front
+ * of each blended entry is recovered from final_T, and with S the colour blended
+ * behind the entry (normalised by the transmittance just behind it):
+ *   dL/drgb   += alpha T g
+ *   dL/dalpha  = sum_c g_c (T (rgb_c - S_c) - final_T bg_c / (1 - alpha))
+ * then through alpha = o exp(-sigma) (nothing when alpha was clamped at 0.99) to
+ * o, to (u, v) and to (A, B, C).  Per-Gaussian sums are reduced across each warp
+ * with shuffles before one vector atomic add per warp.  grad2d is accumulated. */
+gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const gs_camera* cam, const float* bg_host, const float* final_T,
+                        const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream);
+
+/* gs_project_bwd -- chain grad2d through gs_project to the parameters (+= into
+ * grads), in double precision: colour to SH coefficients (zero where the colour
+ * was clamped) and to the mean through the viewing direction; (u, v) to the mean;
+ * the conic through the 2x2 inverse, the EWA product and the Jacobian to the mean,
+ * the log-scales and the quaternion (through its normalisation); opacity to its
+ * logit.  Culled Gaussians get nothing.  When densify_accum and densify_count are
+ * non-NULL, every visible Gaussian also gets densify_accum += |(dL/du, dL/dv)| and
+ * densify_count += 1 (the screen-space mean-gradient statistic that adaptive
+ * density control thresholds, gsplat guide §4.1).  [n] floats / int32. */
+gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
+                         const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
+                         int32_t* densify_count, void* stream);
+
+/* gs_adam -- one bias-corrected Adam step on `count` floats (gsplat guide §4.2:
+ * one call per parameter group with its own lr; betas 0.9, 0.99; eps 1e-15):
+ *   m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2;
+ *   param -= lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps).
+ * step >= 1.  All four arrays 16-byte aligned. */
+gs_status gs_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
+                  float beta2, float eps, int32_t step, void* stream);
+
+/* gs_l1_loss_grad -- the L1 photometric term of the gsplat guide §4.1 over `count`
+ * values: dL_dimage = sign(image - target) / count (sign(0) = 0), and
+ * *loss_dev += mean |image - target| (one double on the device).
+ * image, target, dL_dimage 16-byte aligned; loss_dev 8-byte aligned. */
+gs_status gs_l1_loss_grad(const float* image, const float* target, int64_t count, float* dL_dimage,
+                          double* loss_dev, void* stream);
+
+/* Number of CUDA kernels this library has launched in the calling process
+ * (a diagnostic counter, incremented on the host at every launch). */
+uint64_t gs_kernel_launches(void);
+
+/* gs_zero -- set `bytes` bytes at `ptr` to zero on the stream (clears the
+ * accumulated gradient outputs between steps; a memset, nothing allocated). */
+gs_status gs_zero(void* ptr, size_t bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GS_H */

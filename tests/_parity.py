@@ -1,0 +1,167 @@
+"""Helpers shared by the parity tests: run the CUDA path through the C ABI, run the
+oracle on the same seeded inputs, and compare with the stated tolerances.
+
+Tolerances (fp32 CUDA path against the double-precision oracle):
+  * integers (radius, rectangle, tiles touched, keys, values, ranges, n_contrib
+    on unambiguous pixels): bit-exact;
+  * projected float32 features: at most 1 ulp apart (both sides compute in
+    double and round once; a 1-ulp difference only when an exp() result differs
+    in its last bit and straddles a float32 rounding boundary);
+  * image and final transmittance: 1e-5 absolute on pixels with no compositing
+    decision inside the ambiguity band (alpha within 1e-5 relative of 1/255,
+    T(1-alpha) within 1e-4 relative of 1e-4);
+  * gradients: |gpu - ref| <= 1e-6 + 1e-4 |ref| per element, on Gaussians that
+    touch no ambiguous pixel.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+
+BAND_ALPHA = 1e-5
+BAND_T = 1e-4
+IMG_TOL = 1e-5
+G_RTOL = 1e-4
+G_ATOL = 1e-6
+
+
+def ulp_diff(a, b):
+    """Distance in float32 ulps (0 for equal values, treating +0 == -0)."""
+    a = np.asarray(a, np.float32).copy()
+    b = np.asarray(b, np.float32).copy()
+    a[a == 0] = 0.0
+    b[b == 0] = 0.0
+    ia = a.view(np.int32).astype(np.int64)
+    ib = b.view(np.int32).astype(np.int64)
+    ia = np.where(ia < 0, -(ia & 0x7fffffff), ia)
+    ib = np.where(ib < 0, -(ib & 0x7fffffff), ib)
+    return np.abs(ia - ib)
+
+
+class GpuRun:
+    """Forward (and optionally backward) of one view through the C ABI."""
+
+    def __init__(self, scene, cam, bg=(0.0, 0.0, 0.0), capacity=0):
+        self.scene = scene
+        self.cam = cam
+        self.bg = bg
+        self.g = pl.Gaussians.from_scene(scene)
+        self.view = pl.View(scene.n, cam, capacity=capacity)
+        self.proj = pl.Projected(scene.n)
+        pl.project(self.g, self.view, self.proj)
+        self.K = pl.bin_sort(self.proj, self.view)
+        pl.raster_fwd(self.proj, self.view, bg)
+        torch.cuda.synchronize()
+
+    def projection(self) -> dict:
+        p = self.proj
+        rect = p.rect.cpu().numpy().astype(np.int32) & 0xffff
+        return {"xy": p.xy.cpu().numpy(), "depth": p.depth.cpu().numpy(),
+                "conic": p.conic_opacity[:, :3].cpu().numpy(), "opacity": p.conic_opacity[:, 3].cpu().numpy(),
+                "rgb": p.rgb[:, :3].cpu().numpy(), "radius": p.radius.cpu().numpy(), "rect": rect,
+                "tiles_touched": p.tiles_touched.cpu().numpy().astype(np.uint32)}
+
+    def sorted_instances(self):
+        K = self.K
+        keys = self.view.keys[:K].cpu().numpy().view(np.uint64)
+        vals = self.view.vals[:K].cpu().numpy().view(np.uint32)
+        ranges = self.view.ranges.cpu().numpy().view(np.uint32)
+        return keys, vals, ranges
+
+    def images(self):
+        return (self.view.image.cpu().numpy().reshape(-1, 3), self.view.final_T.cpu().numpy().reshape(-1),
+                self.view.n_contrib.cpu().numpy().reshape(-1))
+
+    def backward(self, dL_dimage: np.ndarray):
+        """Raster backward for an upstream [H,W,3] gradient; returns grad2d rows [n,9]."""
+        self.view.dL_dimage.copy_(torch.from_numpy(np.ascontiguousarray(dL_dimage, np.float32)))
+        self.g2 = pl.Grad2D(self.scene.n)
+        pl.raster_bwd(self.proj, self.view, self.g2, self.bg)
+        torch.cuda.synchronize()
+        return self.g2.as_rows()
+
+    def project_bwd(self, grad2d_rows: np.ndarray, densify=False):
+        """Project backward from given 2D gradient rows [n,9]; returns natural-layout grads."""
+        n = self.scene.n
+        g2 = pl.Grad2D(n)
+        rows = np.asarray(grad2d_rows, np.float32)
+        g2.xy.copy_(torch.from_numpy(np.ascontiguousarray(rows[:, 0:2])))
+        g2.conic_opacity.copy_(torch.from_numpy(np.ascontiguousarray(rows[:, 2:6])))
+        rgb = np.zeros((n, 4), np.float32)
+        rgb[:, :3] = rows[:, 6:9]
+        g2.rgb.copy_(torch.from_numpy(rgb))
+        grads = self.g.zeros_like()
+        acc = torch.zeros((n,), device="cuda", dtype=torch.float32) if densify else None
+        cnt = torch.zeros((n,), device="cuda", dtype=torch.int32) if densify else None
+        pl.project_bwd(self.g, self.view, self.proj, g2, grads, acc, cnt)
+        torch.cuda.synchronize()
+        out = grads.to_numpy()
+        if densify:
+            out["densify_accum"] = acc.cpu().numpy()
+            out["densify_count"] = cnt.cpu().numpy()
+        return out
+
+
+def check_projection(gpu: dict, ref: dict, idx=None):
+    sel = (lambda a: a) if idx is None else (lambda a: a[idx])
+    assert np.array_equal(sel(gpu["radius"]), ref["radius"])
+    assert np.array_equal(sel(gpu["rect"]), ref["rect"])
+    assert np.array_equal(sel(gpu["tiles_touched"]), ref["tiles_touched"])
+    for k in ("xy", "depth", "conic", "opacity", "rgb"):
+        d = ulp_diff(sel(gpu[k]), ref[k])
+        assert d.max(initial=0) <= 1, (k, int(d.max()), int((d > 1).sum()))
+    # the sort key uses the depth bits: they must be identical
+    assert np.array_equal(np.float32(sel(gpu["depth"])).view(np.uint32), np.float32(ref["depth"]).view(np.uint32))
+
+
+def check_images(gpu_img, gpu_T, gpu_nc, ref_img, ref_T, ref_nc, amb, max_amb_frac=1e-3):
+    ok = amb == 0
+    n_amb = int((~ok).sum())
+    assert n_amb <= max(2, max_amb_frac * len(amb)), f"{n_amb} ambiguous pixels of {len(amb)}"
+    err = np.abs(gpu_img[ok] - ref_img[ok])
+    assert err.max(initial=0.0) <= IMG_TOL, f"image max err {err.max()}"
+    errT = np.abs(gpu_T[ok] - ref_T[ok])
+    assert errT.max(initial=0.0) <= IMG_TOL, f"final_T max err {errT.max()}"
+    assert np.array_equal(gpu_nc[ok], ref_nc[ok]), int((gpu_nc[ok] != ref_nc[ok]).sum())
+    return float(err.max(initial=0.0)), n_amb
+
+
+def grad_mismatch(gpu, ref, rtol=G_RTOL, atol=G_ATOL):
+    """Boolean mask of elements outside |gpu - ref| <= atol + rtol |ref|."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return np.abs(gpu - ref) > atol + rtol * np.abs(ref)
+
+
+# A float32 sum of m terms t_i carries an error up to about c * eps32 * sum|t_i|
+# (c grows with the depth of the summation tree and the rounding of each term);
+# an element whose reference is a cancellation (sum|t_i| >> |sum t_i|) can miss
+# the relative tolerance by that much.  SUM_BOUND is c * eps32 with c = 64.
+SUM_BOUND = 64 * float(np.finfo(np.float32).eps)
+
+
+def check_grads(gpu, ref, name, rows=None, ref_abs=None, max_bad_frac=0.0):
+    """Elementwise gradient tolerance |gpu - ref| <= 1e-6 + 1e-4 |ref|.  An element
+    outside it is accepted only when ref_abs (the reference's sum of |terms|)
+    is given and |gpu - ref| <= SUM_BOUND * ref_abs, and only for up to
+    max_bad_frac of the elements; their count is reported."""
+    g = np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    if rows is not None:
+        g, r = g[rows], r[rows]
+        ref_abs = None if ref_abs is None else np.asarray(ref_abs)[rows]
+    bad = grad_mismatch(g, r)
+    nbad = int(bad.sum())
+    if nbad:
+        d = np.abs(g - r)
+        bounded = np.zeros_like(bad) if ref_abs is None else d <= G_ATOL + SUM_BOUND * np.abs(ref_abs)
+        explained = bad & bounded
+        worst = np.argmax(d * bad)
+        ratio = (np.abs(ref_abs).flat[worst] / max(abs(r.flat[worst]), 1e-30)) if ref_abs is not None else float("nan")
+        msg = (f"{name}: {nbad}/{bad.size} outside tol, {int(explained.sum())} within the float32 summation "
+               f"bound; worst gpu={g.flat[worst]!r} ref={r.flat[worst]!r} sum|t|/|ref|={ratio:.3g}")
+        assert nbad == int(explained.sum()) and nbad <= max_bad_frac * bad.size, msg
+        print(f"  {msg}")
+    return nbad

@@ -1,0 +1,129 @@
+"""Host-side checks of the C ABI (no GPU needed): libgs.so loads, exports every
+function include/gs.h declares, and rejects bad arguments before it touches
+the device."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gs.h")
+
+
+@pytest.fixture(scope="module")
+def gs():
+    from gaussian_splatting_differentiable_02_b200 import build
+    build.build()
+    from gaussian_splatting_differentiable_02_b200 import abi
+    abi.lib()
+    return abi
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gs_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for f in ("gs_project", "gs_bin_sort", "gs_raster_fwd", "gs_raster_bwd", "gs_project_bwd", "gs_adam"):
+        assert f in names
+
+
+def test_library_exports_every_declared_function(gs):
+    out = subprocess.run(["nm", "-D", "--defined-only", gs.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gs_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    # the binding covers every declared function with the same name
+    assert set(declared_functions()) == set(gs.SIGNATURES)
+    for f in declared_functions():
+        assert hasattr(gs, f)
+
+
+def test_status_strings(gs):
+    for code in range(5):
+        assert gs.gs_status_string(code).startswith("GS_")
+    assert "unknown" in gs.gs_status_string(99)
+
+
+def test_sh_planes(gs):
+    assert [gs.gs_sh_planes(d) for d in range(5)] == [1, 3, 7, 12, 0]
+
+
+def cam(**kw):
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    c = dict(scenes.tiny().cameras[0])
+    c.update(kw)
+    return c
+
+
+def test_tile_grid_and_camera_checks(gs):
+    assert gs.gs_tile_grid(gs.make_camera(cam())) == (8, 8)
+    assert gs.gs_tile_grid(gs.make_camera(cam(width=100, height=37))) == (7, 3)
+    with pytest.raises(gs.GsError) as e:
+        gs.gs_tile_grid(gs.make_camera(cam(width=0)))
+    assert e.value.status == gs.GS_ERR_UNSUPPORTED
+    with pytest.raises(gs.GsError) as e:
+        gs.gs_tile_grid(gs.make_camera(cam(width=20000)))
+    assert e.value.status == gs.GS_ERR_UNSUPPORTED
+    with pytest.raises(gs.GsError) as e:
+        gs.gs_tile_grid(gs.make_camera(cam(fx=-1.0)))
+    assert e.value.status == gs.GS_ERR_INVALID_ARG
+    with pytest.raises(gs.GsError) as e:
+        gs.gs_tile_grid(gs.make_camera(cam(near=0.0)))
+    assert e.value.status == gs.GS_ERR_INVALID_ARG
+
+
+def test_invalid_arguments_rejected_before_launch(gs):
+    L = gs.lib()
+    c = gs.make_camera(cam())
+    out = gs.gs_projected()
+    # NULL params
+    assert L.gs_project(None, C.byref(c), C.byref(out), None) == gs.GS_ERR_INVALID_ARG
+    # unsupported SH degree
+    p = gs.gs_params(16, 16, 16, 16, 16, 4, 10)
+    assert L.gs_project(C.byref(p), C.byref(c), C.byref(out), None) == gs.GS_ERR_UNSUPPORTED
+    assert "SH degree" in gs.gs_last_error_detail()
+    # misaligned means
+    p = gs.gs_params(16 + 4, 16, 16, 16, 16, 0, 10)
+    assert L.gs_project(C.byref(p), C.byref(c), C.byref(out), None) == gs.GS_ERR_INVALID_ARG
+    assert "aligned" in gs.gs_last_error_detail()
+    # negative n
+    p = gs.gs_params(16, 16, 16, 16, 16, 0, -1)
+    assert L.gs_project(C.byref(p), C.byref(c), C.byref(out), None) == gs.GS_ERR_INVALID_ARG
+    # NULL outputs of the projection
+    p = gs.gs_params(16, 16, 16, 16, 16, 0, 10)
+    assert L.gs_project(C.byref(p), C.byref(c), C.byref(out), None) == gs.GS_ERR_INVALID_ARG
+    # Adam: step 0, misaligned buffers
+    assert L.gs_adam(16, 16, 16, 16, 8, 1e-3, 0.9, 0.99, 1e-15, 0, None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_adam(18, 16, 16, 16, 8, 1e-3, 0.9, 0.99, 1e-15, 1, None) == gs.GS_ERR_INVALID_ARG
+    # bin sort: workspace too small, capacity out of range
+    K = C.c_int64()
+    proj = gs.gs_projected(16, 16, 16, 16, 16, 16, 16)
+    assert L.gs_bin_sort(C.byref(proj), 10, C.byref(c), 256, 16, 256, 256, 100, C.byref(K), 256, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "workspace" in gs.gs_last_error_detail()
+    assert L.gs_bin_sort(C.byref(proj), 10, C.byref(c), 256, 1 << 30, 256, 256, -5, C.byref(K), 256, None) == \
+        gs.GS_ERR_INVALID_ARG
+    # densify buffers must come in pairs
+    g2 = gs.gs_grad2d(16, 16, 16)
+    gr = gs.gs_param_grads(16, 16, 16, 16, 16)
+    p = gs.gs_params(16, 16, 16, 16, 16, 0, 10)
+    assert L.gs_project_bwd(C.byref(p), C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr), 256, None, None) == \
+        gs.GS_ERR_INVALID_ARG
+    # zero-size work needs no pointers and launches nothing
+    assert L.gs_adam(None, None, None, None, 0, 1e-3, 0.9, 0.99, 1e-15, 1, None) == gs.GS_OK
+    assert L.gs_l1_loss_grad(None, None, 0, None, None, None) == gs.GS_OK
+    assert L.gs_zero(None, 0, None) == gs.GS_OK
+
+
+def test_workspace_grows_with_capacity(gs):
+    c = gs.make_camera(cam())
+    a = gs.gs_bin_sort_workspace_bytes(1000, 10_000, c)
+    b = gs.gs_bin_sort_workspace_bytes(1000, 1_000_000, c)
+    assert 0 < a < b
+    assert b >= 12 * 1_000_000          # the ping-pong key/value copy
