@@ -66,6 +66,8 @@ SIGNATURES = {
     "gs_bin_sort_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.POINTER(gs_camera)]),
     "gs_bin_sort": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, C.c_size_t, _P, _P,
                                 C.c_int64, C.POINTER(C.c_int64), _P, _P]),
+    "gs_bin_sort_static": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, _P, C.c_int64,
+                                       C.POINTER(C.c_int64), _P, _P]),
     "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
                                   _P, _P, _P]),
     "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
@@ -152,6 +154,21 @@ def gs_bin_sort(proj: gs_projected, n: int, cam: gs_camera, workspace: int, work
     K = C.c_int64(0)
     st = lib().gs_bin_sort(C.byref(proj), n, C.byref(cam), workspace, workspace_bytes, keys, vals, capacity,
                            C.byref(K), tile_ranges, stream)
+    if check or st not in (GS_OK, GS_ERR_CAPACITY):
+        _check(st)
+    return st, K.value
+
+
+GS_STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def gs_bin_sort_static(proj: gs_projected, n: int, cam: gs_camera, keys: int, vals: int, capacity: int,
+                       tile_ranges: int, stream: int = 0, check: bool = True):
+    """gs_bin_sort with the library's static scratch instead of a caller workspace
+    (for callers that cannot allocate device memory).  Returns (status, K)."""
+    K = C.c_int64(0)
+    st = lib().gs_bin_sort_static(C.byref(proj), n, C.byref(cam), keys, vals, capacity, C.byref(K), tile_ranges,
+                                  stream)
     if check or st not in (GS_OK, GS_ERR_CAPACITY):
         _check(st)
     return st, K.value

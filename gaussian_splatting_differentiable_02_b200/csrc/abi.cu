@@ -55,6 +55,18 @@ gs_status ok() {
     return GS_OK;
 }
 
+}  // namespace
+
+gs_status gsk::fail_detail(gs_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+namespace {
+
 gs_status cuda_status(cudaError_t e, const char* where) {
     if (e == cudaSuccess) return ok();
     return fail(GS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));

@@ -81,6 +81,9 @@ cudaError_t launch_l1(const float* image, const float* target, int64_t count, fl
 // host-side count of kernel launches (gs_kernel_launches)
 void count_launches(int k);
 
+// record a failure for gs_last_error_detail() and return `st`
+gs_status fail_detail(gs_status st, const char* fmt, ...);
+
 // grid size: a multiple of the SM count, capped by the work
 inline unsigned grid_for(int64_t work, int block, int per_sm = 8) {
     int64_t g = (work + block - 1) / block;

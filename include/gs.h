@@ -168,6 +168,30 @@ gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam,
                       size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
                       int64_t* num_instances_host, uint32_t* tile_ranges, void* stream);
 
+/* Size of the device array gs_bin_sort_static uses as its workspace (32 MiB). */
+#define GS_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* gs_bin_sort_static -- gs_bin_sort for callers that cannot allocate device
+ * memory.  The paper has no counterpart: it is an interface for hosts that own
+ * the whole device budget, frame loops where a cudaMalloc would stall every
+ * stream, and foreign runtimes that can pass device pointers but cannot
+ * allocate.  Same arguments and results as gs_bin_sort minus the workspace,
+ * which is a library-owned device array of GS_STATIC_SCRATCH_BYTES held on
+ * every device that loads the library until the process exits.
+ *   - n and capacity whose workspace (gs_bin_sort_workspace_bytes) exceeds
+ *     GS_STATIC_SCRATCH_BYTES return GS_ERR_UNSUPPORTED (about 2.7 million
+ *     instances for a million Gaussians).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the array.  Calls whose GPU work overlaps (other streams,
+ *     other threads on the same device) race on it: serialise them.  No state
+ *     carries over between calls; nothing in it needs clearing.
+ *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call). */
+gs_status gs_bin_sort_static(const gs_projected* proj, int64_t n, const gs_camera* cam, uint64_t* keys,
+                             uint32_t* vals, int64_t capacity, int64_t* num_instances_host, uint32_t* tile_ranges,
+                             void* stream);
+
 /* gs_raster_fwd -- stage 3 (gsplat guide §2.1), one CTA per 16x16 tile.  For each
  * pixel, front to back over its tile's sorted list: sigma as above with
  * d = (u, v) - pixel centre; entries with sigma < 0 are skipped;
