@@ -1,18 +1,30 @@
-// gs_bin_sort: tile binning with a (tile_id << 32 | depth) key and a stable LSD
-// radix sort (the "culling and reordering" stage the MUSA co-design article,
-// qwbw.cn/news/278220 §1, lists among the four 3DGS bottlenecks; the packed
-// screen-space ordering of the gsplat guide, lmnt.cn/news/262699 §4.1).
+// gs_bin_sort: tile binning with a (tile_id << 32 | depth) key (the "culling and
+// reordering" stage the MUSA co-design article, qwbw.cn/news/278220 §1, lists
+// among the four 3DGS bottlenecks; the screen-space ordering of the gsplat
+// guide, lmnt.cn/news/262699 §4.1).
+//
+// The result is the list of instances sorted by (key, Gaussian index).  It is
+// produced without sorting 64-bit keys: the Gaussians are first sorted by depth
+// (a stable LSD radix sort of N 32-bit keys, culled Gaussians last), instances
+// are emitted in that order as 32-bit (tile, gid) pairs, and a stable LSD radix
+// sort over the tile bits alone finishes the job, since a stable sort by tile
+// of a sequence ordered by (depth, gid) is ordered by (tile, depth, gid).  The
+// last tile pass writes the 64-bit key, taking the depth bits from the
+// Gaussian.  This moves about a third of the bytes of a 64-bit key sort.
 //
 // Kernels (no kernel waits on another block, so nothing here can spin):
-//   count_kernel      per-block sum of tiles_touched
+//   depth_keys        key = float32 bits of the depth (culled: 0xffffffff), val = gid
+//   upsweep           per-block 256-bin histogram of one 8-bit digit
+//   scan_hist         per digit: exclusive scan of the block histograms
+//   downsweep         stable rank of every element among equal digits of its
+//                     block (warp match + per-warp counters), reorder in shared
+//                     memory, coalesced scatter; the final tile pass writes
+//                     64-bit keys
+//   count_sorted      per-block sum of tiles_touched in depth order
 //   scan_blocks       one CTA: exclusive scan of the block sums, total K
-//   emit_kernel       per block: in-block scan, then every visible Gaussian
-//                     writes its (key, gid) instances, row-major over its rect
-//   upsweep_kernel    per-block 256-bin digit histogram of one 8-bit digit
-//   scan_hist_kernel  per digit: exclusive scan of the block histograms
-//   downsweep_kernel  stable rank of every element among equal digits of its
-//                     block (warp match + per-warp counters), scatter
-//   ranges_kernel     [begin, end) of each tile in the sorted keys
+//   emit              every visible Gaussian, in depth order, writes its
+//                     instances (row-major over its tile rectangle)
+//   ranges            [begin, end) of each tile in the sorted keys
 #include "internal.cuh"
 
 namespace gsk {
@@ -58,63 +70,17 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, unsigned lon
     return before + inc - v;
 }
 
-__global__ void __launch_bounds__(kEmitBlock) count_kernel(const uint32_t* __restrict__ touched, int64_t n,
-                                                           unsigned long long* block_sums) {
-    const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
-    unsigned long long s = 0;
-    for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
-        const int64_t i = base + k;
-        if (i < n) s += __ldg(touched + i);
-    }
-    unsigned long long tot;
-    block_excl_scan(s, &tot);
-    if (threadIdx.x == 0) block_sums[blockIdx.x] = tot;
-}
-
-__global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
-                                                           unsigned long long* total) {
-    unsigned long long carry = 0;
-    for (int64_t base = 0; base < nb; base += 1024) {
-        const int64_t i = base + threadIdx.x;
-        const unsigned long long v = i < nb ? block_sums[i] : 0ull;
-        unsigned long long tot;
-        const unsigned long long ex = block_excl_scan(v, &tot);
-        if (i < nb) block_sums[i] = carry + ex;
-        carry += tot;
-    }
-    if (threadIdx.x == 0) *total = carry;
-}
-
-__global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
-                                                          const uint2* __restrict__ rect,
-                                                          const float* __restrict__ depth, int64_t n, int tiles_x,
-                                                          const unsigned long long* __restrict__ block_offsets,
-                                                          uint64_t* __restrict__ keys, uint32_t* __restrict__ vals) {
-    const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
-    unsigned long long mine = 0;
-#pragma unroll
-    for (int k = 0; k < kEmitPerThread; ++k)
-        if (first + k < n) mine += __ldg(touched + first + k);
-    unsigned long long tot;
-    unsigned long long off = block_excl_scan(mine, &tot) + block_offsets[blockIdx.x];
-    for (int k = 0; k < kEmitPerThread; ++k) {
-        const int64_t i = first + k;
-        if (i >= n) break;
-        if (__ldg(touched + i) == 0u) continue;
-        const uint2 r = __ldg(rect + i);
-        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, x1 = r.y & 0xffffu, y1 = r.y >> 16;
-        const uint64_t zb = __float_as_uint(__ldg(depth + i));
-        for (uint32_t ty = y0; ty < y1; ++ty)
-            for (uint32_t tx = x0; tx < x1; ++tx) {
-                keys[off] = (uint64_t(ty * uint32_t(tiles_x) + tx) << 32) | zb;
-                vals[off] = uint32_t(i);
-                ++off;
-            }
+__global__ void __launch_bounds__(256) depth_keys_kernel(const uint32_t* __restrict__ touched,
+                                                         const float* __restrict__ depth, int64_t n,
+                                                         uint32_t* __restrict__ keys, uint32_t* __restrict__ vals) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+        keys[i] = __ldg(touched + i) > 0u ? __float_as_uint(__ldg(depth + i)) : 0xffffffffu;
+        vals[i] = uint32_t(i);
     }
 }
 
-__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint64_t* __restrict__ keys, int64_t K, int shift,
-                                                             uint32_t* __restrict__ hist, int64_t nb) {
+__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __restrict__ keys, int64_t count,
+                                                             int shift, uint32_t* __restrict__ hist, int64_t nb) {
     __shared__ uint32_t h[kSortWarps][256];
     const int warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&h[0][0])[k] = 0u;
@@ -123,7 +89,7 @@ __global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint64_t* __r
 #pragma unroll 4
     for (int k = 0; k < kSortPerThread; ++k) {
         const int64_t e = base + int64_t(k) * kSortBlock + threadIdx.x;
-        if (e < K) atomicAdd(&h[warp][uint32_t(__ldg(keys + e) >> shift) & 0xffu], 1u);
+        if (e < count) atomicAdd(&h[warp][(__ldg(keys + e) >> shift) & 0xffu], 1u);
     }
     __syncthreads();
     for (int d = threadIdx.x; d < 256; d += kSortBlock) {
@@ -149,17 +115,23 @@ __global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t
     if (threadIdx.x == 0) digit_totals[blockIdx.x] = uint32_t(carry);
 }
 
-__global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint64_t* __restrict__ keys_in,
+// kFinal: write 64-bit keys (key32 << 32 | depth bits of the Gaussian) to keys_out64.
+template <bool kFinal>
+__global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* __restrict__ keys_in,
                                                                const uint32_t* __restrict__ vals_in,
-                                                               uint64_t* __restrict__ keys_out,
-                                                               uint32_t* __restrict__ vals_out, int64_t K, int shift,
-                                                               const uint32_t* __restrict__ hist, int64_t nb,
-                                                               const uint32_t* __restrict__ digit_totals) {
+                                                               uint32_t* __restrict__ keys_out,
+                                                               uint64_t* __restrict__ keys_out64,
+                                                               uint32_t* __restrict__ vals_out, int64_t count,
+                                                               int shift, const uint32_t* __restrict__ hist,
+                                                               int64_t nb, const uint32_t* __restrict__ digit_totals,
+                                                               const float* __restrict__ depth) {
     __shared__ uint32_t wcount[kSortWarps][256];
-    __shared__ uint32_t gbase[256];
+    __shared__ uint32_t gbase[256];   // global start of each digit's run from this block
+    __shared__ uint32_t lstart[256];  // start of each digit's run within the block
+    __shared__ uint32_t sk[kSortTile];
+    __shared__ uint32_t sv[kSortTile];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&wcount[0][0])[k] = 0u;
-    // digit base: exclusive prefix of the digit totals plus this block's offset
     {
         unsigned long long tot;
         const unsigned long long ex = block_excl_scan(threadIdx.x < 256 ? digit_totals[threadIdx.x] : 0u, &tot);
@@ -167,18 +139,17 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint64_t* _
     }
     __syncthreads();
 
-    const int64_t base = int64_t(blockIdx.x) * kSortTile + int64_t(warp) * kWarpSpan;
+    const int64_t tile0 = int64_t(blockIdx.x) * kSortTile;
+    const int64_t base = tile0 + int64_t(warp) * kWarpSpan;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    uint64_t key[kSortPerThread];
-    uint32_t val[kSortPerThread];
-    uint32_t rank[kSortPerThread];
+    uint32_t key[kSortPerThread], val[kSortPerThread], rank[kSortPerThread];
 #pragma unroll
     for (int r = 0; r < kSortPerThread; ++r) {
         const int64_t e = base + r * 32 + lane;
-        const bool in = e < K;
-        key[r] = in ? __ldg(keys_in + e) : 0ull;
+        const bool in = e < count;
+        key[r] = in ? __ldg(keys_in + e) : 0u;
         val[r] = in ? __ldg(vals_in + e) : 0u;
-        const uint32_t digit = in ? (uint32_t(key[r] >> shift) & 0xffu) : 256u;
+        const uint32_t digit = in ? ((key[r] >> shift) & 0xffu) : 256u;
         const uint32_t peers = __match_any_sync(0xffffffffu, digit);
         const uint32_t before = in ? wcount[warp][digit] : 0u;
         __syncwarp();
@@ -187,26 +158,103 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint64_t* _
         rank[r] = before + __popc(peers & lt_mask);
     }
     __syncthreads();
-    // exclusive prefix over warps for each digit
-    for (int d = threadIdx.x; d < 256; d += kSortBlock) {
-        uint32_t run = 0;
+    // per digit: block total, then the exclusive prefix over warps
+    uint32_t dtot = 0;
+    if (threadIdx.x < 256) {
 #pragma unroll
         for (int w = 0; w < kSortWarps; ++w) {
-            const uint32_t c = wcount[w][d];
-            wcount[w][d] = run;
-            run += c;
+            const uint32_t c = wcount[w][threadIdx.x];
+            wcount[w][threadIdx.x] = dtot;
+            dtot += c;
         }
     }
+    {
+        unsigned long long tot;
+        const unsigned long long ex = block_excl_scan(dtot, &tot);
+        if (threadIdx.x < 256) lstart[threadIdx.x] = uint32_t(ex);
+    }
     __syncthreads();
+    // reorder by digit inside the block (stable), then write runs out coalesced
 #pragma unroll
     for (int r = 0; r < kSortPerThread; ++r) {
         const int64_t e = base + r * 32 + lane;
-        if (e < K) {
-            const uint32_t digit = uint32_t(key[r] >> shift) & 0xffu;
-            const uint32_t pos = gbase[digit] + wcount[warp][digit] + rank[r];
-            keys_out[pos] = key[r];
-            vals_out[pos] = val[r];
+        if (e < count) {
+            const uint32_t digit = (key[r] >> shift) & 0xffu;
+            const uint32_t p = lstart[digit] + wcount[warp][digit] + rank[r];
+            sk[p] = key[r];
+            sv[p] = val[r];
         }
+    }
+    __syncthreads();
+    const int in_block = int(min(int64_t(kSortTile), count - tile0));
+    for (int p = threadIdx.x; p < in_block; p += kSortBlock) {
+        const uint32_t k = sk[p], v = sv[p];
+        const uint32_t digit = (k >> shift) & 0xffu;
+        const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
+        if (kFinal) {
+            keys_out64[g] = (uint64_t(k) << 32) | __float_as_uint(__ldg(depth + v));
+        } else {
+            keys_out[g] = k;
+        }
+        vals_out[g] = v;
+    }
+}
+
+__global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const uint32_t* __restrict__ touched,
+                                                                  const uint32_t* __restrict__ order, int64_t n,
+                                                                  unsigned long long* block_sums) {
+    const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
+    unsigned long long s = 0;
+    for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
+        const int64_t i = base + k;
+        if (i < n) s += __ldg(touched + __ldg(order + i));
+    }
+    unsigned long long tot;
+    block_excl_scan(s, &tot);
+    if (threadIdx.x == 0) block_sums[blockIdx.x] = tot;
+}
+
+__global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
+                                                           unsigned long long* total) {
+    unsigned long long carry = 0;
+    for (int64_t base = 0; base < nb; base += 1024) {
+        const int64_t i = base + threadIdx.x;
+        const unsigned long long v = i < nb ? block_sums[i] : 0ull;
+        unsigned long long tot;
+        const unsigned long long ex = block_excl_scan(v, &tot);
+        if (i < nb) block_sums[i] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) *total = carry;
+}
+
+__global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
+                                                          const uint2* __restrict__ rect,
+                                                          const uint32_t* __restrict__ order, int64_t n, int tiles_x,
+                                                          const unsigned long long* __restrict__ block_offsets,
+                                                          uint32_t* __restrict__ tkeys, uint32_t* __restrict__ tvals) {
+    const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
+    uint32_t gid[kEmitPerThread], tt[kEmitPerThread];
+    unsigned long long mine = 0;
+#pragma unroll
+    for (int k = 0; k < kEmitPerThread; ++k) {
+        gid[k] = first + k < n ? __ldg(order + first + k) : 0u;
+        tt[k] = first + k < n ? __ldg(touched + gid[k]) : 0u;
+        mine += tt[k];
+    }
+    unsigned long long tot;
+    unsigned long long off = block_excl_scan(mine, &tot) + block_offsets[blockIdx.x];
+#pragma unroll
+    for (int k = 0; k < kEmitPerThread; ++k) {
+        if (tt[k] == 0u) continue;
+        const uint2 r = __ldg(rect + gid[k]);
+        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, x1 = r.y & 0xffffu, y1 = r.y >> 16;
+        for (uint32_t ty = y0; ty < y1; ++ty)
+            for (uint32_t tx = x0; tx < x1; ++tx) {
+                tkeys[off] = ty * uint32_t(tiles_x) + tx;
+                tvals[off] = gid[k];
+                ++off;
+            }
     }
 }
 
@@ -221,11 +269,27 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict_
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
+// One LSD pass over `count` (key, val) pairs.  Final passes write 64-bit keys.
+void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout, uint64_t* kout64, uint32_t* vout,
+                int64_t count, int shift, const SortWorkspace& ws, const float* depth, cudaStream_t s) {
+    const int64_t nb = (count + kSortTile - 1) / kSortTile;
+    upsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(kin, count, shift, ws.hist, nb);
+    scan_hist_kernel<<<256, 1024, 0, s>>>(ws.hist, nb, ws.digit_totals);
+    if (kout64)
+        downsweep_kernel<true><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, count, shift,
+                                                                   ws.hist, nb, ws.digit_totals, depth);
+    else
+        downsweep_kernel<false><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, count, shift,
+                                                                    ws.hist, nb, ws.digit_totals, depth);
+    count_launches(3);
+}
+
 }  // namespace
 
 size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws) {
     const int64_t nb_emit = (n + kEmitChunk - 1) / kEmitChunk;
-    const int64_t nb_sort = (capacity + kSortTile - 1) / kSortTile;
+    const int64_t slots = capacity > n ? capacity : n;  // the depth sort borrows the tile buffers
+    const int64_t nb_sort = (slots + kSortTile - 1) / kSortTile;
     size_t off = 0;
     char* b = static_cast<char*>(base);
     SortWorkspace w;
@@ -235,10 +299,12 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
     off += align_up(sizeof(unsigned long long) * size_t(nb_emit > 0 ? nb_emit : 1));
     w.total = reinterpret_cast<unsigned long long*>(b + off);
     off += align_up(sizeof(unsigned long long));
-    w.keys_alt = reinterpret_cast<uint64_t*>(b + off);
-    off += align_up(sizeof(uint64_t) * size_t(capacity > 0 ? capacity : 1));
-    w.vals_alt = reinterpret_cast<uint32_t*>(b + off);
-    off += align_up(sizeof(uint32_t) * size_t(capacity > 0 ? capacity : 1));
+    for (int r = 0; r < 2; ++r) {
+        w.tkey[r] = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * size_t(slots > 0 ? slots : 1));
+        w.tval[r] = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * size_t(slots > 0 ? slots : 1));
+    }
     w.hist = reinterpret_cast<uint32_t*>(b + off);
     off += align_up(sizeof(uint32_t) * 256 * size_t(nb_sort > 0 ? nb_sort : 1));
     w.digit_totals = reinterpret_cast<uint32_t*>(b + off);
@@ -247,14 +313,23 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
     return off;
 }
 
+// Depth order of the Gaussians (into tkey/tval[1], so that tval[1] holds the
+// order while the instances are emitted into buffer 0), then the instance count.
 cudaError_t launch_count_instances(const gs_projected& proj, int64_t n, const SortWorkspace& ws, cudaStream_t s) {
-    if (n > 0) {
-        count_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, n, ws.block_sums);
-        scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total);
-        count_launches(2);
-    } else {
+    if (n == 0) {
         cudaMemsetAsync(ws.total, 0, sizeof(unsigned long long), s);
+        return cudaGetLastError();
     }
+    depth_keys_kernel<<<grid_for(n, 256, 8), 256, 0, s>>>(proj.tiles_touched, proj.depth, n, ws.tkey[1], ws.tval[1]);
+    count_launches(1);
+    for (int p = 0; p < 4; ++p) {  // 4 passes: the order ends in buffer 1 again
+        const int src = (p & 1) ? 0 : 1;
+        radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], n, 8 * p, ws, nullptr, s);
+    }
+    count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, ws.tval[1], n,
+                                                                    ws.block_sums);
+    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total);
+    count_launches(2);
     return cudaGetLastError();
 }
 
@@ -263,26 +338,18 @@ cudaError_t launch_emit_sort_ranges(const gs_projected& proj, int64_t n, const C
     const int64_t T = int64_t(cam.TX) * cam.TY;
     cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint32_t) * 2 * size_t(T), s);
     if (e != cudaSuccess || K == 0) return e;
-    const int key_bits = 32 + tile_bits(T);
-    const int passes = (key_bits + 7) / 8;
-    // emit into the buffer that makes the last pass land in `keys`
-    uint64_t* k_cur = (passes & 1) ? ws.keys_alt : keys;
-    uint32_t* v_cur = (passes & 1) ? ws.vals_alt : vals;
-    uint64_t* k_oth = (passes & 1) ? keys : ws.keys_alt;
-    uint32_t* v_oth = (passes & 1) ? vals : ws.vals_alt;
     emit_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, reinterpret_cast<const uint2*>(proj.rect),
-                                                            proj.depth, n, cam.TX, ws.block_sums, k_cur, v_cur);
+                                                            ws.tval[1], n, cam.TX, ws.block_sums, ws.tkey[0],
+                                                            ws.tval[0]);
     count_launches(1);
-    const int64_t nb = (K + kSortTile - 1) / kSortTile;
+    const int bits = tile_bits(T);
+    const int passes = bits > 0 ? (bits + 7) / 8 : 1;
+    int cur = 0;
     for (int p = 0; p < passes; ++p) {
-        const int shift = 8 * p;
-        upsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(k_cur, K, shift, ws.hist, nb);
-        scan_hist_kernel<<<256, 1024, 0, s>>>(ws.hist, nb, ws.digit_totals);
-        downsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(k_cur, v_cur, k_oth, v_oth, K, shift, ws.hist, nb,
-                                                             ws.digit_totals);
-        count_launches(3);
-        uint64_t* tk = k_cur; k_cur = k_oth; k_oth = tk;
-        uint32_t* tv = v_cur; v_cur = v_oth; v_oth = tv;
+        const bool last = p == passes - 1;
+        radix_pass(ws.tkey[cur], ws.tval[cur], last ? nullptr : ws.tkey[cur ^ 1], last ? keys : nullptr,
+                   last ? vals : ws.tval[cur ^ 1], K, 8 * p, ws, proj.depth, s);
+        cur ^= 1;
     }
     ranges_kernel<<<grid_for(K, 256, 8), 256, 0, s>>>(keys, K, reinterpret_cast<uint2*>(ranges));
     count_launches(1);

@@ -52,8 +52,8 @@ cudaError_t launch_project_bwd(const gs_params& p, const CamArgs& cam, const gs_
 struct SortWorkspace {
     unsigned long long* block_sums;  // [nb_emit]
     unsigned long long* total;       // [1]
-    uint64_t* keys_alt;              // [capacity]
-    uint32_t* vals_alt;              // [capacity]
+    uint32_t* tkey[2];               // [max(capacity, n)] 32-bit keys, ping-pong
+    uint32_t* tval[2];               // [max(capacity, n)] Gaussian indices, ping-pong
     uint32_t* hist;                  // [256][nb_sort]
     uint32_t* digit_totals;          // [256]
     int64_t nb_emit, nb_sort;

@@ -3,18 +3,35 @@
 // §2.1: shared-memory prefetch of the tile's Gaussians, SoA features, warp-level
 // synchronisation; §2.2: a standalone backward entry).
 //
-// One CTA per tile, one pixel per thread.  Each batch of up to 256 list entries
-// is gathered by Gaussian index into shared memory with cp.async (16-byte
-// LDGSTS), double-buffered so the next batch is in flight while the current one
-// is composited.  Both passes evaluate alpha with the same inline function and
-// explicit rounding intrinsics, so the backward pass makes exactly the skip and
-// clamp decisions the forward pass made.
+// Work decomposition: one warp per tile, each lane owns a column of 8 pixels
+// (lane & 15 selects the column, lane >> 4 the upper or lower half), four tiles
+// per block.  The warp walks its tile's sorted list in batches of 32 entries:
+// every lane gathers one entry's 40 bytes (xy, conic + opacity, colour) by
+// Gaussian index into shared memory with cp.async, double-buffered so the next
+// batch is in flight while the current one is composited; the lane that
+// gathered an entry also derives its per-entry constants.  Every lane then
+// reads each entry once (broadcast loads) and applies it to its 8 pixels, whose
+// terms that depend only on dx are shared.  No block-wide barrier is used:
+// warps synchronise with __syncwarp and finish independently.
+//
+// Forward: a warp stops as soon as all 256 pixels have terminated (warp vote
+// per entry).  Backward: back to front from the largest n_contrib of the tile;
+// each lane sums its 8 pixels' contributions, the 9 per-Gaussian sums are
+// reduce-scattered across the warp (18 shuffles) and three lanes issue one
+// float2 / float4 atomic add each (batched atomics, MUSA co-design article
+// qwbw.cn/news/278220 §2.2).  The gradient with respect to (u, v, A, B, C) is
+// accumulated as three moments of dL/dsigma over the lane's pixels, then
+// combined with dx and the conic once per entry.
+//
+// Both passes evaluate alpha with the same inline code built from explicit
+// rounding intrinsics, so the backward pass repeats the forward pass's skip and
+// clamp decisions exactly.
 //
 // Conditioning: sigma = 1/2 (A dx^2 + C dy^2) + B dx dy cancels badly far along
 // the long axis of a needle-shaped Gaussian (the terms grow with the condition
-// number of the conic).  Entries whose conic has a condition number above
-// kCondMax evaluate the quadratic form (and its derivatives in the backward pass)
-// in double; the rest stay in float32, where the error is a few ulp of sigma.
+// number of the conic).  Entries whose conic has an eigenvalue ratio above 8
+// evaluate the quadratic form, and in the backward pass dsigma/du and
+// dsigma/dv, per pixel in double; the rest stay float32.
 #include "internal.cuh"
 
 namespace gsk {
@@ -25,17 +42,35 @@ constexpr float kAlphaMin = 1.0f / 255.0f;
 constexpr float kTMin = 1e-4f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr double kLog2eD = 1.4426950408889634;
-// trace^2 / det = kappa + 1/kappa + 2 for the eigenvalue ratio kappa; 8 -> 10.125
+// trace^2 / det = kappa + 1/kappa + 2 for the eigenvalue ratio kappa; kappa = 8 -> 10.125
 constexpr float kCondMaxTraceSqOverDet = 10.125f;
 
-constexpr int kBlock = kTilePixels;  // 256 threads, one pixel each
+#ifndef GS_RASTER_PX
+#define GS_RASTER_PX 4
+#endif
+constexpr int kPx = GS_RASTER_PX;    // pixels per lane (a column segment): 8 or 4
+constexpr int kSub = 8 / kPx;        // warps per tile (a warp covers 16 x 2 kPx pixels)
+constexpr int kWarps = 4;            // warps per block
+// resident blocks per SM the register allocation is sized for (launch bounds)
+#ifndef GS_RASTER_FWD_MIN_BLOCKS
+#define GS_RASTER_FWD_MIN_BLOCKS 6
+#endif
+#ifndef GS_RASTER_BWD_MIN_BLOCKS
+#define GS_RASTER_BWD_MIN_BLOCKS 5
+#endif
+constexpr int kBatch = 32;  // list entries staged per warp per batch
+constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
@@ -47,79 +82,90 @@ __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
 
-// Raw features of one list entry as gathered from global memory.
-struct RawBuf {
-    float2 xy[kBlock];
-    float4 con[kBlock];  // A, B, C, o
-    float4 rgb[kBlock];
-    uint32_t gid[kBlock];
+// Per-warp staging area: raw gathered features (double-buffered) and the
+// per-entry constants derived from them.
+struct WarpStage {
+    float2 xy[2][kBatch];
+    float4 con[2][kBatch];  // A, B, C, o
+    float4 rgb[2][kBatch];
+    uint32_t gid[2][kBatch];
+    float4 pa[kBatch];  // u, v, log2(o), 1/o
+    float4 pb[kBatch];  // -log2e A/2, -log2e B, -log2e C/2, ill-conditioned flag (0 / 1)
 };
 
-// Derived per-entry constants used by the per-pixel loop.
-struct Prepped {
-    float4 xyl;   // u, v, log2(o), ill-conditioned flag (0 or 1)
-    float4 q;     // -log2e * A/2, -log2e * B, -log2e * C/2, 1/o
-};
-
-__device__ __forceinline__ Prepped prep(float2 xy, float4 con) {
-    Prepped p;
-    const float A = con.x, B = con.y, C = con.z, o = con.w;
-    const float tr = A + C, det = A * C - B * B;
-    const bool ill = !(det > 0.f) || (tr * tr > kCondMaxTraceSqOverDet * det);
-    p.xyl = make_float4(xy.x, xy.y, log2f(o), ill ? 1.f : 0.f);
-    p.q = make_float4(__fmul_rn(-0.5f * kLog2e, A), __fmul_rn(-kLog2e, B), __fmul_rn(-0.5f * kLog2e, C), 1.f / o);
-    return p;
-}
-
-struct AlphaOut {
-    float alpha;    // < kAlphaMin means "not blended"
-    bool clamped;   // alpha hit 0.99
-    float dx, dy;   // mean minus pixel centre
-};
-
-// alpha = min(0.99, o exp(-sigma)); 0 when sigma < 0.
-__device__ __forceinline__ AlphaOut splat_alpha(const Prepped& p, const float4& con, float px, float py) {
-    AlphaOut r;
-    float s;  // -log2(e) * sigma
-    if (p.xyl.w != 0.f) {
-        const double dx = double(p.xyl.x) - double(px), dy = double(p.xyl.y) - double(py);
-        const double sig = 0.5 * (double(con.x) * dx * dx + double(con.z) * dy * dy) + double(con.y) * dx * dy;
-        s = float(-sig * kLog2eD);
-        r.dx = float(dx);
-        r.dy = float(dy);
-    } else {
-        r.dx = __fsub_rn(p.xyl.x, px);
-        r.dy = __fsub_rn(p.xyl.y, py);
-        const float qx = __fmaf_rn(p.q.y, r.dy, __fmul_rn(p.q.x, r.dx));
-        s = __fmaf_rn(qx, r.dx, __fmul_rn(__fmul_rn(p.q.z, r.dy), r.dy));
-    }
-    if (s > 0.f) {
-        r.alpha = 0.f;
-        r.clamped = false;
-        return r;
-    }
-    const float a = ex2_approx(__fadd_rn(s, p.xyl.z));
-    r.clamped = a > kAlphaMax;
-    r.alpha = r.clamped ? kAlphaMax : a;
-    return r;
-}
-
-// Gather entries [first, first + count) of the sorted list into `buf`
-// (entry e -> slot e - first, or reversed for the backward pass).
+// Lane l < count gathers list entry first + l (reverse: first + count - 1 - l).
 template <bool kReverse>
-__device__ __forceinline__ void gather(RawBuf& buf, const uint32_t* __restrict__ vals, const float2* __restrict__ xy,
-                                       const float4* __restrict__ con, const float4* __restrict__ rgb, uint32_t first,
-                                       int count) {
-    const int t = threadIdx.x;
-    if (t < count) {
-        const uint32_t e = kReverse ? first + uint32_t(count - 1 - t) : first + uint32_t(t);
+__device__ __forceinline__ void gather(WarpStage& S, int buf, const uint32_t* __restrict__ vals,
+                                       const float2* __restrict__ xy, const float4* __restrict__ con,
+                                       const float4* __restrict__ rgb, uint32_t first, int count, int lane) {
+    if (lane < count) {
+        const uint32_t e = kReverse ? first + uint32_t(count - 1 - lane) : first + uint32_t(lane);
         const uint32_t g = __ldg(vals + e);
-        buf.gid[t] = g;
-        cp_async8(&buf.xy[t], xy + g);
-        cp_async16(&buf.con[t], con + g);
-        cp_async16(&buf.rgb[t], rgb + g);
+        S.gid[buf][lane] = g;
+        cp_async8(&S.xy[buf][lane], xy + g);
+        cp_async16(&S.con[buf][lane], con + g);
+        cp_async16(&S.rgb[buf][lane], rgb + g);
     }
     cp_async_commit();
+}
+
+// Lane l < count derives the constants of staged entry l.
+__device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane) {
+    if (lane < count) {
+        const float2 xy = S.xy[buf][lane];
+        const float4 c = S.con[buf][lane];
+        const float tr = __fadd_rn(c.x, c.z);
+        const float det = __fsub_rn(__fmul_rn(c.x, c.z), __fmul_rn(c.y, c.y));
+        const bool ill = !(det > 0.f) || (__fmul_rn(tr, tr) > __fmul_rn(kCondMaxTraceSqOverDet, det));
+        S.pa[lane] = make_float4(xy.x, xy.y, log2f(c.w), 1.f / c.w);
+        S.pb[lane] = make_float4(__fmul_rn(-0.5f * kLog2e, c.x), __fmul_rn(-kLog2e, c.y),
+                                 __fmul_rn(-0.5f * kLog2e, c.z), ill ? 1.f : 0.f);
+    }
+}
+
+// alpha of one entry at the lane's 8 pixels, and the offsets dx (shared) and
+// dy[i] of the mean from the pixel centres.  Bit i of `blend` is set when
+// pixel i passes sigma >= 0 and alpha >= 1/255; bit i of `clamp` when alpha
+// was clamped at 0.99.
+__device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float4& con, float px, int y0,
+                                           float (&alpha)[kPx], unsigned& blend, unsigned& clamp, float& dx,
+                                           float (&dy)[kPx]) {
+    blend = 0u;
+    clamp = 0u;
+    if (pb.w != 0.f) {
+        const double dxd = __dsub_rn(double(pa.x), double(px));
+        dx = __double2float_rn(dxd);
+        const double A = con.x, B = con.y, C = con.z;
+        const double adx2 = __dmul_rn(__dmul_rn(A, dxd), dxd);
+        const double bdx = __dmul_rn(B, dxd);
+#pragma unroll
+        for (int i = 0; i < kPx; ++i) {
+            const double dyd = __dsub_rn(double(pa.y), double(y0 + i) + 0.5);
+            const double sig = __dadd_rn(__dmul_rn(0.5, __dadd_rn(adx2, __dmul_rn(__dmul_rn(C, dyd), dyd))),
+                                         __dmul_rn(bdx, dyd));
+            const float s = __double2float_rn(__dmul_rn(-sig, kLog2eD));
+            dy[i] = __double2float_rn(dyd);
+            const float a = ex2_approx(__fadd_rn(s, pa.z));
+            const bool c = a > kAlphaMax;
+            alpha[i] = c ? kAlphaMax : a;
+            if (s <= 0.f && alpha[i] >= kAlphaMin) blend |= 1u << i;
+            if (c) clamp |= 1u << i;
+        }
+    } else {
+        dx = __fsub_rn(pa.x, px);
+        const float a0 = __fmul_rn(__fmul_rn(pb.x, dx), dx);
+        const float c1 = __fmul_rn(pb.y, dx);
+#pragma unroll
+        for (int i = 0; i < kPx; ++i) {
+            dy[i] = __fsub_rn(pa.y, __fadd_rn(float(y0 + i), 0.5f));
+            const float s = __fmaf_rn(dy[i], __fmaf_rn(pb.z, dy[i], c1), a0);
+            const float a = ex2_approx(__fadd_rn(s, pa.z));
+            const bool c = a > kAlphaMax;
+            alpha[i] = c ? kAlphaMax : a;
+            if (s <= 0.f && alpha[i] >= kAlphaMin) blend |= 1u << i;
+            if (c) clamp |= 1u << i;
+        }
+    }
 }
 
 struct FwdArgs {
@@ -128,71 +174,98 @@ struct FwdArgs {
     const float4* rgb;
     const uint32_t* vals;
     const uint2* ranges;
-    int W, H, TX;
+    int W, H, TX, tiles;
     float bg0, bg1, bg2;
     float* image;
     float* final_T;
     int32_t* n_contrib;
 };
 
-__global__ void __launch_bounds__(kBlock) raster_fwd_kernel(const FwdArgs a) {
-    __shared__ RawBuf buf[2];
-    __shared__ Prepped pre[kBlock];
-    const int tile = blockIdx.x;
-    const int tx = tile % a.TX, ty = tile / a.TX;
-    const int x = tx * kTile + (threadIdx.x & (kTile - 1));
-    const int y = ty * kTile + (threadIdx.x >> 4);
-    const bool inside = x < a.W && y < a.H;
-    const float px = float(x) + 0.5f, py = float(y) + 0.5f;
+__global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_fwd_kernel(const FwdArgs a) {
+    __shared__ WarpStage stage[kWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kWarps + warp;
+    const int tile = gw / kSub, sub = gw % kSub;
+    if (tile >= a.tiles) return;
+    WarpStage& S = stage[warp];
+    const int x = (tile % a.TX) * kTile + (lane & 15);
+    const int y0 = (tile / a.TX) * kTile + sub * 2 * kPx + (lane >> 4) * kPx;
+    const float px = float(x) + 0.5f;
     const uint2 range = a.ranges[tile];
-    const int total = int(range.y - range.x);
+    const int n = int(range.y - range.x);
 
-    float T = 1.f, Cr = 0.f, Cg = 0.f, Cb = 0.f;
-    int last = 0;
-    bool done = !inside;
+    float T[kPx], Cr[kPx], Cg[kPx], Cb[kPx];
+    int last[kPx];
+    unsigned done = 0u;
+#pragma unroll
+    for (int i = 0; i < kPx; ++i) {
+        T[i] = 1.f;
+        Cr[i] = Cg[i] = Cb[i] = 0.f;
+        last[i] = 0;
+        if (x >= a.W || y0 + i >= a.H) done |= 1u << i;
+    }
+    constexpr unsigned kAll = (1u << kPx) - 1u;
+    static_assert(kPx == 8 || kPx == 4, "a warp covers whole rows of a tile");
 
-    int cur = 0;
-    if (total > 0) gather<false>(buf[0], a.vals, a.xy, a.con, a.rgb, range.x, min(total, kBlock));
-    for (int start = 0; start < total; start += kBlock) {
-        const int count = min(total - start, kBlock);
+    const int nb = (n + kBatch - 1) / kBatch;
+    if (n > 0) gather<false>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x, min(n, kBatch), lane);
+    for (int b = 0; b < nb; ++b) {
+        const int buf = b & 1;
+        const int cnt = min(n - b * kBatch, kBatch);
         cp_async_wait_all();
-        __syncthreads();  // batch `cur` landed; everyone finished reading `pre` and buf[cur ^ 1]
-        if (__syncthreads_count(done) == kBlock) break;
-        if (start + kBlock < total)
-            gather<false>(buf[cur ^ 1], a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(start + kBlock),
-                          min(total - start - kBlock, kBlock));
-        if (threadIdx.x < count) pre[threadIdx.x] = prep(buf[cur].xy[threadIdx.x], buf[cur].con[threadIdx.x]);
-        __syncthreads();
-        if (!done) {
-            for (int j = 0; j < count; ++j) {
-                const Prepped p = pre[j];
-                const float4 con = buf[cur].con[j];
-                const AlphaOut al = splat_alpha(p, con, px, py);
-                if (al.alpha < kAlphaMin) continue;
-                const float Tn = __fmul_rn(T, __fsub_rn(1.f, al.alpha));
-                if (Tn < kTMin) {
-                    done = true;
-                    break;
-                }
-                const float4 c = buf[cur].rgb[j];
-                const float w = __fmul_rn(al.alpha, T);
-                Cr = __fmaf_rn(c.x, w, Cr);
-                Cg = __fmaf_rn(c.y, w, Cg);
-                Cb = __fmaf_rn(c.z, w, Cb);
-                T = Tn;
-                last = start + j + 1;
+        __syncwarp();
+        if (b + 1 < nb)
+            gather<false>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t((b + 1) * kBatch),
+                          min(n - (b + 1) * kBatch, kBatch), lane);
+        prep(S, buf, cnt, lane);
+        __syncwarp();
+        bool finished = false;
+        for (int j = 0; j < cnt; ++j) {
+            if (__all_sync(kFull, done == kAll)) {
+                finished = true;
+                break;
+            }
+            const float4 pa = S.pa[j], pb = S.pb[j];
+            const float4 con = S.con[buf][j];
+            const float4 c = S.rgb[buf][j];
+            float al[kPx], dy[kPx], dx;
+            unsigned blend, clamp;
+            eval_alpha(pa, pb, con, px, y0, al, blend, clamp, dx, dy);
+            blend &= ~done;
+            const int pos = b * kBatch + j + 1;
+            // branch-free so the 8 independent pixel chains interleave; a pixel
+            // that does not take the entry adds c * 0 (exactly nothing)
+#pragma unroll
+            for (int i = 0; i < kPx; ++i) {
+                const bool act = (blend >> i) & 1u;
+                const float Tn = __fmul_rn(T[i], __fsub_rn(1.f, al[i]));
+                const bool low = Tn < kTMin;
+                const bool take = act && !low;
+                const float w = take ? __fmul_rn(al[i], T[i]) : 0.f;
+                Cr[i] = __fmaf_rn(c.x, w, Cr[i]);
+                Cg[i] = __fmaf_rn(c.y, w, Cg[i]);
+                Cb[i] = __fmaf_rn(c.z, w, Cb[i]);
+                T[i] = take ? Tn : T[i];
+                last[i] = take ? pos : last[i];
+                done |= (act && low) ? (1u << i) : 0u;
             }
         }
-        cur ^= 1;
+        __syncwarp();
+        if (finished) break;
     }
     cp_async_wait_all();
-    if (inside) {
-        const int64_t pix = int64_t(y) * a.W + x;
-        a.image[3 * pix + 0] = __fmaf_rn(T, a.bg0, Cr);
-        a.image[3 * pix + 1] = __fmaf_rn(T, a.bg1, Cg);
-        a.image[3 * pix + 2] = __fmaf_rn(T, a.bg2, Cb);
-        a.final_T[pix] = T;
-        a.n_contrib[pix] = last;
+    if (x < a.W) {
+#pragma unroll
+        for (int i = 0; i < kPx; ++i) {
+            if (y0 + i < a.H) {
+                const int64_t pix = int64_t(y0 + i) * a.W + x;
+                a.image[3 * pix + 0] = __fmaf_rn(T[i], a.bg0, Cr[i]);
+                a.image[3 * pix + 1] = __fmaf_rn(T[i], a.bg1, Cg[i]);
+                a.image[3 * pix + 2] = __fmaf_rn(T[i], a.bg2, Cb[i]);
+                a.final_T[pix] = T[i];
+                a.n_contrib[pix] = last[i];
+            }
+        }
     }
 }
 
@@ -202,7 +275,7 @@ struct BwdArgs {
     const float4* rgb;
     const uint32_t* vals;
     const uint2* ranges;
-    int W, H, TX;
+    int W, H, TX, tiles;
     float bg0, bg1, bg2;
     const float* final_T;
     const int32_t* n_contrib;
@@ -212,116 +285,164 @@ struct BwdArgs {
     float4* g_rgb;
 };
 
-__device__ __forceinline__ float warp_sum(float v) {
+// Sum 9 per-lane values over the warp and add them to the Gaussian's three
+// gradient records with one vector atomic each (lanes 0, 1, 2).
+__device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int lane, uint32_t gid,
+                                                    const BwdArgs& a) {
+    // reduce-scatter of 8 values: after it, lanes 4k..4k+3 hold the total of value k
+    {
+        const bool hi = (lane >> 4) & 1;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+        for (int k = 0; k < 4; ++k) {
+            const float send = hi ? v[k] : v[k + 4];
+            const float keep = hi ? v[k + 4] : v[k];
+            v[k] = keep + __shfl_xor_sync(kFull, send, 16);
+        }
+    }
+    {
+        const bool hi = (lane >> 3) & 1;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const float send = hi ? v[k] : v[k + 2];
+            const float keep = hi ? v[k + 2] : v[k];
+            v[k] = keep + __shfl_xor_sync(kFull, send, 8);
+        }
+    }
+    {
+        const bool hi = (lane >> 2) & 1;
+        const float send = hi ? v[0] : v[1];
+        const float keep = hi ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(kFull, send, 4);
+    }
+    v[0] += __shfl_xor_sync(kFull, v[0], 2);
+    v[0] += __shfl_xor_sync(kFull, v[0], 1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v8 += __shfl_xor_sync(kFull, v8, o);
+    // gather: lane 0 <- values 0,1 (du, dv); lane 1 <- 2..5 (dA, dB, dC, do); lane 2 <- 6,7 (dr, dg) + v8 (db)
+    const int i0 = lane == 0 ? 0 : (lane == 1 ? 2 : 6);
+    const int i1 = i0 + 1;
+    const int i2 = lane == 1 ? 4 : 0;
+    const int i3 = lane == 1 ? 5 : 0;
+    const float f0 = __shfl_sync(kFull, v[0], 4 * i0);
+    const float f1 = __shfl_sync(kFull, v[0], 4 * i1);
+    const float f2 = __shfl_sync(kFull, v[0], 4 * i2);
+    const float f3 = __shfl_sync(kFull, v[0], 4 * i3);
+    if (lane == 0) atomicAdd(a.g_xy + gid, make_float2(f0, f1));
+    if (lane == 1) atomicAdd(a.g_con + gid, make_float4(f0, f1, f2, f3));
+    if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
-__global__ void __launch_bounds__(kBlock) raster_bwd_kernel(const BwdArgs a) {
-    __shared__ RawBuf buf[2];
-    __shared__ Prepped pre[kBlock];
-    __shared__ int max_last;
-    const int tile = blockIdx.x;
-    const int tx = tile % a.TX, ty = tile / a.TX;
-    const int x = tx * kTile + (threadIdx.x & (kTile - 1));
-    const int y = ty * kTile + (threadIdx.x >> 4);
-    const bool inside = x < a.W && y < a.H;
-    const float px = float(x) + 0.5f, py = float(y) + 0.5f;
+__global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_bwd_kernel(const BwdArgs a) {
+    __shared__ WarpStage stage[kWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kWarps + warp;
+    const int tile = gw / kSub, sub = gw % kSub;
+    if (tile >= a.tiles) return;
+    WarpStage& S = stage[warp];
+    const int x = (tile % a.TX) * kTile + (lane & 15);
+    const int y0 = (tile / a.TX) * kTile + sub * 2 * kPx + (lane >> 4) * kPx;
+    const float px = float(x) + 0.5f;
     const uint2 range = a.ranges[tile];
-    const int lane = threadIdx.x & 31;
 
-    float T = 1.f, gr = 0.f, gg = 0.f, gb = 0.f, Tfinal = 1.f;
-    int last = 0;
-    if (inside) {
-        const int64_t pix = int64_t(y) * a.W + x;
-        Tfinal = a.final_T[pix];
-        T = Tfinal;
-        last = a.n_contrib[pix];
-        gr = a.dL_dimage[3 * pix + 0];
-        gg = a.dL_dimage[3 * pix + 1];
-        gb = a.dL_dimage[3 * pix + 2];
-    }
-    const float bgg = a.bg0 * gr + a.bg1 * gg + a.bg2 * gb;
-    float Sr = 0.f, Sg = 0.f, Sb = 0.f;
-
-    if (threadIdx.x == 0) max_last = 0;
-    __syncthreads();
-    atomicMax(&max_last, last);
-    __syncthreads();
-    const int total = max_last;  // entries beyond every pixel's last blended one are never needed
-
-    int cur = 0;
-    // batches walk the list from the back: batch b covers positions [hi - count, hi)
-    if (total > 0) {
-        const int count0 = min(total, kBlock);
-        gather<true>(buf[0], a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(total - count0), count0);
-    }
-    for (int hi = total; hi > 0; hi -= kBlock) {
-        const int count = min(hi, kBlock);
-        cp_async_wait_all();
-        __syncthreads();
-        if (hi - kBlock > 0) {
-            const int nhi = hi - kBlock, ncount = min(nhi, kBlock);
-            gather<true>(buf[cur ^ 1], a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncount), ncount);
-        }
-        if (threadIdx.x < count) pre[threadIdx.x] = prep(buf[cur].xy[threadIdx.x], buf[cur].con[threadIdx.x]);
-        __syncthreads();
-        for (int j = 0; j < count; ++j) {
-            const int pos = hi - 1 - j;  // list position of this entry
-            const Prepped p = pre[j];
-            const float4 con = buf[cur].con[j];
-            float g9[9] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            bool contrib = false;
-            if (pos < last) {
-                const AlphaOut al = splat_alpha(p, con, px, py);
-                if (al.alpha >= kAlphaMin) {
-                    contrib = true;
-                    const float om = __fsub_rn(1.f, al.alpha);
-                    const float rom = __frcp_rn(om);
-                    T = __fmul_rn(T, rom);  // transmittance in front of this entry
-                    const float4 c = buf[cur].rgb[j];
-                    const float w = al.alpha * T;
-                    g9[6] = w * gr;
-                    g9[7] = w * gg;
-                    g9[8] = w * gb;
-                    const float dLda =
-                        T * (gr * (c.x - Sr) + gg * (c.y - Sg) + gb * (c.z - Sb)) - Tfinal * bgg * rom;
-                    Sr = __fmaf_rn(c.x, al.alpha, om * Sr);
-                    Sg = __fmaf_rn(c.y, al.alpha, om * Sg);
-                    Sb = __fmaf_rn(c.z, al.alpha, om * Sb);
-                    if (!al.clamped) {
-                        g9[5] = dLda * al.alpha * p.q.w;  // d alpha / d o = alpha / o
-                        const float dLds = -dLda * al.alpha;
-                        float su, sv;
-                        if (p.xyl.w != 0.f) {
-                            const double dx = double(p.xyl.x) - double(px), dy = double(p.xyl.y) - double(py);
-                            su = float(double(con.x) * dx + double(con.y) * dy);
-                            sv = float(double(con.y) * dx + double(con.z) * dy);
-                        } else {
-                            su = con.x * al.dx + con.y * al.dy;
-                            sv = con.y * al.dx + con.z * al.dy;
-                        }
-                        g9[0] = dLds * su;
-                        g9[1] = dLds * sv;
-                        g9[2] = 0.5f * dLds * al.dx * al.dx;
-                        g9[3] = dLds * al.dx * al.dy;
-                        g9[4] = 0.5f * dLds * al.dy * al.dy;
-                    }
-                }
-            }
-            if (__any_sync(0xffffffffu, contrib)) {
+    float T[kPx], Sr[kPx], Sg[kPx], Sb[kPx], gr[kPx], gg[kPx], gb[kPx], ngb[kPx];
+    int last[kPx];
+    int lmax = 0;
 #pragma unroll
-                for (int q = 0; q < 9; ++q) g9[q] = warp_sum(g9[q]);
-                if (lane == 0) {
-                    const uint32_t gid = buf[cur].gid[j];
-                    atomicAdd(a.g_xy + gid, make_float2(g9[0], g9[1]));
-                    atomicAdd(a.g_con + gid, make_float4(g9[2], g9[3], g9[4], g9[5]));
-                    atomicAdd(a.g_rgb + gid, make_float4(g9[6], g9[7], g9[8], 0.f));
+    for (int i = 0; i < kPx; ++i) {
+        Sr[i] = Sg[i] = Sb[i] = 0.f;
+        if (x < a.W && y0 + i < a.H) {
+            const int64_t pix = int64_t(y0 + i) * a.W + x;
+            T[i] = a.final_T[pix];
+            last[i] = a.n_contrib[pix];
+            gr[i] = a.dL_dimage[3 * pix + 0];
+            gg[i] = a.dL_dimage[3 * pix + 1];
+            gb[i] = a.dL_dimage[3 * pix + 2];
+        } else {
+            T[i] = 1.f;
+            last[i] = 0;
+            gr[i] = gg[i] = gb[i] = 0.f;
+        }
+        ngb[i] = -T[i] * (a.bg0 * gr[i] + a.bg1 * gg[i] + a.bg2 * gb[i]);
+        lmax = max(lmax, last[i]);
+    }
+    // entries past every pixel's last are never needed; never read past the list
+    const int total = min(__reduce_max_sync(kFull, lmax), int(range.y - range.x));
+    const int nb = (total + kBatch - 1) / kBatch;
+    if (total > 0) {
+        const int c0 = min(total, kBatch);
+        gather<true>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(total - c0), c0, lane);
+    }
+    for (int b = 0; b < nb; ++b) {
+        const int buf = b & 1;
+        const int hi = total - b * kBatch;  // this batch covers positions [hi - cnt, hi)
+        const int cnt = min(hi, kBatch);
+        cp_async_wait_all();
+        __syncwarp();
+        if (b + 1 < nb) {
+            const int nhi = hi - kBatch, ncnt = min(nhi, kBatch);
+            gather<true>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncnt), ncnt, lane);
+        }
+        prep(S, buf, cnt, lane);
+        __syncwarp();
+        for (int j = 0; j < cnt; ++j) {
+            const int pos = hi - 1 - j;  // 0-based list position of this entry
+            const float4 pa = S.pa[j], pb = S.pb[j];
+            const float4 con = S.con[buf][j];
+            const float4 c = S.rgb[buf][j];
+            float al[kPx], dy[kPx], m[kPx], dx;
+            unsigned blend, clamp;
+            eval_alpha(pa, pb, con, px, y0, al, blend, clamp, dx, dy);
+            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s0 = 0.f, s1 = 0.f, s2 = 0.f;
+            bool any = false;
+            // branch-free: every pixel runs the same instructions, inactive ones
+            // with zero weight and unchanged state
+#pragma unroll
+            for (int i = 0; i < kPx; ++i) {
+                const bool act = ((blend >> i) & 1u) && pos < last[i];
+                any = any || act;
+                // an inactive pixel runs the same instructions with alpha 0: T, S and
+                // every sum stay unchanged
+                const float ae = act ? al[i] : 0.f;
+                const float rom = rcp_approx(__fsub_rn(1.f, ae));
+                T[i] = T[i] * rom;  // transmittance in front of this entry
+                const float w = ae * T[i];
+                dr = fmaf(w, gr[i], dr);
+                dg = fmaf(w, gg[i], dg);
+                db = fmaf(w, gb[i], db);
+                const float xr = c.x - Sr[i], xg = c.y - Sg[i], xb = c.z - Sb[i];
+                const float dLda = fmaf(T[i], fmaf(gr[i], xr, fmaf(gg[i], xg, gb[i] * xb)), ngb[i] * rom);
+                Sr[i] = fmaf(ae, xr, Sr[i]);  // S <- c alpha + (1 - alpha) S
+                Sg[i] = fmaf(ae, xg, Sg[i]);
+                Sb[i] = fmaf(ae, xb, Sb[i]);
+                m[i] = ((clamp >> i) & 1u) ? 0.f : dLda * ae;  // dL/dsigma = -m, dL/do = m / o
+                mo += m[i];
+                s0 -= m[i];
+                s1 = fmaf(-m[i], dy[i], s1);
+                s2 = fmaf(-m[i] * dy[i], dy[i], s2);
+            }
+            if (__any_sync(kFull, any)) {
+                float du, dv;
+                if (pb.w != 0.f) {
+                    // ill-conditioned: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
+                    const double dxd = __dsub_rn(double(pa.x), double(px));
+                    du = dv = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kPx; ++i) {
+                        const double dyd = __dsub_rn(double(pa.y), double(y0 + i) + 0.5);
+                        const float su = __double2float_rn(double(con.x) * dxd + double(con.y) * dyd);
+                        const float sv = __double2float_rn(double(con.y) * dxd + double(con.z) * dyd);
+                        du = fmaf(-m[i], su, du);
+                        dv = fmaf(-m[i], sv, dv);
+                    }
+                } else {
+                    du = fmaf(con.x * dx, s0, con.y * s1);
+                    dv = fmaf(con.y * dx, s0, con.z * s1);
                 }
+                float v[8] = {du, dv, 0.5f * dx * dx * s0, dx * s1, 0.5f * s2, mo * pa.w, dr, dg};
+                warp_reduce_and_add(v, db, lane, S.gid[buf][j], a);
             }
         }
-        cur ^= 1;
+        __syncwarp();
     }
     cp_async_wait_all();
 }
@@ -340,13 +461,14 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
     a.W = cam.W;
     a.H = cam.H;
     a.TX = cam.TX;
+    a.tiles = cam.TX * cam.TY;
     a.bg0 = bg[0];
     a.bg1 = bg[1];
     a.bg2 = bg[2];
     a.image = image;
     a.final_T = final_T;
     a.n_contrib = n_contrib;
-    raster_fwd_kernel<<<unsigned(cam.TX * cam.TY), kBlock, 0, s>>>(a);
+    raster_fwd_kernel<<<unsigned((a.tiles * kSub + kWarps - 1) / kWarps), kWarps * 32, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -363,6 +485,7 @@ cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, co
     a.W = cam.W;
     a.H = cam.H;
     a.TX = cam.TX;
+    a.tiles = cam.TX * cam.TY;
     a.bg0 = bg[0];
     a.bg1 = bg[1];
     a.bg2 = bg[2];
@@ -372,7 +495,7 @@ cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, co
     a.g_xy = reinterpret_cast<float2*>(g2.xy);
     a.g_con = reinterpret_cast<float4*>(g2.conic_opacity);
     a.g_rgb = reinterpret_cast<float4*>(g2.rgb);
-    raster_bwd_kernel<<<unsigned(cam.TX * cam.TY), kBlock, 0, s>>>(a);
+    raster_bwd_kernel<<<unsigned((a.tiles * kSub + kWarps - 1) / kWarps), kWarps * 32, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -156,10 +156,12 @@ size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera*
 
 /* gs_bin_sort -- tile binning.  Every visible Gaussian emits one instance per tile
  * of its rectangle, key = (ty * tiles_x + tx) << 32 | float32 bits of its depth,
- * value = Gaussian index; the instances are sorted by key with a stable LSD radix
- * sort over the low 32 + ceil(log2(tiles)) key bits (equal keys keep ascending
- * Gaussian index), and tile_ranges[2t], [2t+1] receive the [begin, end) of tile t
- * in the sorted list ([0, 0) when empty).
+ * value = Gaussian index; the instances are sorted by key, equal keys keeping
+ * ascending Gaussian index, and tile_ranges[2t], [2t+1] receive the [begin, end)
+ * of tile t in the sorted list ([0, 0) when empty).  Method: a stable LSD radix
+ * sort of the Gaussians by depth bits, instances emitted in that order, then a
+ * stable LSD radix sort by tile id (ceil(log2(tiles)) bits); the last pass writes
+ * the 64-bit keys.
  *   keys [capacity] (8-byte aligned), vals [capacity] (4-byte aligned),
  *   tile_ranges [tiles][2] uint32 (8-byte aligned), workspace as sized above.
  * *num_instances_host receives K, the instance count.  K > capacity returns
@@ -179,8 +181,8 @@ gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam,
  * which is a library-owned device array of GS_STATIC_SCRATCH_BYTES held on
  * every device that loads the library until the process exits.
  *   - n and capacity whose workspace (gs_bin_sort_workspace_bytes) exceeds
- *     GS_STATIC_SCRATCH_BYTES return GS_ERR_UNSUPPORTED (about 2.7 million
- *     instances for a million Gaussians).
+ *     GS_STATIC_SCRATCH_BYTES return GS_ERR_UNSUPPORTED (the workspace is
+ *     about 16 bytes per slot of max(capacity, n): about 2 million).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make that
  *     first call before any stream capture.
