@@ -48,9 +48,17 @@ constexpr float kCondMaxTraceSqOverDet = 10.125f;
 #ifndef GS_RASTER_PX
 #define GS_RASTER_PX 4
 #endif
-constexpr int kPx = GS_RASTER_PX;    // pixels per lane (a column segment): 8 or 4
-constexpr int kSub = 8 / kPx;        // warps per tile (a warp covers 16 x 2 kPx pixels)
-constexpr int kWarps = 4;            // warps per block
+#ifndef GS_RASTER_BOXW
+#define GS_RASTER_BOXW 16
+#endif
+constexpr int kPx = GS_RASTER_PX;        // pixels per lane (a column segment)
+constexpr int kBoxW = GS_RASTER_BOXW;    // width of a warp's pixel box (16 or 8)
+constexpr int kLaneRows = 32 / kBoxW;    // lanes stacked vertically in the box
+constexpr int kBoxH = kLaneRows * kPx;   // height of a warp's pixel box
+constexpr int kSubX = kTile / kBoxW, kSubY = kTile / kBoxH;
+constexpr int kSub = kSubX * kSubY;      // warps per tile
+constexpr int kWarps = 4;                // warps per block
+static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
 // resident blocks per SM the register allocation is sized for (launch bounds)
 #ifndef GS_RASTER_FWD_MIN_BLOCKS
 #define GS_RASTER_FWD_MIN_BLOCKS 6
@@ -90,7 +98,7 @@ struct WarpStage {
     float4 rgb[2][kBatch];
     uint32_t gid[2][kBatch];
     float4 pa[kBatch];  // u, v, log2(o), 1/o
-    float4 pb[kBatch];  // -log2e A/2, -log2e B, -log2e C/2, ill-conditioned flag (0 / 1)
+    float4 pb[kBatch];  // -log2e A/2, -log2e B, -log2e C/2, flag (0 float32, 1 double, 2 skip)
 };
 
 // Lane l < count gathers list entry first + l (reverse: first + count - 1 - l).
@@ -109,17 +117,44 @@ __device__ __forceinline__ void gather(WarpStage& S, int buf, const uint32_t* __
     cp_async_commit();
 }
 
-// Lane l < count derives the constants of staged entry l.
-__device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane) {
+// Smallest sigma = 1/2 (A dx^2 + 2 B dx dy + C dy^2) with dx fixed and dy in
+// [dylo, dyhi] (a positive definite form is minimised at dy = -B dx / C).
+__device__ __forceinline__ float edge_min(float A, float B, float C, float dx, float dylo, float dyhi) {
+    const float dy = fminf(fmaxf(-B * dx / C, dylo), dyhi);
+    return 0.5f * (A * dx * dx + 2.f * B * dx * dy + C * dy * dy);
+}
+
+// Lane l < count derives the constants of staged entry l.  pb.w: 0 = evaluate
+// in float32, 1 = ill-conditioned (evaluate in double), 2 = skip: the smallest
+// sigma over this warp's pixel box [bx0, bx0 + kBoxW - 1] x [by0, by0 + kBoxH - 1]
+// (pixel centres) puts alpha below 1/255 everywhere in it, with a margin far
+// above the rounding of either evaluation, so no pixel of the warp would blend
+// it.  Ill-conditioned entries are never skipped.
+__device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
     if (lane < count) {
         const float2 xy = S.xy[buf][lane];
         const float4 c = S.con[buf][lane];
         const float tr = __fadd_rn(c.x, c.z);
         const float det = __fsub_rn(__fmul_rn(c.x, c.z), __fmul_rn(c.y, c.y));
         const bool ill = !(det > 0.f) || (__fmul_rn(tr, tr) > __fmul_rn(kCondMaxTraceSqOverDet, det));
-        S.pa[lane] = make_float4(xy.x, xy.y, log2f(c.w), 1.f / c.w);
+        const float lo = log2f(c.w);
+        float flag = ill ? 1.f : 0.f;
+        if (!ill) {
+            const float bx1 = bx0 + float(kBoxW - 1), by1 = by0 + float(kBoxH - 1);
+            const bool inside = xy.x >= bx0 && xy.x <= bx1 && xy.y >= by0 && xy.y <= by1;
+            if (!inside) {
+                const float dxlo = xy.x - bx1, dxhi = xy.x - bx0, dylo = xy.y - by1, dyhi = xy.y - by0;
+                float smin = fminf(edge_min(c.x, c.y, c.z, dxlo, dylo, dyhi), edge_min(c.x, c.y, c.z, dxhi, dylo, dyhi));
+                smin = fminf(smin, edge_min(c.z, c.y, c.x, dylo, dxlo, dxhi));
+                smin = fminf(smin, edge_min(c.z, c.y, c.x, dyhi, dxlo, dxhi));
+                // alpha >= 1/255 needs sigma <= ln(255 o) = ln 255 + lo ln 2
+                const float cut = 5.541263545158426f + lo * 0.6931471805599453f;
+                if (smin * (1.f - 1e-4f) > cut + 1e-4f) flag = 2.f;
+            }
+        }
+        S.pa[lane] = make_float4(xy.x, xy.y, lo, 1.f / c.w);
         S.pb[lane] = make_float4(__fmul_rn(-0.5f * kLog2e, c.x), __fmul_rn(-kLog2e, c.y),
-                                 __fmul_rn(-0.5f * kLog2e, c.z), ill ? 1.f : 0.f);
+                                 __fmul_rn(-0.5f * kLog2e, c.z), flag);
     }
 }
 
@@ -132,7 +167,7 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
                                            float (&dy)[kPx]) {
     blend = 0u;
     clamp = 0u;
-    if (pb.w != 0.f) {
+    if (pb.w == 1.f) {
         const double dxd = __dsub_rn(double(pa.x), double(px));
         dx = __double2float_rn(dxd);
         const double A = con.x, B = con.y, C = con.z;
@@ -188,9 +223,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     const int tile = gw / kSub, sub = gw % kSub;
     if (tile >= a.tiles) return;
     WarpStage& S = stage[warp];
-    const int x = (tile % a.TX) * kTile + (lane & 15);
-    const int y0 = (tile / a.TX) * kTile + sub * 2 * kPx + (lane >> 4) * kPx;
+    const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
+    const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
+    const int x = xb + lane % kBoxW;
+    const int y0 = yb + (lane / kBoxW) * kPx;
     const float px = float(x) + 0.5f;
+    const float bx0 = float(xb) + 0.5f, by0 = float(yb) + 0.5f;  // box corner (pixel centre)
     const uint2 range = a.ranges[tile];
     const int n = int(range.y - range.x);
 
@@ -205,7 +243,6 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (x >= a.W || y0 + i >= a.H) done |= 1u << i;
     }
     constexpr unsigned kAll = (1u << kPx) - 1u;
-    static_assert(kPx == 8 || kPx == 4, "a warp covers whole rows of a tile");
 
     const int nb = (n + kBatch - 1) / kBatch;
     if (n > 0) gather<false>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x, min(n, kBatch), lane);
@@ -217,7 +254,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (b + 1 < nb)
             gather<false>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t((b + 1) * kBatch),
                           min(n - (b + 1) * kBatch, kBatch), lane);
-        prep(S, buf, cnt, lane);
+        prep(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         bool finished = false;
         for (int j = 0; j < cnt; ++j) {
@@ -226,6 +263,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 break;
             }
             const float4 pa = S.pa[j], pb = S.pb[j];
+            if (pb.w == 2.f) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
             float al[kPx], dy[kPx], dx;
@@ -339,9 +377,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     const int tile = gw / kSub, sub = gw % kSub;
     if (tile >= a.tiles) return;
     WarpStage& S = stage[warp];
-    const int x = (tile % a.TX) * kTile + (lane & 15);
-    const int y0 = (tile / a.TX) * kTile + sub * 2 * kPx + (lane >> 4) * kPx;
+    const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
+    const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
+    const int x = xb + lane % kBoxW;
+    const int y0 = yb + (lane / kBoxW) * kPx;
     const float px = float(x) + 0.5f;
+    const float bx0 = float(xb) + 0.5f, by0 = float(yb) + 0.5f;  // box corner (pixel centre)
     const uint2 range = a.ranges[tile];
 
     float T[kPx], Sr[kPx], Sg[kPx], Sb[kPx], gr[kPx], gg[kPx], gb[kPx], ngb[kPx];
@@ -382,11 +423,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             const int nhi = hi - kBatch, ncnt = min(nhi, kBatch);
             gather<true>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncnt), ncnt, lane);
         }
-        prep(S, buf, cnt, lane);
+        prep(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         for (int j = 0; j < cnt; ++j) {
             const int pos = hi - 1 - j;  // 0-based list position of this entry
             const float4 pa = S.pa[j], pb = S.pb[j];
+            if (pb.w == 2.f) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
             float al[kPx], dy[kPx], m[kPx], dx;
@@ -422,7 +464,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             }
             if (__any_sync(kFull, any)) {
                 float du, dv;
-                if (pb.w != 0.f) {
+                if (pb.w == 1.f) {
                     // ill-conditioned: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
                     const double dxd = __dsub_rn(double(pa.x), double(px));
                     du = dv = 0.f;
