@@ -80,19 +80,20 @@ def make_workload(name: str):
 
 def step_bytes(n, sh_degree, views_stats, tiles, pixels):
     """Algorithmic HBM bytes of one step: per view, the sum of the stage terms,
-    then Adam over the 59 floats (SH degree 3) per Gaussian."""
+    then the fused multi-view backward through the projection with Adam."""
     pb = 4 * (11 + 3 * (sh_degree + 1) ** 2)
     total = 0
     for (K, V, passes) in views_stats:
         total += n * (pb + 52)                 # project
-        total += n * 24 + K * 12               # count/scan + emit
-        total += K * (8 + 24 * passes)         # radix sort
+        total += n * (8 + 20 * 4)              # depth keys + 4 depth passes
+        total += n * 16 + K * 8                # count (depth order) + emit (tile, gid)
+        total += K * 20 * passes + K * 4       # tile passes (the last writes 12 instead of 8)
         total += K * 8 + tiles * 8             # tile ranges
         total += K * 4 + V * 36 + pixels * 20  # raster forward
         total += pixels * 36                   # L1 + dL/dimage
         total += K * 4 + V * 108 + pixels * 20  # raster backward
-        total += n * (pb + 36 + 2 * pb + 8)    # project backward: params, grad2d, grads (+=), densify
-    total += n * pb // 4 * 28                  # Adam: param, m, v read+write, grad read
+        total += n * 44                        # this view's radius + 2D gradients, read by the fused pass
+    total += n * 6 * pb + n * 8                # fused pass: params read+write, m and v read+write, densify
     return total
 
 
@@ -281,8 +282,8 @@ def run_ours(args, world, rank, local):
 
     # ---- timed region: K steps on resident inputs
     ev_dom = []
-    orig = {"raster_bwd": pl.raster_bwd, "raster_fwd": pl.raster_fwd, "project_bwd": pl.project_bwd,
-            "project": pl.project}
+    orig = {"raster_bwd": pl.raster_bwd, "raster_fwd": pl.raster_fwd,
+            "project_bwd_adam": pl.project_bwd_views_adam, "project": pl.project}
 
     def wrap(fn):
         def inner(*a, **k):
@@ -322,8 +323,8 @@ def run_ours(args, world, rank, local):
     pairs = 0
     for v in views:
         T = v.tiles_x * v.tiles_y
-        passes = (32 + max(1, math.ceil(math.log2(T))) + 7) // 8
-        stats.append((v.num_instances, int((tr.proj.radius > 0).sum().item()), passes))
+        passes = max(1, (math.ceil(math.log2(T)) + 7) // 8)
+        stats.append((v.num_instances, int((tr.radii[len(stats)] > 0).sum().item()), passes))
         pairs += int(v.n_contrib.sum().item())
     cam0 = wl.cameras[0]
     P = cam0["width"] * cam0["height"]
@@ -377,18 +378,18 @@ def stage_breakdown(tr, pl, torch):
         acc.setdefault(name, []).append((e0, e1))
         return r
 
-    tr.grads.zero_()
-    for view, tgt in zip(tr.views, tr.targets):
-        timed("project", pl.project, tr.gauss, view, tr.proj)
-        timed("bin_sort", pl.bin_sort, tr.proj, view)
-        timed("raster_fwd", pl.raster_fwd, tr.proj, view, tr.bg)
+    for k, (view, tgt) in enumerate(zip(tr.views, tr.targets)):
+        r = tr.radii[k]
+        g2 = tr.grad2ds[k]
+        timed("project", pl.project, tr.gauss, view, tr.proj, r)
+        timed("bin_sort", pl.bin_sort, tr.proj, view, r)
+        timed("raster_fwd", pl.raster_fwd, tr.proj, view, tr.bg, r)
         timed("l1", pl.l1_loss_grad, view, tgt, tr.loss)
-        tr.grad2d.zero_()
-        timed("raster_bwd", pl.raster_bwd, tr.proj, view, tr.grad2d, tr.bg)
-        timed("project_bwd", pl.project_bwd, tr.gauss, view, tr.proj, tr.grad2d, tr.grads, tr.densify_accum,
-              tr.densify_count)
+        g2.zero_()
+        timed("raster_bwd", pl.raster_bwd, tr.proj, view, g2, tr.bg, None, r)
     tr.step_count += 1
-    timed("adam", pl.adam_step, tr.gauss, tr.grads, tr.m, tr.v, tr.lrs, tr.step_count)
+    timed("project_bwd_adam", pl.project_bwd_views_adam, tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m,
+          tr.v, tr.lrs, tr.step_count, None, tr.densify_accum, tr.densify_count)
     torch.cuda.synchronize()
     return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
 
@@ -411,7 +412,8 @@ def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks):
                 "work": f"{pairs_per_view:.4g} (pixel, entry) pairs x {per_pair} flops per launch",
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"}
     n = scene.n
-    per_launch = {"project_bwd": n * (pb + 36 + 2 * pb + 8), "project": n * (pb + 52),
+    nv = len(stats)
+    per_launch = {"project_bwd_adam": n * (6 * pb + 44 * nv + 8), "project": n * (pb + 52),
                   "bin_sort": n * 24 + K * 12 + K * (8 + 24 * stats[0][2]) + K * 8,
                   "adam": n * pb // 4 * 28, "l1": P * 36}.get(stage, 0)
     achieved = per_launch / (ms * 1e-3) / 1e9
@@ -439,7 +441,6 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
         nonlocal done
         done = [torch.cuda.Event() for _ in range(nv)]
         s = stream.cuda_stream
-        tr.grads.zero_()
         abi.gs_zero(tr.loss.data_ptr(), 8, s)
         copy_events = []
         with torch.cuda.stream(copy_stream):
@@ -448,12 +449,9 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
                 e = torch.cuda.Event()
                 e.record(copy_stream)
                 copy_events.append(e)
-        for v, view in enumerate(tr.views):
+        for v in range(nv):
             stream.wait_event(copy_events[v])
-            pl.project(tr.gauss, view, tr.proj)
-            pl.bin_sort(tr.proj, view)
-            pl.raster_fwd(tr.proj, view, tr.bg)
-            pl.l1_loss_grad(view, bufs[v % 2], tr.loss)
+            tr.view_forward_backward(v, bufs[v % 2])
             done[v].record(stream)
             if v + 2 < nv:
                 with torch.cuda.stream(copy_stream):
@@ -462,11 +460,9 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
                     e = torch.cuda.Event()
                     e.record(copy_stream)
                     copy_events.append(e)
-            tr.grad2d.zero_()
-            pl.raster_bwd(tr.proj, view, tr.grad2d, tr.bg)
-            pl.project_bwd(tr.gauss, view, tr.proj, tr.grad2d, tr.grads, tr.densify_accum, tr.densify_count)
         tr.step_count += 1
-        pl.adam_step(tr.gauss, tr.grads, tr.m, tr.v, tr.lrs, tr.step_count)
+        pl.project_bwd_views_adam(tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m, tr.v, tr.lrs,
+                                  tr.step_count, None, tr.densify_accum, tr.densify_count)
         loss_host.copy_(tr.loss, non_blocking=True)
 
     done = []

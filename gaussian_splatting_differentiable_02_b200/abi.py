@@ -74,6 +74,14 @@ SIGNATURES = {
                                   _P, _P, C.POINTER(gs_grad2d), _P]),
     "gs_project_bwd": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected),
                                    C.POINTER(gs_grad2d), C.POINTER(gs_param_grads), _P, _P, _P]),
+    "gs_project_bwd_views": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
+                                         C.POINTER(gs_projected), C.POINTER(gs_grad2d), C.POINTER(gs_param_grads),
+                                         _P, _P, _P]),
+    "gs_project_bwd_views_adam": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
+                                              C.POINTER(gs_projected), C.POINTER(gs_grad2d),
+                                              C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
+                                              C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float, C.c_float,
+                                              C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P]),
     "gs_adam": (C.c_int32, [_P, _P, _P, _P, C.c_int64, C.c_float, C.c_float, C.c_float, C.c_float, C.c_int32, _P]),
     "gs_l1_loss_grad": (C.c_int32, [_P, _P, C.c_int64, _P, _P, _P]),
     "gs_zero": (C.c_int32, [_P, C.c_size_t, _P]),
@@ -192,6 +200,40 @@ def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d
                    densify_accum: int = 0, densify_count: int = 0, stream: int = 0):
     return _check(lib().gs_project_bwd(C.byref(params), C.byref(cam), C.byref(proj), C.byref(grad2d),
                                        C.byref(grads), densify_accum or None, densify_count or None, stream))
+
+
+GS_MAX_VIEWS = 16
+
+
+def _arr(ctype, items):
+    items = list(items)
+    a = (ctype * len(items))()
+    for i, x in enumerate(items):
+        a[i] = x
+    return a
+
+
+def gs_project_bwd_views(params: gs_params, cams, projs, grad2ds, grads: gs_param_grads, densify_accum: int = 0,
+                         densify_count: int = 0, stream: int = 0):
+    """cams, projs, grad2ds: sequences of gs_camera / gs_projected / gs_grad2d (one per view)."""
+    V = len(cams)
+    return _check(lib().gs_project_bwd_views(C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs),
+                                             _arr(gs_grad2d, grad2ds), C.byref(grads), densify_accum or None,
+                                             densify_count or None, stream))
+
+
+def gs_project_bwd_views_adam(params: gs_params, cams, projs, grad2ds, params_inout: gs_param_grads,
+                              adam_m: gs_param_grads, adam_v: gs_param_grads, lrs, beta1: float, beta2: float,
+                              eps: float, step: int, grads: gs_param_grads = None, densify_accum: int = 0,
+                              densify_count: int = 0, stream: int = 0):
+    """Multi-view backward through the projection with the Adam step fused; lrs = 5 learning rates
+    (means, quats, log_scales, opacity_logits, sh)."""
+    V = len(cams)
+    lr = (C.c_float * 5)(*[float(x) for x in lrs])
+    return _check(lib().gs_project_bwd_views_adam(
+        C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _arr(gs_grad2d, grad2ds),
+        C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps, step,
+        C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None, stream))
 
 
 def gs_adam(param: int, grad: int, m: int, v: int, count: int, lr: float, beta1: float, beta2: float, eps: float,

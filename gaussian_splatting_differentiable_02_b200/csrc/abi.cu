@@ -252,35 +252,114 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
                        fn);
 }
 
-gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
-                         const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
-                         int32_t* densify_count, void* stream) {
-    const char* fn = "gs_project_bwd";
+}  // extern "C"
+
+namespace {
+
+gs_status check_grad_arrays(const char* fn, const gs_param_grads* g, const char* what) {
+    if (!g) return fail(GS_ERR_INVALID_ARG, "%s: %s is NULL", fn, what);
+    CHECK_PTR(g->means, 16);
+    CHECK_PTR(g->quats, 16);
+    CHECK_PTR(g->log_scales, 16);
+    CHECK_PTR(g->opacity_logits, 4);
+    CHECK_PTR(g->sh, 16);
+    return GS_OK;
+}
+
+// Shared checks and launch of the (multi-view) backward through the projection.
+gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t num_views, const gs_camera* cams,
+                             const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
+                             float* densify_accum, int32_t* densify_count, const gsk::AdamStep* adam,
+                             void* stream) {
     gs_status st;
     if ((st = check_params(fn, params)) != GS_OK) return st;
-    if ((st = check_camera(fn, cam)) != GS_OK) return st;
-    if ((st = check_projected(fn, proj, params->n, false)) != GS_OK) return st;
-    if (!grad2d || !grads) return fail(GS_ERR_INVALID_ARG, "%s: grad2d or grads is NULL", fn);
+    if (num_views < 1 || num_views > GS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: num_views = %d (1..%d)", fn, int(num_views), GS_MAX_VIEWS);
+    if (!cams || !projs || !grad2d) return fail(GS_ERR_INVALID_ARG, "%s: cams, projs or grad2d is NULL", fn);
     if ((densify_accum == nullptr) != (densify_count == nullptr))
         return fail(GS_ERR_INVALID_ARG, "%s: densify_accum and densify_count must both be set or both NULL", fn);
+    if (!grads && !adam) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
+    gsk::CamArgs c[GS_MAX_VIEWS];
+    for (int v = 0; v < num_views; ++v) {
+        if ((st = check_camera(fn, cams + v)) != GS_OK) return st;
+        c[v] = gsk::make_cam(cams[v]);
+        if (params->n > 0) {
+            CHECK_PTR(projs[v].radius, 4);
+            CHECK_PTR(grad2d[v].xy, 8);
+            CHECK_PTR(grad2d[v].conic_opacity, 16);
+            CHECK_PTR(grad2d[v].rgb, 16);
+        }
+    }
     if (params->n > 0) {
-        CHECK_PTR(grad2d->xy, 8);
-        CHECK_PTR(grad2d->conic_opacity, 16);
-        CHECK_PTR(grad2d->rgb, 16);
-        CHECK_PTR(grads->means, 16);
-        CHECK_PTR(grads->quats, 16);
-        CHECK_PTR(grads->log_scales, 16);
-        CHECK_PTR(grads->opacity_logits, 4);
-        CHECK_PTR(grads->sh, 16);
+        if (grads && (st = check_grad_arrays(fn, grads, "grads")) != GS_OK) return st;
         if (densify_accum) {
             CHECK_PTR(densify_accum, 4);
             CHECK_PTR(densify_count, 4);
         }
+        if (adam) {
+            if ((st = check_grad_arrays(fn, adam->params, "params_inout")) != GS_OK) return st;
+            if ((st = check_grad_arrays(fn, adam->m, "adam_m")) != GS_OK) return st;
+            if ((st = check_grad_arrays(fn, adam->v, "adam_v")) != GS_OK) return st;
+        }
     }
-    const gsk::CamArgs c = gsk::make_cam(*cam);
-    return cuda_status(gsk::launch_project_bwd(*params, c, *proj, *grad2d, *grads, densify_accum, densify_count,
-                                               static_cast<cudaStream_t>(stream)),
+    return cuda_status(gsk::launch_project_bwd_views(*params, num_views, c, cams, projs, grad2d, grads, densify_accum,
+                                                     densify_count, adam, static_cast<cudaStream_t>(stream)),
                        fn);
+}
+
+gs_status check_adam_hyper(const char* fn, float lr, float beta1, float beta2, float eps, int32_t step) {
+    if (step < 1) return fail(GS_ERR_INVALID_ARG, "%s: step must be >= 1", fn);
+    if (!std::isfinite(lr) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f))
+        return fail(GS_ERR_INVALID_ARG, "%s: invalid hyper-parameters", fn);
+    return GS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
+                         const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
+                         int32_t* densify_count, void* stream) {
+    const char* fn = "gs_project_bwd";
+    if (!grads) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
+    return project_bwd_common(fn, params, 1, cam, proj, grad2d, grads, densify_accum, densify_count, nullptr, stream);
+}
+
+gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                               const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
+                               float* densify_accum, int32_t* densify_count, void* stream) {
+    const char* fn = "gs_project_bwd_views";
+    if (!grads) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
+    return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
+                              nullptr, stream);
+}
+
+gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                    const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
+                                    gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                    float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                    float* densify_accum, int32_t* densify_count, void* stream) {
+    const char* fn = "gs_project_bwd_views_adam";
+    if (!lr_host) return fail(GS_ERR_INVALID_ARG, "%s: lr_host is NULL", fn);
+    gsk::AdamStep a;
+    gs_status st;
+    for (int g = 0; g < 5; ++g) {
+        if ((st = check_adam_hyper(fn, lr_host[g], beta1, beta2, eps, step)) != GS_OK) return st;
+        a.lr[g] = lr_host[g];
+    }
+    if (!params_inout || !adam_m || !adam_v) return fail(GS_ERR_INVALID_ARG, "%s: Adam arrays are NULL", fn);
+    if (params && (params_inout->means != params->means || params_inout->sh != params->sh))
+        return fail(GS_ERR_INVALID_ARG, "%s: params_inout must be the arrays of params", fn);
+    a.params = params_inout;
+    a.m = adam_m;
+    a.v = adam_v;
+    a.beta1 = beta1;
+    a.beta2 = beta2;
+    a.eps = eps;
+    a.step = step;
+    return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count, &a,
+                              stream);
 }
 
 gs_status gs_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,

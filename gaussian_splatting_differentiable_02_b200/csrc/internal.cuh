@@ -45,9 +45,22 @@ inline int tile_bits(int64_t tiles) {
 
 cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s);
 
-cudaError_t launch_project_bwd(const gs_params& p, const CamArgs& cam, const gs_projected& proj,
-                               const gs_grad2d& g2, const gs_param_grads& g, float* densify_accum,
-                               int32_t* densify_count, cudaStream_t s);
+// One Adam step fused into the backward pass (parameters updated in place).
+struct AdamStep {
+    const gs_param_grads* params;  // the parameter arrays (same as gs_params), written
+    const gs_param_grads* m;
+    const gs_param_grads* v;
+    float lr[5];  // means, quats, log_scales, opacity_logits, sh
+    float beta1, beta2, eps;
+    int step;
+};
+
+// Backward through the projection for V <= GS_MAX_VIEWS views of the same
+// Gaussians; grads (+=) may be null when adam is given.
+cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* cams, const gs_camera* raw,
+                                     const gs_projected* projs, const gs_grad2d* g2d, const gs_param_grads* grads,
+                                     float* densify_accum, int32_t* densify_count, const AdamStep* adam,
+                                     cudaStream_t s);
 
 struct SortWorkspace {
     unsigned long long* block_sums;  // [nb_emit]

@@ -120,9 +120,11 @@ class Projected:
         self.rect = torch.zeros((n, 4), device=device, dtype=torch.int16)   # uint16 values < 2^15
         self.tiles_touched = torch.zeros((n,), **i)                         # uint32 values < 2^31
 
-    def struct(self) -> abi.gs_projected:
+    def struct(self, radius: torch.Tensor = None) -> abi.gs_projected:
+        """The C struct; `radius` replaces the radius array (a view's own copy)."""
+        r = self.radius if radius is None else radius
         return abi.gs_projected(_ptr(self.xy), _ptr(self.depth), _ptr(self.conic_opacity), _ptr(self.rgb),
-                                _ptr(self.radius), _ptr(self.rect), _ptr(self.tiles_touched))
+                                _ptr(r), _ptr(self.rect), _ptr(self.tiles_touched))
 
 
 class Grad2D:
@@ -175,15 +177,15 @@ class View:
         self.workspace = torch.zeros((nbytes,), device=self.device, dtype=torch.uint8)
 
 
-def project(g: Gaussians, view: View, proj: Projected):
-    abi.gs_project(g.params(), view.gcam, proj.struct(), _stream())
+def project(g: Gaussians, view: View, proj: Projected, radius: torch.Tensor = None):
+    abi.gs_project(g.params(), view.gcam, proj.struct(radius), _stream())
 
 
-def bin_sort(proj: Projected, view: View):
+def bin_sort(proj: Projected, view: View, radius: torch.Tensor = None):
     """Sort the instances; grows the view's buffers when they are too small.  Returns K."""
     s = _stream()
     while True:
-        st, K = abi.gs_bin_sort(proj.struct(), view.n, view.gcam, _ptr(view.workspace), view.workspace.numel(),
+        st, K = abi.gs_bin_sort(proj.struct(radius), view.n, view.gcam, _ptr(view.workspace), view.workspace.numel(),
                                 _ptr(view.keys), _ptr(view.vals), view.capacity, _ptr(view.ranges), s, check=False)
         if st == abi.GS_OK:
             view.num_instances = K
@@ -191,21 +193,23 @@ def bin_sort(proj: Projected, view: View):
         view._alloc(int(K * 1.25) + 1024)
 
 
-def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0)):
-    abi.gs_raster_fwd(proj.struct(), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.image),
+def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Tensor = None):
+    abi.gs_raster_fwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.image),
                       _ptr(view.final_T), _ptr(view.n_contrib), _stream())
 
 
-def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), dL_dimage: torch.Tensor = None):
+def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), dL_dimage: torch.Tensor = None,
+               radius: torch.Tensor = None):
     d = view.dL_dimage if dL_dimage is None else dL_dimage
-    abi.gs_raster_bwd(proj.struct(), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.final_T),
+    abi.gs_raster_bwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.final_T),
                       _ptr(view.n_contrib), _ptr(d), grad2d.struct(), _stream())
 
 
 def project_bwd(g: Gaussians, view: View, proj: Projected, grad2d: Grad2D, grads: Gaussians,
-                densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None):
-    abi.gs_project_bwd(g.params(), view.gcam, proj.struct(), grad2d.struct(), grads.grads(), _ptr(densify_accum),
-                       _ptr(densify_count), _stream())
+                densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
+                radius: torch.Tensor = None):
+    abi.gs_project_bwd(g.params(), view.gcam, proj.struct(radius), grad2d.struct(), grads.grads(),
+                       _ptr(densify_accum), _ptr(densify_count), _stream())
 
 
 def l1_loss_grad(view: View, target: torch.Tensor, loss_dev: torch.Tensor):
@@ -222,23 +226,46 @@ def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: d
                     lrs[name], betas[0], betas[1], eps, step, s)
 
 
+def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: torch.Tensor, grad2ds: list,
+                           m: Gaussians, v: Gaussians, lrs: dict, step: int, grads: Gaussians = None,
+                           densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
+                           betas=(0.9, 0.99), eps=1e-15):
+    """Backward through the projection for all views (each with its own radius row and 2D
+    gradients) with the Adam step of all five groups fused in."""
+    abi.gs_project_bwd_views_adam(
+        g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
+        [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES],
+        betas[0], betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum),
+        _ptr(densify_count), _stream())
+
+
 @dataclass
 class Trainer:
     """One or several views of L1 training with Adam (the training loop of the gsplat guide §4.1-4.2),
-    optionally accumulating the densification statistic."""
+    optionally accumulating the densification statistic.
+
+    fused=True (default, up to GS_MAX_VIEWS views): every view keeps its own 2D
+    gradients and visibility, and one pass chains all views back to the parameters
+    and applies Adam.  fused=False: per view project_bwd into a gradient buffer,
+    then gs_adam per parameter group."""
     gauss: Gaussians
     views: list
     targets: list
     lrs: dict
     bg: tuple = (0.0, 0.0, 0.0)
     densify: bool = False
+    fused: bool = True
 
     def __post_init__(self):
         n = self.gauss.n
         dev = self.gauss.means.device
+        self.fused = self.fused and len(self.views) <= abi.GS_MAX_VIEWS
         self.proj = Projected(n, dev)
-        self.grad2d = Grad2D(n, dev)
-        self.grads = self.gauss.zeros_like()
+        nv = len(self.views) if self.fused else 1
+        self.grad2ds = [Grad2D(n, dev) for _ in range(nv)]
+        self.grad2d = self.grad2ds[0]
+        self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
+        self.grads = None if self.fused else self.gauss.zeros_like()
         self.m = self.gauss.zeros_like()
         self.v = self.gauss.zeros_like()
         self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
@@ -246,18 +273,32 @@ class Trainer:
         self.densify_count = torch.zeros((n,), device=dev, dtype=torch.int32) if self.densify else None
         self.step_count = 0
 
+    def view_forward_backward(self, k: int, target: torch.Tensor) -> None:
+        """project -> sort -> raster forward -> L1 -> raster backward of view k."""
+        view = self.views[k]
+        r = self.radii[k if self.fused else 0]
+        g2 = self.grad2ds[k if self.fused else 0]
+        project(self.gauss, view, self.proj, r)
+        bin_sort(self.proj, view, r)
+        raster_fwd(self.proj, view, self.bg, r)
+        l1_loss_grad(view, target, self.loss)
+        g2.zero_()
+        raster_bwd(self.proj, view, g2, self.bg, radius=r)
+
     def step(self) -> None:
         """forward + L1 + backward for every view, then one Adam step; loss stays on the device."""
         s = _stream()
-        self.grads.zero_()
         abi.gs_zero(_ptr(self.loss), 8, s)
-        for view, tgt in zip(self.views, self.targets):
-            project(self.gauss, view, self.proj)
-            bin_sort(self.proj, view)
-            raster_fwd(self.proj, view, self.bg)
-            l1_loss_grad(view, tgt, self.loss)
-            self.grad2d.zero_()
-            raster_bwd(self.proj, view, self.grad2d, self.bg)
-            project_bwd(self.gauss, view, self.proj, self.grad2d, self.grads, self.densify_accum, self.densify_count)
+        if not self.fused:
+            self.grads.zero_()
+        for k, tgt in enumerate(self.targets):
+            self.view_forward_backward(k, tgt)
+            if not self.fused:
+                project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
+                            self.densify_count, radius=self.radii[0])
         self.step_count += 1
-        adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)
+        if self.fused:
+            project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
+                                   self.lrs, self.step_count, None, self.densify_accum, self.densify_count)
+        else:
+            adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)

@@ -233,6 +233,35 @@ gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs
                          const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
                          int32_t* densify_count, void* stream);
 
+/* Most views one multi-view backward call takes. */
+#define GS_MAX_VIEWS 16
+
+/* gs_project_bwd_views -- gs_project_bwd for num_views (1..GS_MAX_VIEWS) views of
+ * the same Gaussians in one pass: cams, projs and grad2d are host arrays of
+ * num_views structs (of projs only `radius` is read: a Gaussian counts as
+ * visible in a view when its radius there is > 0).  Every Gaussian reads its
+ * parameters once, adds every visible view's contribution in registers and
+ * accumulates the sum over views into grads (+=); densify statistics as in
+ * gs_project_bwd, summed over views.  Equal, up to rounding, to num_views calls
+ * of gs_project_bwd. */
+gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                               const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
+                               float* densify_accum, int32_t* densify_count, void* stream);
+
+/* gs_project_bwd_views_adam -- gs_project_bwd_views followed by the Adam step of
+ * gs_adam for all five parameter groups in the same pass (gsplat guide §4.2:
+ * lr_host[5] for means, quats, log_scales, opacity_logits, sh; shared betas,
+ * eps and step).  params_inout holds the same arrays as params and is updated
+ * in place; adam_m and adam_v are the first and second moments in the
+ * parameter layout.  The summed gradient goes straight into Adam; grads, when
+ * non-NULL, also receives it (+=).  Every Gaussian is updated, visible or not,
+ * as gs_adam updates every element. */
+gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                    const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
+                                    gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                    float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                    float* densify_accum, int32_t* densify_count, void* stream);
+
 /* gs_adam -- one bias-corrected Adam step on `count` floats (gsplat guide §4.2:
  * one call per parameter group with its own lr; betas 0.9, 0.99; eps 1e-15):
  *   m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2;

@@ -1,0 +1,159 @@
+"""Parity of the multi-view backward through the projection (gs_project_bwd_views)
+and of the fused Adam step (gs_project_bwd_views_adam) with the oracle: the sum
+over views of the oracle's dual-number chain, then the oracle's Adam."""
+import numpy as np
+import pytest
+import torch
+
+from gaussian_splatting_differentiable_02_b200 import abi, scenes
+from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+
+from _parity import check_grads
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("means", "quats", "log_scales", "opacity_logits", "sh")
+LRS = {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3, "opacity_logits": 5e-2, "sh": 2.5e-3}
+
+
+def _views(n_views, seed=0):
+    rng = np.random.default_rng(seed)
+    cams = []
+    for k in range(n_views):
+        eye = rng.standard_normal(3)
+        eye = 4.0 * eye / np.linalg.norm(eye)
+        R, t = scenes.look_at(eye)
+        cams.append(scenes.camera(R, t, 128.0, 128.0, 64.0, 64.0, 128, 128))
+    return cams
+
+
+def _setup(orc, n_views=3, deg=2, seed=5):
+    rng = np.random.default_rng(seed)
+    scene = scenes.random_scene(rng, 800, deg, mean_box=1.0, log_scale=(-4.0, -2.0))
+    cams = _views(n_views, seed)
+    g = pl.Gaussians.from_scene(scene)
+    proj = pl.Projected(scene.n)
+    radii = torch.zeros((n_views, scene.n), dtype=torch.int32, device="cuda")
+    views, g2s, g2_rows = [], [], []
+    for k, cam in enumerate(cams):
+        view = pl.View(scene.n, cam)
+        pl.project(g, view, proj, radii[k])
+        views.append(view)
+        ref = orc.project(scene, cam)
+        assert np.array_equal(radii[k].cpu().numpy(), ref["radius"])
+        up = rng.standard_normal((128 * 128, 3))
+        g2, _, _ = orc.render_bwd(ref, cam, up)
+        rows = g2.astype(np.float32)
+        g2_rows.append(rows)
+        gd = pl.Grad2D(scene.n)
+        gd.xy.copy_(torch.from_numpy(np.ascontiguousarray(rows[:, 0:2])))
+        gd.conic_opacity.copy_(torch.from_numpy(np.ascontiguousarray(rows[:, 2:6])))
+        rgb = np.zeros((scene.n, 4), np.float32)
+        rgb[:, :3] = rows[:, 6:9]
+        gd.rgb.copy_(torch.from_numpy(rgb))
+        g2s.append(gd)
+    torch.cuda.synchronize()
+    want = {k: 0.0 for k in NAMES}
+    acc = np.zeros(scene.n)
+    cnt = np.zeros(scene.n, np.int64)
+    for cam, rows in zip(cams, g2_rows):
+        o = orc.project_bwd(scene, cam, rows.astype(np.float64), densify=True)
+        for k in NAMES:
+            want[k] = want[k] + o[k]
+        acc += o["densify_accum"]
+        cnt += o["densify_count"]
+    return scene, cams, g, proj, radii, views, g2s, want, acc, cnt
+
+
+def test_views_equal_sum_of_single_view_chains(orc):
+    scene, cams, g, proj, radii, views, g2s, want, acc, cnt = _setup(orc)
+    grads = g.zeros_like()
+    da = torch.zeros(scene.n, device="cuda")
+    dc = torch.zeros(scene.n, dtype=torch.int32, device="cuda")
+    abi.gs_project_bwd_views(g.params(), [v.gcam for v in views], [proj.struct(radii[k]) for k in range(len(views))],
+                             [x.struct() for x in g2s], grads.grads(), da.data_ptr(), dc.data_ptr(),
+                             torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    got = grads.to_numpy()
+    vis = np.nonzero(cnt > 0)[0]
+    assert len(vis) > 500
+    for k in NAMES:
+        check_grads(got[k].reshape(scene.n, -1), np.asarray(want[k]).reshape(scene.n, -1), k, rows=vis)
+    np.testing.assert_allclose(da.cpu().numpy(), acc, rtol=1e-5, atol=1e-9)
+    assert np.array_equal(dc.cpu().numpy(), cnt)
+
+
+@pytest.mark.parametrize("deg", [0, 3])
+def test_fused_adam_matches_oracle_adam_of_summed_gradients(orc, deg):
+    scene, cams, g, proj, radii, views, g2s, want, acc, cnt = _setup(orc, n_views=4, deg=deg, seed=9)
+    rng = np.random.default_rng(3)
+    m, v = g.zeros_like(), g.zeros_like()
+    for t in list(m.tensors().values()) + list(v.tensors().values()):
+        t.copy_(torch.from_numpy((0.01 * rng.random(tuple(t.shape))).astype(np.float32)))
+    p0 = {k: getattr(g, k).cpu().numpy().copy() for k in NAMES}
+    m0 = {k: getattr(m, k).cpu().numpy().copy() for k in NAMES}
+    v0 = {k: getattr(v, k).cpu().numpy().copy() for k in NAMES}
+    grads = g.zeros_like()
+    step = 3
+    b1, b2, eps = (float(np.float32(x)) for x in (0.9, 0.99, 1e-15))
+    lrs = [float(np.float32(LRS[k])) for k in NAMES]
+    abi.gs_project_bwd_views_adam(g.params(), [vw.gcam for vw in views],
+                                  [proj.struct(radii[k]) for k in range(len(views))], [x.struct() for x in g2s],
+                                  g.grads(), m.grads(), v.grads(), lrs, b1, b2, eps, step, grads.grads(), 0, 0,
+                                  torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    # the summed gradient it applied
+    got_g = grads.to_numpy()
+    vis = np.nonzero(cnt > 0)[0]
+    for k in NAMES:
+        check_grads(got_g[k].reshape(scene.n, -1), np.asarray(want[k]).reshape(scene.n, -1), k, rows=vis)
+    # Adam on the device layout: compare with the oracle's Adam of the reference gradient, rows where the
+    # reference gradient is not a near-zero cancellation (there Adam's direction is not determined)
+    eps32 = float(np.finfo(np.float32).eps)
+    for gi, k in enumerate(NAMES):
+        gref = np.zeros_like(p0[k])
+        w = np.asarray(want[k])
+        if k in ("means", "log_scales"):
+            gref[:, :3] = w
+        elif k == "sh":
+            gref[:] = pl.sh_to_planes(w.astype(np.float32))
+        else:
+            gref[:] = w.reshape(gref.shape)
+        p1, m1, v1 = orc.adam(p0[k], gref.astype(np.float32), m0[k], v0[k], lrs[gi], b1, b2, eps, step)
+        gp, gm, gv = getattr(g, k).cpu().numpy(), getattr(m, k).cpu().numpy(), getattr(v, k).cpu().numpy()
+        gerr = np.abs(getattr(grads, k).cpu().numpy() - gref)
+        assert np.all(np.abs(gm - m1) <= 3 * eps32 * (np.abs(m1) + 0.1 * np.abs(gref)) + 0.1 * gerr + 1e-12), k
+        assert np.all(np.abs(gv - v1) <= 3 * eps32 * (np.abs(v1) + 0.01 * gref ** 2) + 0.02 * gerr * np.abs(gref)
+                      + 1e-12), k
+        upd = np.abs(p1.astype(np.float64) - p0[k])
+        bound = eps32 * np.maximum(np.abs(p1), np.abs(p0[k])) + 1e-3 * upd + 1e-9
+        assert np.all(np.abs(gp - p1) <= bound), (k, float(np.max(np.abs(gp - p1) - bound)))
+
+
+def test_trainer_fused_equals_unfused():
+    """The fused multi-view step and the per-view step + gs_adam update the same
+    parameters (both CUDA paths; a consistency check next to the oracle parity)."""
+    rng = np.random.default_rng(12)
+    scene = scenes.random_scene(rng, 600, 1, mean_box=1.0, log_scale=(-3.5, -2.0))
+    cams = _views(3, 4)
+    targets = [torch.from_numpy(rng.random((128, 128, 3)).astype(np.float32)).cuda() for _ in cams]
+    out = []
+    for fused in (True, False):
+        g = pl.Gaussians.from_scene(scene)
+        tr = pl.Trainer(g, [pl.View(scene.n, c) for c in cams], targets, dict(LRS), densify=True, fused=fused)
+        tr.step()
+        tr.step()
+        torch.cuda.synchronize()
+        out.append((g.to_numpy(), tr.densify_accum.cpu().numpy(), tr.densify_count.cpu().numpy(), tr.loss.item()))
+    (a, da, ca, la), (b, db, cb, lb) = out
+    assert np.array_equal(ca, cb)
+    np.testing.assert_allclose(da, db, rtol=1e-5, atol=1e-9)
+    assert abs(la - lb) <= 1e-9 * max(1.0, abs(la))
+    for k in NAMES:
+        # identical up to the rounding of the per-view float32 accumulation; Adam's first
+        # steps move by about lr * sign(g), so an element whose gradient is a near-zero
+        # cancellation may move the other way (at most 2 lr per step)
+        d = np.abs(a[k] - b[k])
+        close = d <= 1e-6 + 1e-6 * np.abs(a[k])
+        assert close.mean() >= 0.999, (k, float(close.mean()))
+        assert d.max() <= 4 * LRS[k] + 1e-6, (k, float(d.max()))
