@@ -68,10 +68,13 @@ SIGNATURES = {
                                 C.c_int64, C.POINTER(C.c_int64), _P, _P]),
     "gs_bin_sort_static": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, _P, C.c_int64,
                                        C.POINTER(C.c_int64), _P, _P]),
-    "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
-                                  _P, _P, _P]),
-    "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float), _P,
-                                  _P, _P, C.POINTER(gs_grad2d), _P]),
+    "gs_bin_sort_async": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, C.c_size_t, _P, _P,
+                                      C.c_int64, _P, _P, _P]),
+    "gs_tile_order": (C.c_int32, [_P, C.POINTER(gs_camera), _P, _P]),
+    "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
+                                  _P, _P, _P, _P]),
+    "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
+                                  _P, _P, _P, C.POINTER(gs_grad2d), _P]),
     "gs_project_bwd": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected),
                                    C.POINTER(gs_grad2d), C.POINTER(gs_param_grads), _P, _P, _P]),
     "gs_project_bwd_views": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
@@ -167,6 +170,13 @@ def gs_bin_sort(proj: gs_projected, n: int, cam: gs_camera, workspace: int, work
     return st, K.value
 
 
+def gs_bin_sort_async(proj: gs_projected, n: int, cam: gs_camera, workspace: int, workspace_bytes: int, keys: int,
+                      vals: int, capacity: int, num_instances_dev: int, tile_ranges: int, stream: int = 0):
+    """gs_bin_sort without a host wait: K goes to the device uint64 at num_instances_dev."""
+    return _check(lib().gs_bin_sort_async(C.byref(proj), n, C.byref(cam), workspace, workspace_bytes, keys, vals,
+                                          capacity, num_instances_dev, tile_ranges, stream))
+
+
 GS_STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -182,18 +192,23 @@ def gs_bin_sort_static(proj: gs_projected, n: int, cam: gs_camera, keys: int, va
     return st, K.value
 
 
-def gs_raster_fwd(proj: gs_projected, vals: int, tile_ranges: int, cam: gs_camera, bg, image: int, final_T: int,
-                  n_contrib: int, stream: int = 0):
-    b = (C.c_float * 3)(*[float(x) for x in bg])
-    return _check(lib().gs_raster_fwd(C.byref(proj), vals, tile_ranges, C.byref(cam), b, image, final_T, n_contrib,
-                                      stream))
+def gs_tile_order(tile_ranges: int, cam: gs_camera, tile_order: int, stream: int = 0):
+    return _check(lib().gs_tile_order(tile_ranges, C.byref(cam), tile_order, stream))
 
 
-def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, cam: gs_camera, bg, final_T: int, n_contrib: int,
-                  dL_dimage: int, grad2d: gs_grad2d, stream: int = 0):
+def gs_raster_fwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg, image: int,
+                  final_T: int, n_contrib: int, stream: int = 0):
+    """tile_order: device pointer from gs_tile_order, or 0 for the natural tile order."""
     b = (C.c_float * 3)(*[float(x) for x in bg])
-    return _check(lib().gs_raster_bwd(C.byref(proj), vals, tile_ranges, C.byref(cam), b, final_T, n_contrib,
-                                      dL_dimage, C.byref(grad2d), stream))
+    return _check(lib().gs_raster_fwd(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b, image,
+                                      final_T, n_contrib, stream))
+
+
+def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg, final_T: int,
+                  n_contrib: int, dL_dimage: int, grad2d: gs_grad2d, stream: int = 0):
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_bwd(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b,
+                                      final_T, n_contrib, dL_dimage, C.byref(grad2d), stream))
 
 
 def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d: gs_grad2d, grads: gs_param_grads,

@@ -173,16 +173,23 @@ size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera*
     return gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
 }
 
-gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
-                      size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
-                      int64_t* num_instances_host, uint32_t* tile_ranges, void* stream) {
-    const char* fn = "gs_bin_sort";
+}  // extern "C"
+
+namespace {
+
+// Checks and launch of the binning + sort.  With num_instances_host the call
+// waits for K and reports GS_ERR_CAPACITY; with count_dev it returns at once.
+gs_status bin_sort_impl(const char* fn, const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                        size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                        int64_t* num_instances_host, unsigned long long* count_dev, uint32_t* tile_ranges,
+                        void* stream) {
     gs_status st;
     if (n < 0 || n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n out of range", fn);
     if (capacity < 0 || capacity > 0xffffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: capacity out of range", fn);
     if ((st = check_camera(fn, cam)) != GS_OK) return st;
     if ((st = check_projected(fn, proj, n, true)) != GS_OK) return st;
-    if (!num_instances_host) return fail(GS_ERR_INVALID_ARG, "%s: num_instances_host is NULL", fn);
+    if (!num_instances_host && !count_dev) return fail(GS_ERR_INVALID_ARG, "%s: instance count output is NULL", fn);
+    if (count_dev) CHECK_PTR(count_dev, 8);
     CHECK_PTR(workspace, 16);
     CHECK_PTR(tile_ranges, 8);
     if (capacity > 0) {
@@ -197,8 +204,10 @@ gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     gsk::SortWorkspace ws;
     gsk::sort_workspace_layout(n, capacity, workspace, &ws);
-    cudaError_t e = gsk::launch_count_instances(*proj, n, ws, s);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    cudaError_t e = gsk::launch_bin_sort(*proj, n, c, ws, keys, vals, capacity, tile_ranges, count_dev, s);
     if (e != cudaSuccess) return cuda_status(e, fn);
+    if (!num_instances_host) return ok();
     unsigned long long K = 0;
     e = cudaMemcpyAsync(&K, ws.total, sizeof K, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -206,13 +215,43 @@ gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam,
     *num_instances_host = int64_t(K);
     if (int64_t(K) > capacity)
         return fail(GS_ERR_CAPACITY, "%s: %llu instances, capacity %lld", fn, K, (long long)capacity);
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                      size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                      int64_t* num_instances_host, uint32_t* tile_ranges, void* stream) {
+    if (!num_instances_host) return fail(GS_ERR_INVALID_ARG, "gs_bin_sort: num_instances_host is NULL");
+    return bin_sort_impl("gs_bin_sort", proj, n, cam, workspace, workspace_bytes, keys, vals, capacity,
+                         num_instances_host, nullptr, tile_ranges, stream);
+}
+
+gs_status gs_bin_sort_async(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                            size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                            uint64_t* num_instances_dev, uint32_t* tile_ranges, void* stream) {
+    if (!num_instances_dev) return fail(GS_ERR_INVALID_ARG, "gs_bin_sort_async: num_instances_dev is NULL");
+    return bin_sort_impl("gs_bin_sort_async", proj, n, cam, workspace, workspace_bytes, keys, vals, capacity,
+                         nullptr, reinterpret_cast<unsigned long long*>(num_instances_dev), tile_ranges, stream);
+}
+
+gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint32_t* tile_order, void* stream) {
+    const char* fn = "gs_tile_order";
+    gs_status st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    CHECK_PTR(tile_ranges, 8);
+    CHECK_PTR(tile_order, 4);
     const gsk::CamArgs c = gsk::make_cam(*cam);
-    return cuda_status(gsk::launch_emit_sort_ranges(*proj, n, c, ws, keys, vals, int64_t(K), tile_ranges, s), fn);
+    return cuda_status(gsk::launch_tile_order(tile_ranges, c.TX * c.TY, tile_order, static_cast<cudaStream_t>(stream)),
+                       fn);
 }
 
 gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const gs_camera* cam, const float* bg_host, float* image, float* final_T,
-                        int32_t* n_contrib, void* stream) {
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
+                        float* final_T, int32_t* n_contrib, void* stream) {
     const char* fn = "gs_raster_fwd";
     gs_status st;
     if ((st = check_camera(fn, cam)) != GS_OK) return st;
@@ -220,17 +259,18 @@ gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const ui
     if (!bg_host) return fail(GS_ERR_INVALID_ARG, "%s: bg_host is NULL", fn);
     CHECK_PTR(vals, 4);
     CHECK_PTR(tile_ranges, 8);
+    if (tile_order) CHECK_PTR(tile_order, 4);
     CHECK_PTR(image, 4);
     CHECK_PTR(final_T, 4);
     CHECK_PTR(n_contrib, 4);
     const gsk::CamArgs c = gsk::make_cam(*cam);
-    return cuda_status(gsk::launch_raster_fwd(*proj, vals, tile_ranges, c, bg_host, image, final_T, n_contrib,
-                                              static_cast<cudaStream_t>(stream)),
+    return cuda_status(gsk::launch_raster_fwd(*proj, vals, tile_ranges, tile_order, c, bg_host, image, final_T,
+                                              n_contrib, static_cast<cudaStream_t>(stream)),
                        fn);
 }
 
 gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const gs_camera* cam, const float* bg_host, const float* final_T,
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* final_T,
                         const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream) {
     const char* fn = "gs_raster_bwd";
     gs_status st;
@@ -240,6 +280,7 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
     if (!grad2d) return fail(GS_ERR_INVALID_ARG, "%s: grad2d is NULL", fn);
     CHECK_PTR(vals, 4);
     CHECK_PTR(tile_ranges, 8);
+    if (tile_order) CHECK_PTR(tile_order, 4);
     CHECK_PTR(final_T, 4);
     CHECK_PTR(n_contrib, 4);
     CHECK_PTR(dL_dimage, 4);
@@ -247,8 +288,8 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
     CHECK_PTR(grad2d->conic_opacity, 16);
     CHECK_PTR(grad2d->rgb, 16);
     const gsk::CamArgs c = gsk::make_cam(*cam);
-    return cuda_status(gsk::launch_raster_bwd(*proj, vals, tile_ranges, c, bg_host, final_T, n_contrib, dL_dimage,
-                                              *grad2d, static_cast<cudaStream_t>(stream)),
+    return cuda_status(gsk::launch_raster_bwd(*proj, vals, tile_ranges, tile_order, c, bg_host, final_T, n_contrib,
+                                              dL_dimage, *grad2d, static_cast<cudaStream_t>(stream)),
                        fn);
 }
 

@@ -1,7 +1,7 @@
-// gs_bin_sort: tile binning with a (tile_id << 32 | depth) key (the "culling and
-// reordering" stage the MUSA co-design article, qwbw.cn/news/278220 §1, lists
-// among the four 3DGS bottlenecks; the screen-space ordering of the gsplat
-// guide, lmnt.cn/news/262699 §4.1).
+// gs_bin_sort / gs_bin_sort_async: tile binning with a (tile_id << 32 | depth)
+// key (the "culling and reordering" stage the MUSA co-design article,
+// qwbw.cn/news/278220 §1, lists among the four 3DGS bottlenecks; the
+// screen-space ordering of the gsplat guide, lmnt.cn/news/262699 §4.1).
 //
 // The result is the list of instances sorted by (key, Gaussian index).  It is
 // produced without sorting 64-bit keys: the Gaussians are first sorted by depth
@@ -11,6 +11,11 @@
 // of a sequence ordered by (depth, gid) is ordered by (tile, depth, gid).  The
 // last tile pass writes the 64-bit key, taking the depth bits from the
 // Gaussian.  This moves about a third of the bytes of a 64-bit key sort.
+//
+// The instance count K stays on the device: the passes over instances are
+// launched for the caller's capacity and read K when they start, so nothing
+// waits for the host.  When K exceeds the capacity nothing is emitted or
+// sorted and every tile range is left empty.
 //
 // Kernels (no kernel waits on another block, so nothing here can spin):
 //   depth_keys        key = float32 bits of the depth (culled: 0xffffffff), val = gid
@@ -34,11 +39,27 @@ constexpr int kEmitBlock = 256;
 constexpr int kEmitPerThread = 8;
 constexpr int kEmitChunk = kEmitBlock * kEmitPerThread;  // Gaussians per emit block
 
+#ifndef GS_SORT_ITEMS
+#define GS_SORT_ITEMS 8
+#endif
 constexpr int kSortBlock = 256;
 constexpr int kSortWarps = kSortBlock / 32;
-constexpr int kSortPerThread = 16;
+constexpr int kSortPerThread = GS_SORT_ITEMS;
 constexpr int kSortTile = kSortBlock * kSortPerThread;  // elements per sort block
 constexpr int kWarpSpan = 32 * kSortPerThread;           // elements per warp
+
+// Number of elements a pass covers: a host count, or the device instance count
+// (0 when it exceeds the capacity).
+struct Count {
+    int64_t host;
+    const unsigned long long* dev;
+    int64_t limit;
+    __device__ __forceinline__ int64_t get() const {
+        if (!dev) return host;
+        const unsigned long long k = *dev;
+        return k <= static_cast<unsigned long long>(limit) ? static_cast<int64_t>(k) : 0;
+    }
+};
 
 __device__ __forceinline__ unsigned long long warp_incl_scan(unsigned long long v) {
     const int lane = threadIdx.x & 31;
@@ -79,9 +100,10 @@ __global__ void __launch_bounds__(256) depth_keys_kernel(const uint32_t* __restr
     }
 }
 
-__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __restrict__ keys, int64_t count,
+__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __restrict__ keys, const Count cnt,
                                                              int shift, uint32_t* __restrict__ hist, int64_t nb) {
     __shared__ uint32_t h[kSortWarps][256];
+    const int64_t count = cnt.get();
     const int warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&h[0][0])[k] = 0u;
     __syncthreads();
@@ -121,7 +143,7 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
                                                                const uint32_t* __restrict__ vals_in,
                                                                uint32_t* __restrict__ keys_out,
                                                                uint64_t* __restrict__ keys_out64,
-                                                               uint32_t* __restrict__ vals_out, int64_t count,
+                                                               uint32_t* __restrict__ vals_out, const Count cnt,
                                                                int shift, const uint32_t* __restrict__ hist,
                                                                int64_t nb, const uint32_t* __restrict__ digit_totals,
                                                                const float* __restrict__ depth) {
@@ -130,6 +152,9 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
     __shared__ uint32_t lstart[256];  // start of each digit's run within the block
     __shared__ uint32_t sk[kSortTile];
     __shared__ uint32_t sv[kSortTile];
+    const int64_t count = cnt.get();
+    const int64_t tile0 = int64_t(blockIdx.x) * kSortTile;
+    if (tile0 >= count) return;  // block-uniform: launched for the capacity
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&wcount[0][0])[k] = 0u;
     {
@@ -139,7 +164,6 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
     }
     __syncthreads();
 
-    const int64_t tile0 = int64_t(blockIdx.x) * kSortTile;
     const int64_t base = tile0 + int64_t(warp) * kWarpSpan;
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t key[kSortPerThread], val[kSortPerThread], rank[kSortPerThread];
@@ -215,7 +239,8 @@ __global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const uint32_t
 }
 
 __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
-                                                           unsigned long long* total) {
+                                                           unsigned long long* total,
+                                                           unsigned long long* total_copy) {
     unsigned long long carry = 0;
     for (int64_t base = 0; base < nb; base += 1024) {
         const int64_t i = base + threadIdx.x;
@@ -225,14 +250,19 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* b
         if (i < nb) block_sums[i] = carry + ex;
         carry += tot;
     }
-    if (threadIdx.x == 0) *total = carry;
+    if (threadIdx.x == 0) {
+        *total = carry;
+        if (total_copy) *total_copy = carry;
+    }
 }
 
 __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
                                                           const uint2* __restrict__ rect,
                                                           const uint32_t* __restrict__ order, int64_t n, int tiles_x,
                                                           const unsigned long long* __restrict__ block_offsets,
-                                                          uint32_t* __restrict__ tkeys, uint32_t* __restrict__ tvals) {
+                                                          const Count cnt, uint32_t* __restrict__ tkeys,
+                                                          uint32_t* __restrict__ tvals) {
+    if (cnt.get() == 0) return;  // nothing fits: emit nothing
     const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
     uint32_t gid[kEmitPerThread], tt[kEmitPerThread];
     unsigned long long mine = 0;
@@ -258,8 +288,9 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __rest
     }
 }
 
-__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict__ keys, int64_t K,
+__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict__ keys, const Count cnt,
                                                      uint2* __restrict__ ranges) {
+    const int64_t K = cnt.get();
     for (int64_t k = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; k < K; k += int64_t(gridDim.x) * blockDim.x) {
         const uint32_t t = uint32_t(__ldg(keys + k) >> 32);
         if (k == 0 || uint32_t(__ldg(keys + k - 1) >> 32) != t) ranges[t].x = uint32_t(k);
@@ -269,17 +300,19 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict_
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
-// One LSD pass over `count` (key, val) pairs.  Final passes write 64-bit keys.
+// One LSD pass over up to `slots` (key, val) pairs (`cnt` of them when the pass
+// starts).  Final passes write 64-bit keys.
 void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout, uint64_t* kout64, uint32_t* vout,
-                int64_t count, int shift, const SortWorkspace& ws, const float* depth, cudaStream_t s) {
-    const int64_t nb = (count + kSortTile - 1) / kSortTile;
-    upsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(kin, count, shift, ws.hist, nb);
+                Count cnt, int64_t slots, int shift, const SortWorkspace& ws, const float* depth, cudaStream_t s) {
+    const int64_t nb = (slots + kSortTile - 1) / kSortTile;
+    if (nb == 0) return;
+    upsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(kin, cnt, shift, ws.hist, nb);
     scan_hist_kernel<<<256, 1024, 0, s>>>(ws.hist, nb, ws.digit_totals);
     if (kout64)
-        downsweep_kernel<true><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, count, shift,
+        downsweep_kernel<true><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, cnt, shift,
                                                                    ws.hist, nb, ws.digit_totals, depth);
     else
-        downsweep_kernel<false><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, count, shift,
+        downsweep_kernel<false><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, cnt, shift,
                                                                     ws.hist, nb, ws.digit_totals, depth);
     count_launches(3);
 }
@@ -313,33 +346,35 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
     return off;
 }
 
-// Depth order of the Gaussians (into tkey/tval[1], so that tval[1] holds the
-// order while the instances are emitted into buffer 0), then the instance count.
-cudaError_t launch_count_instances(const gs_projected& proj, int64_t n, const SortWorkspace& ws, cudaStream_t s) {
+cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
+                            uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* ranges,
+                            unsigned long long* count_out, cudaStream_t s) {
+    const int64_t T = int64_t(cam.TX) * cam.TY;
+    cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint32_t) * 2 * size_t(T), s);
+    if (e != cudaSuccess) return e;
     if (n == 0) {
-        cudaMemsetAsync(ws.total, 0, sizeof(unsigned long long), s);
-        return cudaGetLastError();
+        e = cudaMemsetAsync(ws.total, 0, sizeof(unsigned long long), s);
+        if (e == cudaSuccess && count_out) e = cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), s);
+        return e;
     }
+    // depth order of the Gaussians: 4 passes from buffer 1 back into buffer 1, so
+    // that tval[1] holds the order while the instances are emitted into buffer 0
     depth_keys_kernel<<<grid_for(n, 256, 8), 256, 0, s>>>(proj.tiles_touched, proj.depth, n, ws.tkey[1], ws.tval[1]);
     count_launches(1);
-    for (int p = 0; p < 4; ++p) {  // 4 passes: the order ends in buffer 1 again
+    const Count all{n, nullptr, 0};
+    for (int p = 0; p < 4; ++p) {
         const int src = (p & 1) ? 0 : 1;
-        radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], n, 8 * p, ws, nullptr, s);
+        radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], all, n, 8 * p, ws,
+                   nullptr, s);
     }
     count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, ws.tval[1], n,
                                                                     ws.block_sums);
-    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total);
+    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total, count_out);
     count_launches(2);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_emit_sort_ranges(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
-                                    uint64_t* keys, uint32_t* vals, int64_t K, uint32_t* ranges, cudaStream_t s) {
-    const int64_t T = int64_t(cam.TX) * cam.TY;
-    cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint32_t) * 2 * size_t(T), s);
-    if (e != cudaSuccess || K == 0) return e;
+    // instances: launched for the capacity, K read on the device
+    const Count inst{0, ws.total, capacity};
     emit_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, reinterpret_cast<const uint2*>(proj.rect),
-                                                            ws.tval[1], n, cam.TX, ws.block_sums, ws.tkey[0],
+                                                            ws.tval[1], n, cam.TX, ws.block_sums, inst, ws.tkey[0],
                                                             ws.tval[0]);
     count_launches(1);
     const int bits = tile_bits(T);
@@ -348,11 +383,13 @@ cudaError_t launch_emit_sort_ranges(const gs_projected& proj, int64_t n, const C
     for (int p = 0; p < passes; ++p) {
         const bool last = p == passes - 1;
         radix_pass(ws.tkey[cur], ws.tval[cur], last ? nullptr : ws.tkey[cur ^ 1], last ? keys : nullptr,
-                   last ? vals : ws.tval[cur ^ 1], K, 8 * p, ws, proj.depth, s);
+                   last ? vals : ws.tval[cur ^ 1], inst, capacity, 8 * p, ws, proj.depth, s);
         cur ^= 1;
     }
-    ranges_kernel<<<grid_for(K, 256, 8), 256, 0, s>>>(keys, K, reinterpret_cast<uint2*>(ranges));
-    count_launches(1);
+    if (capacity > 0) {
+        ranges_kernel<<<grid_for(capacity, 256, 8), 256, 0, s>>>(keys, inst, reinterpret_cast<uint2*>(ranges));
+        count_launches(1);
+    }
     return cudaGetLastError();
 }
 

@@ -73,17 +73,22 @@ struct SortWorkspace {
 };
 size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws);
 
-cudaError_t launch_count_instances(const gs_projected& proj, int64_t n, const SortWorkspace& ws, cudaStream_t s);
-cudaError_t launch_emit_sort_ranges(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
-                                    uint64_t* keys, uint32_t* vals, int64_t K, uint32_t* ranges, cudaStream_t s);
+// Enqueues the whole binning and sort; the instance count stays on the device
+// (ws.total, and *count_out when given).  K > capacity: nothing emitted, ranges empty.
+cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
+                            uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* ranges,
+                            unsigned long long* count_out, cudaStream_t s);
+
+cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s);
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
-                              const CamArgs& cam, const float bg[3], float* image, float* final_T,
-                              int32_t* n_contrib, cudaStream_t s);
+                              const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
+                              float* final_T, int32_t* n_contrib, cudaStream_t s);
 
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
-                              const CamArgs& cam, const float bg[3], const float* final_T, const int32_t* n_contrib,
-                              const float* dL_dimage, const gs_grad2d& g2, cudaStream_t s);
+                              const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,
+                              const int32_t* n_contrib, const float* dL_dimage, const gs_grad2d& g2,
+                              cudaStream_t s);
 
 cudaError_t launch_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
                         float beta2, float eps, int32_t step, cudaStream_t s);

@@ -209,6 +209,7 @@ struct FwdArgs {
     const float4* rgb;
     const uint32_t* vals;
     const uint2* ranges;
+    const uint32_t* order;  // tile processing order (nullable)
     int W, H, TX, tiles;
     float bg0, bg1, bg2;
     float* image;
@@ -220,8 +221,9 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
-    const int tile = gw / kSub, sub = gw % kSub;
-    if (tile >= a.tiles) return;
+    const int slot = gw / kSub, sub = gw % kSub;
+    if (slot >= a.tiles) return;
+    const int tile = a.order ? int(__ldg(a.order + slot)) : slot;  // longest lists first when ordered
     WarpStage& S = stage[warp];
     const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
     const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
@@ -313,6 +315,7 @@ struct BwdArgs {
     const float4* rgb;
     const uint32_t* vals;
     const uint2* ranges;
+    const uint32_t* order;  // tile processing order (nullable)
     int W, H, TX, tiles;
     float bg0, bg1, bg2;
     const float* final_T;
@@ -374,8 +377,9 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
-    const int tile = gw / kSub, sub = gw % kSub;
-    if (tile >= a.tiles) return;
+    const int slot = gw / kSub, sub = gw % kSub;
+    if (slot >= a.tiles) return;
+    const int tile = a.order ? int(__ldg(a.order + slot)) : slot;  // longest lists first when ordered
     WarpStage& S = stage[warp];
     const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
     const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
@@ -385,12 +389,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     const float bx0 = float(xb) + 0.5f, by0 = float(yb) + 0.5f;  // box corner (pixel centre)
     const uint2 range = a.ranges[tile];
 
-    float T[kPx], Sr[kPx], Sg[kPx], Sb[kPx], gr[kPx], gg[kPx], gb[kPx], ngb[kPx];
+    float T[kPx], P[kPx], gr[kPx], gg[kPx], gb[kPx], ngb[kPx];
     int last[kPx];
     int lmax = 0;
 #pragma unroll
     for (int i = 0; i < kPx; ++i) {
-        Sr[i] = Sg[i] = Sb[i] = 0.f;
+        P[i] = 0.f;
         if (x < a.W && y0 + i < a.H) {
             const int64_t pix = int64_t(y0 + i) * a.W + x;
             T[i] = a.final_T[pix];
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             float al[kPx], dy[kPx], m[kPx], dx;
             unsigned blend, clamp;
             eval_alpha(pa, pb, con, px, y0, al, blend, clamp, dx, dy);
-            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s0 = 0.f, s1 = 0.f, s2 = 0.f;
+            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s1 = 0.f, s2 = 0.f;
             bool any = false;
             // branch-free: every pixel runs the same instructions, inactive ones
             // with zero weight and unchanged state
@@ -451,17 +455,16 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                 dr = fmaf(w, gr[i], dr);
                 dg = fmaf(w, gg[i], dg);
                 db = fmaf(w, gb[i], db);
-                const float xr = c.x - Sr[i], xg = c.y - Sg[i], xb = c.z - Sb[i];
-                const float dLda = fmaf(T[i], fmaf(gr[i], xr, fmaf(gg[i], xg, gb[i] * xb)), ngb[i] * rom);
-                Sr[i] = fmaf(ae, xr, Sr[i]);  // S <- c alpha + (1 - alpha) S
-                Sg[i] = fmaf(ae, xg, Sg[i]);
-                Sb[i] = fmaf(ae, xb, Sb[i]);
+                // only g . S enters the gradient: P = g . S with S <- c alpha + (1 - alpha) S
+                const float x = fmaf(gr[i], c.x, fmaf(gg[i], c.y, gb[i] * c.z)) - P[i];
+                const float dLda = fmaf(T[i], x, ngb[i] * rom);
+                P[i] = fmaf(ae, x, P[i]);
                 m[i] = ((clamp >> i) & 1u) ? 0.f : dLda * ae;  // dL/dsigma = -m, dL/do = m / o
                 mo += m[i];
-                s0 -= m[i];
                 s1 = fmaf(-m[i], dy[i], s1);
                 s2 = fmaf(-m[i] * dy[i], dy[i], s2);
             }
+            const float s0 = -mo;
             if (__any_sync(kFull, any)) {
                 float du, dv;
                 if (pb.w == 1.f) {
@@ -489,17 +492,52 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     cp_async_wait_all();
 }
 
+// Tiles ordered by decreasing list length (bucketed by floor(sqrt(length)),
+// 256 buckets; order inside a bucket unspecified), so that the longest tiles
+// start first and the kernel's tail holds short ones.  One CTA.
+__global__ void __launch_bounds__(1024) tile_order_kernel(const uint2* __restrict__ ranges, int tiles,
+                                                         uint32_t* __restrict__ order) {
+    __shared__ uint32_t count[256];
+    __shared__ uint32_t start[256];
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) count[b] = 0u;
+    __syncthreads();
+    auto bucket = [&](int t) {
+        const uint2 r = __ldg(ranges + t);
+        const float len = float(r.y - r.x);
+        return 255u - min(255u, uint32_t(sqrtf(len)));  // longest first
+    };
+    for (int t = threadIdx.x; t < tiles; t += blockDim.x) atomicAdd(&count[bucket(t)], 1u);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t run = 0;
+        for (int b = 0; b < 256; ++b) {
+            start[b] = run;
+            run += count[b];
+        }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < tiles; t += blockDim.x) order[atomicAdd(&start[bucket(t)], 1u)] = uint32_t(t);
+}
+
 }  // namespace
 
+cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s) {
+    if (tiles <= 0) return cudaSuccess;
+    tile_order_kernel<<<1, 1024, 0, s>>>(reinterpret_cast<const uint2*>(ranges), tiles, order);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
-                              const CamArgs& cam, const float bg[3], float* image, float* final_T,
-                              int32_t* n_contrib, cudaStream_t s) {
+                              const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
+                              float* final_T, int32_t* n_contrib, cudaStream_t s) {
     FwdArgs a;
     a.xy = reinterpret_cast<const float2*>(proj.xy);
     a.con = reinterpret_cast<const float4*>(proj.conic_opacity);
     a.rgb = reinterpret_cast<const float4*>(proj.rgb);
     a.vals = vals;
     a.ranges = reinterpret_cast<const uint2*>(ranges);
+    a.order = order;
     a.W = cam.W;
     a.H = cam.H;
     a.TX = cam.TX;
@@ -516,14 +554,16 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
 }
 
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
-                              const CamArgs& cam, const float bg[3], const float* final_T, const int32_t* n_contrib,
-                              const float* dL_dimage, const gs_grad2d& g2, cudaStream_t s) {
+                              const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,
+                              const int32_t* n_contrib, const float* dL_dimage, const gs_grad2d& g2,
+                              cudaStream_t s) {
     BwdArgs a;
     a.xy = reinterpret_cast<const float2*>(proj.xy);
     a.con = reinterpret_cast<const float4*>(proj.conic_opacity);
     a.rgb = reinterpret_cast<const float4*>(proj.rgb);
     a.vals = vals;
     a.ranges = reinterpret_cast<const uint2*>(ranges);
+    a.order = order;
     a.W = cam.W;
     a.H = cam.H;
     a.TX = cam.TX;

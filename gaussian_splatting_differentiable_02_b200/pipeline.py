@@ -165,6 +165,7 @@ class View:
         self.final_T = torch.zeros((H, W), device=device, dtype=torch.float32)
         self.n_contrib = torch.zeros((H, W), device=device, dtype=torch.int32)
         self.dL_dimage = torch.zeros((H, W, 3), device=device, dtype=torch.float32)
+        self.order = torch.zeros((T,), device=device, dtype=torch.int32)  # longest tiles first
         self.num_instances = 0
         self.capacity = 0
         self._alloc(max(capacity, 4 * n, 1024))
@@ -189,20 +190,30 @@ def bin_sort(proj: Projected, view: View, radius: torch.Tensor = None):
                                 _ptr(view.keys), _ptr(view.vals), view.capacity, _ptr(view.ranges), s, check=False)
         if st == abi.GS_OK:
             view.num_instances = K
+            abi.gs_tile_order(_ptr(view.ranges), view.gcam, _ptr(view.order), s)
             return K
         view._alloc(int(K * 1.25) + 1024)
 
 
+def bin_sort_async(proj: Projected, view: View, counter: torch.Tensor, radius: torch.Tensor = None):
+    """Sort without waiting; K lands in `counter` (one int64 on the device).  The
+    caller checks K against view.capacity later and repeats the view if it overflowed."""
+    abi.gs_bin_sort_async(proj.struct(radius), view.n, view.gcam, _ptr(view.workspace), view.workspace.numel(),
+                          _ptr(view.keys), _ptr(view.vals), view.capacity, _ptr(counter), _ptr(view.ranges),
+                          _stream())
+    abi.gs_tile_order(_ptr(view.ranges), view.gcam, _ptr(view.order), _stream())
+
+
 def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Tensor = None):
-    abi.gs_raster_fwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.image),
-                      _ptr(view.final_T), _ptr(view.n_contrib), _stream())
+    abi.gs_raster_fwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam, bg,
+                      _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _stream())
 
 
 def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), dL_dimage: torch.Tensor = None,
                radius: torch.Tensor = None):
     d = view.dL_dimage if dL_dimage is None else dL_dimage
-    abi.gs_raster_bwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), view.gcam, bg, _ptr(view.final_T),
-                      _ptr(view.n_contrib), _ptr(d), grad2d.struct(), _stream())
+    abi.gs_raster_bwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam, bg,
+                      _ptr(view.final_T), _ptr(view.n_contrib), _ptr(d), grad2d.struct(), _stream())
 
 
 def project_bwd(g: Gaussians, view: View, proj: Projected, grad2d: Grad2D, grads: Gaussians,
@@ -271,15 +282,20 @@ class Trainer:
         self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
         self.densify_accum = torch.zeros((n,), device=dev, dtype=torch.float32) if self.densify else None
         self.densify_count = torch.zeros((n,), device=dev, dtype=torch.int32) if self.densify else None
+        self.kcount = torch.zeros((len(self.views),), device=dev, dtype=torch.int64)
         self.step_count = 0
 
     def view_forward_backward(self, k: int, target: torch.Tensor) -> None:
-        """project -> sort -> raster forward -> L1 -> raster backward of view k."""
+        """project -> sort -> raster forward -> L1 -> raster backward of view k.
+        The fused path sorts without waiting (instance count checked once per step)."""
         view = self.views[k]
         r = self.radii[k if self.fused else 0]
         g2 = self.grad2ds[k if self.fused else 0]
         project(self.gauss, view, self.proj, r)
-        bin_sort(self.proj, view, r)
+        if self.fused:
+            bin_sort_async(self.proj, view, self.kcount[k:k + 1], r)
+        else:
+            bin_sort(self.proj, view, r)
         raster_fwd(self.proj, view, self.bg, r)
         l1_loss_grad(view, target, self.loss)
         g2.zero_()
@@ -288,14 +304,26 @@ class Trainer:
     def step(self) -> None:
         """forward + L1 + backward for every view, then one Adam step; loss stays on the device."""
         s = _stream()
-        abi.gs_zero(_ptr(self.loss), 8, s)
-        if not self.fused:
-            self.grads.zero_()
-        for k, tgt in enumerate(self.targets):
-            self.view_forward_backward(k, tgt)
+        while True:
+            abi.gs_zero(_ptr(self.loss), 8, s)
             if not self.fused:
-                project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
-                            self.densify_count, radius=self.radii[0])
+                self.grads.zero_()
+            for k, tgt in enumerate(self.targets):
+                self.view_forward_backward(k, tgt)
+                if not self.fused:
+                    project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
+                                self.densify_count, radius=self.radii[0])
+            if not self.fused:
+                break
+            # one wait per step: every view's instance count against its capacity
+            counts = self.kcount.cpu().tolist()
+            over = [k for k, K in enumerate(counts) if K > self.views[k].capacity]
+            for k, K in enumerate(counts):
+                self.views[k].num_instances = K
+            if not over:
+                break
+            for k in over:  # grow and repeat the step's views (nothing was applied yet)
+                self.views[k]._alloc(int(counts[k] * 1.25) + 1024)
         self.step_count += 1
         if self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,

@@ -165,10 +165,22 @@ size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera*
  *   keys [capacity] (8-byte aligned), vals [capacity] (4-byte aligned),
  *   tile_ranges [tiles][2] uint32 (8-byte aligned), workspace as sized above.
  * *num_instances_host receives K, the instance count.  K > capacity returns
- * GS_ERR_CAPACITY with nothing else written; call again with a larger buffer. */
+ * GS_ERR_CAPACITY with keys and vals untouched and every tile range empty; call
+ * again with a larger buffer.  The call waits for K (one 8-byte device-to-host
+ * copy); gs_bin_sort_async does not. */
 gs_status gs_bin_sort(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
                       size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
                       int64_t* num_instances_host, uint32_t* tile_ranges, void* stream);
+
+/* gs_bin_sort_async -- gs_bin_sort without waiting: the passes over instances
+ * are launched for `capacity` and read K on the device, and K is written to
+ * *num_instances_dev (one uint64 on the device, 8-byte aligned) instead of the
+ * host.  If K > capacity nothing is emitted or sorted and every tile range is
+ * empty, so the later raster calls see no instances; the caller reads K when it
+ * synchronises anyway and repeats the view with larger buffers. */
+gs_status gs_bin_sort_async(const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
+                            size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                            uint64_t* num_instances_dev, uint32_t* tile_ranges, void* stream);
 
 /* Size of the device array gs_bin_sort_static uses as its workspace (32 MiB). */
 #define GS_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -194,18 +206,26 @@ gs_status gs_bin_sort_static(const gs_projected* proj, int64_t n, const gs_camer
                              uint32_t* vals, int64_t capacity, int64_t* num_instances_host, uint32_t* tile_ranges,
                              void* stream);
 
-/* gs_raster_fwd -- stage 3 (gsplat guide §2.1), one CTA per 16x16 tile.  For each
+/* gs_tile_order -- the tiles ordered by decreasing length of their sorted lists
+ * (tile_ranges as written by gs_bin_sort; tile_order [tiles] uint32, 4-byte
+ * aligned).  Passed to the raster calls it starts the longest tiles first, so
+ * that the end of each launch is not held by a few long tiles; results do not
+ * depend on the order. */
+gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint32_t* tile_order, void* stream);
+
+/* gs_raster_fwd -- stage 3 (gsplat guide §2.1) over 16x16 tiles.  For each
  * pixel, front to back over its tile's sorted list: sigma as above with
  * d = (u, v) - pixel centre; entries with sigma < 0 are skipped;
  * alpha = min(0.99, o exp(-sigma)); entries with alpha < 1/255 are skipped; if
  * T (1 - alpha) < 1e-4 the pixel stops without blending that entry; otherwise
  * C += rgb alpha T and T *= 1 - alpha.
+ *   tile_order  optional processing order from gs_tile_order (NULL: tile order)
  *   image   [H][W][3] = C + T bg (bg_host: 3 floats read during the call)
  *   final_T [H][W]    transmittance after the last blended entry
  *   n_contrib [H][W]  1 + list position of the last blended entry (0 if none) */
 gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const gs_camera* cam, const float* bg_host, float* image, float* final_T,
-                        int32_t* n_contrib, void* stream);
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
+                        float* final_T, int32_t* n_contrib, void* stream);
 
 /* gs_raster_bwd -- the reverse of gs_raster_fwd for an upstream dL/dimage
  * [H][W][3]: per pixel, back to front from n_contrib, the transmittance in front
@@ -215,9 +235,10 @@ gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const ui
  *   dL/dalpha  = sum_c g_c (T (rgb_c - S_c) - final_T bg_c / (1 - alpha))
  * then through alpha = o exp(-sigma) (nothing when alpha was clamped at 0.99) to
  * o, to (u, v) and to (A, B, C).  Per-Gaussian sums are reduced across each warp
- * with shuffles before one vector atomic add per warp.  grad2d is accumulated. */
+ * with shuffles before one vector atomic add per warp.  grad2d is accumulated.
+ * tile_order as for gs_raster_fwd. */
 gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const gs_camera* cam, const float* bg_host, const float* final_T,
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* final_T,
                         const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream);
 
 /* gs_project_bwd -- chain grad2d through gs_project to the parameters (+= into

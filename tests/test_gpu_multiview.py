@@ -130,6 +130,34 @@ def test_fused_adam_matches_oracle_adam_of_summed_gradients(orc, deg):
         assert np.all(np.abs(gp - p1) <= bound), (k, float(np.max(np.abs(gp - p1) - bound)))
 
 
+def test_bin_sort_async_matches_sync_and_reports_overflow(orc):
+    wl = scenes.tiny()
+    cam = wl.cameras[0]
+    g = pl.Gaussians.from_scene(wl.scene)
+    view = pl.View(wl.scene.n, cam)
+    proj = pl.Projected(wl.scene.n)
+    pl.project(g, view, proj)
+    ref = orc.project(wl.scene, cam)
+    keys, vals, ranges = orc.keys(ref, cam)
+    K = len(keys)
+    counter = torch.zeros(1, dtype=torch.int64, device="cuda")
+    view._alloc(K + 100)
+    pl.bin_sort_async(proj, view, counter)
+    torch.cuda.synchronize()
+    assert int(counter.item()) == K
+    assert np.array_equal(view.keys[:K].cpu().numpy().view(np.uint64), keys)
+    assert np.array_equal(view.vals[:K].cpu().numpy().view(np.uint32), vals)
+    assert np.array_equal(view.ranges.cpu().numpy().view(np.uint32), ranges)
+    # too small: K still reported, nothing emitted, every range empty
+    view._alloc(64)
+    view.keys.fill_(-7)
+    pl.bin_sort_async(proj, view, counter)
+    torch.cuda.synchronize()
+    assert int(counter.item()) == K
+    assert torch.all(view.ranges == 0)
+    assert torch.all(view.keys == -7)
+
+
 def test_trainer_fused_equals_unfused():
     """The fused multi-view step and the per-view step + gs_adam update the same
     parameters (both CUDA paths; a consistency check next to the oracle parity)."""
