@@ -60,10 +60,10 @@ def measured_peaks():
 
 # --------------------------------------------------------------------- workloads
 
-def make_workload(name: str):
+def make_workload(name: str, views: int = 16):
     from gaussian_splatting_differentiable_02_b200 import scenes
     if name == "multiview":
-        return scenes.multiview1m(views=16)
+        return scenes.multiview1m(views=views)
     if name == "mixture":
         return scenes.mixture1m()
     if name == "box":
@@ -225,7 +225,7 @@ def cpu_oracle_sample(wl, fraction: float, seed: int = 0):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.views)
     fraction = args.cpu_fraction
     vals = []
     per_iter = threads = desc = None
@@ -259,7 +259,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     abi.lib()
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.views)
     scene = wl.scene
     nv = len(wl.cameras)
     gauss = pl.Gaussians.from_scene(scene)
@@ -334,7 +334,7 @@ def run_ours(args, world, rank, local):
     step_gbs = nbytes / (ms_per_step * 1e-3) / 1e9
 
     dom_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev_dom) if ev_dom else stages[dominant]
-    roof = roofline_for(dominant, dom_ms, stats, pairs / nv, scene, P, clk, peaks)
+    roof = roofline_for(dominant, dom_ms, stats, pairs / nv, scene, P, clk, peaks, profile_key(wl))
 
     line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -394,7 +394,57 @@ def stage_breakdown(tr, pl, torch):
     return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
 
 
-def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks):
+# Source files each stage's kernels are built from: a DRAM traffic figure taken
+# by ncu is reported only while these files are unchanged since the capture.
+STAGE_SOURCES = {
+    "raster_bwd": ["csrc/raster.cu", "csrc/internal.cuh", "../include/gs.h"],
+    "raster_fwd": ["csrc/raster.cu", "csrc/internal.cuh", "../include/gs.h"],
+    "project_bwd_adam": ["csrc/project_bwd.cu", "csrc/internal.cuh", "../include/gs.h"],
+}
+
+
+def profile_key(wl):
+    """File-name key of a workload's ncu summaries: the scene and the image size
+    (one launch of a stage does the same work whatever the number of views)."""
+    cam = wl.cameras[0]
+    scene = wl.name.split("-")[0] + wl.name.split("-")[1]
+    return f"{scene}_{cam['width']}x{cam['height']}"
+
+
+def stage_source_digest(stage):
+    import hashlib
+    pkg = os.path.join(ROOT, "gaussian_splatting_differentiable_02_b200")
+    h = hashlib.sha256()
+    for rel in STAGE_SOURCES[stage]:
+        with open(os.path.normpath(os.path.join(pkg, rel)), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(stage, workload):
+    """DRAM bytes per launch (read + write) of the stage's kernel from the ncu
+    summary under profiles/, or None when there is none for this workload or the
+    kernel's sources changed since it was taken."""
+    if stage not in STAGE_SOURCES:
+        return None
+    path = os.path.join(ROOT, "profiles", f"{stage}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- `"):
+                k, v = line[3:].split("`", 1)[0], line.split(":", 1)[1].strip().strip("`")
+                fields[k] = v
+    try:
+        if fields.get("source_sha256") != stage_source_digest(stage):
+            return None
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks, workload=""):
     """Roofline object of the dominant kernel: the raster kernels against the
     float32 ALU peak (148 SMs x 128 lanes x 2 x max SM clock), the streaming
     kernels against the measured HBM copy bandwidth."""
@@ -408,7 +458,7 @@ def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks):
         flops = pairs_per_view * per_pair
         achieved = flops / (ms * 1e-3) / 1e12
         return {"kernel": stage, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                "frac": achieved / alu_peak, "traffic": None,
+                "frac": achieved / alu_peak, "traffic": profiled_traffic(stage, workload),
                 "work": f"{pairs_per_view:.4g} (pixel, entry) pairs x {per_pair} flops per launch",
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"}
     n = scene.n
@@ -418,7 +468,8 @@ def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks):
                   "adam": n * pb // 4 * 28, "l1": P * 36}.get(stage, 0)
     achieved = per_launch / (ms * 1e-3) / 1e9
     return {"kernel": stage, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"]}
+            "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(stage, workload),
+            "peak_source": peaks["source"]}
 
 
 def run_e2e(tr, targets_host, targets, args, world, torch):
@@ -493,7 +544,12 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["multiview", "mixture", "box", "city", "tiny"], default="multiview")
     ap.add_argument("--cpu-fraction", type=float, default=1.0 / 256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--views", type=int, default=16,
+                    help="views per step of the multiview workload (fewer: the first poses of the 16; "
+                         "for small profiler captures, not a bench line)")
     args = ap.parse_args(argv)
+    if not 1 <= args.views <= 16:
+        ap.error("--views must be in 1..16")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()

@@ -207,7 +207,8 @@ def city3m(seed: int = 0, poses: int = 50, n: int = 3_000_000) -> Workload:
 
 def multiview1m(seed: int = 0, views: int = 16, n: int = 1_000_000) -> Workload:
     """The 1M mixture seen from a fixed batch of 16 poses on a radius-6 sphere at 1920x1080,
-    each view with its own L1 target ~ U[0,1]."""
+    each view with its own L1 target ~ U[0,1]. A smaller `views` keeps the first poses
+    of the 16 (the poses are drawn before the targets)."""
     rng = np.random.default_rng(seed)
     scene = _mixture_scene(rng, n)
     cams, targets = [], []
@@ -216,7 +217,7 @@ def multiview1m(seed: int = 0, views: int = 16, n: int = 1_000_000) -> Workload:
         cams.append(camera(R, t, 1600.0, 1600.0, 960.0, 540.0, 1920, 1080))
     for _ in range(views):
         targets.append(rng.uniform(0.0, 1.0, (1080, 1920, 3)).astype(np.float32))
-    return Workload("multiview-1m-16x1920x1080-train", scene, cams, targets=targets, adam_lr=dict(ADAM_LR))
+    return Workload(f"multiview-1m-{views}x1920x1080-train", scene, cams, targets=targets, adam_lr=dict(ADAM_LR))
 
 
 WORKLOADS = {1: tiny, 2: box100k, 3: mixture1m, 4: city3m, 5: multiview1m}

@@ -57,6 +57,11 @@ def lib():
         L.orc_l1.argtypes = [C.c_int64, _f32p, _f32p, _f32p]
         L.orc_l1.restype = C.c_double
         L.orc_sh_basis.argtypes = [C.c_int64, _f64p, C.c_int, _f64p]
+        L.orc_densify.argtypes = [C.c_int64, C.c_int, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _i32p, _i32p,
+                                  _f64p, C.c_double, C.c_double, C.c_double, C.c_int32, _u8p,
+                                  np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS"), _u8p, _f64p, _f64p, _f64p,
+                                  _f64p, _f64p]
+        L.orc_densify.restype = C.c_int64
         L.orc_set_threads.argtypes = [C.c_int]
         L.orc_set_threads.restype = C.c_int
         _lib = L
@@ -227,3 +232,46 @@ def sh_basis(dirs, deg: int):
     Y = np.zeros((len(d), nc))
     lib().orc_sh_basis(len(d), d.reshape(-1), deg, Y.reshape(-1))
     return Y
+
+
+def densify(scene, accum, count, max_radius, noise, grad_threshold, scale_threshold, min_opacity,
+            max_screen_radius, moments=(), quantize: bool = True) -> dict:
+    """Adaptive density control of oracle.cpp's orc_densify.
+
+    accum [n] float, count [n] int, max_radius [n] int, noise [n, 2, 3] (the N(0, I)
+    draws of the two split children).  Thresholds are taken as given (pass float32
+    values to decide in the same precision as a float32 configuration).  moments:
+    optimizer-state arrays laid out like the parameters, a dict per state with the
+    keys means, quats, log_scales, opacity_logits, sh; each is carried to the
+    outputs (kept Gaussians keep theirs, new ones start at zero).  Returns the
+    decision per input, source / fresh per output, the output scene arrays
+    (float32 values when quantize) and the carried moments."""
+    n = scene.n
+    nc = (scene.sh_degree + 1) ** 2
+    mu, q, ls, lo, sh = _scene_arrays(scene)
+    cap = 2 * n
+    out = {"means": np.zeros((cap, 3)), "quats": np.zeros((cap, 4)), "log_scales": np.zeros((cap, 3)),
+           "opacity_logits": np.zeros(cap), "sh": np.zeros((cap, nc, 3))}
+    decision = np.zeros(n, np.uint8)
+    source = np.zeros(cap, np.int64)
+    fresh = np.zeros(cap, np.uint8)
+    k = lib().orc_densify(n, nc, mu, q, ls, lo, sh, _c(accum, np.float64), _c(count, np.int32),
+                          _c(max_radius, np.int32), _c(noise, np.float64).reshape(-1), float(grad_threshold),
+                          float(scale_threshold), float(min_opacity), int(max_screen_radius), decision, source, fresh,
+                          out["means"].reshape(-1), out["quats"].reshape(-1), out["log_scales"].reshape(-1),
+                          out["opacity_logits"], out["sh"].reshape(-1))
+    res = {"decision": decision, "n_out": int(k), "source": source[:k], "fresh": fresh[:k].astype(bool)}
+    for key, a in out.items():
+        a = a[:k]
+        res[key] = a.astype(np.float32).astype(np.float64) if quantize else a
+    carried = []
+    for mom in moments:
+        c = {}
+        for key, a in mom.items():
+            a = np.asarray(a)
+            o = a[res["source"]].copy()
+            o[res["fresh"]] = 0
+            c[key] = o
+        carried.append(c)
+    res["moments"] = carried
+    return res

@@ -32,6 +32,10 @@
  *                      parameter), contracted with the 2D gradients.
  *   - orc_adam, orc_l1: Adam (gsplat guide §4.2: betas 0.9/0.99, eps 1e-15) and
  *                      the L1 photometric loss (gsplat guide §4.1) with its gradient.
+ *   - orc_densify:     adaptive density control (gsplat guide §4.1): prune,
+ *                      clone or split each Gaussian from its accumulated
+ *                      screen-space gradient statistic, opacity, scale and the
+ *                      largest screen radius it reached.
  *
  * Readings where the pages are silent (pixel centres at +0.5, near plane and
  * dilation as camera fields, 1.3x Jacobian clamp, radius = ceil(3 sqrt(lmax)),
@@ -689,6 +693,83 @@ double orc_l1(int64_t count, const float* img, const float* tgt, float* grad) {
         grad[i] = d > 0.0 ? inv : (d < 0.0 ? -inv : 0.0f);
     }
     return s / (double)count;
+}
+
+/* Adaptive density control (gsplat guide, lmnt.cn/news/262699, §4.1: every
+ * 100 steps densify_and_prune with a gradient threshold, a minimum opacity, a
+ * spatial extent and a maximum screen size; 3DGS deploy guide, hmyw.cn/news/140031,
+ * §3.2: --densify_grad_threshold 0.0002).  The pages give only the four
+ * parameters; the decision per Gaussian i, in this order:
+ *   prune  unless sigmoid(logit) >= min_opacity, or when max_screen_radius > 0
+ *          and the largest radius seen max_radius[i] > max_screen_radius;
+ *   densify when count[i] > 0 and accum[i] / count[i] >= grad_threshold:
+ *          clone (the Gaussian and an exact copy) if its largest scale
+ *          exp(log_scale) <= scale_threshold, else split it into two children
+ *          with means mu + R(q) (s * z_j) (z_j = noise[i][j], N(0, I) draws
+ *          passed in), log-scales log_scale - log(1.6), the same rotation,
+ *          opacity and SH;
+ *   keep   otherwise.
+ * Outputs keep input order: input i contributes 0 (prune), 1 (keep), or 2
+ * (clone: itself then the copy; split: child 0 then child 1) consecutive
+ * Gaussians.  source[k] is the input of output k and fresh[k] = 1 marks a new
+ * Gaussian (the copy, both children), whose optimizer state starts at zero.
+ * Decisions and values in double; returns the output count. */
+int64_t orc_densify(int64_t n, int nc, const double* means, const double* quats, const double* log_scales,
+                    const double* logits, const double* sh, const double* accum, const int32_t* count,
+                    const int32_t* max_radius, const double* noise, double grad_threshold, double scale_threshold,
+                    double min_opacity, int32_t max_screen_radius, uint8_t* decision, int64_t* source,
+                    uint8_t* fresh, double* out_means, double* out_quats, double* out_log_scales,
+                    double* out_logits, double* out_sh) {
+    const double log_split = std::log(1.6);
+    int64_t k = 0;
+    auto emit = [&](int64_t i, bool is_new) {
+        source[k] = i;
+        fresh[k] = is_new ? 1 : 0;
+        for (int c = 0; c < 3; ++c) out_means[3 * k + c] = means[3 * i + c];
+        for (int c = 0; c < 4; ++c) out_quats[4 * k + c] = quats[4 * i + c];
+        for (int c = 0; c < 3; ++c) out_log_scales[3 * k + c] = log_scales[3 * i + c];
+        out_logits[k] = logits[i];
+        for (int c = 0; c < 3 * nc; ++c) out_sh[3 * nc * k + c] = sh[3 * nc * i + c];
+        return k++;
+    };
+    for (int64_t i = 0; i < n; ++i) {
+        const double opacity = 1.0 / (1.0 + std::exp(-logits[i]));
+        const bool prune = !(opacity >= min_opacity) || (max_screen_radius > 0 && max_radius[i] > max_screen_radius);
+        const bool densify = count[i] > 0 && accum[i] / count[i] >= grad_threshold;
+        if (prune) {
+            decision[i] = 0;
+            continue;
+        }
+        if (!densify) {
+            decision[i] = 1;
+            emit(i, false);
+            continue;
+        }
+        const double ls_max = std::max(log_scales[3 * i], std::max(log_scales[3 * i + 1], log_scales[3 * i + 2]));
+        if (std::exp(ls_max) <= scale_threshold) {
+            decision[i] = 2;
+            emit(i, false);
+            emit(i, true);
+            continue;
+        }
+        decision[i] = 3;
+        // rotation of the normalised quaternion (w, x, y, z)
+        const double* q = quats + 4 * i;
+        const double qn = std::sqrt(q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3]);
+        const double w = q[0] / qn, x = q[1] / qn, y = q[2] / qn, z = q[3] / qn;
+        const double R[3][3] = {{1 - 2 * (y * y + z * z), 2 * (x * y - w * z), 2 * (x * z + w * y)},
+                                {2 * (x * y + w * z), 1 - 2 * (x * x + z * z), 2 * (y * z - w * x)},
+                                {2 * (x * z - w * y), 2 * (y * z + w * x), 1 - 2 * (x * x + y * y)}};
+        for (int j = 0; j < 2; ++j) {
+            const int64_t o = emit(i, true);
+            double sz[3];
+            for (int c = 0; c < 3; ++c) sz[c] = std::exp(log_scales[3 * i + c]) * noise[6 * i + 3 * j + c];
+            for (int r = 0; r < 3; ++r)
+                out_means[3 * o + r] = means[3 * i + r] + (R[r][0] * sz[0] + R[r][1] * sz[1] + R[r][2] * sz[2]);
+            for (int c = 0; c < 3; ++c) out_log_scales[3 * o + c] = log_scales[3 * i + c] - log_split;
+        }
+    }
+    return k;
 }
 
 /* Real SH basis values at unit directions dirs[3*k..] (degree <= 3), for pins. */
