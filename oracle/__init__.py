@@ -62,6 +62,8 @@ def lib():
                                   np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS"), _u8p, _f64p, _f64p, _f64p,
                                   _f64p, _f64p]
         L.orc_densify.restype = C.c_int64
+        L.orc_ssim.argtypes = [C.c_int, C.c_int, C.c_int, _f64p, _f64p, _vp, _vp]
+        L.orc_ssim.restype = C.c_double
         L.orc_set_threads.argtypes = [C.c_int]
         L.orc_set_threads.restype = C.c_int
         _lib = L
@@ -275,3 +277,29 @@ def densify(scene, accum, count, max_radius, noise, grad_threshold, scale_thresh
         carried.append(c)
     res["moments"] = carried
     return res
+
+
+def ssim(x, y, want_map: bool = False, want_grad: bool = False):
+    """Mean structural similarity of two [H, W, ch] images (11x11 Gaussian window,
+    sigma 1.5, zero outside the image); optionally the per-pixel map and the
+    gradient with respect to x.  Returns (ssim, map or None, grad or None)."""
+    xa = _c(x, np.float64)
+    ya = _c(y, np.float64)
+    H, W, ch = xa.shape
+    m = np.zeros_like(xa) if want_map else None
+    g = np.zeros_like(xa) if want_grad else None
+    v = lib().orc_ssim(H, W, ch, xa.reshape(-1), ya.reshape(-1), m.ctypes.data_as(_vp) if want_map else None,
+                       g.ctypes.data_as(_vp) if want_grad else None)
+    return v, m, g
+
+
+def l1_dssim(image, target, l1_weight: float = 1.0, ssim_weight: float = 0.2):
+    """loss = l1_weight * mean|image - target| + ssim_weight * (1 - ssim(image, target))
+    and its gradient with respect to image (gsplat guide §4.1)."""
+    img = _c(image, np.float64)
+    tgt = _c(target, np.float64)
+    n = img.size
+    l1v = float(np.abs(img - tgt).mean())
+    s, _, gs = ssim(img, tgt, want_grad=True)
+    g = l1_weight * np.sign(img - tgt) / n - ssim_weight * gs
+    return l1_weight * l1v + ssim_weight * (1.0 - s), g

@@ -32,6 +32,8 @@
  *                      parameter), contracted with the 2D gradients.
  *   - orc_adam, orc_l1: Adam (gsplat guide §4.2: betas 0.9/0.99, eps 1e-15) and
  *                      the L1 photometric loss (gsplat guide §4.1) with its gradient.
+ *   - orc_ssim:        the structural similarity of the L1 + D-SSIM loss
+ *                      (gsplat guide §4.1) and its gradient.
  *   - orc_densify:     adaptive density control (gsplat guide §4.1): prune,
  *                      clone or split each Gaussian from its accumulated
  *                      screen-space gradient statistic, opacity, scale and the
@@ -770,6 +772,81 @@ int64_t orc_densify(int64_t n, int nc, const double* means, const double* quats,
         }
     }
     return k;
+}
+
+/* Structural similarity of the L1 + D-SSIM photometric loss (gsplat guide,
+ * lmnt.cn/news/262699, §4.1: loss = l1_loss + 0.2 * (1 - ssim(render, gt))).
+ * The pages do not define ssim(); this is the standard structural similarity:
+ * per channel and pixel p, with w an 11x11 Gaussian window (standard deviation
+ * 1.5, normalised to sum 1) centred on p and the images taken as 0 outside
+ * their bounds,
+ *   mx = sum w x, my = sum w y, sxx = sum w x^2 - mx^2, syy = sum w y^2 - my^2,
+ *   sxy = sum w x y - mx my,
+ *   S(p) = (2 mx my + C1)(2 sxy + C2) / ((mx^2 + my^2 + C1)(sxx + syy + C2)),
+ * C1 = 0.01^2, C2 = 0.03^2 (dynamic range 1), and ssim = the mean of S over
+ * pixels and channels.  Images are [H][W][ch].  Returns ssim; `map` (nullable)
+ * receives S; `grad` (nullable) receives d ssim / d x, from
+ *   dS(p)/dmx = S (2 my / a - 2 my / b - 2 mx / c + 2 mx / d),
+ *   dS(p)/d(sum w x^2) = -S / d,  dS(p)/d(sum w x y) = 2 S / b
+ * (a, b, c, d the four factors above) and the window weights, summed over
+ * every p whose window covers the pixel.  Plain sums over the 2D window. */
+double orc_ssim(int H, int W, int ch, const double* x, const double* y, double* map, double* grad) {
+    const int R = 5;
+    double g[2 * R + 1], gs = 0.0;
+    for (int k = -R; k <= R; ++k) gs += g[k + R] = std::exp(-(double)(k * k) / (2.0 * 1.5 * 1.5));
+    for (int k = 0; k <= 2 * R; ++k) g[k] /= gs;
+    const double C1 = 0.01 * 0.01, C2 = 0.03 * 0.03;
+    const int64_t n = (int64_t)H * W * ch;
+    std::vector<double> dmx(grad ? n : 0), dxx(grad ? n : 0), dxy(grad ? n : 0);
+    double total = 0.0;
+#pragma omp parallel for reduction(+ : total) schedule(static)
+    for (int py = 0; py < H; ++py)
+        for (int px = 0; px < W; ++px)
+            for (int c = 0; c < ch; ++c) {
+                double mx = 0, my = 0, exx = 0, eyy = 0, exy = 0;
+                for (int dy = -R; dy <= R; ++dy)
+                    for (int dx = -R; dx <= R; ++dx) {
+                        const int qy = py + dy, qx = px + dx;
+                        if (qy < 0 || qy >= H || qx < 0 || qx >= W) continue;
+                        const double w = g[dy + R] * g[dx + R];
+                        const double xv = x[((int64_t)qy * W + qx) * ch + c], yv = y[((int64_t)qy * W + qx) * ch + c];
+                        mx += w * xv;
+                        my += w * yv;
+                        exx += w * xv * xv;
+                        eyy += w * yv * yv;
+                        exy += w * xv * yv;
+                    }
+                const double a = 2 * mx * my + C1, b = 2 * (exy - mx * my) + C2;
+                const double cc = mx * mx + my * my + C1, d = (exx - mx * mx) + (eyy - my * my) + C2;
+                const double S = a * b / (cc * d);
+                const int64_t i = ((int64_t)py * W + px) * ch + c;
+                if (map) map[i] = S;
+                total += S;
+                if (grad) {
+                    dmx[i] = S * (2 * my / a - 2 * my / b - 2 * mx / cc + 2 * mx / d);
+                    dxx[i] = -S / d;
+                    dxy[i] = 2 * S / b;
+                }
+            }
+    if (grad) {
+#pragma omp parallel for schedule(static)
+        for (int qy = 0; qy < H; ++qy)
+            for (int qx = 0; qx < W; ++qx)
+                for (int c = 0; c < ch; ++c) {
+                    const int64_t q = ((int64_t)qy * W + qx) * ch + c;
+                    double s = 0.0;
+                    for (int dy = -R; dy <= R; ++dy)
+                        for (int dx = -R; dx <= R; ++dx) {
+                            const int py = qy + dy, px = qx + dx;
+                            if (py < 0 || py >= H || px < 0 || px >= W) continue;
+                            const double w = g[dy + R] * g[dx + R];
+                            const int64_t p = ((int64_t)py * W + px) * ch + c;
+                            s += w * (dmx[p] + 2.0 * x[q] * dxx[p] + y[q] * dxy[p]);
+                        }
+                    grad[q] = s / (double)n;
+                }
+    }
+    return total / (double)n;
 }
 
 /* Real SH basis values at unit directions dirs[3*k..] (degree <= 3), for pins. */
