@@ -354,6 +354,10 @@ def run_ours(args, world, rank, local):
     # e2e: the same step with the per-step inputs (16 target images) copied from
     # pinned host memory and the loss read back, inside the timed region
     line["e2e"] = run_e2e(tr, targets_host, targets, args, world, torch)
+    # rows outside the per-step path, measured after the step timing
+    with_oracle = rank == 0 and not args.no_cpu_baseline and world == 1
+    line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
+                    "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
         line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
@@ -363,17 +367,133 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def measure_dssim(tr, wl, peaks, torch, with_oracle: bool, reps: int = 10):
+    """The L1 + D-SSIM loss and gradient (weights 1 and 0.2) of the first view's
+    rendered image against its target, timed with CUDA events over `reps` calls,
+    against the HBM roofline of its algorithmic bytes (image and target read
+    twice, the 72-byte-per-pixel derivative maps written and read, dL/dimage
+    written); the oracle timed on a 256 x 256 crop and scaled by pixel count."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    view, target = tr.views[0], tr.targets[0]
+    H, W = view.image.shape[0], view.image.shape[1]
+    loss = torch.zeros((1,), device=view.image.device, dtype=torch.float64)
+    s = torch.cuda.current_stream()
+    for _ in range(3):
+        pl.l1_dssim_loss_grad(view, target, loss)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        pl.l1_dssim_loss_grad(view, target, loss)
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = H * W * (24 + 72 + 72 + 24 + 12)
+    hbm = peaks["hbm_gbs"]
+    res = {"image": f"{W}x{H}", "ms": ms,
+           "roofline": {"kernel": "ssim_moments + ssim_grad", "bound": "hbm", "achieved": nbytes / ms / 1e6,
+                        "peak": hbm, "unit": "GB/s", "frac": nbytes / ms / 1e6 / hbm, "traffic": None,
+                        "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
+    if with_oracle:
+        import oracle
+        c = 256
+        x = view.image[:c, :c].double().cpu().numpy()
+        y = target[:c, :c].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.l1_dssim(x, y)
+        dt = time.perf_counter() - t0
+        res["cpu_oracle"] = {"ms": dt * 1e3 * (H * W) / (c * c), "cores": oracle.set_threads(0), "kind": "oracle",
+                             "sample": f"{c}x{c} crop, scaled by pixel count"}
+    return res
+
+
+def measure_densify(tr, wl, peaks, torch, with_oracle: bool, reps: int = 10):
+    """Adaptive density control on the trainer's Gaussians and statistics (the
+    gradient threshold at the median of the visible Gaussians' mean statistic, so
+    that about half of them densify): gs_densify_plan and gs_densify_apply timed
+    with CUDA events over `reps` launches each, against the HBM roofline of their
+    algorithmic bytes; the oracle timed on the same inputs."""
+    from gaussian_splatting_differentiable_02_b200 import abi
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    g, n = tr.gauss, tr.gauss.n
+    s = torch.cuda.current_stream()
+    acc, cnt = tr.densify_accum[:n], tr.densify_count[:n]
+    vis = cnt > 0
+    thr = float((acc[vis] / cnt[vis]).median().item()) if bool(vis.any()) else 0.0
+    cam = wl.cameras[0]
+    cfg = pl.densify_config(cam["width"], cam["height"], grad_threshold=thr)
+    gen = torch.Generator(device=g.means.device)
+    gen.manual_seed(1)
+    noise = torch.randn((n, 6), device=g.means.device, generator=gen)
+    ws_bytes = abi.gs_densify_workspace_bytes(n)
+    ws = torch.empty((ws_bytes,), device=g.means.device, dtype=torch.uint8)
+    dec = torch.empty((n,), device=g.means.device, dtype=torch.uint8)
+    num = torch.zeros((1,), device=g.means.device, dtype=torch.int64)
+    mr = tr.densify_max_radius[:n]
+
+    def plan():
+        abi.gs_densify_plan(g.params(), pl._ptr(acc), pl._ptr(cnt), pl._ptr(mr), cfg, pl._ptr(ws), ws_bytes,
+                            pl._ptr(dec), pl._ptr(num), s.cuda_stream)
+
+    plan()
+    n_out = int(num.item())
+    out, om, ov = (pl.Gaussians(n_out, g.sh_degree, g.means.device) for _ in range(3))
+
+    def apply():
+        abi.gs_densify_apply(g.params(), tr.m.params(), tr.v.params(), pl._ptr(noise), pl._ptr(dec), pl._ptr(ws),
+                             ws_bytes, n_out, out.grads(), om.grads(), ov.grads(), s.cuda_stream)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    plan_ms = timed(plan)
+    apply_ms = timed(apply)
+    d = torch.bincount(dec.long(), minlength=4).tolist()
+    pb = 4 * (11 + 3 * (g.sh_degree + 1) ** 2)
+    plan_bytes = n * (4 + 12 + 4 + 4 + 4 + 1)
+    apply_bytes = (n + (d[1] + d[2]) * 3 * pb + d[3] * (pb + 24) + n_out * 3 * pb)
+    hbm = peaks["hbm_gbs"]
+    res = {"gaussians_in": n, "gaussians_out": n_out, "decisions": {"prune": d[0], "keep": d[1], "clone": d[2],
+                                                                      "split": d[3]},
+           "grad_threshold": thr, "plan_ms": plan_ms, "apply_ms": apply_ms,
+           "roofline": {"kernel": "densify_apply", "bound": "hbm", "achieved": apply_bytes / apply_ms / 1e6,
+                        "peak": hbm, "unit": "GB/s", "frac": apply_bytes / apply_ms / 1e6 / hbm,
+                        "traffic": None, "algorithmic_bytes": apply_bytes, "peak_source": peaks["source"]},
+           "plan_roofline_frac": plan_bytes / plan_ms / 1e6 / hbm}
+    if with_oracle:
+        import oracle
+        from gaussian_splatting_differentiable_02_b200 import scenes
+        p = g.to_numpy()
+        sc = scenes.Scene(p["means"], p["quats"], p["log_scales"], p["opacity_logits"], p["sh"], g.sh_degree)
+        a_h, c_h, r_h = acc.cpu().numpy(), cnt.cpu().numpy(), mr.cpu().numpy()
+        z = noise.cpu().numpy().reshape(n, 2, 3)
+        t0 = time.perf_counter()
+        want = oracle.densify(sc, a_h, c_h, r_h, z, cfg.grad_threshold, cfg.scale_threshold, cfg.min_opacity,
+                              cfg.max_screen_radius)
+        res["cpu_oracle"] = {"ms": (time.perf_counter() - t0) * 1e3, "cores": 1, "kind": "oracle",
+                             "sample": "all Gaussians, parameters only (no moments)",
+                             "decisions_equal": bool(np.array_equal(want["decision"], dec.cpu().numpy()))}
+    return res
+
+
 def stage_breakdown(tr, pl, torch):
     """Milliseconds per step of each stage, from CUDA events around every call of
     one untimed step."""
     stream = torch.cuda.current_stream()
     acc = {}
 
-    def timed(name, fn, *a):
+    def timed(name, fn, *a, **kw):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        r = fn(*a)
+        r = fn(*a, **kw)
         e1.record(stream)
         acc.setdefault(name, []).append((e0, e1))
         return r
@@ -389,7 +509,8 @@ def stage_breakdown(tr, pl, torch):
         timed("raster_bwd", pl.raster_bwd, tr.proj, view, g2, tr.bg, None, r)
     tr.step_count += 1
     timed("project_bwd_adam", pl.project_bwd_views_adam, tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m,
-          tr.v, tr.lrs, tr.step_count, None, tr.densify_accum, tr.densify_count)
+          tr.v, tr.lrs, tr.step_count, None, tr.densify_accum, tr.densify_count,
+          densify_max_radius=tr.densify_max_radius)
     torch.cuda.synchronize()
     return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
 
@@ -513,7 +634,8 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
                     copy_events.append(e)
         tr.step_count += 1
         pl.project_bwd_views_adam(tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m, tr.v, tr.lrs,
-                                  tr.step_count, None, tr.densify_accum, tr.densify_count)
+                                  tr.step_count, None, tr.densify_accum, tr.densify_count,
+                                  densify_max_radius=tr.densify_max_radius)
         loss_host.copy_(tr.loss, non_blocking=True)
 
     done = []

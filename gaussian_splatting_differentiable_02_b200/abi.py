@@ -55,6 +55,17 @@ class gs_grad2d(C.Structure):
     _fields_ = [("xy", C.c_void_p), ("conic_opacity", C.c_void_p), ("rgb", C.c_void_p)]
 
 
+class gs_densify_config(C.Structure):
+    _fields_ = [("grad_threshold", C.c_float), ("scale_threshold", C.c_float), ("min_opacity", C.c_float),
+                ("max_screen_radius", C.c_int32)]
+
+
+GS_DENSIFY_PRUNE = 0
+GS_DENSIFY_KEEP = 1
+GS_DENSIFY_CLONE = 2
+GS_DENSIFY_SPLIT = 3
+
+
 # name -> (restype, argtypes), exactly the declarations of include/gs.h
 _P = C.c_void_p
 SIGNATURES = {
@@ -76,15 +87,24 @@ SIGNATURES = {
     "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, C.POINTER(gs_grad2d), _P]),
     "gs_project_bwd": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected),
-                                   C.POINTER(gs_grad2d), C.POINTER(gs_param_grads), _P, _P, _P]),
+                                   C.POINTER(gs_grad2d), C.POINTER(gs_param_grads), _P, _P, _P, _P]),
     "gs_project_bwd_views": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
                                          C.POINTER(gs_projected), C.POINTER(gs_grad2d), C.POINTER(gs_param_grads),
-                                         _P, _P, _P]),
+                                         _P, _P, _P, _P]),
     "gs_project_bwd_views_adam": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
                                               C.POINTER(gs_projected), C.POINTER(gs_grad2d),
                                               C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
                                               C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float, C.c_float,
-                                              C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P]),
+                                              C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P, _P]),
+    "gs_l1_dssim_workspace_bytes": (C.c_size_t, [C.c_int32, C.c_int32]),
+    "gs_l1_dssim_loss_grad": (C.c_int32, [_P, _P, C.c_int32, C.c_int32, C.c_float, C.c_float, _P, C.c_size_t, _P, _P,
+                                          _P]),
+    "gs_densify_workspace_bytes": (C.c_size_t, [C.c_int64]),
+    "gs_densify_plan": (C.c_int32, [C.POINTER(gs_params), _P, _P, _P, C.POINTER(gs_densify_config), _P, C.c_size_t,
+                                    _P, _P, _P]),
+    "gs_densify_apply": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_params), C.POINTER(gs_params), _P, _P, _P,
+                                     C.c_size_t, C.c_int64, C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
+                                     C.POINTER(gs_param_grads), _P]),
     "gs_adam": (C.c_int32, [_P, _P, _P, _P, C.c_int64, C.c_float, C.c_float, C.c_float, C.c_float, C.c_int32, _P]),
     "gs_l1_loss_grad": (C.c_int32, [_P, _P, C.c_int64, _P, _P, _P]),
     "gs_zero": (C.c_int32, [_P, C.c_size_t, _P]),
@@ -212,9 +232,10 @@ def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: i
 
 
 def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d: gs_grad2d, grads: gs_param_grads,
-                   densify_accum: int = 0, densify_count: int = 0, stream: int = 0):
+                   densify_accum: int = 0, densify_count: int = 0, densify_max_radius: int = 0, stream: int = 0):
     return _check(lib().gs_project_bwd(C.byref(params), C.byref(cam), C.byref(proj), C.byref(grad2d),
-                                       C.byref(grads), densify_accum or None, densify_count or None, stream))
+                                       C.byref(grads), densify_accum or None, densify_count or None,
+                                       densify_max_radius or None, stream))
 
 
 GS_MAX_VIEWS = 16
@@ -229,18 +250,18 @@ def _arr(ctype, items):
 
 
 def gs_project_bwd_views(params: gs_params, cams, projs, grad2ds, grads: gs_param_grads, densify_accum: int = 0,
-                         densify_count: int = 0, stream: int = 0):
+                         densify_count: int = 0, densify_max_radius: int = 0, stream: int = 0):
     """cams, projs, grad2ds: sequences of gs_camera / gs_projected / gs_grad2d (one per view)."""
     V = len(cams)
     return _check(lib().gs_project_bwd_views(C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs),
                                              _arr(gs_grad2d, grad2ds), C.byref(grads), densify_accum or None,
-                                             densify_count or None, stream))
+                                             densify_count or None, densify_max_radius or None, stream))
 
 
 def gs_project_bwd_views_adam(params: gs_params, cams, projs, grad2ds, params_inout: gs_param_grads,
                               adam_m: gs_param_grads, adam_v: gs_param_grads, lrs, beta1: float, beta2: float,
                               eps: float, step: int, grads: gs_param_grads = None, densify_accum: int = 0,
-                              densify_count: int = 0, stream: int = 0):
+                              densify_count: int = 0, densify_max_radius: int = 0, stream: int = 0):
     """Multi-view backward through the projection with the Adam step fused; lrs = 5 learning rates
     (means, quats, log_scales, opacity_logits, sh)."""
     V = len(cams)
@@ -248,7 +269,40 @@ def gs_project_bwd_views_adam(params: gs_params, cams, projs, grad2ds, params_in
     return _check(lib().gs_project_bwd_views_adam(
         C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _arr(gs_grad2d, grad2ds),
         C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps, step,
-        C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None, stream))
+        C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None,
+        densify_max_radius or None, stream))
+
+
+def gs_l1_dssim_workspace_bytes(width: int, height: int) -> int:
+    return lib().gs_l1_dssim_workspace_bytes(width, height)
+
+
+def gs_l1_dssim_loss_grad(image: int, target: int, width: int, height: int, l1_weight: float, ssim_weight: float,
+                          workspace: int, workspace_bytes: int, dL_dimage: int, loss_dev: int, stream: int = 0):
+    return _check(lib().gs_l1_dssim_loss_grad(image, target, width, height, l1_weight, ssim_weight, workspace,
+                                              workspace_bytes, dL_dimage, loss_dev, stream))
+
+
+def gs_densify_workspace_bytes(n: int) -> int:
+    return lib().gs_densify_workspace_bytes(n)
+
+
+def gs_densify_plan(params: gs_params, densify_accum: int, densify_count: int, densify_max_radius: int,
+                    cfg: gs_densify_config, workspace: int, workspace_bytes: int, decision: int, num_out_dev: int,
+                    stream: int = 0):
+    return _check(lib().gs_densify_plan(C.byref(params), densify_accum or None, densify_count or None,
+                                        densify_max_radius or None, C.byref(cfg), workspace, workspace_bytes,
+                                        decision or None, num_out_dev, stream))
+
+
+def gs_densify_apply(params: gs_params, adam_m, adam_v, split_noise: int, decision: int, workspace: int,
+                     workspace_bytes: int, n_out: int, out_params: gs_param_grads, out_m=None, out_v=None,
+                     stream: int = 0):
+    """adam_m / adam_v: gs_params of the moments or None; out_m / out_v: gs_param_grads or None."""
+    ref = lambda x: C.byref(x) if x is not None else None  # noqa: E731
+    return _check(lib().gs_densify_apply(C.byref(params), ref(adam_m), ref(adam_v), split_noise or None,
+                                         decision or None, workspace, workspace_bytes, n_out, C.byref(out_params),
+                                         ref(out_m), ref(out_v), stream))
 
 
 def gs_adam(param: int, grad: int, m: int, v: int, count: int, lr: float, beta1: float, beta2: float, eps: float,

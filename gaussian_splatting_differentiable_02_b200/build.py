@@ -22,7 +22,7 @@ LIB = os.path.join(HERE, "libgs.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
           "--expt-relaxed-constexpr"]
-PER_FILE = {"project_fwd.cu": ["-fmad=false"]}
+PER_FILE = {"project_fwd.cu": ["-fmad=false"], "densify.cu": ["-fmad=false"]}
 
 
 def sources():

@@ -310,8 +310,8 @@ gs_status check_grad_arrays(const char* fn, const gs_param_grads* g, const char*
 // Shared checks and launch of the (multi-view) backward through the projection.
 gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t num_views, const gs_camera* cams,
                              const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
-                             float* densify_accum, int32_t* densify_count, const gsk::AdamStep* adam,
-                             void* stream) {
+                             float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                             const gsk::AdamStep* adam, void* stream) {
     gs_status st;
     if ((st = check_params(fn, params)) != GS_OK) return st;
     if (num_views < 1 || num_views > GS_MAX_VIEWS)
@@ -337,6 +337,7 @@ gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t nu
             CHECK_PTR(densify_accum, 4);
             CHECK_PTR(densify_count, 4);
         }
+        if (densify_max_radius) CHECK_PTR(densify_max_radius, 4);
         if (adam) {
             if ((st = check_grad_arrays(fn, adam->params, "params_inout")) != GS_OK) return st;
             if ((st = check_grad_arrays(fn, adam->m, "adam_m")) != GS_OK) return st;
@@ -344,7 +345,8 @@ gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t nu
         }
     }
     return cuda_status(gsk::launch_project_bwd_views(*params, num_views, c, cams, projs, grad2d, grads, densify_accum,
-                                                     densify_count, adam, static_cast<cudaStream_t>(stream)),
+                                                     densify_count, densify_max_radius, adam,
+                                                     static_cast<cudaStream_t>(stream)),
                        fn);
 }
 
@@ -361,26 +363,29 @@ extern "C" {
 
 gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
                          const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
-                         int32_t* densify_count, void* stream) {
+                         int32_t* densify_count, int32_t* densify_max_radius, void* stream) {
     const char* fn = "gs_project_bwd";
     if (!grads) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
-    return project_bwd_common(fn, params, 1, cam, proj, grad2d, grads, densify_accum, densify_count, nullptr, stream);
+    return project_bwd_common(fn, params, 1, cam, proj, grad2d, grads, densify_accum, densify_count,
+                              densify_max_radius, nullptr, stream);
 }
 
 gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const gs_camera* cams,
                                const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
-                               float* densify_accum, int32_t* densify_count, void* stream) {
+                               float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                               void* stream) {
     const char* fn = "gs_project_bwd_views";
     if (!grads) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
     return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
-                              nullptr, stream);
+                              densify_max_radius, nullptr, stream);
 }
 
 gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
                                     const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
                                     gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
                                     float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
-                                    float* densify_accum, int32_t* densify_count, void* stream) {
+                                    float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                    void* stream) {
     const char* fn = "gs_project_bwd_views_adam";
     if (!lr_host) return fail(GS_ERR_INVALID_ARG, "%s: lr_host is NULL", fn);
     gsk::AdamStep a;
@@ -399,8 +404,116 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
     a.beta2 = beta2;
     a.eps = eps;
     a.step = step;
-    return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count, &a,
-                              stream);
+    return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
+                              densify_max_radius, &a, stream);
+}
+
+size_t gs_l1_dssim_workspace_bytes(int32_t width, int32_t height) {
+    if (width <= 0 || height <= 0) return 0;
+    return (size_t(width) * size_t(height) * 9 * sizeof(double) + 255) & ~size_t(255);
+}
+
+gs_status gs_l1_dssim_loss_grad(const float* image, const float* target, int32_t width, int32_t height,
+                                float l1_weight, float ssim_weight, void* workspace, size_t workspace_bytes,
+                                float* dL_dimage, double* loss_dev, void* stream) {
+    const char* fn = "gs_l1_dssim_loss_grad";
+    if (width <= 0 || height <= 0 || width > 16384 || height > 16384)
+        return fail(GS_ERR_UNSUPPORTED, "%s: image %d x %d (1..16384 supported)", fn, int(width), int(height));
+    if (!std::isfinite(l1_weight) || !std::isfinite(ssim_weight))
+        return fail(GS_ERR_INVALID_ARG, "%s: non-finite weight", fn);
+    CHECK_PTR(image, 4);
+    CHECK_PTR(target, 4);
+    CHECK_PTR(dL_dimage, 4);
+    CHECK_PTR(loss_dev, 8);
+    CHECK_PTR(workspace, 16);
+    if (workspace_bytes < gs_l1_dssim_workspace_bytes(width, height))
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes,
+                    gs_l1_dssim_workspace_bytes(width, height));
+    return cuda_status(gsk::launch_l1_dssim(image, target, width, height, l1_weight, ssim_weight,
+                                            static_cast<double*>(workspace), dL_dimage, loss_dev,
+                                            static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+size_t gs_densify_workspace_bytes(int64_t n) {
+    if (n < 0) n = 0;
+    return gsk::densify_workspace_layout(n, nullptr, nullptr);
+}
+
+gs_status gs_densify_plan(const gs_params* params, const float* densify_accum, const int32_t* densify_count,
+                          const int32_t* densify_max_radius, const gs_densify_config* cfg, void* workspace,
+                          size_t workspace_bytes, uint8_t* decision, uint64_t* num_out_dev, void* stream) {
+    const char* fn = "gs_densify_plan";
+    gs_status st;
+    if ((st = check_params(fn, params)) != GS_OK) return st;
+    if (!cfg) return fail(GS_ERR_INVALID_ARG, "%s: cfg is NULL", fn);
+    if (!std::isfinite(cfg->grad_threshold) || !std::isfinite(cfg->scale_threshold) ||
+        !std::isfinite(cfg->min_opacity))
+        return fail(GS_ERR_INVALID_ARG, "%s: non-finite threshold", fn);
+    CHECK_PTR(workspace, 16);
+    CHECK_PTR(num_out_dev, 8);
+    if (workspace_bytes < gs_densify_workspace_bytes(params->n))
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes,
+                    gs_densify_workspace_bytes(params->n));
+    if (params->n > 0) {
+        CHECK_PTR(densify_accum, 4);
+        CHECK_PTR(densify_count, 4);
+        CHECK_PTR(decision, 1);
+        if (densify_max_radius) CHECK_PTR(densify_max_radius, 4);
+    }
+    gsk::DensifyWorkspace ws;
+    gsk::densify_workspace_layout(params->n, workspace, &ws);
+    return cuda_status(gsk::launch_densify_plan(*params, densify_accum, densify_count, densify_max_radius, *cfg, ws,
+                                                decision, num_out_dev, static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+gs_status gs_densify_apply(const gs_params* params, const gs_params* adam_m, const gs_params* adam_v,
+                           const float* split_noise, const uint8_t* decision, const void* workspace,
+                           size_t workspace_bytes, int64_t n_out, gs_param_grads* out_params, gs_param_grads* out_m,
+                           gs_param_grads* out_v, void* stream) {
+    const char* fn = "gs_densify_apply";
+    gs_status st;
+    if ((st = check_params(fn, params)) != GS_OK) return st;
+    const bool moments = adam_m || adam_v || out_m || out_v;
+    if (moments && !(adam_m && adam_v && out_m && out_v))
+        return fail(GS_ERR_INVALID_ARG, "%s: adam_m, adam_v, out_m and out_v must all be set or all NULL", fn);
+    if (moments) {
+        for (const gs_params* g : {adam_m, adam_v}) {
+            if (g->n != params->n || g->sh_degree != params->sh_degree)
+                return fail(GS_ERR_INVALID_ARG, "%s: moments differ from params in n or SH degree", fn);
+            if ((st = check_params(fn, g)) != GS_OK) return st;
+        }
+    }
+    if (n_out < 0 || n_out > 2 * params->n) return fail(GS_ERR_INVALID_ARG, "%s: n_out = %lld", fn, (long long)n_out);
+    CHECK_PTR(workspace, 16);
+    if (workspace_bytes < gs_densify_workspace_bytes(params->n))
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes,
+                    gs_densify_workspace_bytes(params->n));
+    if (params->n > 0) {
+        CHECK_PTR(split_noise, 4);
+        CHECK_PTR(decision, 1);
+    }
+    if (n_out > 0) {
+        if ((st = check_grad_arrays(fn, out_params, "out_params")) != GS_OK) return st;
+        if (moments) {
+            if ((st = check_grad_arrays(fn, out_m, "out_m")) != GS_OK) return st;
+            if ((st = check_grad_arrays(fn, out_v, "out_v")) != GS_OK) return st;
+        }
+    }
+    gsk::DensifyWorkspace ws;
+    gsk::densify_workspace_layout(params->n, const_cast<void*>(workspace), &ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned long long planned = 0;
+    if (cudaMemcpyAsync(&planned, ws.total, sizeof(planned), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return cuda_status(cudaGetLastError(), fn);
+    if ((long long)planned != n_out)
+        return fail(GS_ERR_INVALID_ARG, "%s: n_out = %lld but the plan has %llu", fn, (long long)n_out, planned);
+    return cuda_status(gsk::launch_densify_apply(*params, adam_m, adam_v, split_noise, decision, ws, n_out,
+                                                 out_params ? *out_params : gs_param_grads{}, out_m, out_v,
+                                                 std::log(1.6), s),
+                       fn);
 }
 
 gs_status gs_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,

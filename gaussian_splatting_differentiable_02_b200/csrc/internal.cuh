@@ -59,8 +59,8 @@ struct AdamStep {
 // Gaussians; grads (+=) may be null when adam is given.
 cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* cams, const gs_camera* raw,
                                      const gs_projected* projs, const gs_grad2d* g2d, const gs_param_grads* grads,
-                                     float* densify_accum, int32_t* densify_count, const AdamStep* adam,
-                                     cudaStream_t s);
+                                     float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                     const AdamStep* adam, cudaStream_t s);
 
 struct SortWorkspace {
     unsigned long long* block_sums;  // [nb_emit]
@@ -95,6 +95,28 @@ cudaError_t launch_adam(float* param, const float* grad, float* m, float* v, int
 
 cudaError_t launch_l1(const float* image, const float* target, int64_t count, float* dL, double* loss,
                       cudaStream_t s);
+
+struct DensifyWorkspace {
+    unsigned long long* chunk_counts;  // [blocks]: output count per chunk, then its offset
+    unsigned long long* total;         // [1]
+    int blocks;
+    int64_t chunk;
+};
+size_t densify_workspace_layout(int64_t n, void* base, DensifyWorkspace* ws);
+
+cudaError_t launch_densify_plan(const gs_params& p, const float* accum, const int32_t* count,
+                                const int32_t* max_radius, const gs_densify_config& cfg,
+                                const DensifyWorkspace& ws, uint8_t* decision, uint64_t* num_out_dev,
+                                cudaStream_t s);
+
+cudaError_t launch_densify_apply(const gs_params& p, const gs_params* m, const gs_params* v, const float* noise,
+                                 const uint8_t* decision, const DensifyWorkspace& ws, int64_t n_out,
+                                 const gs_param_grads& op, const gs_param_grads* om, const gs_param_grads* ov,
+                                 double log_split, cudaStream_t s);
+
+// maps: [9][H][W] doubles of workspace
+cudaError_t launch_l1_dssim(const float* image, const float* target, int W, int H, float l1_weight,
+                            float ssim_weight, double* maps, float* dL, double* loss, cudaStream_t s);
 
 // host-side count of kernel launches (gs_kernel_launches)
 void count_launches(int k);

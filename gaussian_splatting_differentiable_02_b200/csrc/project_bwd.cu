@@ -61,6 +61,7 @@ struct Args {
     float4* d_sh;
     float* densify_accum;
     int32_t* densify_count;
+    int32_t* densify_max_radius;
     // Adam (kAdam): parameters updated in place, first and second moments
     float4* p_means;
     float4* p_quats;
@@ -165,9 +166,14 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
     const int t = threadIdx.x;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + t; i < a.n; i += int64_t(gridDim.x) * blockDim.x) {
         unsigned vis = 0u;
-        for (int v = 0; v < a.V; ++v)
-            if (__ldg(a.view[v].radius + i) > 0) vis |= 1u << v;
+        int rmax = 0;
+        for (int v = 0; v < a.V; ++v) {
+            const int r = __ldg(a.view[v].radius + i);
+            if (r > 0) vis |= 1u << v;
+            rmax = max(rmax, r);
+        }
         if (!kAdam && vis == 0u) continue;
+        if (a.densify_max_radius && rmax > a.densify_max_radius[i]) a.densify_max_radius[i] = rmax;
 
         double gS[6] = {0, 0, 0, 0, 0, 0};  // symmetric dL/dSigma: xx, xy, xz, yy, yz, zz
         double gmu[3] = {0, 0, 0};
@@ -479,8 +485,8 @@ void fill_grads(float4*& m, float4*& q, float4*& l, float*& o, float4*& s, const
 
 cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* cams, const gs_camera* raw,
                                      const gs_projected* projs, const gs_grad2d* g2d, const gs_param_grads* grads,
-                                     float* densify_accum, int32_t* densify_count, const AdamStep* adam,
-                                     cudaStream_t s) {
+                                     float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                     const AdamStep* adam, cudaStream_t s) {
     if (p.n == 0) return cudaSuccess;
     Args a;
     fill_params(a, p);
@@ -488,6 +494,7 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
     fill_grads(a.d_means, a.d_quats, a.d_log_scales, a.d_logits, a.d_sh, grads);
     a.densify_accum = densify_accum;
     a.densify_count = densify_count;
+    a.densify_max_radius = densify_max_radius;
     const unsigned grid = grid_for(p.n, kBwdBlock, 16);
     if (adam) {
         fill_grads(a.p_means, a.p_quats, a.p_log_scales, a.p_logits, a.p_sh, adam->params);

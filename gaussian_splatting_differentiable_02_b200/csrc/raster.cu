@@ -30,8 +30,11 @@
 // Conditioning: sigma = 1/2 (A dx^2 + C dy^2) + B dx dy cancels badly far along
 // the long axis of a needle-shaped Gaussian (the terms grow with the condition
 // number of the conic).  Entries whose conic has an eigenvalue ratio above 8
-// evaluate the quadratic form, and in the backward pass dsigma/du and
-// dsigma/dv, per pixel in double; the rest stay float32.
+// use the factored form sigma = 1/2 A t^2 + 1/2 D dy^2 with t = dx + (B/A) dy
+// and D = det / A: both terms are non-negative, and t is formed with B/A split
+// into two floats, so the float32 evaluation keeps a relative error of a few
+// ulps whatever the conditioning; dsigma/du = A t and dsigma/dv = B t + D dy.
+// The factors are derived once per entry in double.
 #include "internal.cuh"
 
 namespace gsk {
@@ -92,13 +95,20 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // Per-warp staging area: raw gathered features (double-buffered) and the
 // per-entry constants derived from them.
+// Evaluation of an entry (WarpStage::pb.w).
+constexpr float kPlain = 0.f;     // expanded quadratic form in float32
+constexpr float kDouble = 1.f;    // quadratic form in double (a conic that is not positive definite)
+constexpr float kSkip = 2.f;      // misses every pixel of the warp's box
+constexpr float kFactored = 3.f;  // factored form 1/2 A t^2 + 1/2 D dy^2 in float32
+
 struct WarpStage {
     float2 xy[2][kBatch];
     float4 con[2][kBatch];  // A, B, C, o
     float4 rgb[2][kBatch];
     uint32_t gid[2][kBatch];
     float4 pa[kBatch];  // u, v, log2(o), 1/o
-    float4 pb[kBatch];  // -log2e A/2, -log2e B, -log2e C/2, flag (0 float32, 1 double, 2 skip)
+    float4 pb[kBatch];  // plain: -log2e A/2, -log2e B, -log2e C/2; factored: B/A (high, low part), D; flag
+    float2 pc[kBatch];  // factored: -log2e A/2, -log2e D/2
 };
 
 // Lane l < count gathers list entry first + l (reverse: first + count - 1 - l).
@@ -119,17 +129,30 @@ __device__ __forceinline__ void gather(WarpStage& S, int buf, const uint32_t* __
 
 // Smallest sigma = 1/2 (A dx^2 + 2 B dx dy + C dy^2) with dx fixed and dy in
 // [dylo, dyhi] (a positive definite form is minimised at dy = -B dx / C).
-__device__ __forceinline__ float edge_min(float A, float B, float C, float dx, float dylo, float dyhi) {
-    const float dy = fminf(fmaxf(-B * dx / C, dylo), dyhi);
-    return 0.5f * (A * dx * dx + 2.f * B * dx * dy + C * dy * dy);
+template <class R>
+__device__ __forceinline__ R edge_min(R A, R B, R C, R dx, R dylo, R dyhi) {
+    const R dy = fmin(fmax(-B * dx / C, dylo), dyhi);
+    return R(0.5) * (A * dx * dx + R(2) * B * dx * dy + C * dy * dy);
 }
 
-// Lane l < count derives the constants of staged entry l.  pb.w: 0 = evaluate
-// in float32, 1 = ill-conditioned (evaluate in double), 2 = skip: the smallest
-// sigma over this warp's pixel box [bx0, bx0 + kBoxW - 1] x [by0, by0 + kBoxH - 1]
-// (pixel centres) puts alpha below 1/255 everywhere in it, with a margin far
-// above the rounding of either evaluation, so no pixel of the warp would blend
-// it.  Ill-conditioned entries are never skipped.
+// Smallest sigma over the box [bx0, bx1] x [by0, by1] of pixel centres: 0 with
+// the mean inside, else the smallest of the four edge minima.
+template <class R>
+__device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by0, R by1) {
+    if (u >= bx0 && u <= bx1 && v >= by0 && v <= by1) return R(0);
+    const R dxlo = u - bx1, dxhi = u - bx0, dylo = v - by1, dyhi = v - by0;
+    R m = fmin(edge_min(A, B, C, dxlo, dylo, dyhi), edge_min(A, B, C, dxhi, dylo, dyhi));
+    m = fmin(m, edge_min(C, B, A, dylo, dxlo, dxhi));
+    return fmin(m, edge_min(C, B, A, dyhi, dxlo, dxhi));
+}
+
+// Lane l < count derives the constants of staged entry l.  pb.w selects the
+// evaluation (kPlain, kFactored, kDouble) or kSkip: the smallest sigma over
+// this warp's pixel box [bx0, bx0 + kBoxW - 1] x [by0, by0 + kBoxH - 1] (pixel
+// centres) puts alpha below 1/255 everywhere in it, with a margin far above
+// the rounding of either evaluation, so no pixel of the warp would blend it.
+// The bound is computed in float32 for well-conditioned conics and in double
+// for the others.
 __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
     if (lane < count) {
         const float2 xy = S.xy[buf][lane];
@@ -138,36 +161,59 @@ __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane,
         const float det = __fsub_rn(__fmul_rn(c.x, c.z), __fmul_rn(c.y, c.y));
         const bool ill = !(det > 0.f) || (__fmul_rn(tr, tr) > __fmul_rn(kCondMaxTraceSqOverDet, det));
         const float lo = log2f(c.w);
-        float flag = ill ? 1.f : 0.f;
+        // alpha >= 1/255 needs sigma <= ln(255 o) = ln 255 + lo ln 2
+        const float cut = 5.541263545158426f + lo * 0.6931471805599453f;
+        const float bx1 = bx0 + float(kBoxW - 1), by1 = by0 + float(kBoxH - 1);
+        float4 pb;
+        float2 pc = make_float2(0.f, 0.f);
         if (!ill) {
-            const float bx1 = bx0 + float(kBoxW - 1), by1 = by0 + float(kBoxH - 1);
-            const bool inside = xy.x >= bx0 && xy.x <= bx1 && xy.y >= by0 && xy.y <= by1;
-            if (!inside) {
-                const float dxlo = xy.x - bx1, dxhi = xy.x - bx0, dylo = xy.y - by1, dyhi = xy.y - by0;
-                float smin = fminf(edge_min(c.x, c.y, c.z, dxlo, dylo, dyhi), edge_min(c.x, c.y, c.z, dxhi, dylo, dyhi));
-                smin = fminf(smin, edge_min(c.z, c.y, c.x, dylo, dxlo, dxhi));
-                smin = fminf(smin, edge_min(c.z, c.y, c.x, dyhi, dxlo, dxhi));
-                // alpha >= 1/255 needs sigma <= ln(255 o) = ln 255 + lo ln 2
-                const float cut = 5.541263545158426f + lo * 0.6931471805599453f;
-                if (smin * (1.f - 1e-4f) > cut + 1e-4f) flag = 2.f;
+            const float smin = box_min<float>(c.x, c.y, c.z, xy.x, xy.y, bx0, bx1, by0, by1);
+            const float flag = smin * (1.f - 1e-4f) > cut + 1e-4f ? kSkip : kPlain;
+            pb = make_float4(__fmul_rn(-0.5f * kLog2e, c.x), __fmul_rn(-kLog2e, c.y), __fmul_rn(-0.5f * kLog2e, c.z),
+                             flag);
+        } else {
+            const double A = c.x, B = c.y, C = c.z;
+            const double D = (A * C - B * B) / A;  // A C and B^2 are exact in double
+            if (A > 0.0 && D > 0.0) {
+                const double smin = box_min<double>(A, B, C, xy.x, xy.y, bx0, bx1, by0, by1);
+                const double r = B / A;
+                const float rh = __double2float_rn(r);
+                pb = make_float4(rh, __double2float_rn(r - double(rh)), float(D),
+                                 smin * (1.0 - 1e-4) > double(cut) + 1e-4 ? kSkip : kFactored);
+                pc = make_float2(__double2float_rn(-0.5 * kLog2eD * A), __double2float_rn(-0.5 * kLog2eD * D));
+            } else {
+                pb = make_float4(0.f, 0.f, 0.f, kDouble);
             }
         }
         S.pa[lane] = make_float4(xy.x, xy.y, lo, 1.f / c.w);
-        S.pb[lane] = make_float4(__fmul_rn(-0.5f * kLog2e, c.x), __fmul_rn(-kLog2e, c.y),
-                                 __fmul_rn(-0.5f * kLog2e, c.z), flag);
+        S.pb[lane] = pb;
+        S.pc[lane] = pc;
     }
 }
 
-// alpha of one entry at the lane's 8 pixels, and the offsets dx (shared) and
-// dy[i] of the mean from the pixel centres.  Bit i of `blend` is set when
-// pixel i passes sigma >= 0 and alpha >= 1/255; bit i of `clamp` when alpha
-// was clamped at 0.99.
-__device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float4& con, float px, int y0,
-                                           float (&alpha)[kPx], unsigned& blend, unsigned& clamp, float& dx,
-                                           float (&dy)[kPx]) {
+// alpha of one entry at the lane's pixels, and the offsets dx (shared) and
+// dy[i] of the mean from the pixel centres (t[i] = dx + (B/A) dy[i] for a
+// factored entry).  Bit i of `blend` is set when pixel i passes sigma >= 0 and
+// alpha >= 1/255; bit i of `clamp` when alpha was clamped at 0.99.
+__device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
+                                           float px, int y0, float (&alpha)[kPx], unsigned& blend, unsigned& clamp,
+                                           float& dx, float (&dy)[kPx], float (&t)[kPx]) {
     blend = 0u;
     clamp = 0u;
-    if (pb.w == 1.f) {
+    if (pb.w == kFactored) {
+        dx = __fsub_rn(pa.x, px);
+#pragma unroll
+        for (int i = 0; i < kPx; ++i) {
+            dy[i] = __fsub_rn(pa.y, __fadd_rn(float(y0 + i), 0.5f));
+            t[i] = __fmaf_rn(pb.y, dy[i], __fmaf_rn(pb.x, dy[i], dx));
+            const float s = __fmaf_rn(__fmul_rn(pc.x, t[i]), t[i], __fmul_rn(__fmul_rn(pc.y, dy[i]), dy[i]));
+            const float a = ex2_approx(__fadd_rn(s, pa.z));
+            const bool c = a > kAlphaMax;
+            alpha[i] = c ? kAlphaMax : a;
+            if (alpha[i] >= kAlphaMin) blend |= 1u << i;  // s <= 0 by construction
+            if (c) clamp |= 1u << i;
+        }
+    } else if (pb.w == kDouble) {
         const double dxd = __dsub_rn(double(pa.x), double(px));
         dx = __double2float_rn(dxd);
         const double A = con.x, B = con.y, C = con.z;
@@ -180,6 +226,7 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
                                          __dmul_rn(bdx, dyd));
             const float s = __double2float_rn(__dmul_rn(-sig, kLog2eD));
             dy[i] = __double2float_rn(dyd);
+            t[i] = 0.f;
             const float a = ex2_approx(__fadd_rn(s, pa.z));
             const bool c = a > kAlphaMax;
             alpha[i] = c ? kAlphaMax : a;
@@ -193,6 +240,7 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
 #pragma unroll
         for (int i = 0; i < kPx; ++i) {
             dy[i] = __fsub_rn(pa.y, __fadd_rn(float(y0 + i), 0.5f));
+            t[i] = 0.f;
             const float s = __fmaf_rn(dy[i], __fmaf_rn(pb.z, dy[i], c1), a0);
             const float a = ex2_approx(__fadd_rn(s, pa.z));
             const bool c = a > kAlphaMax;
@@ -265,12 +313,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 break;
             }
             const float4 pa = S.pa[j], pb = S.pb[j];
-            if (pb.w == 2.f) continue;  // misses every pixel of this warp
+            if (pb.w == kSkip) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
-            float al[kPx], dy[kPx], dx;
+            float al[kPx], dy[kPx], tt[kPx], dx;
             unsigned blend, clamp;
-            eval_alpha(pa, pb, con, px, y0, al, blend, clamp, dx, dy);
+            eval_alpha(pa, pb, S.pc[j], con, px, y0, al, blend, clamp, dx, dy, tt);
             blend &= ~done;
             const int pos = b * kBatch + j + 1;
             // branch-free so the 8 independent pixel chains interleave; a pixel
@@ -432,13 +480,13 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
         for (int j = 0; j < cnt; ++j) {
             const int pos = hi - 1 - j;  // 0-based list position of this entry
             const float4 pa = S.pa[j], pb = S.pb[j];
-            if (pb.w == 2.f) continue;  // misses every pixel of this warp
+            if (pb.w == kSkip) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
-            float al[kPx], dy[kPx], m[kPx], dx;
+            float al[kPx], dy[kPx], tt[kPx], m[kPx], dx;
             unsigned blend, clamp;
-            eval_alpha(pa, pb, con, px, y0, al, blend, clamp, dx, dy);
-            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s1 = 0.f, s2 = 0.f;
+            eval_alpha(pa, pb, S.pc[j], con, px, y0, al, blend, clamp, dx, dy, tt);
+            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s1 = 0.f, s2 = 0.f, st = 0.f;
             bool any = false;
             // branch-free: every pixel runs the same instructions, inactive ones
             // with zero weight and unchanged state
@@ -463,12 +511,17 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                 mo += m[i];
                 s1 = fmaf(-m[i], dy[i], s1);
                 s2 = fmaf(-m[i] * dy[i], dy[i], s2);
+                st = fmaf(-m[i], tt[i], st);  // factored entries only (tt = 0 otherwise)
             }
             const float s0 = -mo;
             if (__any_sync(kFull, any)) {
                 float du, dv;
-                if (pb.w == 1.f) {
-                    // ill-conditioned: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
+                if (pb.w == kFactored) {
+                    // dsigma/du = A t, dsigma/dv = B t + D dy
+                    du = con.x * st;
+                    dv = fmaf(con.y, st, pb.z * s1);
+                } else if (pb.w == kDouble) {
+                    // not positive definite: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
                     const double dxd = __dsub_rn(double(pa.x), double(px));
                     du = dv = 0.f;
 #pragma unroll

@@ -170,6 +170,11 @@ class View:
         self.capacity = 0
         self._alloc(max(capacity, 4 * n, 1024))
 
+    def set_n(self, n: int):
+        """Resize for a new Gaussian count (after densification): the sort workspace depends on n."""
+        self.n = int(n)
+        self._alloc(max(self.capacity, 4 * self.n, 1024))
+
     def _alloc(self, capacity: int):
         self.capacity = int(capacity)
         self.keys = torch.zeros((self.capacity,), device=self.device, dtype=torch.int64)
@@ -218,14 +223,27 @@ def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), 
 
 def project_bwd(g: Gaussians, view: View, proj: Projected, grad2d: Grad2D, grads: Gaussians,
                 densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
-                radius: torch.Tensor = None):
+                radius: torch.Tensor = None, densify_max_radius: torch.Tensor = None):
     abi.gs_project_bwd(g.params(), view.gcam, proj.struct(radius), grad2d.struct(), grads.grads(),
-                       _ptr(densify_accum), _ptr(densify_count), _stream())
+                       _ptr(densify_accum), _ptr(densify_count), _ptr(densify_max_radius), _stream())
 
 
 def l1_loss_grad(view: View, target: torch.Tensor, loss_dev: torch.Tensor):
     abi.gs_l1_loss_grad(_ptr(view.image), _ptr(target), view.image.numel(), _ptr(view.dL_dimage), _ptr(loss_dev),
                         _stream())
+
+
+def l1_dssim_loss_grad(view: View, target: torch.Tensor, loss_dev: torch.Tensor, l1_weight: float = 1.0,
+                       ssim_weight: float = 0.2):
+    """loss += l1_weight L1 + ssim_weight (1 - SSIM) of the view's image against target, and
+    dL/dimage into the view (gsplat guide §4.1); the view keeps the SSIM workspace."""
+    H, W = view.image.shape[0], view.image.shape[1]
+    nbytes = abi.gs_l1_dssim_workspace_bytes(W, H)
+    if getattr(view, "ssim_workspace", None) is None or view.ssim_workspace.numel() < nbytes:
+        view.ssim_workspace = torch.empty((nbytes,), device=view.image.device, dtype=torch.uint8)
+    abi.gs_l1_dssim_loss_grad(_ptr(view.image), _ptr(target), W, H, l1_weight, ssim_weight,
+                              _ptr(view.ssim_workspace), view.ssim_workspace.numel(), _ptr(view.dL_dimage),
+                              _ptr(loss_dev), _stream())
 
 
 def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: dict, step: int,
@@ -240,20 +258,58 @@ def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: d
 def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: torch.Tensor, grad2ds: list,
                            m: Gaussians, v: Gaussians, lrs: dict, step: int, grads: Gaussians = None,
                            densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
-                           betas=(0.9, 0.99), eps=1e-15):
+                           betas=(0.9, 0.99), eps=1e-15, densify_max_radius: torch.Tensor = None):
     """Backward through the projection for all views (each with its own radius row and 2D
     gradients) with the Adam step of all five groups fused in."""
     abi.gs_project_bwd_views_adam(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES],
         betas[0], betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum),
-        _ptr(densify_count), _stream())
+        _ptr(densify_count), _ptr(densify_max_radius), _stream())
+
+
+# densify_and_prune parameters of the gsplat guide §4.1 (every 100 steps): gradient
+# threshold, minimum opacity, extent (read as the largest scale, in world units,
+# up to which a densified Gaussian is cloned rather than split) and maximum screen
+# size (read as a fraction of the image's larger side).
+DENSIFY_DEFAULTS = {"grad_threshold": 0.0002, "min_opacity": 0.005, "extent": 0.01, "max_screen_size": 0.02}
+
+
+def densify_config(width: int, height: int, grad_threshold=0.0002, min_opacity=0.005, extent=0.01,
+                   max_screen_size=0.02) -> abi.gs_densify_config:
+    return abi.gs_densify_config(grad_threshold, extent, min_opacity,
+                                 int(max_screen_size * max(width, height)) if max_screen_size > 0 else 0)
+
+
+def densify(g: Gaussians, accum: torch.Tensor, count: torch.Tensor, max_radius: torch.Tensor, noise: torch.Tensor,
+            cfg: abi.gs_densify_config, m: Gaussians = None, v: Gaussians = None):
+    """Prune / clone / split (gs_densify_plan, one wait for the output count, gs_densify_apply).
+    noise: [n, 6] float32 N(0, 1) draws for the split children.  Returns the new Gaussians,
+    the carried moments (None without m, v) and the per-Gaussian decisions."""
+    s = _stream()
+    dev = g.means.device
+    ws_bytes = abi.gs_densify_workspace_bytes(g.n)
+    ws = torch.empty((ws_bytes,), device=dev, dtype=torch.uint8)
+    decision = torch.empty((max(g.n, 1),), device=dev, dtype=torch.uint8)
+    num_out = torch.zeros((1,), device=dev, dtype=torch.int64)
+    abi.gs_densify_plan(g.params(), _ptr(accum), _ptr(count), _ptr(max_radius), cfg, _ptr(ws), ws_bytes,
+                        _ptr(decision), _ptr(num_out), s)
+    n_out = int(num_out.item())
+    out = Gaussians(n_out, g.sh_degree, dev)
+    om = ov = None
+    if m is not None:
+        om = Gaussians(n_out, g.sh_degree, dev)
+        ov = Gaussians(n_out, g.sh_degree, dev)
+    abi.gs_densify_apply(g.params(), m.params() if m is not None else None, v.params() if v is not None else None,
+                         _ptr(noise), _ptr(decision), _ptr(ws), ws_bytes, n_out, out.grads(),
+                         om.grads() if om is not None else None, ov.grads() if ov is not None else None, s)
+    return out, om, ov, decision[:g.n]
 
 
 @dataclass
 class Trainer:
-    """One or several views of L1 training with Adam (the training loop of the gsplat guide §4.1-4.2),
-    optionally accumulating the densification statistic.
+    """One or several views of L1 (or L1 + D-SSIM) training with Adam (the training loop of the
+    gsplat guide §4.1-4.2), optionally accumulating the densification statistics.
 
     fused=True (default, up to GS_MAX_VIEWS views): every view keeps its own 2D
     gradients and visibility, and one pass chains all views back to the parameters
@@ -266,24 +322,56 @@ class Trainer:
     bg: tuple = (0.0, 0.0, 0.0)
     densify: bool = False
     fused: bool = True
+    ssim_weight: float = 0.0   # > 0: L1 + ssim_weight * (1 - SSIM) (the gsplat guide §4.1 uses 0.2)
 
     def __post_init__(self):
         n = self.gauss.n
         dev = self.gauss.means.device
         self.fused = self.fused and len(self.views) <= abi.GS_MAX_VIEWS
-        self.proj = Projected(n, dev)
+        self._alloc_per_gaussian(n)
+        self.m = self.gauss.zeros_like()
+        self.v = self.gauss.zeros_like()
+        self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
+        self.kcount = torch.zeros((len(self.views),), device=dev, dtype=torch.int64)
+        self.step_count = 0
+        self.noise_gen = torch.Generator(device=dev)
+        self.noise_gen.manual_seed(0)
+
+    def _alloc_per_gaussian(self, n: int):
+        """Buffers sized by the Gaussian count (the projection, 2D gradients, visibility rows,
+        gradients and densification statistics)."""
+        dev = self.gauss.means.device
         nv = len(self.views) if self.fused else 1
+        self.proj = Projected(n, dev)
         self.grad2ds = [Grad2D(n, dev) for _ in range(nv)]
         self.grad2d = self.grad2ds[0]
         self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
         self.grads = None if self.fused else self.gauss.zeros_like()
-        self.m = self.gauss.zeros_like()
-        self.v = self.gauss.zeros_like()
-        self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
-        self.densify_accum = torch.zeros((n,), device=dev, dtype=torch.float32) if self.densify else None
-        self.densify_count = torch.zeros((n,), device=dev, dtype=torch.int32) if self.densify else None
-        self.kcount = torch.zeros((len(self.views),), device=dev, dtype=torch.int64)
-        self.step_count = 0
+        self.densify_accum = torch.zeros((max(n, 1),), device=dev, dtype=torch.float32) if self.densify else None
+        self.densify_count = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
+        self.densify_max_radius = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
+
+    def densify_and_prune(self, **kw) -> torch.Tensor:
+        """Adaptive density control from the statistics accumulated since the last call
+        (thresholds as in DENSIFY_DEFAULTS, overridable by keyword; the screen limit is a
+        fraction of the first view's larger side).  Parameters and Adam moments are
+        compacted into new arrays, every per-Gaussian buffer is resized and the
+        statistics restart from zero.  Returns the per-Gaussian decisions."""
+        if not self.densify:
+            raise RuntimeError("Trainer(densify=True) accumulates the statistics densification needs")
+        p = dict(DENSIFY_DEFAULTS)
+        p.update(kw)
+        cam = self.views[0].cam
+        cfg = densify_config(cam["width"], cam["height"], **p)
+        noise = torch.randn((max(self.gauss.n, 1), 6), device=self.gauss.means.device, dtype=torch.float32,
+                            generator=self.noise_gen)
+        g, m, v, decision = densify(self.gauss, self.densify_accum, self.densify_count, self.densify_max_radius,
+                                    noise, cfg, self.m, self.v)
+        self.gauss, self.m, self.v = g, m, v
+        for view in self.views:
+            view.set_n(g.n)
+        self._alloc_per_gaussian(g.n)
+        return decision
 
     def view_forward_backward(self, k: int, target: torch.Tensor) -> None:
         """project -> sort -> raster forward -> L1 -> raster backward of view k.
@@ -297,7 +385,10 @@ class Trainer:
         else:
             bin_sort(self.proj, view, r)
         raster_fwd(self.proj, view, self.bg, r)
-        l1_loss_grad(view, target, self.loss)
+        if self.ssim_weight > 0.0:
+            l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
+        else:
+            l1_loss_grad(view, target, self.loss)
         g2.zero_()
         raster_bwd(self.proj, view, g2, self.bg, radius=r)
 
@@ -312,7 +403,7 @@ class Trainer:
                 self.view_forward_backward(k, tgt)
                 if not self.fused:
                     project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
-                                self.densify_count, radius=self.radii[0])
+                                self.densify_count, radius=self.radii[0], densify_max_radius=self.densify_max_radius)
             if not self.fused:
                 break
             # one wait per step: every view's instance count against its capacity
@@ -327,6 +418,7 @@ class Trainer:
         self.step_count += 1
         if self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
-                                   self.lrs, self.step_count, None, self.densify_accum, self.densify_count)
+                                   self.lrs, self.step_count, None, self.densify_accum, self.densify_count,
+                                   densify_max_radius=self.densify_max_radius)
         else:
             adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)

@@ -249,10 +249,12 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
  * logit.  Culled Gaussians get nothing.  When densify_accum and densify_count are
  * non-NULL, every visible Gaussian also gets densify_accum += |(dL/du, dL/dv)| and
  * densify_count += 1 (the screen-space mean-gradient statistic that adaptive
- * density control thresholds, gsplat guide §4.1).  [n] floats / int32. */
+ * density control thresholds, gsplat guide §4.1).  [n] floats / int32.  When
+ * densify_max_radius [n] int32 is non-NULL it becomes the largest of itself and
+ * the view's radius (the screen-size statistic that gs_densify_plan prunes on). */
 gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs_projected* proj,
                          const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
-                         int32_t* densify_count, void* stream);
+                         int32_t* densify_count, int32_t* densify_max_radius, void* stream);
 
 /* Most views one multi-view backward call takes. */
 #define GS_MAX_VIEWS 16
@@ -263,11 +265,12 @@ gs_status gs_project_bwd(const gs_params* params, const gs_camera* cam, const gs
  * visible in a view when its radius there is > 0).  Every Gaussian reads its
  * parameters once, adds every visible view's contribution in registers and
  * accumulates the sum over views into grads (+=); densify statistics as in
- * gs_project_bwd, summed over views.  Equal, up to rounding, to num_views calls
- * of gs_project_bwd. */
+ * gs_project_bwd, summed (the largest radius: maximised) over views.  Equal, up
+ * to rounding, to num_views calls of gs_project_bwd. */
 gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const gs_camera* cams,
                                const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
-                               float* densify_accum, int32_t* densify_count, void* stream);
+                               float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                               void* stream);
 
 /* gs_project_bwd_views_adam -- gs_project_bwd_views followed by the Adam step of
  * gs_adam for all five parameter groups in the same pass (gsplat guide §4.2:
@@ -281,7 +284,64 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
                                     const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
                                     gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
                                     float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
-                                    float* densify_accum, int32_t* densify_count, void* stream);
+                                    float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                    void* stream);
+
+/* Adaptive density control (gsplat guide §4.1: every 100 steps,
+ * densify_and_prune with a gradient threshold of 0.0002, a minimum opacity of
+ * 0.005, an extent of 0.01 and a maximum screen size of 0.02; 3DGS deploy guide
+ * §3.2: --densify_grad_threshold 0.0002).  Per Gaussian, in this order:
+ *   prune   unless sigmoid(logit) >= min_opacity, or when max_screen_radius > 0
+ *           and the largest radius it reached (densify_max_radius of the
+ *           backward calls) exceeds max_screen_radius pixels;
+ *   densify when densify_count > 0 and densify_accum / densify_count >=
+ *           grad_threshold: clone (the Gaussian and an exact copy) when its
+ *           largest scale exp(log_scale) <= scale_threshold, else split it into
+ *           two children with means mu + R(q) (exp(log_scale) * z_j), z_j the
+ *           caller's N(0, I) draws, log-scales reduced by log(1.6), the same
+ *           rotation, opacity and SH;
+ *   keep    otherwise.
+ * Decisions are taken in double precision from the float32 values. */
+typedef struct gs_densify_config {
+    float grad_threshold;       /* units of densify_accum (pixels) */
+    float scale_threshold;      /* world units */
+    float min_opacity;
+    int32_t max_screen_radius;  /* pixels; <= 0 disables the screen test */
+} gs_densify_config;
+
+#define GS_DENSIFY_PRUNE 0
+#define GS_DENSIFY_KEEP 1
+#define GS_DENSIFY_CLONE 2
+#define GS_DENSIFY_SPLIT 3
+
+/* Bytes of device workspace the densify calls need for n Gaussians (a few KB). */
+size_t gs_densify_workspace_bytes(int64_t n);
+
+/* gs_densify_plan -- the decisions and the output count.
+ *   densify_accum [n] float, densify_count [n] int32 (as accumulated by the
+ *   backward calls), densify_max_radius [n] int32 or NULL (then no screen test),
+ *   decision [n] uint8 receives GS_DENSIFY_*, *num_out_dev (one uint64 on the
+ *   device, 8-byte aligned) the number of output Gaussians: 1 per kept, 2 per
+ *   cloned or split Gaussian.  workspace (16-byte aligned, caller-owned) carries
+ *   the plan to gs_densify_apply and must not be touched in between.  Asynchronous. */
+gs_status gs_densify_plan(const gs_params* params, const float* densify_accum, const int32_t* densify_count,
+                          const int32_t* densify_max_radius, const gs_densify_config* cfg, void* workspace,
+                          size_t workspace_bytes, uint8_t* decision, uint64_t* num_out_dev, void* stream);
+
+/* gs_densify_apply -- write the planned Gaussians into new arrays, in input
+ * order: a kept Gaussian once, a cloned one itself then its copy, a split one
+ * child 0 then child 1.  out_params holds n_out Gaussians in the layout of
+ * gs_params (SH planes of n_out rows).  adam_m / adam_v (the moments, laid out as
+ * params) and out_m / out_v are all set or all NULL: surviving Gaussians keep
+ * their moments, new ones (copies, children) start at zero.  split_noise [n][6]
+ * float holds z_0 then z_1 for every Gaussian (read only for split ones).
+ * n_out must equal the planned count (the call reads it from the workspace,
+ * one 8-byte copy and wait, and returns GS_ERR_INVALID_ARG otherwise).  The
+ * output arrays must not overlap the inputs. */
+gs_status gs_densify_apply(const gs_params* params, const gs_params* adam_m, const gs_params* adam_v,
+                           const float* split_noise, const uint8_t* decision, const void* workspace,
+                           size_t workspace_bytes, int64_t n_out, gs_param_grads* out_params, gs_param_grads* out_m,
+                           gs_param_grads* out_v, void* stream);
 
 /* gs_adam -- one bias-corrected Adam step on `count` floats (gsplat guide §4.2:
  * one call per parameter group with its own lr; betas 0.9, 0.99; eps 1e-15):
@@ -297,6 +357,26 @@ gs_status gs_adam(float* param, const float* grad, float* m, float* v, int64_t c
  * image, target, dL_dimage 16-byte aligned; loss_dev 8-byte aligned. */
 gs_status gs_l1_loss_grad(const float* image, const float* target, int64_t count, float* dL_dimage,
                           double* loss_dev, void* stream);
+
+/* Bytes of device workspace gs_l1_dssim_loss_grad needs for a width x height
+ * image (72 bytes per pixel). */
+size_t gs_l1_dssim_workspace_bytes(int32_t width, int32_t height);
+
+/* gs_l1_dssim_loss_grad -- the L1 + D-SSIM photometric loss of the gsplat guide
+ * §4.1, loss = l1_weight mean|image - target| + ssim_weight (1 - ssim(image,
+ * target)) (the guide trains with weights 1 and 0.2), added to *loss_dev (one
+ * double on the device), and its gradient with respect to the image written to
+ * dL_dimage.  The pages do not define ssim: it is the standard structural
+ * similarity, per channel and pixel with an 11x11 Gaussian window of standard
+ * deviation 1.5 (normalised), C1 = 0.01^2, C2 = 0.03^2, the images zero outside
+ * their bounds, averaged over all pixels and channels; the L1 term's gradient
+ * is sign(image - target) / count with sign(0) = 0.  Double precision inside.
+ *   image, target, dL_dimage [height][width][3] float (4-byte aligned);
+ *   workspace (16-byte aligned, caller-owned) as sized above; loss_dev 8-byte
+ *   aligned.  Asynchronous. */
+gs_status gs_l1_dssim_loss_grad(const float* image, const float* target, int32_t width, int32_t height,
+                                float l1_weight, float ssim_weight, void* workspace, size_t workspace_bytes,
+                                float* dL_dimage, double* loss_dev, void* stream);
 
 /* Number of CUDA kernels this library has launched in the calling process
  * (a diagnostic counter, incremented on the host at every launch). */

@@ -113,8 +113,23 @@ def test_invalid_arguments_rejected_before_launch(gs):
     g2 = gs.gs_grad2d(16, 16, 16)
     gr = gs.gs_param_grads(16, 16, 16, 16, 16)
     p = gs.gs_params(16, 16, 16, 16, 16, 0, 10)
-    assert L.gs_project_bwd(C.byref(p), C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr), 256, None, None) == \
+    assert L.gs_project_bwd(C.byref(p), C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr), 256, None, None,
+                            None) == gs.GS_ERR_INVALID_ARG
+    # densify: no config, non-finite threshold, small workspace, moments not all given, n_out out of range
+    cfg = gs.gs_densify_config(2e-4, 0.01, 0.005, 38)
+    ws = gs.gs_densify_workspace_bytes(10)
+    assert L.gs_densify_plan(C.byref(p), 256, 256, None, None, 256, ws, 256, 256, None) == gs.GS_ERR_INVALID_ARG
+    bad = gs.gs_densify_config(float("nan"), 0.01, 0.005, 38)
+    assert L.gs_densify_plan(C.byref(p), 256, 256, None, C.byref(bad), 256, ws, 256, 256, None) == \
         gs.GS_ERR_INVALID_ARG
+    assert L.gs_densify_plan(C.byref(p), 256, 256, None, C.byref(cfg), 256, 8, 256, 256, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "workspace" in gs.gs_last_error_detail()
+    assert L.gs_densify_apply(C.byref(p), C.byref(p), None, 256, 256, 256, ws, 12, C.byref(gr), None, None,
+                              None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_densify_apply(C.byref(p), None, None, 256, 256, 256, ws, 21, C.byref(gr), None, None, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "n_out" in gs.gs_last_error_detail()
     # zero-size work needs no pointers and launches nothing
     assert L.gs_adam(None, None, None, None, 0, 1e-3, 0.9, 0.99, 1e-15, 1, None) == gs.GS_OK
     assert L.gs_l1_loss_grad(None, None, 0, None, None, None) == gs.GS_OK
