@@ -1,13 +1,15 @@
 """Build libgs.so (the CUDA library behind include/gs.h) for sm_100a, in-tree.
 
-Each .cu compiles to its own object with nvcc; project_fwd.cu is built with
--fmad=false so that the projection rounds every product and sum as written.
+Each .cu compiles to its own object with nvcc; project_fwd.cu, densify.cu and
+ssim.cu are built with -fmad=false so that they round every product and sum as
+written.
 The objects link with the static CUDA runtime into one shared library beside
 this file.
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
+import hashlib
 import os
 import subprocess
 import sys
@@ -22,7 +24,7 @@ LIB = os.path.join(HERE, "libgs.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
           "--expt-relaxed-constexpr"]
-PER_FILE = {"project_fwd.cu": ["-fmad=false"], "densify.cu": ["-fmad=false"]}
+PER_FILE = {"project_fwd.cu": ["-fmad=false"], "densify.cu": ["-fmad=false"], "ssim.cu": ["-fmad=false"]}
 
 
 def sources():
@@ -52,10 +54,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     objs = []
     for f in sources():
         src = os.path.join(CSRC, f)
-        obj = os.path.join(OBJ, f[:-3] + ".o")
+        flags = [*ARCH, *COMMON, *PER_FILE.get(f, [])]
+        # the object's name carries its flags, so a change of flags rebuilds it
+        tag = hashlib.sha1(" ".join(flags).encode()).hexdigest()[:10]
+        obj = os.path.join(OBJ, f"{f[:-3]}.{tag}.o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [nvcc, *ARCH, *COMMON, *PER_FILE.get(f, []), "-c", src, "-o", obj]
+            cmd = [nvcc, *flags, "-c", src, "-o", obj]
             if ptxas_info:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)

@@ -38,6 +38,7 @@ namespace {
 constexpr int kEmitBlock = 256;
 constexpr int kEmitPerThread = 8;
 constexpr int kEmitChunk = kEmitBlock * kEmitPerThread;  // Gaussians per emit block
+static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halves a power of two");
 
 #ifndef GS_SORT_ITEMS
 #define GS_SORT_ITEMS 8
@@ -256,12 +257,20 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* b
     }
 }
 
+// Instances of the block's Gaussians (depth order), load-balanced: the block's
+// output slots [0, total) are dealt to its threads round-robin, and each slot
+// finds its Gaussian by a binary search over the block's exclusive offsets in
+// shared memory, then its tile from its index inside the Gaussian's tile
+// rectangle (row-major).  Consecutive slots are written by consecutive threads.
 __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
                                                           const uint2* __restrict__ rect,
                                                           const uint32_t* __restrict__ order, int64_t n, int tiles_x,
                                                           const unsigned long long* __restrict__ block_offsets,
                                                           const Count cnt, uint32_t* __restrict__ tkeys,
                                                           uint32_t* __restrict__ tvals) {
+    __shared__ uint32_t s_start[kEmitChunk];
+    __shared__ uint32_t s_gid[kEmitChunk];
+    __shared__ uint2 s_rect[kEmitChunk];
     if (cnt.get() == 0) return;  // nothing fits: emit nothing
     const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
     uint32_t gid[kEmitPerThread], tt[kEmitPerThread];
@@ -272,19 +281,30 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __rest
         tt[k] = first + k < n ? __ldg(touched + gid[k]) : 0u;
         mine += tt[k];
     }
-    unsigned long long tot;
-    unsigned long long off = block_excl_scan(mine, &tot) + block_offsets[blockIdx.x];
+    unsigned long long total;
+    uint32_t run = uint32_t(block_excl_scan(mine, &total));
+    const unsigned long long base = block_offsets[blockIdx.x];
 #pragma unroll
     for (int k = 0; k < kEmitPerThread; ++k) {
-        if (tt[k] == 0u) continue;
-        const uint2 r = __ldg(rect + gid[k]);
-        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, x1 = r.y & 0xffffu, y1 = r.y >> 16;
-        for (uint32_t ty = y0; ty < y1; ++ty)
-            for (uint32_t tx = x0; tx < x1; ++tx) {
-                tkeys[off] = ty * uint32_t(tiles_x) + tx;
-                tvals[off] = gid[k];
-                ++off;
-            }
+        const int idx = threadIdx.x * kEmitPerThread + k;
+        s_start[idx] = run;
+        s_gid[idx] = gid[k];
+        s_rect[idx] = tt[k] ? __ldg(rect + gid[k]) : make_uint2(0u, 0u);
+        run += tt[k];
+    }
+    __syncthreads();
+    for (uint32_t slot = threadIdx.x; slot < uint32_t(total); slot += kEmitBlock) {
+        // the last Gaussian whose first slot is <= slot (it has at least one instance)
+        int lo = 0;
+#pragma unroll
+        for (int step = kEmitChunk / 2; step > 0; step >>= 1)
+            if (s_start[lo + step] <= slot) lo += step;
+        const uint32_t j = slot - s_start[lo];
+        const uint2 r = s_rect[lo];
+        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, w = (r.y & 0xffffu) - x0;
+        const uint32_t ty = y0 + j / w, tx = x0 + j % w;
+        tkeys[base + slot] = ty * uint32_t(tiles_x) + tx;
+        tvals[base + slot] = s_gid[lo];
     }
 }
 

@@ -21,7 +21,7 @@
 namespace gsk {
 namespace {
 
-constexpr int kBlock = 256;
+constexpr int kBlock = 128;
 constexpr int kMaxChunks = kNumSMs * 8;
 
 struct Chunking {
@@ -175,13 +175,32 @@ struct ApplyArgs {
     int64_t n, n_out, chunk;
 };
 
-__device__ __forceinline__ void copy_group(const Group& g, const OutGroup& o, int64_t i, int64_t k, int planes,
-                                           int64_t n, int64_t n_out) {
-    o.means[k] = __ldg(g.means + i);
-    o.quats[k] = __ldg(g.quats + i);
-    o.log_scales[k] = __ldg(g.log_scales + i);
-    o.logits[k] = __ldg(g.logits + i);
-    for (int p = 0; p < planes; ++p) o.sh[int64_t(p) * n_out + k] = __ldg(g.sh + int64_t(p) * n + i);
+// One Gaussian's record of a parameter-shaped group, held in registers so that
+// every load is issued before the first store.
+struct Record {
+    float4 means, quats, log_scales, sh[12];
+    float logit;
+};
+
+__device__ __forceinline__ void load_record(const Group& g, int64_t i, int planes, int64_t n, Record& r) {
+    r.means = __ldg(g.means + i);
+    r.quats = __ldg(g.quats + i);
+    r.log_scales = __ldg(g.log_scales + i);
+    r.logit = __ldg(g.logits + i);
+#pragma unroll
+    for (int p = 0; p < 12; ++p)
+        if (p < planes) r.sh[p] = __ldg(g.sh + int64_t(p) * n + i);
+}
+
+__device__ __forceinline__ void store_record(const OutGroup& o, int64_t k, int planes, int64_t n_out,
+                                             const Record& r) {
+    o.means[k] = r.means;
+    o.quats[k] = r.quats;
+    o.log_scales[k] = r.log_scales;
+    o.logits[k] = r.logit;
+#pragma unroll
+    for (int p = 0; p < 12; ++p)
+        if (p < planes) o.sh[int64_t(p) * n_out + k] = r.sh[p];
 }
 
 __device__ __forceinline__ void zero_group(const OutGroup& o, int64_t k, int planes, int64_t n_out) {
@@ -190,32 +209,35 @@ __device__ __forceinline__ void zero_group(const OutGroup& o, int64_t k, int pla
     o.quats[k] = z;
     o.log_scales[k] = z;
     o.logits[k] = 0.f;
-    for (int p = 0; p < planes; ++p) o.sh[int64_t(p) * n_out + k] = z;
+#pragma unroll
+    for (int p = 0; p < 12; ++p)
+        if (p < planes) o.sh[int64_t(p) * n_out + k] = z;
 }
 
-// Child j of a split: mean + R(q) (exp(log_scale) * z_j), log_scale - log(1.6),
-// rotation, opacity and SH copied.  Double precision, rounded once.
-__device__ __forceinline__ void write_child(const ApplyArgs& a, int64_t i, int64_t k, int j) {
-    const float4 mu = __ldg(a.p.means + i);
-    const float4 q4 = __ldg(a.p.quats + i);
-    const float4 ls = __ldg(a.p.log_scales + i);
+// Child j of a split from the parent's record: mean + R(q) (exp(log_scale) * z_j)
+// and log_scale - log(1.6) (double precision, rounded once); the rotation,
+// opacity and SH are the parent's.
+__device__ __forceinline__ void store_child(const OutGroup& o, int64_t k, int planes, int64_t n_out,
+                                            const Record& p, const float* z, double log_split) {
+    const float4 mu = p.means, q4 = p.quats, ls = p.log_scales;
     const double qw = q4.x, qx = q4.y, qy = q4.z, qz = q4.w;
     const double qn = sqrt(((qw * qw + qx * qx) + qy * qy) + qz * qz);
-    const double w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
-    const double R00 = 1.0 - 2.0 * (y * y + z * z), R01 = 2.0 * (x * y - w * z), R02 = 2.0 * (x * z + w * y);
-    const double R10 = 2.0 * (x * y + w * z), R11 = 1.0 - 2.0 * (x * x + z * z), R12 = 2.0 * (y * z - w * x);
-    const double R20 = 2.0 * (x * z - w * y), R21 = 2.0 * (y * z + w * x), R22 = 1.0 - 2.0 * (x * x + y * y);
-    const float* zj = a.noise + 6 * i + 3 * j;
-    const double s0 = exp(double(ls.x)) * double(__ldg(zj)), s1 = exp(double(ls.y)) * double(__ldg(zj + 1)),
-                 s2 = exp(double(ls.z)) * double(__ldg(zj + 2));
-    a.op.means[k] = make_float4(float(double(mu.x) + ((R00 * s0 + R01 * s1) + R02 * s2)),
-                                float(double(mu.y) + ((R10 * s0 + R11 * s1) + R12 * s2)),
-                                float(double(mu.z) + ((R20 * s0 + R21 * s1) + R22 * s2)), 0.f);
-    a.op.quats[k] = q4;
-    a.op.log_scales[k] = make_float4(float(double(ls.x) - a.log_split), float(double(ls.y) - a.log_split),
-                                     float(double(ls.z) - a.log_split), 0.f);
-    a.op.logits[k] = __ldg(a.p.logits + i);
-    for (int p = 0; p < a.planes; ++p) a.op.sh[int64_t(p) * a.n_out + k] = __ldg(a.p.sh + int64_t(p) * a.n + i);
+    const double w = qw / qn, x = qx / qn, y = qy / qn, zz = qz / qn;
+    const double R00 = 1.0 - 2.0 * (y * y + zz * zz), R01 = 2.0 * (x * y - w * zz), R02 = 2.0 * (x * zz + w * y);
+    const double R10 = 2.0 * (x * y + w * zz), R11 = 1.0 - 2.0 * (x * x + zz * zz), R12 = 2.0 * (y * zz - w * x);
+    const double R20 = 2.0 * (x * zz - w * y), R21 = 2.0 * (y * zz + w * x), R22 = 1.0 - 2.0 * (x * x + y * y);
+    const double s0 = exp(double(ls.x)) * double(__ldg(z)), s1 = exp(double(ls.y)) * double(__ldg(z + 1)),
+                 s2 = exp(double(ls.z)) * double(__ldg(z + 2));
+    o.means[k] = make_float4(float(double(mu.x) + ((R00 * s0 + R01 * s1) + R02 * s2)),
+                             float(double(mu.y) + ((R10 * s0 + R11 * s1) + R12 * s2)),
+                             float(double(mu.z) + ((R20 * s0 + R21 * s1) + R22 * s2)), 0.f);
+    o.log_scales[k] = make_float4(float(double(ls.x) - log_split), float(double(ls.y) - log_split),
+                                  float(double(ls.z) - log_split), 0.f);
+    o.quats[k] = q4;
+    o.logits[k] = p.logit;
+#pragma unroll
+    for (int pl = 0; pl < 12; ++pl)
+        if (pl < planes) o.sh[int64_t(pl) * n_out + k] = p.sh[pl];
 }
 
 __global__ void __launch_bounds__(kBlock) densify_apply_kernel(const ApplyArgs a) {
@@ -232,9 +254,11 @@ __global__ void __launch_bounds__(kBlock) densify_apply_kernel(const ApplyArgs a
         const int64_t k = int64_t(run + (incl - c));
         run += tile_total;
         if (c == 0 || k + c > a.n_out) continue;
+        Record r;
+        load_record(a.p, i, a.planes, a.n, r);
         if (d == GS_DENSIFY_SPLIT) {
-            write_child(a, i, k, 0);
-            write_child(a, i, k + 1, 1);
+            store_child(a.op, k, a.planes, a.n_out, r, a.noise + 6 * i, a.log_split);
+            store_child(a.op, k + 1, a.planes, a.n_out, r, a.noise + 6 * i + 3, a.log_split);
             if (a.moments) {
                 zero_group(a.om, k, a.planes, a.n_out);
                 zero_group(a.om, k + 1, a.planes, a.n_out);
@@ -243,14 +267,14 @@ __global__ void __launch_bounds__(kBlock) densify_apply_kernel(const ApplyArgs a
             }
             continue;
         }
-        copy_group(a.p, a.op, i, k, a.planes, a.n, a.n_out);
+        store_record(a.op, k, a.planes, a.n_out, r);
+        if (d == GS_DENSIFY_CLONE) store_record(a.op, k + 1, a.planes, a.n_out, r);
         if (a.moments) {
-            copy_group(a.m, a.om, i, k, a.planes, a.n, a.n_out);
-            copy_group(a.v, a.ov, i, k, a.planes, a.n, a.n_out);
-        }
-        if (d == GS_DENSIFY_CLONE) {
-            copy_group(a.p, a.op, i, k + 1, a.planes, a.n, a.n_out);
-            if (a.moments) {
+            load_record(a.m, i, a.planes, a.n, r);
+            store_record(a.om, k, a.planes, a.n_out, r);
+            load_record(a.v, i, a.planes, a.n, r);
+            store_record(a.ov, k, a.planes, a.n_out, r);
+            if (d == GS_DENSIFY_CLONE) {
                 zero_group(a.om, k + 1, a.planes, a.n_out);
                 zero_group(a.ov, k + 1, a.planes, a.n_out);
             }

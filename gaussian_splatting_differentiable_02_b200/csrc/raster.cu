@@ -3,25 +3,32 @@
 // §2.1: shared-memory prefetch of the tile's Gaussians, SoA features, warp-level
 // synchronisation; §2.2: a standalone backward entry).
 //
-// Work decomposition: one warp per tile, each lane owns a column of 8 pixels
-// (lane & 15 selects the column, lane >> 4 the upper or lower half), four tiles
-// per block.  The warp walks its tile's sorted list in batches of 32 entries:
-// every lane gathers one entry's 40 bytes (xy, conic + opacity, colour) by
-// Gaussian index into shared memory with cp.async, double-buffered so the next
-// batch is in flight while the current one is composited; the lane that
-// gathered an entry also derives its per-entry constants.  Every lane then
-// reads each entry once (broadcast loads) and applies it to its 8 pixels, whose
-// terms that depend only on dx are shared.  No block-wide barrier is used:
-// warps synchronise with __syncwarp and finish independently.
+// Work decomposition: one warp per 16x8 pixel box (two warps per tile, four
+// warps per block, blocks launched in the tile order of gs_tile_order when one
+// is given); each lane owns a column segment of 4 pixels (lane & 15 selects the
+// column, lane >> 4 the upper or lower half of the box).  The warp walks its
+// tile's sorted list in batches of 32 entries: every lane gathers one entry's
+// 40 bytes (xy, conic + opacity, colour) by Gaussian index into shared memory
+// with cp.async, double-buffered so the next batch is in flight while the
+// current one is composited; the lane that gathered an entry also derives its
+// per-entry constants and tests the entry against the warp's whole box (an
+// entry whose smallest sigma over the box leaves alpha below 1/255 is skipped
+// by the warp).  Every lane then reads each entry once (broadcast loads) and
+// applies it to its 4 pixels, whose terms that depend only on dx are shared;
+// the pixels go in pairs through the paired float32 instructions of sm_100
+// (fma/mul/add on two floats at once).  No block-wide barrier is used: warps
+// synchronise with __syncwarp and finish independently.
 //
-// Forward: a warp stops as soon as all 256 pixels have terminated (warp vote
-// per entry).  Backward: back to front from the largest n_contrib of the tile;
-// each lane sums its 8 pixels' contributions, the 9 per-Gaussian sums are
-// reduce-scattered across the warp (18 shuffles) and three lanes issue one
-// float2 / float4 atomic add each (batched atomics, MUSA co-design article
-// qwbw.cn/news/278220 §2.2).  The gradient with respect to (u, v, A, B, C) is
-// accumulated as three moments of dL/dsigma over the lane's pixels, then
-// combined with dx and the conic once per entry.
+// Forward: a warp stops as soon as all 128 pixels have terminated (warp vote
+// per entry).  Backward: back to front from the largest n_contrib of the box,
+// the transmittance in front of each entry recovered with rcp(1 - alpha) and
+// g . S (S the colour blended behind) tracked per pixel; each lane sums its
+// pixels' contributions, the 9 per-Gaussian sums are reduce-scattered across
+// the warp (18 shuffles) and three lanes issue one float2 / float4 atomic add
+// each (batched atomics, MUSA co-design article qwbw.cn/news/278220 §2.2).  The
+// gradient with respect to (u, v, A, B, C) is accumulated as moments of
+// dL/dsigma over the lane's pixels, then combined with dx and the conic once
+// per entry.
 //
 // Both passes evaluate alpha with the same inline code built from explicit
 // rounding intrinsics, so the backward pass repeats the forward pass's skip and
@@ -64,7 +71,7 @@ constexpr int kWarps = 4;                // warps per block
 static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
 // resident blocks per SM the register allocation is sized for (launch bounds)
 #ifndef GS_RASTER_FWD_MIN_BLOCKS
-#define GS_RASTER_FWD_MIN_BLOCKS 6
+#define GS_RASTER_FWD_MIN_BLOCKS 5
 #endif
 #ifndef GS_RASTER_BWD_MIN_BLOCKS
 #define GS_RASTER_BWD_MIN_BLOCKS 5
@@ -153,8 +160,13 @@ __device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by
 // the rounding of either evaluation, so no pixel of the warp would blend it.
 // The bound is computed in float32 for well-conditioned conics and in double
 // for the others.
+template <bool kNegRgb>
 __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
     if (lane < count) {
+        if (kNegRgb) {  // the forward pass blends with -alpha T weights
+            const float4 c = S.rgb[buf][lane];
+            S.rgb[buf][lane] = make_float4(-c.x, -c.y, -c.z, c.w);
+        }
         const float2 xy = S.xy[buf][lane];
         const float4 c = S.con[buf][lane];
         const float tr = __fadd_rn(c.x, c.z);
@@ -191,62 +203,87 @@ __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane,
     }
 }
 
-// alpha of one entry at the lane's pixels, and the offsets dx (shared) and
-// dy[i] of the mean from the pixel centres (t[i] = dx + (B/A) dy[i] for a
-// factored entry).  Bit i of `blend` is set when pixel i passes sigma >= 0 and
-// alpha >= 1/255; bit i of `clamp` when alpha was clamped at 0.99.
+// Pairs of pixels go through the paired float32 instructions of sm_100
+// (two IEEE operations per instruction, rounded as two scalar ones).
+constexpr int kPairs = kPx / 2;
+static_assert(kPx % 2 == 0, "pixels per lane come in pairs");
+using f2 = float2;
+__device__ __forceinline__ f2 splat(float v) { return make_float2(v, v); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
+
+// One entry at the lane's pixels: -alpha per pixel (pairs 2p, 2p + 1), the
+// offsets dx (shared) and dy of the mean from the pixel centres, t = dx +
+// (B/A) dy for a factored entry; bit i of `blend` is set when pixel i passes
+// sigma >= 0 and alpha >= 1/255, bit i of `clamp` when alpha was clamped at 0.99.
+struct Alpha {
+    f2 nal[kPairs];
+    f2 dy[kPairs];
+    f2 t[kPairs];
+    unsigned blend, clamp;
+    float dx;
+};
+
+__device__ __forceinline__ void alpha_at(float e, bool sign_ok, int i, float& nal, unsigned& blend,
+                                         unsigned& clamp) {
+    const float a = ex2_approx(e);
+    nal = fmaxf(-a, -kAlphaMax);  // -min(a, 0.99)
+    if (sign_ok && nal <= -kAlphaMin) blend |= 1u << i;
+    if (a > kAlphaMax) clamp |= 1u << i;
+}
+
+// nyc[p]: minus the centres' y of the lane's pixels 2p and 2p + 1.
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
-                                           float px, int y0, float (&alpha)[kPx], unsigned& blend, unsigned& clamp,
-                                           float& dx, float (&dy)[kPx], float (&t)[kPx]) {
-    blend = 0u;
-    clamp = 0u;
+                                           float px, const f2 (&nyc)[kPairs], Alpha& r) {
+    r.blend = 0u;
+    r.clamp = 0u;
+    const f2 vy = splat(pa.y), lo = splat(pa.z);
     if (pb.w == kFactored) {
-        dx = __fsub_rn(pa.x, px);
+        r.dx = __fsub_rn(pa.x, px);
+        const f2 dx2 = splat(r.dx), rh = splat(pb.x), rl = splat(pb.y), ka = splat(pc.x), kd = splat(pc.y);
 #pragma unroll
-        for (int i = 0; i < kPx; ++i) {
-            dy[i] = __fsub_rn(pa.y, __fadd_rn(float(y0 + i), 0.5f));
-            t[i] = __fmaf_rn(pb.y, dy[i], __fmaf_rn(pb.x, dy[i], dx));
-            const float s = __fmaf_rn(__fmul_rn(pc.x, t[i]), t[i], __fmul_rn(__fmul_rn(pc.y, dy[i]), dy[i]));
-            const float a = ex2_approx(__fadd_rn(s, pa.z));
-            const bool c = a > kAlphaMax;
-            alpha[i] = c ? kAlphaMax : a;
-            if (alpha[i] >= kAlphaMin) blend |= 1u << i;  // s <= 0 by construction
-            if (c) clamp |= 1u << i;
+        for (int p = 0; p < kPairs; ++p) {
+            r.dy[p] = add2(vy, nyc[p]);
+            r.t[p] = fma2(rl, r.dy[p], fma2(rh, r.dy[p], dx2));
+            const f2 e = add2(fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p])), lo);
+            alpha_at(e.x, true, 2 * p, r.nal[p].x, r.blend, r.clamp);  // sigma >= 0 by construction
+            alpha_at(e.y, true, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
         }
     } else if (pb.w == kDouble) {
         const double dxd = __dsub_rn(double(pa.x), double(px));
-        dx = __double2float_rn(dxd);
+        r.dx = __double2float_rn(dxd);
         const double A = con.x, B = con.y, C = con.z;
         const double adx2 = __dmul_rn(__dmul_rn(A, dxd), dxd);
         const double bdx = __dmul_rn(B, dxd);
 #pragma unroll
         for (int i = 0; i < kPx; ++i) {
-            const double dyd = __dsub_rn(double(pa.y), double(y0 + i) + 0.5);
+            const double dyd = __dsub_rn(double(pa.y), -double(i & 1 ? nyc[i / 2].y : nyc[i / 2].x));
             const double sig = __dadd_rn(__dmul_rn(0.5, __dadd_rn(adx2, __dmul_rn(__dmul_rn(C, dyd), dyd))),
                                          __dmul_rn(bdx, dyd));
-            const float s = __double2float_rn(__dmul_rn(-sig, kLog2eD));
-            dy[i] = __double2float_rn(dyd);
-            t[i] = 0.f;
-            const float a = ex2_approx(__fadd_rn(s, pa.z));
-            const bool c = a > kAlphaMax;
-            alpha[i] = c ? kAlphaMax : a;
-            if (s <= 0.f && alpha[i] >= kAlphaMin) blend |= 1u << i;
-            if (c) clamp |= 1u << i;
+            const float sv = __double2float_rn(__dmul_rn(-sig, kLog2eD));
+            const float dyf = __double2float_rn(dyd);
+            float nal;
+            alpha_at(__fadd_rn(sv, pa.z), sv <= 0.f, i, nal, r.blend, r.clamp);
+            if (i & 1) {
+                r.dy[i / 2].y = dyf;
+                r.nal[i / 2].y = nal;
+            } else {
+                r.dy[i / 2].x = dyf;
+                r.nal[i / 2].x = nal;
+            }
         }
     } else {
-        dx = __fsub_rn(pa.x, px);
-        const float a0 = __fmul_rn(__fmul_rn(pb.x, dx), dx);
-        const float c1 = __fmul_rn(pb.y, dx);
+        r.dx = __fsub_rn(pa.x, px);
+        const f2 a0 = splat(__fmul_rn(__fmul_rn(pb.x, r.dx), r.dx)), c1 = splat(__fmul_rn(pb.y, r.dx));
+        const f2 cz = splat(pb.z);
 #pragma unroll
-        for (int i = 0; i < kPx; ++i) {
-            dy[i] = __fsub_rn(pa.y, __fadd_rn(float(y0 + i), 0.5f));
-            t[i] = 0.f;
-            const float s = __fmaf_rn(dy[i], __fmaf_rn(pb.z, dy[i], c1), a0);
-            const float a = ex2_approx(__fadd_rn(s, pa.z));
-            const bool c = a > kAlphaMax;
-            alpha[i] = c ? kAlphaMax : a;
-            if (s <= 0.f && alpha[i] >= kAlphaMin) blend |= 1u << i;
-            if (c) clamp |= 1u << i;
+        for (int p = 0; p < kPairs; ++p) {
+            r.dy[p] = add2(vy, nyc[p]);
+            const f2 sv = fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0);
+            const f2 e = add2(sv, lo);
+            alpha_at(e.x, sv.x <= 0.f, 2 * p, r.nal[p].x, r.blend, r.clamp);
+            alpha_at(e.y, sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
         }
     }
 }
@@ -282,17 +319,22 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     const uint2 range = a.ranges[tile];
     const int n = int(range.y - range.x);
 
-    float T[kPx], Cr[kPx], Cg[kPx], Cb[kPx];
+    f2 nyc[kPairs], T[kPairs], Cr[kPairs], Cg[kPairs], Cb[kPairs];
     int last[kPx];
     unsigned done = 0u;
 #pragma unroll
+    for (int p = 0; p < kPairs; ++p) {
+        nyc[p] = make_float2(-(float(y0 + 2 * p) + 0.5f), -(float(y0 + 2 * p + 1) + 0.5f));
+        T[p] = splat(1.f);
+        Cr[p] = Cg[p] = Cb[p] = splat(0.f);
+    }
+#pragma unroll
     for (int i = 0; i < kPx; ++i) {
-        T[i] = 1.f;
-        Cr[i] = Cg[i] = Cb[i] = 0.f;
         last[i] = 0;
         if (x >= a.W || y0 + i >= a.H) done |= 1u << i;
     }
     constexpr unsigned kAll = (1u << kPx) - 1u;
+    const f2 one = splat(1.f);
 
     const int nb = (n + kBatch - 1) / kBatch;
     if (n > 0) gather<false>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x, min(n, kBatch), lane);
@@ -304,7 +346,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (b + 1 < nb)
             gather<false>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t((b + 1) * kBatch),
                           min(n - (b + 1) * kBatch, kBatch), lane);
-        prep(S, buf, cnt, lane, bx0, by0);
+        prep<true>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         bool finished = false;
         for (int j = 0; j < cnt; ++j) {
@@ -315,27 +357,32 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
             const float4 pa = S.pa[j], pb = S.pb[j];
             if (pb.w == kSkip) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
-            const float4 c = S.rgb[buf][j];
-            float al[kPx], dy[kPx], tt[kPx], dx;
-            unsigned blend, clamp;
-            eval_alpha(pa, pb, S.pc[j], con, px, y0, al, blend, clamp, dx, dy, tt);
-            blend &= ~done;
+            const float4 nc = S.rgb[buf][j];  // minus the colour
+            Alpha r;
+            eval_alpha(pa, pb, S.pc[j], con, px, nyc, r);
+            const unsigned blend = r.blend & ~done;
             const int pos = b * kBatch + j + 1;
-            // branch-free so the 8 independent pixel chains interleave; a pixel
-            // that does not take the entry adds c * 0 (exactly nothing)
+            const f2 ncr = splat(nc.x), ncg = splat(nc.y), ncb = splat(nc.z);
+            // branch-free so the pixel chains interleave; a pixel that does not
+            // take the entry adds c * 0 (exactly nothing)
 #pragma unroll
-            for (int i = 0; i < kPx; ++i) {
-                const bool act = (blend >> i) & 1u;
-                const float Tn = __fmul_rn(T[i], __fsub_rn(1.f, al[i]));
-                const bool low = Tn < kTMin;
-                const bool take = act && !low;
-                const float w = take ? __fmul_rn(al[i], T[i]) : 0.f;
-                Cr[i] = __fmaf_rn(c.x, w, Cr[i]);
-                Cg[i] = __fmaf_rn(c.y, w, Cg[i]);
-                Cb[i] = __fmaf_rn(c.z, w, Cb[i]);
-                T[i] = take ? Tn : T[i];
-                last[i] = take ? pos : last[i];
-                done |= (act && low) ? (1u << i) : 0u;
+            for (int p = 0; p < kPairs; ++p) {
+                const f2 Tn = mul2(T[p], add2(one, r.nal[p]));  // T (1 - alpha)
+                f2 nw = mul2(r.nal[p], T[p]);                    // -alpha T
+                const bool act0 = (blend >> (2 * p)) & 1u, act1 = (blend >> (2 * p + 1)) & 1u;
+                const bool low0 = Tn.x < kTMin, low1 = Tn.y < kTMin;
+                const bool take0 = act0 && !low0, take1 = act1 && !low1;
+                nw.x = take0 ? nw.x : 0.f;
+                nw.y = take1 ? nw.y : 0.f;
+                Cr[p] = fma2(ncr, nw, Cr[p]);
+                Cg[p] = fma2(ncg, nw, Cg[p]);
+                Cb[p] = fma2(ncb, nw, Cb[p]);
+                T[p].x = take0 ? Tn.x : T[p].x;
+                T[p].y = take1 ? Tn.y : T[p].y;
+                last[2 * p] = take0 ? pos : last[2 * p];
+                last[2 * p + 1] = take1 ? pos : last[2 * p + 1];
+                done |= (act0 && low0) ? (1u << (2 * p)) : 0u;
+                done |= (act1 && low1) ? (1u << (2 * p + 1)) : 0u;
             }
         }
         __syncwarp();
@@ -347,10 +394,11 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         for (int i = 0; i < kPx; ++i) {
             if (y0 + i < a.H) {
                 const int64_t pix = int64_t(y0 + i) * a.W + x;
-                a.image[3 * pix + 0] = __fmaf_rn(T[i], a.bg0, Cr[i]);
-                a.image[3 * pix + 1] = __fmaf_rn(T[i], a.bg1, Cg[i]);
-                a.image[3 * pix + 2] = __fmaf_rn(T[i], a.bg2, Cb[i]);
-                a.final_T[pix] = T[i];
+                const float Ti = i & 1 ? T[i / 2].y : T[i / 2].x;
+                a.image[3 * pix + 0] = __fmaf_rn(Ti, a.bg0, i & 1 ? Cr[i / 2].y : Cr[i / 2].x);
+                a.image[3 * pix + 1] = __fmaf_rn(Ti, a.bg1, i & 1 ? Cg[i / 2].y : Cg[i / 2].x);
+                a.image[3 * pix + 2] = __fmaf_rn(Ti, a.bg2, i & 1 ? Cb[i / 2].y : Cb[i / 2].x);
+                a.final_T[pix] = Ti;
                 a.n_contrib[pix] = last[i];
             }
         }
@@ -437,27 +485,35 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     const float bx0 = float(xb) + 0.5f, by0 = float(yb) + 0.5f;  // box corner (pixel centre)
     const uint2 range = a.ranges[tile];
 
-    float T[kPx], P[kPx], gr[kPx], gg[kPx], gb[kPx], ngb[kPx];
+    // per pixel pair: transmittance, minus g . S (S the colour blended behind),
+    // dL/dimage, -final_T (bg . g)
+    f2 nyc[kPairs], T[kPairs], nP[kPairs], gr[kPairs], gg[kPairs], gb[kPairs], ngb[kPairs];
     int last[kPx];
     int lmax = 0;
 #pragma unroll
     for (int i = 0; i < kPx; ++i) {
-        P[i] = 0.f;
+        float Ti = 1.f, r = 0.f, g = 0.f, bb = 0.f;
+        last[i] = 0;
         if (x < a.W && y0 + i < a.H) {
             const int64_t pix = int64_t(y0 + i) * a.W + x;
-            T[i] = a.final_T[pix];
+            Ti = a.final_T[pix];
             last[i] = a.n_contrib[pix];
-            gr[i] = a.dL_dimage[3 * pix + 0];
-            gg[i] = a.dL_dimage[3 * pix + 1];
-            gb[i] = a.dL_dimage[3 * pix + 2];
-        } else {
-            T[i] = 1.f;
-            last[i] = 0;
-            gr[i] = gg[i] = gb[i] = 0.f;
+            r = a.dL_dimage[3 * pix + 0];
+            g = a.dL_dimage[3 * pix + 1];
+            bb = a.dL_dimage[3 * pix + 2];
         }
-        ngb[i] = -T[i] * (a.bg0 * gr[i] + a.bg1 * gg[i] + a.bg2 * gb[i]);
+        const float nb = -Ti * (a.bg0 * r + a.bg1 * g + a.bg2 * bb);
+        const float ny = -(float(y0 + i) + 0.5f);
+        if (i & 1) {
+            T[i / 2].y = Ti; gr[i / 2].y = r; gg[i / 2].y = g; gb[i / 2].y = bb; ngb[i / 2].y = nb; nyc[i / 2].y = ny;
+        } else {
+            T[i / 2].x = Ti; gr[i / 2].x = r; gg[i / 2].x = g; gb[i / 2].x = bb; ngb[i / 2].x = nb; nyc[i / 2].x = ny;
+        }
         lmax = max(lmax, last[i]);
     }
+#pragma unroll
+    for (int p = 0; p < kPairs; ++p) nP[p] = splat(0.f);
+    const f2 one = splat(1.f), zero = splat(0.f);
     // entries past every pixel's last are never needed; never read past the list
     const int total = min(__reduce_max_sync(kFull, lmax), int(range.y - range.x));
     const int nb = (total + kBatch - 1) / kBatch;
@@ -475,7 +531,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             const int nhi = hi - kBatch, ncnt = min(nhi, kBatch);
             gather<true>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncnt), ncnt, lane);
         }
-        prep(S, buf, cnt, lane, bx0, by0);
+        prep<false>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         for (int j = 0; j < cnt; ++j) {
             const int pos = hi - 1 - j;  // 0-based list position of this entry
@@ -483,61 +539,69 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             if (pb.w == kSkip) continue;  // misses every pixel of this warp
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
-            float al[kPx], dy[kPx], tt[kPx], m[kPx], dx;
-            unsigned blend, clamp;
-            eval_alpha(pa, pb, S.pc[j], con, px, y0, al, blend, clamp, dx, dy, tt);
-            float dr = 0.f, dg = 0.f, db = 0.f, mo = 0.f, s1 = 0.f, s2 = 0.f, st = 0.f;
+            Alpha r;
+            eval_alpha(pa, pb, S.pc[j], con, px, nyc, r);
+            const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
+            f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
             bool any = false;
             // branch-free: every pixel runs the same instructions, inactive ones
-            // with zero weight and unchanged state
+            // with alpha 0, so T, P and every sum stay unchanged
 #pragma unroll
-            for (int i = 0; i < kPx; ++i) {
-                const bool act = ((blend >> i) & 1u) && pos < last[i];
-                any = any || act;
-                // an inactive pixel runs the same instructions with alpha 0: T, S and
-                // every sum stay unchanged
-                const float ae = act ? al[i] : 0.f;
-                const float rom = rcp_approx(__fsub_rn(1.f, ae));
-                T[i] = T[i] * rom;  // transmittance in front of this entry
-                const float w = ae * T[i];
-                dr = fmaf(w, gr[i], dr);
-                dg = fmaf(w, gg[i], dg);
-                db = fmaf(w, gb[i], db);
+            for (int p = 0; p < kPairs; ++p) {
+                const bool act0 = ((r.blend >> (2 * p)) & 1u) && pos < last[2 * p];
+                const bool act1 = ((r.blend >> (2 * p + 1)) & 1u) && pos < last[2 * p + 1];
+                any = any || act0 || act1;
+                const f2 nae = make_float2(act0 ? r.nal[p].x : 0.f, act1 ? r.nal[p].y : 0.f);  // -alpha
+                const f2 om = add2(one, nae);                                                  // 1 - alpha
+                const f2 rom = make_float2(rcp_approx(om.x), rcp_approx(om.y));
+                T[p] = mul2(T[p], rom);  // transmittance in front of this entry
+                const f2 nw = mul2(nae, T[p]);
+                ndr = fma2(nw, gr[p], ndr);
+                ndg = fma2(nw, gg[p], ndg);
+                ndb = fma2(nw, gb[p], ndb);
                 // only g . S enters the gradient: P = g . S with S <- c alpha + (1 - alpha) S
-                const float x = fmaf(gr[i], c.x, fmaf(gg[i], c.y, gb[i] * c.z)) - P[i];
-                const float dLda = fmaf(T[i], x, ngb[i] * rom);
-                P[i] = fmaf(ae, x, P[i]);
-                m[i] = ((clamp >> i) & 1u) ? 0.f : dLda * ae;  // dL/dsigma = -m, dL/do = m / o
-                mo += m[i];
-                s1 = fmaf(-m[i], dy[i], s1);
-                s2 = fmaf(-m[i] * dy[i], dy[i], s2);
-                st = fmaf(-m[i], tt[i], st);  // factored entries only (tt = 0 otherwise)
+                const f2 xg = add2(fma2(gr[p], cr, fma2(gg[p], cg, mul2(gb[p], cb))), nP[p]);  // g . c - P
+                const f2 dLda = fma2(T[p], xg, mul2(ngb[p], rom));
+                nP[p] = fma2(nae, xg, nP[p]);
+                f2 q = mul2(dLda, nae);  // -dL/dalpha alpha = dL/dsigma (zero when clamped)
+                q.x = ((r.clamp >> (2 * p)) & 1u) ? 0.f : q.x;
+                q.y = ((r.clamp >> (2 * p + 1)) & 1u) ? 0.f : q.y;
+                nm[p] = q;
+                nmo = add2(nmo, q);
+                s1 = fma2(q, r.dy[p], s1);
+                s2 = fma2(mul2(q, r.dy[p]), r.dy[p], s2);
             }
-            const float s0 = -mo;
             if (__any_sync(kFull, any)) {
+                const float s0 = nmo.x + nmo.y, mo = -s0, m1 = s1.x + s1.y;
                 float du, dv;
                 if (pb.w == kFactored) {
                     // dsigma/du = A t, dsigma/dv = B t + D dy
-                    du = con.x * st;
-                    dv = fmaf(con.y, st, pb.z * s1);
+                    f2 st = zero;
+#pragma unroll
+                    for (int p = 0; p < kPairs; ++p) st = fma2(nm[p], r.t[p], st);
+                    const float stt = st.x + st.y;
+                    du = con.x * stt;
+                    dv = fmaf(con.y, stt, pb.z * m1);
                 } else if (pb.w == kDouble) {
                     // not positive definite: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
                     const double dxd = __dsub_rn(double(pa.x), double(px));
                     du = dv = 0.f;
 #pragma unroll
                     for (int i = 0; i < kPx; ++i) {
-                        const double dyd = __dsub_rn(double(pa.y), double(y0 + i) + 0.5);
+                        const double dyd = __dsub_rn(double(pa.y), -double(i & 1 ? nyc[i / 2].y : nyc[i / 2].x));
                         const float su = __double2float_rn(double(con.x) * dxd + double(con.y) * dyd);
                         const float sv = __double2float_rn(double(con.y) * dxd + double(con.z) * dyd);
-                        du = fmaf(-m[i], su, du);
-                        dv = fmaf(-m[i], sv, dv);
+                        const float qi = i & 1 ? nm[i / 2].y : nm[i / 2].x;
+                        du = fmaf(qi, su, du);
+                        dv = fmaf(qi, sv, dv);
                     }
                 } else {
-                    du = fmaf(con.x * dx, s0, con.y * s1);
-                    dv = fmaf(con.y * dx, s0, con.z * s1);
+                    du = fmaf(con.x * r.dx, s0, con.y * m1);
+                    dv = fmaf(con.y * r.dx, s0, con.z * m1);
                 }
-                float v[8] = {du, dv, 0.5f * dx * dx * s0, dx * s1, 0.5f * s2, mo * pa.w, dr, dg};
-                warp_reduce_and_add(v, db, lane, S.gid[buf][j], a);
+                float v[8] = {du, dv, 0.5f * r.dx * r.dx * s0, r.dx * m1, 0.5f * (s2.x + s2.y), mo * pa.w,
+                              -(ndr.x + ndr.y), -(ndg.x + ndg.y)};
+                warp_reduce_and_add(v, -(ndb.x + ndb.y), lane, S.gid[buf][j], a);
             }
         }
         __syncwarp();

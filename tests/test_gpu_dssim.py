@@ -29,8 +29,10 @@ def _gpu(img, tgt, l1w=1.0, sw=0.2):
 
 def _compare(orc, img, tgt, l1w=1.0, sw=0.2):
     loss, g = _gpu(img, tgt, l1w, sw)
+    # the weights cross the C boundary as float32
     want_loss, want_g = orc.l1_dssim(img.astype(np.float32).astype(np.float64),
-                                     tgt.astype(np.float32).astype(np.float64), l1w, sw)
+                                     tgt.astype(np.float32).astype(np.float64), float(np.float32(l1w)),
+                                     float(np.float32(sw)))
     assert abs(loss - want_loss) <= 1e-12 * max(1.0, abs(want_loss)), (loss, want_loss)
     w32 = want_g.astype(np.float32)
     ulp = np.spacing(np.abs(w32)).astype(np.float64)
