@@ -357,7 +357,8 @@ def run_ours(args, world, rank, local):
     # rows outside the per-step path, measured after the step timing
     with_oracle = rank == 0 and not args.no_cpu_baseline and world == 1
     line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
-                    "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle)}
+                    "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
+                    "absgrad_and_sparse_adam": measure_variants(tr, torch)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
         line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
@@ -365,6 +366,45 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_variants(tr, torch, reps: int = 10):
+    """Cost of the absgrad option (raster backward with the absolute 2D gradient) on
+    the first view, and of the sparse Adam option of the fused backward, each
+    against the default, with CUDA events over `reps` launches."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    s = torch.cuda.current_stream()
+    view, r = tr.views[0], tr.radii[0]
+    pl.project(tr.gauss, view, tr.proj, r)
+    pl.bin_sort(tr.proj, view, r)
+    pl.raster_fwd(tr.proj, view, tr.bg, r)
+    plain = pl.Grad2D(tr.gauss.n)
+    absg = pl.Grad2D(tr.gauss.n, absgrad=True)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    res = {"raster_bwd_ms": timed(lambda: pl.raster_bwd(tr.proj, view, plain, tr.bg, radius=r)),
+           "raster_bwd_absgrad_ms": timed(lambda: pl.raster_bwd(tr.proj, view, absg, tr.bg, radius=r))}
+    # the fused backward with Adam on copies of the parameters and moments
+    g, m, v = (x.zeros_like() for x in (tr.gauss, tr.gauss, tr.gauss))
+    for dst, src in ((g, tr.gauss), (m, tr.m), (v, tr.v)):
+        for a, b in zip(dst.tensors().values(), src.tensors().values()):
+            a.copy_(b)
+    for sparse in (False, True):
+        res["project_bwd_adam_sparse_ms" if sparse else "project_bwd_adam_ms"] = timed(
+            lambda: pl.project_bwd_views_adam(g, tr.views, tr.proj, tr.radii, tr.grad2ds, m, v, tr.lrs,
+                                              tr.step_count + 1, sparse=sparse))
+    res["visible_fraction"] = float((tr.radii > 0).any(dim=0).float().mean().item())
+    return res
 
 
 def measure_dssim(tr, wl, peaks, torch, with_oracle: bool, reps: int = 10):
@@ -602,8 +642,10 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
     stream = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
     nv = len(tr.views)
+    side = tr.side_streams()
+    nbuf = min(nv, 2 * len(side))   # targets in flight: the views running plus the next ones
     loss_host = torch.zeros(1, dtype=torch.float64).pin_memory()
-    bufs = [torch.empty_like(targets[0]) for _ in range(2)]
+    bufs = [torch.empty_like(targets[0]) for _ in range(nbuf)]
 
     # the view loop mirrors Trainer.step with the target taken from the copy buffers
     from gaussian_splatting_differentiable_02_b200 import pipeline as pl
@@ -612,26 +654,31 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
     def step():
         nonlocal done
         done = [torch.cuda.Event() for _ in range(nv)]
-        s = stream.cuda_stream
-        abi.gs_zero(tr.loss.data_ptr(), 8, s)
-        copy_events = []
+        abi.gs_zero(tr.loss.data_ptr(), 8, stream.cuda_stream)
+        begin = stream.record_event()
+        copy_events = {}
         with torch.cuda.stream(copy_stream):
-            for v in range(min(2, nv)):
-                bufs[v % 2].copy_(targets_host[v], non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(copy_stream)
-                copy_events.append(e)
+            copy_stream.wait_event(begin)   # the previous step's views are done with the buffers
+            for v in range(nbuf):
+                bufs[v].copy_(targets_host[v], non_blocking=True)
+                copy_events[v] = copy_stream.record_event()
         for v in range(nv):
-            stream.wait_event(copy_events[v])
-            tr.view_forward_backward(v, bufs[v % 2])
-            done[v].record(stream)
-            if v + 2 < nv:
+            st = side[v % len(side)]
+            st.wait_event(begin)
+            st.wait_event(copy_events[v])
+            with torch.cuda.stream(st):
+                tr.view_forward_backward(v, bufs[v % nbuf], tr.projs[v % len(side)])
+            done[v].record(st)
+            if v + nbuf < nv:
                 with torch.cuda.stream(copy_stream):
                     copy_stream.wait_event(done[v])
-                    bufs[v % 2].copy_(targets_host[v + 2], non_blocking=True)
-                    e = torch.cuda.Event()
-                    e.record(copy_stream)
-                    copy_events.append(e)
+                    bufs[v % nbuf].copy_(targets_host[v + nbuf], non_blocking=True)
+                    copy_events[v + nbuf] = copy_stream.record_event()
+        for st in side:
+            stream.wait_stream(st)
+        # the step's one wait: the instance counts (buffers were sized in the warm-up)
+        if any(K > vw.capacity for K, vw in zip(tr.kcount.cpu().tolist(), tr.views)):
+            raise RuntimeError("instance buffers overflowed after the warm-up")
         tr.step_count += 1
         pl.project_bwd_views_adam(tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m, tr.v, tr.lrs,
                                   tr.step_count, None, tr.densify_accum, tr.densify_count,

@@ -52,7 +52,7 @@ class gs_projected(C.Structure):
 
 
 class gs_grad2d(C.Structure):
-    _fields_ = [("xy", C.c_void_p), ("conic_opacity", C.c_void_p), ("rgb", C.c_void_p)]
+    _fields_ = [("xy", C.c_void_p), ("conic_opacity", C.c_void_p), ("rgb", C.c_void_p), ("xy_abs", C.c_void_p)]
 
 
 class gs_densify_config(C.Structure):
@@ -95,7 +95,8 @@ SIGNATURES = {
                                               C.POINTER(gs_projected), C.POINTER(gs_grad2d),
                                               C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
                                               C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float, C.c_float,
-                                              C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P, _P]),
+                                              C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P, C.c_int32,
+                                              _P]),
     "gs_l1_dssim_workspace_bytes": (C.c_size_t, [C.c_int32, C.c_int32]),
     "gs_l1_dssim_loss_grad": (C.c_int32, [_P, _P, C.c_int32, C.c_int32, C.c_float, C.c_float, _P, C.c_size_t, _P, _P,
                                           _P]),
@@ -261,16 +262,17 @@ def gs_project_bwd_views(params: gs_params, cams, projs, grad2ds, grads: gs_para
 def gs_project_bwd_views_adam(params: gs_params, cams, projs, grad2ds, params_inout: gs_param_grads,
                               adam_m: gs_param_grads, adam_v: gs_param_grads, lrs, beta1: float, beta2: float,
                               eps: float, step: int, grads: gs_param_grads = None, densify_accum: int = 0,
-                              densify_count: int = 0, densify_max_radius: int = 0, stream: int = 0):
+                              densify_count: int = 0, densify_max_radius: int = 0, sparse_adam: int = 0,
+                              stream: int = 0):
     """Multi-view backward through the projection with the Adam step fused; lrs = 5 learning rates
-    (means, quats, log_scales, opacity_logits, sh)."""
+    (means, quats, log_scales, opacity_logits, sh); sparse_adam = 1 skips Gaussians visible in no view."""
     V = len(cams)
     lr = (C.c_float * 5)(*[float(x) for x in lrs])
     return _check(lib().gs_project_bwd_views_adam(
         C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _arr(gs_grad2d, grad2ds),
         C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps, step,
         C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None,
-        densify_max_radius or None, stream))
+        densify_max_radius or None, int(sparse_adam), stream))
 
 
 def gs_l1_dssim_workspace_bytes(width: int, height: int) -> int:

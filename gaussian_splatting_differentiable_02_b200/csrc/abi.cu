@@ -287,6 +287,7 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
     CHECK_PTR(grad2d->xy, 8);
     CHECK_PTR(grad2d->conic_opacity, 16);
     CHECK_PTR(grad2d->rgb, 16);
+    if (grad2d->xy_abs) CHECK_PTR(grad2d->xy_abs, 8);
     const gsk::CamArgs c = gsk::make_cam(*cam);
     return cuda_status(gsk::launch_raster_bwd(*proj, vals, tile_ranges, tile_order, c, bg_host, final_T, n_contrib,
                                               dL_dimage, *grad2d, static_cast<cudaStream_t>(stream)),
@@ -329,6 +330,7 @@ gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t nu
             CHECK_PTR(grad2d[v].xy, 8);
             CHECK_PTR(grad2d[v].conic_opacity, 16);
             CHECK_PTR(grad2d[v].rgb, 16);
+            if (grad2d[v].xy_abs) CHECK_PTR(grad2d[v].xy_abs, 8);
         }
     }
     if (params->n > 0) {
@@ -385,8 +387,9 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
                                     gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
                                     float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
                                     float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
-                                    void* stream) {
+                                    int32_t sparse_adam, void* stream) {
     const char* fn = "gs_project_bwd_views_adam";
+    if (sparse_adam != 0 && sparse_adam != 1) return fail(GS_ERR_INVALID_ARG, "%s: sparse_adam must be 0 or 1", fn);
     if (!lr_host) return fail(GS_ERR_INVALID_ARG, "%s: lr_host is NULL", fn);
     gsk::AdamStep a;
     gs_status st;
@@ -404,6 +407,7 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
     a.beta2 = beta2;
     a.eps = eps;
     a.step = step;
+    a.sparse = sparse_adam == 1;
     return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
                               densify_max_radius, &a, stream);
 }

@@ -53,6 +53,7 @@ struct AdamStep {
     float lr[5];  // means, quats, log_scales, opacity_logits, sh
     float beta1, beta2, eps;
     int step;
+    bool sparse;  // skip Gaussians visible in no view (parameters and moments untouched)
 };
 
 // Backward through the projection for V <= GS_MAX_VIEWS views of the same

@@ -40,6 +40,7 @@ struct ViewArgs {
     float R[9], t[3], fx, fy;
     const int32_t* radius;
     const float2* g_xy;
+    const float2* g_xy_abs;  // absolute 2D gradient for the densification statistic (nullable)
     const float4* g_con;
     const float4* g_rgb;
 };
@@ -62,6 +63,7 @@ struct Args {
     float* densify_accum;
     int32_t* densify_count;
     int32_t* densify_max_radius;
+    bool sparse;  // Adam: leave Gaussians visible in no view untouched
     // Adam (kAdam): parameters updated in place, first and second moments
     float4* p_means;
     float4* p_quats;
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
             if (r > 0) vis |= 1u << v;
             rmax = max(rmax, r);
         }
-        if (!kAdam && vis == 0u) continue;
+        if ((!kAdam || a.sparse) && vis == 0u) continue;  // nothing to add (sparse Adam: nothing to update)
         if (a.densify_max_radius && rmax > a.densify_max_radius[i]) a.densify_max_radius[i] = rmax;
 
         double gS[6] = {0, 0, 0, 0, 0, 0};  // symmetric dL/dSigma: xx, xy, xz, yy, yz, zz
@@ -365,7 +367,8 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
                 gmu[1] += (gdir[1] - uy * dproj) / dn;
                 gmu[2] += (gdir[2] - uz * dproj) / dn;
 
-                dacc += sqrtf(gxy.x * gxy.x + gxy.y * gxy.y);
+                const float2 sxy = cam.g_xy_abs ? __ldg(cam.g_xy_abs + i) : gxy;
+                dacc += sqrtf(sxy.x * sxy.x + sxy.y * sxy.y);
                 dcnt += 1;
                 v = vn;
             }
@@ -457,6 +460,7 @@ void fill_views(Args& a, const CamArgs* cams, const gs_projected* projs, const g
         w.fy = raw[v].fy;
         w.radius = projs[v].radius;
         w.g_xy = reinterpret_cast<const float2*>(g2d[v].xy);
+        w.g_xy_abs = reinterpret_cast<const float2*>(g2d[v].xy_abs);
         w.g_con = reinterpret_cast<const float4*>(g2d[v].conic_opacity);
         w.g_rgb = reinterpret_cast<const float4*>(g2d[v].rgb);
     }
@@ -495,6 +499,7 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
     a.densify_accum = densify_accum;
     a.densify_count = densify_count;
     a.densify_max_radius = densify_max_radius;
+    a.sparse = adam && adam->sparse;
     const unsigned grid = grid_for(p.n, kBwdBlock, 16);
     if (adam) {
         fill_grads(a.p_means, a.p_quats, a.p_log_scales, a.p_logits, a.p_sh, adam->params);

@@ -420,6 +420,7 @@ struct BwdArgs {
     float2* g_xy;
     float4* g_con;
     float4* g_rgb;
+    float2* g_xy_abs;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv| (kAbs only)
 };
 
 // Sum 9 per-lane values over the warp and add them to the Gaussian's three
@@ -469,6 +470,7 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
     if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
+template <bool kAbs>
 __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_bwd_kernel(const BwdArgs a) {
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -574,6 +576,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             if (__any_sync(kFull, any)) {
                 const float s0 = nmo.x + nmo.y, mo = -s0, m1 = s1.x + s1.y;
                 float du, dv;
+                float au = 0.f, av = 0.f;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv|
                 if (pb.w == kFactored) {
                     // dsigma/du = A t, dsigma/dv = B t + D dy
                     f2 st = zero;
@@ -582,6 +585,15 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                     const float stt = st.x + st.y;
                     du = con.x * stt;
                     dv = fmaf(con.y, stt, pb.z * m1);
+                    if (kAbs) {
+#pragma unroll
+                        for (int p = 0; p < kPairs; ++p) {
+                            const f2 pu = mul2(nm[p], mul2(splat(con.x), r.t[p]));
+                            const f2 pv = mul2(nm[p], fma2(splat(con.y), r.t[p], mul2(splat(pb.z), r.dy[p])));
+                            au += fabsf(pu.x) + fabsf(pu.y);
+                            av += fabsf(pv.x) + fabsf(pv.y);
+                        }
+                    }
                 } else if (pb.w == kDouble) {
                     // not positive definite: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
                     const double dxd = __dsub_rn(double(pa.x), double(px));
@@ -594,14 +606,37 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                         const float qi = i & 1 ? nm[i / 2].y : nm[i / 2].x;
                         du = fmaf(qi, su, du);
                         dv = fmaf(qi, sv, dv);
+                        if (kAbs) {
+                            au += fabsf(qi * su);
+                            av += fabsf(qi * sv);
+                        }
                     }
                 } else {
                     du = fmaf(con.x * r.dx, s0, con.y * m1);
                     dv = fmaf(con.y * r.dx, s0, con.z * m1);
+                    if (kAbs) {
+                        // per pixel dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy
+                        const f2 adx = splat(con.x * r.dx), bdx = splat(con.y * r.dx);
+#pragma unroll
+                        for (int p = 0; p < kPairs; ++p) {
+                            const f2 pu = mul2(nm[p], fma2(splat(con.y), r.dy[p], adx));
+                            const f2 pv = mul2(nm[p], fma2(splat(con.z), r.dy[p], bdx));
+                            au += fabsf(pu.x) + fabsf(pu.y);
+                            av += fabsf(pv.x) + fabsf(pv.y);
+                        }
+                    }
                 }
                 float v[8] = {du, dv, 0.5f * r.dx * r.dx * s0, r.dx * m1, 0.5f * (s2.x + s2.y), mo * pa.w,
                               -(ndr.x + ndr.y), -(ndg.x + ndg.y)};
                 warp_reduce_and_add(v, -(ndb.x + ndb.y), lane, S.gid[buf][j], a);
+                if (kAbs) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        au += __shfl_xor_sync(kFull, au, o);
+                        av += __shfl_xor_sync(kFull, av, o);
+                    }
+                    if (lane == 3) atomicAdd(a.g_xy_abs + S.gid[buf][j], make_float2(au, av));
+                }
             }
         }
         __syncwarp();
@@ -694,7 +729,12 @@ cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, co
     a.g_xy = reinterpret_cast<float2*>(g2.xy);
     a.g_con = reinterpret_cast<float4*>(g2.conic_opacity);
     a.g_rgb = reinterpret_cast<float4*>(g2.rgb);
-    raster_bwd_kernel<<<unsigned((a.tiles * kSub + kWarps - 1) / kWarps), kWarps * 32, 0, s>>>(a);
+    a.g_xy_abs = reinterpret_cast<float2*>(g2.xy_abs);
+    const unsigned grid = unsigned((a.tiles * kSub + kWarps - 1) / kWarps);
+    if (a.g_xy_abs)
+        raster_bwd_kernel<true><<<grid, kWarps * 32, 0, s>>>(a);
+    else
+        raster_bwd_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }

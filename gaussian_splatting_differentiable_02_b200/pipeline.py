@@ -128,20 +128,24 @@ class Projected:
 
 
 class Grad2D:
-    def __init__(self, n: int, device="cuda"):
+    """2D gradients of one view; absgrad=True also keeps the absolute gradient xy_abs."""
+
+    def __init__(self, n: int, device="cuda", absgrad: bool = False):
         f = dict(device=device, dtype=torch.float32)
         n = max(n, 1)
         self.xy = torch.zeros((n, 2), **f)
         self.conic_opacity = torch.zeros((n, 4), **f)
         self.rgb = torch.zeros((n, 4), **f)
+        self.xy_abs = torch.zeros((n, 2), **f) if absgrad else None
 
     def struct(self) -> abi.gs_grad2d:
-        return abi.gs_grad2d(_ptr(self.xy), _ptr(self.conic_opacity), _ptr(self.rgb))
+        return abi.gs_grad2d(_ptr(self.xy), _ptr(self.conic_opacity), _ptr(self.rgb), _ptr(self.xy_abs))
 
     def zero_(self):
         s = _stream()
-        for t in (self.xy, self.conic_opacity, self.rgb):
-            abi.gs_zero(_ptr(t), t.numel() * 4, s)
+        for t in (self.xy, self.conic_opacity, self.rgb, self.xy_abs):
+            if t is not None:
+                abi.gs_zero(_ptr(t), t.numel() * 4, s)
 
     def as_rows(self) -> np.ndarray:
         """[n, 9]: u, v, A, B, C, o, r, g, b (the oracle's order)."""
@@ -258,14 +262,16 @@ def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: d
 def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: torch.Tensor, grad2ds: list,
                            m: Gaussians, v: Gaussians, lrs: dict, step: int, grads: Gaussians = None,
                            densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
-                           betas=(0.9, 0.99), eps=1e-15, densify_max_radius: torch.Tensor = None):
+                           betas=(0.9, 0.99), eps=1e-15, densify_max_radius: torch.Tensor = None,
+                           sparse: bool = False):
     """Backward through the projection for all views (each with its own radius row and 2D
-    gradients) with the Adam step of all five groups fused in."""
+    gradients) with the Adam step of all five groups fused in; sparse=True leaves Gaussians
+    visible in no view untouched (the gsplat guide §4.1 sparse_grad option)."""
     abi.gs_project_bwd_views_adam(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES],
         betas[0], betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum),
-        _ptr(densify_count), _ptr(densify_max_radius), _stream())
+        _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
 # densify_and_prune parameters of the gsplat guide §4.1 (every 100 steps): gradient
@@ -323,6 +329,10 @@ class Trainer:
     densify: bool = False
     fused: bool = True
     ssim_weight: float = 0.0   # > 0: L1 + ssim_weight * (1 - SSIM) (the gsplat guide §4.1 uses 0.2)
+    absgrad: bool = False      # densify on the absolute 2D gradient (the gsplat guide §4.1 absgrad option)
+    sparse_grad: bool = False  # Adam skips Gaussians seen in no view of the step (sparse_grad option; fused only)
+    streams: int = 2           # fused path: views alternate over this many CUDA streams, so that one
+                               # view's projection and sort overlap another view's compositing
 
     def __post_init__(self):
         n = self.gauss.n
@@ -343,7 +353,10 @@ class Trainer:
         dev = self.gauss.means.device
         nv = len(self.views) if self.fused else 1
         self.proj = Projected(n, dev)
-        self.grad2ds = [Grad2D(n, dev) for _ in range(nv)]
+        # concurrent views need their own projected features
+        self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
+            if self.fused else [self.proj]
+        self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
         self.grad2d = self.grad2ds[0]
         self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
         self.grads = None if self.fused else self.gauss.zeros_like()
@@ -373,24 +386,51 @@ class Trainer:
         self._alloc_per_gaussian(g.n)
         return decision
 
-    def view_forward_backward(self, k: int, target: torch.Tensor) -> None:
-        """project -> sort -> raster forward -> L1 -> raster backward of view k.
-        The fused path sorts without waiting (instance count checked once per step)."""
+    def view_forward_backward(self, k: int, target: torch.Tensor, proj: Projected = None) -> None:
+        """project -> sort -> raster forward -> L1 -> raster backward of view k (on the
+        current stream).  The fused path sorts without waiting (instance count checked
+        once per step)."""
         view = self.views[k]
+        proj = self.proj if proj is None else proj
         r = self.radii[k if self.fused else 0]
         g2 = self.grad2ds[k if self.fused else 0]
-        project(self.gauss, view, self.proj, r)
+        project(self.gauss, view, proj, r)
         if self.fused:
-            bin_sort_async(self.proj, view, self.kcount[k:k + 1], r)
+            bin_sort_async(proj, view, self.kcount[k:k + 1], r)
         else:
-            bin_sort(self.proj, view, r)
-        raster_fwd(self.proj, view, self.bg, r)
+            bin_sort(proj, view, r)
+        raster_fwd(proj, view, self.bg, r)
         if self.ssim_weight > 0.0:
             l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
         else:
             l1_loss_grad(view, target, self.loss)
         g2.zero_()
-        raster_bwd(self.proj, view, g2, self.bg, radius=r)
+        raster_bwd(proj, view, g2, self.bg, radius=r)
+
+    def _all_views(self) -> None:
+        """Every view's forward and backward; in the fused path view k runs on stream
+        k mod `streams` (each with its own projected features), joined before return."""
+        if not self.fused or len(self.projs) == 1:
+            for k, tgt in enumerate(self.targets):
+                self.view_forward_backward(k, tgt)
+            return
+        main = torch.cuda.current_stream()
+        side = self.side_streams()
+        start = main.record_event()
+        for st in side:
+            st.wait_event(start)
+        for k, tgt in enumerate(self.targets):
+            j = k % len(side)
+            with torch.cuda.stream(side[j]):
+                self.view_forward_backward(k, tgt, self.projs[j])
+        for st in side:
+            main.wait_stream(st)
+
+    def side_streams(self) -> list:
+        """The streams the fused path runs views on (one per projected-feature buffer)."""
+        if getattr(self, "_side", None) is None:
+            self._side = [torch.cuda.Stream(device=self.gauss.means.device) for _ in self.projs]
+        return self._side
 
     def step(self) -> None:
         """forward + L1 + backward for every view, then one Adam step; loss stays on the device."""
@@ -399,13 +439,12 @@ class Trainer:
             abi.gs_zero(_ptr(self.loss), 8, s)
             if not self.fused:
                 self.grads.zero_()
-            for k, tgt in enumerate(self.targets):
-                self.view_forward_backward(k, tgt)
-                if not self.fused:
+                for k, tgt in enumerate(self.targets):
+                    self.view_forward_backward(k, tgt)
                     project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
                                 self.densify_count, radius=self.radii[0], densify_max_radius=self.densify_max_radius)
-            if not self.fused:
                 break
+            self._all_views()
             # one wait per step: every view's instance count against its capacity
             counts = self.kcount.cpu().tolist()
             over = [k for k, K in enumerate(counts) if K > self.views[k].capacity]
@@ -419,6 +458,6 @@ class Trainer:
         if self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
                                    self.lrs, self.step_count, None, self.densify_accum, self.densify_count,
-                                   densify_max_radius=self.densify_max_radius)
+                                   densify_max_radius=self.densify_max_radius, sparse=self.sparse_grad)
         else:
             adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)

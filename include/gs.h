@@ -118,11 +118,18 @@ typedef struct gs_projected {
 /* Gradients with respect to the projected features, written by gs_raster_bwd (+=):
  *   xy            [n][2]  dL/du, dL/dv                              (8-byte aligned)
  *   conic_opacity [n][4]  dL/dA, dL/dB, dL/dC, dL/do                (16-byte aligned)
- *   rgb           [n][4]  dL/dr, dL/dg, dL/db, 0                    (16-byte aligned) */
+ *   rgb           [n][4]  dL/dr, dL/dg, dL/db, 0                    (16-byte aligned)
+ *   xy_abs        [n][2]  NULL, or the absolute gradient (the absgrad option of
+ *                         the gsplat guide §4.1): the sum over pixels of the
+ *                         absolute value of each pixel's contribution to dL/du
+ *                         and to dL/dv                               (8-byte aligned)
+ * When xy_abs is set, the densification statistic of the backward calls
+ * through the projection accumulates |xy_abs| instead of |xy|. */
 typedef struct gs_grad2d {
     float* xy;
     float* conic_opacity;
     float* rgb;
+    float* xy_abs;
 } gs_grad2d;
 
 /* Text for a status code (static storage). */
@@ -278,14 +285,18 @@ gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const
  * eps and step).  params_inout holds the same arrays as params and is updated
  * in place; adam_m and adam_v are the first and second moments in the
  * parameter layout.  The summed gradient goes straight into Adam; grads, when
- * non-NULL, also receives it (+=).  Every Gaussian is updated, visible or not,
- * as gs_adam updates every element. */
+ * non-NULL, also receives it (+=).  With sparse_adam = 0 every Gaussian is
+ * updated, visible or not, as gs_adam updates every element.  With
+ * sparse_adam = 1 (the sparse_grad option of the gsplat guide §4.1) a Gaussian
+ * visible in none of the views keeps its parameters and moments unchanged (no
+ * decay of the moments), as a sparse Adam skips absent rows; the bias
+ * correction still uses `step`. */
 gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
                                     const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
                                     gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
                                     float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
                                     float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
-                                    void* stream);
+                                    int32_t sparse_adam, void* stream);
 
 /* Adaptive density control (gsplat guide §4.1: every 100 steps,
  * densify_and_prune with a gradient threshold of 0.0002, a minimum opacity of

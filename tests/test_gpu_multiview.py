@@ -71,8 +71,8 @@ def test_views_equal_sum_of_single_view_chains(orc):
     da = torch.zeros(scene.n, device="cuda")
     dc = torch.zeros(scene.n, dtype=torch.int32, device="cuda")
     abi.gs_project_bwd_views(g.params(), [v.gcam for v in views], [proj.struct(radii[k]) for k in range(len(views))],
-                             [x.struct() for x in g2s], grads.grads(), da.data_ptr(), dc.data_ptr(),
-                             torch.cuda.current_stream().cuda_stream)
+                             [x.struct() for x in g2s], grads.grads(), densify_accum=da.data_ptr(),
+                             densify_count=dc.data_ptr(), stream=torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     got = grads.to_numpy()
     vis = np.nonzero(cnt > 0)[0]
@@ -99,8 +99,8 @@ def test_fused_adam_matches_oracle_adam_of_summed_gradients(orc, deg):
     lrs = [float(np.float32(LRS[k])) for k in NAMES]
     abi.gs_project_bwd_views_adam(g.params(), [vw.gcam for vw in views],
                                   [proj.struct(radii[k]) for k in range(len(views))], [x.struct() for x in g2s],
-                                  g.grads(), m.grads(), v.grads(), lrs, b1, b2, eps, step, grads.grads(), 0, 0,
-                                  torch.cuda.current_stream().cuda_stream)
+                                  g.grads(), m.grads(), v.grads(), lrs, b1, b2, eps, step, grads=grads.grads(),
+                                  stream=torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     # the summed gradient it applied
     got_g = grads.to_numpy()
@@ -185,3 +185,53 @@ def test_trainer_fused_equals_unfused():
         close = d <= 1e-6 + 1e-6 * np.abs(a[k])
         assert close.mean() >= 0.999, (k, float(close.mean()))
         assert d.max() <= 4 * LRS[k] + 1e-6, (k, float(d.max()))
+
+
+def test_sparse_adam_skips_gaussians_seen_in_no_view():
+    """sparse_adam = 1: Gaussians visible in no view keep parameters and moments bit for
+    bit; every other Gaussian gets exactly the dense update (same inputs, same arithmetic)."""
+    rng = np.random.default_rng(41)
+    scene = scenes.random_scene(rng, 700, 1, mean_box=1.0, log_scale=(-4.0, -2.0))
+    scene.means[:120] += 40.0   # far outside every view
+    cams = _views(3, 6)
+    views = [pl.View(scene.n, c) for c in cams]
+    g = pl.Gaussians.from_scene(scene)
+    proj = pl.Projected(scene.n)
+    radii = torch.zeros((len(cams), scene.n), dtype=torch.int32, device="cuda")
+    g2s = []
+    for k, vw in enumerate(views):
+        pl.project(g, vw, proj, radii[k])
+        pl.bin_sort(proj, vw, radii[k])
+        pl.raster_fwd(proj, vw, radius=radii[k])
+        vw.dL_dimage.copy_(torch.from_numpy(rng.standard_normal(tuple(vw.dL_dimage.shape)).astype(np.float32)))
+        gd = pl.Grad2D(scene.n)
+        pl.raster_bwd(proj, vw, gd, radius=radii[k])
+        g2s.append(gd)
+    torch.cuda.synchronize()
+    vis = (radii.cpu().numpy() > 0).any(axis=0)
+    assert not vis[:120].any() and vis.sum() > 400
+    m0 = g.zeros_like()
+    v0 = g.zeros_like()
+    for t in list(m0.tensors().values()) + list(v0.tensors().values()):
+        t.copy_(torch.from_numpy((0.01 * rng.random(tuple(t.shape))).astype(np.float32)))
+    out = []
+    for sparse in (False, True):
+        gg = pl.Gaussians.from_scene(scene)
+        m, v = gg.zeros_like(), gg.zeros_like()
+        for a, b in zip(list(m.tensors().values()) + list(v.tensors().values()),
+                        list(m0.tensors().values()) + list(v0.tensors().values())):
+            a.copy_(b)
+        pl.project_bwd_views_adam(gg, views, proj, radii, g2s, m, v, LRS, 2, sparse=sparse)
+        torch.cuda.synchronize()
+        out.append([{k: getattr(x, k).cpu().numpy() for k in NAMES} for x in (gg, m, v)])
+    g_init = {k: getattr(g, k).cpu().numpy() for k in NAMES}
+    init = [g_init, {k: getattr(m0, k).cpu().numpy() for k in NAMES}, {k: getattr(v0, k).cpu().numpy() for k in NAMES}]
+    for dense, sparse, before in zip(out[0], out[1], init):
+        for k in NAMES:
+            d, s, b = dense[k], sparse[k], before[k]
+            if k == "sh":   # [P][n][4]
+                d, s, b = (np.moveaxis(x, 1, 0) for x in (d, s, b))
+            assert np.array_equal(s[vis], d[vis]), k
+            assert np.array_equal(s[~vis], b[~vis]), k
+    # the dense step did move the unseen Gaussians' moments (they decay)
+    assert not np.array_equal(out[0][1]["means"][~vis], init[1]["means"][~vis])
