@@ -286,12 +286,14 @@ def run_ours(args, world, rank, local):
             "project_bwd_adam": pl.project_bwd_views_adam, "project": pl.project}
 
     def wrap(fn):
+        # events on the stream the kernel is launched on (the Trainer spreads views over streams)
         def inner(*a, **k):
+            st = torch.cuda.current_stream()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+            e0.record(st)
             fn(*a, **k)
-            e1.record(stream)
+            e1.record(st)
             ev_dom.append((e0, e1))
         return inner
 

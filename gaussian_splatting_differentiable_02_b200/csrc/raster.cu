@@ -103,10 +103,11 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Per-warp staging area: raw gathered features (double-buffered) and the
 // per-entry constants derived from them.
 // Evaluation of an entry (WarpStage::pb.w).
-constexpr float kPlain = 0.f;     // expanded quadratic form in float32
-constexpr float kDouble = 1.f;    // quadratic form in double (a conic that is not positive definite)
-constexpr float kSkip = 2.f;      // misses every pixel of the warp's box
-constexpr float kFactored = 3.f;  // factored form 1/2 A t^2 + 1/2 D dy^2 in float32
+constexpr float kPlain = 0.f;          // expanded quadratic form in float32
+constexpr float kSkip = 2.f;           // misses every pixel of the warp's box
+constexpr float kFactored = 3.f;       // factored form 1/2 A t^2 + 1/2 D dy^2 in float32 (D > 0)
+constexpr float kFactoredIndef = 4.f;  // the same with D <= 0 (a float32 conic that rounded to indefinite):
+                                       // sigma can be negative, and such pixels are skipped
 
 struct WarpStage {
     float2 xy[2][kBatch];
@@ -154,12 +155,12 @@ __device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by
 }
 
 // Lane l < count derives the constants of staged entry l.  pb.w selects the
-// evaluation (kPlain, kFactored, kDouble) or kSkip: the smallest sigma over
+// evaluation (kPlain, kFactored, kFactoredIndef) or kSkip: the smallest sigma over
 // this warp's pixel box [bx0, bx0 + kBoxW - 1] x [by0, by0 + kBoxH - 1] (pixel
 // centres) puts alpha below 1/255 everywhere in it, with a margin far above
 // the rounding of either evaluation, so no pixel of the warp would blend it.
 // The bound is computed in float32 for well-conditioned conics and in double
-// for the others.
+// for the others (never for an indefinite one).
 template <bool kNegRgb>
 __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
     if (lane < count) {
@@ -185,16 +186,21 @@ __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane,
                              flag);
         } else {
             const double A = c.x, B = c.y, C = c.z;
-            const double D = (A * C - B * B) / A;  // A C and B^2 are exact in double
-            if (A > 0.0 && D > 0.0) {
-                const double smin = box_min<double>(A, B, C, xy.x, xy.y, bx0, bx1, by0, by1);
+            if (A > 0.0) {
+                const double D = (A * C - B * B) / A;  // A C and B^2 are exact in double
                 const double r = B / A;
                 const float rh = __double2float_rn(r);
-                pb = make_float4(rh, __double2float_rn(r - double(rh)), float(D),
-                                 smin * (1.0 - 1e-4) > double(cut) + 1e-4 ? kSkip : kFactored);
+                float flag = kFactoredIndef;
+                if (D > 0.0) {
+                    const double smin = box_min<double>(A, B, C, xy.x, xy.y, bx0, bx1, by0, by1);
+                    flag = smin * (1.0 - 1e-4) > double(cut) + 1e-4 ? kSkip : kFactored;
+                }
+                pb = make_float4(rh, __double2float_rn(r - double(rh)), float(D), flag);
                 pc = make_float2(__double2float_rn(-0.5 * kLog2eD * A), __double2float_rn(-0.5 * kLog2eD * D));
             } else {
-                pb = make_float4(0.f, 0.f, 0.f, kDouble);
+                // A = Sigma'_yy / det > 0 for every conic the projection writes; a
+                // non-positive one has no meaningful footprint
+                pb = make_float4(0.f, 0.f, 0.f, kSkip);
             }
         }
         S.pa[lane] = make_float4(xy.x, xy.y, lo, 1.f / c.w);
@@ -239,39 +245,19 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
     r.blend = 0u;
     r.clamp = 0u;
     const f2 vy = splat(pa.y), lo = splat(pa.z);
-    if (pb.w == kFactored) {
+    if (pb.w >= kFactored) {
+        const bool indef = pb.w == kFactoredIndef;
         r.dx = __fsub_rn(pa.x, px);
         const f2 dx2 = splat(r.dx), rh = splat(pb.x), rl = splat(pb.y), ka = splat(pc.x), kd = splat(pc.y);
 #pragma unroll
         for (int p = 0; p < kPairs; ++p) {
             r.dy[p] = add2(vy, nyc[p]);
             r.t[p] = fma2(rl, r.dy[p], fma2(rh, r.dy[p], dx2));
-            const f2 e = add2(fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p])), lo);
-            alpha_at(e.x, true, 2 * p, r.nal[p].x, r.blend, r.clamp);  // sigma >= 0 by construction
-            alpha_at(e.y, true, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
-        }
-    } else if (pb.w == kDouble) {
-        const double dxd = __dsub_rn(double(pa.x), double(px));
-        r.dx = __double2float_rn(dxd);
-        const double A = con.x, B = con.y, C = con.z;
-        const double adx2 = __dmul_rn(__dmul_rn(A, dxd), dxd);
-        const double bdx = __dmul_rn(B, dxd);
-#pragma unroll
-        for (int i = 0; i < kPx; ++i) {
-            const double dyd = __dsub_rn(double(pa.y), -double(i & 1 ? nyc[i / 2].y : nyc[i / 2].x));
-            const double sig = __dadd_rn(__dmul_rn(0.5, __dadd_rn(adx2, __dmul_rn(__dmul_rn(C, dyd), dyd))),
-                                         __dmul_rn(bdx, dyd));
-            const float sv = __double2float_rn(__dmul_rn(-sig, kLog2eD));
-            const float dyf = __double2float_rn(dyd);
-            float nal;
-            alpha_at(__fadd_rn(sv, pa.z), sv <= 0.f, i, nal, r.blend, r.clamp);
-            if (i & 1) {
-                r.dy[i / 2].y = dyf;
-                r.nal[i / 2].y = nal;
-            } else {
-                r.dy[i / 2].x = dyf;
-                r.nal[i / 2].x = nal;
-            }
+            const f2 sv = fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p]));
+            const f2 e = add2(sv, lo);
+            // sigma >= 0 by construction unless the conic is indefinite
+            alpha_at(e.x, !indef || sv.x <= 0.f, 2 * p, r.nal[p].x, r.blend, r.clamp);
+            alpha_at(e.y, !indef || sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
         }
     } else {
         r.dx = __fsub_rn(pa.x, px);
@@ -577,7 +563,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                 const float s0 = nmo.x + nmo.y, mo = -s0, m1 = s1.x + s1.y;
                 float du, dv;
                 float au = 0.f, av = 0.f;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv|
-                if (pb.w == kFactored) {
+                if (pb.w >= kFactored) {
                     // dsigma/du = A t, dsigma/dv = B t + D dy
                     f2 st = zero;
 #pragma unroll
@@ -592,23 +578,6 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                             const f2 pv = mul2(nm[p], fma2(splat(con.y), r.t[p], mul2(splat(pb.z), r.dy[p])));
                             au += fabsf(pu.x) + fabsf(pu.y);
                             av += fabsf(pv.x) + fabsf(pv.y);
-                        }
-                    }
-                } else if (pb.w == kDouble) {
-                    // not positive definite: dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy per pixel in double
-                    const double dxd = __dsub_rn(double(pa.x), double(px));
-                    du = dv = 0.f;
-#pragma unroll
-                    for (int i = 0; i < kPx; ++i) {
-                        const double dyd = __dsub_rn(double(pa.y), -double(i & 1 ? nyc[i / 2].y : nyc[i / 2].x));
-                        const float su = __double2float_rn(double(con.x) * dxd + double(con.y) * dyd);
-                        const float sv = __double2float_rn(double(con.y) * dxd + double(con.z) * dyd);
-                        const float qi = i & 1 ? nm[i / 2].y : nm[i / 2].x;
-                        du = fmaf(qi, su, du);
-                        dv = fmaf(qi, sv, dv);
-                        if (kAbs) {
-                            au += fabsf(qi * su);
-                            av += fabsf(qi * sv);
                         }
                     }
                 } else {

@@ -65,7 +65,9 @@ def test_identical_images_give_zero():
     img = rng.random((45, 61, 3)).astype(np.float32)
     loss, g = _gpu(img, img)
     assert loss == 0.0
-    assert np.all(g == 0.0)
+    # the partial derivative with respect to the windowed mean cancels to rounding
+    # (four terms summed in order), so the gradient is zero up to that
+    assert np.max(np.abs(g)) < 1e-15
 
 
 def test_full_hd_rendered_image(orc):

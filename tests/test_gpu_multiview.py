@@ -235,3 +235,31 @@ def test_sparse_adam_skips_gaussians_seen_in_no_view():
             assert np.array_equal(s[~vis], b[~vis]), k
     # the dense step did move the unseen Gaussians' moments (they decay)
     assert not np.array_equal(out[0][1]["means"][~vis], init[1]["means"][~vis])
+
+
+def test_trainer_two_streams_equals_one():
+    """Views spread over two CUDA streams (each with its own projected features) give
+    the step of the single-stream order: same losses, counts and parameters up to the
+    order of the atomic adds."""
+    rng = np.random.default_rng(13)
+    scene = scenes.random_scene(rng, 600, 1, mean_box=1.0, log_scale=(-3.5, -2.0))
+    cams = _views(5, 8)
+    targets = [torch.from_numpy(rng.random((128, 128, 3)).astype(np.float32)).cuda() for _ in cams]
+    out = []
+    for streams in (1, 2):
+        g = pl.Gaussians.from_scene(scene)
+        tr = pl.Trainer(g, [pl.View(scene.n, c) for c in cams], targets, dict(LRS), densify=True, streams=streams)
+        assert len(tr.projs) == streams
+        tr.step()   # the first step starts from identical parameters: counts and K agree exactly
+        torch.cuda.synchronize()
+        first = (tr.loss.item(), tr.densify_count.cpu().numpy(), tr.kcount.cpu().numpy())
+        tr.step()
+        tr.step()
+        torch.cuda.synchronize()
+        out.append((tr.gauss.to_numpy(), first))
+    (a, (la, ca, ka)), (b, (lb, cb, kb)) = out
+    assert np.array_equal(ca, cb) and np.array_equal(ka, kb)
+    assert abs(la - lb) <= 1e-9 * abs(la)
+    for k in NAMES:
+        close = np.abs(a[k] - b[k]) <= 1e-6 + 1e-5 * np.abs(a[k])
+        assert close.mean() >= 0.999, (k, float(close.mean()))

@@ -242,3 +242,48 @@ def test_opaque_stack_terminates_early(orc):
     gi, gT, gn = run.images()
     centre = 64 * 128 + 64
     assert 0 < gn[centre] < 10 and gT[centre] >= 1e-4
+
+
+def test_needle_and_indefinite_conics(orc):
+    """Conics written straight into the projected features (the rectangles and the
+    sort stay those of the projection): needles with eigenvalue ratios up to 1e6 take
+    the factored float32 evaluation, and conics that are indefinite in float32 (which
+    the projection never writes) blend only where sigma >= 0, as the oracle's direct
+    evaluation does."""
+    wl = scenes.tiny()
+    cam = wl.cameras[0]
+    run = GpuRun(wl.scene, cam)
+    p = run.projection()
+    vis = np.argsort(-p["radius"])[:12]   # the largest footprints
+    assert np.all(p["radius"][vis] > 4)
+    con = run.proj.conic_opacity.cpu().numpy()
+    rng = np.random.default_rng(5)
+    for k, i in enumerate(vis[:12]):
+        A = np.float32(rng.uniform(0.05, 0.5))
+        ang = rng.uniform(0, np.pi)
+        if k < 8:   # needle: eigenvalues A and A / kappa, rotated
+            kappa = 10.0 ** rng.uniform(2, 6)
+            l1, l2 = A, A / kappa
+        else:       # indefinite
+            l1, l2 = A, -A / 50
+        c, s = np.cos(ang), np.sin(ang)
+        con[i, 0] = l1 * c * c + l2 * s * s
+        con[i, 1] = (l1 - l2) * c * s
+        con[i, 2] = l1 * s * s + l2 * c * c
+        con[i, 3] = 0.9
+    run.proj.conic_opacity.copy_(torch.from_numpy(con))
+    pl.raster_fwd(run.proj, run.view, run.bg)
+    torch.cuda.synchronize()
+    # the oracle composites exactly the features the kernels see
+    ref = {k: np.asarray(v, np.float64) if v.dtype.kind == "f" else v for k, v in run.projection().items()}
+    img, T, nc, amb = orc.render(ref, cam, band_alpha=BAND_ALPHA, band_T=BAND_T)
+    gi, gT, gn = run.images()
+    check_images(gi, gT, gn, img, T, nc, amb, max_amb_frac=0.01)
+    # and the backward agrees on the same features
+    up = wl.upstream[0]
+    g2_gpu = run.backward(up)
+    g2, g2a, touched = orc.render_bwd(ref, cam, up.reshape(-1, 3).astype(np.float64), band_alpha=BAND_ALPHA,
+                                      band_T=BAND_T)
+    rows = np.nonzero(touched == 0)[0]
+    for q, name in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
+        check_grads(g2_gpu[:, q], g2[:, q], name, rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.002)
