@@ -268,7 +268,7 @@ def run_ours(args, world, rank, local):
     targets = targets_host.cuda() if targets_host is not None else None
     lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
                                                   "opacity_logits": 5e-2, "sh": 2.5e-3}
-    tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True)
+    tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams)
     stream = torch.cuda.current_stream()
 
     # warm-up (also sizes every view's instance buffers)
@@ -341,7 +341,7 @@ def run_ours(args, world, rank, local):
     line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv,
+            "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -715,6 +715,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["multiview", "mixture", "box", "city", "tiny"], default="multiview")
     ap.add_argument("--cpu-fraction", type=float, default=1.0 / 256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--streams", type=int, default=2,
+                    help="CUDA streams the views of a step alternate over (1 = serial)")
     ap.add_argument("--views", type=int, default=16,
                     help="views per step of the multiview workload (fewer: the first poses of the 16; "
                          "for small profiler captures, not a bench line)")

@@ -278,7 +278,9 @@ def test_needle_and_indefinite_conics(orc):
     ref = {k: np.asarray(v, np.float64) if v.dtype.kind == "f" else v for k, v in run.projection().items()}
     img, T, nc, amb = orc.render(ref, cam, band_alpha=BAND_ALPHA, band_T=BAND_T)
     gi, gT, gn = run.images()
-    check_images(gi, gT, gn, img, T, nc, amb, max_amb_frac=0.01)
+    # an indefinite form is zero along two lines through the mean, where sigma changes
+    # sign: the pixels near them are ambiguous by construction (excluded, counted)
+    check_images(gi, gT, gn, img, T, nc, amb, max_amb_frac=0.08)
     # and the backward agrees on the same features
     up = wl.upstream[0]
     g2_gpu = run.backward(up)

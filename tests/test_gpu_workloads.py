@@ -7,13 +7,14 @@ workloads, in the launch configuration the benchmark uses:
     random tiles) for the forward pass,
   * the backward pass for an upstream gradient that is N(0,1) on those sampled
     pixels and zero elsewhere, so that every Gaussian's 2D gradient is a sum the
-    oracle computes exactly,
+    oracle computes exactly, with and without the absolute 2D gradient (absgrad),
   * project_bwd on a sample of Gaussians from random 2D gradients.
 """
 import numpy as np
 import pytest
 import torch
 
+from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 from gaussian_splatting_differentiable_02_b200 import scenes
 
 from _parity import (BAND_ALPHA, BAND_T, GpuRun, check_grads, check_images, check_projection)
@@ -92,6 +93,14 @@ def test_workload_parity(orc, workload):
         assert len(rows) > 50
         for q, qn in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
             check_grads(g2_gpu[:, q], g2[:, q], f"{name}:{qn}", rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.003)
+        # the absolute 2D gradient: sums of |per-pixel terms|, no cancellation allowance needed
+        g2abs = pl.Grad2D(scene.n, absgrad=True)
+        pl.raster_bwd(run.proj, run.view, g2abs, run.bg)
+        torch.cuda.synchronize()
+        xa = g2abs.xy_abs.cpu().numpy()
+        check_grads(xa[:, 0], g2a[:, 0], f"{name}:|du|", rows=rows)
+        check_grads(xa[:, 1], g2a[:, 1], f"{name}:|dv|", rows=rows)
+        del g2abs
 
         # project_bwd on a sample of visible Gaussians from random 2D gradients
         vis = np.nonzero(ref["radius"] > 0)[0]
