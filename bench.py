@@ -715,7 +715,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["multiview", "mixture", "box", "city", "tiny"], default="multiview")
     ap.add_argument("--cpu-fraction", type=float, default=1.0 / 256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--streams", type=int, default=2,
+    ap.add_argument("--streams", type=int, default=3,
                     help="CUDA streams the views of a step alternate over (1 = serial)")
     ap.add_argument("--views", type=int, default=16,
                     help="views per step of the multiview workload (fewer: the first poses of the 16; "

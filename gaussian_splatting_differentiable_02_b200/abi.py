@@ -12,6 +12,8 @@ from __future__ import annotations
 import ctypes as C
 import os
 
+import numpy as np
+
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgs.so")
 
@@ -139,8 +141,8 @@ def _check(status: int):
 def make_camera(cam: dict) -> gs_camera:
     """gs_camera from a scene camera dict (R 3x3 row-major, t, fx, fy, cx, cy, width, height, near, eps2d)."""
     c = gs_camera()
-    R = [float(v) for v in __import__("numpy").asarray(cam["R"], "float32").reshape(9)]
-    t = [float(v) for v in __import__("numpy").asarray(cam["t"], "float32").reshape(3)]
+    R = [float(v) for v in np.asarray(cam["R"], np.float32).reshape(9)]
+    t = [float(v) for v in np.asarray(cam["t"], np.float32).reshape(3)]
     for i in range(9):
         c.R[i] = R[i]
     for i in range(3):

@@ -36,7 +36,10 @@ namespace gsk {
 namespace {
 
 constexpr int kEmitBlock = 256;
-constexpr int kEmitPerThread = 8;
+#ifndef GS_EMIT_ITEMS
+#define GS_EMIT_ITEMS 2
+#endif
+constexpr int kEmitPerThread = GS_EMIT_ITEMS;
 constexpr int kEmitChunk = kEmitBlock * kEmitPerThread;  // Gaussians per emit block
 static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halves a power of two");
 

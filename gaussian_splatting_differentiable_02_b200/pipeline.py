@@ -331,7 +331,7 @@ class Trainer:
     ssim_weight: float = 0.0   # > 0: L1 + ssim_weight * (1 - SSIM) (the gsplat guide §4.1 uses 0.2)
     absgrad: bool = False      # densify on the absolute 2D gradient (the gsplat guide §4.1 absgrad option)
     sparse_grad: bool = False  # Adam skips Gaussians seen in no view of the step (sparse_grad option; fused only)
-    streams: int = 2           # fused path: views alternate over this many CUDA streams, so that one
+    streams: int = 3           # fused path: views alternate over this many CUDA streams, so that one
                                # view's projection and sort overlap another view's compositing
 
     def __post_init__(self):
