@@ -268,7 +268,8 @@ def run_ours(args, world, rank, local):
     targets = targets_host.cuda() if targets_host is not None else None
     lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
                                                   "opacity_logits": 5e-2, "sh": 2.5e-3}
-    tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams)
+    tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams,
+                    batched_sort=not args.per_view_sort)
     stream = torch.cuda.current_stream()
 
     # warm-up (also sizes every view's instance buffers)
@@ -342,6 +343,7 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
+                       "depth_sort": "per view" if args.per_view_sort else "batched over the views",
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -540,15 +542,24 @@ def stage_breakdown(tr, pl, torch):
         acc.setdefault(name, []).append((e0, e1))
         return r
 
+    batched = getattr(tr, "depth_order", None) is not None
+    if batched:   # the Trainer's order: every projection, one batched depth sort, then per view
+        for k, view in enumerate(tr.views):
+            timed("project", pl.project, tr.gauss, view, tr.projs[k], tr.radii[k])
+        timed("bin_sort", pl.depth_order_views, tr.projs, tr.radii, tr.depth_order)
     for k, (view, tgt) in enumerate(zip(tr.views, tr.targets)):
         r = tr.radii[k]
         g2 = tr.grad2ds[k]
-        timed("project", pl.project, tr.gauss, view, tr.proj, r)
-        timed("bin_sort", pl.bin_sort, tr.proj, view, r)
-        timed("raster_fwd", pl.raster_fwd, tr.proj, view, tr.bg, r)
+        proj = tr.projs[k] if batched else tr.proj
+        if batched:
+            timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.depth_order.order[k], tr.kcount[k:k + 1], r)
+        else:
+            timed("project", pl.project, tr.gauss, view, proj, r)
+            timed("bin_sort", pl.bin_sort, proj, view, r)
+        timed("raster_fwd", pl.raster_fwd, proj, view, tr.bg, r)
         timed("l1", pl.l1_loss_grad, view, tgt, tr.loss)
         g2.zero_()
-        timed("raster_bwd", pl.raster_bwd, tr.proj, view, g2, tr.bg, None, r)
+        timed("raster_bwd", pl.raster_bwd, proj, view, g2, tr.bg, None, r)
     tr.step_count += 1
     timed("project_bwd_adam", pl.project_bwd_views_adam, tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m,
           tr.v, tr.lrs, tr.step_count, None, tr.densify_accum, tr.densify_count,
@@ -664,12 +675,17 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
             for v in range(nbuf):
                 bufs[v].copy_(targets_host[v], non_blocking=True)
                 copy_events[v] = copy_stream.record_event()
+        batched = tr.depth_order is not None
+        if batched:
+            tr.project_and_order()
+            begin = stream.record_event()
         for v in range(nv):
             st = side[v % len(side)]
             st.wait_event(begin)
             st.wait_event(copy_events[v])
             with torch.cuda.stream(st):
-                tr.view_forward_backward(v, bufs[v % nbuf], tr.projs[v % len(side)])
+                tr.view_forward_backward(v, bufs[v % nbuf], tr.projs[v if batched else v % len(side)],
+                                         projected=batched)
             done[v].record(st)
             if v + nbuf < nv:
                 with torch.cuda.stream(copy_stream):
@@ -717,6 +733,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--streams", type=int, default=3,
                     help="CUDA streams the views of a step alternate over (1 = serial)")
+    ap.add_argument("--per-view-sort", action="store_true",
+                    help="sort each view on its own stream instead of one batched depth sort of all views")
     ap.add_argument("--views", type=int, default=16,
                     help="views per step of the multiview workload (fewer: the first poses of the 16; "
                          "for small profiler captures, not a bench line)")

@@ -83,6 +83,10 @@ SIGNATURES = {
                                        C.POINTER(C.c_int64), _P, _P]),
     "gs_bin_sort_async": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, C.POINTER(gs_camera), _P, C.c_size_t, _P, _P,
                                       C.c_int64, _P, _P, _P]),
+    "gs_depth_order_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int32]),
+    "gs_depth_order_views": (C.c_int32, [C.POINTER(gs_projected), C.c_int32, C.c_int64, _P, C.c_size_t, _P, _P]),
+    "gs_bin_sort_ordered_async": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, _P, C.POINTER(gs_camera), _P,
+                                              C.c_size_t, _P, _P, C.c_int64, _P, _P, _P]),
     "gs_tile_order": (C.c_int32, [_P, C.POINTER(gs_camera), _P, _P]),
     "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, _P]),
@@ -213,6 +217,25 @@ def gs_bin_sort_static(proj: gs_projected, n: int, cam: gs_camera, keys: int, va
     if check or st not in (GS_OK, GS_ERR_CAPACITY):
         _check(st)
     return st, K.value
+
+
+def gs_depth_order_workspace_bytes(n: int, num_views: int) -> int:
+    return lib().gs_depth_order_workspace_bytes(n, num_views)
+
+
+def gs_depth_order_views(projs, n: int, workspace: int, workspace_bytes: int, order: int, stream: int = 0):
+    """projs: a sequence of gs_projected (one per view); order: device [views][n] uint32."""
+    projs = list(projs)
+    return _check(lib().gs_depth_order_views(_arr(gs_projected, projs), len(projs), n, workspace, workspace_bytes,
+                                             order, stream))
+
+
+def gs_bin_sort_ordered_async(proj: gs_projected, n: int, order: int, cam: gs_camera, workspace: int,
+                              workspace_bytes: int, keys: int, vals: int, capacity: int, num_instances_dev: int,
+                              tile_ranges: int, stream: int = 0):
+    return _check(lib().gs_bin_sort_ordered_async(C.byref(proj), n, order or None, C.byref(cam), workspace,
+                                                  workspace_bytes, keys, vals, capacity, num_instances_dev,
+                                                  tile_ranges, stream))
 
 
 def gs_tile_order(tile_ranges: int, cam: gs_camera, tile_order: int, stream: int = 0):

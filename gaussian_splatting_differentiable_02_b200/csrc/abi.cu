@@ -182,7 +182,7 @@ namespace {
 gs_status bin_sort_impl(const char* fn, const gs_projected* proj, int64_t n, const gs_camera* cam, void* workspace,
                         size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
                         int64_t* num_instances_host, unsigned long long* count_dev, uint32_t* tile_ranges,
-                        void* stream) {
+                        void* stream, const uint32_t* order = nullptr) {
     gs_status st;
     if (n < 0 || n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n out of range", fn);
     if (capacity < 0 || capacity > 0xffffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: capacity out of range", fn);
@@ -205,7 +205,9 @@ gs_status bin_sort_impl(const char* fn, const gs_projected* proj, int64_t n, con
     gsk::SortWorkspace ws;
     gsk::sort_workspace_layout(n, capacity, workspace, &ws);
     const gsk::CamArgs c = gsk::make_cam(*cam);
-    cudaError_t e = gsk::launch_bin_sort(*proj, n, c, ws, keys, vals, capacity, tile_ranges, count_dev, s);
+    cudaError_t e = order ? gsk::launch_bin_sort_ordered(*proj, n, order, c, ws, keys, vals, capacity, tile_ranges,
+                                                         count_dev, s)
+                          : gsk::launch_bin_sort(*proj, n, c, ws, keys, vals, capacity, tile_ranges, count_dev, s);
     if (e != cudaSuccess) return cuda_status(e, fn);
     if (!num_instances_host) return ok();
     unsigned long long K = 0;
@@ -236,6 +238,48 @@ gs_status gs_bin_sort_async(const gs_projected* proj, int64_t n, const gs_camera
     if (!num_instances_dev) return fail(GS_ERR_INVALID_ARG, "gs_bin_sort_async: num_instances_dev is NULL");
     return bin_sort_impl("gs_bin_sort_async", proj, n, cam, workspace, workspace_bytes, keys, vals, capacity,
                          nullptr, reinterpret_cast<unsigned long long*>(num_instances_dev), tile_ranges, stream);
+}
+
+gs_status gs_bin_sort_ordered_async(const gs_projected* proj, int64_t n, const uint32_t* order, const gs_camera* cam,
+                                    void* workspace, size_t workspace_bytes, uint64_t* keys, uint32_t* vals,
+                                    int64_t capacity, uint64_t* num_instances_dev, uint32_t* tile_ranges,
+                                    void* stream) {
+    const char* fn = "gs_bin_sort_ordered_async";
+    if (!num_instances_dev) return fail(GS_ERR_INVALID_ARG, "%s: num_instances_dev is NULL", fn);
+    if (n > 0 && !order) return fail(GS_ERR_INVALID_ARG, "%s: order is NULL", fn);
+    if (n > 0) CHECK_PTR(order, 4);
+    return bin_sort_impl(fn, proj, n, cam, workspace, workspace_bytes, keys, vals, capacity, nullptr,
+                         reinterpret_cast<unsigned long long*>(num_instances_dev), tile_ranges, stream,
+                         n > 0 ? order : nullptr);
+}
+
+size_t gs_depth_order_workspace_bytes(int64_t n, int32_t num_views) {
+    if (n < 0) n = 0;
+    if (num_views < 1) num_views = 1;
+    return gsk::depth_order_workspace_layout(n, num_views, nullptr, nullptr);
+}
+
+gs_status gs_depth_order_views(const gs_projected* projs, int32_t num_views, int64_t n, void* workspace,
+                               size_t workspace_bytes, uint32_t* order, void* stream) {
+    const char* fn = "gs_depth_order_views";
+    if (num_views < 1 || num_views > GS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: num_views = %d (1..%d)", fn, int(num_views), GS_MAX_VIEWS);
+    if (n < 0 || n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n out of range", fn);
+    if (!projs) return fail(GS_ERR_INVALID_ARG, "%s: projs is NULL", fn);
+    CHECK_PTR(workspace, 16);
+    if (workspace_bytes < gs_depth_order_workspace_bytes(n, num_views))
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes,
+                    gs_depth_order_workspace_bytes(n, num_views));
+    if (n > 0) {
+        CHECK_PTR(order, 4);
+        for (int v = 0; v < num_views; ++v) {
+            CHECK_PTR(projs[v].tiles_touched, 4);
+            CHECK_PTR(projs[v].depth, 4);
+        }
+    }
+    gsk::DepthOrderWorkspace ws;
+    gsk::depth_order_workspace_layout(n, num_views, workspace, &ws);
+    return cuda_status(gsk::launch_depth_order(projs, num_views, n, ws, order, static_cast<cudaStream_t>(stream)), fn);
 }
 
 gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint32_t* tile_order, void* stream) {

@@ -104,9 +104,36 @@ __global__ void __launch_bounds__(256) depth_keys_kernel(const uint32_t* __restr
     }
 }
 
+// The depth keys of several views at once: view blockIdx.y fills segment
+// blockIdx.y (n elements) of keys and vals.
+struct ViewDepths {
+    const uint32_t* touched[GS_MAX_VIEWS];
+    const float* depth[GS_MAX_VIEWS];
+};
+
+__global__ void __launch_bounds__(256) depth_keys_views_kernel(const ViewDepths src, int64_t n,
+                                                               uint32_t* __restrict__ keys,
+                                                               uint32_t* __restrict__ vals) {
+    const int v = blockIdx.y;
+    const uint32_t* touched = src.touched[v];
+    const float* depth = src.depth[v];
+    keys += int64_t(v) * n;
+    vals += int64_t(v) * n;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+        keys[i] = __ldg(touched + i) > 0u ? __float_as_uint(__ldg(depth + i)) : 0xffffffffu;
+        vals[i] = uint32_t(i);
+    }
+}
+
+// Radix passes over several independent segments at once (one per view): block
+// row blockIdx.y works on segment blockIdx.y, whose keys and values start
+// seg_stride elements further on and whose histograms start 256 nb further on.
 __global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __restrict__ keys, const Count cnt,
-                                                             int shift, uint32_t* __restrict__ hist, int64_t nb) {
+                                                             int shift, uint32_t* __restrict__ hist, int64_t nb,
+                                                             int64_t seg_stride) {
     __shared__ uint32_t h[kSortWarps][256];
+    keys += int64_t(blockIdx.y) * seg_stride;
+    hist += int64_t(blockIdx.y) * 256 * nb;
     const int64_t count = cnt.get();
     const int warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&h[0][0])[k] = 0u;
@@ -128,6 +155,8 @@ __global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __r
 
 // One CTA per digit: exclusive scan over the blocks' counts of that digit.
 __global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t nb, uint32_t* digit_totals) {
+    hist += int64_t(blockIdx.y) * 256 * nb;  // segment blockIdx.y
+    digit_totals += int64_t(blockIdx.y) * 256;
     uint32_t* row = hist + int64_t(blockIdx.x) * nb;
     unsigned long long carry = 0;
     for (int64_t base = 0; base < nb; base += 1024) {
@@ -150,12 +179,24 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
                                                                uint32_t* __restrict__ vals_out, const Count cnt,
                                                                int shift, const uint32_t* __restrict__ hist,
                                                                int64_t nb, const uint32_t* __restrict__ digit_totals,
-                                                               const float* __restrict__ depth) {
+                                                               const float* __restrict__ depth, int64_t seg_stride) {
     __shared__ uint32_t wcount[kSortWarps][256];
     __shared__ uint32_t gbase[256];   // global start of each digit's run from this block
     __shared__ uint32_t lstart[256];  // start of each digit's run within the block
     __shared__ uint32_t sk[kSortTile];
     __shared__ uint32_t sv[kSortTile];
+    {
+        const int64_t so = int64_t(blockIdx.y) * seg_stride;  // segment blockIdx.y
+        keys_in += so;
+        vals_in += so;
+        vals_out += so;
+        if (kFinal)
+            keys_out64 += so;
+        else
+            keys_out += so;
+        hist += int64_t(blockIdx.y) * 256 * nb;
+        digit_totals += int64_t(blockIdx.y) * 256;
+    }
     const int64_t count = cnt.get();
     const int64_t tile0 = int64_t(blockIdx.x) * kSortTile;
     if (tile0 >= count) return;  // block-uniform: launched for the capacity
@@ -326,17 +367,19 @@ size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 // One LSD pass over up to `slots` (key, val) pairs (`cnt` of them when the pass
 // starts).  Final passes write 64-bit keys.
 void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout, uint64_t* kout64, uint32_t* vout,
-                Count cnt, int64_t slots, int shift, const SortWorkspace& ws, const float* depth, cudaStream_t s) {
+                Count cnt, int64_t slots, int shift, uint32_t* hist, uint32_t* digit_totals, const float* depth,
+                cudaStream_t s, int segments = 1, int64_t seg_stride = 0) {
     const int64_t nb = (slots + kSortTile - 1) / kSortTile;
     if (nb == 0) return;
-    upsweep_kernel<<<unsigned(nb), kSortBlock, 0, s>>>(kin, cnt, shift, ws.hist, nb);
-    scan_hist_kernel<<<256, 1024, 0, s>>>(ws.hist, nb, ws.digit_totals);
+    const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>(segments));
+    upsweep_kernel<<<grid, kSortBlock, 0, s>>>(kin, cnt, shift, hist, nb, seg_stride);
+    scan_hist_kernel<<<dim3(256, unsigned(segments)), 1024, 0, s>>>(hist, nb, digit_totals);
     if (kout64)
-        downsweep_kernel<true><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, cnt, shift,
-                                                                   ws.hist, nb, ws.digit_totals, depth);
+        downsweep_kernel<true><<<grid, kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, cnt, shift, hist, nb,
+                                                           digit_totals, depth, seg_stride);
     else
-        downsweep_kernel<false><<<unsigned(nb), kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, cnt, shift,
-                                                                    ws.hist, nb, ws.digit_totals, depth);
+        downsweep_kernel<false><<<grid, kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, cnt, shift, hist, nb,
+                                                            digit_totals, depth, seg_stride);
     count_launches(3);
 }
 
@@ -369,9 +412,71 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
     return off;
 }
 
+size_t depth_order_workspace_layout(int64_t n, int views, void* base, DepthOrderWorkspace* ws) {
+    const int64_t total = n * views;
+    const int64_t nb = (n + kSortTile - 1) / kSortTile;
+    size_t off = 0;
+    char* b = static_cast<char*>(base);
+    DepthOrderWorkspace w;
+    w.nb = nb;
+    for (int r = 0; r < 2; ++r) {
+        w.key[r] = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * size_t(total > 0 ? total : 1));
+        w.val[r] = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * size_t(total > 0 ? total : 1));
+    }
+    w.hist = reinterpret_cast<uint32_t*>(b + off);
+    off += align_up(sizeof(uint32_t) * 256 * size_t(nb > 0 ? nb : 1) * size_t(views > 0 ? views : 1));
+    w.digit_totals = reinterpret_cast<uint32_t*>(b + off);
+    off += align_up(sizeof(uint32_t) * 256 * size_t(views > 0 ? views : 1));
+    if (ws) *ws = w;
+    return off;
+}
+
+cudaError_t launch_depth_order(const gs_projected* projs, int views, int64_t n, const DepthOrderWorkspace& ws,
+                               uint32_t* order, cudaStream_t s) {
+    if (n == 0 || views == 0) return cudaSuccess;
+    ViewDepths src;
+    for (int v = 0; v < views; ++v) {
+        src.touched[v] = projs[v].tiles_touched;
+        src.depth[v] = projs[v].depth;
+    }
+    const dim3 kgrid(grid_for(n, 256, 8), static_cast<unsigned>(views));
+    depth_keys_views_kernel<<<kgrid, 256, 0, s>>>(src, n, ws.key[0], ws.val[0]);
+    count_launches(1);
+    // four stable 8-bit passes A -> B -> A -> B -> (A, order), every view a segment
+    const Count all{n, nullptr, 0};
+    for (int p = 0; p < 4; ++p) {
+        const int a = p & 1;
+        uint32_t* vout = p == 3 ? order : ws.val[a ^ 1];
+        radix_pass(ws.key[a], ws.val[a], ws.key[a ^ 1], nullptr, vout, all, n, 8 * p, ws.hist, ws.digit_totals,
+                   nullptr, s, views, n);
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& cam, const SortWorkspace& ws,
                             uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* ranges,
                             unsigned long long* count_out, cudaStream_t s) {
+    if (n > 0) {
+        // depth order of the Gaussians: 4 passes from buffer 1 back into buffer 1, so
+        // that tval[1] holds the order while the instances are emitted into buffer 0
+        depth_keys_kernel<<<grid_for(n, 256, 8), 256, 0, s>>>(proj.tiles_touched, proj.depth, n, ws.tkey[1],
+                                                               ws.tval[1]);
+        count_launches(1);
+        const Count all{n, nullptr, 0};
+        for (int p = 0; p < 4; ++p) {
+            const int src = (p & 1) ? 0 : 1;
+            radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], all, n, 8 * p,
+                       ws.hist, ws.digit_totals, nullptr, s);
+        }
+    }
+    return launch_bin_sort_ordered(proj, n, ws.tval[1], cam, ws, keys, vals, capacity, ranges, count_out, s);
+}
+
+cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const uint32_t* order, const CamArgs& cam,
+                                    const SortWorkspace& ws, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                                    uint32_t* ranges, unsigned long long* count_out, cudaStream_t s) {
     const int64_t T = int64_t(cam.TX) * cam.TY;
     cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint32_t) * 2 * size_t(T), s);
     if (e != cudaSuccess) return e;
@@ -380,24 +485,13 @@ cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& 
         if (e == cudaSuccess && count_out) e = cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), s);
         return e;
     }
-    // depth order of the Gaussians: 4 passes from buffer 1 back into buffer 1, so
-    // that tval[1] holds the order while the instances are emitted into buffer 0
-    depth_keys_kernel<<<grid_for(n, 256, 8), 256, 0, s>>>(proj.tiles_touched, proj.depth, n, ws.tkey[1], ws.tval[1]);
-    count_launches(1);
-    const Count all{n, nullptr, 0};
-    for (int p = 0; p < 4; ++p) {
-        const int src = (p & 1) ? 0 : 1;
-        radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], all, n, 8 * p, ws,
-                   nullptr, s);
-    }
-    count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, ws.tval[1], n,
-                                                                    ws.block_sums);
+    count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, order, n, ws.block_sums);
     scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total, count_out);
     count_launches(2);
     // instances: launched for the capacity, K read on the device
     const Count inst{0, ws.total, capacity};
     emit_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, reinterpret_cast<const uint2*>(proj.rect),
-                                                            ws.tval[1], n, cam.TX, ws.block_sums, inst, ws.tkey[0],
+                                                            order, n, cam.TX, ws.block_sums, inst, ws.tkey[0],
                                                             ws.tval[0]);
     count_launches(1);
     const int bits = tile_bits(T);
@@ -406,7 +500,7 @@ cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& 
     for (int p = 0; p < passes; ++p) {
         const bool last = p == passes - 1;
         radix_pass(ws.tkey[cur], ws.tval[cur], last ? nullptr : ws.tkey[cur ^ 1], last ? keys : nullptr,
-                   last ? vals : ws.tval[cur ^ 1], inst, capacity, 8 * p, ws, proj.depth, s);
+                   last ? vals : ws.tval[cur ^ 1], inst, capacity, 8 * p, ws.hist, ws.digit_totals, proj.depth, s);
         cur ^= 1;
     }
     if (capacity > 0) {

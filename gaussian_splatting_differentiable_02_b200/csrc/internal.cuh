@@ -80,6 +80,25 @@ cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& 
                             uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* ranges,
                             unsigned long long* count_out, cudaStream_t s);
 
+// The rest of the binning from a given depth order of the Gaussians (order [n]):
+// emission, the passes by tile id, ranges.
+cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const uint32_t* order, const CamArgs& cam,
+                                    const SortWorkspace& ws, uint64_t* keys, uint32_t* vals, int64_t capacity,
+                                    uint32_t* ranges, unsigned long long* count_out, cudaStream_t s);
+
+// Stable depth order of the Gaussians of several views (at most GS_MAX_VIEWS) in
+// one launch per radix pass: order [views][n].
+struct DepthOrderWorkspace {
+    uint32_t* key[2];        // [views][n], ping-pong
+    uint32_t* val[2];        // [views][n], ping-pong
+    uint32_t* hist;          // [views][256][nb]
+    uint32_t* digit_totals;  // [views][256]
+    int64_t nb;
+};
+size_t depth_order_workspace_layout(int64_t n, int views, void* base, DepthOrderWorkspace* ws);
+cudaError_t launch_depth_order(const gs_projected* projs, int views, int64_t n, const DepthOrderWorkspace& ws,
+                               uint32_t* order, cudaStream_t s);
+
 cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s);
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,

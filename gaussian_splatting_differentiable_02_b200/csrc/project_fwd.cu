@@ -59,6 +59,12 @@ __global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
         const float4 q4 = __ldg(a.quats + i);
         const float4 s4 = __ldg(a.log_scales + i);
         const float lg = __ldg(a.logits + i);
+#ifndef GS_PROJECT_NO_PREFETCH
+        // the SH planes are read only after the covariance arithmetic: start moving
+        // them into L2 now so that their loads do not wait on DRAM then
+        for (int p = 0; p < a.planes; ++p)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.sh + int64_t(p) * a.n + i));
+#endif
         const double mu[3] = {m4.x, m4.y, m4.z};
         const double q[4] = {q4.x, q4.y, q4.z, q4.w};
         const double ls[3] = {s4.x, s4.y, s4.z};

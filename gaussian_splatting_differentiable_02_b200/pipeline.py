@@ -213,6 +213,32 @@ def bin_sort_async(proj: Projected, view: View, counter: torch.Tensor, radius: t
     abi.gs_tile_order(_ptr(view.ranges), view.gcam, _ptr(view.order), _stream())
 
 
+class DepthOrder:
+    """Depth orders of several views of the same n Gaussians ([views, n] uint32) and the
+    workspace of the batched sort that computes them."""
+
+    def __init__(self, n: int, views: int, device="cuda"):
+        self.n, self.views = int(n), int(views)
+        self.order = torch.empty((views, max(n, 1)), device=device, dtype=torch.int32)
+        nbytes = abi.gs_depth_order_workspace_bytes(n, views)
+        self.workspace = torch.empty((nbytes,), device=device, dtype=torch.uint8)
+
+
+def depth_order_views(projs: list, radii: torch.Tensor, d: DepthOrder):
+    """Every view's stable depth order in one batched sort (projs[k] with radius row radii[k])."""
+    abi.gs_depth_order_views([p.struct(radii[k]) for k, p in enumerate(projs)], d.n, _ptr(d.workspace),
+                             d.workspace.numel(), _ptr(d.order), _stream())
+
+
+def bin_sort_ordered_async(proj: Projected, view: View, order_row: torch.Tensor, counter: torch.Tensor,
+                           radius: torch.Tensor = None):
+    """bin_sort_async from a precomputed depth order (a row of DepthOrder.order)."""
+    abi.gs_bin_sort_ordered_async(proj.struct(radius), view.n, _ptr(order_row), view.gcam, _ptr(view.workspace),
+                                  view.workspace.numel(), _ptr(view.keys), _ptr(view.vals), view.capacity,
+                                  _ptr(counter), _ptr(view.ranges), _stream())
+    abi.gs_tile_order(_ptr(view.ranges), view.gcam, _ptr(view.order), _stream())
+
+
 def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Tensor = None):
     abi.gs_raster_fwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam, bg,
                       _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _stream())
@@ -332,7 +358,9 @@ class Trainer:
     absgrad: bool = False      # densify on the absolute 2D gradient (the gsplat guide §4.1 absgrad option)
     sparse_grad: bool = False  # Adam skips Gaussians seen in no view of the step (sparse_grad option; fused only)
     streams: int = 3           # fused path: views alternate over this many CUDA streams, so that one
-                               # view's projection and sort overlap another view's compositing
+                               # view's sort overlaps another view's compositing
+    batched_sort: bool = True  # fused path: project every view first and sort all views by depth in one
+                               # batched sort (gs_depth_order_views), then bin and composite per view
 
     def __post_init__(self):
         n = self.gauss.n
@@ -354,8 +382,14 @@ class Trainer:
         nv = len(self.views) if self.fused else 1
         self.proj = Projected(n, dev)
         # concurrent views need their own projected features
-        self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
-            if self.fused else [self.proj]
+        if self.fused and self.batched_sort:
+            # every view's projection is kept until its binning
+            self.projs = [self.proj] + [Projected(n, dev) for _ in range(nv - 1)]
+            self.depth_order = DepthOrder(n, nv, dev)
+        else:
+            self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
+                if self.fused else [self.proj]
+            self.depth_order = None
         self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
         self.grad2d = self.grad2ds[0]
         self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
@@ -386,19 +420,24 @@ class Trainer:
         self._alloc_per_gaussian(g.n)
         return decision
 
-    def view_forward_backward(self, k: int, target: torch.Tensor, proj: Projected = None) -> None:
+    def view_forward_backward(self, k: int, target: torch.Tensor, proj: Projected = None,
+                              projected: bool = False) -> None:
         """project -> sort -> raster forward -> L1 -> raster backward of view k (on the
         current stream).  The fused path sorts without waiting (instance count checked
-        once per step)."""
+        once per step); with `projected` the view was projected and depth-ordered
+        already (the batched sort) and only the binning from that order runs here."""
         view = self.views[k]
         proj = self.proj if proj is None else proj
         r = self.radii[k if self.fused else 0]
         g2 = self.grad2ds[k if self.fused else 0]
-        project(self.gauss, view, proj, r)
-        if self.fused:
-            bin_sort_async(proj, view, self.kcount[k:k + 1], r)
+        if projected:
+            bin_sort_ordered_async(proj, view, self.depth_order.order[k], self.kcount[k:k + 1], r)
         else:
-            bin_sort(proj, view, r)
+            project(self.gauss, view, proj, r)
+            if self.fused:
+                bin_sort_async(proj, view, self.kcount[k:k + 1], r)
+            else:
+                bin_sort(proj, view, r)
         raster_fwd(proj, view, self.bg, r)
         if self.ssim_weight > 0.0:
             l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
@@ -410,26 +449,36 @@ class Trainer:
     def _all_views(self) -> None:
         """Every view's forward and backward; in the fused path view k runs on stream
         k mod `streams` (each with its own projected features), joined before return."""
-        if not self.fused or len(self.projs) == 1:
+        if not self.fused or (self.depth_order is None and len(self.projs) == 1):
             for k, tgt in enumerate(self.targets):
                 self.view_forward_backward(k, tgt)
             return
         main = torch.cuda.current_stream()
         side = self.side_streams()
+        batched = self.depth_order is not None
+        if batched:
+            self.project_and_order()
         start = main.record_event()
         for st in side:
             st.wait_event(start)
         for k, tgt in enumerate(self.targets):
             j = k % len(side)
             with torch.cuda.stream(side[j]):
-                self.view_forward_backward(k, tgt, self.projs[j])
+                self.view_forward_backward(k, tgt, self.projs[k if batched else j], projected=batched)
         for st in side:
             main.wait_stream(st)
 
+    def project_and_order(self) -> None:
+        """Every view's projection, then the batched depth sort of all views (current stream)."""
+        for k, view in enumerate(self.views):
+            project(self.gauss, view, self.projs[k], self.radii[k])
+        depth_order_views(self.projs, self.radii, self.depth_order)
+
     def side_streams(self) -> list:
-        """The streams the fused path runs views on (one per projected-feature buffer)."""
+        """The streams the fused path runs views on."""
         if getattr(self, "_side", None) is None:
-            self._side = [torch.cuda.Stream(device=self.gauss.means.device) for _ in self.projs]
+            count = min(self.streams, len(self.views))
+            self._side = [torch.cuda.Stream(device=self.gauss.means.device) for _ in range(count)]
         return self._side
 
     def step(self) -> None:

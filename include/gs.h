@@ -189,6 +189,30 @@ gs_status gs_bin_sort_async(const gs_projected* proj, int64_t n, const gs_camera
                             size_t workspace_bytes, uint64_t* keys, uint32_t* vals, int64_t capacity,
                             uint64_t* num_instances_dev, uint32_t* tile_ranges, void* stream);
 
+/* Bytes of device workspace gs_depth_order_views needs for n Gaussians seen
+ * from num_views views (about 16 bytes per Gaussian and view). */
+size_t gs_depth_order_workspace_bytes(int64_t n, int32_t num_views);
+
+/* gs_depth_order_views -- the first half of gs_bin_sort for several views of the
+ * same Gaussians at once: for each view v (1..GS_MAX_VIEWS views, projs[v] as
+ * written by gs_project; tiles_touched and depth are read), the stable order of
+ * the Gaussians by the float32 bits of their depth, culled Gaussians last,
+ * written to order[v * n ... v * n + n - 1] (uint32, 4-byte aligned).  One launch
+ * per radix pass serves every view.  Asynchronous; workspace (16-byte aligned,
+ * caller-owned) as sized above. */
+gs_status gs_depth_order_views(const gs_projected* projs, int32_t num_views, int64_t n, void* workspace,
+                               size_t workspace_bytes, uint32_t* order, void* stream);
+
+/* gs_bin_sort_ordered_async -- gs_bin_sort_async from a depth order computed by
+ * gs_depth_order_views (order [n], this view's row): emission of the instances
+ * in that order, the stable passes by tile id, the ranges.  Same arguments,
+ * results and capacity behaviour as gs_bin_sort_async otherwise (the same
+ * workspace size). */
+gs_status gs_bin_sort_ordered_async(const gs_projected* proj, int64_t n, const uint32_t* order, const gs_camera* cam,
+                                    void* workspace, size_t workspace_bytes, uint64_t* keys, uint32_t* vals,
+                                    int64_t capacity, uint64_t* num_instances_dev, uint32_t* tile_ranges,
+                                    void* stream);
+
 /* Size of the device array gs_bin_sort_static uses as its workspace (32 MiB). */
 #define GS_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 

@@ -237,29 +237,69 @@ def test_sparse_adam_skips_gaussians_seen_in_no_view():
     assert not np.array_equal(out[0][1]["means"][~vis], init[1]["means"][~vis])
 
 
-def test_trainer_two_streams_equals_one():
-    """Views spread over two CUDA streams (each with its own projected features) give
-    the step of the single-stream order: same losses, counts and parameters up to the
-    order of the atomic adds."""
+def test_trainer_stream_and_sort_configurations_agree():
+    """Views on one stream with a sort per view, on two streams, and on three streams
+    after one batched depth sort of all views: the first step (identical inputs) gives
+    the same loss, counts and instance numbers; later steps agree up to the order of
+    the atomic adds."""
     rng = np.random.default_rng(13)
     scene = scenes.random_scene(rng, 600, 1, mean_box=1.0, log_scale=(-3.5, -2.0))
     cams = _views(5, 8)
     targets = [torch.from_numpy(rng.random((128, 128, 3)).astype(np.float32)).cuda() for _ in cams]
     out = []
-    for streams in (1, 2):
+    for streams, batched in ((1, False), (2, False), (3, True)):
         g = pl.Gaussians.from_scene(scene)
-        tr = pl.Trainer(g, [pl.View(scene.n, c) for c in cams], targets, dict(LRS), densify=True, streams=streams)
-        assert len(tr.projs) == streams
-        tr.step()   # the first step starts from identical parameters: counts and K agree exactly
+        tr = pl.Trainer(g, [pl.View(scene.n, c) for c in cams], targets, dict(LRS), densify=True, streams=streams,
+                        batched_sort=batched)
+        tr.step()
         torch.cuda.synchronize()
-        first = (tr.loss.item(), tr.densify_count.cpu().numpy(), tr.kcount.cpu().numpy())
+        first = (tr.loss.item(), tr.densify_count.cpu().numpy(), tr.kcount.cpu().numpy(),
+                 [vw.keys[:int(K)].cpu().numpy() for vw, K in zip(tr.views, tr.kcount.cpu().tolist())])
         tr.step()
         tr.step()
         torch.cuda.synchronize()
         out.append((tr.gauss.to_numpy(), first))
-    (a, (la, ca, ka)), (b, (lb, cb, kb)) = out
-    assert np.array_equal(ca, cb) and np.array_equal(ka, kb)
-    assert abs(la - lb) <= 1e-9 * abs(la)
-    for k in NAMES:
-        close = np.abs(a[k] - b[k]) <= 1e-6 + 1e-5 * np.abs(a[k])
-        assert close.mean() >= 0.999, (k, float(close.mean()))
+    (a, (la, ca, ka, keys_a)) = out[0]
+    for b, (lb, cb, kb, keys_b) in out[1:]:
+        assert np.array_equal(ca, cb) and np.array_equal(ka, kb)
+        assert all(np.array_equal(x, y) for x, y in zip(keys_a, keys_b))
+        assert abs(la - lb) <= 1e-9 * abs(la)
+        for k in NAMES:
+            close = np.abs(a[k] - b[k]) <= 1e-6 + 1e-5 * np.abs(a[k])
+            assert close.mean() >= 0.999, (k, float(close.mean()))
+
+
+def test_batched_depth_order_matches_the_per_view_sort(orc):
+    """gs_depth_order_views + gs_bin_sort_ordered_async give, for every view, the keys,
+    values and ranges of gs_bin_sort (bit for bit) and of the oracle."""
+    rng = np.random.default_rng(14)
+    scene = scenes.random_scene(rng, 3000, 1, mean_box=1.0, log_scale=(-4.0, -2.0))
+    scene.means[:100] += 30.0   # some Gaussians culled in every view
+    cams = _views(6, 9)
+    g = pl.Gaussians.from_scene(scene)
+    projs = [pl.Projected(scene.n) for _ in cams]
+    views = [pl.View(scene.n, c, capacity=40 * scene.n) for c in cams]
+    radii = torch.zeros((len(cams), scene.n), dtype=torch.int32, device="cuda")
+    for k, vw in enumerate(views):
+        pl.project(g, vw, projs[k], radii[k])
+    d = pl.DepthOrder(scene.n, len(cams))
+    pl.depth_order_views(projs, radii, d)
+    counts = torch.zeros((len(cams),), dtype=torch.int64, device="cuda")
+    for k, vw in enumerate(views):
+        pl.bin_sort_ordered_async(projs[k], vw, d.order[k], counts[k:k + 1], radii[k])
+    torch.cuda.synchronize()
+    for k, (vw, cam) in enumerate(zip(views, cams)):
+        K = int(counts[k].item())
+        assert K <= vw.capacity
+        ref = orc.project(scene, cam)
+        keys, vals, ranges = orc.keys(ref, cam)
+        assert K == len(keys)
+        assert np.array_equal(vw.keys[:K].cpu().numpy().view(np.uint64), keys)
+        assert np.array_equal(vw.vals[:K].cpu().numpy().view(np.uint32), vals)
+        assert np.array_equal(vw.ranges.cpu().numpy().view(np.uint32), ranges)
+        # the depth order itself: visible Gaussians by (depth bits, index), culled ones after
+        order = d.order[k].cpu().numpy().view(np.uint32)
+        r = radii[k].cpu().numpy()
+        z = projs[k].depth.cpu().numpy().view(np.uint32).astype(np.uint64)
+        keyz = np.where(r > 0, z, 0xFFFFFFFF)
+        assert np.array_equal(order, np.lexsort((np.arange(scene.n), keyz)).astype(np.uint32))
