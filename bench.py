@@ -568,12 +568,12 @@ def stage_breakdown(tr, pl, torch):
     return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
 
 
-# Source files each stage's kernels are built from: a DRAM traffic figure taken
-# by ncu is reported only while these files are unchanged since the capture.
+# Source file of each stage's kernels: a DRAM traffic figure taken by ncu is
+# reported only while this file is unchanged since the capture.
 STAGE_SOURCES = {
-    "raster_bwd": ["csrc/raster.cu", "csrc/internal.cuh", "../include/gs.h"],
-    "raster_fwd": ["csrc/raster.cu", "csrc/internal.cuh", "../include/gs.h"],
-    "project_bwd_adam": ["csrc/project_bwd.cu", "csrc/internal.cuh", "../include/gs.h"],
+    "raster_bwd": ["csrc/raster.cu"],
+    "raster_fwd": ["csrc/raster.cu"],
+    "project_bwd_adam": ["csrc/project_bwd.cu"],
 }
 
 
@@ -648,8 +648,9 @@ def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks, workloa
 
 def run_e2e(tr, targets_host, targets, args, world, torch):
     """Steps whose target images arrive from pinned host memory (copied on a side
-    stream one view ahead, overlapping the previous view's kernels) and whose
-    loss is read back every step."""
+    stream a few views ahead, overlapping the kernels of the views before) and
+    whose loss is read back every step; the views run through the Trainer's own
+    view loop."""
     if targets_host is None:
         return None
     stream = torch.cuda.current_stream()
@@ -665,8 +666,6 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
     from gaussian_splatting_differentiable_02_b200 import abi
 
     def step():
-        nonlocal done
-        done = [torch.cuda.Event() for _ in range(nv)]
         abi.gs_zero(tr.loss.data_ptr(), 8, stream.cuda_stream)
         begin = stream.record_event()
         copy_events = {}
@@ -675,25 +674,19 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
             for v in range(nbuf):
                 bufs[v].copy_(targets_host[v], non_blocking=True)
                 copy_events[v] = copy_stream.record_event()
-        batched = tr.depth_order is not None
-        if batched:
-            tr.project_and_order()
-            begin = stream.record_event()
-        for v in range(nv):
-            st = side[v % len(side)]
-            st.wait_event(begin)
-            st.wait_event(copy_events[v])
-            with torch.cuda.stream(st):
-                tr.view_forward_backward(v, bufs[v % nbuf], tr.projs[v if batched else v % len(side)],
-                                         projected=batched)
-            done[v].record(st)
+
+        class Ready:   # the copy event of view v exists by the time the Trainer asks for it
+            def __getitem__(self, v):
+                return copy_events[v]
+
+        def after_view(v, ev):
             if v + nbuf < nv:
                 with torch.cuda.stream(copy_stream):
-                    copy_stream.wait_event(done[v])
+                    copy_stream.wait_event(ev)
                     bufs[v % nbuf].copy_(targets_host[v + nbuf], non_blocking=True)
                     copy_events[v + nbuf] = copy_stream.record_event()
-        for st in side:
-            stream.wait_stream(st)
+
+        tr._all_views(targets=[bufs[v % nbuf] for v in range(nv)], ready=Ready(), after_view=after_view)
         # the step's one wait: the instance counts (buffers were sized in the warm-up)
         if any(K > vw.capacity for K, vw in zip(tr.kcount.cpu().tolist(), tr.views)):
             raise RuntimeError("instance buffers overflowed after the warm-up")
@@ -703,7 +696,6 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
                                   densify_max_radius=tr.densify_max_radius)
         loss_host.copy_(tr.loss, non_blocking=True)
 
-    done = []
     for _ in range(max(1, args.warmup // 2)):
         step()
     torch.cuda.synchronize()

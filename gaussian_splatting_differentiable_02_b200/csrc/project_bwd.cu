@@ -176,6 +176,28 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
         }
         if ((!kAdam || a.sparse) && vis == 0u) continue;  // nothing to add (sparse Adam: nothing to update)
         if (a.densify_max_radius && rmax > a.densify_max_radius[i]) a.densify_max_radius[i] = rmax;
+#ifndef GS_PBWD_NO_PREFETCH
+        // everything this Gaussian reads after the long double-precision chain (the
+        // visible views' 2D gradients, the Adam moments) starts moving into L2 now
+        for (unsigned rest = vis; rest; rest &= rest - 1u) {
+            const ViewArgs& w = a.view[__ffs(rest) - 1];
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_xy + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_con + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_rgb + i));
+        }
+        if (kAdam) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.m_means + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.v_means + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.m_quats + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.v_quats + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.m_log_scales + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.v_log_scales + i));
+            for (int p = 0; p < a.planes; ++p) {
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.m_sh + int64_t(p) * a.n + i));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.v_sh + int64_t(p) * a.n + i));
+            }
+        }
+#endif
 
         double gS[6] = {0, 0, 0, 0, 0, 0};  // symmetric dL/dSigma: xx, xy, xz, yy, yz, zz
         double gmu[3] = {0, 0, 0};

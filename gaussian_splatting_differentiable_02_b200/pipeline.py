@@ -446,27 +446,81 @@ class Trainer:
         g2.zero_()
         raster_bwd(proj, view, g2, self.bg, radius=r)
 
-    def _all_views(self) -> None:
+    def _all_views(self, targets=None, ready=None, after_view=None) -> None:
         """Every view's forward and backward; in the fused path view k runs on stream
-        k mod `streams` (each with its own projected features), joined before return."""
+        k mod `streams`, joined before return.  targets: per-view target images
+        (default self.targets); ready: per-view CUDA events view k's compositing waits
+        for (e.g. the copy of its target); after_view(k, event): called once view k
+        is enqueued, with an event recorded after it."""
+        targets = self.targets if targets is None else targets
         if not self.fused or (self.depth_order is None and len(self.projs) == 1):
-            for k, tgt in enumerate(self.targets):
+            for k, tgt in enumerate(targets):
+                if ready is not None:
+                    torch.cuda.current_stream().wait_event(ready[k])
                 self.view_forward_backward(k, tgt)
+                if after_view is not None:
+                    after_view(k, torch.cuda.current_stream().record_event())
             return
         main = torch.cuda.current_stream()
         side = self.side_streams()
         batched = self.depth_order is not None
         if batched:
             self.project_and_order()
+            # binning of every view on a high-priority stream: its small, latency-bound
+            # kernels take SM slots as soon as compositing blocks retire, instead of
+            # queueing behind whole compositing launches
+            bin_stream = self.bin_stream()
+            bin_stream.wait_stream(main)
+            binned = []
+            with torch.cuda.stream(bin_stream):
+                for k, view in enumerate(self.views):
+                    bin_sort_ordered_async(self.projs[k], view, self.depth_order.order[k], self.kcount[k:k + 1],
+                                           self.radii[k])
+                    binned.append(bin_stream.record_event())
+            for k, tgt in enumerate(targets):
+                st = side[k % len(side)]
+                st.wait_event(binned[k])
+                if ready is not None:
+                    st.wait_event(ready[k])
+                with torch.cuda.stream(st):
+                    self.view_composite(k, tgt, self.projs[k])
+                if after_view is not None:
+                    after_view(k, st.record_event())
+            for st in side + [bin_stream]:
+                main.wait_stream(st)
+            return
         start = main.record_event()
         for st in side:
             st.wait_event(start)
-        for k, tgt in enumerate(self.targets):
+        for k, tgt in enumerate(targets):
             j = k % len(side)
+            if ready is not None:
+                side[j].wait_event(ready[k])
             with torch.cuda.stream(side[j]):
-                self.view_forward_backward(k, tgt, self.projs[k if batched else j], projected=batched)
+                self.view_forward_backward(k, tgt, self.projs[j])
+            if after_view is not None:
+                after_view(k, side[j].record_event())
         for st in side:
             main.wait_stream(st)
+
+    def view_composite(self, k: int, target: torch.Tensor, proj: Projected) -> None:
+        """raster forward -> loss -> raster backward of an already binned view k."""
+        view = self.views[k]
+        r = self.radii[k]
+        raster_fwd(proj, view, self.bg, r)
+        if self.ssim_weight > 0.0:
+            l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
+        else:
+            l1_loss_grad(view, target, self.loss)
+        self.grad2ds[k].zero_()
+        raster_bwd(proj, view, self.grad2ds[k], self.bg, radius=r)
+
+    def bin_stream(self) -> torch.cuda.Stream:
+        """The high-priority stream the batched path bins every view on."""
+        if getattr(self, "_bin_stream", None) is None:
+            hi = torch.cuda.Stream.priority_range()[1] if hasattr(torch.cuda.Stream, "priority_range") else -1
+            self._bin_stream = torch.cuda.Stream(device=self.gauss.means.device, priority=hi)
+        return self._bin_stream
 
     def project_and_order(self) -> None:
         """Every view's projection, then the batched depth sort of all views (current stream)."""

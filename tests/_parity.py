@@ -40,7 +40,7 @@ def ulp_diff(a, b):
     return np.abs(ia - ib)
 
 
-class GpuRun:
+class CudaRun:
     """Forward (and optionally backward) of one view through the C ABI."""
 
     def __init__(self, scene, cam, bg=(0.0, 0.0, 0.0), capacity=0):

@@ -10,7 +10,7 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 from gaussian_splatting_differentiable_02_b200 import scenes
 
-from _parity import BAND_ALPHA, BAND_T, GpuRun, check_grads
+from _parity import BAND_ALPHA, BAND_T, CudaRun, check_grads
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,7 @@ def test_absgrad_matches_oracle(orc, case):
         R, t = scenes.look_at((0.5, 0.2, -4.0))
         cam = scenes.camera(R, t, 120.0, 120.0, 50.0, 18.5, 100, 37)
         up = rng.standard_normal((37, 100, 3)).astype(np.float32)
-    run = GpuRun(scene, cam)
+    run = CudaRun(scene, cam)
     plain = run.backward(up)
     g2 = _absgrad(run, up)
     # the option leaves the ordinary gradients as they were (same arithmetic; the
@@ -56,7 +56,7 @@ def test_absgrad_matches_oracle(orc, case):
 
 def test_densify_statistic_uses_the_absolute_gradient(orc):
     wl = scenes.tiny()
-    run = GpuRun(wl.scene, wl.cameras[0])
+    run = CudaRun(wl.scene, wl.cameras[0])
     g2 = _absgrad(run, wl.upstream[0])
     n = wl.scene.n
     grads = run.g.zeros_like()

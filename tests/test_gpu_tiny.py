@@ -10,7 +10,7 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import abi, scenes
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 
-from _parity import (BAND_ALPHA, BAND_T, GpuRun, check_grads, check_images, check_projection, grad_mismatch,
+from _parity import (BAND_ALPHA, BAND_T, CudaRun, check_grads, check_images, check_projection, grad_mismatch,
                      ulp_diff)
 
 pytestmark = pytest.mark.gpu
@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 def tiny(orc):
     wl = scenes.tiny()
     cam = wl.cameras[0]
-    run = GpuRun(wl.scene, cam)
+    run = CudaRun(wl.scene, cam)
     ref = orc.project(wl.scene, cam)
     return wl, cam, run, ref
 
@@ -156,7 +156,7 @@ def test_l1_matches_oracle(orc):
 # ------------------------------------------------------------------ edge cases
 
 def _run_and_compare(orc, scene, cam, bg=(0.0, 0.0, 0.0), max_amb_frac=1e-3):
-    run = GpuRun(scene, cam, bg=bg)
+    run = CudaRun(scene, cam, bg=bg)
     ref = orc.project(scene, cam)
     check_projection(run.projection(), ref)
     keys, vals, ranges = orc.keys(ref, cam)
@@ -171,7 +171,7 @@ def _run_and_compare(orc, scene, cam, bg=(0.0, 0.0, 0.0), max_amb_frac=1e-3):
 def test_empty_scene(orc):
     scene = scenes.random_scene(np.random.default_rng(0), 0, 0)
     cam = scenes.tiny().cameras[0]
-    run = GpuRun(scene, cam, bg=(0.1, 0.2, 0.3))
+    run = CudaRun(scene, cam, bg=(0.1, 0.2, 0.3))
     assert run.K == 0
     gi, gT, gn = run.images()
     assert np.all(gi == np.float32([0.1, 0.2, 0.3])) and np.all(gT == 1.0) and np.all(gn == 0)
@@ -252,7 +252,7 @@ def test_needle_and_indefinite_conics(orc):
     evaluation does."""
     wl = scenes.tiny()
     cam = wl.cameras[0]
-    run = GpuRun(wl.scene, cam)
+    run = CudaRun(wl.scene, cam)
     p = run.projection()
     vis = np.argsort(-p["radius"])[:12]   # the largest footprints
     assert np.all(p["radius"][vis] > 4)

@@ -17,7 +17,7 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 from gaussian_splatting_differentiable_02_b200 import scenes
 
-from _parity import (BAND_ALPHA, BAND_T, GpuRun, check_grads, check_images, check_projection)
+from _parity import (BAND_ALPHA, BAND_T, CudaRun, check_grads, check_images, check_projection)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +57,7 @@ def test_workload_parity(orc, workload):
     name, scene, cams = workload
     rng = np.random.default_rng(0)
     for ci, cam in enumerate(cams):
-        run = GpuRun(scene, cam)
+        run = CudaRun(scene, cam)
         ref = orc.project(scene, cam)
         check_projection(run.projection(), ref)
 
