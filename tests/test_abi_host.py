@@ -130,6 +130,29 @@ def test_invalid_arguments_rejected_before_launch(gs):
     assert L.gs_densify_apply(C.byref(p), None, None, 256, 256, 256, ws, 21, C.byref(gr), None, None, None) == \
         gs.GS_ERR_INVALID_ARG
     assert "n_out" in gs.gs_last_error_detail()
+    # batched depth order: view count bounds, small workspace, NULL order
+    projs = (gs.gs_projected * 2)(proj, proj)
+    wsd = gs.gs_depth_order_workspace_bytes(10, 2)
+    assert wsd >= 4 * 4 * 10 * 2
+    assert L.gs_depth_order_views(projs, 0, 10, 256, wsd, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_depth_order_views(projs, 17, 10, 256, wsd, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_depth_order_views(projs, 2, 10, 256, 16, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert "workspace" in gs.gs_last_error_detail()
+    assert L.gs_depth_order_views(projs, 2, 10, 256, wsd, None, None) == gs.GS_ERR_INVALID_ARG
+    # binning from an order: the order is required
+    cnt = C.c_uint64()
+    assert L.gs_bin_sort_ordered_async(C.byref(proj), 10, None, C.byref(c), 256, 1 << 30, 256, 256, 100, 256, 256,
+                                       None) == gs.GS_ERR_INVALID_ARG
+    assert "order" in gs.gs_last_error_detail()
+    # the sparse Adam flag is 0 or 1
+    lr = (C.c_float * 5)(1e-3, 1e-3, 1e-3, 1e-3, 1e-3)
+    assert L.gs_project_bwd_views_adam(C.byref(p), 1, C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr),
+                                       C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None, None, None, None, 2,
+                                       None) == gs.GS_ERR_INVALID_ARG
+    # D-SSIM: image size limits and workspace
+    assert L.gs_l1_dssim_loss_grad(256, 256, 0, 10, 1.0, 0.2, 256, 1 << 20, 256, 256, None) == gs.GS_ERR_UNSUPPORTED
+    assert L.gs_l1_dssim_loss_grad(256, 256, 10, 10, 1.0, 0.2, 256, 8, 256, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert gs.gs_l1_dssim_workspace_bytes(10, 10) >= 72 * 100
     # zero-size work needs no pointers and launches nothing
     assert L.gs_adam(None, None, None, None, 0, 1e-3, 0.9, 0.99, 1e-15, 1, None) == gs.GS_OK
     assert L.gs_l1_loss_grad(None, None, 0, None, None, None) == gs.GS_OK
