@@ -266,10 +266,11 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
 #pragma unroll
         for (int p = 0; p < kPairs; ++p) {
             r.dy[p] = add2(vy, nyc[p]);
-            const f2 sv = fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0);
-            const f2 e = add2(sv, lo);
-            alpha_at(e.x, sv.x <= 0.f, 2 * p, r.nal[p].x, r.blend, r.clamp);
-            alpha_at(e.y, sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
+            // a positive-definite form has sigma >= 0; the float32 value can round
+            // below zero only within rounding of the mean, where alpha is o either way
+            const f2 e = add2(fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0), lo);
+            alpha_at(e.x, true, 2 * p, r.nal[p].x, r.blend, r.clamp);
+            alpha_at(e.y, true, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
         }
     }
 }
