@@ -10,6 +10,11 @@ algorithmic HBM bytes against the measured copy bandwidth.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload multiview|mixture|box|city|tiny]
 
+Other workloads: mixture (the 1M mixture, one 1296x840 view per training step),
+tiny (1,000 Gaussians at 128x128), and the forward-only box (100k Gaussians, 1080p,
+a step renders its 100 poses) and city (3M Gaussians, 3840x2160, 50 poses), which
+report frames/s.
+
 --impl reference times the CPU oracle (the plain double-precision per-pixel
 renderer the tests use as ground truth) on a bounded sample of the same
 workload.  With N > 1 every rank runs an independent replica (the path has no
@@ -34,6 +39,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 METRIC = "fwd+bwd iterations/s and HBM GB/s vs roofline at 1M Gaussians, 1920x1080"
+RENDER_METRIC = "forward rendering frames/s"
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 # FP32 lanes per SM and SMs of a B200; the ALU roofline uses the max SM clock
 FP32_LANES_PER_SM = 128
@@ -67,10 +73,9 @@ def make_workload(name: str, views: int = 16):
     if name == "mixture":
         return scenes.mixture1m()
     if name == "box":
-        wl = scenes.box100k(poses=16)
-        return wl
+        return scenes.box100k(poses=100)     # forward only, timed over the 100 poses
     if name == "city":
-        return scenes.city3m(poses=4)
+        return scenes.city3m(poses=50)       # forward only, timed over the 50 poses
     if name == "tiny":
         wl = scenes.tiny()
         wl.targets = [np.full((128, 128, 3), 0.5, np.float32)]
@@ -227,26 +232,148 @@ def run_reference(args, world, rank):
         return 0
     wl = make_workload(args.workload, args.views)
     fraction = args.cpu_fraction
+    render = args.workload in ("box", "city")
+    sample = cpu_oracle_render_sample if render else cpu_oracle_sample
     vals = []
     per_iter = threads = desc = None
     for i in range(args.warmup + args.steps):
-        per_iter, threads, desc = cpu_oracle_sample(wl, fraction, seed=i)
+        per_iter, threads, desc = sample(wl, fraction, seed=i)
         if i >= args.warmup:
             vals.append(per_iter)
     sec = statistics.mean(vals)
     value = 1.0 / sec
-    line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": args.gpus, "steps": args.steps,
+    unit = "frames/s" if render else "iterations/s"
+    line = {"metric": RENDER_METRIC if render else METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": wl.name, "gaussians": wl.scene.n, "views_per_step": len(wl.cameras)},
-            "cpu_baseline": {"value": value, "unit": "iterations/s", "cores": threads, "kind": "oracle",
-                             "sample": desc},
-            "e2e": {"value": value, "unit": "iterations/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ----------------------------------------------------------------------- our arm
+
+def cpu_oracle_render_sample(wl, fraction: float, seed: int = 0):
+    """The oracle's forward pass on a bounded sample of one pose (projection and keys
+    of all Gaussians, compositing of a fraction of the tiles), scaled to one frame."""
+    import oracle
+    threads = oracle.set_threads(0)
+    rng = np.random.default_rng(seed)
+    scene, cam = wl.scene, wl.cameras[0]
+    W, H = cam["width"], cam["height"]
+    tx, ty = (W + 15) // 16, (H + 15) // 16
+    ntiles = max(1, int(round(fraction * tx * ty)))
+    tiles = rng.choice(tx * ty, ntiles, replace=False)
+    pix = np.concatenate([[(t // tx) * 16 * W + (t % tx) * 16 + yy * W + xx for yy in range(16) for xx in range(16)
+                           if (t // tx) * 16 + yy < H and (t % tx) * 16 + xx < W] for t in tiles]).astype(np.int64)
+    t0 = time.perf_counter()
+    proj = oracle.project(scene, cam)
+    oracle.keys(proj, cam)
+    t_all = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.render(proj, cam, pix=pix)
+    t_pix = time.perf_counter() - t0
+    per_frame = t_all + t_pix * (tx * ty) / ntiles
+    desc = (f"1 pose: projection+sort of all {scene.n} Gaussians, compositing of {ntiles} of {tx * ty} tiles, "
+            f"scaled to the whole frame")
+    return per_frame, threads, desc
+
+
+def run_render(args, world, rank, local):
+    """Forward-only workloads (the 100k box at 1080p over 100 poses, the 3M city at
+    4K over 50 poses): one step renders every pose once (projection, binning,
+    compositing); the metric is frames/s."""
+    import torch
+
+    from gaussian_splatting_differentiable_02_b200 import abi
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    abi.lib()
+    wl = make_workload(args.workload, args.views)
+    scene, cams = wl.scene, wl.cameras
+    g = pl.Gaussians.from_scene(scene)
+    view = pl.View(scene.n, cams[0])
+    proj = pl.Projected(scene.n)
+    stream = torch.cuda.current_stream()
+    # size the instance buffers for the largest pose
+    for cam in cams:
+        view.set_camera(cam)
+        pl.project(g, view, proj)
+        pl.bin_sort(proj, view)
+    counter = torch.zeros((len(cams),), device=g.means.device, dtype=torch.int64)
+    fwd_ev = []
+
+    def frame(k, cam, record):
+        view.set_camera(cam)
+        pl.project(g, view, proj)
+        pl.bin_sort_async(proj, view, counter[k:k + 1])
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        pl.raster_fwd(proj, view)
+        if record:
+            e1.record(stream)
+            fwd_ev.append((e0, e1))
+
+    for _ in range(args.warmup):
+        for k, cam in enumerate(cams):
+            frame(k, cam, False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    barrier(world)
+    launches0 = abi.gs_kernel_launches()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        for k, cam in enumerate(cams):
+            frame(k, cam, True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = abi.gs_kernel_launches() - launches0
+    barrier(world)
+    clk = clocks.stop()
+    if any(K > view.capacity for K in counter.cpu().tolist()):
+        raise RuntimeError("instance buffers overflowed after the warm-up")
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    frames = args.steps * len(cams)
+    # compositing pairs of the last pose's frame for the ALU roofline of raster_fwd
+    pairs = int(view.n_contrib.sum().item())
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev[-len(cams):])
+    peaks = measured_peaks()
+    smax = clk.get("sm_max_mhz") or 1965.0
+    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
+    per_pair = FLOPS_ALPHA + FLOPS_FWD_BLEND
+    last_ms = fwd_ev[-1][0].elapsed_time(fwd_ev[-1][1])
+    achieved = pairs * per_pair / (last_ms * 1e-3) / 1e12
+    cam0 = cams[0]
+    line = {"metric": RENDER_METRIC, "value": world * frames / (ms / 1e3), "unit": "frames/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "gaussians": scene.n, "poses_per_step": len(cams),
+                       "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "a step renders every pose once; the instance lists of a pose exceed L2"},
+            "stages_ms_per_frame": {"raster_fwd": fwd_ms, "frame": ms / frames},
+            "roofline": {"kernel": "raster_fwd", "bound": "alu", "achieved": achieved, "peak": alu_peak,
+                         "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
+                         "work": f"{pairs} (pixel, entry) pairs x {per_pair} flops (last pose)",
+                         "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"},
+            "gpu_launches": int(launches), "clocks": clk,
+            "e2e": None, "hbm_peak_gbs": peaks["hbm_gbs"]}
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        per_frame, threads, desc = cpu_oracle_render_sample(wl, args.cpu_fraction)
+        line["cpu_baseline"] = {"value": 1.0 / per_frame, "unit": "frames/s", "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
 
 def run_ours(args, world, rank, local):
     import torch
@@ -739,6 +866,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.workload in ("box", "city"):
+            return run_render(args, world, rank, local)
         return run_ours(args, world, rank, local)
     finally:
         if world > 1:

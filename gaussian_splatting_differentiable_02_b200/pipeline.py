@@ -174,6 +174,13 @@ class View:
         self.capacity = 0
         self._alloc(max(capacity, 4 * n, 1024))
 
+    def set_camera(self, cam: dict):
+        """Another pose of the same image size (the tile grid and the buffers stay)."""
+        if (cam["width"], cam["height"]) != (self.cam["width"], self.cam["height"]):
+            raise ValueError("set_camera keeps the image size")
+        self.cam = cam
+        self.gcam = abi.make_camera(cam)
+
     def set_n(self, n: int):
         """Resize for a new Gaussian count (after densification): the sort workspace depends on n."""
         self.n = int(n)
