@@ -249,7 +249,11 @@ gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint3
  * d = (u, v) - pixel centre; entries with sigma < 0 are skipped;
  * alpha = min(0.99, o exp(-sigma)); entries with alpha < 1/255 are skipped; if
  * T (1 - alpha) < 1e-4 the pixel stops without blending that entry; otherwise
- * C += rgb alpha T and T *= 1 - alpha.
+ * C += rgb alpha T and T *= 1 - alpha.  sigma is evaluated in float32, for
+ * conics with an eigenvalue ratio above 8 in the factored form
+ * 1/2 A t^2 + 1/2 (det/A) dy^2, t = dx + (B/A) dy, which keeps a few ulps of
+ * relative accuracy at any ratio; for a positive-definite conic sigma >= 0
+ * holds and is not tested.
  *   tile_order  optional processing order from gs_tile_order (NULL: tile order)
  *   image   [H][W][3] = C + T bg (bg_host: 3 floats read during the call)
  *   final_T [H][W]    transmittance after the last blended entry
