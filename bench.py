@@ -489,7 +489,8 @@ def run_ours(args, world, rank, local):
     with_oracle = rank == 0 and not args.no_cpu_baseline and world == 1
     line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
                     "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
-                    "absgrad_and_sparse_adam": measure_variants(tr, torch)}
+                    "absgrad_and_sparse_adam": measure_variants(tr, torch),
+                    "packed": measure_packed(tr, wl, peaks, torch)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
         line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
@@ -535,6 +536,60 @@ def measure_variants(tr, torch, reps: int = 10):
             lambda: pl.project_bwd_views_adam(g, tr.views, tr.proj, tr.radii, tr.grad2ds, m, v, tr.lrs,
                                               tr.step_count + 1, sparse=sparse))
     res["visible_fraction"] = float((tr.radii > 0).any(dim=0).float().mean().item())
+    return res
+
+
+def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
+    """The packed layout (gs_project_packed): the training step with packed views against
+    the same step unpacked (CUDA events over `steps` steps each, after 3 warm-up steps of
+    the packed Trainer), and the packed projection of the first view against the plain
+    projection, with the HBM roofline of its algorithmic bytes (the projection's bytes as
+    in step_bytes, the visibility read twice and the slot map written, and the visible
+    Gaussians' 52 bytes of features read, written packed, and their ids written)."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    s = torch.cuda.current_stream()
+    scene = wl.scene
+    trp = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
+                     dict(tr.lrs), densify=True, streams=tr.streams, packed=True)
+
+    def step_ms(t):
+        for _ in range(3):
+            t.step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            t.step()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    res = {"step_ms_packed": step_ms(trp), "step_ms_unpacked": step_ms(tr)}
+    visible = trp.counts[1].cpu().numpy()
+    res["visible_fraction_per_view"] = float(visible.mean() / max(scene.n, 1))
+    res["slot_capacity"] = int(trp.pcap)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    view = trp.views[0]
+    res["project_ms"] = timed(lambda: pl.project(tr.gauss, tr.views[0], tr.projs[0], tr.radii[0]))
+    ms = timed(lambda: pl.project_packed(trp.gauss, view, trp.packs[0], trp.pack_ws))
+    res["project_packed_ms"] = ms
+    n, V = scene.n, int(visible[0])
+    pb = 4 * (11 + 3 * (scene.sh_degree + 1) ** 2)
+    nbytes = n * (pb + 52) + n * 12 + V * (52 + 52 + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res["project_packed_roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                      "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes}
+    del trp
     return res
 
 

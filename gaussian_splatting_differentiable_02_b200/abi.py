@@ -103,6 +103,18 @@ SIGNATURES = {
                                               C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float, C.c_float,
                                               C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P, _P, _P, C.c_int32,
                                               _P]),
+    "gs_project_packed_workspace_bytes": (C.c_size_t, [C.c_int64]),
+    "gs_project_packed": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), _P, C.c_size_t,
+                                      C.POINTER(gs_projected), C.c_int64, _P, _P, _P, _P]),
+    "gs_project_bwd_views_packed": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
+                                                C.POINTER(gs_projected), C.POINTER(_P), C.POINTER(gs_grad2d),
+                                                C.POINTER(gs_param_grads), _P, _P, _P, _P]),
+    "gs_project_bwd_views_adam_packed": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
+                                                     C.POINTER(gs_projected), C.POINTER(_P), C.POINTER(gs_grad2d),
+                                                     C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
+                                                     C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float,
+                                                     C.c_float, C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P,
+                                                     _P, _P, C.c_int32, _P]),
     "gs_l1_dssim_workspace_bytes": (C.c_size_t, [C.c_int32, C.c_int32]),
     "gs_l1_dssim_loss_grad": (C.c_int32, [_P, _P, C.c_int32, C.c_int32, C.c_float, C.c_float, _P, C.c_size_t, _P, _P,
                                           _P]),
@@ -297,6 +309,50 @@ def gs_project_bwd_views_adam(params: gs_params, cams, projs, grad2ds, params_in
         C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _arr(gs_grad2d, grad2ds),
         C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps, step,
         C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None,
+        densify_max_radius or None, int(sparse_adam), stream))
+
+
+def gs_project_packed_workspace_bytes(n: int) -> int:
+    return lib().gs_project_packed_workspace_bytes(n)
+
+
+def gs_project_packed(params: gs_params, cam: gs_camera, workspace: int, workspace_bytes: int,
+                      packed: gs_projected, capacity: int, gaussian_ids: int, slot_of: int, num_visible_dev: int,
+                      stream: int = 0):
+    """The packed projection: packed arrays of `capacity` slots, their Gaussian ids, the slot of every
+    Gaussian, the visible count on the device."""
+    return _check(lib().gs_project_packed(C.byref(params), C.byref(cam), workspace, workspace_bytes,
+                                          C.byref(packed), capacity, gaussian_ids or None, slot_of or None,
+                                          num_visible_dev, stream))
+
+
+def _slots(slot_of):
+    return _arr(_P, [int(p) for p in slot_of])
+
+
+def gs_project_bwd_views_packed(params: gs_params, cams, projs, slot_of, grad2ds, grads: gs_param_grads,
+                                densify_accum: int = 0, densify_count: int = 0, densify_max_radius: int = 0,
+                                stream: int = 0):
+    """gs_project_bwd_views for packed views; slot_of: one device pointer per view."""
+    V = len(cams)
+    return _check(lib().gs_project_bwd_views_packed(C.byref(params), V, _arr(gs_camera, cams),
+                                                    _arr(gs_projected, projs), _slots(slot_of),
+                                                    _arr(gs_grad2d, grad2ds), C.byref(grads), densify_accum or None,
+                                                    densify_count or None, densify_max_radius or None, stream))
+
+
+def gs_project_bwd_views_adam_packed(params: gs_params, cams, projs, slot_of, grad2ds, params_inout: gs_param_grads,
+                                     adam_m: gs_param_grads, adam_v: gs_param_grads, lrs, beta1: float, beta2: float,
+                                     eps: float, step: int, grads: gs_param_grads = None, densify_accum: int = 0,
+                                     densify_count: int = 0, densify_max_radius: int = 0, sparse_adam: int = 0,
+                                     stream: int = 0):
+    """gs_project_bwd_views_adam for packed views; slot_of: one device pointer per view."""
+    V = len(cams)
+    lr = (C.c_float * 5)(*[float(x) for x in lrs])
+    return _check(lib().gs_project_bwd_views_adam_packed(
+        C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _slots(slot_of),
+        _arr(gs_grad2d, grad2ds), C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps,
+        step, C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None,
         densify_max_radius or None, int(sparse_adam), stream))
 
 

@@ -356,7 +356,8 @@ gs_status check_grad_arrays(const char* fn, const gs_param_grads* g, const char*
 gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t num_views, const gs_camera* cams,
                              const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* grads,
                              float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
-                             const gsk::AdamStep* adam, void* stream) {
+                             const gsk::AdamStep* adam, void* stream, const int32_t* const* slots = nullptr,
+                             bool packed = false) {
     gs_status st;
     if ((st = check_params(fn, params)) != GS_OK) return st;
     if (num_views < 1 || num_views > GS_MAX_VIEWS)
@@ -370,6 +371,10 @@ gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t nu
         if ((st = check_camera(fn, cams + v)) != GS_OK) return st;
         c[v] = gsk::make_cam(cams[v]);
         if (params->n > 0) {
+            if (packed) {
+                if (!slots) return fail(GS_ERR_INVALID_ARG, "%s: slot_of is NULL", fn);
+                CHECK_PTR(slots[v], 4);
+            }
             CHECK_PTR(projs[v].radius, 4);
             CHECK_PTR(grad2d[v].xy, 8);
             CHECK_PTR(grad2d[v].conic_opacity, 16);
@@ -390,7 +395,8 @@ gs_status project_bwd_common(const char* fn, const gs_params* params, int32_t nu
             if ((st = check_grad_arrays(fn, adam->v, "adam_v")) != GS_OK) return st;
         }
     }
-    return cuda_status(gsk::launch_project_bwd_views(*params, num_views, c, cams, projs, grad2d, grads, densify_accum,
+    return cuda_status(gsk::launch_project_bwd_views(*params, num_views, c, cams, projs, packed ? slots : nullptr,
+                                                     grad2d, grads, densify_accum,
                                                      densify_count, densify_max_radius, adam,
                                                      static_cast<cudaStream_t>(stream)),
                        fn);
@@ -426,13 +432,16 @@ gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const
                               densify_max_radius, nullptr, stream);
 }
 
-gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
-                                    const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
-                                    gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
-                                    float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
-                                    float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
-                                    int32_t sparse_adam, void* stream) {
-    const char* fn = "gs_project_bwd_views_adam";
+}  // extern "C"
+
+namespace {
+
+gs_status project_bwd_adam_common(const char* fn, const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                  const gs_projected* projs, const int32_t* const* slots, bool packed,
+                                  const gs_grad2d* grad2d, gs_param_grads* params_inout, gs_param_grads* adam_m,
+                                  gs_param_grads* adam_v, const float* lr_host, float beta1, float beta2, float eps,
+                                  int32_t step, gs_param_grads* grads, float* densify_accum, int32_t* densify_count,
+                                  int32_t* densify_max_radius, int32_t sparse_adam, void* stream) {
     if (sparse_adam != 0 && sparse_adam != 1) return fail(GS_ERR_INVALID_ARG, "%s: sparse_adam must be 0 or 1", fn);
     if (!lr_host) return fail(GS_ERR_INVALID_ARG, "%s: lr_host is NULL", fn);
     gsk::AdamStep a;
@@ -453,7 +462,74 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
     a.step = step;
     a.sparse = sparse_adam == 1;
     return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
-                              densify_max_radius, &a, stream);
+                              densify_max_radius, &a, stream, slots, packed);
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                    const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
+                                    gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                    float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                    float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                    int32_t sparse_adam, void* stream) {
+    return project_bwd_adam_common("gs_project_bwd_views_adam", params, num_views, cams, projs, nullptr, false,
+                                   grad2d, params_inout, adam_m, adam_v, lr_host, beta1, beta2, eps, step, grads,
+                                   densify_accum, densify_count, densify_max_radius, sparse_adam, stream);
+}
+
+gs_status gs_project_bwd_views_adam_packed(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                           const gs_projected* projs, const int32_t* const* slot_of,
+                                           const gs_grad2d* grad2d, gs_param_grads* params_inout,
+                                           gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                           float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                           float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                           int32_t sparse_adam, void* stream) {
+    return project_bwd_adam_common("gs_project_bwd_views_adam_packed", params, num_views, cams, projs, slot_of, true,
+                                   grad2d, params_inout, adam_m, adam_v, lr_host, beta1, beta2, eps, step, grads,
+                                   densify_accum, densify_count, densify_max_radius, sparse_adam, stream);
+}
+
+gs_status gs_project_bwd_views_packed(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                      const gs_projected* projs, const int32_t* const* slot_of,
+                                      const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
+                                      int32_t* densify_count, int32_t* densify_max_radius, void* stream) {
+    const char* fn = "gs_project_bwd_views_packed";
+    if (!grads) return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL", fn);
+    return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
+                              densify_max_radius, nullptr, stream, slot_of, true);
+}
+
+size_t gs_project_packed_workspace_bytes(int64_t n) {
+    if (n < 0) n = 0;
+    return gsk::pack_workspace_layout(n, nullptr, nullptr);
+}
+
+gs_status gs_project_packed(const gs_params* params, const gs_camera* cam, void* workspace, size_t workspace_bytes,
+                            gs_projected* packed, int64_t capacity, uint32_t* gaussian_ids, int32_t* slot_of,
+                            uint64_t* num_visible_dev, void* stream) {
+    const char* fn = "gs_project_packed";
+    gs_status st;
+    if ((st = check_params(fn, params)) != GS_OK) return st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if (capacity < 0 || capacity > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: capacity out of range", fn);
+    if ((st = check_projected(fn, packed, capacity, true)) != GS_OK) return st;
+    CHECK_PTR(num_visible_dev, 8);
+    CHECK_PTR(workspace, 16);
+    if (capacity > 0) CHECK_PTR(gaussian_ids, 4);
+    if (params->n > 0) CHECK_PTR(slot_of, 4);
+    const size_t need = gsk::pack_workspace_layout(params->n, nullptr, nullptr);
+    if (workspace_bytes < need)
+        return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
+    gsk::PackWorkspace ws;
+    gsk::pack_workspace_layout(params->n, workspace, &ws);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_project_packed(*params, c, ws, *packed, capacity, gaussian_ids, slot_of,
+                                                  reinterpret_cast<unsigned long long*>(num_visible_dev),
+                                                  static_cast<cudaStream_t>(stream)),
+                       fn);
 }
 
 size_t gs_l1_dssim_workspace_bytes(int32_t width, int32_t height) {

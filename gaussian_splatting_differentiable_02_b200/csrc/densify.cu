@@ -8,7 +8,8 @@
 // Three launches:
 //   plan     one block per contiguous chunk of Gaussians: decision per
 //            Gaussian (uint8), and the chunk's output count;
-//   offsets  one block: exclusive scan of the chunk counts, the total;
+//   offsets  one block: exclusive scan of the chunk counts, the total
+//            (compact.cuh);
 //   apply    the same chunks: block-wide scan of the per-Gaussian output counts
 //            gives every Gaussian its output slot; parameters and moments are
 //            copied (keep, clone), or the two split children are written.
@@ -16,28 +17,16 @@
 // the parameters and both moments (3 x 236 bytes at SH degree 3) in and out.
 #include <cuda_runtime.h>
 
+#include "compact.cuh"
 #include "internal.cuh"
 
 namespace gsk {
 namespace {
 
-constexpr int kBlock = 128;
-constexpr int kMaxChunks = kNumSMs * 8;
-
-struct Chunking {
-    int64_t chunk;  // Gaussians per block, a multiple of kBlock
-    int blocks;
-};
-
-Chunking chunking(int64_t n) {
-    int64_t tiles = (n + kBlock - 1) / kBlock;
-    int64_t blocks = tiles < kMaxChunks ? tiles : kMaxChunks;
-    if (blocks < 1) blocks = 1;
-    const int64_t tiles_per_block = (tiles + blocks - 1) / blocks;
-    blocks = tiles_per_block > 0 ? (tiles + tiles_per_block - 1) / tiles_per_block : 1;
-    if (blocks < 1) blocks = 1;
-    return {tiles_per_block * kBlock, int(blocks)};
-}
+using compact::block_inclusive_scan;
+using compact::chunking;
+using compact::Chunking;
+using compact::kBlock;
 
 struct PlanArgs {
     const float* logits;
@@ -71,32 +60,6 @@ __device__ __forceinline__ int decide(const PlanArgs& a, int64_t i) {
 
 __device__ __forceinline__ int outputs_of(int d) { return d == GS_DENSIFY_PRUNE ? 0 : (d == GS_DENSIFY_KEEP ? 1 : 2); }
 
-// Inclusive block-wide sum scan of one value per thread (kBlock threads).
-__device__ __forceinline__ unsigned block_inclusive_scan(unsigned x, unsigned* warp_tot, unsigned& block_total) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, x, d);
-        if (lane >= d) x += y;
-    }
-    if (lane == 31) warp_tot[w] = x;
-    __syncthreads();
-    if (w == 0) {
-        unsigned t = lane < kBlock / 32 ? warp_tot[lane] : 0u;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const unsigned y = __shfl_up_sync(0xffffffffu, t, d);
-            if (lane >= d) t += y;
-        }
-        if (lane < kBlock / 32) warp_tot[lane] = t;
-    }
-    __syncthreads();
-    const unsigned before = w > 0 ? warp_tot[w - 1] : 0u;
-    block_total = warp_tot[kBlock / 32 - 1];
-    __syncthreads();
-    return x + before;
-}
-
 __global__ void __launch_bounds__(kBlock) densify_plan_kernel(const PlanArgs a) {
     __shared__ unsigned warp_tot[kBlock / 32];
     const int64_t begin = int64_t(blockIdx.x) * a.chunk;
@@ -115,37 +78,6 @@ __global__ void __launch_bounds__(kBlock) densify_plan_kernel(const PlanArgs a) 
         total += tile_total;
     }
     if (threadIdx.x == 0) a.chunk_counts[blockIdx.x] = total;
-}
-
-// Exclusive scan of the chunk counts in place (one block of 1024 threads, each
-// owning a contiguous run), the total to *total and *total_copy.
-__global__ void __launch_bounds__(1024) densify_offsets_kernel(unsigned long long* counts, int nb,
-                                                               unsigned long long* total,
-                                                               unsigned long long* total_copy) {
-    __shared__ unsigned long long part[1024];
-    const int per = (nb + 1023) / 1024;
-    const int b0 = threadIdx.x * per;
-    const int b1 = b0 + per < nb ? b0 + per : nb;
-    unsigned long long s = 0;
-    for (int b = b0; b < b1; ++b) s += counts[b];
-    part[threadIdx.x] = s;
-    __syncthreads();
-    for (int d = 1; d < 1024; d <<= 1) {
-        const unsigned long long y = threadIdx.x >= d ? part[threadIdx.x - d] : 0ull;
-        __syncthreads();
-        part[threadIdx.x] += y;
-        __syncthreads();
-    }
-    unsigned long long run = part[threadIdx.x] - s;
-    for (int b = b0; b < b1; ++b) {
-        const unsigned long long c = counts[b];
-        counts[b] = run;
-        run += c;
-    }
-    if (threadIdx.x == 1023) {
-        *total = part[1023];
-        if (total_copy) *total_copy = part[1023];
-    }
 }
 
 struct Group {  // one set of parameter-shaped arrays
@@ -296,14 +228,13 @@ OutGroup out_group_of(const gs_param_grads& g) {
 
 size_t densify_workspace_layout(int64_t n, void* base, DensifyWorkspace* ws) {
     const Chunking ch = chunking(n);
-    const size_t bytes = (size_t(ch.blocks) + 1) * sizeof(unsigned long long);
     if (ws) {
         ws->chunk_counts = static_cast<unsigned long long*>(base);
         ws->total = ws->chunk_counts + ch.blocks;
         ws->blocks = ch.blocks;
         ws->chunk = ch.chunk;
     }
-    return (bytes + 255) & ~size_t(255);
+    return compact::workspace_bytes(n);
 }
 
 cudaError_t launch_densify_plan(const gs_params& p, const float* accum, const int32_t* count,
@@ -330,7 +261,7 @@ cudaError_t launch_densify_plan(const gs_params& p, const float* accum, const in
     } else {
         cudaMemsetAsync(ws.chunk_counts, 0, sizeof(unsigned long long) * ws.blocks, s);
     }
-    densify_offsets_kernel<<<1, 1024, 0, s>>>(ws.chunk_counts, ws.blocks, ws.total,
+    compact::chunk_offsets_kernel<<<1, 1024, 0, s>>>(ws.chunk_counts, ws.blocks, ws.total,
                                               reinterpret_cast<unsigned long long*>(num_out_dev));
     count_launches(1);
     return cudaGetLastError();

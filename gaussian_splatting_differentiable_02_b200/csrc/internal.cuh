@@ -56,10 +56,27 @@ struct AdamStep {
     bool sparse;  // skip Gaussians visible in no view (parameters and moments untouched)
 };
 
+// The packed projection: every Gaussian projected into `full` (workspace), then
+// the visible ones compacted in ascending order into `capacity` packed slots.
+struct PackWorkspace {
+    gs_projected full;                 // [n] projection of every Gaussian
+    unsigned long long* chunk_counts;  // [blocks]
+    unsigned long long* total;         // [1] visible count
+    int blocks;
+    int64_t chunk;
+};
+size_t pack_workspace_layout(int64_t n, void* base, PackWorkspace* ws);
+cudaError_t launch_project_packed(const gs_params& p, const CamArgs& cam, const PackWorkspace& ws,
+                                  const gs_projected& packed, int64_t capacity, uint32_t* ids, int32_t* slot_of,
+                                  unsigned long long* num_visible_dev, cudaStream_t s);
+
 // Backward through the projection for V <= GS_MAX_VIEWS views of the same
-// Gaussians; grads (+=) may be null when adam is given.
+// Gaussians; grads (+=) may be null when adam is given.  slots: null (projs and
+// g2d indexed by Gaussian), or per view the slot of every Gaussian in the packed
+// projs and g2d (-1: not in the view).
 cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* cams, const gs_camera* raw,
-                                     const gs_projected* projs, const gs_grad2d* g2d, const gs_param_grads* grads,
+                                     const gs_projected* projs, const int32_t* const* slots, const gs_grad2d* g2d,
+                                     const gs_param_grads* grads,
                                      float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
                                      const AdamStep* adam, cudaStream_t s);
 

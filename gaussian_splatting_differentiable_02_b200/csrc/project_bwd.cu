@@ -11,7 +11,9 @@
 // values), dL/dmean, dL/dlogit and the 48 SH gradients, all held in registers;
 // the chain from dL/dSigma to the scales and the quaternion runs once at the end.
 // With Adam fused the gradients never reach memory: parameters, moments and the
-// views' 2D gradients each make exactly one pass through HBM.
+// views' 2D gradients each make exactly one pass through HBM.  In the packed
+// layout (gs_project_packed) a view's features and 2D gradients are read at the
+// Gaussian's slot, found through the view's slot map.
 //
 // The geometric chain is double precision: the inverse of a 2x2 conic and the
 // EWA product are badly conditioned for needle-shaped Gaussians.  The colour
@@ -38,6 +40,7 @@ constexpr int kBwdBlock = 128;
 struct ViewArgs {
     double limx, limy, cc[3], eps2d;
     float R[9], t[3], fx, fy;
+    const int32_t* slot;  // packed layout: entry of each Gaussian (-1: none); else null
     const int32_t* radius;
     const float2* g_xy;
     const float2* g_xy_abs;  // absolute 2D gradient for the densification statistic (nullable)
@@ -158,11 +161,18 @@ __device__ __forceinline__ void add4(float4* d, int64_t i, float4 g) {
     d[i] = make_float4(x.x + g.x, x.y + g.y, x.z + g.z, x.w + g.w);
 }
 
+// Index of Gaussian i's entry in a view's projected features and 2D gradients:
+// i itself, or its slot in the packed layout.
+template <bool kPacked>
+__device__ __forceinline__ int64_t entry(const ViewArgs& w, int64_t i) {
+    return kPacked ? int64_t(__ldg(w.slot + i)) : i;
+}
+
 #ifndef GS_PBWD_MIN_BLOCKS
 #define GS_PBWD_MIN_BLOCKS 2
 #endif
 
-template <bool kAdam>
+template <bool kAdam, bool kPacked>
 __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_kernel(const Args a) {
     __shared__ float shs[48][kBwdBlock];  // this thread's SH coefficients, column threadIdx.x
     const int t = threadIdx.x;
@@ -170,7 +180,8 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
         unsigned vis = 0u;
         int rmax = 0;
         for (int v = 0; v < a.V; ++v) {
-            const int r = __ldg(a.view[v].radius + i);
+            const int64_t j = entry<kPacked>(a.view[v], i);
+            const int r = j >= 0 ? __ldg(a.view[v].radius + j) : 0;
             if (r > 0) vis |= 1u << v;
             rmax = max(rmax, r);
         }
@@ -181,9 +192,10 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
         // visible views' 2D gradients, the Adam moments) starts moving into L2 now
         for (unsigned rest = vis; rest; rest &= rest - 1u) {
             const ViewArgs& w = a.view[__ffs(rest) - 1];
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_xy + i));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_con + i));
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_rgb + i));
+            const int64_t j = entry<kPacked>(w, i);
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_xy + j));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_con + j));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(w.g_rgb + j));
         }
         if (kAdam) {
             asm volatile("prefetch.global.L2 [%0];" ::"l"(a.m_means + i));
@@ -249,20 +261,23 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
             // visible views in order; the next view's 2D gradients are loaded while
             // the current one is processed
             int v = __ffs(vis) - 1;
-            float2 nxy = __ldg(a.view[v].g_xy + i);
-            float4 nco = __ldg(a.view[v].g_con + i);
-            float4 nrg = __ldg(a.view[v].g_rgb + i);
+            int64_t nj = entry<kPacked>(a.view[v], i);
+            float2 nxy = __ldg(a.view[v].g_xy + nj);
+            float4 nco = __ldg(a.view[v].g_con + nj);
+            float4 nrg = __ldg(a.view[v].g_rgb + nj);
             while (v >= 0) {
                 const ViewArgs& cam = a.view[v];
                 const float2 gxy = nxy;
                 const float4 gco = nco;
                 const float4 grg = nrg;
+                const int64_t cj = nj;
                 const unsigned rest = vis & ~((2u << v) - 1u);
                 const int vn = rest ? __ffs(rest) - 1 : -1;
                 if (vn >= 0) {
-                    nxy = __ldg(a.view[vn].g_xy + i);
-                    nco = __ldg(a.view[vn].g_con + i);
-                    nrg = __ldg(a.view[vn].g_rgb + i);
+                    nj = entry<kPacked>(a.view[vn], i);
+                    nxy = __ldg(a.view[vn].g_xy + nj);
+                    nco = __ldg(a.view[vn].g_con + nj);
+                    nrg = __ldg(a.view[vn].g_rgb + nj);
                 }
                 const double fx = cam.fx, fy = cam.fy;
                 double pc[3];
@@ -389,7 +404,7 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
                 gmu[1] += (gdir[1] - uy * dproj) / dn;
                 gmu[2] += (gdir[2] - uz * dproj) / dn;
 
-                const float2 sxy = cam.g_xy_abs ? __ldg(cam.g_xy_abs + i) : gxy;
+                const float2 sxy = cam.g_xy_abs ? __ldg(cam.g_xy_abs + cj) : gxy;
                 dacc += sqrtf(sxy.x * sxy.x + sxy.y * sxy.y);
                 dcnt += 1;
                 v = vn;
@@ -467,8 +482,8 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
     }
 }
 
-void fill_views(Args& a, const CamArgs* cams, const gs_projected* projs, const gs_grad2d* g2d, int V,
-                const gs_camera* raw) {
+void fill_views(Args& a, const CamArgs* cams, const gs_projected* projs, const int32_t* const* slots,
+                const gs_grad2d* g2d, int V, const gs_camera* raw) {
     a.V = V;
     for (int v = 0; v < V; ++v) {
         ViewArgs& w = a.view[v];
@@ -480,6 +495,7 @@ void fill_views(Args& a, const CamArgs* cams, const gs_projected* projs, const g
         for (int j = 0; j < 3; ++j) w.t[j] = raw[v].t[j];
         w.fx = raw[v].fx;
         w.fy = raw[v].fy;
+        w.slot = slots ? slots[v] : nullptr;
         w.radius = projs[v].radius;
         w.g_xy = reinterpret_cast<const float2*>(g2d[v].xy);
         w.g_xy_abs = reinterpret_cast<const float2*>(g2d[v].xy_abs);
@@ -510,13 +526,14 @@ void fill_grads(float4*& m, float4*& q, float4*& l, float*& o, float4*& s, const
 }  // namespace
 
 cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* cams, const gs_camera* raw,
-                                     const gs_projected* projs, const gs_grad2d* g2d, const gs_param_grads* grads,
+                                     const gs_projected* projs, const int32_t* const* slots, const gs_grad2d* g2d,
+                                     const gs_param_grads* grads,
                                      float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
                                      const AdamStep* adam, cudaStream_t s) {
     if (p.n == 0) return cudaSuccess;
     Args a;
     fill_params(a, p);
-    fill_views(a, cams, projs, g2d, V, raw);
+    fill_views(a, cams, projs, slots, g2d, V, raw);
     fill_grads(a.d_means, a.d_quats, a.d_log_scales, a.d_logits, a.d_sh, grads);
     a.densify_accum = densify_accum;
     a.densify_count = densify_count;
@@ -534,9 +551,14 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
         a.b1 = adam->beta1;
         a.b2 = adam->beta2;
         a.eps = adam->eps;
-        project_bwd_kernel<true><<<grid, kBwdBlock, 0, s>>>(a);
+        if (slots)
+            project_bwd_kernel<true, true><<<grid, kBwdBlock, 0, s>>>(a);
+        else
+            project_bwd_kernel<true, false><<<grid, kBwdBlock, 0, s>>>(a);
+    } else if (slots) {
+        project_bwd_kernel<false, true><<<grid, kBwdBlock, 0, s>>>(a);
     } else {
-        project_bwd_kernel<false><<<grid, kBwdBlock, 0, s>>>(a);
+        project_bwd_kernel<false, false><<<grid, kBwdBlock, 0, s>>>(a);
     }
     count_launches(1);
     return cudaGetLastError();

@@ -153,6 +153,32 @@ class Grad2D:
                                self.rgb[:, :3].cpu().numpy()], axis=1)
 
 
+class Packed:
+    """One view's projection in the packed layout (gs_project_packed, the gsplat guide §4.1
+    packed option): `capacity` slots of projected features (`proj`), the Gaussian of every
+    slot (`ids`), the slot of every Gaussian (`slot_of`, -1: not in the view) and the number
+    of Gaussians the view keeps (`num_visible`, on the device)."""
+
+    def __init__(self, n: int, capacity: int, device="cuda", num_visible: torch.Tensor = None):
+        self.n, self.capacity = int(n), int(capacity)
+        self.proj = Projected(self.capacity, device)
+        self.ids = torch.zeros((max(self.capacity, 1),), device=device, dtype=torch.int32)
+        self.slot_of = torch.zeros((max(self.n, 1),), device=device, dtype=torch.int32)
+        self.num_visible = torch.zeros((1,), device=device, dtype=torch.int64) if num_visible is None \
+            else num_visible
+
+
+def project_packed_workspace(n: int, device="cuda") -> torch.Tensor:
+    return torch.empty((abi.gs_project_packed_workspace_bytes(n),), device=device, dtype=torch.uint8)
+
+
+def project_packed(g: Gaussians, view: View, packed: Packed, workspace: torch.Tensor):
+    """gs_project_packed into `packed` (visible count left on the device)."""
+    abi.gs_project_packed(g.params(), view.gcam, _ptr(workspace), workspace.numel(), packed.proj.struct(),
+                          packed.capacity, _ptr(packed.ids), _ptr(packed.slot_of), _ptr(packed.num_visible),
+                          _stream())
+
+
 class View:
     """Per-camera buffers: sorted instances, tile ranges, image and its gradient."""
 
@@ -182,9 +208,16 @@ class View:
         self.gcam = abi.make_camera(cam)
 
     def set_n(self, n: int):
-        """Resize for a new Gaussian count (after densification): the sort workspace depends on n."""
+        """Resize for a new Gaussian (or packed slot) count: the sort workspace depends on n.
+        The instance buffers and their contents stay unless the capacity has to grow."""
         self.n = int(n)
-        self._alloc(max(self.capacity, 4 * self.n, 1024))
+        cap = max(self.capacity, 4 * self.n, 1024)
+        if cap != self.capacity:
+            self._alloc(cap)
+            return
+        nbytes = abi.gs_bin_sort_workspace_bytes(self.n, self.capacity, self.gcam)
+        if nbytes > self.workspace.numel():
+            self.workspace = torch.zeros((nbytes,), device=self.device, dtype=torch.uint8)
 
     def _alloc(self, capacity: int):
         self.capacity = int(capacity)
@@ -233,7 +266,8 @@ class DepthOrder:
 
 def depth_order_views(projs: list, radii: torch.Tensor, d: DepthOrder):
     """Every view's stable depth order in one batched sort (projs[k] with radius row radii[k])."""
-    abi.gs_depth_order_views([p.struct(radii[k]) for k, p in enumerate(projs)], d.n, _ptr(d.workspace),
+    abi.gs_depth_order_views([p.struct(None if radii is None else radii[k]) for k, p in enumerate(projs)], d.n,
+                             _ptr(d.workspace),
                              d.workspace.numel(), _ptr(d.order), _stream())
 
 
@@ -307,6 +341,18 @@ def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: to
         _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
+def project_bwd_views_adam_packed(g: Gaussians, views: list, packs: list, grad2ds: list, m: Gaussians, v: Gaussians,
+                                  lrs: dict, step: int, grads: Gaussians = None, densify_accum: torch.Tensor = None,
+                                  densify_count: torch.Tensor = None, betas=(0.9, 0.99), eps=1e-15,
+                                  densify_max_radius: torch.Tensor = None, sparse: bool = False):
+    """project_bwd_views_adam for views in the packed layout (packs[k]: view k's Packed)."""
+    abi.gs_project_bwd_views_adam_packed(
+        g.params(), [vw.gcam for vw in views], [pk.proj.struct() for pk in packs], [_ptr(pk.slot_of) for pk in packs],
+        [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES], betas[0],
+        betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum), _ptr(densify_count),
+        _ptr(densify_max_radius), int(sparse), _stream())
+
+
 # densify_and_prune parameters of the gsplat guide §4.1 (every 100 steps): gradient
 # threshold, minimum opacity, extent (read as the largest scale, in world units,
 # up to which a densified Gaussian is cloned rather than split) and maximum screen
@@ -368,16 +414,23 @@ class Trainer:
                                # view's sort overlaps another view's compositing
     batched_sort: bool = True  # fused path: project every view first and sort all views by depth in one
                                # batched sort (gs_depth_order_views), then bin and composite per view
+    packed: bool = False       # fused batched path: views in the packed layout (gs_project_packed, the
+                               # gsplat guide §4.1 packed option); the slot capacity follows the largest
+                               # visible count seen
 
     def __post_init__(self):
         n = self.gauss.n
         dev = self.gauss.means.device
         self.fused = self.fused and len(self.views) <= abi.GS_MAX_VIEWS
+        if self.packed and not (self.fused and self.batched_sort):
+            raise ValueError("packed=True runs on the fused path with the batched sort")
+        # per view: instance count and (packed) visible count, read back with one wait per step
+        self.counts = torch.zeros((2, len(self.views)), device=dev, dtype=torch.int64)
+        self.kcount = self.counts[0]
         self._alloc_per_gaussian(n)
         self.m = self.gauss.zeros_like()
         self.v = self.gauss.zeros_like()
         self.loss = torch.zeros((1,), device=dev, dtype=torch.float64)
-        self.kcount = torch.zeros((len(self.views),), device=dev, dtype=torch.int64)
         self.step_count = 0
         self.noise_gen = torch.Generator(device=dev)
         self.noise_gen.manual_seed(0)
@@ -387,23 +440,46 @@ class Trainer:
         gradients and densification statistics)."""
         dev = self.gauss.means.device
         nv = len(self.views) if self.fused else 1
-        self.proj = Projected(n, dev)
-        # concurrent views need their own projected features
-        if self.fused and self.batched_sort:
-            # every view's projection is kept until its binning
-            self.projs = [self.proj] + [Projected(n, dev) for _ in range(nv - 1)]
-            self.depth_order = DepthOrder(n, nv, dev)
+        if self.packed:
+            self.pack_ws = project_packed_workspace(n, dev)
+            self.radii = None
+            self._alloc_packed(n)
         else:
-            self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
-                if self.fused else [self.proj]
-            self.depth_order = None
-        self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
-        self.grad2d = self.grad2ds[0]
-        self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
+            self.proj = Projected(n, dev)
+            # concurrent views need their own projected features
+            if self.fused and self.batched_sort:
+                # every view's projection is kept until its binning
+                self.projs = [self.proj] + [Projected(n, dev) for _ in range(nv - 1)]
+                self.depth_order = DepthOrder(n, nv, dev)
+            else:
+                self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
+                    if self.fused else [self.proj]
+                self.depth_order = None
+            self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
+            self.grad2d = self.grad2ds[0]
+            self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
         self.grads = None if self.fused else self.gauss.zeros_like()
         self.densify_accum = torch.zeros((max(n, 1),), device=dev, dtype=torch.float32) if self.densify else None
         self.densify_count = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
         self.densify_max_radius = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
+
+    def _alloc_packed(self, capacity: int):
+        """Packed views of `capacity` slots: features, 2D gradients, depth order and sort buffers."""
+        dev = self.gauss.means.device
+        n, nv = self.gauss.n, len(self.views)
+        self.pcap = int(capacity)
+        self.packs = [Packed(n, self.pcap, dev, self.counts[1][k:k + 1]) for k in range(nv)]
+        self.projs = [pk.proj for pk in self.packs]
+        self.proj = self.projs[0]
+        self.depth_order = DepthOrder(self.pcap, nv, dev)
+        self.grad2ds = [Grad2D(self.pcap, dev, absgrad=self.absgrad) for _ in range(nv)]
+        self.grad2d = self.grad2ds[0]
+        for view in self.views:
+            view.set_n(self.pcap)
+
+    def _radius(self, k: int):
+        """View k's radius row (None: the packed projection's own)."""
+        return None if self.packed else self.radii[k if self.fused else 0]
 
     def densify_and_prune(self, **kw) -> torch.Tensor:
         """Adaptive density control from the statistics accumulated since the last call
@@ -482,7 +558,7 @@ class Trainer:
             with torch.cuda.stream(bin_stream):
                 for k, view in enumerate(self.views):
                     bin_sort_ordered_async(self.projs[k], view, self.depth_order.order[k], self.kcount[k:k + 1],
-                                           self.radii[k])
+                                           self._radius(k))
                     binned.append(bin_stream.record_event())
             for k, tgt in enumerate(targets):
                 st = side[k % len(side)]
@@ -513,7 +589,7 @@ class Trainer:
     def view_composite(self, k: int, target: torch.Tensor, proj: Projected) -> None:
         """raster forward -> loss -> raster backward of an already binned view k."""
         view = self.views[k]
-        r = self.radii[k]
+        r = self._radius(k)
         raster_fwd(proj, view, self.bg, r)
         if self.ssim_weight > 0.0:
             l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
@@ -530,9 +606,13 @@ class Trainer:
         return self._bin_stream
 
     def project_and_order(self) -> None:
-        """Every view's projection, then the batched depth sort of all views (current stream)."""
+        """Every view's projection (packed or not), then the batched depth sort of all views
+        (current stream)."""
         for k, view in enumerate(self.views):
-            project(self.gauss, view, self.projs[k], self.radii[k])
+            if self.packed:
+                project_packed(self.gauss, view, self.packs[k], self.pack_ws)
+            else:
+                project(self.gauss, view, self.projs[k], self.radii[k])
         depth_order_views(self.projs, self.radii, self.depth_order)
 
     def side_streams(self) -> list:
@@ -555,8 +635,14 @@ class Trainer:
                                 self.densify_count, radius=self.radii[0], densify_max_radius=self.densify_max_radius)
                 break
             self._all_views()
-            # one wait per step: every view's instance count against its capacity
-            counts = self.kcount.cpu().tolist()
+            # one wait per step: every view's instance count against its capacity (and in the
+            # packed layout its visible count against the slot capacity)
+            both = self.counts.cpu().tolist()
+            counts, visible = both[0], both[1]
+            if self.packed and max(visible) > self.pcap:
+                # some view kept more Gaussians than there are slots: more slots, repeat the step
+                self._alloc_packed(min(self.gauss.n, int(max(visible) * 1.25) + 1024))
+                continue
             over = [k for k, K in enumerate(counts) if K > self.views[k].capacity]
             for k, K in enumerate(counts):
                 self.views[k].num_instances = K
@@ -565,7 +651,15 @@ class Trainer:
             for k in over:  # grow and repeat the step's views (nothing was applied yet)
                 self.views[k]._alloc(int(counts[k] * 1.25) + 1024)
         self.step_count += 1
-        if self.fused:
+        if self.packed:
+            project_bwd_views_adam_packed(self.gauss, self.views, self.packs, self.grad2ds, self.m, self.v, self.lrs,
+                                          self.step_count, None, self.densify_accum, self.densify_count,
+                                          densify_max_radius=self.densify_max_radius, sparse=self.sparse_grad)
+            # far more slots than Gaussians kept (the first step starts with n): fewer slots from
+            # the next step on
+            if self.pcap > 1.5 * max(visible) + 4096:
+                self._alloc_packed(min(self.gauss.n, int(max(visible) * 1.25) + 1024))
+        elif self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
                                    self.lrs, self.step_count, None, self.densify_accum, self.densify_count,
                                    densify_max_radius=self.densify_max_radius, sparse=self.sparse_grad)

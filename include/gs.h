@@ -326,6 +326,56 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
                                     float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
                                     int32_t sparse_adam, void* stream);
 
+/* The packed layout (the packed option of rasterize_gaussians, gsplat guide
+ * §4.1): a view's projected features are stored only for the Gaussians it keeps
+ * (radius > 0), contiguously in ascending Gaussian order.  Slot k holds
+ * Gaussian gaussian_ids[k]; slot_of[i] is the slot of Gaussian i, or -1.  Every
+ * later call takes the packed arrays as it takes gs_project's, with n replaced
+ * by the capacity: the binning's values, the raster calls' 2D gradients and the
+ * instance lists are then indexed by slot.  Because slots ascend with the
+ * Gaussian id, the sort keys, the order of equal keys, the images and the
+ * gradients are those of the unpacked layout with every value v replaced by
+ * gaussian_ids[v].
+ *
+ * gs_project_packed_workspace_bytes -- device workspace for n Gaussians (about
+ * 60 bytes per Gaussian: gs_project's outputs for all of them, before packing).
+ *
+ * gs_project_packed -- gs_project of every Gaussian into the workspace, then
+ * the order-preserving compaction into `capacity` packed slots:
+ *   packed         gs_projected arrays of `capacity` entries (the alignments of
+ *                  gs_projected);
+ *   gaussian_ids   [capacity] uint32, 0xffffffff for an unused slot;
+ *   slot_of        [params->n] int32;
+ *   num_visible_dev  one uint64 on the device: the number V of Gaussians kept.
+ * Slots V..capacity-1 hold culled entries (radius 0, tiles_touched 0, zero
+ * features), so the later calls skip them.  V > capacity is not an error of the
+ * call: slots up to capacity are filled, slot_of is -1 for the Gaussians that got
+ * none, and the caller compares V (read when convenient) with the capacity and
+ * repeats with more room before using the results.  Asynchronous, no host wait. */
+size_t gs_project_packed_workspace_bytes(int64_t n);
+gs_status gs_project_packed(const gs_params* params, const gs_camera* cam, void* workspace, size_t workspace_bytes,
+                            gs_projected* packed, int64_t capacity, uint32_t* gaussian_ids, int32_t* slot_of,
+                            uint64_t* num_visible_dev, void* stream);
+
+/* gs_project_bwd_views_packed, gs_project_bwd_views_adam_packed --
+ * gs_project_bwd_views and gs_project_bwd_views_adam for views in the packed
+ * layout: projs[v] and grad2d[v] are view v's packed arrays and slot_of[v]
+ * (a host array of num_views device pointers) its slot map; a Gaussian is in
+ * view v when slot_of[v][i] >= 0.  Parameters, gradients and the densification
+ * statistics stay indexed by Gaussian.  Results equal those of the unpacked
+ * calls given the same per-Gaussian 2D gradients. */
+gs_status gs_project_bwd_views_packed(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                      const gs_projected* projs, const int32_t* const* slot_of,
+                                      const gs_grad2d* grad2d, gs_param_grads* grads, float* densify_accum,
+                                      int32_t* densify_count, int32_t* densify_max_radius, void* stream);
+gs_status gs_project_bwd_views_adam_packed(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                           const gs_projected* projs, const int32_t* const* slot_of,
+                                           const gs_grad2d* grad2d, gs_param_grads* params_inout,
+                                           gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                           float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                           float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                           int32_t sparse_adam, void* stream);
+
 /* Adaptive density control (gsplat guide §4.1: every 100 steps,
  * densify_and_prune with a gradient threshold of 0.0002, a minimum opacity of
  * 0.005, an extent of 0.01 and a maximum screen size of 0.02; 3DGS deploy guide

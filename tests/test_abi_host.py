@@ -149,6 +149,32 @@ def test_invalid_arguments_rejected_before_launch(gs):
     assert L.gs_project_bwd_views_adam(C.byref(p), 1, C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr),
                                        C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None, None, None, None, 2,
                                        None) == gs.GS_ERR_INVALID_ARG
+    # packed projection: workspace size, capacity, the visible counter and the slot map
+    wsp = gs.gs_project_packed_workspace_bytes(10)
+    assert wsp >= 60 * 10
+    packed = gs.gs_projected(16, 16, 16, 16, 16, 16, 16)
+    cntp = 256
+    assert L.gs_project_packed(C.byref(p), C.byref(c), 256, 8, C.byref(packed), 10, 256, 256, cntp, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "workspace" in gs.gs_last_error_detail()
+    assert L.gs_project_packed(C.byref(p), C.byref(c), 256, wsp, C.byref(packed), -1, 256, 256, cntp, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert L.gs_project_packed(C.byref(p), C.byref(c), 256, wsp, C.byref(packed), 10, 256, 256, None, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert L.gs_project_packed(C.byref(p), C.byref(c), 256, wsp, C.byref(packed), 10, 256, None, cntp, None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "slot_of" in gs.gs_last_error_detail()
+    assert L.gs_project_packed(C.byref(p), C.byref(c), 256, wsp, C.byref(packed), 10, None, 256, cntp, None) == \
+        gs.GS_ERR_INVALID_ARG
+    # packed backward: the slot maps are required
+    assert L.gs_project_bwd_views_packed(C.byref(p), 1, C.byref(c), C.byref(proj), None, C.byref(g2), C.byref(gr),
+                                         None, None, None, None) == gs.GS_ERR_INVALID_ARG
+    assert "slot_of" in gs.gs_last_error_detail()
+    bad_slots = (C.c_void_p * 1)(258)
+    assert L.gs_project_bwd_views_adam_packed(C.byref(p), 1, C.byref(c), C.byref(proj), bad_slots, C.byref(g2),
+                                              C.byref(gr), C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None,
+                                              None, None, None, 0, None) == gs.GS_ERR_INVALID_ARG
+    assert "aligned" in gs.gs_last_error_detail()
     # D-SSIM: image size limits and workspace
     assert L.gs_l1_dssim_loss_grad(256, 256, 0, 10, 1.0, 0.2, 256, 1 << 20, 256, 256, None) == gs.GS_ERR_UNSUPPORTED
     assert L.gs_l1_dssim_loss_grad(256, 256, 10, 10, 1.0, 0.2, 256, 8, 256, 256, None) == gs.GS_ERR_INVALID_ARG
