@@ -490,7 +490,8 @@ def run_ours(args, world, rank, local):
     line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
                     "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
                     "absgrad_and_sparse_adam": measure_variants(tr, torch),
-                    "packed": measure_packed(tr, wl, peaks, torch)}
+                    "packed": measure_packed(tr, wl, peaks, torch),
+                    "sh16": measure_sh16(tr, wl, peaks, torch)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
         line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
@@ -590,6 +591,44 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     res["project_packed_roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                       "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes}
     del trp
+    return res
+
+
+def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
+    """16-bit SH storage: the training step with the projections reading the half copy
+    (Trainer(sh16=True)) against the float32 step, and the projection of the first view
+    from half against float32 coefficients, each with the HBM roofline of its algorithmic
+    bytes (the parameters read, with 2 or 4 bytes per SH coefficient, and 52 bytes of
+    projected features written)."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    s = torch.cuda.current_stream()
+    scene = wl.scene
+    trh = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
+                     dict(tr.lrs), densify=True, streams=tr.streams, sh16=True)
+
+    def timed(fn, count):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(count):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / count
+
+    res = {"step_ms_sh16": timed(trh.step, steps), "step_ms_f32": timed(tr.step, steps)}
+    n, nc = scene.n, 3 * (scene.sh_degree + 1) ** 2
+    for name, fn, sh_bytes in (
+            ("f32", lambda: pl.project(tr.gauss, tr.views[0], tr.projs[0], tr.radii[0]), 4),
+            ("sh16", lambda: pl.project_sh16(trh.gauss, trh.sh_half, trh.views[0], trh.projs[0], trh.radii[0]), 2)):
+        ms = timed(fn, reps)
+        nbytes = n * (44 + sh_bytes * nc + 52)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[f"project_{name}_ms"] = ms
+        res[f"project_{name}_roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                           "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes}
+    del trh
     return res
 
 

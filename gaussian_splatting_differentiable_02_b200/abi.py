@@ -115,6 +115,14 @@ SIGNATURES = {
                                                      C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float,
                                                      C.c_float, C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P,
                                                      _P, _P, C.c_int32, _P]),
+    "gs_to_half": (C.c_int32, [_P, C.c_int64, _P, _P]),
+    "gs_project_sh16": (C.c_int32, [C.POINTER(gs_params), _P, C.POINTER(gs_camera), C.POINTER(gs_projected), _P]),
+    "gs_project_bwd_views_adam_sh16": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
+                                                   C.POINTER(gs_projected), C.POINTER(gs_grad2d), _P, _P,
+                                                   C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
+                                                   C.POINTER(gs_param_grads), C.POINTER(C.c_float), C.c_float,
+                                                   C.c_float, C.c_float, C.c_int32, C.POINTER(gs_param_grads), _P,
+                                                   _P, _P, C.c_int32, _P]),
     "gs_l1_dssim_workspace_bytes": (C.c_size_t, [C.c_int32, C.c_int32]),
     "gs_l1_dssim_loss_grad": (C.c_int32, [_P, _P, C.c_int32, C.c_int32, C.c_float, C.c_float, _P, C.c_size_t, _P, _P,
                                           _P]),
@@ -354,6 +362,32 @@ def gs_project_bwd_views_adam_packed(params: gs_params, cams, projs, slot_of, gr
         _arr(gs_grad2d, grad2ds), C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1, beta2, eps,
         step, C.byref(grads) if grads is not None else None, densify_accum or None, densify_count or None,
         densify_max_radius or None, int(sparse_adam), stream))
+
+
+def gs_to_half(x: int, count: int, out: int, stream: int = 0):
+    """float32 -> IEEE half, round to nearest even (count values)."""
+    return _check(lib().gs_to_half(x or None, count, out or None, stream))
+
+
+def gs_project_sh16(params: gs_params, sh_half: int, cam: gs_camera, out: gs_projected, stream: int = 0):
+    """gs_project with the SH coefficients read from a 16-bit copy."""
+    return _check(lib().gs_project_sh16(C.byref(params), sh_half or None, C.byref(cam), C.byref(out), stream))
+
+
+def gs_project_bwd_views_adam_sh16(params: gs_params, cams, projs, grad2ds, sh_half: int, sh_half_out: int,
+                                   params_inout: gs_param_grads, adam_m: gs_param_grads, adam_v: gs_param_grads, lrs,
+                                   beta1: float, beta2: float, eps: float, step: int, grads: gs_param_grads = None,
+                                   densify_accum: int = 0, densify_count: int = 0, densify_max_radius: int = 0,
+                                   sparse_adam: int = 0, stream: int = 0):
+    """gs_project_bwd_views_adam for views projected from 16-bit SH; the updated SH is
+    rounded into sh_half_out."""
+    V = len(cams)
+    lr = (C.c_float * 5)(*[float(x) for x in lrs])
+    return _check(lib().gs_project_bwd_views_adam_sh16(
+        C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, projs), _arr(gs_grad2d, grad2ds),
+        sh_half or None, sh_half_out or None, C.byref(params_inout), C.byref(adam_m), C.byref(adam_v), lr, beta1,
+        beta2, eps, step, C.byref(grads) if grads is not None else None, densify_accum or None,
+        densify_count or None, densify_max_radius or None, int(sparse_adam), stream))
 
 
 def gs_l1_dssim_workspace_bytes(width: int, height: int) -> int:

@@ -98,7 +98,7 @@ gs_status check_camera(const char* fn, const gs_camera* cam) {
     return GS_OK;
 }
 
-gs_status check_params(const char* fn, const gs_params* p) {
+gs_status check_params(const char* fn, const gs_params* p, bool need_sh = true) {
     if (!p) return fail(GS_ERR_INVALID_ARG, "%s: params is NULL", fn);
     if (p->n < 0 || p->n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n = %lld out of range", fn, (long long)p->n);
     if (p->sh_degree < 0 || p->sh_degree > 3)
@@ -108,7 +108,7 @@ gs_status check_params(const char* fn, const gs_params* p) {
     CHECK_PTR(p->quats, 16);
     CHECK_PTR(p->log_scales, 16);
     CHECK_PTR(p->opacity_logits, 4);
-    CHECK_PTR(p->sh, 16);
+    if (need_sh) CHECK_PTR(p->sh, 16);
     return GS_OK;
 }
 
@@ -154,6 +154,27 @@ gs_status gs_tile_grid(const gs_camera* cam, int32_t* tiles_x_host, int32_t* til
     *tiles_x_host = (cam->width + GS_TILE - 1) / GS_TILE;
     *tiles_y_host = (cam->height + GS_TILE - 1) / GS_TILE;
     return ok();
+}
+
+gs_status gs_project_sh16(const gs_params* params, const uint16_t* sh_half, const gs_camera* cam, gs_projected* out,
+                          void* stream) {
+    const char* fn = "gs_project_sh16";
+    gs_status st;
+    if ((st = check_params(fn, params, false)) != GS_OK) return st;
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if ((st = check_projected(fn, out, params->n, true)) != GS_OK) return st;
+    if (params->n > 0) CHECK_PTR(sh_half, 8);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_project_fwd(*params, c, *out, static_cast<cudaStream_t>(stream), sh_half), fn);
+}
+
+gs_status gs_to_half(const float* x, int64_t count, uint16_t* out, void* stream) {
+    const char* fn = "gs_to_half";
+    if (count < 0) return fail(GS_ERR_INVALID_ARG, "%s: count < 0", fn);
+    if (count == 0) return ok();
+    CHECK_PTR(x, 16);
+    CHECK_PTR(out, 8);
+    return cuda_status(gsk::launch_to_half(x, count, out, static_cast<cudaStream_t>(stream)), fn);
 }
 
 gs_status gs_project(const gs_params* params, const gs_camera* cam, gs_projected* out, void* stream) {
@@ -441,8 +462,14 @@ gs_status project_bwd_adam_common(const char* fn, const gs_params* params, int32
                                   const gs_grad2d* grad2d, gs_param_grads* params_inout, gs_param_grads* adam_m,
                                   gs_param_grads* adam_v, const float* lr_host, float beta1, float beta2, float eps,
                                   int32_t step, gs_param_grads* grads, float* densify_accum, int32_t* densify_count,
-                                  int32_t* densify_max_radius, int32_t sparse_adam, void* stream) {
+                                  int32_t* densify_max_radius, int32_t sparse_adam, void* stream,
+                                  const uint16_t* sh_half = nullptr, uint16_t* sh_half_out = nullptr,
+                                  bool sh16 = false) {
     if (sparse_adam != 0 && sparse_adam != 1) return fail(GS_ERR_INVALID_ARG, "%s: sparse_adam must be 0 or 1", fn);
+    if (sh16 && params && params->n > 0) {
+        CHECK_PTR(sh_half, 8);
+        CHECK_PTR(sh_half_out, 8);
+    }
     if (!lr_host) return fail(GS_ERR_INVALID_ARG, "%s: lr_host is NULL", fn);
     gsk::AdamStep a;
     gs_status st;
@@ -461,6 +488,10 @@ gs_status project_bwd_adam_common(const char* fn, const gs_params* params, int32
     a.eps = eps;
     a.step = step;
     a.sparse = sparse_adam == 1;
+    if (sh16) {
+        a.sh_half = sh_half;
+        a.sh_half_out = sh_half_out;
+    }
     return project_bwd_common(fn, params, num_views, cams, projs, grad2d, grads, densify_accum, densify_count,
                               densify_max_radius, &a, stream, slots, packed);
 }
@@ -490,6 +521,19 @@ gs_status gs_project_bwd_views_adam_packed(const gs_params* params, int32_t num_
     return project_bwd_adam_common("gs_project_bwd_views_adam_packed", params, num_views, cams, projs, slot_of, true,
                                    grad2d, params_inout, adam_m, adam_v, lr_host, beta1, beta2, eps, step, grads,
                                    densify_accum, densify_count, densify_max_radius, sparse_adam, stream);
+}
+
+gs_status gs_project_bwd_views_adam_sh16(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                         const gs_projected* projs, const gs_grad2d* grad2d,
+                                         const uint16_t* sh_half, uint16_t* sh_half_out, gs_param_grads* params_inout,
+                                         gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                         float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                         float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                         int32_t sparse_adam, void* stream) {
+    return project_bwd_adam_common("gs_project_bwd_views_adam_sh16", params, num_views, cams, projs, nullptr, false,
+                                   grad2d, params_inout, adam_m, adam_v, lr_host, beta1, beta2, eps, step, grads,
+                                   densify_accum, densify_count, densify_max_radius, sparse_adam, stream, sh_half,
+                                   sh_half_out, true);
 }
 
 gs_status gs_project_bwd_views_packed(const gs_params* params, int32_t num_views, const gs_camera* cams,

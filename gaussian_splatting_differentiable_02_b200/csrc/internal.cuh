@@ -43,7 +43,12 @@ inline int tile_bits(int64_t tiles) {
 // ------------------------------------------------------------------ launchers
 // Each returns the launch's cudaGetLastError().
 
-cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s);
+// sh_half: null, or a 16-bit copy of the SH planes read instead of p.sh
+cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s,
+                               const uint16_t* sh_half = nullptr);
+
+// float32 -> IEEE half (round to nearest even), count values
+cudaError_t launch_to_half(const float* x, int64_t count, uint16_t* out, cudaStream_t s);
 
 // One Adam step fused into the backward pass (parameters updated in place).
 struct AdamStep {
@@ -54,6 +59,10 @@ struct AdamStep {
     float beta1, beta2, eps;
     int step;
     bool sparse;  // skip Gaussians visible in no view (parameters and moments untouched)
+    // 16-bit SH: the chain reads sh_half (the values the forward used) instead of the
+    // float32 SH, and the updated float32 SH is written back rounded into sh_half_out
+    const uint16_t* sh_half = nullptr;
+    uint16_t* sh_half_out = nullptr;
 };
 
 // The packed projection: every Gaussian projected into `full` (workspace), then

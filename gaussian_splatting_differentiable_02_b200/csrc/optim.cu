@@ -1,7 +1,10 @@
 // gs_adam and gs_l1_loss_grad: the optimiser step and the L1 photometric term
-// of the training loop in the gsplat guide (lmnt.cn/news/262699) §4.1-4.2.
-// Both are streaming kernels: 128-bit loads and stores, grid a multiple of the
-// SM count.
+// of the training loop in the gsplat guide (lmnt.cn/news/262699) §4.1-4.2; and
+// gs_to_half, the float32 -> FP16 rounding of parameters (the guides' FP16
+// parameter storage).  All are streaming kernels: 128-bit loads, grid a multiple
+// of the SM count.
+#include <cuda_fp16.h>
+
 #include "internal.cuh"
 
 namespace gsk {
@@ -78,7 +81,35 @@ __global__ void __launch_bounds__(256) l1_kernel(const float* __restrict__ img, 
     }
 }
 
+// Round to nearest even into IEEE half: four values per thread and step, then the tail.
+__global__ void __launch_bounds__(256) to_half_kernel(const float* __restrict__ x, int64_t count,
+                                                      uint16_t* __restrict__ out) {
+    const int64_t q = count / 4;
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t first = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    for (int64_t i = first; i < q; i += stride) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(x) + i);
+        const __half2 lo = __floats2half2_rn(v.x, v.y);
+        const __half2 hi = __floats2half2_rn(v.z, v.w);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(out)[i] = w;
+    }
+    for (int64_t i = 4 * q + first; i < count; i += stride) {
+        const __half h = __float2half_rn(__ldg(x + i));
+        out[i] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_to_half(const float* x, int64_t count, uint16_t* out, cudaStream_t s) {
+    if (count == 0) return cudaSuccess;
+    to_half_kernel<<<grid_for((count + 3) / 4, 256, 8), 256, 0, s>>>(x, count, out);
+    count_launches(1);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
                         float beta2, float eps, int32_t step, cudaStream_t s) {

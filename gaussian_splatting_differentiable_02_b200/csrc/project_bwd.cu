@@ -13,12 +13,16 @@
 // With Adam fused the gradients never reach memory: parameters, moments and the
 // views' 2D gradients each make exactly one pass through HBM.  In the packed
 // layout (gs_project_packed) a view's features and 2D gradients are read at the
-// Gaussian's slot, found through the view's slot map.
+// Gaussian's slot, found through the view's slot map.  With 16-bit SH storage the
+// colour chain takes the half-precision coefficients the forward pass used, Adam
+// updates the float32 coefficients, and their rounding to half is written back.
 //
 // The geometric chain is double precision: the inverse of a 2x2 conic and the
 // EWA product are badly conditioned for needle-shaped Gaussians.  The colour
 // (SH) chain is float32 except the sign test of the raw colour, which repeats the
 // forward pass's double-precision decision.
+#include <cuda_fp16.h>
+
 #include "internal.cuh"
 
 namespace gsk {
@@ -54,6 +58,8 @@ struct Args {
     const float4* log_scales;
     const float* logits;
     const float4* sh;
+    const uint2* sh_half;  // kHalf: the 16-bit SH the forward used (four halves per element)
+    uint2* sh_half_out;    // kHalf: the updated SH rounded to 16 bits (may alias sh_half)
     int deg, planes, V;
     int64_t n;
     ViewArgs view[kMaxViews];
@@ -144,8 +150,8 @@ __device__ __forceinline__ float adam_one(float p, float g, float& m, float& v, 
     return p - lr_t * m / (sqrtf(v) * a.inv_sqrt_bc2 + a.eps);
 }
 
-__device__ __forceinline__ void adam4(float4* p, float4* m, float4* v, int64_t i, float4 g, float lr_t,
-                                      const Args& a) {
+__device__ __forceinline__ float4 adam4(float4* p, float4* m, float4* v, int64_t i, float4 g, float lr_t,
+                                        const Args& a) {
     float4 pp = p[i], mm = m[i], vv = v[i];
     pp.x = adam_one(pp.x, g.x, mm.x, vv.x, lr_t, a);
     pp.y = adam_one(pp.y, g.y, mm.y, vv.y, lr_t, a);
@@ -154,6 +160,22 @@ __device__ __forceinline__ void adam4(float4* p, float4* m, float4* v, int64_t i
     p[i] = pp;
     m[i] = mm;
     v[i] = vv;
+    return pp;
+}
+
+__device__ __forceinline__ float4 widen(uint2 h) {
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+__device__ __forceinline__ uint2 narrow(float4 f) {
+    const __half2 lo = __floats2half2_rn(f.x, f.y);
+    const __half2 hi = __floats2half2_rn(f.z, f.w);
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&lo);
+    w.y = *reinterpret_cast<const uint32_t*>(&hi);
+    return w;
 }
 
 __device__ __forceinline__ void add4(float4* d, int64_t i, float4 g) {
@@ -172,7 +194,7 @@ __device__ __forceinline__ int64_t entry(const ViewArgs& w, int64_t i) {
 #define GS_PBWD_MIN_BLOCKS 2
 #endif
 
-template <bool kAdam, bool kPacked>
+template <bool kAdam, bool kPacked, bool kHalf>
 __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_kernel(const Args a) {
     __shared__ float shs[48][kBwdBlock];  // this thread's SH coefficients, column threadIdx.x
     const int t = threadIdx.x;
@@ -229,7 +251,8 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
             const double logit = __ldg(a.logits + i);
             const double mu[3] = {m4.x, m4.y, m4.z};
             for (int p = 0; p < a.planes; ++p) {
-                const float4 c4 = __ldg(a.sh + int64_t(p) * a.n + i);
+                const float4 c4 = kHalf ? widen(__ldg(a.sh_half + int64_t(p) * a.n + i))
+                                        : __ldg(a.sh + int64_t(p) * a.n + i);
                 shs[4 * p + 0][t] = c4.x;
                 shs[4 * p + 1][t] = c4.y;
                 shs[4 * p + 2][t] = c4.z;
@@ -472,8 +495,12 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
 #pragma unroll
             for (int p = 0; p < 12; ++p)
                 if (p < a.planes)
-                    adam4(a.p_sh, a.m_sh, a.v_sh, int64_t(p) * a.n + i,
-                          make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]), a.lr_t[4], a);
+                {
+                    const float4 up = adam4(a.p_sh, a.m_sh, a.v_sh, int64_t(p) * a.n + i,
+                                            make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]),
+                                            a.lr_t[4], a);
+                    if (kHalf) a.sh_half_out[int64_t(p) * a.n + i] = narrow(up);
+                }
         }
         if (a.densify_accum && dcnt) {
             a.densify_accum[i] += dacc;
@@ -551,14 +578,18 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
         a.b1 = adam->beta1;
         a.b2 = adam->beta2;
         a.eps = adam->eps;
-        if (slots)
-            project_bwd_kernel<true, true><<<grid, kBwdBlock, 0, s>>>(a);
+        a.sh_half = reinterpret_cast<const uint2*>(adam->sh_half);
+        a.sh_half_out = reinterpret_cast<uint2*>(adam->sh_half_out);
+        if (adam->sh_half)
+            project_bwd_kernel<true, false, true><<<grid, kBwdBlock, 0, s>>>(a);
+        else if (slots)
+            project_bwd_kernel<true, true, false><<<grid, kBwdBlock, 0, s>>>(a);
         else
-            project_bwd_kernel<true, false><<<grid, kBwdBlock, 0, s>>>(a);
+            project_bwd_kernel<true, false, false><<<grid, kBwdBlock, 0, s>>>(a);
     } else if (slots) {
-        project_bwd_kernel<false, true><<<grid, kBwdBlock, 0, s>>>(a);
+        project_bwd_kernel<false, true, false><<<grid, kBwdBlock, 0, s>>>(a);
     } else {
-        project_bwd_kernel<false, false><<<grid, kBwdBlock, 0, s>>>(a);
+        project_bwd_kernel<false, false, false><<<grid, kBwdBlock, 0, s>>>(a);
     }
     count_launches(1);
     return cudaGetLastError();

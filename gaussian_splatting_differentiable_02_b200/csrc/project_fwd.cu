@@ -5,9 +5,13 @@
 // written, so the integer decisions taken from floating point (culling, the
 // 3-sigma radius, the tile rectangle) and the float32 depth used in the sort key
 // come out the same on any IEEE double implementation that evaluates the same
-// expressions in the same order.  The projection is streaming work (about 290
+// expressions in the same order.  The SH coefficients may come from a 16-bit
+// (IEEE half) copy; widening a half is exact, so the result is the float32 path's
+// on the rounded coefficients.  The projection is streaming work (about 290
 // bytes per Gaussian) and sits far below the device's double-precision rate, so
 // the wider arithmetic costs no time.
+#include <cuda_fp16.h>
+
 #include "internal.cuh"
 
 namespace gsk {
@@ -28,6 +32,7 @@ struct FwdArgs {
     const float4* log_scales;
     const float* logits;
     const float4* sh;
+    const uint2* sh_half;  // 16-bit copy of the SH planes (four IEEE halves per element), or null
     int deg, planes;
     int64_t n;
     CamArgs cam;
@@ -52,6 +57,18 @@ __device__ void write_culled(const FwdArgs& a, int64_t i) {
     a.tiles_touched[i] = 0u;
 }
 
+// One float4 element of SH plane p: from the float32 array, or widened exactly from
+// the 16-bit copy.
+template <bool kHalf>
+__device__ __forceinline__ float4 sh_element(const FwdArgs& a, int p, int64_t i) {
+    if (!kHalf) return __ldg(a.sh + int64_t(p) * a.n + i);
+    const uint2 h = __ldg(a.sh_half + int64_t(p) * a.n + i);
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+template <bool kHalf>
 __global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
     const CamArgs& cam = a.cam;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < a.n; i += int64_t(gridDim.x) * blockDim.x) {
@@ -62,8 +79,12 @@ __global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
 #ifndef GS_PROJECT_NO_PREFETCH
         // the SH planes are read only after the covariance arithmetic: start moving
         // them into L2 now so that their loads do not wait on DRAM then
-        for (int p = 0; p < a.planes; ++p)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.sh + int64_t(p) * a.n + i));
+        for (int p = 0; p < a.planes; ++p) {
+            if (kHalf)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.sh_half + int64_t(p) * a.n + i));
+            else
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.sh + int64_t(p) * a.n + i));
+        }
 #endif
         const double mu[3] = {m4.x, m4.y, m4.z};
         const double q[4] = {q4.x, q4.y, q4.z, q4.w};
@@ -182,7 +203,7 @@ __global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
         const int nc = (a.deg + 1) * (a.deg + 1);
         double col[3] = {0.0, 0.0, 0.0};
         for (int p = 0; p < a.planes; ++p) {
-            const float4 c4 = __ldg(a.sh + int64_t(p) * a.n + i);
+            const float4 c4 = sh_element<kHalf>(a, p, i);
             const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -215,13 +236,15 @@ __global__ void __launch_bounds__(256) project_fwd_kernel(const FwdArgs a) {
 
 }  // namespace
 
-cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s) {
+cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s,
+                               const uint16_t* sh_half) {
     FwdArgs a;
     a.means = reinterpret_cast<const float4*>(p.means);
     a.quats = reinterpret_cast<const float4*>(p.quats);
     a.log_scales = reinterpret_cast<const float4*>(p.log_scales);
     a.logits = p.opacity_logits;
     a.sh = reinterpret_cast<const float4*>(p.sh);
+    a.sh_half = reinterpret_cast<const uint2*>(sh_half);
     a.deg = p.sh_degree;
     a.planes = sh_planes(p.sh_degree);
     a.n = p.n;
@@ -234,7 +257,10 @@ cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_
     a.rect = reinterpret_cast<uint2*>(out.rect);
     a.tiles_touched = out.tiles_touched;
     if (p.n == 0) return cudaSuccess;
-    project_fwd_kernel<<<grid_for(p.n, 256, 16), 256, 0, s>>>(a);
+    if (sh_half)
+        project_fwd_kernel<true><<<grid_for(p.n, 256, 16), 256, 0, s>>>(a);
+    else
+        project_fwd_kernel<false><<<grid_for(p.n, 256, 16), 256, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }

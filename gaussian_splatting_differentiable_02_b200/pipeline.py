@@ -231,6 +231,22 @@ def project(g: Gaussians, view: View, proj: Projected, radius: torch.Tensor = No
     abi.gs_project(g.params(), view.gcam, proj.struct(radius), _stream())
 
 
+def to_half(x: torch.Tensor, out: torch.Tensor = None) -> torch.Tensor:
+    """x (float32) rounded to IEEE half, nearest even (gs_to_half); out: an int16 tensor of
+    x's shape holding the bit patterns (allocated when None)."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise TypeError("to_half takes a contiguous float32 tensor")
+    if out is None:
+        out = torch.empty(x.shape, device=x.device, dtype=torch.int16)
+    abi.gs_to_half(_ptr(x), x.numel(), _ptr(out), _stream())
+    return out
+
+
+def project_sh16(g: Gaussians, sh_half: torch.Tensor, view: View, proj: Projected, radius: torch.Tensor = None):
+    """gs_project with the SH coefficients read from their 16-bit copy sh_half ([P, n, 4] halves)."""
+    abi.gs_project_sh16(g.params(), _ptr(sh_half), view.gcam, proj.struct(radius), _stream())
+
+
 def bin_sort(proj: Projected, view: View, radius: torch.Tensor = None):
     """Sort the instances; grows the view's buffers when they are too small.  Returns K."""
     s = _stream()
@@ -341,6 +357,20 @@ def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: to
         _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
+def project_bwd_views_adam_sh16(g: Gaussians, sh_half: torch.Tensor, views: list, proj: Projected,
+                                radii: torch.Tensor, grad2ds: list, m: Gaussians, v: Gaussians, lrs: dict, step: int,
+                                grads: Gaussians = None, densify_accum: torch.Tensor = None,
+                                densify_count: torch.Tensor = None, betas=(0.9, 0.99), eps=1e-15,
+                                densify_max_radius: torch.Tensor = None, sparse: bool = False):
+    """project_bwd_views_adam for views projected from the 16-bit SH copy: the chain reads
+    sh_half, Adam updates the float32 SH, and sh_half is refreshed from it in place."""
+    abi.gs_project_bwd_views_adam_sh16(
+        g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
+        [gd.struct() for gd in grad2ds], _ptr(sh_half), _ptr(sh_half), g.grads(), m.grads(), v.grads(),
+        [lrs[k] for k in PARAM_NAMES], betas[0], betas[1], eps, step, grads.grads() if grads is not None else None,
+        _ptr(densify_accum), _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
+
+
 def project_bwd_views_adam_packed(g: Gaussians, views: list, packs: list, grad2ds: list, m: Gaussians, v: Gaussians,
                                   lrs: dict, step: int, grads: Gaussians = None, densify_accum: torch.Tensor = None,
                                   densify_count: torch.Tensor = None, betas=(0.9, 0.99), eps=1e-15,
@@ -417,6 +447,8 @@ class Trainer:
     packed: bool = False       # fused batched path: views in the packed layout (gs_project_packed, the
                                # gsplat guide §4.1 packed option); the slot capacity follows the largest
                                # visible count seen
+    sh16: bool = False         # fused unpacked path: the projections read a 16-bit (FP16) copy of the SH
+                               # coefficients, which the fused Adam step refreshes from the float32 ones
 
     def __post_init__(self):
         n = self.gauss.n
@@ -424,6 +456,8 @@ class Trainer:
         self.fused = self.fused and len(self.views) <= abi.GS_MAX_VIEWS
         if self.packed and not (self.fused and self.batched_sort):
             raise ValueError("packed=True runs on the fused path with the batched sort")
+        if self.sh16 and (self.packed or not self.fused):
+            raise ValueError("sh16=True runs on the fused path with unpacked views")
         # per view: instance count and (packed) visible count, read back with one wait per step
         self.counts = torch.zeros((2, len(self.views)), device=dev, dtype=torch.int64)
         self.kcount = self.counts[0]
@@ -459,6 +493,7 @@ class Trainer:
             self.grad2d = self.grad2ds[0]
             self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
         self.grads = None if self.fused else self.gauss.zeros_like()
+        self.sh_half = to_half(self.gauss.sh) if self.sh16 else None
         self.densify_accum = torch.zeros((max(n, 1),), device=dev, dtype=torch.float32) if self.densify else None
         self.densify_count = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
         self.densify_max_radius = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
@@ -476,6 +511,12 @@ class Trainer:
         self.grad2d = self.grad2ds[0]
         for view in self.views:
             view.set_n(self.pcap)
+
+    def _project(self, view: View, proj: Projected, radius: torch.Tensor):
+        if self.sh16:
+            project_sh16(self.gauss, self.sh_half, view, proj, radius)
+        else:
+            project(self.gauss, view, proj, radius)
 
     def _radius(self, k: int):
         """View k's radius row (None: the packed projection's own)."""
@@ -516,7 +557,7 @@ class Trainer:
         if projected:
             bin_sort_ordered_async(proj, view, self.depth_order.order[k], self.kcount[k:k + 1], r)
         else:
-            project(self.gauss, view, proj, r)
+            self._project(view, proj, r)
             if self.fused:
                 bin_sort_async(proj, view, self.kcount[k:k + 1], r)
             else:
@@ -612,7 +653,7 @@ class Trainer:
             if self.packed:
                 project_packed(self.gauss, view, self.packs[k], self.pack_ws)
             else:
-                project(self.gauss, view, self.projs[k], self.radii[k])
+                self._project(view, self.projs[k], self.radii[k])
         depth_order_views(self.projs, self.radii, self.depth_order)
 
     def side_streams(self) -> list:
@@ -659,6 +700,11 @@ class Trainer:
             # the next step on
             if self.pcap > 1.5 * max(visible) + 4096:
                 self._alloc_packed(min(self.gauss.n, int(max(visible) * 1.25) + 1024))
+        elif self.sh16:
+            project_bwd_views_adam_sh16(self.gauss, self.sh_half, self.views, self.proj, self.radii, self.grad2ds,
+                                        self.m, self.v, self.lrs, self.step_count, None, self.densify_accum,
+                                        self.densify_count, densify_max_radius=self.densify_max_radius,
+                                        sparse=self.sparse_grad)
         elif self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
                                    self.lrs, self.step_count, None, self.densify_accum, self.densify_count,

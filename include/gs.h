@@ -376,6 +376,37 @@ gs_status gs_project_bwd_views_adam_packed(const gs_params* params, int32_t num_
                                            float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
                                            int32_t sparse_adam, void* stream);
 
+/* 16-bit SH storage (the guides' FP16 mode: FP16 parameters for rendering, mixed
+ * precision in training).  The SH coefficients are kept as IEEE binary16 in the
+ * float4-plane layout of gs_params.sh: [planes][n][4] halves, 8-byte aligned.
+ * All arithmetic stays double / float32; widening a half is exact, so every
+ * result equals the float32 path's on the rounded coefficients.
+ *
+ * gs_to_half -- out[i] = x[i] rounded to the nearest binary16, ties to even
+ * (magnitudes past 65504 round to infinity, as IEEE 754 rounds); count floats,
+ * x 16-byte and out 8-byte aligned.
+ *
+ * gs_project_sh16 -- gs_project with the SH coefficients read from sh_half
+ * instead of params->sh (which may be NULL).  A coefficient that rounded to
+ * infinity makes the colour non-finite, and the Gaussian is culled.
+ *
+ * gs_project_bwd_views_adam_sh16 -- gs_project_bwd_views_adam for views
+ * projected by gs_project_sh16: the colour chain uses the half-precision
+ * coefficients in sh_half (the values the forward pass used), Adam updates the
+ * float32 coefficients params_inout->sh (the master copy), and each updated
+ * float32 coefficient is written, rounded as by gs_to_half, to sh_half_out
+ * (which may be sh_half itself).  Unpacked views only. */
+gs_status gs_to_half(const float* x, int64_t count, uint16_t* out, void* stream);
+gs_status gs_project_sh16(const gs_params* params, const uint16_t* sh_half, const gs_camera* cam, gs_projected* out,
+                          void* stream);
+gs_status gs_project_bwd_views_adam_sh16(const gs_params* params, int32_t num_views, const gs_camera* cams,
+                                         const gs_projected* projs, const gs_grad2d* grad2d,
+                                         const uint16_t* sh_half, uint16_t* sh_half_out, gs_param_grads* params_inout,
+                                         gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,
+                                         float beta1, float beta2, float eps, int32_t step, gs_param_grads* grads,
+                                         float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
+                                         int32_t sparse_adam, void* stream);
+
 /* Adaptive density control (gsplat guide §4.1: every 100 steps,
  * densify_and_prune with a gradient threshold of 0.0002, a minimum opacity of
  * 0.005, an extent of 0.01 and a maximum screen size of 0.02; 3DGS deploy guide

@@ -175,6 +175,17 @@ def test_invalid_arguments_rejected_before_launch(gs):
                                               C.byref(gr), C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None,
                                               None, None, None, 0, None) == gs.GS_ERR_INVALID_ARG
     assert "aligned" in gs.gs_last_error_detail()
+    # 16-bit SH: negative count, misaligned input, missing half copy
+    assert L.gs_to_half(256, -1, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_to_half(260, 8, 256, None) == gs.GS_ERR_INVALID_ARG
+    assert "aligned" in gs.gs_last_error_detail()
+    assert L.gs_to_half(None, 0, None, None) == gs.GS_OK
+    p_nosh = gs.gs_params(16, 16, 16, 16, None, 3, 10)
+    assert L.gs_project_sh16(C.byref(p_nosh), None, C.byref(c), C.byref(packed), None) == gs.GS_ERR_INVALID_ARG
+    assert "sh_half" in gs.gs_last_error_detail()
+    assert L.gs_project_bwd_views_adam_sh16(C.byref(p), 1, C.byref(c), C.byref(proj), C.byref(g2), None, 256,
+                                            C.byref(gr), C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None,
+                                            None, None, None, 0, None) == gs.GS_ERR_INVALID_ARG
     # D-SSIM: image size limits and workspace
     assert L.gs_l1_dssim_loss_grad(256, 256, 0, 10, 1.0, 0.2, 256, 1 << 20, 256, 256, None) == gs.GS_ERR_UNSUPPORTED
     assert L.gs_l1_dssim_loss_grad(256, 256, 10, 10, 1.0, 0.2, 256, 8, 256, 256, None) == gs.GS_ERR_INVALID_ARG
