@@ -396,7 +396,7 @@ def run_ours(args, world, rank, local):
     lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
                                                   "opacity_logits": 5e-2, "sh": 2.5e-3}
     tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams,
-                    batched_sort=not args.per_view_sort)
+                    batched_sort=not args.per_view_sort, groups=args.groups)
     stream = torch.cuda.current_stream()
 
     # warm-up (also sizes every view's instance buffers)
@@ -470,7 +470,8 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
-                       "depth_sort": "per view" if args.per_view_sort else "batched over the views",
+                       "depth_sort": "per view" if args.per_view_sort else
+                       f"batched over the views, in {len(tr.view_groups())} pipelined view groups",
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -551,7 +552,7 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     s = torch.cuda.current_stream()
     scene = wl.scene
     trp = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, packed=True)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, packed=True)
 
     def step_ms(t):
         for _ in range(3):
@@ -604,7 +605,7 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     s = torch.cuda.current_stream()
     scene = wl.scene
     trh = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, sh16=True)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, sh16=True)
 
     def timed(fn, count):
         for _ in range(3):
@@ -763,17 +764,18 @@ def stage_breakdown(tr, pl, torch):
         acc.setdefault(name, []).append((e0, e1))
         return r
 
-    batched = getattr(tr, "depth_order", None) is not None
-    if batched:   # the Trainer's order: every projection, one batched depth sort, then per view
-        for k, view in enumerate(tr.views):
-            timed("project", pl.project, tr.gauss, view, tr.projs[k], tr.radii[k])
-        timed("bin_sort", pl.depth_order_views, tr.projs, tr.radii, tr.depth_order)
+    batched = getattr(tr, "depth_orders", None) is not None
+    if batched:   # the Trainer's order: per view group the projections and one batched depth sort, then per view
+        for ks, d in zip(tr.view_groups(), tr.depth_orders):
+            for k in ks:
+                timed("project", pl.project, tr.gauss, tr.views[k], tr.projs[k], tr.radii[k])
+            timed("bin_sort", pl.depth_order_views, [tr.projs[k] for k in ks], [tr.radii[k] for k in ks], d)
     for k, (view, tgt) in enumerate(zip(tr.views, tr.targets)):
         r = tr.radii[k]
         g2 = tr.grad2ds[k]
         proj = tr.projs[k] if batched else tr.proj
         if batched:
-            timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.depth_order.order[k], tr.kcount[k:k + 1], r)
+            timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.order_row(k), tr.kcount[k:k + 1], r)
         else:
             timed("project", pl.project, tr.gauss, view, proj, r)
             timed("bin_sort", pl.bin_sort, proj, view, r)
@@ -946,6 +948,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--streams", type=int, default=3,
                     help="CUDA streams the views of a step alternate over (1 = serial)")
+    ap.add_argument("--groups", type=int, default=1,
+                    help="view groups of the batched path (projection and depth sort of a group overlap "
+                         "the compositing of the groups before it)")
     ap.add_argument("--per-view-sort", action="store_true",
                     help="sort each view on its own stream instead of one batched depth sort of all views")
     ap.add_argument("--views", type=int, default=16,

@@ -444,6 +444,11 @@ class Trainer:
                                # view's sort overlaps another view's compositing
     batched_sort: bool = True  # fused path: project every view first and sort all views by depth in one
                                # batched sort (gs_depth_order_views), then bin and composite per view
+    groups: int = 1            # fused batched path: the views are projected, depth-sorted and binned in
+                               # this many consecutive groups, so that a group's projection and depth sort
+                               # overlap the compositing of the groups before it (on the 16-view 1080p
+                               # step 1, 2, 4, 8 groups take 44.4, 44.6, 44.8, 45.1 ms: compositing
+                               # already fills the device, and the overlap only adds launches)
     packed: bool = False       # fused batched path: views in the packed layout (gs_project_packed, the
                                # gsplat guide §4.1 packed option); the slot capacity follows the largest
                                # visible count seen
@@ -484,11 +489,11 @@ class Trainer:
             if self.fused and self.batched_sort:
                 # every view's projection is kept until its binning
                 self.projs = [self.proj] + [Projected(n, dev) for _ in range(nv - 1)]
-                self.depth_order = DepthOrder(n, nv, dev)
+                self._alloc_orders(n)
             else:
                 self.projs = [self.proj] + [Projected(n, dev) for _ in range(min(self.streams, nv) - 1)] \
                     if self.fused else [self.proj]
-                self.depth_order = None
+                self.depth_orders = None
             self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
             self.grad2d = self.grad2ds[0]
             self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
@@ -506,11 +511,29 @@ class Trainer:
         self.packs = [Packed(n, self.pcap, dev, self.counts[1][k:k + 1]) for k in range(nv)]
         self.projs = [pk.proj for pk in self.packs]
         self.proj = self.projs[0]
-        self.depth_order = DepthOrder(self.pcap, nv, dev)
+        self._alloc_orders(self.pcap)
         self.grad2ds = [Grad2D(self.pcap, dev, absgrad=self.absgrad) for _ in range(nv)]
         self.grad2d = self.grad2ds[0]
         for view in self.views:
             view.set_n(self.pcap)
+
+    def view_groups(self) -> list:
+        """The consecutive groups of view indices the batched path projects, sorts and bins together."""
+        nv = len(self.views)
+        size = -(-nv // max(1, min(self.groups, nv)))
+        return [list(range(i, min(i + size, nv))) for i in range(0, nv, size)]
+
+    def _alloc_orders(self, n: int):
+        """One batched depth order (and its workspace) per view group, over n entries."""
+        dev = self.gauss.means.device
+        groups = self.view_groups()
+        self.depth_orders = [DepthOrder(n, len(ks), dev) for ks in groups]
+        self._order_at = {k: (gi, j) for gi, ks in enumerate(groups) for j, k in enumerate(ks)}
+
+    def order_row(self, k: int) -> torch.Tensor:
+        """View k's depth order (a row of its group's DepthOrder)."""
+        gi, j = self._order_at[k]
+        return self.depth_orders[gi].order[j]
 
     def _project(self, view: View, proj: Projected, radius: torch.Tensor):
         if self.sh16:
@@ -555,7 +578,7 @@ class Trainer:
         r = self.radii[k if self.fused else 0]
         g2 = self.grad2ds[k if self.fused else 0]
         if projected:
-            bin_sort_ordered_async(proj, view, self.depth_order.order[k], self.kcount[k:k + 1], r)
+            bin_sort_ordered_async(proj, view, self.order_row(k), self.kcount[k:k + 1], r)
         else:
             self._project(view, proj, r)
             if self.fused:
@@ -577,7 +600,7 @@ class Trainer:
         for (e.g. the copy of its target); after_view(k, event): called once view k
         is enqueued, with an event recorded after it."""
         targets = self.targets if targets is None else targets
-        if not self.fused or (self.depth_order is None and len(self.projs) == 1):
+        if not self.fused or (self.depth_orders is None and len(self.projs) == 1):
             for k, tgt in enumerate(targets):
                 if ready is not None:
                     torch.cuda.current_stream().wait_event(ready[k])
@@ -587,29 +610,32 @@ class Trainer:
             return
         main = torch.cuda.current_stream()
         side = self.side_streams()
-        batched = self.depth_order is not None
+        batched = self.depth_orders is not None
         if batched:
-            self.project_and_order()
             # binning of every view on a high-priority stream: its small, latency-bound
             # kernels take SM slots as soon as compositing blocks retire, instead of
             # queueing behind whole compositing launches
             bin_stream = self.bin_stream()
-            bin_stream.wait_stream(main)
-            binned = []
-            with torch.cuda.stream(bin_stream):
-                for k, view in enumerate(self.views):
-                    bin_sort_ordered_async(self.projs[k], view, self.depth_order.order[k], self.kcount[k:k + 1],
-                                           self._radius(k))
-                    binned.append(bin_stream.record_event())
-            for k, tgt in enumerate(targets):
-                st = side[k % len(side)]
-                st.wait_event(binned[k])
-                if ready is not None:
-                    st.wait_event(ready[k])
-                with torch.cuda.stream(st):
-                    self.view_composite(k, tgt, self.projs[k])
-                if after_view is not None:
-                    after_view(k, st.record_event())
+            for gi, ks in enumerate(self.view_groups()):
+                # this group's projections and depth sort on the current stream run while
+                # the groups before it composite
+                self.project_and_order(gi)
+                bin_stream.wait_stream(main)
+                binned = {}
+                with torch.cuda.stream(bin_stream):
+                    for k in ks:
+                        bin_sort_ordered_async(self.projs[k], self.views[k], self.order_row(k),
+                                               self.kcount[k:k + 1], self._radius(k))
+                        binned[k] = bin_stream.record_event()
+                for k in ks:
+                    st = side[k % len(side)]
+                    st.wait_event(binned[k])
+                    if ready is not None:
+                        st.wait_event(ready[k])
+                    with torch.cuda.stream(st):
+                        self.view_composite(k, targets[k], self.projs[k])
+                    if after_view is not None:
+                        after_view(k, st.record_event())
             for st in side + [bin_stream]:
                 main.wait_stream(st)
             return
@@ -646,15 +672,19 @@ class Trainer:
             self._bin_stream = torch.cuda.Stream(device=self.gauss.means.device, priority=hi)
         return self._bin_stream
 
-    def project_and_order(self) -> None:
-        """Every view's projection (packed or not), then the batched depth sort of all views
-        (current stream)."""
-        for k, view in enumerate(self.views):
-            if self.packed:
-                project_packed(self.gauss, view, self.packs[k], self.pack_ws)
-            else:
-                self._project(view, self.projs[k], self.radii[k])
-        depth_order_views(self.projs, self.radii, self.depth_order)
+    def project_and_order(self, group: int = None) -> None:
+        """The projection of every view of a view group (packed or not), then the batched
+        depth sort of the group (current stream); every group when group is None."""
+        groups = self.view_groups()
+        for gi in range(len(groups)) if group is None else [group]:
+            ks = groups[gi]
+            for k in ks:
+                if self.packed:
+                    project_packed(self.gauss, self.views[k], self.packs[k], self.pack_ws)
+                else:
+                    self._project(self.views[k], self.projs[k], self.radii[k])
+            depth_order_views([self.projs[k] for k in ks], None if self.radii is None else [self.radii[k] for k in ks],
+                              self.depth_orders[gi])
 
     def side_streams(self) -> list:
         """The streams the fused path runs views on."""

@@ -239,18 +239,18 @@ def test_sparse_adam_skips_gaussians_seen_in_no_view():
 
 def test_trainer_stream_and_sort_configurations_agree():
     """Views on one stream with a sort per view, on two streams, and on three streams
-    after one batched depth sort of all views: the first step (identical inputs) gives
-    the same loss, counts and instance numbers; later steps agree up to the order of
-    the atomic adds."""
+    after batched depth sorts of all views at once, of two view groups and of one view
+    per group: the first step (identical inputs) gives the same loss, counts and
+    instance numbers; later steps agree up to the order of the atomic adds."""
     rng = np.random.default_rng(13)
     scene = scenes.random_scene(rng, 600, 1, mean_box=1.0, log_scale=(-3.5, -2.0))
     cams = _views(5, 8)
     targets = [torch.from_numpy(rng.random((128, 128, 3)).astype(np.float32)).cuda() for _ in cams]
     out = []
-    for streams, batched in ((1, False), (2, False), (3, True)):
+    for streams, batched, groups in ((1, False, 1), (2, False, 1), (3, True, 1), (3, True, 2), (2, True, 5)):
         g = pl.Gaussians.from_scene(scene)
         tr = pl.Trainer(g, [pl.View(scene.n, c) for c in cams], targets, dict(LRS), densify=True, streams=streams,
-                        batched_sort=batched)
+                        batched_sort=batched, groups=groups)
         tr.step()
         torch.cuda.synchronize()
         first = (tr.loss.item(), tr.densify_count.cpu().numpy(), tr.kcount.cpu().numpy(),
