@@ -12,8 +12,10 @@
 // with cp.async, double-buffered so the next batch is in flight while the
 // current one is composited; the lane that gathered an entry also derives its
 // per-entry constants and tests the entry against the warp's whole box (an
-// entry whose smallest sigma over the box leaves alpha below 1/255 is skipped
-// by the warp).  Every lane then reads each entry once (broadcast loads) and
+// entry whose smallest sigma over the box leaves alpha below 1/255 is dropped,
+// and the constants of the others are compacted, so the warp's loop visits only
+// entries that can reach its box).  Every lane then reads each entry once
+// (broadcast loads) and
 // applies it to its 4 pixels, whose terms that depend only on dx are shared;
 // the pixels go in pairs through the paired float32 instructions of sm_100
 // (fma/mul/add on two floats at once).  No block-wide barrier is used: warps
@@ -114,9 +116,12 @@ struct WarpStage {
     float4 con[2][kBatch];  // A, B, C, o
     float4 rgb[2][kBatch];
     uint32_t gid[2][kBatch];
+    // per-entry constants of the batch's entries that reach the warp's box, compacted
+    // in list order; idx is the entry's index in the batch
     float4 pa[kBatch];  // u, v, log2(o), 1/o
     float4 pb[kBatch];  // plain: -log2e A/2, -log2e B, -log2e C/2; factored: B/A (high, low part), D; flag
     float2 pc[kBatch];  // factored: -log2e A/2, -log2e D/2
+    int idx[kBatch];
 };
 
 // Lane l < count gathers list entry first + l (reverse: first + count - 1 - l).
@@ -160,9 +165,13 @@ __device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by
 // centres) puts alpha below 1/255 everywhere in it, with a margin far above
 // the rounding of either evaluation, so no pixel of the warp would blend it.
 // The bound is computed in float32 for well-conditioned conics and in double
-// for the others (never for an indefinite one).
+// for the others (never for an indefinite one).  The entries not skipped are
+// written compacted, in batch order, to S.pa / S.pb / S.pc with their batch index
+// in S.idx; returns their number.  Called by the whole warp.
 template <bool kNegRgb>
-__device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
+__device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
+    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = make_float4(0.f, 0.f, 0.f, kSkip);
+    float2 pc = make_float2(0.f, 0.f);
     if (lane < count) {
         if (kNegRgb) {  // the forward pass blends with -alpha T weights
             const float4 c = S.rgb[buf][lane];
@@ -177,8 +186,6 @@ __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane,
         // alpha >= 1/255 needs sigma <= ln(255 o) = ln 255 + lo ln 2
         const float cut = 5.541263545158426f + lo * 0.6931471805599453f;
         const float bx1 = bx0 + float(kBoxW - 1), by1 = by0 + float(kBoxH - 1);
-        float4 pb;
-        float2 pc = make_float2(0.f, 0.f);
         if (!ill) {
             const float smin = box_min<float>(c.x, c.y, c.z, xy.x, xy.y, bx0, bx1, by0, by1);
             const float flag = smin * (1.f - 1e-4f) > cut + 1e-4f ? kSkip : kPlain;
@@ -203,10 +210,17 @@ __device__ __forceinline__ void prep(WarpStage& S, int buf, int count, int lane,
                 pb = make_float4(0.f, 0.f, 0.f, kSkip);
             }
         }
-        S.pa[lane] = make_float4(xy.x, xy.y, lo, 1.f / c.w);
-        S.pb[lane] = pb;
-        S.pc[lane] = pc;
+        pa = make_float4(xy.x, xy.y, lo, 1.f / c.w);
     }
+    const unsigned keep = __ballot_sync(kFull, pb.w != kSkip);
+    if (pb.w != kSkip) {
+        const int k = __popc(keep & ((1u << lane) - 1u));
+        S.pa[k] = pa;
+        S.pb[k] = pb;
+        S.pc[k] = pc;
+        S.idx[k] = lane;
+    }
+    return __popc(keep);
 }
 
 // Pairs of pixels go through the paired float32 instructions of sm_100
@@ -333,20 +347,20 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (b + 1 < nb)
             gather<false>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t((b + 1) * kBatch),
                           min(n - (b + 1) * kBatch, kBatch), lane);
-        prep<true>(S, buf, cnt, lane, bx0, by0);
+        const int live = prep<true>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         bool finished = false;
-        for (int j = 0; j < cnt; ++j) {
+        for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
             if (__all_sync(kFull, done == kAll)) {
                 finished = true;
                 break;
             }
-            const float4 pa = S.pa[j], pb = S.pb[j];
-            if (pb.w == kSkip) continue;  // misses every pixel of this warp
+            const int j = S.idx[e];
+            const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
             const float4 nc = S.rgb[buf][j];  // minus the colour
             Alpha r;
-            eval_alpha(pa, pb, S.pc[j], con, px, nyc, r);
+            eval_alpha(pa, pb, S.pc[e], con, px, nyc, r);
             const unsigned blend = r.blend & ~done;
             const int pos = b * kBatch + j + 1;
             const f2 ncr = splat(nc.x), ncg = splat(nc.y), ncb = splat(nc.z);
@@ -520,16 +534,16 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             const int nhi = hi - kBatch, ncnt = min(nhi, kBatch);
             gather<true>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncnt), ncnt, lane);
         }
-        prep<false>(S, buf, cnt, lane, bx0, by0);
+        const int live = prep<false>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
-        for (int j = 0; j < cnt; ++j) {
+        for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
+            const int j = S.idx[e];
             const int pos = hi - 1 - j;  // 0-based list position of this entry
-            const float4 pa = S.pa[j], pb = S.pb[j];
-            if (pb.w == kSkip) continue;  // misses every pixel of this warp
+            const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
             Alpha r;
-            eval_alpha(pa, pb, S.pc[j], con, px, nyc, r);
+            eval_alpha(pa, pb, S.pc[e], con, px, nyc, r);
             const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
             f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
             bool any = false;
