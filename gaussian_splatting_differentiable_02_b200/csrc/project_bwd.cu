@@ -11,7 +11,10 @@
 // values), dL/dmean, dL/dlogit and the 48 SH gradients, all held in registers;
 // the chain from dL/dSigma to the scales and the quaternion runs once at the end.
 // With Adam fused the gradients never reach memory: parameters, moments and the
-// views' 2D gradients each make exactly one pass through HBM.  In the packed
+// views' 2D gradients each make exactly one pass through HBM.  For one or two
+// views the 48 SH gradients are summed in a second pass over the visible views
+// (their masked colour gradients kept in shared memory), which lets the kernel
+// run at twice the occupancy.  In the packed
 // layout (gs_project_packed) a view's features and 2D gradients are read at the
 // Gaussian's slot, found through the view's slot map.  With 16-bit SH storage the
 // colour chain takes the half-precision coefficients the forward pass used, Adam
@@ -193,10 +196,17 @@ __device__ __forceinline__ int64_t entry(const ViewArgs& w, int64_t i) {
 #ifndef GS_PBWD_MIN_BLOCKS
 #define GS_PBWD_MIN_BLOCKS 2
 #endif
+// Launches with at most this many views defer the SH gradient to a second pass
+// (kSplit): the 48 accumulators then never share registers with the geometric
+// chain, and the kernel runs at 4 blocks per SM instead of 2.  With many views the
+// single pass is faster (the second pass recomputes every view's SH basis).
+constexpr int kSplitMaxViews = 2;
 
-template <bool kAdam, bool kPacked, bool kHalf>
-__global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_kernel(const Args a) {
+template <bool kAdam, bool kPacked, bool kHalf, bool kSplit>
+__global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) project_bwd_kernel(const Args a) {
     __shared__ float shs[48][kBwdBlock];  // this thread's SH coefficients, column threadIdx.x
+    // kSplit: this thread's masked colour gradient of every view, kept for the SH pass
+    __shared__ float gcs[kSplit ? 3 * kMaxViews : 1][kBwdBlock];
     const int t = threadIdx.x;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + t; i < a.n; i += int64_t(gridDim.x) * blockDim.x) {
         unsigned vis = 0u;
@@ -407,14 +417,21 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
                 }
                 const float gcol[3] = {raw[0] < 0.f ? 0.f : grg.x, raw[1] < 0.f ? 0.f : grg.y,
                                        raw[2] < 0.f ? 0.f : grg.z};
+                if (kSplit) {
+                    gcs[3 * v + 0][t] = gcol[0];
+                    gcs[3 * v + 1][t] = gcol[1];
+                    gcs[3 * v + 2][t] = gcol[2];
+                }
                 float wk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     if (k < nc) {
                         const float s0 = shs[3 * k][t], s1 = shs[3 * k + 1][t], s2 = shs[3 * k + 2][t];
-                        gsh[3 * k + 0] = fmaf(Y[k], gcol[0], gsh[3 * k + 0]);
-                        gsh[3 * k + 1] = fmaf(Y[k], gcol[1], gsh[3 * k + 1]);
-                        gsh[3 * k + 2] = fmaf(Y[k], gcol[2], gsh[3 * k + 2]);
+                        if (!kSplit) {
+                            gsh[3 * k + 0] = fmaf(Y[k], gcol[0], gsh[3 * k + 0]);
+                            gsh[3 * k + 1] = fmaf(Y[k], gcol[1], gsh[3 * k + 1]);
+                            gsh[3 * k + 2] = fmaf(Y[k], gcol[2], gsh[3 * k + 2]);
+                        }
                         wk[k] = s0 * gcol[0] + s1 * gcol[1] + s2 * gcol[2];
                     } else {
                         wk[k] = 0.f;
@@ -478,11 +495,6 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
             add4(a.d_quats, i, g_quats);
             add4(a.d_log_scales, i, g_ls);
             a.d_logits[i] += g_logit;
-#pragma unroll
-            for (int p = 0; p < 12; ++p)
-                if (p < a.planes)
-                    add4(a.d_sh, int64_t(p) * a.n + i,
-                         make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]));
         }
         if (kAdam) {
             adam4(a.p_means, a.m_means, a.v_means, i, g_means, a.lr_t[0], a);
@@ -492,6 +504,39 @@ __global__ void __launch_bounds__(kBwdBlock, GS_PBWD_MIN_BLOCKS) project_bwd_ker
             a.p_logits[i] = adam_one(a.p_logits[i], g_logit, mm, vv, a.lr_t[3], a);
             a.m_logits[i] = mm;
             a.v_logits[i] = vv;
+        }
+        if (kSplit && vis) {
+            // the SH pass, after the geometric chain has released its registers:
+            // dL/dc_k = sum over the visible views of Y_k(direction) x the masked colour
+            // gradient, the basis recomputed as in the first pass
+            const float4 m4 = __ldg(a.means + i);
+            const double mu[3] = {m4.x, m4.y, m4.z};
+            for (unsigned rest = vis; rest; rest &= rest - 1u) {
+                const int v = __ffs(rest) - 1;
+                const ViewArgs& cam = a.view[v];
+                const double dvx = mu[0] - cam.cc[0], dvy = mu[1] - cam.cc[1], dvz = mu[2] - cam.cc[2];
+                const double dn = sqrt(dvx * dvx + dvy * dvy + dvz * dvz);
+                float Y[16];
+                sh_basis<float>(a.deg, float(dvx / dn), float(dvy / dn), float(dvz / dn), Y);
+                const float gcol[3] = {gcs[3 * v][t], gcs[3 * v + 1][t], gcs[3 * v + 2][t]};
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    if (k < nc) {
+                        gsh[3 * k + 0] = fmaf(Y[k], gcol[0], gsh[3 * k + 0]);
+                        gsh[3 * k + 1] = fmaf(Y[k], gcol[1], gsh[3 * k + 1]);
+                        gsh[3 * k + 2] = fmaf(Y[k], gcol[2], gsh[3 * k + 2]);
+                    }
+                }
+            }
+        }
+        if (a.d_means) {
+#pragma unroll
+            for (int p = 0; p < 12; ++p)
+                if (p < a.planes)
+                    add4(a.d_sh, int64_t(p) * a.n + i,
+                         make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]));
+        }
+        if (kAdam) {
 #pragma unroll
             for (int p = 0; p < 12; ++p)
                 if (p < a.planes)
@@ -581,15 +626,19 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
         a.sh_half = reinterpret_cast<const uint2*>(adam->sh_half);
         a.sh_half_out = reinterpret_cast<uint2*>(adam->sh_half_out);
         if (adam->sh_half)
-            project_bwd_kernel<true, false, true><<<grid, kBwdBlock, 0, s>>>(a);
+            project_bwd_kernel<true, false, true, false><<<grid, kBwdBlock, 0, s>>>(a);
         else if (slots)
-            project_bwd_kernel<true, true, false><<<grid, kBwdBlock, 0, s>>>(a);
+            project_bwd_kernel<true, true, false, false><<<grid, kBwdBlock, 0, s>>>(a);
+        else if (V <= kSplitMaxViews)
+            project_bwd_kernel<true, false, false, true><<<grid, kBwdBlock, 0, s>>>(a);
         else
-            project_bwd_kernel<true, false, false><<<grid, kBwdBlock, 0, s>>>(a);
+            project_bwd_kernel<true, false, false, false><<<grid, kBwdBlock, 0, s>>>(a);
     } else if (slots) {
-        project_bwd_kernel<false, true, false><<<grid, kBwdBlock, 0, s>>>(a);
+        project_bwd_kernel<false, true, false, false><<<grid, kBwdBlock, 0, s>>>(a);
+    } else if (V <= kSplitMaxViews) {
+        project_bwd_kernel<false, false, false, true><<<grid, kBwdBlock, 0, s>>>(a);
     } else {
-        project_bwd_kernel<false, false, false><<<grid, kBwdBlock, 0, s>>>(a);
+        project_bwd_kernel<false, false, false, false><<<grid, kBwdBlock, 0, s>>>(a);
     }
     count_launches(1);
     return cudaGetLastError();
