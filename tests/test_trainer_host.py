@@ -1,0 +1,74 @@
+"""Host logic of the Trainer that runs without a GPU: the view groups of the
+batched path, the lookup of a view's depth-order row, the packed layout's buffers
+and their resizing after densification, and the option checks.  Device work is
+not called: the Trainer is built on CPU tensors, whose allocations and the
+library's host-side size queries need no GPU."""
+import numpy as np
+import pytest
+import torch
+
+from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+from gaussian_splatting_differentiable_02_b200 import scenes
+
+LRS = dict(scenes.ADAM_LR)
+
+
+def _trainer(n_views=5, n=300, **kw):
+    rng = np.random.default_rng(0)
+    scene = scenes.random_scene(rng, n, 1)
+    cams = []
+    for k in range(n_views):
+        R, t = scenes.look_at((np.cos(k), 0.3, np.sin(k) - 4.0))
+        cams.append(scenes.camera(R, t, 64.0, 64.0, 32.0, 32.0, 64, 64))
+    views = [pl.View(n, c, device="cpu") for c in cams]
+    targets = [torch.zeros((64, 64, 3)) for _ in cams]
+    return pl.Trainer(pl.Gaussians.from_scene(scene, device="cpu"), views, targets, dict(LRS), densify=True, **kw)
+
+
+@pytest.mark.parametrize("n_views,groups,want", [
+    (5, 1, [[0, 1, 2, 3, 4]]),
+    (5, 2, [[0, 1, 2], [3, 4]]),
+    (5, 5, [[0], [1], [2], [3], [4]]),
+    (5, 9, [[0], [1], [2], [3], [4]]),
+    (16, 3, [list(range(0, 6)), list(range(6, 12)), list(range(12, 16))]),
+    (1, 4, [[0]]),
+])
+def test_view_groups_cover_every_view_once_in_order(n_views, groups, want):
+    tr = _trainer(n_views, groups=groups)
+    got = tr.view_groups()
+    assert got == want
+    assert [k for ks in got for k in ks] == list(range(n_views))
+    # one depth order per group, each row the view's own
+    assert len(tr.depth_orders) == len(got)
+    for gi, ks in enumerate(got):
+        assert tr.depth_orders[gi].views == len(ks)
+        for j, k in enumerate(ks):
+            assert tr.order_row(k).data_ptr() == tr.depth_orders[gi].order[j].data_ptr()
+
+
+def test_packed_buffers_follow_the_slot_capacity():
+    tr = _trainer(3, n=500, packed=True)
+    assert tr.pcap == 500 and tr.radii is None
+    assert all(pk.slot_of.numel() == 500 and pk.capacity == 500 for pk in tr.packs)
+    assert [p is pk.proj for p, pk in zip(tr.projs, tr.packs)] == [True] * 3
+    assert all(vw.n == 500 for vw in tr.views)
+    keys_before = tr.views[0].keys
+    tr._alloc_packed(200)
+    assert tr.pcap == 200
+    assert all(pk.proj.xy.shape[0] == 200 and pk.ids.numel() == 200 for pk in tr.packs)
+    assert all(d.n == 200 for d in tr.depth_orders)
+    assert all(g.xy.shape[0] == 200 for g in tr.grad2ds)
+    # the visible counters are rows of the step's single read-back tensor
+    for k, pk in enumerate(tr.packs):
+        assert pk.num_visible.data_ptr() == tr.counts[1][k:k + 1].data_ptr()
+    # fewer slots keep the instance buffers (and their contents) of the views
+    assert tr.views[0].keys is keys_before
+
+
+def test_option_checks():
+    with pytest.raises(ValueError):
+        _trainer(2, packed=True, batched_sort=False)
+    with pytest.raises(ValueError):
+        _trainer(2, sh16=True, packed=True)
+    with pytest.raises(ValueError):
+        _trainer(2, sh16=True, fused=False)
