@@ -470,8 +470,8 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
-                       "depth_sort": "per view" if args.per_view_sort else
-                       f"batched over the views, in {len(tr.view_groups())} pipelined view groups",
+                       "depth_sort": "per view" if args.per_view_sort else "batched over the views" + (
+                           f", in {len(tr.view_groups())} pipelined view groups" if len(tr.view_groups()) > 1 else ""),
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -541,31 +541,42 @@ def measure_variants(tr, torch, reps: int = 10):
     return res
 
 
+def paired_step_ms(tr_a, tr_b, steps, torch, rounds: int = 2):
+    """Mean step time of two Trainers, timed in alternating segments of `steps` steps
+    (a, b, a, b, ...) after 3 warm-up steps each, so that a drift of the clocks over
+    the run affects both alike."""
+    s = torch.cuda.current_stream()
+    for t in (tr_a, tr_b):
+        for _ in range(3):
+            t.step()
+    tot = [0.0, 0.0]
+    for _ in range(rounds):
+        for i, t in enumerate((tr_a, tr_b)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(steps):
+                t.step()
+            e1.record(s)
+            torch.cuda.synchronize()
+            tot[i] += e0.elapsed_time(e1)
+    return tot[0] / (rounds * steps), tot[1] / (rounds * steps)
+
+
 def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     """The packed layout (gs_project_packed): the training step with packed views against
-    the same step unpacked (CUDA events over `steps` steps each, after 3 warm-up steps of
-    the packed Trainer), and the packed projection of the first view against the plain
-    projection, with the HBM roofline of its algorithmic bytes (the projection's bytes as
-    in step_bytes, the visibility read twice and the slot map written, and the visible
-    Gaussians' 52 bytes of features read, written packed, and their ids written)."""
+    the same step unpacked (paired_step_ms), and the packed projection of the first view
+    against the plain projection, with the HBM roofline of its algorithmic bytes (the
+    projection's bytes as in step_bytes, the visibility read twice and the slot map
+    written, and the visible Gaussians' 52 bytes of features read, written packed, and
+    their ids written)."""
     from gaussian_splatting_differentiable_02_b200 import pipeline as pl
     s = torch.cuda.current_stream()
     scene = wl.scene
     trp = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
                      dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, packed=True)
 
-    def step_ms(t):
-        for _ in range(3):
-            t.step()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        for _ in range(steps):
-            t.step()
-        e1.record(s)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / steps
-
-    res = {"step_ms_packed": step_ms(trp), "step_ms_unpacked": step_ms(tr)}
+    ms_packed, ms_unpacked = paired_step_ms(trp, tr, steps, torch)
+    res = {"step_ms_packed": ms_packed, "step_ms_unpacked": ms_unpacked}
     visible = trp.counts[1].cpu().numpy()
     res["visible_fraction_per_view"] = float(visible.mean() / max(scene.n, 1))
     res["slot_capacity"] = int(trp.pcap)
@@ -597,7 +608,7 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
 
 def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     """16-bit SH storage: the training step with the projections reading the half copy
-    (Trainer(sh16=True)) against the float32 step, and the projection of the first view
+    (Trainer(sh16=True)) against the float32 step (paired_step_ms), and the projection of the first view
     from half against float32 coefficients, each with the HBM roofline of its algorithmic
     bytes (the parameters read, with 2 or 4 bytes per SH coefficient, and 52 bytes of
     projected features written)."""
@@ -618,7 +629,8 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / count
 
-    res = {"step_ms_sh16": timed(trh.step, steps), "step_ms_f32": timed(tr.step, steps)}
+    ms_sh16, ms_f32 = paired_step_ms(trh, tr, steps, torch)
+    res = {"step_ms_sh16": ms_sh16, "step_ms_f32": ms_f32}
     n, nc = scene.n, 3 * (scene.sh_degree + 1) ** 2
     for name, fn, sh_bytes in (
             ("f32", lambda: pl.project(tr.gauss, tr.views[0], tr.projs[0], tr.radii[0]), 4),
