@@ -3,9 +3,9 @@
 // §2.1: shared-memory prefetch of the tile's Gaussians, SoA features, warp-level
 // synchronisation; §2.2: a standalone backward entry).
 //
-// Work decomposition: one warp per 16x8 pixel box (two warps per tile, four
-// warps per block, blocks launched in the tile order of gs_tile_order when one
-// is given); each lane owns a column segment of 4 pixels (lane & 15 selects the
+// Work decomposition: one warp per 16x8 pixel box (two warps per tile, one tile
+// per block, blocks launched in the tile order of gs_tile_order when one is
+// given); each lane owns a column segment of 4 pixels (lane & 15 selects the
 // column, lane >> 4 the upper or lower half of the box).  The warp walks its
 // tile's sorted list in batches of 32 entries: every lane gathers one entry's
 // 40 bytes (xy, conic + opacity, colour) by Gaussian index into shared memory
@@ -69,14 +69,19 @@ constexpr int kLaneRows = 32 / kBoxW;    // lanes stacked vertically in the box
 constexpr int kBoxH = kLaneRows * kPx;   // height of a warp's pixel box
 constexpr int kSubX = kTile / kBoxW, kSubY = kTile / kBoxH;
 constexpr int kSub = kSubX * kSubY;      // warps per tile
-constexpr int kWarps = 4;                // warps per block
+#ifndef GS_RASTER_WARPS
+#define GS_RASTER_WARPS 2
+#endif
+// warps per block: one tile's two boxes, so that a block retires with its own tile
+// (two tiles per block: 1% slower, the block waiting for the slower tile)
+constexpr int kWarps = GS_RASTER_WARPS;
 static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
 // resident blocks per SM the register allocation is sized for (launch bounds)
 #ifndef GS_RASTER_FWD_MIN_BLOCKS
-#define GS_RASTER_FWD_MIN_BLOCKS 5
+#define GS_RASTER_FWD_MIN_BLOCKS 10
 #endif
 #ifndef GS_RASTER_BWD_MIN_BLOCKS
-#define GS_RASTER_BWD_MIN_BLOCKS 5
+#define GS_RASTER_BWD_MIN_BLOCKS 10
 #endif
 constexpr int kBatch = 32;  // list entries staged per warp per batch
 constexpr unsigned kFull = 0xffffffffu;
