@@ -542,9 +542,9 @@ def measure_variants(tr, torch, reps: int = 10):
 
 
 def paired_step_ms(tr_a, tr_b, steps, torch, rounds: int = 2):
-    """Mean step time of two Trainers, timed in alternating segments of `steps` steps
-    (a, b, a, b, ...) after 3 warm-up steps each, so that a drift of the clocks over
-    the run affects both alike."""
+    """Mean step time of two Trainers started from the same scene, timed in alternating
+    segments of `steps` steps (a, b, a, b, ...) after 3 warm-up steps each, so that a
+    drift of the clocks over the run affects both alike."""
     s = torch.cuda.current_stream()
     for t in (tr_a, tr_b):
         for _ in range(3):
@@ -575,7 +575,12 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     trp = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
                      dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, packed=True)
 
-    ms_packed, ms_unpacked = paired_step_ms(trp, tr, steps, torch)
+    # the unpacked arm starts from the same scene (the benchmark's own Trainer has
+    # trained for many steps by now, and its Gaussians have moved)
+    tru = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups)
+    ms_packed, ms_unpacked = paired_step_ms(trp, tru, steps, torch)
+    del tru
     res = {"step_ms_packed": ms_packed, "step_ms_unpacked": ms_unpacked}
     visible = trp.counts[1].cpu().numpy()
     res["visible_fraction_per_view"] = float(visible.mean() / max(scene.n, 1))
@@ -629,7 +634,10 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / count
 
-    ms_sh16, ms_f32 = paired_step_ms(trh, tr, steps, torch)
+    trf = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups)
+    ms_sh16, ms_f32 = paired_step_ms(trh, trf, steps, torch)
+    del trf
     res = {"step_ms_sh16": ms_sh16, "step_ms_f32": ms_f32}
     n, nc = scene.n, 3 * (scene.sh_degree + 1) ** 2
     for name, fn, sh_bytes in (
