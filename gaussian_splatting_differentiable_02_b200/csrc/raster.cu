@@ -238,30 +238,34 @@ __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c
 __device__ __forceinline__ f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 
-// One entry at the lane's pixels: -alpha per pixel (pairs 2p, 2p + 1), the
-// offsets dx (shared) and dy of the mean from the pixel centres, t = dx +
-// (B/A) dy for a factored entry; bit i of `blend` is set when pixel i passes
-// sigma >= 0 and alpha >= 1/255, bit i of `clamp` when alpha was clamped at 0.99.
+// One entry at the lane's pixels: -alpha per pixel (pairs 2p, 2p + 1; 0 where the
+// pixel fails sigma >= 0 or alpha >= 1/255, so that it does not blend the entry),
+// the offsets dx (shared) and dy of the mean from the pixel centres, t = dx +
+// (B/A) dy for a factored entry; bit i of `clamp` is set when alpha was clamped at
+// 0.99 (backward pass only).  The masks are floats rather than bits: a pixel that
+// does not take an entry runs the same paired instructions with alpha 0.
 struct Alpha {
     f2 nal[kPairs];
     f2 dy[kPairs];
     f2 t[kPairs];
-    unsigned blend, clamp;
+    unsigned clamp;
     float dx;
 };
 
-__device__ __forceinline__ void alpha_at(float e, bool sign_ok, int i, float& nal, unsigned& blend,
-                                         unsigned& clamp) {
+// -alpha at one pixel, 0 for a pixel that does not blend the entry (sigma < 0 or
+// alpha < 1/255); with kClamp, bit i of `clamp` is set when alpha was clamped at 0.99.
+template <bool kClamp>
+__device__ __forceinline__ void alpha_at(float e, bool sign_ok, int i, float& nal, unsigned& clamp) {
     const float a = ex2_approx(e);
     nal = fmaxf(-a, -kAlphaMax);  // -min(a, 0.99)
-    if (sign_ok && nal <= -kAlphaMin) blend |= 1u << i;
-    if (a > kAlphaMax) clamp |= 1u << i;
+    nal = (sign_ok && nal <= -kAlphaMin) ? nal : 0.f;
+    if (kClamp && a > kAlphaMax) clamp |= 1u << i;
 }
 
 // nyc[p]: minus the centres' y of the lane's pixels 2p and 2p + 1.
+template <bool kClamp>
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
                                            float px, const f2 (&nyc)[kPairs], Alpha& r) {
-    r.blend = 0u;
     r.clamp = 0u;
     const f2 vy = splat(pa.y), lo = splat(pa.z);
     if (pb.w >= kFactored) {
@@ -275,8 +279,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             const f2 sv = fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p]));
             const f2 e = add2(sv, lo);
             // sigma >= 0 by construction unless the conic is indefinite
-            alpha_at(e.x, !indef || sv.x <= 0.f, 2 * p, r.nal[p].x, r.blend, r.clamp);
-            alpha_at(e.y, !indef || sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
+            alpha_at<kClamp>(e.x, !indef || sv.x <= 0.f, 2 * p, r.nal[p].x, r.clamp);
+            alpha_at<kClamp>(e.y, !indef || sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.clamp);
         }
     } else {
         r.dx = __fsub_rn(pa.x, px);
@@ -288,8 +292,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             // a positive-definite form has sigma >= 0; the float32 value can round
             // below zero only within rounding of the mean, where alpha is o either way
             const f2 e = add2(fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0), lo);
-            alpha_at(e.x, true, 2 * p, r.nal[p].x, r.blend, r.clamp);
-            alpha_at(e.y, true, 2 * p + 1, r.nal[p].y, r.blend, r.clamp);
+            alpha_at<kClamp>(e.x, true, 2 * p, r.nal[p].x, r.clamp);
+            alpha_at<kClamp>(e.y, true, 2 * p + 1, r.nal[p].y, r.clamp);
         }
     }
 }
@@ -328,16 +332,24 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     f2 nyc[kPairs], T[kPairs], Cr[kPairs], Cg[kPairs], Cb[kPairs];
     int last[kPx];
     unsigned done = 0u;
+    f2 on[kPairs];  // 1 while the pixel composites, 0 once it has stopped (or lies outside the image)
 #pragma unroll
     for (int p = 0; p < kPairs; ++p) {
         nyc[p] = make_float2(-(float(y0 + 2 * p) + 0.5f), -(float(y0 + 2 * p + 1) + 0.5f));
         T[p] = splat(1.f);
         Cr[p] = Cg[p] = Cb[p] = splat(0.f);
+        on[p] = splat(1.f);
     }
 #pragma unroll
     for (int i = 0; i < kPx; ++i) {
         last[i] = 0;
-        if (x >= a.W || y0 + i >= a.H) done |= 1u << i;
+        if (x >= a.W || y0 + i >= a.H) {
+            done |= 1u << i;
+            if (i & 1)
+                on[i / 2].y = 0.f;
+            else
+                on[i / 2].x = 0.f;
+        }
     }
     constexpr unsigned kAll = (1u << kPx) - 1u;
     const f2 one = splat(1.f);
@@ -365,30 +377,32 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
             const float4 con = S.con[buf][j];
             const float4 nc = S.rgb[buf][j];  // minus the colour
             Alpha r;
-            eval_alpha(pa, pb, S.pc[e], con, px, nyc, r);
-            const unsigned blend = r.blend & ~done;
             const int pos = b * kBatch + j + 1;
             const f2 ncr = splat(nc.x), ncg = splat(nc.y), ncb = splat(nc.z);
-            // branch-free so the pixel chains interleave; a pixel that does not
-            // take the entry adds c * 0 (exactly nothing)
+            eval_alpha<false>(pa, pb, S.pc[e], con, px, nyc, r);
+            // branch-free with float masks: -alpha is 0 for a pixel that does not blend
+            // the entry or has stopped (on 0), so T (1 - alpha) = T and -alpha T = 0
+            // leave it exactly as it was; T (1 - alpha) < 1e-4 then only happens for a
+            // pixel that blends, which stops there without taking the entry
 #pragma unroll
             for (int p = 0; p < kPairs; ++p) {
-                const f2 Tn = mul2(T[p], add2(one, r.nal[p]));  // T (1 - alpha)
-                f2 nw = mul2(r.nal[p], T[p]);                    // -alpha T
-                const bool act0 = (blend >> (2 * p)) & 1u, act1 = (blend >> (2 * p + 1)) & 1u;
+                const f2 na = mul2(r.nal[p], on[p]);
+                const f2 Tn = mul2(T[p], add2(one, na));  // T (1 - alpha)
+                f2 nw = mul2(na, T[p]);                    // -alpha T
                 const bool low0 = Tn.x < kTMin, low1 = Tn.y < kTMin;
-                const bool take0 = act0 && !low0, take1 = act1 && !low1;
-                nw.x = take0 ? nw.x : 0.f;
-                nw.y = take1 ? nw.y : 0.f;
+                nw.x = low0 ? 0.f : nw.x;
+                nw.y = low1 ? 0.f : nw.y;
                 Cr[p] = fma2(ncr, nw, Cr[p]);
                 Cg[p] = fma2(ncg, nw, Cg[p]);
                 Cb[p] = fma2(ncb, nw, Cb[p]);
-                T[p].x = take0 ? Tn.x : T[p].x;
-                T[p].y = take1 ? Tn.y : T[p].y;
-                last[2 * p] = take0 ? pos : last[2 * p];
-                last[2 * p + 1] = take1 ? pos : last[2 * p + 1];
-                done |= (act0 && low0) ? (1u << (2 * p)) : 0u;
-                done |= (act1 && low1) ? (1u << (2 * p + 1)) : 0u;
+                T[p].x = low0 ? T[p].x : Tn.x;
+                T[p].y = low1 ? T[p].y : Tn.y;
+                last[2 * p] = (na.x != 0.f && !low0) ? pos : last[2 * p];
+                last[2 * p + 1] = (na.y != 0.f && !low1) ? pos : last[2 * p + 1];
+                on[p].x = low0 ? 0.f : on[p].x;
+                on[p].y = low1 ? 0.f : on[p].y;
+                done |= low0 ? (1u << (2 * p)) : 0u;
+                done |= low1 ? (1u << (2 * p + 1)) : 0u;
             }
         }
         __syncwarp();
@@ -548,7 +562,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
             Alpha r;
-            eval_alpha(pa, pb, S.pc[e], con, px, nyc, r);
+            eval_alpha<true>(pa, pb, S.pc[e], con, px, nyc, r);
             const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
             f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
             bool any = false;
@@ -556,10 +570,10 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             // with alpha 0, so T, P and every sum stay unchanged
 #pragma unroll
             for (int p = 0; p < kPairs; ++p) {
-                const bool act0 = ((r.blend >> (2 * p)) & 1u) && pos < last[2 * p];
-                const bool act1 = ((r.blend >> (2 * p + 1)) & 1u) && pos < last[2 * p + 1];
-                any = any || act0 || act1;
-                const f2 nae = make_float2(act0 ? r.nal[p].x : 0.f, act1 ? r.nal[p].y : 0.f);  // -alpha
+                // -alpha, 0 where the pixel does not blend the entry or has not reached it
+                const f2 nae = make_float2(pos < last[2 * p] ? r.nal[p].x : 0.f,
+                                           pos < last[2 * p + 1] ? r.nal[p].y : 0.f);
+                any = any || nae.x != 0.f || nae.y != 0.f;
                 const f2 om = add2(one, nae);                                                  // 1 - alpha
                 const f2 rom = make_float2(rcp_approx(om.x), rcp_approx(om.y));
                 T[p] = mul2(T[p], rom);  // transmittance in front of this entry
