@@ -241,32 +241,32 @@ __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 // One entry at the lane's pixels: -alpha per pixel (pairs 2p, 2p + 1; 0 where the
 // pixel fails sigma >= 0 or alpha >= 1/255, so that it does not blend the entry),
 // the offsets dx (shared) and dy of the mean from the pixel centres, t = dx +
-// (B/A) dy for a factored entry; bit i of `clamp` is set when alpha was clamped at
-// 0.99 (backward pass only).  The masks are floats rather than bits: a pixel that
-// does not take an entry runs the same paired instructions with alpha 0.
+// (B/A) dy for a factored entry, and (backward pass) a gate that is 0 where alpha
+// was clamped at 0.99 and 1 elsewhere.  The masks are floats rather than bits: a
+// pixel that does not take an entry runs the same paired instructions with alpha
+// 0, and a clamped pixel's dL/dsigma is multiplied by 0.
 struct Alpha {
     f2 nal[kPairs];
     f2 dy[kPairs];
     f2 t[kPairs];
-    unsigned clamp;
+    f2 gate[kPairs];  // 0 where alpha was clamped at 0.99, else 1 (backward pass)
     float dx;
 };
 
 // -alpha at one pixel, 0 for a pixel that does not blend the entry (sigma < 0 or
-// alpha < 1/255); with kClamp, bit i of `clamp` is set when alpha was clamped at 0.99.
+// alpha < 1/255); with kClamp, gate = 0 when alpha was clamped at 0.99, else 1.
 template <bool kClamp>
-__device__ __forceinline__ void alpha_at(float e, bool sign_ok, int i, float& nal, unsigned& clamp) {
+__device__ __forceinline__ void alpha_at(float e, bool sign_ok, float& nal, float& gate) {
     const float a = ex2_approx(e);
     nal = fmaxf(-a, -kAlphaMax);  // -min(a, 0.99)
     nal = (sign_ok && nal <= -kAlphaMin) ? nal : 0.f;
-    if (kClamp && a > kAlphaMax) clamp |= 1u << i;
+    if (kClamp) gate = a > kAlphaMax ? 0.f : 1.f;
 }
 
 // nyc[p]: minus the centres' y of the lane's pixels 2p and 2p + 1.
 template <bool kClamp>
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
                                            float px, const f2 (&nyc)[kPairs], Alpha& r) {
-    r.clamp = 0u;
     const f2 vy = splat(pa.y), lo = splat(pa.z);
     if (pb.w >= kFactored) {
         const bool indef = pb.w == kFactoredIndef;
@@ -279,8 +279,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             const f2 sv = fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p]));
             const f2 e = add2(sv, lo);
             // sigma >= 0 by construction unless the conic is indefinite
-            alpha_at<kClamp>(e.x, !indef || sv.x <= 0.f, 2 * p, r.nal[p].x, r.clamp);
-            alpha_at<kClamp>(e.y, !indef || sv.y <= 0.f, 2 * p + 1, r.nal[p].y, r.clamp);
+            alpha_at<kClamp>(e.x, !indef || sv.x <= 0.f, r.nal[p].x, r.gate[p].x);
+            alpha_at<kClamp>(e.y, !indef || sv.y <= 0.f, r.nal[p].y, r.gate[p].y);
         }
     } else {
         r.dx = __fsub_rn(pa.x, px);
@@ -292,8 +292,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             // a positive-definite form has sigma >= 0; the float32 value can round
             // below zero only within rounding of the mean, where alpha is o either way
             const f2 e = add2(fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0), lo);
-            alpha_at<kClamp>(e.x, true, 2 * p, r.nal[p].x, r.clamp);
-            alpha_at<kClamp>(e.y, true, 2 * p + 1, r.nal[p].y, r.clamp);
+            alpha_at<kClamp>(e.x, true, r.nal[p].x, r.gate[p].x);
+            alpha_at<kClamp>(e.y, true, r.nal[p].y, r.gate[p].y);
         }
     }
 }
@@ -585,9 +585,8 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                 const f2 xg = add2(fma2(gr[p], cr, fma2(gg[p], cg, mul2(gb[p], cb))), nP[p]);  // g . c - P
                 const f2 dLda = fma2(T[p], xg, mul2(ngb[p], rom));
                 nP[p] = fma2(nae, xg, nP[p]);
-                f2 q = mul2(dLda, nae);  // -dL/dalpha alpha = dL/dsigma (zero when clamped)
-                q.x = ((r.clamp >> (2 * p)) & 1u) ? 0.f : q.x;
-                q.y = ((r.clamp >> (2 * p + 1)) & 1u) ? 0.f : q.y;
+                // -dL/dalpha alpha = dL/dsigma, zero where alpha was clamped (times a 0/1 gate)
+                const f2 q = mul2(mul2(dLda, nae), r.gate[p]);
                 nm[p] = q;
                 nmo = add2(nmo, q);
                 s1 = fma2(q, r.dy[p], s1);
