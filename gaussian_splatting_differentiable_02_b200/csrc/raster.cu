@@ -331,7 +331,6 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
 
     f2 nyc[kPairs], T[kPairs], Cr[kPairs], Cg[kPairs], Cb[kPairs];
     int last[kPx];
-    unsigned done = 0u;
     f2 on[kPairs];  // 1 while the pixel composites, 0 once it has stopped (or lies outside the image)
 #pragma unroll
     for (int p = 0; p < kPairs; ++p) {
@@ -344,14 +343,12 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     for (int i = 0; i < kPx; ++i) {
         last[i] = 0;
         if (x >= a.W || y0 + i >= a.H) {
-            done |= 1u << i;
             if (i & 1)
                 on[i / 2].y = 0.f;
             else
                 on[i / 2].x = 0.f;
         }
     }
-    constexpr unsigned kAll = (1u << kPx) - 1u;
     const f2 one = splat(1.f);
 
     const int nb = (n + kBatch - 1) / kBatch;
@@ -368,7 +365,10 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         __syncwarp();
         bool finished = false;
         for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
-            if (__all_sync(kFull, done == kAll)) {
+            f2 alive = on[0];  // nonzero while some pixel of the lane composites
+#pragma unroll
+            for (int p = 1; p < kPairs; ++p) alive = add2(alive, on[p]);
+            if (__all_sync(kFull, alive.x + alive.y == 0.f)) {
                 finished = true;
                 break;
             }
@@ -401,8 +401,6 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 last[2 * p + 1] = (na.y != 0.f && !low1) ? pos : last[2 * p + 1];
                 on[p].x = low0 ? 0.f : on[p].x;
                 on[p].y = low1 ? 0.f : on[p].y;
-                done |= low0 ? (1u << (2 * p)) : 0u;
-                done |= low1 ? (1u << (2 * p + 1)) : 0u;
             }
         }
         __syncwarp();
