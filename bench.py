@@ -478,7 +478,8 @@ def run_ours(args, world, rank, local):
                        "l2": "inputs larger than L2: each step streams %.2f GB of parameters, optimizer state, "
                              "instances and images" % (nbytes / 1e9)},
             "hbm": {"algorithmic_bytes_per_step": nbytes, "achieved_gbs": step_gbs, "peak_gbs": hbm_peak,
-                    "frac": step_gbs / hbm_peak, "peak_source": peaks["source"]},
+                    "frac": step_gbs / hbm_peak, "peak_source": peaks["source"],
+                    "frac_of_nominal_8000_gbs": step_gbs / 8000.0},
             "stages_ms_per_step": {k: round(v, 4) for k, v in stages.items()},
             "roofline": roof,
             "gpu_launches": int(launches),
