@@ -446,9 +446,9 @@ class Trainer:
                                # batched sort (gs_depth_order_views), then bin and composite per view
     groups: int = 1            # fused batched path: the views are projected, depth-sorted and binned in
                                # this many consecutive groups, so that a group's projection and depth sort
-                               # overlap the compositing of the groups before it (on the 16-view 1080p
-                               # step 1, 2, 4, 8 groups take 44.4, 44.6, 44.8, 45.1 ms: compositing
-                               # already fills the device, and the overlap only adds launches)
+                               # overlap the compositing of the groups before it (slower on the 16-view
+                               # 1080p step: compositing already fills the device, and the overlap only
+                               # adds launches)
     packed: bool = False       # fused batched path: views in the packed layout (gs_project_packed, the
                                # gsplat guide §4.1 packed option); the slot capacity follows the largest
                                # visible count seen
