@@ -72,3 +72,19 @@ def test_option_checks():
         _trainer(2, sh16=True, packed=True)
     with pytest.raises(ValueError):
         _trainer(2, sh16=True, fused=False)
+
+
+def test_view_set_n_keeps_or_grows_the_instance_buffers():
+    R, t = scenes.look_at((0.0, 0.0, -4.0))
+    cam = scenes.camera(R, t, 64.0, 64.0, 32.0, 32.0, 64, 64)
+    view = pl.View(1000, cam, device="cpu")
+    assert view.capacity == 4000
+    keys = view.keys
+    view.set_n(200)                      # fewer Gaussians: same buffers, same contents
+    assert view.keys is keys and view.capacity == 4000 and view.n == 200
+    ws = view.workspace.numel()
+    view.set_n(3000)                     # more: the capacity grows to 4 n, new buffers
+    assert view.capacity == 12000 and view.keys is not keys
+    assert view.workspace.numel() >= ws
+    from gaussian_splatting_differentiable_02_b200 import abi
+    assert view.workspace.numel() >= abi.gs_bin_sort_workspace_bytes(3000, 12000, view.gcam)
