@@ -202,3 +202,16 @@ def test_workspace_grows_with_capacity(gs):
     b = gs.gs_bin_sort_workspace_bytes(1000, 1_000_000, c)
     assert 0 < a < b
     assert b >= 12 * 1_000_000          # the ping-pong key/value copy
+
+
+def test_binding_argument_counts_match_the_header(gs):
+    """Every prototype of include/gs.h takes as many parameters as the ctypes binding
+    passes (a missing or extra argument would be undefined behaviour at the call)."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"\b(?:gs_status|size_t|int32_t|uint64_t|const char\s*\*)\s+(gs_[a-z0-9_]+)\s*\(([^;]*?)\)\s*;",
+                       text, flags=re.S)
+    assert {name for name, _ in decls} == set(declared_functions())
+    for name, params in decls:
+        p = params.strip()
+        n = 0 if p in ("", "void") else p.count(",") + 1
+        assert n == len(gs.SIGNATURES[name][1]), (name, n, len(gs.SIGNATURES[name][1]))
