@@ -333,9 +333,10 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
  * later call takes the packed arrays as it takes gs_project's, with n replaced
  * by the capacity: the binning's values, the raster calls' 2D gradients and the
  * instance lists are then indexed by slot.  Because slots ascend with the
- * Gaussian id, the sort keys, the order of equal keys, the images and the
- * gradients are those of the unpacked layout with every value v replaced by
- * gaussian_ids[v].
+ * Gaussian id, the sort keys and the order of equal keys are those of the
+ * unpacked layout with every value v replaced by gaussian_ids[v], the images are
+ * the same bit for bit, and the 2D gradients are the same sums (added in an order
+ * the atomics choose, as in the unpacked layout).
  *
  * gs_project_packed_workspace_bytes -- device workspace for n Gaussians (about
  * 60 bytes per Gaussian: gs_project's outputs for all of them, before packing).
@@ -351,7 +352,10 @@ gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, 
  * features), so the later calls skip them.  V > capacity is not an error of the
  * call: slots up to capacity are filled, slot_of is -1 for the Gaussians that got
  * none, and the caller compares V (read when convenient) with the capacity and
- * repeats with more room before using the results.  Asynchronous, no host wait. */
+ * repeats with more room before using the results.  Asynchronous, no host wait.
+ * Errors (nothing launched): GS_ERR_INVALID_ARG for a NULL or misaligned pointer,
+ * a capacity outside 0..2^31-1 or a workspace smaller than
+ * gs_project_packed_workspace_bytes(params->n); GS_ERR_UNSUPPORTED as gs_project. */
 size_t gs_project_packed_workspace_bytes(int64_t n);
 gs_status gs_project_packed(const gs_params* params, const gs_camera* cam, void* workspace, size_t workspace_bytes,
                             gs_projected* packed, int64_t capacity, uint32_t* gaussian_ids, int32_t* slot_of,
