@@ -399,7 +399,11 @@ gs_status gs_project_bwd_views_adam_packed(const gs_params* params, int32_t num_
  * coefficients in sh_half (the values the forward pass used), Adam updates the
  * float32 coefficients params_inout->sh (the master copy), and each updated
  * float32 coefficient is written, rounded as by gs_to_half, to sh_half_out
- * (which may be sh_half itself).  Unpacked views only. */
+ * (which may be sh_half itself).  Unpacked views only.
+ *
+ * Errors (nothing launched): GS_ERR_INVALID_ARG for a negative count, a NULL or
+ * misaligned pointer (sh_half and sh_half_out 8-byte aligned when n > 0), and
+ * otherwise as the float32 calls. */
 gs_status gs_to_half(const float* x, int64_t count, uint16_t* out, void* stream);
 gs_status gs_project_sh16(const gs_params* params, const uint16_t* sh_half, const gs_camera* cam, gs_projected* out,
                           void* stream);
