@@ -11,40 +11,30 @@
 // The array is a file-scope __device__ variable, so every device that loads
 // the library holds GS_STATIC_SCRATCH_BYTES of it until the process exits.  In
 // host code its name is a host-side shadow, not a device address: the address
-// comes from cudaGetSymbolAddress, taken once per device (with that device
-// current) on the first call on that device and cached.
+// comes from cudaGetSymbolAddress, looked up on every call in the current
+// device's current context.  An address belongs to a context, not to a device
+// number: after cudaDeviceReset, or in a host that creates its own contexts,
+// a cached one would point at memory the new context never mapped.  The lookup
+// allocates nothing; the first one in a context loads the library's module
+// there (which is when the array itself comes into being).
 //
 // All calls share the one array and it keeps whatever the previous call left:
 // every word the sort reads is written earlier in the same call (block sums,
 // total, histograms, digit totals, the ping-pong copy), so nothing needs to be
 // cleared first.  Calls whose work overlaps on the GPU (different streams,
 // or threads racing on one device) corrupt each other's scratch: serialise them.
-#include <mutex>
-
 #include "internal.cuh"
 
 namespace {
 
 __device__ __align__(256) unsigned char g_static_scratch[GS_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device (set-up on first use).
+// Device address of the scratch array in the current context.
 cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return e;
-        g_addr[dev] = p;
-    }
-    *out = g_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

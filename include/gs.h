@@ -226,9 +226,11 @@ gs_status gs_bin_sort_ordered_async(const gs_projected* proj, int64_t n, const u
  *   - n and capacity whose workspace (gs_bin_sort_workspace_bytes) exceeds
  *     GS_STATIC_SCRATCH_BYTES return GS_ERR_UNSUPPORTED (the workspace is
  *     about 16 bytes per slot of max(capacity, n): about 2 million).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make that
- *     first call before any stream capture.
+ *   - Every call looks up the array's address in the current context
+ *     (cudaGetSymbolAddress, no allocation), so it stays valid after a
+ *     cudaDeviceReset and in contexts the host creates itself.  The first call
+ *     in a context loads the library's module there, which is when the array
+ *     comes into being: make that first call before any stream capture.
  *   - All calls share the array.  Calls whose GPU work overlaps (other streams,
  *     other threads on the same device) race on it: serialise them.  No state
  *     carries over between calls; nothing in it needs clearing.

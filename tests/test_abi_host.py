@@ -215,3 +215,36 @@ def test_binding_argument_counts_match_the_header(gs):
         p = params.strip()
         n = 0 if p in ("", "void") else p.count(",") + 1
         assert n == len(gs.SIGNATURES[name][1]), (name, n, len(gs.SIGNATURES[name][1]))
+
+
+def test_static_scratch_size_matches_the_header(gs):
+    """The binding's GS_STATIC_SCRATCH_BYTES is the header's #define, not a stale copy."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+GS_STATIC_SCRATCH_BYTES\s+\(\(size_t\)\s*(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "GS_STATIC_SCRATCH_BYTES not found in gs.h"
+    assert int(m.group(1)) << int(m.group(2)) == gs.GS_STATIC_SCRATCH_BYTES
+
+
+def test_static_scratch_limit_is_checked_at_the_boundary(gs):
+    """gs_bin_sort_static rejects, before it touches a device, the smallest capacity whose
+    workspace exceeds the static scratch, and lets the largest one that fits through to
+    its next checks (here the missing device or the NULL buffers, never the size)."""
+    c = gs.make_camera(cam())
+    n = 1000
+    lo, hi = 1, 1 << 26   # workspace(lo) fits, workspace(hi) does not
+    assert gs.gs_bin_sort_workspace_bytes(n, lo, c) <= gs.GS_STATIC_SCRATCH_BYTES
+    assert gs.gs_bin_sort_workspace_bytes(n, hi, c) > gs.GS_STATIC_SCRATCH_BYTES
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if gs.gs_bin_sort_workspace_bytes(n, mid, c) <= gs.GS_STATIC_SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid
+    proj = gs.gs_projected()
+    K = C.c_int64(0)
+    L = gs.lib()
+    st = L.gs_bin_sort_static(C.byref(proj), n, C.byref(c), None, None, hi, C.byref(K), None, None)
+    assert st == gs.GS_ERR_UNSUPPORTED
+    assert "static scratch" in L.gs_last_error_detail().decode()
+    st = L.gs_bin_sort_static(C.byref(proj), n, C.byref(c), None, None, lo, C.byref(K), None, None)
+    assert st not in (gs.GS_OK, gs.GS_ERR_UNSUPPORTED)

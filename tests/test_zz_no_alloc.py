@@ -30,15 +30,27 @@ def _with_workspace(proj, view):
     return K, view.keys[:K].clone(), view.vals[:K].clone(), view.ranges.clone()
 
 
-def _with_static_scratch(proj, view, capacity):
+def _outputs(capacity, view):
     keys = torch.zeros(capacity, dtype=torch.int64, device="cuda")
     vals = torch.zeros(capacity, dtype=torch.int32, device="cuda")
     ranges = torch.full_like(view.ranges, -1)
-    st, K = abi.gs_bin_sort_static(proj.struct(), view.n, view.gcam, keys.data_ptr(), vals.data_ptr(), capacity,
+    torch.cuda.synchronize()
+    return keys, vals, ranges
+
+
+def _with_static_scratch(proj, view, out):
+    """One gs_bin_sort_static call into the preallocated `out`; returns its results and
+    the device's free bytes and torch's allocated bytes before and after the call."""
+    keys, vals, ranges = out
+    ranges.fill_(-1)
+    torch.cuda.synchronize()
+    before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated())
+    st, K = abi.gs_bin_sort_static(proj.struct(), view.n, view.gcam, keys.data_ptr(), vals.data_ptr(), keys.numel(),
                                    ranges.data_ptr(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
+    after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated())
     assert st == abi.GS_OK
-    return K, keys[:K], vals[:K], ranges
+    return (K, keys[:K], vals[:K], ranges), before, after
 
 
 def test_static_scratch_matches_caller_workspace_on_consecutive_calls():
@@ -51,11 +63,16 @@ def test_static_scratch_matches_caller_workspace_on_consecutive_calls():
     for scene, cam in cases:
         g, view, proj = _inputs(scene, cam)
         want = _with_workspace(proj, view)
-        for _ in range(2):                       # two calls in a row on the shared scratch
-            got = _with_static_scratch(proj, view, capacity=want[0] + 1000)
+        out = _outputs(want[0] + 1000, view)
+        for call in range(2):                    # two calls in a row on the shared scratch
+            got, before, after = _with_static_scratch(proj, view, out)
             assert got[0] == want[0] > 0
             for a, b in zip(got[1:], want[1:]):
                 assert torch.equal(a, b)
+            if call == 1:
+                # the module (and with it the array) was loaded by the first call; the
+                # second one takes no device memory, neither from the driver nor from torch
+                assert after == before, (before, after)
 
 
 def test_sizes_beyond_the_static_scratch_are_rejected():
