@@ -443,16 +443,38 @@ std::vector<int64_t> tile_candidates(int64_t n, const Features& f, int tx, int t
     return c;
 }
 
+/* The candidates whose alpha at pixel (px, py) could reach the 1/255 threshold
+ * under a relative perturbation of band_alpha (o exp(-sigma) >= (1 - band_alpha)
+ * / 255, or a form so close to indefinite that its sign is not decided), i.e.
+ * every Gaussian a float32 evaluation might blend there, before or after the
+ * pixel's stop.  A Gaussian outside this set takes no gradient from the pixel
+ * whatever the pixel's straddling decisions are. */
+std::vector<int64_t> reachable(const Features& f, const std::vector<int64_t>& cand, int px, int py,
+                               double band_alpha) {
+    std::vector<int64_t> r;
+    const double X = px + 0.5, Yp = py + 0.5;
+    for (int64_t i : cand) {
+        const double dx = f.xy[2 * i] - X, dy = f.xy[2 * i + 1] - Yp;
+        const double A = f.conic[3 * i], B = f.conic[3 * i + 1], Cc = f.conic[3 * i + 2];
+        const double sigma = 0.5 * (A * dx * dx + Cc * dy * dy) + B * dx * dy;
+        const double scale = 0.5 * (std::fabs(A) * dx * dx + std::fabs(Cc) * dy * dy) + std::fabs(B * dx * dy);
+        const double s = sigma <= 1e-6 * scale ? 0.0 : sigma;  // undecided sign: as if at the mean
+        if (f.opac[i] * std::exp(-s) >= (1.0 - band_alpha) * ALPHA_MIN) r.push_back(i);
+    }
+    return r;
+}
+
 /* Composite one pixel front to back over its depth-sorted candidate list.
  * Returns the blended entries (for the reverse pass) and the ambiguity flags:
  *   bit 0: a skip/stop decision lay within the relative band of its threshold
  *          (alpha vs 1/255 or T(1-alpha) vs 1e-4), so float32 evaluation may
  *          legitimately decide the other way;
  *   bit 1: an unclamped alpha lay within the band of the 0.99 clamp (gradients
- *          switch on or off there; values are continuous). */
+ *          switch on or off there; values are continuous); those entries are
+ *          appended to clamp_band when given. */
 int composite_pixel(const Features& f, std::vector<int64_t> cand, int px, int py, const double* bg,
                     double band_alpha, double band_T, double* color, double* finalT, int32_t* ncontrib,
-                    std::vector<Blended>* blended) {
+                    std::vector<Blended>* blended, std::vector<int64_t>* clamp_band = nullptr) {
     // full depth sort of this pixel's candidates: by float32 depth bits, then gid
     std::sort(cand.begin(), cand.end(), [&](int64_t a, int64_t b) {
         uint32_t za = f32_bits(f.depth[a]), zb = f32_bits(f.depth[b]);
@@ -477,7 +499,10 @@ int composite_pixel(const Features& f, std::vector<int64_t> cand, int px, int py
         const double alpha = std::min(ALPHA_MAX, a);
         if (std::fabs(alpha - ALPHA_MIN) <= band_alpha * ALPHA_MIN) amb |= 1;
         if (alpha < ALPHA_MIN) continue;
-        if (std::fabs(a - ALPHA_MAX) <= band_alpha * ALPHA_MAX) amb |= 2;
+        if (std::fabs(a - ALPHA_MAX) <= band_alpha * ALPHA_MAX) {
+            amb |= 2;
+            if (clamp_band) clamp_band->push_back(i);
+        }
         const double Tn = T * (1.0 - alpha);
         if (std::fabs(Tn - T_MIN) <= band_T * T_MIN) amb |= 1;
         if (Tn < T_MIN) break;
@@ -539,7 +564,11 @@ int orc_render(int64_t n, const double* xy, const double* depth, const double* c
  * dL_dpix[3*k..] (all other pixels contribute nothing).  Accumulates (+=) into
  * grad2d[9*i..] = dL/d(u, v, A, B, C, o, r, g, b) and grad2d_abs (the sum of
  * the absolute values of the accumulated terms, a conditioning measure).
- * touched_amb[i] is set when Gaussian i is a candidate of an ambiguous pixel. */
+ * touched_amb[i] is set for the Gaussians whose gradient a straddling decision at
+ * one of the pixels can change: with a skip/stop straddle (bit 0) every Gaussian
+ * reachable at that pixel (it may blend there or not, and every blended entry's
+ * T and S move with it); with only a clamp straddle (bit 1) the entries in the
+ * clamp band (their alpha is continuous, only their own dalpha switches). */
 int orc_render_bwd(int64_t n, const double* xy, const double* depth, const double* conic, const double* opac,
                    const double* rgb, const int32_t* radius, const int32_t* rect, const orc_camera* ocam,
                    const double* bg, int64_t npix, const int64_t* pix, const double* dL_dpix, double band_alpha,
@@ -565,18 +594,25 @@ int orc_render_bwd(int64_t n, const double* xy, const double* depth, const doubl
         const int tx = (int)(t % cam.tiles_x()), ty = (int)(t / cam.tiles_x());
         const std::vector<int64_t> cand = tile_candidates(n, f, tx, ty);
         std::vector<Blended> bl;
+        std::vector<int64_t> cb;
         for (int64_t j = starts[s]; j < starts[s + 1]; ++j) {
             const int64_t k = order[j];
             const int64_t p = pix ? pix[k] : k;
             const double* g = dL_dpix + 3 * k;
             if (g[0] == 0.0 && g[1] == 0.0 && g[2] == 0.0) continue;
             bl.clear();
+            cb.clear();
             double color[3], T_final;
             int32_t nc;
             const int amb = composite_pixel(f, cand, (int)(p % W), (int)(p / W), bg, band_alpha, band_T, color,
-                                            &T_final, &nc, &bl);
-            if (amb) {
-                for (int64_t i : cand) {
+                                            &T_final, &nc, &bl, &cb);
+            if (amb & 1) {
+                for (int64_t i : reachable(f, cand, (int)(p % W), (int)(p / W), band_alpha)) {
+#pragma omp atomic write
+                    touched_amb[i] = 1;
+                }
+            } else if (amb & 2) {
+                for (int64_t i : cb) {
 #pragma omp atomic write
                     touched_amb[i] = 1;
                 }

@@ -47,7 +47,7 @@ def test_absgrad_matches_oracle(orc, case):
     want, want_abs, touched = orc.render_bwd(ref, cam, up.reshape(-1, 3).astype(np.float64), band_alpha=BAND_ALPHA,
                                              band_T=BAND_T)
     rows = np.nonzero(touched == 0)[0]
-    assert len(rows) > 0.5 * scene.n
+    assert len(rows) > 0.8 * scene.n
     got = g2.xy_abs.cpu().numpy()
     check_grads(got[:, 0], want_abs[:, 0], "abs du", rows=rows)
     check_grads(got[:, 1], want_abs[:, 1], "abs dv", rows=rows)

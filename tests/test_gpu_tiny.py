@@ -10,8 +10,8 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import abi, scenes
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 
-from _parity import (BAND_ALPHA, BAND_T, CudaRun, check_grads, check_images, check_projection, grad_mismatch,
-                     ulp_diff)
+from _parity import (BAND_ALPHA, BAND_T, G_ATOL, G_RTOL, CudaRun, chain_abs_bound, check_grads, check_images,
+                     check_projection, grad_mismatch, ulp_diff)
 
 pytestmark = pytest.mark.gpu
 
@@ -86,7 +86,11 @@ def test_project_backward_from_reference_grad2d(orc, tiny):
 
 
 def test_end_to_end_parameter_gradients(orc, tiny):
-    """Whole backward: CUDA raster_bwd -> CUDA project_bwd against oracle render_bwd -> oracle project_bwd."""
+    """Whole backward: CUDA raster_bwd -> CUDA project_bwd against oracle render_bwd -> oracle
+    project_bwd, element by element.  The two sides start from different 2D gradients (each
+    side's own, which agree element by element within their tolerance), so each parameter
+    gradient may differ by what that 2D difference moves it through the chain, |J| |d2D|,
+    plus the chain's own tolerance; nothing passes outside that bound."""
     wl, cam, run, ref = tiny
     g = wl.upstream[0]
     g2_gpu = run.backward(g)
@@ -94,14 +98,21 @@ def test_end_to_end_parameter_gradients(orc, tiny):
     g2, g2a, touched = orc.render_bwd(ref, cam, g.reshape(-1, 3).astype(np.float64), band_alpha=BAND_ALPHA,
                                       band_T=BAND_T)
     want = orc.project_bwd(wl.scene, cam, g2)
+    prop = chain_abs_bound(orc, wl.scene, cam, g2_gpu.astype(np.float64) - g2)
     rows = np.nonzero((touched == 0) & (ref["radius"] > 0))[0]
     for k in ("means", "quats", "log_scales", "opacity_logits", "sh"):
-        a = gpu[k].reshape(wl.scene.n, -1)
-        b = want[k].reshape(wl.scene.n, -1)
+        a = gpu[k].reshape(wl.scene.n, -1)[rows].astype(np.float64)
+        b = want[k].reshape(wl.scene.n, -1)[rows]
+        p = prop[k][rows]
         # the chain of fp32-accumulated 2D sums: report the norm-wise error too
-        rel = np.linalg.norm(a[rows] - b[rows]) / np.linalg.norm(b[rows])
+        rel = np.linalg.norm(a - b) / np.linalg.norm(b)
         assert rel < 1e-5, (k, rel)
-        check_grads(a, b, k, rows=rows, max_bad_frac=0.01, ref_abs=np.full_like(b, np.inf))
+        d = np.abs(a - b)
+        within_tol = d <= G_ATOL + G_RTOL * np.abs(b)
+        bound = G_ATOL + G_RTOL * (np.abs(b) + p) + 1.01 * p
+        assert np.all(d <= bound), (k, float(np.max(d - bound)))
+        print(f"  {k}: {int((~within_tol).sum())} of {d.size} elements outside 1e-6 + 1e-4|ref|, all within the "
+              f"propagated 2D difference")
 
 
 def test_adam_matches_oracle(orc):

@@ -436,3 +436,38 @@ def test_clamped_alpha_has_no_opacity_or_shape_gradient(orc):
     grads = orc.project_bwd(sc, cam, g2)
     for name in ("means", "opacity_logits", "log_scales"):
         assert np.all(grads[name] == 0.0)
+
+
+def _hand_projection(rows):
+    """A projection dict built by hand: rows of (u, v, depth, isotropic conic c, opacity)."""
+    n = len(rows)
+    a = np.asarray(rows, np.float64)
+    return {"xy": a[:, 0:2].copy(), "depth": a[:, 2].copy(),
+            "conic": np.stack([a[:, 3], np.zeros(n), a[:, 3]], 1), "opacity": a[:, 4].copy(),
+            "rgb": np.full((n, 3), 0.5), "radius": np.full(n, 3, np.int32),
+            "rect": np.tile(np.array([0, 0, 1, 1], np.int32), (n, 1)),
+            "tiles_touched": np.ones(n, np.uint32)}
+
+
+def test_straddle_marks_only_the_gaussians_the_decision_can_change(orc):
+    """The reverse pass excludes from comparison (touched) only the Gaussians whose gradient
+    a straddling decision can change: after a skip/stop straddle every Gaussian that can
+    blend at that pixel, not the far ones that merely share its tile; after a clamp
+    straddle only the clamped entry (alpha is continuous across the clamp)."""
+    cam = scenes.camera(np.eye(3), np.zeros(3), 16.0, 16.0, 8.0, 8.0, 16, 16)
+    d = math.sqrt(2.0 * math.log(255.0 / 1.2))          # alpha = 1.2 / 255 at pixel (4, 4)
+    rows = [(4.5, 4.5, 1.0, 1.0, 0.5),                   # C: blended at (4, 4)
+            (4.5 + d, 4.5, 2.0, 1.0, 1.0),               # A: alpha 1.2/255 at (4, 4), inside a 0.5 band
+            (14.5, 14.5, 3.0, 1.0, 0.9),                 # B: alpha ~ 1e-44 at (4, 4); 0.0017 at (12, 12)
+            (12.5, 12.5, 4.0, 1.0, 0.99 * 1.001),        # D: clamped at (12, 12), inside a 0.01 band
+            (12.5, 12.5, 5.0, 1.0, 0.3)]                 # E: blended at (12, 12) behind D
+    p = _hand_projection(rows)
+    up = np.array([[1.0, -0.5, 0.25]])
+    _, amb = orc.render(p, cam, pix=np.array([4 * 16 + 4]), band_alpha=0.5, band_T=1e-4)[2:]
+    assert amb[0] & 1
+    _, _, touched = orc.render_bwd(p, cam, up, pix=np.array([4 * 16 + 4]), band_alpha=0.5, band_T=1e-4)
+    assert list(touched) == [1, 1, 0, 0, 0]
+    _, amb = orc.render(p, cam, pix=np.array([12 * 16 + 12]), band_alpha=0.01, band_T=1e-4)[2:]
+    assert amb[0] == 2
+    _, _, touched = orc.render_bwd(p, cam, up, pix=np.array([12 * 16 + 12]), band_alpha=0.01, band_T=1e-4)
+    assert list(touched) == [0, 0, 0, 1, 0]
