@@ -41,17 +41,22 @@ import numpy as np  # noqa: E402
 METRIC = "fwd+bwd iterations/s and HBM GB/s vs roofline at 1M Gaussians, 1920x1080"
 RENDER_METRIC = "forward rendering frames/s"
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
-# FP32 lanes per SM and SMs of a B200; the ALU roofline uses the max SM clock
+# FP32 lanes per SM and SMs of a B200 (the nominal ALU peak, context beside the measured one)
 FP32_LANES_PER_SM = 128
 NUM_SMS = 148
 # float32 operations per (pixel, list entry) pair, counted from the kernels'
 # arithmetic with an FMA as two: alpha evaluation (dx, dy, quadratic form,
-# exponent, clamp, threshold tests) = 14; forward blend = 8; backward
-# transmittance recovery, colour/alpha gradients and the chain to
-# (u, v, A, B, C, o) = 46.
+# exponent, clamp, threshold tests) = 14, done for every pair a pixel traverses
+# (its list up to n_contrib); forward blend = 8 and backward transmittance
+# recovery, colour/alpha gradients and the chain to (u, v, A, B, C, o) = 46,
+# done only for the pairs the pixel blends.
 FLOPS_ALPHA = 14
 FLOPS_FWD_BLEND = 8
 FLOPS_BWD_GRAD = 46
+# special-function instructions per evaluated (pixel, entry) pair: ex2 for alpha;
+# the reverse pass adds rcp(1 - alpha)
+SFU_FWD = 1
+SFU_BWD = 2
 
 
 def measured_peaks():
@@ -188,7 +193,7 @@ def cpu_oracle_sample(wl, fraction: float, seed: int = 0):
     """Time the oracle on a bounded sample of one view of the workload and scale
     to one iteration.  Returns (seconds per iteration, threads, description)."""
     import oracle
-    threads = oracle.set_threads(0)
+    threads = oracle.set_threads(0)   # 0: keep the current thread count, return it
     rng = np.random.default_rng(seed)
     scene, cam = wl.scene, wl.cameras[0]
     n = scene.n
@@ -227,6 +232,23 @@ def cpu_oracle_sample(wl, fraction: float, seed: int = 0):
     return per_iter, threads, desc
 
 
+def cpu_baseline(sample, wl, fraction, unit):
+    """The oracle timed on the host on a bounded sample (`sample` returns seconds per
+    unit, threads, description): once on every core OpenMP is given and once on a
+    single thread (a quarter of the sample, scaled the same way)."""
+    import oracle
+    per_all, threads, desc = sample(wl, fraction)
+    oracle.set_threads(1)
+    try:
+        per_one, _, desc_one = sample(wl, fraction / 4)
+    finally:
+        oracle.set_threads(threads)
+    return {"value": 1.0 / per_all, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc,
+            "host_cpu_count": os.cpu_count(),
+            "single_thread": {"value": 1.0 / per_one, "unit": unit, "cores": 1, "sample": desc_one},
+            "thread_speedup": per_one / per_all}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -260,7 +282,7 @@ def cpu_oracle_render_sample(wl, fraction: float, seed: int = 0):
     """The oracle's forward pass on a bounded sample of one pose (projection and keys
     of all Gaussians, compositing of a fraction of the tiles), scaled to one frame."""
     import oracle
-    threads = oracle.set_threads(0)
+    threads = oracle.set_threads(0)   # 0: keep the current thread count, return it
     rng = np.random.default_rng(seed)
     scene, cam = wl.scene, wl.cameras[0]
     W, H = cam["width"], cam["height"]
@@ -342,15 +364,19 @@ def run_render(args, world, rank, local):
         raise RuntimeError("instance buffers overflowed after the warm-up")
     ms = max_over_ranks(start.elapsed_time(end), world)
     frames = args.steps * len(cams)
-    # compositing pairs of the last pose's frame for the ALU roofline of raster_fwd
-    pairs = int(view.n_contrib.sum().item())
+    # work counters of the last pose's compositing (counted variant, outside the timing) and
+    # the measured float32 / special-function peaks, for the roofline of raster_fwd
+    counts = torch.zeros(4, device="cuda", dtype=torch.int64)
+    pl.raster_fwd_counted(proj, view, counts)
+    torch.cuda.synchronize()
+    c = counts.cpu().tolist()
+    work = {"traversed_pairs": float(view.n_contrib.sum().item()), "fwd_evaluated_pairs": float(c[0]),
+            "fwd_blended_pairs": float(c[1]), "fwd_staged_entries": float(c[2])}
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev[-len(cams):])
     peaks = measured_peaks()
-    smax = clk.get("sm_max_mhz") or 1965.0
-    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
-    per_pair = FLOPS_ALPHA + FLOPS_FWD_BLEND
+    alu = measure_alu_peaks(torch, local)
     last_ms = fwd_ev[-1][0].elapsed_time(fwd_ev[-1][1])
-    achieved = pairs * per_pair / (last_ms * 1e-3) / 1e12
+    roof = raster_roofline("raster_fwd", last_ms, work, alu)
     cam0 = cams[0]
     line = {"metric": RENDER_METRIC, "value": world * frames / (ms / 1e3), "unit": "frames/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -360,16 +386,11 @@ def run_render(args, world, rank, local):
                        "parallelism": f"replicas x{world}",
                        "l2": "a step renders every pose once; the instance lists of a pose exceed L2"},
             "stages_ms_per_frame": {"raster_fwd": fwd_ms, "frame": ms / frames},
-            "roofline": {"kernel": "raster_fwd", "bound": "alu", "achieved": achieved, "peak": alu_peak,
-                         "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
-                         "work": f"{pairs} (pixel, entry) pairs x {per_pair} flops (last pose)",
-                         "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"},
+            "roofline": roof, "raster_work_last_pose": work, "alu_peaks": alu,
             "gpu_launches": int(launches), "clocks": clk,
             "e2e": None, "hbm_peak_gbs": peaks["hbm_gbs"]}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        per_frame, threads, desc = cpu_oracle_render_sample(wl, args.cpu_fraction)
-        line["cpu_baseline"] = {"value": 1.0 / per_frame, "unit": "frames/s", "cores": threads, "kind": "oracle",
-                                "sample": desc}
+        line["cpu_baseline"] = cpu_baseline(cpu_oracle_render_sample, wl, args.cpu_fraction, "frames/s")
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -378,7 +399,6 @@ def run_render(args, world, rank, local):
 def run_ours(args, world, rank, local):
     import torch
 
-    import oracle  # noqa: F401  (only for the cpu_baseline leg below)
     from gaussian_splatting_differentiable_02_b200 import abi
     from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 
@@ -464,7 +484,12 @@ def run_ours(args, world, rank, local):
     step_gbs = nbytes / (ms_per_step * 1e-3) / 1e9
 
     dom_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev_dom) if ev_dom else stages[dominant]
-    roof = roofline_for(dominant, dom_ms, stats, pairs / nv, scene, P, clk, peaks, profile_key(wl))
+    # measured float32 / special-function peaks and the compositing kernels' work counters
+    # (both after the timed region)
+    alu = measure_alu_peaks(torch, local)
+    work = raster_work_counts(tr, torch)
+    roof = roofline_for(dominant, dom_ms, stats, scene, P, peaks, profile_key(wl), work=work, alu=alu)
+    raster_roofs = {st: raster_roofline(st, stages[st] / nv, work, alu) for st in ("raster_fwd", "raster_bwd")}
 
     line = {"metric": METRIC, "value": value, "unit": "iterations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -482,6 +507,9 @@ def run_ours(args, world, rank, local):
                     "frac_of_nominal_8000_gbs": step_gbs / 8000.0},
             "stages_ms_per_step": {k: round(v, 4) for k, v in stages.items()},
             "roofline": roof,
+            "raster_alone": {k: {x: v[x] for x in ("achieved", "peak", "frac", "sfu")} for k, v in raster_roofs.items()},
+            "raster_work_per_view": work,
+            "alu_peaks": alu,
             "gpu_launches": int(launches),
             "clocks": clk}
     # e2e: the same step with the per-step inputs (16 target images) copied from
@@ -495,9 +523,7 @@ def run_ours(args, world, rank, local):
                     "packed": measure_packed(tr, wl, peaks, torch),
                     "sh16": measure_sh16(tr, wl, peaks, torch)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        per_iter, threads, desc = cpu_oracle_sample(wl, args.cpu_fraction)
-        line["cpu_baseline"] = {"value": 1.0 / per_iter, "unit": "iterations/s", "cores": threads,
-                                "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = cpu_baseline(cpu_oracle_sample, wl, args.cpu_fraction, "iterations/s")
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -770,6 +796,74 @@ def measure_densify(tr, wl, peaks, torch, with_oracle: bool, reps: int = 10):
     return res
 
 
+def measure_alu_peaks(torch, local, target_ms: float = 60.0, reps: int = 5):
+    """Measured instruction throughputs of this device (gs_alu_probe): float32 FMA
+    scalar and paired (TFLOP/s, an FMA counting two) and ex2 / rcp.approx
+    (T instructions x lanes per second); each op is calibrated to about
+    `target_ms` per launch and the best of `reps` launches is kept (CUDA events)."""
+    from gaussian_splatting_differentiable_02_b200 import abi
+    out = torch.empty(abi.gs_alu_probe_slots(), device="cuda", dtype=torch.float32)
+    s = torch.cuda.current_stream()
+    names = {abi.GS_PROBE_FFMA: "ffma", abi.GS_PROBE_FFMA2: "ffma2", abi.GS_PROBE_EX2: "ex2",
+             abi.GS_PROBE_RCP: "rcp"}
+    res = {}
+    clocks = ClockSampler(local)
+
+    def once(op, iters):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        ops = abi.gs_alu_probe(op, iters, out.data_ptr(), out.numel(), s.cuda_stream)
+        e1.record(s)
+        torch.cuda.synchronize()
+        return ops, e0.elapsed_time(e1)
+
+    for op, name in names.items():
+        once(op, 256)
+        ops, ms = once(op, 4096)
+        iters = max(4096, int(4096 * target_ms / max(ms, 1e-3)))
+        best = None
+        for _ in range(reps):
+            ops, ms = once(op, iters)
+            rate = ops / (ms * 1e-3) / 1e12
+            best = rate if best is None else max(best, rate)
+        res[name] = best
+    clk = clocks.stop()
+    return {"ffma_tflops": res["ffma"], "ffma2_tflops": res["ffma2"], "ex2_tops": res["ex2"],
+            "rcp_tops": res["rcp"], "fp32_tflops": max(res["ffma"], res["ffma2"]), "clocks": clk,
+            "source": "measured: gs_alu_probe, 8 blocks x 256 threads per SM, best of %d launches of ~%.0f ms"
+                      % (reps, target_ms)}
+
+
+def raster_work_counts(tr, torch):
+    """Work counters of the compositing kernels over the step's views, from the
+    counted variants run once on the last step's lists (outside any timing):
+    per view mean of the pairs a pixel traverses (sum of n_contrib), the pairs
+    it blends, the pairs the warps evaluate, and the list entries staged."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    nv = len(tr.views)
+    cf = torch.zeros(4, device="cuda", dtype=torch.int64)
+    cb = torch.zeros(4, device="cuda", dtype=torch.int64)
+    traversed = 0
+    g2 = pl.Grad2D(tr.gauss.n)
+    batched = getattr(tr, "depth_orders", None) is not None
+    for k in range(nv):
+        view, r = tr.views[k], tr._radius(k)
+        if batched:
+            proj = tr.projs[k]   # the view's projection, kept with its lists
+        else:                    # the projections were reused across views: redo this view's
+            proj = tr.proj
+            pl.project(tr.gauss, view, proj, r)
+            pl.bin_sort(proj, view, r)
+        pl.raster_fwd_counted(proj, view, cf, tr.bg, r)
+        traversed += int(view.n_contrib.sum().item())
+        pl.raster_bwd_counted(proj, view, g2, cb, tr.bg, r)
+    torch.cuda.synchronize()
+    f, b = cf.cpu().tolist(), cb.cpu().tolist()
+    return {"traversed_pairs": traversed / nv, "fwd_evaluated_pairs": f[0] / nv, "fwd_blended_pairs": f[1] / nv,
+            "fwd_staged_entries": f[2] / nv, "bwd_evaluated_pairs": b[0] / nv, "bwd_gradient_pairs": b[1] / nv,
+            "bwd_staged_entries": b[2] / nv}
+
+
 def stage_breakdown(tr, pl, torch):
     """Milliseconds per step of each stage, from CUDA events around every call of
     one untimed step."""
@@ -862,23 +956,39 @@ def profiled_traffic(stage, workload):
         return None
 
 
-def roofline_for(stage, ms, stats, pairs_per_view, scene, P, clk, peaks, workload=""):
+def raster_roofline(stage, ms, work, alu, workload=""):
+    """Roofline object of a compositing kernel against the measured float32 FMA
+    peak: achieved = the method's flops per launch (FLOPS_ALPHA per traversed
+    pair, plus the blend or gradient flops per blended pair) / the mean launch
+    time.  The special-function unit (ex2, rcp per evaluated pair) is reported
+    beside it against its own measured rate."""
+    fwd = stage == "raster_fwd"
+    blended = work["fwd_blended_pairs"] if fwd else work["bwd_gradient_pairs"]
+    evaluated = work["fwd_evaluated_pairs"] if fwd else work["bwd_evaluated_pairs"]
+    flops = FLOPS_ALPHA * work["traversed_pairs"] + (FLOPS_FWD_BLEND if fwd else FLOPS_BWD_GRAD) * blended
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = alu["fp32_tflops"]
+    sfu_ops = evaluated * (SFU_FWD if fwd else SFU_BWD)
+    sfu_rate = sfu_ops / (ms * 1e-3) / 1e12
+    return {"kernel": stage, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": profiled_traffic(stage, workload),
+            "work": (f"{work['traversed_pairs']:.4g} traversed pairs x {FLOPS_ALPHA} + {blended:.4g} blended pairs x "
+                     f"{FLOPS_FWD_BLEND if fwd else FLOPS_BWD_GRAD} flops per launch (mean over views)"),
+            "peak_source": f"measured float32 FMA throughput ({alu['source']})",
+            "sfu": {"achieved_tops": sfu_rate, "peak_tops": alu["ex2_tops"], "frac": sfu_rate / alu["ex2_tops"],
+                    "ops": f"{evaluated:.4g} evaluated pairs x {SFU_FWD if fwd else SFU_BWD} (ex2{'' if fwd else ' + rcp'})"},
+            "evaluated_over_traversed": evaluated / max(work["traversed_pairs"], 1.0),
+            "nominal_fp32_tflops": NUM_SMS * FP32_LANES_PER_SM * 2 * 1965.0 * 1e6 / 1e12}
+
+
+def roofline_for(stage, ms, stats, scene, P, peaks, workload="", work=None, alu=None):
     """Roofline object of the dominant kernel: the raster kernels against the
-    float32 ALU peak (148 SMs x 128 lanes x 2 x max SM clock), the streaming
-    kernels against the measured HBM copy bandwidth."""
+    measured float32 FMA peak (raster_roofline), the streaming kernels against
+    the measured HBM copy bandwidth."""
     K = float(np.mean([s[0] for s in stats]))
-    V = float(np.mean([s[1] for s in stats]))
     pb = 4 * (11 + 3 * (scene.sh_degree + 1) ** 2)
-    smax = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    alu_peak = NUM_SMS * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
     if stage in ("raster_bwd", "raster_fwd"):
-        per_pair = FLOPS_ALPHA + (FLOPS_BWD_GRAD if stage == "raster_bwd" else FLOPS_FWD_BLEND)
-        flops = pairs_per_view * per_pair
-        achieved = flops / (ms * 1e-3) / 1e12
-        return {"kernel": stage, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                "frac": achieved / alu_peak, "traffic": profiled_traffic(stage, workload),
-                "work": f"{pairs_per_view:.4g} (pixel, entry) pairs x {per_pair} flops per launch",
-                "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"}
+        return raster_roofline(stage, ms, work, alu, workload)
     n = scene.n
     nv = len(stats)
     per_launch = {"project_bwd_adam": n * (6 * pb + 44 * nv + 8), "project": n * (pb + 52),

@@ -136,6 +136,12 @@ SIGNATURES = {
     "gs_l1_loss_grad": (C.c_int32, [_P, _P, C.c_int64, _P, _P, _P]),
     "gs_zero": (C.c_int32, [_P, C.c_size_t, _P]),
     "gs_kernel_launches": (C.c_uint64, []),
+    "gs_raster_fwd_counted": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera),
+                                          C.POINTER(C.c_float), _P, _P, _P, _P, _P]),
+    "gs_raster_bwd_counted": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera),
+                                          C.POINTER(C.c_float), _P, _P, _P, C.POINTER(gs_grad2d), _P, _P]),
+    "gs_alu_probe_slots": (C.c_int64, []),
+    "gs_alu_probe": (C.c_int32, [C.c_int32, C.c_int64, _P, C.c_int64, C.POINTER(C.c_double), _P]),
 }
 
 _lib = None
@@ -275,6 +281,37 @@ def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: i
     b = (C.c_float * 3)(*[float(x) for x in bg])
     return _check(lib().gs_raster_bwd(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b,
                                       final_T, n_contrib, dL_dimage, C.byref(grad2d), stream))
+
+
+def gs_raster_fwd_counted(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg,
+                          image: int, final_T: int, n_contrib: int, counts: int, stream: int = 0):
+    """gs_raster_fwd that also adds its work counters to counts (4 uint64 on the device)."""
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_fwd_counted(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b,
+                                              image, final_T, n_contrib, counts, stream))
+
+
+def gs_raster_bwd_counted(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg,
+                          final_T: int, n_contrib: int, dL_dimage: int, grad2d: gs_grad2d, counts: int,
+                          stream: int = 0):
+    """gs_raster_bwd that also adds its work counters to counts (4 uint64 on the device)."""
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_bwd_counted(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b,
+                                              final_T, n_contrib, dL_dimage, C.byref(grad2d), counts, stream))
+
+
+GS_PROBE_FFMA, GS_PROBE_FFMA2, GS_PROBE_EX2, GS_PROBE_RCP = 0, 1, 2, 3
+
+
+def gs_alu_probe_slots() -> int:
+    return lib().gs_alu_probe_slots()
+
+
+def gs_alu_probe(op: int, iters: int, out: int, out_count: int, stream: int = 0) -> float:
+    """One throughput-probe launch; returns the operations it performs."""
+    ops = C.c_double(0.0)
+    _check(lib().gs_alu_probe(op, iters, out, out_count, C.byref(ops), stream))
+    return ops.value
 
 
 def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d: gs_grad2d, grads: gs_param_grads,

@@ -314,10 +314,14 @@ gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint3
                        fn);
 }
 
-gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
-                        float* final_T, int32_t* n_contrib, void* stream) {
-    const char* fn = "gs_raster_fwd";
+}  // extern "C"
+
+namespace {
+
+gs_status raster_fwd_common(const char* fn, const gs_projected* proj, const uint32_t* vals,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order, const gs_camera* cam,
+                            const float* bg_host, float* image, float* final_T, int32_t* n_contrib,
+                            unsigned long long* counts, void* stream) {
     gs_status st;
     if ((st = check_camera(fn, cam)) != GS_OK) return st;
     if ((st = check_projected(fn, proj, 1, false)) != GS_OK) return st;
@@ -330,14 +334,14 @@ gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const ui
     CHECK_PTR(n_contrib, 4);
     const gsk::CamArgs c = gsk::make_cam(*cam);
     return cuda_status(gsk::launch_raster_fwd(*proj, vals, tile_ranges, tile_order, c, bg_host, image, final_T,
-                                              n_contrib, static_cast<cudaStream_t>(stream)),
+                                              n_contrib, static_cast<cudaStream_t>(stream), counts),
                        fn);
 }
 
-gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
-                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* final_T,
-                        const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream) {
-    const char* fn = "gs_raster_bwd";
+gs_status raster_bwd_common(const char* fn, const gs_projected* proj, const uint32_t* vals,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order, const gs_camera* cam,
+                            const float* bg_host, const float* final_T, const int32_t* n_contrib,
+                            const float* dL_dimage, gs_grad2d* grad2d, unsigned long long* counts, void* stream) {
     gs_status st;
     if ((st = check_camera(fn, cam)) != GS_OK) return st;
     if ((st = check_projected(fn, proj, 1, false)) != GS_OK) return st;
@@ -355,8 +359,45 @@ gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const ui
     if (grad2d->xy_abs) CHECK_PTR(grad2d->xy_abs, 8);
     const gsk::CamArgs c = gsk::make_cam(*cam);
     return cuda_status(gsk::launch_raster_bwd(*proj, vals, tile_ranges, tile_order, c, bg_host, final_T, n_contrib,
-                                              dL_dimage, *grad2d, static_cast<cudaStream_t>(stream)),
+                                              dL_dimage, *grad2d, static_cast<cudaStream_t>(stream), counts),
                        fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
+                        float* final_T, int32_t* n_contrib, void* stream) {
+    return raster_fwd_common("gs_raster_fwd", proj, vals, tile_ranges, tile_order, cam, bg_host, image, final_T,
+                             n_contrib, nullptr, stream);
+}
+
+gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                        const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* final_T,
+                        const int32_t* n_contrib, const float* dL_dimage, gs_grad2d* grad2d, void* stream) {
+    return raster_bwd_common("gs_raster_bwd", proj, vals, tile_ranges, tile_order, cam, bg_host, final_T, n_contrib,
+                             dL_dimage, grad2d, nullptr, stream);
+}
+
+gs_status gs_raster_fwd_counted(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                                const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
+                                float* final_T, int32_t* n_contrib, uint64_t* counts, void* stream) {
+    const char* fn = "gs_raster_fwd_counted";
+    CHECK_PTR(counts, 8);
+    return raster_fwd_common(fn, proj, vals, tile_ranges, tile_order, cam, bg_host, image, final_T, n_contrib,
+                             reinterpret_cast<unsigned long long*>(counts), stream);
+}
+
+gs_status gs_raster_bwd_counted(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                                const uint32_t* tile_order, const gs_camera* cam, const float* bg_host,
+                                const float* final_T, const int32_t* n_contrib, const float* dL_dimage,
+                                gs_grad2d* grad2d, uint64_t* counts, void* stream) {
+    const char* fn = "gs_raster_bwd_counted";
+    CHECK_PTR(counts, 8);
+    return raster_bwd_common(fn, proj, vals, tile_ranges, tile_order, cam, bg_host, final_T, n_contrib, dL_dimage,
+                             grad2d, reinterpret_cast<unsigned long long*>(counts), stream);
 }
 
 }  // extern "C"

@@ -129,12 +129,13 @@ cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
-                              float* final_T, int32_t* n_contrib, cudaStream_t s);
+                              float* final_T, int32_t* n_contrib, cudaStream_t s,
+                              unsigned long long* counts = nullptr);
 
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,
                               const int32_t* n_contrib, const float* dL_dimage, const gs_grad2d& g2,
-                              cudaStream_t s);
+                              cudaStream_t s, unsigned long long* counts = nullptr);
 
 cudaError_t launch_adam(float* param, const float* grad, float* m, float* v, int64_t count, float lr, float beta1,
                         float beta2, float eps, int32_t step, cudaStream_t s);

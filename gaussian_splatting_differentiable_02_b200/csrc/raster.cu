@@ -310,8 +310,26 @@ struct FwdArgs {
     float* image;
     float* final_T;
     int32_t* n_contrib;
+    unsigned long long* counts;  // kCount only: work counters (gs_raster_fwd_counted)
 };
 
+// Work counters of the counted variants (one atomic per warp at its end): pairs
+// the warp evaluated (entries that reach its box x its pixels), pairs that did
+// the method's work (blended in the forward pass, took a gradient in the
+// reverse pass), list entries staged, and entries that reached the box.
+__device__ __forceinline__ void add_counts(unsigned long long* counts, int evaluated_entries, int work_pairs,
+                                           int staged, int lane) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) work_pairs += __shfl_xor_sync(kFull, work_pairs, o);
+    if (lane == 0) {
+        atomicAdd(counts + 0, (unsigned long long)evaluated_entries * (32 * kPx));
+        atomicAdd(counts + 1, (unsigned long long)work_pairs);
+        atomicAdd(counts + 2, (unsigned long long)staged);
+        atomicAdd(counts + 3, (unsigned long long)evaluated_entries);
+    }
+}
+
+template <bool kCount>
 __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_fwd_kernel(const FwdArgs a) {
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -350,6 +368,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         }
     }
     const f2 one = splat(1.f);
+    int c_eval = 0, c_work = 0, c_staged = 0;  // kCount only
 
     const int nb = (n + kBatch - 1) / kBatch;
     if (n > 0) gather<false>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x, min(n, kBatch), lane);
@@ -363,6 +382,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                           min(n - (b + 1) * kBatch, kBatch), lane);
         const int live = prep<true>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
+        if (kCount) c_staged += cnt;
         bool finished = false;
         for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
             f2 alive = on[0];  // nonzero while some pixel of the lane composites
@@ -372,6 +392,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 finished = true;
                 break;
             }
+            if (kCount) ++c_eval;
             const int j = S.idx[e];
             const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
@@ -399,6 +420,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 T[p].y = low1 ? T[p].y : Tn.y;
                 last[2 * p] = (na.x != 0.f && !low0) ? pos : last[2 * p];
                 last[2 * p + 1] = (na.y != 0.f && !low1) ? pos : last[2 * p + 1];
+                if (kCount) c_work += int(na.x != 0.f && !low0) + int(na.y != 0.f && !low1);
                 on[p].x = low0 ? 0.f : on[p].x;
                 on[p].y = low1 ? 0.f : on[p].y;
             }
@@ -407,6 +429,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (finished) break;
     }
     cp_async_wait_all();
+    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane);
     if (x < a.W) {
 #pragma unroll
         for (int i = 0; i < kPx; ++i) {
@@ -439,6 +462,7 @@ struct BwdArgs {
     float4* g_con;
     float4* g_rgb;
     float2* g_xy_abs;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv| (kAbs only)
+    unsigned long long* counts;  // kCount only: work counters (gs_raster_bwd_counted)
 };
 
 // Sum 9 per-lane values over the warp and add them to the Gaussian's three
@@ -488,7 +512,7 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
     if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
-template <bool kAbs>
+template <bool kAbs, bool kCount>
 __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_bwd_kernel(const BwdArgs a) {
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -537,6 +561,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     // entries past every pixel's last are never needed; never read past the list
     const int total = min(__reduce_max_sync(kFull, lmax), int(range.y - range.x));
     const int nb = (total + kBatch - 1) / kBatch;
+    int c_eval = 0, c_work = 0, c_staged = 0;  // kCount only
     if (total > 0) {
         const int c0 = min(total, kBatch);
         gather<true>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(total - c0), c0, lane);
@@ -553,6 +578,10 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
         }
         const int live = prep<false>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
+        if (kCount) {
+            c_staged += cnt;
+            c_eval += live;
+        }
         for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
             const int j = S.idx[e];
             const int pos = hi - 1 - j;  // 0-based list position of this entry
@@ -572,6 +601,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                 const f2 nae = make_float2(pos < last[2 * p] ? r.nal[p].x : 0.f,
                                            pos < last[2 * p + 1] ? r.nal[p].y : 0.f);
                 any = any || nae.x != 0.f || nae.y != 0.f;
+                if (kCount) c_work += int(nae.x != 0.f) + int(nae.y != 0.f);
                 const f2 om = add2(one, nae);                                                  // 1 - alpha
                 const f2 rom = make_float2(rcp_approx(om.x), rcp_approx(om.y));
                 T[p] = mul2(T[p], rom);  // transmittance in front of this entry
@@ -642,6 +672,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
         __syncwarp();
     }
     cp_async_wait_all();
+    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane);
 }
 
 // Tiles ordered by decreasing list length (bucketed by floor(sqrt(length)),
@@ -682,7 +713,7 @@ cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
-                              float* final_T, int32_t* n_contrib, cudaStream_t s) {
+                              float* final_T, int32_t* n_contrib, cudaStream_t s, unsigned long long* counts) {
     FwdArgs a;
     a.xy = reinterpret_cast<const float2*>(proj.xy);
     a.con = reinterpret_cast<const float4*>(proj.conic_opacity);
@@ -700,7 +731,12 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
     a.image = image;
     a.final_T = final_T;
     a.n_contrib = n_contrib;
-    raster_fwd_kernel<<<unsigned((a.tiles * kSub + kWarps - 1) / kWarps), kWarps * 32, 0, s>>>(a);
+    a.counts = counts;
+    const unsigned grid = unsigned((a.tiles * kSub + kWarps - 1) / kWarps);
+    if (counts)
+        raster_fwd_kernel<true><<<grid, kWarps * 32, 0, s>>>(a);
+    else
+        raster_fwd_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -708,7 +744,7 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,
                               const int32_t* n_contrib, const float* dL_dimage, const gs_grad2d& g2,
-                              cudaStream_t s) {
+                              cudaStream_t s, unsigned long long* counts) {
     BwdArgs a;
     a.xy = reinterpret_cast<const float2*>(proj.xy);
     a.con = reinterpret_cast<const float4*>(proj.conic_opacity);
@@ -730,11 +766,18 @@ cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, co
     a.g_con = reinterpret_cast<float4*>(g2.conic_opacity);
     a.g_rgb = reinterpret_cast<float4*>(g2.rgb);
     a.g_xy_abs = reinterpret_cast<float2*>(g2.xy_abs);
+    a.counts = counts;
     const unsigned grid = unsigned((a.tiles * kSub + kWarps - 1) / kWarps);
-    if (a.g_xy_abs)
-        raster_bwd_kernel<true><<<grid, kWarps * 32, 0, s>>>(a);
-    else
-        raster_bwd_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
+    if (counts) {
+        if (a.g_xy_abs)
+            raster_bwd_kernel<true, true><<<grid, kWarps * 32, 0, s>>>(a);
+        else
+            raster_bwd_kernel<false, true><<<grid, kWarps * 32, 0, s>>>(a);
+    } else if (a.g_xy_abs) {
+        raster_bwd_kernel<true, false><<<grid, kWarps * 32, 0, s>>>(a);
+    } else {
+        raster_bwd_kernel<false, false><<<grid, kWarps * 32, 0, s>>>(a);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

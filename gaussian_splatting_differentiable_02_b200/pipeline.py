@@ -308,6 +308,22 @@ def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), 
                       _ptr(view.final_T), _ptr(view.n_contrib), _ptr(d), grad2d.struct(), _stream())
 
 
+def raster_fwd_counted(proj: Projected, view: View, counts: torch.Tensor, bg=(0.0, 0.0, 0.0),
+                       radius: torch.Tensor = None):
+    """raster_fwd that also adds its work counters to counts (4 int64 on the device)."""
+    abi.gs_raster_fwd_counted(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam,
+                              bg, _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _ptr(counts),
+                              _stream())
+
+
+def raster_bwd_counted(proj: Projected, view: View, grad2d: Grad2D, counts: torch.Tensor, bg=(0.0, 0.0, 0.0),
+                       radius: torch.Tensor = None):
+    """raster_bwd (upstream view.dL_dimage) that also adds its work counters to counts."""
+    abi.gs_raster_bwd_counted(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam,
+                              bg, _ptr(view.final_T), _ptr(view.n_contrib), _ptr(view.dL_dimage), grad2d.struct(),
+                              _ptr(counts), _stream())
+
+
 def project_bwd(g: Gaussians, view: View, proj: Projected, grad2d: Grad2D, grads: Gaussians,
                 densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
                 radius: torch.Tensor = None, densify_max_radius: torch.Tensor = None):

@@ -508,6 +508,52 @@ gs_status gs_l1_dssim_loss_grad(const float* image, const float* target, int32_t
                                 float l1_weight, float ssim_weight, void* workspace, size_t workspace_bytes,
                                 float* dL_dimage, double* loss_dev, void* stream);
 
+/* ------------------------------------------------------------ measurement
+ * Diagnostics for the roofline of the compositing kernels; not part of the
+ * pipeline.  The compositing stage is the one the gsplat guide §2.1 calls the
+ * performance black hole; it is bound by arithmetic issue rather than by HBM,
+ * so its denominators are measured instruction throughputs and its numerator
+ * the work the method actually does. */
+
+/* gs_raster_fwd_counted / gs_raster_bwd_counted -- gs_raster_fwd / gs_raster_bwd
+ * (same arguments, same results, bit for bit) that also add work counters to
+ * counts[0..3] (uint64 on the device, 8-byte aligned, +=):
+ *   counts[0]  (pixel, entry) pairs evaluated: entries that reached a warp's
+ *              16x8 pixel box times its 128 pixels (pixels outside the image
+ *              included);
+ *   counts[1]  pairs that did the method's work: in the forward pass the
+ *              entries a pixel blended, in the reverse pass the entries a pixel
+ *              takes a gradient from (the same blended set);
+ *   counts[2]  list entries staged into shared memory, summed over warps;
+ *   counts[3]  entries that reached a warp's box, summed over warps.
+ * One atomic add per warp and counter at the warp's end. */
+gs_status gs_raster_fwd_counted(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                                const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
+                                float* final_T, int32_t* n_contrib, uint64_t* counts, void* stream);
+gs_status gs_raster_bwd_counted(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                                const uint32_t* tile_order, const gs_camera* cam, const float* bg_host,
+                                const float* final_T, const int32_t* n_contrib, const float* dL_dimage,
+                                gs_grad2d* grad2d, uint64_t* counts, void* stream);
+
+/* Instruction classes gs_alu_probe measures. */
+#define GS_PROBE_FFMA 0  /* float32 fma, one per lane per instruction */
+#define GS_PROBE_FFMA2 1 /* paired float32 fma of sm_100, two per lane per instruction */
+#define GS_PROBE_EX2 2   /* ex2.approx.ftz.f32 (special-function unit) */
+#define GS_PROBE_RCP 3   /* rcp.approx.ftz.f32 (special-function unit) */
+
+/* Number of floats gs_alu_probe writes (one per thread of its grid). */
+int64_t gs_alu_probe_slots(void);
+
+/* gs_alu_probe -- one launch that executes `iters` (1..2^30) iterations of 8
+ * independent dependency chains of instruction class `op` in every thread of a
+ * grid of 8 blocks x 256 threads per SM, all in registers.  *ops_host receives
+ * the operations the launch performs (flops for the fma forms, an fma counting
+ * two; instructions x lanes for ex2 and rcp); the caller times the launch with
+ * events on `stream`.  out: gs_alu_probe_slots() floats (4-byte aligned), the
+ * chains' final values.  Asynchronous; op outside GS_PROBE_* or iters out of
+ * range -> GS_ERR_INVALID_ARG. */
+gs_status gs_alu_probe(int32_t op, int64_t iters, float* out, int64_t out_count, double* ops_host, void* stream);
+
 /* Number of CUDA kernels this library has launched in the calling process
  * (a diagnostic counter, incremented on the host at every launch). */
 uint64_t gs_kernel_launches(void);

@@ -208,7 +208,7 @@ def test_binding_argument_counts_match_the_header(gs):
     """Every prototype of include/gs.h takes as many parameters as the ctypes binding
     passes (a missing or extra argument would be undefined behaviour at the call)."""
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
-    decls = re.findall(r"\b(?:gs_status|size_t|int32_t|uint64_t|const char\s*\*)\s+(gs_[a-z0-9_]+)\s*\(([^;]*?)\)\s*;",
+    decls = re.findall(r"\b(?:gs_status|size_t|int32_t|int64_t|uint64_t|const char\s*\*)\s+(gs_[a-z0-9_]+)\s*\(([^;]*?)\)\s*;",
                        text, flags=re.S)
     assert {name for name, _ in decls} == set(declared_functions())
     for name, params in decls:
@@ -248,3 +248,27 @@ def test_static_scratch_limit_is_checked_at_the_boundary(gs):
     assert "static scratch" in L.gs_last_error_detail().decode()
     st = L.gs_bin_sort_static(C.byref(proj), n, C.byref(c), None, None, lo, C.byref(K), None, None)
     assert st not in (gs.GS_OK, gs.GS_ERR_UNSUPPORTED)
+
+
+def test_alu_probe_argument_checks(gs):
+    L = gs.lib()
+    ops = C.c_double(0.0)
+    slots = gs.gs_alu_probe_slots()
+    assert slots == 148 * 8 * 256
+    assert L.gs_alu_probe(7, 10, C.c_void_p(256), slots, C.byref(ops), None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_alu_probe(gs.GS_PROBE_EX2, 0, C.c_void_p(256), slots, C.byref(ops), None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_alu_probe(gs.GS_PROBE_EX2, 10, None, slots, C.byref(ops), None) == gs.GS_ERR_INVALID_ARG
+    assert L.gs_alu_probe(gs.GS_PROBE_FFMA, 10, C.c_void_p(256), slots - 1, C.byref(ops), None) == \
+        gs.GS_ERR_INVALID_ARG
+    assert "needed" in L.gs_last_error_detail().decode()
+
+
+def test_counted_raster_calls_check_their_counter(gs):
+    L = gs.lib()
+    c = gs.make_camera(cam())
+    proj = gs.gs_projected()
+    bg = (C.c_float * 3)(0, 0, 0)
+    st = L.gs_raster_fwd_counted(C.byref(proj), None, None, None, C.byref(c), bg, None, None, None, None, None)
+    assert st == gs.GS_ERR_INVALID_ARG and "counts" in L.gs_last_error_detail().decode()
+    st = L.gs_raster_bwd_counted(C.byref(proj), None, None, None, C.byref(c), bg, None, None, None, None, None, None)
+    assert st == gs.GS_ERR_INVALID_ARG and "counts" in L.gs_last_error_detail().decode()

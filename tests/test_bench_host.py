@@ -87,3 +87,33 @@ def test_clock_parser(tmp_path):
     r = bench.ClockSampler.stop(c)
     assert r["sm_mhz"] == 1900.0 and r["sm_max_mhz"] == 1965.0 and r["reasons"] == ["sw_power_cap"]
     assert r["samples"] == 3
+
+
+def test_raster_roofline_counts_the_method_work():
+    """achieved = (14 per traversed pair + 46 per blended pair) / time against the measured
+    float32 peak; the special-function rate counts ex2 + rcp per evaluated pair."""
+    sys.path.insert(0, ROOT)
+    import bench
+    work = {"traversed_pairs": 1e9, "fwd_evaluated_pairs": 2e9, "fwd_blended_pairs": 4e8,
+            "bwd_evaluated_pairs": 1.5e9, "bwd_gradient_pairs": 4e8}
+    alu = {"fp32_tflops": 70.0, "ex2_tops": 4.0, "source": "test"}
+    r = bench.raster_roofline("raster_bwd", 2.0, work, alu)
+    assert r["bound"] == "alu" and r["unit"] == "TFLOP/s" and r["peak"] == 70.0
+    assert abs(r["achieved"] - (14 * 1e9 + 46 * 4e8) / 2e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 70.0) < 1e-12
+    assert abs(r["sfu"]["achieved_tops"] - 2 * 1.5e9 / 2e-3 / 1e12) < 1e-9
+    f = bench.raster_roofline("raster_fwd", 1.0, work, alu)
+    assert abs(f["achieved"] - (14 * 1e9 + 8 * 4e8) / 1e-3 / 1e12) < 1e-9
+    assert abs(f["sfu"]["achieved_tops"] - 2e9 / 1e-3 / 1e12) < 1e-9
+
+
+def test_cpu_baseline_times_all_cores_and_one_thread():
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    wl = bench.make_workload("tiny")
+    before = oracle.set_threads(0)
+    cb = bench.cpu_baseline(bench.cpu_oracle_sample, wl, 0.25, "iterations/s")
+    assert oracle.set_threads(0) == before          # the thread count is restored
+    assert cb["kind"] == "oracle" and cb["cores"] == before and cb["host_cpu_count"] == os.cpu_count()
+    assert cb["single_thread"]["cores"] == 1 and cb["value"] > 0 and cb["single_thread"]["value"] > 0
