@@ -517,11 +517,12 @@ def run_ours(args, world, rank, local):
     line["e2e"] = run_e2e(tr, targets_host, targets, args, world, torch)
     # rows outside the per-step path, measured after the step timing
     with_oracle = rank == 0 and not args.no_cpu_baseline and world == 1
-    line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
-                    "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
-                    "absgrad_and_sparse_adam": measure_variants(tr, torch),
-                    "packed": measure_packed(tr, wl, peaks, torch),
-                    "sh16": measure_sh16(tr, wl, peaks, torch)}
+    if not args.no_rows:
+        line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
+                        "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
+                        "absgrad_and_sparse_adam": measure_variants(tr, torch),
+                        "packed": measure_packed(tr, wl, peaks, torch),
+                        "sh16": measure_sh16(tr, wl, peaks, torch)}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cpu_oracle_sample, wl, args.cpu_fraction, "iterations/s")
     if rank == 0:
@@ -1077,6 +1078,9 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["multiview", "mixture", "box", "city", "tiny"], default="multiview")
     ap.add_argument("--cpu-fraction", type=float, default=1.0 / 256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the rows of the other options (densification, D-SSIM, absgrad, packed, FP16 SH): "
+                         "for short profiler captures, not a bench line")
     ap.add_argument("--streams", type=int, default=3,
                     help="CUDA streams the views of a step alternate over (1 = serial)")
     ap.add_argument("--groups", type=int, default=1,
