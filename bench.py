@@ -89,12 +89,13 @@ def make_workload(name: str, views: int = 16):
 
 
 def step_bytes(n, sh_degree, views_stats, tiles, pixels):
-    """Algorithmic HBM bytes of one step: per view, the sum of the stage terms,
-    then the fused multi-view backward through the projection with Adam."""
+    """Algorithmic HBM bytes of one step: the multi-view projection (parameters once,
+    outputs per view), per view the sum of the other stage terms, then the fused
+    multi-view backward through the projection with Adam."""
     pb = 4 * (11 + 3 * (sh_degree + 1) ** 2)
-    total = 0
+    total = n * pb                             # project: the parameters, read once for all views
     for (K, V, passes) in views_stats:
-        total += n * (pb + 52)                 # project
+        total += n * 52                        # project: this view's outputs
         total += n * (8 + 20 * 4)              # depth keys + 4 depth passes
         total += n * 16 + K * 8                # count (depth order) + emit (tile, gid)
         total += K * 20 * passes + K * 4       # tile passes (the last writes 12 instead of 8)
@@ -431,7 +432,7 @@ def run_ours(args, world, rank, local):
     # ---- timed region: K steps on resident inputs
     ev_dom = []
     orig = {"raster_bwd": pl.raster_bwd, "raster_fwd": pl.raster_fwd,
-            "project_bwd_adam": pl.project_bwd_views_adam, "project": pl.project}
+            "project_bwd_adam": pl.project_bwd_views_adam, "project": pl.project_views}
 
     def wrap(fn):
         # events on the stream the kernel is launched on (the Trainer spreads views over streams)
@@ -883,8 +884,8 @@ def stage_breakdown(tr, pl, torch):
     batched = getattr(tr, "depth_orders", None) is not None
     if batched:   # the Trainer's order: per view group the projections and one batched depth sort, then per view
         for ks, d in zip(tr.view_groups(), tr.depth_orders):
-            for k in ks:
-                timed("project", pl.project, tr.gauss, tr.views[k], tr.projs[k], tr.radii[k])
+            timed("project", pl.project_views, tr.gauss, [tr.views[k] for k in ks], [tr.projs[k] for k in ks],
+                  [tr.radii[k] for k in ks])
             timed("bin_sort", pl.depth_order_views, [tr.projs[k] for k in ks], [tr.radii[k] for k in ks], d)
     for k, (view, tgt) in enumerate(zip(tr.views, tr.targets)):
         r = tr.radii[k]
@@ -992,7 +993,7 @@ def roofline_for(stage, ms, stats, scene, P, peaks, workload="", work=None, alu=
         return raster_roofline(stage, ms, work, alu, workload)
     n = scene.n
     nv = len(stats)
-    per_launch = {"project_bwd_adam": n * (6 * pb + 44 * nv + 8), "project": n * (pb + 52),
+    per_launch = {"project_bwd_adam": n * (6 * pb + 44 * nv + 8), "project": n * (pb + 52 * nv),
                   "bin_sort": n * 24 + K * 12 + K * (8 + 24 * stats[0][2]) + K * 8,
                   "adam": n * pb // 4 * 28, "l1": P * 36}.get(stage, 0)
     achieved = per_launch / (ms * 1e-3) / 1e9

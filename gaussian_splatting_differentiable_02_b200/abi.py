@@ -117,6 +117,8 @@ SIGNATURES = {
                                                      _P, _P, C.c_int32, _P]),
     "gs_to_half": (C.c_int32, [_P, C.c_int64, _P, _P]),
     "gs_project_sh16": (C.c_int32, [C.POINTER(gs_params), _P, C.POINTER(gs_camera), C.POINTER(gs_projected), _P]),
+    "gs_project_views": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera), C.POINTER(gs_projected),
+                                     _P, _P]),
     "gs_project_bwd_views_adam_sh16": (C.c_int32, [C.POINTER(gs_params), C.c_int32, C.POINTER(gs_camera),
                                                    C.POINTER(gs_projected), C.POINTER(gs_grad2d), _P, _P,
                                                    C.POINTER(gs_param_grads), C.POINTER(gs_param_grads),
@@ -404,6 +406,13 @@ def gs_project_bwd_views_adam_packed(params: gs_params, cams, projs, slot_of, gr
 def gs_to_half(x: int, count: int, out: int, stream: int = 0):
     """float32 -> IEEE half, round to nearest even (count values)."""
     return _check(lib().gs_to_half(x or None, count, out or None, stream))
+
+
+def gs_project_views(params: gs_params, cams, outs, sh_half: int = 0, stream: int = 0):
+    """gs_project of every view in cams into the matching gs_projected of outs, in one launch."""
+    V = len(cams)
+    return _check(lib().gs_project_views(C.byref(params), V, _arr(gs_camera, cams), _arr(gs_projected, outs),
+                                         sh_half or None, stream))
 
 
 def gs_project_sh16(params: gs_params, sh_half: int, cam: gs_camera, out: gs_projected, stream: int = 0):

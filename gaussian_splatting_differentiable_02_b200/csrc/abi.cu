@@ -187,6 +187,25 @@ gs_status gs_project(const gs_params* params, const gs_camera* cam, gs_projected
     return cuda_status(gsk::launch_project_fwd(*params, c, *out, static_cast<cudaStream_t>(stream)), fn);
 }
 
+gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_camera* cams, gs_projected* outs,
+                           const uint16_t* sh_half, void* stream) {
+    const char* fn = "gs_project_views";
+    gs_status st;
+    if ((st = check_params(fn, params, sh_half == nullptr)) != GS_OK) return st;
+    if (num_views < 1 || num_views > GS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: num_views %d outside 1..%d", fn, int(num_views), GS_MAX_VIEWS);
+    if (!cams || !outs) return fail(GS_ERR_INVALID_ARG, "%s: cams or outs is NULL", fn);
+    if (sh_half && params->n > 0) CHECK_PTR(sh_half, 8);
+    gsk::CamArgs c[GS_MAX_VIEWS];
+    for (int v = 0; v < num_views; ++v) {
+        if ((st = check_camera(fn, cams + v)) != GS_OK) return st;
+        if ((st = check_projected(fn, outs + v, params->n, true)) != GS_OK) return st;
+        c[v] = gsk::make_cam(cams[v]);
+    }
+    return cuda_status(
+        gsk::launch_project_views(*params, num_views, c, outs, static_cast<cudaStream_t>(stream), sh_half), fn);
+}
+
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam) {
     (void)cam;
     if (n < 0) n = 0;

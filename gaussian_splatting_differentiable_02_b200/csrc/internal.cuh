@@ -47,6 +47,11 @@ inline int tile_bits(int64_t tiles) {
 cudaError_t launch_project_fwd(const gs_params& p, const CamArgs& cam, const gs_projected& out, cudaStream_t s,
                                const uint16_t* sh_half = nullptr);
 
+// Several views (1..GS_MAX_VIEWS) of the same Gaussians in one pass; view v's
+// outputs are launch_project_fwd's with cams[v] bit for bit.
+cudaError_t launch_project_views(const gs_params& p, int V, const CamArgs* cams, const gs_projected* outs,
+                                 cudaStream_t s, const uint16_t* sh_half = nullptr);
+
 // float32 -> IEEE half (round to nearest even), count values
 cudaError_t launch_to_half(const float* x, int64_t count, uint16_t* out, cudaStream_t s);
 

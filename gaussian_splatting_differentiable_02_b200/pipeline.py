@@ -231,6 +231,14 @@ def project(g: Gaussians, view: View, proj: Projected, radius: torch.Tensor = No
     abi.gs_project(g.params(), view.gcam, proj.struct(radius), _stream())
 
 
+def project_views(g: Gaussians, views: list, projs: list, radii: list = None, sh_half: torch.Tensor = None):
+    """gs_project of every view in one launch (projs[k] with radius row radii[k] for view k;
+    sh_half: project from the 16-bit SH copy)."""
+    abi.gs_project_views(g.params(), [vw.gcam for vw in views],
+                         [p.struct(None if radii is None else radii[k]) for k, p in enumerate(projs)],
+                         _ptr(sh_half), _stream())
+
+
 def to_half(x: torch.Tensor, out: torch.Tensor = None) -> torch.Tensor:
     """x (float32) rounded to IEEE half, nearest even (gs_to_half); out: an int16 tensor of
     x's shape holding the bit patterns (allocated when None)."""
@@ -694,11 +702,13 @@ class Trainer:
         groups = self.view_groups()
         for gi in range(len(groups)) if group is None else [group]:
             ks = groups[gi]
-            for k in ks:
-                if self.packed:
+            if self.packed:
+                for k in ks:
                     project_packed(self.gauss, self.views[k], self.packs[k], self.pack_ws)
-                else:
-                    self._project(self.views[k], self.projs[k], self.radii[k])
+            else:
+                # every view of the group in one launch (the parameters are read once)
+                project_views(self.gauss, [self.views[k] for k in ks], [self.projs[k] for k in ks],
+                              [self.radii[k] for k in ks], self.sh_half if self.sh16 else None)
             depth_order_views([self.projs[k] for k in ks], None if self.radii is None else [self.radii[k] for k in ks],
                               self.depth_orders[gi])
 

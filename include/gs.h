@@ -157,6 +157,17 @@ gs_status gs_tile_grid(const gs_camera* cam, int32_t* tiles_x_host, int32_t* til
  * Arithmetic is double precision; outputs are rounded to float32. */
 gs_status gs_project(const gs_params* params, const gs_camera* cam, gs_projected* out, void* stream);
 
+/* gs_project_views -- gs_project for num_views (1..GS_MAX_VIEWS) views of the same
+ * Gaussians in one launch: outs[v] receives, bit for bit, what gs_project writes
+ * for cams[v].  The view-independent part of stages 1-2 of the gsplat guide §2.1
+ * (the 3D covariance from quaternion and scales, the opacity) and the reading of
+ * the parameters are shared by the views instead of repeated per view.  sh_half:
+ * NULL, or the 16-bit copy of the SH planes that gs_project_sh16 reads (params->sh
+ * is then not read).  Every outs[v] as gs_project's out; the views' arrays must
+ * not overlap.  Asynchronous. */
+gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_camera* cams, gs_projected* outs,
+                           const uint16_t* sh_half, void* stream);
+
 /* Bytes of device workspace gs_bin_sort needs for n Gaussians and up to `capacity`
  * instances (16-byte aligned buffer, owned by the caller). */
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam);
