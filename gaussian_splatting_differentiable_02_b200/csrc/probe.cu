@@ -7,9 +7,11 @@
 // transmittance recovery of the reverse pass).
 //
 // Each thread runs kChains independent dependency chains of one instruction
-// for `iters` iterations, entirely in registers; the grid is 8 blocks of 256
-// threads per SM, so every scheduler has many warps to hide the latency.  The
-// chains' final values are written out so that nothing is optimised away.
+// for `iters` iterations, entirely in registers (the rcp chain adds 1 before
+// each reciprocal, an add on the FMA pipe, so that no two reciprocals cancel);
+// the grid is 8 blocks of 256 threads per SM, so every scheduler has many warps
+// to hide the latency.  The chains' final values are written out so that
+// nothing is optimised away.
 #include "internal.cuh"
 
 namespace gsk {
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(kProbeBlock) alu_probe_kernel(int64_t iters, f
             for (int i = 0; i < kChains; ++i) {
                 if (kOp == 0) a[i] = fmaf(a[i], 0.9999f, 1e-7f);
                 if (kOp == 2) a[i] = probe_ex2(-a[i]);  // stays in [0.5, 1]
-                if (kOp == 3) a[i] = probe_rcp(a[i]);   // alternates between x and 1/x
+                if (kOp == 3) a[i] = probe_rcp(a[i] + 1.f);  // x -> 1/(1 + x) stays in [0.5, 1]
             }
         }
 #pragma unroll
