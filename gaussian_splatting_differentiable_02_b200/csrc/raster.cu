@@ -44,6 +44,8 @@
 // into two floats, so the float32 evaluation keeps a relative error of a few
 // ulps whatever the conditioning; dsigma/du = A t and dsigma/dv = B t + D dy.
 // The factors are derived once per entry in double.
+#include <type_traits>
+
 #include "internal.cuh"
 
 namespace gsk {
@@ -58,7 +60,7 @@ constexpr double kLog2eD = 1.4426950408889634;
 constexpr float kCondMaxTraceSqOverDet = 10.125f;
 
 #ifndef GS_RASTER_PX
-#define GS_RASTER_PX 4
+#define GS_RASTER_PX 8
 #endif
 #ifndef GS_RASTER_BOXW
 #define GS_RASTER_BOXW 16
@@ -70,7 +72,7 @@ constexpr int kBoxH = kLaneRows * kPx;   // height of a warp's pixel box
 constexpr int kSubX = kTile / kBoxW, kSubY = kTile / kBoxH;
 constexpr int kSub = kSubX * kSubY;      // warps per tile
 #ifndef GS_RASTER_WARPS
-#define GS_RASTER_WARPS 2
+#define GS_RASTER_WARPS 1
 #endif
 // warps per block: one tile's two boxes, so that a block retires with its own tile
 // (two tiles per block: 1% slower, the block waiting for the slower tile)
@@ -78,10 +80,10 @@ constexpr int kWarps = GS_RASTER_WARPS;
 static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
 // resident blocks per SM the register allocation is sized for (launch bounds)
 #ifndef GS_RASTER_FWD_MIN_BLOCKS
-#define GS_RASTER_FWD_MIN_BLOCKS 10
+#define GS_RASTER_FWD_MIN_BLOCKS 16
 #endif
 #ifndef GS_RASTER_BWD_MIN_BLOCKS
-#define GS_RASTER_BWD_MIN_BLOCKS 10
+#define GS_RASTER_BWD_MIN_BLOCKS 16
 #endif
 constexpr int kBatch = 32;  // list entries staged per warp per batch
 constexpr unsigned kFull = 0xffffffffu;
@@ -115,6 +117,7 @@ constexpr float kSkip = 2.f;           // misses every pixel of the warp's box
 constexpr float kFactored = 3.f;       // factored form 1/2 A t^2 + 1/2 D dy^2 in float32 (D > 0)
 constexpr float kFactoredIndef = 4.f;  // the same with D <= 0 (a float32 conic that rounded to indefinite):
                                        // sigma can be negative, and such pixels are skipped
+constexpr int kMayClampBit = 32;       // WarpStage::idx: the entry's alpha can reach the 0.99 clamp
 
 struct WarpStage {
     float2 xy[2][kBatch];
@@ -172,11 +175,14 @@ __device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by
 // The bound is computed in float32 for well-conditioned conics and in double
 // for the others (never for an indefinite one).  The entries not skipped are
 // written compacted, in batch order, to S.pa / S.pb / S.pc with their batch index
-// in S.idx; returns their number.  Called by the whole warp.
+// in S.idx (bits 0-4) and kMayClamp (bit 5) when the entry's opacity is high
+// enough for its alpha to reach the 0.99 clamp; returns their number.  Called by
+// the whole warp.
 template <bool kNegRgb>
 __device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = make_float4(0.f, 0.f, 0.f, kSkip);
     float2 pc = make_float2(0.f, 0.f);
+    bool may_clamp = false;
     if (lane < count) {
         if (kNegRgb) {  // the forward pass blends with -alpha T weights
             const float4 c = S.rgb[buf][lane];
@@ -216,6 +222,10 @@ __device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, 
             }
         }
         pa = make_float4(xy.x, xy.y, lo, 1.f / c.w);
+        // o e^-sigma evaluates to at most o (1 + a few 1e-7) (ex2.approx and the
+        // rounding of the exponent near the mean), so an opacity 1e-5 below 0.99
+        // never reaches the clamp: such entries skip the clamp and its gate
+        may_clamp = c.w > kAlphaMax * (1.f - 1e-5f);
     }
     const unsigned keep = __ballot_sync(kFull, pb.w != kSkip);
     if (pb.w != kSkip) {
@@ -223,7 +233,7 @@ __device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, 
         S.pa[k] = pa;
         S.pb[k] = pb;
         S.pc[k] = pc;
-        S.idx[k] = lane;
+        S.idx[k] = lane | (may_clamp ? kMayClampBit : 0);
     }
     return __popc(keep);
 }
@@ -254,17 +264,18 @@ struct Alpha {
 };
 
 // -alpha at one pixel, 0 for a pixel that does not blend the entry (sigma < 0 or
-// alpha < 1/255); with kClamp, gate = 0 when alpha was clamped at 0.99, else 1.
-template <bool kClamp>
+// alpha < 1/255); with kMayClamp alpha is clamped at 0.99 and (kGate) gate = 0 when
+// it was, else 1; without, alpha cannot reach the clamp and no gate is formed.
+template <bool kGate, bool kMayClamp>
 __device__ __forceinline__ void alpha_at(float e, bool sign_ok, float& nal, float& gate) {
     const float a = ex2_approx(e);
-    nal = fmaxf(-a, -kAlphaMax);  // -min(a, 0.99)
+    nal = kMayClamp ? fmaxf(-a, -kAlphaMax) : -a;  // -min(a, 0.99)
     nal = (sign_ok && nal <= -kAlphaMin) ? nal : 0.f;
-    if (kClamp) gate = a > kAlphaMax ? 0.f : 1.f;
+    if (kGate && kMayClamp) gate = a > kAlphaMax ? 0.f : 1.f;
 }
 
 // nyc[p]: minus the centres' y of the lane's pixels 2p and 2p + 1.
-template <bool kClamp>
+template <bool kGate, bool kMayClamp>
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
                                            float px, const f2 (&nyc)[kPairs], Alpha& r) {
     const f2 vy = splat(pa.y), lo = splat(pa.z);
@@ -279,8 +290,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             const f2 sv = fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p]));
             const f2 e = add2(sv, lo);
             // sigma >= 0 by construction unless the conic is indefinite
-            alpha_at<kClamp>(e.x, !indef || sv.x <= 0.f, r.nal[p].x, r.gate[p].x);
-            alpha_at<kClamp>(e.y, !indef || sv.y <= 0.f, r.nal[p].y, r.gate[p].y);
+            alpha_at<kGate, kMayClamp>(e.x, !indef || sv.x <= 0.f, r.nal[p].x, r.gate[p].x);
+            alpha_at<kGate, kMayClamp>(e.y, !indef || sv.y <= 0.f, r.nal[p].y, r.gate[p].y);
         }
     } else {
         r.dx = __fsub_rn(pa.x, px);
@@ -292,8 +303,8 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             // a positive-definite form has sigma >= 0; the float32 value can round
             // below zero only within rounding of the mean, where alpha is o either way
             const f2 e = add2(fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0), lo);
-            alpha_at<kClamp>(e.x, true, r.nal[p].x, r.gate[p].x);
-            alpha_at<kClamp>(e.y, true, r.nal[p].y, r.gate[p].y);
+            alpha_at<kGate, kMayClamp>(e.x, true, r.nal[p].x, r.gate[p].x);
+            alpha_at<kGate, kMayClamp>(e.y, true, r.nal[p].y, r.gate[p].y);
         }
     }
 }
@@ -393,14 +404,18 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
                 break;
             }
             if (kCount) ++c_eval;
-            const int j = S.idx[e];
+            const int ij = S.idx[e];
+            const int j = ij & (kBatch - 1);
             const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
             const float4 nc = S.rgb[buf][j];  // minus the colour
             Alpha r;
             const int pos = b * kBatch + j + 1;
             const f2 ncr = splat(nc.x), ncg = splat(nc.y), ncb = splat(nc.z);
-            eval_alpha<false>(pa, pb, S.pc[e], con, px, nyc, r);
+            if (ij & kMayClampBit)
+                eval_alpha<false, true>(pa, pb, S.pc[e], con, px, nyc, r);
+            else
+                eval_alpha<false, false>(pa, pb, S.pc[e], con, px, nyc, r);
             // branch-free with float masks: -alpha is 0 for a pixel that does not blend
             // the entry or has stopped (on 0), so T (1 - alpha) = T and -alpha T = 0
             // leave it exactly as it was; T (1 - alpha) < 1e-4 then only happens for a
@@ -583,44 +598,50 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             c_eval += live;
         }
         for (int e = 0; e < live; ++e) {  // the batch's entries that reach this warp's box
-            const int j = S.idx[e];
+            const int ij = S.idx[e];
+            const int j = ij & (kBatch - 1);
             const int pos = hi - 1 - j;  // 0-based list position of this entry
             const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
             const float4 c = S.rgb[buf][j];
-            Alpha r;
-            eval_alpha<true>(pa, pb, S.pc[e], con, px, nyc, r);
-            const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
-            f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
-            bool any = false;
-            // branch-free: every pixel runs the same instructions, inactive ones
-            // with alpha 0, so T, P and every sum stay unchanged
+            // the entry at the lane's pixels; kMC: its alpha can reach the 0.99 clamp,
+            // whose gate then multiplies dL/dsigma (else the gate is 1 and not formed)
+            const auto entry = [&](auto may_clamp) {
+                constexpr bool kMC = decltype(may_clamp)::value;
+                Alpha r;
+                eval_alpha<true, kMC>(pa, pb, S.pc[e], con, px, nyc, r);
+                const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
+                f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
+                // branch-free: every pixel runs the same instructions, inactive ones
+                // with alpha 0, so T, P and every sum stay unchanged
 #pragma unroll
-            for (int p = 0; p < kPairs; ++p) {
-                // -alpha, 0 where the pixel does not blend the entry or has not reached it
-                const f2 nae = make_float2(pos < last[2 * p] ? r.nal[p].x : 0.f,
-                                           pos < last[2 * p + 1] ? r.nal[p].y : 0.f);
-                any = any || nae.x != 0.f || nae.y != 0.f;
-                if (kCount) c_work += int(nae.x != 0.f) + int(nae.y != 0.f);
-                const f2 om = add2(one, nae);                                                  // 1 - alpha
-                const f2 rom = make_float2(rcp_approx(om.x), rcp_approx(om.y));
-                T[p] = mul2(T[p], rom);  // transmittance in front of this entry
-                const f2 nw = mul2(nae, T[p]);
-                ndr = fma2(nw, gr[p], ndr);
-                ndg = fma2(nw, gg[p], ndg);
-                ndb = fma2(nw, gb[p], ndb);
-                // only g . S enters the gradient: P = g . S with S <- c alpha + (1 - alpha) S
-                const f2 xg = add2(fma2(gr[p], cr, fma2(gg[p], cg, mul2(gb[p], cb))), nP[p]);  // g . c - P
-                const f2 dLda = fma2(T[p], xg, mul2(ngb[p], rom));
-                nP[p] = fma2(nae, xg, nP[p]);
-                // -dL/dalpha alpha = dL/dsigma, zero where alpha was clamped (times a 0/1 gate)
-                const f2 q = mul2(mul2(dLda, nae), r.gate[p]);
-                nm[p] = q;
-                nmo = add2(nmo, q);
-                s1 = fma2(q, r.dy[p], s1);
-                s2 = fma2(mul2(q, r.dy[p]), r.dy[p], s2);
-            }
-            if (__any_sync(kFull, any)) {
+                for (int p = 0; p < kPairs; ++p) {
+                    // -alpha, 0 where the pixel does not blend the entry or has not reached it
+                    const f2 nae = make_float2(pos < last[2 * p] ? r.nal[p].x : 0.f,
+                                               pos < last[2 * p + 1] ? r.nal[p].y : 0.f);
+                    if (kCount) c_work += int(nae.x != 0.f) + int(nae.y != 0.f);
+                    const f2 om = add2(one, nae);                                                  // 1 - alpha
+                    const f2 rom = make_float2(rcp_approx(om.x), rcp_approx(om.y));
+                    T[p] = mul2(T[p], rom);  // transmittance in front of this entry
+                    const f2 nw = mul2(nae, T[p]);
+                    ndr = fma2(nw, gr[p], ndr);
+                    ndg = fma2(nw, gg[p], ndg);
+                    ndb = fma2(nw, gb[p], ndb);
+                    // only g . S enters the gradient: P = g . S with S <- c alpha + (1 - alpha) S
+                    const f2 xg = add2(fma2(gr[p], cr, fma2(gg[p], cg, mul2(gb[p], cb))), nP[p]);  // g . c - P
+                    const f2 dLda = fma2(T[p], xg, mul2(ngb[p], rom));
+                    nP[p] = fma2(nae, xg, nP[p]);
+                    // -dL/dalpha alpha = dL/dsigma, zero where alpha was clamped (times a 0/1 gate)
+                    f2 q = mul2(dLda, nae);
+                    if (kMC) q = mul2(q, r.gate[p]);
+                    nm[p] = q;
+                    nmo = add2(nmo, q);
+                    s1 = fma2(q, r.dy[p], s1);
+                    s2 = fma2(mul2(q, r.dy[p]), r.dy[p], s2);
+                }
+                // no vote on whether any pixel took the entry: 9 in 10 entries that reach
+                // the box take a gradient somewhere in it, and the test costs more than the
+                // reductions of zeros it would save
                 const float s0 = nmo.x + nmo.y, mo = -s0, m1 = s1.x + s1.y;
                 float du, dv;
                 float au = 0.f, av = 0.f;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv|
@@ -667,7 +688,11 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
                     }
                     if (lane == 3) atomicAdd(a.g_xy_abs + S.gid[buf][j], make_float2(au, av));
                 }
-            }
+            };
+            if (ij & kMayClampBit)
+                entry(std::true_type{});
+            else
+                entry(std::false_type{});
         }
         __syncwarp();
     }

@@ -49,7 +49,7 @@ def lib():
                                  _f64p, C.c_int64, _vp, C.c_double, C.c_double, _f64p, _f64p, _i32p, _u8p]
         L.orc_render_bwd.argtypes = [C.c_int64, _f64p, _f64p, _f64p, _f64p, _f64p, _i32p, _i32p,
                                      C.POINTER(OrcCamera), _f64p, C.c_int64, _vp, _f64p, C.c_double, C.c_double,
-                                     _f64p, _f64p, _u8p]
+                                     _f64p, _f64p, _u8p, _vp]
         L.orc_project_bwd.argtypes = [C.c_int64, _f64p, _f64p, _f64p, _f64p, _f64p, C.c_int, C.POINTER(OrcCamera),
                                       _vp, C.c_int64, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _vp, _vp]
         L.orc_adam.argtypes = [C.c_int64, _f32p, _f32p, _f32p, _f32p, C.c_double, C.c_double, C.c_double,
@@ -164,23 +164,28 @@ def render(proj: dict, cam: dict, bg=(0.0, 0.0, 0.0), pix=None, band_alpha=1e-5,
     return image, fT, nc, amb
 
 
-def render_bwd(proj: dict, cam: dict, dL_dpix, bg=(0.0, 0.0, 0.0), pix=None, band_alpha=1e-5, band_T=1e-4):
+def render_bwd(proj: dict, cam: dict, dL_dpix, bg=(0.0, 0.0, 0.0), pix=None, band_alpha=1e-5, band_T=1e-4,
+               straddle: bool = False):
     """Reverse compositing.  dL_dpix is [npix,3] for the listed pixels (or the
     whole image, row-major, when pix is None).  Returns grad2d [n,9]
     (u, v, A, B, C, o, r, g, b), the per-element sum of |terms|, and the
-    touched-ambiguous flags [n]."""
+    touched-ambiguous flags [n]; with straddle=True also [n,9], the sum over the
+    straddling decisions of |terms with the decision taken the other way - terms|."""
     n = len(proj["depth"])
     ip, ni, keep = _idx(pix)
     g2 = np.zeros((n, 9))
     g2a = np.zeros((n, 9))
     touched = np.zeros(n, np.uint8)
+    st = np.zeros((n, 9)) if straddle else None
     oc = camera(cam)
     lib().orc_render_bwd(n, _c(proj["xy"], np.float64).reshape(-1), _c(proj["depth"], np.float64),
                          _c(proj["conic"], np.float64).reshape(-1), _c(proj["opacity"], np.float64),
                          _c(proj["rgb"], np.float64).reshape(-1), _c(proj["radius"], np.int32),
                          _c(proj["rect"], np.int32).reshape(-1), C.byref(oc), _c(bg, np.float64), ni, ip,
                          _c(dL_dpix, np.float64).reshape(-1), band_alpha, band_T, g2.reshape(-1),
-                         g2a.reshape(-1), touched)
+                         g2a.reshape(-1), touched, None if st is None else st.ctypes.data_as(C.c_void_p))
+    if straddle:
+        return g2, g2a, touched, st
     return g2, g2a, touched
 
 

@@ -56,6 +56,10 @@
 #include <vector>
 #include <omp.h>
 
+#include <array>
+#include <map>
+#include <utility>
+
 namespace {
 
 /* ---------------------------------------------------------------- dual numbers */
@@ -464,22 +468,38 @@ std::vector<int64_t> reachable(const Features& f, const std::vector<int64_t>& ca
     return r;
 }
 
+/* A decision of the compositing that float32 evaluation may legitimately take the
+ * other way: entry k of the pixel's depth-sorted list and the test. */
+enum StraddleKind { kSignTest = 1, kSkipTest = 2, kClampTest = 3, kStopTest = 4 };
+struct Straddle {
+    size_t k;
+    int kind;
+};
+
 /* Composite one pixel front to back over its depth-sorted candidate list.
  * Returns the blended entries (for the reverse pass) and the ambiguity flags:
  *   bit 0: a skip/stop decision lay within the relative band of its threshold
- *          (alpha vs 1/255 or T(1-alpha) vs 1e-4), so float32 evaluation may
- *          legitimately decide the other way;
+ *          (alpha vs 1/255 or T(1-alpha) vs 1e-4, or the sign of a form this
+ *          close to indefinite), so float32 evaluation may legitimately decide
+ *          the other way;
  *   bit 1: an unclamped alpha lay within the band of the 0.99 clamp (gradients
  *          switch on or off there; values are continuous); those entries are
- *          appended to clamp_band when given. */
+ *          appended to clamp_band when given.
+ * Every such decision is appended to `straddles` when given; with `invert` the
+ * one decision it names is taken the other way (the alternative result). */
 int composite_pixel(const Features& f, std::vector<int64_t> cand, int px, int py, const double* bg,
                     double band_alpha, double band_T, double* color, double* finalT, int32_t* ncontrib,
-                    std::vector<Blended>* blended, std::vector<int64_t>* clamp_band = nullptr) {
+                    std::vector<Blended>* blended, std::vector<int64_t>* clamp_band = nullptr,
+                    std::vector<Straddle>* straddles = nullptr, const Straddle* invert = nullptr) {
     // full depth sort of this pixel's candidates: by float32 depth bits, then gid
     std::sort(cand.begin(), cand.end(), [&](int64_t a, int64_t b) {
         uint32_t za = f32_bits(f.depth[a]), zb = f32_bits(f.depth[b]);
         return za != zb ? za < zb : a < b;
     });
+    const auto flipped = [&](size_t k, int kind) { return invert && invert->k == k && invert->kind == kind; };
+    const auto record = [&](size_t k, int kind) {
+        if (straddles) straddles->push_back({k, kind});
+    };
     const double X = px + 0.5, Yp = py + 0.5;
     double T = 1.0, C[3] = {0, 0, 0};
     int32_t last = 0;
@@ -491,23 +511,35 @@ int composite_pixel(const Features& f, std::vector<int64_t> cand, int px, int py
         const double sigma = 0.5 * (A * dx * dx + Cc * dy * dy) + B * dx * dy;
         // a form this close to indefinite may round below zero in float32
         if (sigma <= 1e-6 * (0.5 * (std::fabs(A) * dx * dx + std::fabs(Cc) * dy * dy) + std::fabs(B * dx * dy)) &&
-            sigma != 0.0)
+            sigma != 0.0) {
             amb |= 1;
-        if (sigma < 0.0) continue;
+            record(k, kSignTest);
+        }
+        if ((sigma < 0.0) != flipped(k, kSignTest)) continue;
         const double G = std::exp(-sigma);
         const double a = f.opac[i] * G;
         const double alpha = std::min(ALPHA_MAX, a);
-        if (std::fabs(alpha - ALPHA_MIN) <= band_alpha * ALPHA_MIN) amb |= 1;
-        if (alpha < ALPHA_MIN) continue;
+        if (std::fabs(alpha - ALPHA_MIN) <= band_alpha * ALPHA_MIN) {
+            amb |= 1;
+            record(k, kSkipTest);
+        }
+        if ((alpha < ALPHA_MIN) != flipped(k, kSkipTest)) continue;
         if (std::fabs(a - ALPHA_MAX) <= band_alpha * ALPHA_MAX) {
             amb |= 2;
             if (clamp_band) clamp_band->push_back(i);
+            record(k, kClampTest);
         }
+        // the clamp changes alpha continuously; what a straddle decides is whether
+        // alpha has a derivative with respect to o and sigma
+        const bool clamped = (a > ALPHA_MAX) != flipped(k, kClampTest);
         const double Tn = T * (1.0 - alpha);
-        if (std::fabs(Tn - T_MIN) <= band_T * T_MIN) amb |= 1;
-        if (Tn < T_MIN) break;
+        if (std::fabs(Tn - T_MIN) <= band_T * T_MIN) {
+            amb |= 1;
+            record(k, kStopTest);
+        }
+        if ((Tn < T_MIN) != flipped(k, kStopTest)) break;
         for (int c = 0; c < 3; ++c) C[c] += f.rgb[3 * i + c] * alpha * T;
-        if (blended) blended->push_back({i, alpha, T, G, dx, dy, a > ALPHA_MAX});
+        if (blended) blended->push_back({i, alpha, T, G, dx, dy, clamped});
         T = Tn;
         last = (int32_t)(k + 1);
     }
@@ -515,6 +547,39 @@ int composite_pixel(const Features& f, std::vector<int64_t> cand, int px, int py
     *finalT = T;
     *ncontrib = last;
     return amb;
+}
+
+/* The reverse pass of one pixel: the 9 gradient terms (u, v, A, B, C, o, r, g,
+ * b) of every blended entry for the upstream g, derived directly from
+ * C = sum_i c_i alpha_i T_i + T_final bg.  Appended to `out` as (gid, terms). */
+void pixel_terms(const Features& f, const std::vector<Blended>& bl, double T_final, const double* g,
+                 const double* bg, std::vector<std::pair<int64_t, std::array<double, 9>>>* out) {
+    // S = colour accumulated behind the current entry, normalised by the
+    // transmittance just behind it
+    double S[3] = {0, 0, 0};
+    for (int e = (int)bl.size() - 1; e >= 0; --e) {
+        const Blended& b = bl[e];
+        const int64_t i = b.gid;
+        const double* c = f.rgb + 3 * i;
+        std::array<double, 9> t9 = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+        double dL_dalpha = 0.0;
+        for (int ch = 0; ch < 3; ++ch) {
+            t9[6 + ch] = b.alpha * b.T * g[ch];
+            dL_dalpha += g[ch] * (b.T * (c[ch] - S[ch]) - T_final * bg[ch] / (1.0 - b.alpha));
+        }
+        for (int ch = 0; ch < 3; ++ch) S[ch] = c[ch] * b.alpha + (1.0 - b.alpha) * S[ch];
+        if (!b.clamped) {
+            const double A = f.conic[3 * i], B = f.conic[3 * i + 1], Cc = f.conic[3 * i + 2];
+            t9[5] = dL_dalpha * b.G;                        // d alpha / d o = G
+            const double dL_dsigma = -dL_dalpha * b.alpha;  // d alpha / d sigma = -o G
+            t9[0] = dL_dsigma * (A * b.dx + B * b.dy);      // d sigma / d u
+            t9[1] = dL_dsigma * (B * b.dx + Cc * b.dy);     // d sigma / d v
+            t9[2] = dL_dsigma * 0.5 * b.dx * b.dx;
+            t9[3] = dL_dsigma * b.dx * b.dy;
+            t9[4] = dL_dsigma * 0.5 * b.dy * b.dy;
+        }
+        out->push_back({i, t9});
+    }
 }
 
 }  // namespace
@@ -568,11 +633,15 @@ int orc_render(int64_t n, const double* xy, const double* depth, const double* c
  * one of the pixels can change: with a skip/stop straddle (bit 0) every Gaussian
  * reachable at that pixel (it may blend there or not, and every blended entry's
  * T and S move with it); with only a clamp straddle (bit 1) the entries in the
- * clamp band (their alpha is continuous, only their own dalpha switches). */
+ * clamp band (their alpha is continuous, only their own dalpha switches).
+ * straddle (nullable, [n][9]) accumulates, over the pixels and over each of their
+ * straddling decisions, |terms with that decision taken the other way - terms as
+ * taken| per Gaussian and component: how far float32 evaluation that legitimately
+ * decides a straddle the other way can move each 2D gradient. */
 int orc_render_bwd(int64_t n, const double* xy, const double* depth, const double* conic, const double* opac,
                    const double* rgb, const int32_t* radius, const int32_t* rect, const orc_camera* ocam,
                    const double* bg, int64_t npix, const int64_t* pix, const double* dL_dpix, double band_alpha,
-                   double band_T, double* grad2d, double* grad2d_abs, uint8_t* touched_amb) {
+                   double band_T, double* grad2d, double* grad2d_abs, uint8_t* touched_amb, double* straddle) {
     const Camera cam = to_cam(ocam);
     const Features f{xy, depth, conic, opac, rgb, radius, rect};
     const int64_t W = cam.width;
@@ -593,21 +662,25 @@ int orc_render_bwd(int64_t n, const double* xy, const double* depth, const doubl
         const int64_t t = tile_of(order[starts[s]]);
         const int tx = (int)(t % cam.tiles_x()), ty = (int)(t / cam.tiles_x());
         const std::vector<int64_t> cand = tile_candidates(n, f, tx, ty);
-        std::vector<Blended> bl;
+        std::vector<Blended> bl, bl2;
         std::vector<int64_t> cb;
+        std::vector<Straddle> events;
+        std::vector<std::pair<int64_t, std::array<double, 9>>> terms, terms2;
         for (int64_t j = starts[s]; j < starts[s + 1]; ++j) {
             const int64_t k = order[j];
             const int64_t p = pix ? pix[k] : k;
+            const int ppx = (int)(p % W), ppy = (int)(p / W);
             const double* g = dL_dpix + 3 * k;
             if (g[0] == 0.0 && g[1] == 0.0 && g[2] == 0.0) continue;
             bl.clear();
             cb.clear();
+            events.clear();
             double color[3], T_final;
             int32_t nc;
-            const int amb = composite_pixel(f, cand, (int)(p % W), (int)(p / W), bg, band_alpha, band_T, color,
-                                            &T_final, &nc, &bl, &cb);
+            const int amb = composite_pixel(f, cand, ppx, ppy, bg, band_alpha, band_T, color, &T_final, &nc, &bl, &cb,
+                                            &events);
             if (amb & 1) {
-                for (int64_t i : reachable(f, cand, (int)(p % W), (int)(p / W), band_alpha)) {
+                for (int64_t i : reachable(f, cand, ppx, ppy, band_alpha)) {
 #pragma omp atomic write
                     touched_amb[i] = 1;
                 }
@@ -617,35 +690,41 @@ int orc_render_bwd(int64_t n, const double* xy, const double* depth, const doubl
                     touched_amb[i] = 1;
                 }
             }
-            // S = colour accumulated behind the current entry, normalised by the
-            // transmittance just behind it
-            double S[3] = {0, 0, 0};
-            for (int e = (int)bl.size() - 1; e >= 0; --e) {
-                const Blended& b = bl[e];
-                const int64_t i = b.gid;
-                const double* c = rgb + 3 * i;
-                double t9[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
-                double dL_dalpha = 0.0;
-                for (int ch = 0; ch < 3; ++ch) {
-                    t9[6 + ch] = b.alpha * b.T * g[ch];
-                    dL_dalpha += g[ch] * (b.T * (c[ch] - S[ch]) - T_final * bg[ch] / (1.0 - b.alpha));
-                }
-                for (int ch = 0; ch < 3; ++ch) S[ch] = c[ch] * b.alpha + (1.0 - b.alpha) * S[ch];
-                if (!b.clamped) {
-                    const double A = conic[3 * i], B = conic[3 * i + 1], Cc = conic[3 * i + 2];
-                    t9[5] = dL_dalpha * b.G;                // d alpha / d o = G
-                    const double dL_dsigma = -dL_dalpha * b.alpha;  // d alpha / d sigma = -o G
-                    t9[0] = dL_dsigma * (A * b.dx + B * b.dy);      // d sigma / d u
-                    t9[1] = dL_dsigma * (B * b.dx + Cc * b.dy);     // d sigma / d v
-                    t9[2] = dL_dsigma * 0.5 * b.dx * b.dx;
-                    t9[3] = dL_dsigma * b.dx * b.dy;
-                    t9[4] = dL_dsigma * 0.5 * b.dy * b.dy;
-                }
+            terms.clear();
+            pixel_terms(f, bl, T_final, g, bg, &terms);
+            for (const auto& it : terms) {
                 for (int q = 0; q < 9; ++q) {
 #pragma omp atomic
-                    grad2d[9 * i + q] += t9[q];
+                    grad2d[9 * it.first + q] += it.second[q];
 #pragma omp atomic
-                    grad2d_abs[9 * i + q] += std::fabs(t9[q]);
+                    grad2d_abs[9 * it.first + q] += std::fabs(it.second[q]);
+                }
+            }
+            if (!straddle) continue;
+            // each straddling decision taken the other way: the difference of every
+            // Gaussian's terms between the two results is what that decision can move
+            for (const Straddle& ev : events) {
+                bl2.clear();
+                double color2[3], T_final2;
+                int32_t nc2;
+                composite_pixel(f, cand, ppx, ppy, bg, band_alpha, band_T, color2, &T_final2, &nc2, &bl2, nullptr,
+                                nullptr, &ev);
+                terms2.clear();
+                pixel_terms(f, bl2, T_final2, g, bg, &terms2);
+                std::map<int64_t, std::array<double, 9>> diff;
+                for (const auto& it : terms2) {
+                    auto& d = diff[it.first];
+                    for (int q = 0; q < 9; ++q) d[q] += it.second[q];
+                }
+                for (const auto& it : terms) {
+                    auto& d = diff[it.first];
+                    for (int q = 0; q < 9; ++q) d[q] -= it.second[q];
+                }
+                for (const auto& it : diff) {
+                    for (int q = 0; q < 9; ++q) {
+#pragma omp atomic
+                        straddle[9 * it.first + q] += std::fabs(it.second[q]);
+                    }
                 }
             }
         }

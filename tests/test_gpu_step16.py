@@ -29,8 +29,8 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 from gaussian_splatting_differentiable_02_b200 import scenes
 
-from _parity import (AMB_FRAC_LONG_LISTS, BAND_ALPHA, BAND_T, G_RTOL, SUM_BOUND, check_grads, check_images,
-                     check_projection)
+from _parity import (AMB_FRAC_LONG_LISTS, BAND_ALPHA, BAND_T, G_ATOL, G_RTOL, SUM_BOUND, check_grads,
+                     check_images, check_projection)
 
 pytestmark = pytest.mark.gpu
 
@@ -134,6 +134,7 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
     per_view = []
     n_amb_total = n_px_total = 0
     sign_amb_total = 0
+    n_allow_total = n_elem_total = 0
     for k, cam in enumerate(cams):
         view = tr.views[k]
         lens = lengths[k]
@@ -166,11 +167,16 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
         assert np.array_equal(gd[cmp], up[cmp].astype(np.float32)), k
         sign_amb_total += int(sign_flip.sum())
 
-        g2, g2a, touched = orc.render_bwd(ref, cam, up, pix=pix, band_alpha=BAND_ALPHA, band_T=BAND_T)
+        g2, g2a, _, straddle = orc.render_bwd(ref, cam, up, pix=pix, band_alpha=BAND_ALPHA, band_T=BAND_T,
+                                              straddle=True)
+        # what a straddling decision the GPU may take the other way moves (the oracle's
+        # difference of the two results), plus, at a pixel whose sign of (image - target)
+        # is not decided, the terms of a reversed upstream on that channel
+        allow = straddle.copy()
         if sign_flip.any():
-            # every Gaussian that takes a term at those pixels (unit upstream) is left out
-            _, ga, _ = orc.render_bwd(ref, cam, np.ones((int(sign_flip.sum()), 3)), pix=pix[sign_flip])
-            touched = touched | (ga.sum(axis=1) > 0)
+            flip_up = np.where(np.abs(img - tgt.astype(np.float64))[sign_flip] <= 1e-5, 2.0 / (3.0 * W * H), 0.0)
+            _, ga, _ = orc.render_bwd(ref, cam, flip_up, pix=pix[sign_flip])
+            allow += ga
         # Gaussians whose whole tile rectangle was rendered: their oracle 2D gradient is complete
         # (a summed-area table of the tiles not rendered, queried over every rectangle)
         vis = visible[k]
@@ -183,13 +189,23 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
         x0, y0, x1, y1 = rc[:, 0], rc[:, 1], rc[:, 2], rc[:, 3]
         missing = sat[y1, x1] - sat[y0, x1] - sat[y1, x0] + sat[y0, x0]
         inside = vis & (missing == 0)
-        rows = np.nonzero(inside & (touched == 0))[0]
+        rows = np.nonzero(inside)[0]
         assert len(rows) > 500, (k, len(rows))
-        g2_gpu = tr.grad2ds[k].as_rows()
-        for q, qn in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
-            check_grads(g2_gpu[:, q], g2[:, q], f"view {k}:{qn}", rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.003)
+        g2_gpu = tr.grad2ds[k].as_rows().astype(np.float64)
+        # per element: the benchmark spec's tolerance (its absolute part scaled to this upstream,
+        # 1 / (3 H W) per pixel instead of N(0, 1)), the float32 summation bound of a
+        # cancelling sum, and the straddle allowance; no Gaussian is left out
+        atol = G_ATOL / (3.0 * W * H)
+        dd = np.abs(g2_gpu[rows] - g2[rows])
+        bound = atol + G_RTOL * np.abs(g2[rows]) + SUM_BOUND * g2a[rows] + 1.01 * allow[rows]
+        assert np.all(dd <= bound), (k, int((dd > bound).sum()), float(np.max(dd - bound)))
+        strict = dd <= atol + G_RTOL * np.abs(g2[rows])
+        n_allow = int((~strict).sum())
         print(f"view {k}: K={int(counts[k])}, {len(tiles)} tiles / {len(pix)} px, max img err {err:.2e}, "
-              f"{namb} ambiguous px, {int(sign_flip.sum())} sign-ambiguous px, {len(rows)} Gaussians' 2D gradients")
+              f"{namb} ambiguous px, {int(sign_flip.sum())} sign-ambiguous px, {len(rows)} Gaussians' 2D gradients, "
+              f"{n_allow} of {dd.size} elements within the summation or straddle allowance only")
+        n_allow_total += n_allow
+        n_elem_total += dd.size
 
         # the sampled Gaussians' 2D gradients and the chain's columns in this view
         Jk = []
@@ -198,16 +214,19 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
             e[:, q] = 1.0
             Jk.append(orc.project_bwd(scene, cam, e, idx=sample))
         pb = orc.project_bwd(scene, cam, g2[sample], idx=sample, densify=True)
-        per_view.append({"g2": g2[sample], "g2a": g2a[sample], "gpu": g2_gpu[sample].astype(np.float64),
-                         "touched": touched[sample] != 0, "vis": vis[sample], "J": Jk, "pb": pb})
+        per_view.append({"g2": g2[sample], "g2a": g2a[sample], "gpu": g2_gpu[sample], "vis": vis[sample], "J": Jk,
+                         "pb": pb})
         del ref, g2, g2a
 
     assert n_amb_total <= AMB_FRAC_LONG_LISTS * n_px_total
 
-    # ---- the update of the sampled Gaussians: sum over views of the oracle's chain, then Adam
+    # at most 1% of the compared 2D gradient elements pass through an allowance only
+    assert n_allow_total <= 0.01 * n_elem_total, (n_allow_total, n_elem_total)
+
+    # ---- the update of the sampled Gaussians: sum over views of the oracle's chain, then Adam;
+    # every sampled Gaussian is checked, the measured 2D differences (bounded above)
+    # propagated through the chain into each tolerance
     m = len(sample)
-    clean = ~np.any([pv["touched"] & pv["vis"] for pv in per_view], axis=0)
-    assert clean.sum() >= 0.8 * m, (int(clean.sum()), m)
     g_ref = {k: 0.0 for k in NAMES}
     prop = {k: 0.0 for k in NAMES}
     sumb = {k: 0.0 for k in NAMES}
@@ -228,7 +247,7 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
     got_acc = tr.densify_accum[torch.from_numpy(sample).cuda()].cpu().numpy()
     got_cnt = tr.densify_count[torch.from_numpy(sample).cuda()].cpu().numpy()
     assert np.array_equal(got_cnt, cnt_ref)
-    assert np.all(np.abs(got_acc - acc_ref)[clean] <= 1.01 * acc_tol[clean] + 1e-6 * acc_ref[clean] + 1e-30)
+    assert np.all(np.abs(got_acc - acc_ref) <= 1.01 * acc_tol + 1e-6 * acc_ref + 1e-30)
 
     after = _natural(tr.gauss, sample, deg)
     m1 = _natural(tr.m, sample, deg)
@@ -248,7 +267,6 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
         gm = np.asarray(m1[k], np.float64).reshape(m, -1)
         gv = np.asarray(v1[k], np.float64).reshape(m, -1)
         gp = np.asarray(after[k], np.float64).reshape(m, -1)
-        c = clean[:, None]
         ok_m = np.abs(gm - m1r) <= (1 - b1) * 1.0001 * tol + 2 * EPS32 * np.abs(m1r)
         ok_v = np.abs(gv - v1r) <= (1 - b2) * 1.0001 * (2 * np.abs(gr) * tol + tol ** 2) + 3 * EPS32 * np.abs(v1r)
         # the first step moves by lr sign(g); where the gradient is within its tolerance of 0 the
@@ -256,10 +274,11 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
         undecided = np.abs(gr) <= tol
         ok_p = np.abs(gp - p1r) <= EPS32 * np.maximum(np.abs(p0), np.abs(p1r)) + 1e-5 * lr + undecided * 2 * lr
         for nm, ok in (("m", ok_m), ("v", ok_v), ("param", ok_p)):
-            bad = ~ok & c
+            bad = ~ok
             assert not bad.any(), (k, nm, int(bad.sum()), np.argwhere(bad)[:3])
-    print(f"step: {int(clean.sum())} of {m} sampled Gaussians checked end to end; {n_amb_total} ambiguous of "
-          f"{n_px_total} rendered px; {sign_amb_total} sign-ambiguous px")
+    print(f"step: all {m} sampled Gaussians checked end to end; {n_amb_total} ambiguous of {n_px_total} rendered "
+          f"px; {sign_amb_total} sign-ambiguous px; {n_allow_total} of {n_elem_total} 2D gradient elements within "
+          f"an allowance only")
 
 
 def test_fused_16_view_backward_with_adam_at_full_size(orc, stepped):

@@ -471,3 +471,62 @@ def test_straddle_marks_only_the_gaussians_the_decision_can_change(orc):
     assert amb[0] == 2
     _, _, touched = orc.render_bwd(p, cam, up, pix=np.array([12 * 16 + 12]), band_alpha=0.01, band_T=1e-4)
     assert list(touched) == [0, 0, 0, 1, 0]
+
+
+def _alt(p, i, scale):
+    q = {k: v.copy() for k, v in p.items()}
+    q["opacity"][i] *= scale
+    return q
+
+
+def test_straddle_allowance_is_the_difference_of_the_two_decisions(orc):
+    """The straddle output of the reverse pass is, per Gaussian and component, the
+    difference between the terms with a straddling decision taken each way.  Pinned
+    against two renders whose opacity is nudged to either side of the threshold (far
+    outside the band, so neither straddles): the skip test at 1/255, the stop test at
+    T(1 - alpha) = 1e-4 and the 0.99 clamp."""
+    cam = scenes.camera(np.eye(3), np.zeros(3), 16.0, 16.0, 8.0, 8.0, 16, 16)
+    pix = np.array([4 * 16 + 4])
+    up = np.array([[1.0, -0.5, 0.25]])
+    band = dict(band_alpha=1e-5, band_T=1e-4)
+    tiny = dict(band_alpha=1e-12, band_T=1e-12)
+    # skip straddle: E's alpha at the pixel is (1/255)(1 + 2e-6)
+    d = math.sqrt(2.0 * math.log(255.0 / (1.0 + 2e-6)))
+    p = _hand_projection([(4.5, 4.5, 1.0, 1.0, 0.5),          # C in front, blended
+                          (4.5 + d, 4.5, 2.0, 1.0, 1.0),      # E straddles the skip test
+                          (4.5, 5.5, 3.0, 0.5, 0.3)])         # D behind, blended
+    p["rgb"] = np.array([[0.9, 0.2, 0.1], [0.1, 0.8, 0.3], [0.3, 0.3, 0.9]])
+    _, _, _, st = orc.render_bwd(p, cam, up, pix=pix, straddle=True, **band)
+    hi = orc.render_bwd(_alt(p, 1, 1 + 2e-4), cam, up, pix=pix, **tiny)[0]
+    lo = orc.render_bwd(_alt(p, 1, 1 - 2e-4), cam, up, pix=pix, **tiny)[0]
+    want = np.abs(hi - lo)
+    # E's own terms appear or vanish; D behind sees its T change; C in front (at its own
+    # centre, so no position or shape terms) sees only the colour behind it change
+    assert st[1].max() > 0 and st[2][6:].min() > 0 and st[0][5] > 0
+    np.testing.assert_allclose(st, want, rtol=1e-3, atol=1e-15)
+
+    # stop straddle: 13 entries of alpha 0.5, then one whose T(1 - alpha) is 1e-4 (1 + 3e-5)
+    T13 = 0.5 ** 13
+    ak = 1.0 - 1e-4 * (1.0 + 3e-5) / T13
+    rows = [(4.5, 4.5, 1.0 + j, 0.5, 0.5) for j in range(13)] + [(4.5, 4.5, 20.0, 0.5, ak), (4.5, 4.5, 21.0, 0.5, 0.4)]
+    p = _hand_projection(rows)
+    p["rgb"] = np.linspace(0.1, 0.9, 3 * len(rows)).reshape(-1, 3)
+    _, _, _, st = orc.render_bwd(p, cam, up, pix=pix, straddle=True, **band)
+    hi = orc.render_bwd(_alt(p, 13, 1 + 1e-3), cam, up, pix=pix, **tiny)[0]   # stops there
+    lo = orc.render_bwd(_alt(p, 13, 1 - 1e-3), cam, up, pix=pix, **tiny)[0]   # blends it
+    want = np.abs(hi - lo)
+    assert st[13].max() > 0 and np.all(st[14] == 0)
+    np.testing.assert_allclose(st, want, rtol=1e-2, atol=1e-15)
+
+    # clamp straddle: a single entry with o e^-sigma = 0.99 (1 + 2e-6) at the pixel
+    p = _hand_projection([(4.5, 4.5, 1.0, 0.5, 0.99 * (1 + 2e-6))])
+    _, _, _, st = orc.render_bwd(p, cam, up, pix=pix, straddle=True, **band)
+    hi = orc.render_bwd(_alt(p, 0, 1 + 1e-3), cam, up, pix=pix, **tiny)[0]   # clamped
+    lo = orc.render_bwd(_alt(p, 0, 1 - 1e-3), cam, up, pix=pix, **tiny)[0]   # not clamped
+    assert np.all(st[0, 6:] == 0)        # the clamp does not change alpha, only its derivatives
+    np.testing.assert_allclose(st[0, :6], np.abs(hi - lo)[0, :6], rtol=5e-3, atol=1e-15)
+
+    # no straddle: nothing
+    p = _hand_projection([(4.5, 4.5, 1.0, 1.0, 0.5)])
+    _, _, _, st = orc.render_bwd(p, cam, up, pix=pix, straddle=True, **band)
+    assert not st.any()
