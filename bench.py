@@ -431,8 +431,10 @@ def run_ours(args, world, rank, local):
 
     # ---- timed region: K steps on resident inputs
     ev_dom = []
-    orig = {"raster_bwd": pl.raster_bwd, "raster_fwd": pl.raster_fwd,
-            "project_bwd_adam": pl.project_bwd_views_adam, "project": pl.project_views}
+    # stage -> the pipeline function whose calls make it
+    stage_fn = {"raster_bwd": "raster_bwd", "raster_fwd": "raster_fwd", "project_bwd_adam": "project_bwd_views_adam",
+                "project": "project_views"}
+    orig = {name: getattr(pl, name) for name in stage_fn.values()}
 
     def wrap(fn):
         # events on the stream the kernel is launched on (the Trainer spreads views over streams)
@@ -446,8 +448,8 @@ def run_ours(args, world, rank, local):
             ev_dom.append((e0, e1))
         return inner
 
-    if dominant in orig:
-        setattr(pl, dominant, wrap(orig[dominant]))
+    if dominant in stage_fn:
+        setattr(pl, stage_fn[dominant], wrap(orig[stage_fn[dominant]]))
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()

@@ -3,10 +3,12 @@
 // §2.1: shared-memory prefetch of the tile's Gaussians, SoA features, warp-level
 // synchronisation; §2.2: a standalone backward entry).
 //
-// Work decomposition: one warp per 16x8 pixel box (two warps per tile, one tile
-// per block, blocks launched in the tile order of gs_tile_order when one is
-// given); each lane owns a column segment of 4 pixels (lane & 15 selects the
-// column, lane >> 4 the upper or lower half of the box).  The warp walks its
+// Work decomposition: one warp per 16x16 tile (one tile per block, blocks
+// launched in the tile order of gs_tile_order when one is given); each lane owns
+// a column segment of 8 pixels (lane & 15 selects the column, lane >> 4 the
+// upper or lower half of the tile), so that the per-entry work of the warp (its
+// shared-memory reads, the gradient reduction, the branches) is spread over 256
+// pixels.  The warp walks its
 // tile's sorted list in batches of 32 entries: every lane gathers one entry's
 // 40 bytes (xy, conic + opacity, colour) by Gaussian index into shared memory
 // with cp.async, double-buffered so the next batch is in flight while the
@@ -16,12 +18,12 @@
 // and the constants of the others are compacted, so the warp's loop visits only
 // entries that can reach its box).  Every lane then reads each entry once
 // (broadcast loads) and
-// applies it to its 4 pixels, whose terms that depend only on dx are shared;
+// applies it to its 8 pixels, whose terms that depend only on dx are shared;
 // the pixels go in pairs through the paired float32 instructions of sm_100
 // (fma/mul/add on two floats at once).  No block-wide barrier is used: warps
 // synchronise with __syncwarp and finish independently.
 //
-// Forward: a warp stops as soon as all 128 pixels have terminated (warp vote
+// Forward: a warp stops as soon as all of its pixels have terminated (warp vote
 // per entry).  Backward: back to front from the largest n_contrib of the box,
 // the transmittance in front of each entry recovered with rcp(1 - alpha) and
 // g . S (S the colour blended behind) tracked per pixel; each lane sums its
@@ -74,13 +76,18 @@ constexpr int kSub = kSubX * kSubY;      // warps per tile
 #ifndef GS_RASTER_WARPS
 #define GS_RASTER_WARPS 1
 #endif
-// warps per block: one tile's two boxes, so that a block retires with its own tile
-// (two tiles per block: 1% slower, the block waiting for the slower tile)
+// warps per block: one tile per block, so that a block retires with its own tile.
+// Measured per 1080p view of the 1M mixture (forward / backward ms): 4 pixels per
+// lane in 16x8 boxes, two warps a block, 10 blocks an SM 0.622 / 1.144; 8 pixels
+// per lane, one warp a block, 12 / 14 / 16 / 20 blocks an SM 0.666 / 1.205,
+// 0.609 / 1.098, 0.618 / 1.069, 0.631 / 1.198; two warps a block, 8 blocks an
+// SM 0.639 / 1.208.
 constexpr int kWarps = GS_RASTER_WARPS;
 static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
-// resident blocks per SM the register allocation is sized for (launch bounds)
+// resident blocks per SM the register allocation is sized for (launch bounds; the
+// forward pass does best at 14, the reverse pass at 16)
 #ifndef GS_RASTER_FWD_MIN_BLOCKS
-#define GS_RASTER_FWD_MIN_BLOCKS 16
+#define GS_RASTER_FWD_MIN_BLOCKS 14
 #endif
 #ifndef GS_RASTER_BWD_MIN_BLOCKS
 #define GS_RASTER_BWD_MIN_BLOCKS 16

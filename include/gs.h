@@ -530,8 +530,8 @@ gs_status gs_l1_dssim_loss_grad(const float* image, const float* target, int32_t
  * (same arguments, same results, bit for bit) that also add work counters to
  * counts[0..3] (uint64 on the device, 8-byte aligned, +=):
  *   counts[0]  (pixel, entry) pairs evaluated: entries that reached a warp's
- *              16x8 pixel box times its 128 pixels (pixels outside the image
- *              included);
+ *              pixel box (its 16x16 tile) times the box's pixels (pixels
+ *              outside the image included);
  *   counts[1]  pairs that did the method's work: in the forward pass the
  *              entries a pixel blended, in the reverse pass the entries a pixel
  *              takes a gradient from (the same blended set);
