@@ -175,6 +175,38 @@ __global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t
 }
 
 // kFinal: write 64-bit keys (key32 << 32 | depth bits of the Gaussian) to keys_out64.
+// Writes the block's elements, reordered by digit in shared memory (sk, sv, n of
+// them), to their global places gbase[digit] + offset within the digit's run: a
+// thread's loads (and, for the final pass, its gathers of the Gaussians' depths)
+// are all issued before its stores, so their latencies overlap.
+template <bool kFinal>
+__device__ __forceinline__ void scatter_runs(const uint32_t* sk, const uint32_t* sv, int n, int shift,
+                                             const uint32_t* gbase, const uint32_t* lstart,
+                                             const float* __restrict__ depth, uint32_t* __restrict__ keys_out,
+                                             uint64_t* __restrict__ keys_out64, uint32_t* __restrict__ vals_out) {
+    uint32_t k[kSortPerThread], v[kSortPerThread], z[kSortPerThread];
+#pragma unroll
+    for (int r = 0; r < kSortPerThread; ++r) {
+        const int p = threadIdx.x + r * kSortBlock;
+        k[r] = p < n ? sk[p] : 0u;
+        v[r] = p < n ? sv[p] : 0u;
+        z[r] = (kFinal && p < n) ? __float_as_uint(__ldg(depth + v[r])) : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < kSortPerThread; ++r) {
+        const int p = threadIdx.x + r * kSortBlock;
+        if (p < n) {
+            const uint32_t digit = (k[r] >> shift) & 0xffu;
+            const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
+            if (kFinal)
+                keys_out64[g] = (uint64_t(k[r]) << 32) | z[r];
+            else
+                keys_out[g] = k[r];
+            vals_out[g] = v[r];
+        }
+    }
+}
+
 // digit_bits: how many of the digit's 8 bits can be set (the last pass over the
 // tile bits has fewer); the rank votes only on those.
 template <bool kFinal>
@@ -273,17 +305,7 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
     }
     __syncthreads();
     const int in_block = int(min(int64_t(kSortTile), count - tile0));
-    for (int p = threadIdx.x; p < in_block; p += kSortBlock) {
-        const uint32_t k = sk[p], v = sv[p];
-        const uint32_t digit = (k >> shift) & 0xffu;
-        const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
-        if (kFinal) {
-            keys_out64[g] = (uint64_t(k) << 32) | __float_as_uint(__ldg(depth + v));
-        } else {
-            keys_out[g] = k;
-        }
-        vals_out[g] = v;
-    }
+    scatter_runs<kFinal>(sk, sv, in_block, shift, gbase, lstart, depth, keys_out, keys_out64, vals_out);
 }
 
 __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
@@ -364,10 +386,18 @@ __global__ void __launch_bounds__(kEmitBlock) count_digits_kernel(const uint32_t
     __shared__ uint32_t h[256];
     for (int d = threadIdx.x; d < 256; d += kEmitBlock) h[d] = 0u;
     const uint32_t total = load_chunk(touched, rect, order, n, s_start, s_gid, s_rect);  // synchronises
-    for (uint32_t slot = threadIdx.x; slot < total; slot += kEmitBlock) {
-        uint32_t tile, gid;
-        slot_instance(s_start, s_gid, s_rect, slot, tiles_x, tile, gid);
-        atomicAdd(&h[tile & 0xffu], 1u);
+    constexpr int kAtOnce = 8;  // independent binary searches in flight per thread
+    for (uint32_t first = threadIdx.x; first < total; first += kAtOnce * kEmitBlock) {
+        uint32_t tile[kAtOnce], gid;
+#pragma unroll
+        for (int r = 0; r < kAtOnce; ++r) {
+            const uint32_t slot = first + r * kEmitBlock;
+            tile[r] = 0u;
+            if (slot < total) slot_instance(s_start, s_gid, s_rect, slot, tiles_x, tile[r], gid);
+        }
+#pragma unroll
+        for (int r = 0; r < kAtOnce; ++r)
+            if (first + r * kEmitBlock < total) atomicAdd(&h[tile[r] & 0xffu], 1u);
     }
     __syncthreads();
     for (int d = threadIdx.x; d < 256; d += kEmitBlock) hist[int64_t(d) * nb + blockIdx.x] = h[d];
@@ -409,13 +439,18 @@ __global__ void __launch_bounds__(kSortBlock) emit_ranked_kernel(
         __syncthreads();
         const uint32_t base = round + uint32_t(warp) * kWarpSpan;
         uint32_t key[kSortPerThread], val[kSortPerThread], rank[kSortPerThread];
+        // the thread's instances first (independent binary searches), then the votes
+#pragma unroll
+        for (int r = 0; r < kSortPerThread; ++r) {
+            const uint32_t slot = base + r * 32 + lane;
+            key[r] = 0u;
+            val[r] = 0u;
+            if (slot < total) slot_instance(s_start, s_gid, s_rect, slot, tiles_x, key[r], val[r]);
+        }
 #pragma unroll
         for (int r = 0; r < kSortPerThread; ++r) {
             const uint32_t slot = base + r * 32 + lane;
             const bool in = slot < total;
-            key[r] = 0u;
-            val[r] = 0u;
-            if (in) slot_instance(s_start, s_gid, s_rect, slot, tiles_x, key[r], val[r]);
             const uint32_t digit = in ? (key[r] & 0xffu) : 256u;
             uint32_t peers = __ballot_sync(0xffffffffu, in);
             peers = in ? peers : ~peers;
@@ -459,16 +494,7 @@ __global__ void __launch_bounds__(kSortBlock) emit_ranked_kernel(
         }
         __syncthreads();
         const int in_round = int(min(uint32_t(kSortTile), total - round));
-        for (int p = threadIdx.x; p < in_round; p += kSortBlock) {
-            const uint32_t k = sk[p], v = sv[p];
-            const uint32_t digit = k & 0xffu;
-            const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
-            if (kFinal)
-                keys_out64[g] = (uint64_t(k) << 32) | __float_as_uint(__ldg(depth + v));
-            else
-                keys_out[g] = k;
-            vals_out[g] = v;
-        }
+        scatter_runs<kFinal>(sk, sv, in_round, 0, gbase, lstart, depth, keys_out, keys_out64, vals_out);
         __syncthreads();
         if (threadIdx.x < 256) gbase[threadIdx.x] += dtot;  // the next round continues every run
     }

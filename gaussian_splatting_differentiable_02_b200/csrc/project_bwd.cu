@@ -194,7 +194,7 @@ __device__ __forceinline__ int64_t entry(const ViewArgs& w, int64_t i) {
 }
 
 #ifndef GS_PBWD_MIN_BLOCKS
-#define GS_PBWD_MIN_BLOCKS 2
+#define GS_PBWD_MIN_BLOCKS 3
 #endif
 // Launches with at most this many views defer the SH gradient to a second pass
 // (kSplit): the 48 accumulators then never share registers with the geometric
@@ -205,8 +205,10 @@ constexpr int kSplitMaxViews = 2;
 template <bool kAdam, bool kPacked, bool kHalf, bool kSplit>
 __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) project_bwd_kernel(const Args a) {
     __shared__ float shs[48][kBwdBlock];  // this thread's SH coefficients, column threadIdx.x
-    // kSplit: this thread's masked colour gradient of every view, kept for the SH pass
-    __shared__ float gcs[kSplit ? 3 * kMaxViews : 1][kBwdBlock];
+    // kSplit: this thread's masked colour gradient of every view, kept for the SH pass;
+    // otherwise the 48 SH gradient sums, accumulated view by view in shared memory
+    // rather than in registers (which keeps the one-pass kernel at 3 blocks per SM)
+    __shared__ float gcs[kSplit ? 3 * kMaxViews : 48][kBwdBlock];
     const int t = threadIdx.x;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + t; i < a.n; i += int64_t(gridDim.x) * blockDim.x) {
         unsigned vis = 0u;
@@ -246,9 +248,13 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
         double gS[6] = {0, 0, 0, 0, 0, 0};  // symmetric dL/dSigma: xx, xy, xz, yy, yz, zz
         double gmu[3] = {0, 0, 0};
         double glogit = 0.0;
-        float gsh[48];
+        float gsh[kSplit ? 48 : 1];  // kSplit: the SH gradient sums (the second pass)
 #pragma unroll
-        for (int k = 0; k < 48; ++k) gsh[k] = 0.f;
+        for (int k = 0; k < (kSplit ? 48 : 1); ++k) gsh[k] = 0.f;
+        if (!kSplit) {
+#pragma unroll
+            for (int k = 0; k < 48; ++k) gcs[k][t] = 0.f;
+        }
         float dacc = 0.f;
         int dcnt = 0;
         double qv[4] = {1, 0, 0, 0}, s3[3] = {0, 0, 0}, qn = 1.0;
@@ -395,7 +401,8 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
                 // colour decides the clamp and is re-taken in double when close to 0
                 const double dvx = mu[0] - cam.cc[0], dvy = mu[1] - cam.cc[1], dvz = mu[2] - cam.cc[2];
                 const double dn = sqrt(dvx * dvx + dvy * dvy + dvz * dvz);
-                const double ux = dvx / dn, uy = dvy / dn, uz = dvz / dn;
+                const double idn = 1.0 / dn;  // one division for the six uses below
+                const double ux = dvx * idn, uy = dvy * idn, uz = dvz * idn;
                 const float fx3 = float(ux), fy3 = float(uy), fz3 = float(uz);
                 float Y[16];
                 sh_basis<float>(a.deg, fx3, fy3, fz3, Y);
@@ -428,9 +435,9 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
                     if (k < nc) {
                         const float s0 = shs[3 * k][t], s1 = shs[3 * k + 1][t], s2 = shs[3 * k + 2][t];
                         if (!kSplit) {
-                            gsh[3 * k + 0] = fmaf(Y[k], gcol[0], gsh[3 * k + 0]);
-                            gsh[3 * k + 1] = fmaf(Y[k], gcol[1], gsh[3 * k + 1]);
-                            gsh[3 * k + 2] = fmaf(Y[k], gcol[2], gsh[3 * k + 2]);
+                            gcs[3 * k + 0][t] = fmaf(Y[k], gcol[0], gcs[3 * k + 0][t]);
+                            gcs[3 * k + 1][t] = fmaf(Y[k], gcol[1], gcs[3 * k + 1][t]);
+                            gcs[3 * k + 2][t] = fmaf(Y[k], gcol[2], gcs[3 * k + 2][t]);
                         }
                         wk[k] = s0 * gcol[0] + s1 * gcol[1] + s2 * gcol[2];
                     } else {
@@ -440,9 +447,9 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
                 float gdir[3] = {0.f, 0.f, 0.f};
                 sh_grad_dir(a.deg, fx3, fy3, fz3, wk, gdir);
                 const double dproj = gdir[0] * ux + gdir[1] * uy + gdir[2] * uz;
-                gmu[0] += (gdir[0] - ux * dproj) / dn;
-                gmu[1] += (gdir[1] - uy * dproj) / dn;
-                gmu[2] += (gdir[2] - uz * dproj) / dn;
+                gmu[0] += (gdir[0] - ux * dproj) * idn;
+                gmu[1] += (gdir[1] - uy * dproj) * idn;
+                gmu[2] += (gdir[2] - uz * dproj) * idn;
 
                 const float2 sxy = cam.g_xy_abs ? __ldg(cam.g_xy_abs + cj) : gxy;
                 dacc += sqrtf(sxy.x * sxy.x + sxy.y * sxy.y);
@@ -516,8 +523,9 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
                 const ViewArgs& cam = a.view[v];
                 const double dvx = mu[0] - cam.cc[0], dvy = mu[1] - cam.cc[1], dvz = mu[2] - cam.cc[2];
                 const double dn = sqrt(dvx * dvx + dvy * dvy + dvz * dvz);
+                const double idn = 1.0 / dn;  // the direction exactly as the first pass formed it
                 float Y[16];
-                sh_basis<float>(a.deg, float(dvx / dn), float(dvy / dn), float(dvz / dn), Y);
+                sh_basis<float>(a.deg, float(dvx * idn), float(dvy * idn), float(dvz * idn), Y);
                 const float gcol[3] = {gcs[3 * v][t], gcs[3 * v + 1][t], gcs[3 * v + 2][t]};
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
@@ -529,21 +537,23 @@ __global__ void __launch_bounds__(kBwdBlock, kSplit ? 4 : GS_PBWD_MIN_BLOCKS) pr
                 }
             }
         }
+        // the SH gradient of plane p (four coefficients): from the registers of the
+        // second pass, or from the shared-memory sums
+        const auto sh_grad = [&](int p) {
+            if (kSplit) return make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]);
+            return make_float4(gcs[4 * p][t], gcs[4 * p + 1][t], gcs[4 * p + 2][t], gcs[4 * p + 3][t]);
+        };
         if (a.d_means) {
 #pragma unroll
             for (int p = 0; p < 12; ++p)
-                if (p < a.planes)
-                    add4(a.d_sh, int64_t(p) * a.n + i,
-                         make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]));
+                if (p < a.planes) add4(a.d_sh, int64_t(p) * a.n + i, sh_grad(p));
         }
         if (kAdam) {
 #pragma unroll
             for (int p = 0; p < 12; ++p)
                 if (p < a.planes)
                 {
-                    const float4 up = adam4(a.p_sh, a.m_sh, a.v_sh, int64_t(p) * a.n + i,
-                                            make_float4(gsh[4 * p], gsh[4 * p + 1], gsh[4 * p + 2], gsh[4 * p + 3]),
-                                            a.lr_t[4], a);
+                    const float4 up = adam4(a.p_sh, a.m_sh, a.v_sh, int64_t(p) * a.n + i, sh_grad(p), a.lr_t[4], a);
                     if (kHalf) a.sh_half_out[int64_t(p) * a.n + i] = narrow(up);
                 }
         }
