@@ -285,7 +285,7 @@ __device__ __forceinline__ void alpha_at(float e, bool sign_ok, float& nal, floa
 template <bool kGate, bool kMayClamp>
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
                                            float px, const f2 (&nyc)[kPairs], Alpha& r) {
-    const f2 vy = splat(pa.y), lo = splat(pa.z);
+    const f2 vy = splat(pa.y);
     if (pb.w >= kFactored) {
         const bool indef = pb.w == kFactoredIndef;
         r.dx = __fsub_rn(pa.x, px);
@@ -295,21 +295,23 @@ __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, c
             r.dy[p] = add2(vy, nyc[p]);
             r.t[p] = fma2(rl, r.dy[p], fma2(rh, r.dy[p], dx2));
             const f2 sv = fma2(mul2(ka, r.t[p]), r.t[p], mul2(mul2(kd, r.dy[p]), r.dy[p]));
-            const f2 e = add2(sv, lo);
+            const f2 e = add2(sv, splat(pa.z));
             // sigma >= 0 by construction unless the conic is indefinite
             alpha_at<kGate, kMayClamp>(e.x, !indef || sv.x <= 0.f, r.nal[p].x, r.gate[p].x);
             alpha_at<kGate, kMayClamp>(e.y, !indef || sv.y <= 0.f, r.nal[p].y, r.gate[p].y);
         }
     } else {
         r.dx = __fsub_rn(pa.x, px);
-        const f2 a0 = splat(__fmul_rn(__fmul_rn(pb.x, r.dx), r.dx)), c1 = splat(__fmul_rn(pb.y, r.dx));
+        // the terms that depend only on dx, with log2(o) added once per entry
+        const f2 a0 = splat(__fadd_rn(__fmul_rn(__fmul_rn(pb.x, r.dx), r.dx), pa.z));
+        const f2 c1 = splat(__fmul_rn(pb.y, r.dx));
         const f2 cz = splat(pb.z);
 #pragma unroll
         for (int p = 0; p < kPairs; ++p) {
             r.dy[p] = add2(vy, nyc[p]);
             // a positive-definite form has sigma >= 0; the float32 value can round
             // below zero only within rounding of the mean, where alpha is o either way
-            const f2 e = add2(fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0), lo);
+            const f2 e = fma2(r.dy[p], fma2(cz, r.dy[p], c1), a0);
             alpha_at<kGate, kMayClamp>(e.x, true, r.nal[p].x, r.gate[p].x);
             alpha_at<kGate, kMayClamp>(e.y, true, r.nal[p].y, r.gate[p].y);
         }
