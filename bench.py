@@ -526,6 +526,11 @@ def run_ours(args, world, rank, local):
                         "absgrad_and_sparse_adam": measure_variants(tr, torch),
                         "packed": measure_packed(tr, wl, peaks, torch),
                         "sh16": measure_sh16(tr, wl, peaks, torch)}
+        # the two options where they are meant to pay: packed views that keep a small part
+        # of the scene, FP16 SH on a single-view step
+        torch.cuda.empty_cache()
+        line["rows"]["packed_narrow_views"] = measure_packed_narrow(torch)
+        line["rows"]["sh16_single_view"] = measure_sh16_single_view(torch)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cpu_oracle_sample, wl, args.cpu_fraction, "iterations/s")
     if rank == 0:
@@ -640,6 +645,78 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
                                       "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes}
     del trp
     return res
+
+
+def narrow_views(views: int = 4, f: float = 3600.0):
+    """The 3M city scene seen through narrow cameras (1920x1080, focal length 3600: a
+    half-angle of 15 degrees horizontally) from the first poses of its radius-8 circle:
+    each view keeps a small part of the scene, the regime the packed layout is for.
+    Seeded random targets for an L1 training step."""
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    wl = scenes.city3m(poses=views)
+    cams = []
+    for c in wl.cameras:
+        R = np.asarray(c["R"], np.float64)
+        eye = -R.T @ np.asarray(c["t"], np.float64)
+        Rn, tn = scenes.look_at(eye)
+        cams.append(scenes.camera(Rn, tn, f, f, 960.0, 540.0, 1920, 1080))
+    rng = np.random.default_rng(7)
+    targets = [rng.uniform(0.0, 1.0, (1080, 1920, 3)).astype(np.float32) for _ in cams]
+    return wl.scene, cams, targets
+
+
+def measure_packed_narrow(torch, steps: int = 5):
+    """The packed layout where a view keeps a small part of the scene (narrow_views):
+    training step time and peak device memory of Trainer(packed=True) against the same
+    step unpacked, both from the same scene."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    scene, cams, targets_h = narrow_views()
+    targets = [torch.from_numpy(t).cuda() for t in targets_h]
+    lrs = dict(scenes.ADAM_LR)
+    res = {"workload": f"city 3M, {len(cams)} views of 1920x1080 at focal length {cams[0]['fx']:.0f}",
+           "gaussians": scene.n}
+    for packed in (True, False):
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+        tr = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in cams], targets, dict(lrs),
+                        densify=True, packed=packed)
+        for _ in range(3):
+            tr.step()
+        torch.cuda.synchronize()
+        s = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            tr.step()
+        e1.record(s)
+        torch.cuda.synchronize()
+        key = "packed" if packed else "unpacked"
+        res[f"step_ms_{key}"] = e0.elapsed_time(e1) / steps
+        res[f"peak_memory_gb_{key}"] = (torch.cuda.max_memory_allocated() - base) / 1e9
+        if packed:
+            res["visible_fraction_per_view"] = float(tr.counts[1].cpu().numpy().mean() / scene.n)
+            res["slot_capacity"] = int(tr.pcap)
+        del tr
+    res["speedup"] = res["step_ms_unpacked"] / res["step_ms_packed"]
+    return res
+
+
+def measure_sh16_single_view(torch, steps: int = 10):
+    """16-bit SH storage on the single-view training step of the 1M mixture at 1296x840,
+    against the float32 step (paired_step_ms), both from the same scene."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    wl = scenes.mixture1m()
+    targets = [torch.from_numpy(t).cuda() for t in wl.targets]
+    mk = [pl.Trainer(pl.Gaussians.from_scene(wl.scene), [pl.View(wl.scene.n, c) for c in wl.cameras], targets,
+                     dict(wl.adam_lr), densify=True, sh16=h) for h in (True, False)]
+    ms_h, ms_f = paired_step_ms(mk[0], mk[1], steps, torch)
+    del mk
+    return {"workload": "mixture 1M, one 1296x840 view per step", "step_ms_sh16": ms_h, "step_ms_f32": ms_f,
+            "speedup": ms_f / ms_h}
 
 
 def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
