@@ -207,9 +207,10 @@ gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_
 }
 
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam) {
+    (void)cam;
     if (n < 0) n = 0;
     if (capacity < 0) capacity = 0;
-    return gsk::sort_workspace_layout(n, capacity, gsk::tile_count(cam), nullptr, nullptr);
+    return gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
 }
 
 }  // extern "C"
@@ -235,14 +236,14 @@ gs_status bin_sort_impl(const char* fn, const gs_projected* proj, int64_t n, con
         CHECK_PTR(keys, 8);
         CHECK_PTR(vals, 4);
     }
-    const size_t need = gsk::sort_workspace_layout(n, capacity, gsk::tile_count(cam), nullptr, nullptr);
+    const size_t need = gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
     if (workspace_bytes < need)
         return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
     const int64_t tiles = int64_t((cam->width + GS_TILE - 1) / GS_TILE) * ((cam->height + GS_TILE - 1) / GS_TILE);
     if (tiles > (int64_t(1) << 20)) return fail(GS_ERR_UNSUPPORTED, "%s: more than 2^20 tiles", fn);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     gsk::SortWorkspace ws;
-    gsk::sort_workspace_layout(n, capacity, gsk::tile_count(cam), workspace, &ws);
+    gsk::sort_workspace_layout(n, capacity, workspace, &ws);
     const gsk::CamArgs c = gsk::make_cam(*cam);
     cudaError_t e = order ? gsk::launch_bin_sort_ordered(*proj, n, order, c, ws, keys, vals, capacity, tile_ranges,
                                                          count_dev, s)

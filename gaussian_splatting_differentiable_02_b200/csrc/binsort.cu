@@ -47,11 +47,6 @@ constexpr int kEmitPerThread = GS_EMIT_ITEMS;
 constexpr int kEmitChunk = kEmitBlock * kEmitPerThread;  // Gaussians per emit block
 static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halves a power of two");
 
-// single-pass binning: chunks per segment of the scan over chunks (a chunk's count
-// for a tile is at most kEmitChunk, so a prefix within a segment fits 16 bits)
-constexpr int kSegChunks = 64;
-static_assert(kSegChunks * kEmitChunk <= 65535, "prefixes within a segment are 16-bit");
-
 #ifndef GS_SORT_ITEMS
 #define GS_SORT_ITEMS 8
 #endif
@@ -505,189 +500,6 @@ __global__ void __launch_bounds__(kSortBlock) emit_ranked_kernel(
     }
 }
 
-// ---------------------------------------------------------------- single pass
-// For tile grids of at most kSinglePassTiles tiles the instances are binned in
-// one pass over the depth order: a chunk's Gaussians cover each tile some number
-// of times (count_tiles: a difference array over every rectangle row, then a
-// scan of each row); the counts are scanned over the chunks (scan_chunks within
-// segments of kSegChunks chunks, scan_segments over the segments) and over the
-// tiles (scan_tiles: the tile ranges and K); then every chunk writes each of its
-// instances straight to its final place (emit_tiles).  Within a tile the chunks
-// come in depth order and a chunk writes its Gaussians in depth order, so the
-// instances of a tile are ordered by (depth, Gaussian index), the key order.
-
-// Per chunk (kEmitChunk Gaussians of the depth order) and tile: how many of the
-// chunk's Gaussians cover the tile (thist[chunk][tile], 16-bit).
-__global__ void __launch_bounds__(kEmitBlock) count_tiles_kernel(const uint32_t* __restrict__ touched,
-                                                                 const uint2* __restrict__ rect,
-                                                                 const uint32_t* __restrict__ order, int64_t n,
-                                                                 int tiles_x, int tiles_y,
-                                                                 uint16_t* __restrict__ thist) {
-    __shared__ int32_t d[kSinglePassTiles];  // per row: +1 where a rectangle row starts, -1 where it ends
-    const int T = tiles_x * tiles_y;
-    for (int t = threadIdx.x; t < T; t += kEmitBlock) d[t] = 0;
-    __syncthreads();
-    const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
-    for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
-        const int64_t i = base + k;
-        if (i >= n) break;
-        const uint32_t g = __ldg(order + i);
-        if (__ldg(touched + g) == 0u) continue;
-        const uint2 r = __ldg(rect + g);
-        const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu), y1 = int(r.y >> 16);
-        for (int y = y0; y < y1; ++y) {
-            atomicAdd(&d[y * tiles_x + x0], 1);
-            if (x1 < tiles_x) atomicAdd(&d[y * tiles_x + x1], -1);
-        }
-    }
-    __syncthreads();
-    // inclusive scan of every row (a warp per row, 32 columns at a time)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int y = warp; y < tiles_y; y += kEmitBlock / 32) {
-        int carry = 0;
-        for (int x0 = 0; x0 < tiles_x; x0 += 32) {
-            const int x = x0 + lane;
-            int v = x < tiles_x ? d[y * tiles_x + x] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            if (x < tiles_x) d[y * tiles_x + x] = v + carry;
-            carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-    }
-    __syncthreads();
-    uint16_t* row = thist + int64_t(blockIdx.x) * T;
-    for (int t = threadIdx.x; t < T; t += kEmitBlock) row[t] = uint16_t(d[t]);
-}
-
-// Per tile (x) and segment (y) of kSegChunks chunks: each chunk's count replaced
-// by the exclusive prefix within the segment; segsum[seg][tile] = the segment's sum.
-__global__ void __launch_bounds__(256) scan_chunks_kernel(uint16_t* __restrict__ thist, int64_t nb, int T,
-                                                          uint32_t* __restrict__ segsum) {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    const int64_t c0 = int64_t(blockIdx.y) * kSegChunks;
-    const int cnt = int(min(int64_t(kSegChunks), nb - c0));
-    uint16_t* col = thist + c0 * T + t;
-    uint32_t v[kSegChunks];
-#pragma unroll
-    for (int c = 0; c < kSegChunks; ++c) v[c] = c < cnt ? col[int64_t(c) * T] : 0u;  // loads first
-    uint32_t run = 0;
-#pragma unroll
-    for (int c = 0; c < kSegChunks; ++c) {
-        if (c < cnt) col[int64_t(c) * T] = uint16_t(run);
-        run += v[c];
-    }
-    segsum[int64_t(blockIdx.y) * T + t] = run;
-}
-
-// Per tile: each segment's sum replaced by the exclusive prefix over segments;
-// tile_count[tile] = the tile's instance count.
-__global__ void __launch_bounds__(256) scan_segments_kernel(uint32_t* __restrict__ segsum, int64_t nseg, int T,
-                                                            uint32_t* __restrict__ tile_count) {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    uint32_t run = 0;
-    for (int64_t g = 0; g < nseg; ++g) {
-        const uint32_t v = segsum[g * T + t];
-        segsum[g * T + t] = run;
-        run += v;
-    }
-    tile_count[t] = run;
-}
-
-// One CTA: the exclusive scan of the tile counts (replaced by each tile's first
-// position), K to *total and *total_copy, and the tile ranges when K fits the
-// capacity (the ranges were cleared before).
-__global__ void __launch_bounds__(1024) scan_tiles_kernel(uint32_t* __restrict__ tile_count, int T,
-                                                          int64_t capacity, uint2* __restrict__ ranges,
-                                                          unsigned long long* total,
-                                                          unsigned long long* total_copy) {
-    constexpr int kPer = kSinglePassTiles / 1024;
-    const int t0 = threadIdx.x * kPer;
-    uint32_t c[kPer];
-    unsigned long long mine = 0;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        c[k] = t0 + k < T ? tile_count[t0 + k] : 0u;
-        mine += c[k];
-    }
-    unsigned long long K;
-    unsigned long long run = block_excl_scan(mine, &K);
-    const bool fits = K <= static_cast<unsigned long long>(capacity);
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        if (t0 + k < T) {
-            tile_count[t0 + k] = uint32_t(run);
-            if (fits && c[k] > 0u) ranges[t0 + k] = make_uint2(uint32_t(run), uint32_t(run + c[k]));
-        }
-        run += c[k];
-    }
-    if (threadIdx.x == 0) {
-        *total = K;
-        if (total_copy) *total_copy = K;
-    }
-}
-
-// Every instance of the chunk to its final place: the chunk's warps split the tile
-// ids into eight bands, and each warp walks all the chunk's Gaussians in depth
-// order, writing the instances that fall in its band (a rectangle row at a time,
-// a lane per tile) at its tile's next position, counted in shared memory from the
-// tile's first position plus the chunk's prefix.  A Gaussian's tiles are distinct,
-// so the lanes never share a counter.
-__global__ void __launch_bounds__(kEmitBlock) emit_tiles_kernel(
-    const uint32_t* __restrict__ touched, const uint2* __restrict__ rect, const uint32_t* __restrict__ order,
-    const float* __restrict__ depth, int64_t n, int tiles_x, int tiles_y, const uint16_t* __restrict__ thist,
-    const uint32_t* __restrict__ segsum, const uint32_t* __restrict__ tile_base, const Count cnt,
-    uint64_t* __restrict__ keys, uint32_t* __restrict__ vals) {
-    __shared__ uint32_t next[kSinglePassTiles];
-    __shared__ uint32_t s_gid[kEmitChunk];
-    __shared__ uint32_t s_depth[kEmitChunk];
-    __shared__ uint2 s_rect[kEmitChunk];
-    if (cnt.get() == 0) return;  // more instances than the capacity (or none): emit nothing
-    const int T = tiles_x * tiles_y;
-    const int64_t seg = int64_t(blockIdx.x) / kSegChunks;
-    const uint16_t* pre = thist + int64_t(blockIdx.x) * T;
-    const uint32_t* spre = segsum + seg * T;
-    for (int t = threadIdx.x; t < T; t += kEmitBlock) next[t] = __ldg(tile_base + t) + __ldg(spre + t) + pre[t];
-    const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
-    const int m = int(min(int64_t(kEmitChunk), n - base));
-    for (int k = threadIdx.x; k < m; k += kEmitBlock) {
-        const uint32_t g = __ldg(order + base + k);
-        s_gid[k] = g;
-        const bool vis = __ldg(touched + g) > 0u;
-        s_rect[k] = vis ? __ldg(rect + g) : make_uint2(0u, 0u);
-        s_depth[k] = vis ? __float_as_uint(__ldg(depth + g)) : 0u;
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int kBands = kEmitBlock / 32;
-    const int lo = int((int64_t(T) * warp) / kBands), hi = int((int64_t(T) * (warp + 1)) / kBands);
-    for (int k = 0; k < m; ++k) {
-        const uint2 r = s_rect[k];
-        const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu), y1 = int(r.y >> 16);
-        // the rectangle's tile ids lie in [y0 TX + x0, (y1 - 1) TX + x1): skip it unless
-        // that meets this warp's band (culled Gaussians have an empty rectangle)
-        if (x1 <= x0 || y0 * tiles_x + x0 >= hi || (y1 - 1) * tiles_x + x1 <= lo) continue;
-        const uint32_t g = s_gid[k];
-        const uint64_t z = s_depth[k];
-        for (int y = y0; y < y1; ++y) {
-            for (int x = x0 + lane; x < x1; x += 32) {
-                const int t = y * tiles_x + x;
-                if (t >= lo && t < hi) {
-                    const uint32_t pos = next[t];
-                    next[t] = pos + 1u;
-                    keys[pos] = (uint64_t(uint32_t(t)) << 32) | z;
-                    vals[pos] = g;
-                }
-            }
-        }
-        __syncwarp();
-    }
-}
-
 __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict__ keys, const Count cnt,
                                                      uint2* __restrict__ ranges) {
     const int64_t K = cnt.get();
@@ -721,19 +533,15 @@ void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout, uint64
 
 }  // namespace
 
-size_t sort_workspace_layout(int64_t n, int64_t capacity, int64_t tiles, void* base, SortWorkspace* ws) {
+size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws) {
     const int64_t nb_emit = (n + kEmitChunk - 1) / kEmitChunk;
     const int64_t slots = capacity > n ? capacity : n;  // the depth sort borrows the tile buffers
     const int64_t nb_sort = (slots + kSortTile - 1) / kSortTile;
-    const bool single = tiles > 0 && tiles <= kSinglePassTiles;
-    const int64_t nseg = (nb_emit + kSegChunks - 1) / kSegChunks;
     size_t off = 0;
     char* b = static_cast<char*>(base);
     SortWorkspace w;
     w.nb_emit = nb_emit;
     w.nb_sort = nb_sort;
-    w.tiles = tiles;
-    w.nseg = nseg;
     w.block_sums = reinterpret_cast<unsigned long long*>(b + off);
     off += align_up(sizeof(unsigned long long) * size_t(nb_emit > 0 ? nb_emit : 1));
     w.total = reinterpret_cast<unsigned long long*>(b + off);
@@ -751,12 +559,6 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, int64_t tiles, void* b
     off += align_up(sizeof(uint32_t) * 256 * size_t(nb_hist > 0 ? nb_hist : 1));
     w.digit_totals = reinterpret_cast<uint32_t*>(b + off);
     off += align_up(sizeof(uint32_t) * 256);
-    w.thist = reinterpret_cast<uint16_t*>(b + off);
-    off += single ? align_up(sizeof(uint16_t) * size_t(nb_emit > 0 ? nb_emit : 1) * size_t(tiles)) : 0;
-    w.segsum = reinterpret_cast<uint32_t*>(b + off);
-    off += single ? align_up(sizeof(uint32_t) * size_t(nseg > 0 ? nseg : 1) * size_t(tiles)) : 0;
-    w.tile_base = reinterpret_cast<uint32_t*>(b + off);
-    off += single ? align_up(sizeof(uint32_t) * size_t(tiles)) : 0;
     if (ws) *ws = w;
     return off;
 }
@@ -834,25 +636,9 @@ cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const u
         if (e == cudaSuccess && count_out) e = cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), s);
         return e;
     }
-    const uint2* rect = reinterpret_cast<const uint2*>(proj.rect);
-    if (T <= kSinglePassTiles) {
-        const int Ti = int(T);
-        const unsigned tblocks = unsigned((T + 255) / 256);
-        count_tiles_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, rect, order, n, cam.TX,
-                                                                        cam.TY, ws.thist);
-        scan_chunks_kernel<<<dim3(tblocks, unsigned(ws.nseg)), 256, 0, s>>>(ws.thist, ws.nb_emit, Ti, ws.segsum);
-        scan_segments_kernel<<<tblocks, 256, 0, s>>>(ws.segsum, ws.nseg, Ti, ws.tile_base);
-        scan_tiles_kernel<<<1, 1024, 0, s>>>(ws.tile_base, Ti, capacity, reinterpret_cast<uint2*>(ranges), ws.total,
-                                             count_out);
-        const Count inst{0, ws.total, capacity};
-        emit_tiles_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, rect, order, proj.depth, n,
-                                                                       cam.TX, cam.TY, ws.thist, ws.segsum,
-                                                                       ws.tile_base, inst, keys, vals);
-        count_launches(5);
-        return cudaGetLastError();
-    }
     const int bits = tile_bits(T);
     const int passes = bits > 0 ? (bits + 7) / 8 : 1;
+    const uint2* rect = reinterpret_cast<const uint2*>(proj.rect);
     // the first pass over the tile id (its low 8 bits) is fused into the emission:
     // per-block digit histograms and instance counts, K, the scanned histograms,
     // then the ranked emission into buffer 0 (or the final keys)

@@ -34,12 +34,6 @@ inline int sh_planes(int deg) {
     }
 }
 
-// Tiles of a camera's grid, 0 for a missing or empty camera (workspace sizing).
-inline int64_t tile_count(const gs_camera* c) {
-    if (!c || c->width <= 0 || c->height <= 0) return 0;
-    return int64_t((c->width + kTile - 1) / kTile) * ((c->height + kTile - 1) / kTile);
-}
-
 inline int tile_bits(int64_t tiles) {
     int b = 0;
     while ((int64_t(1) << b) < tiles) ++b;
@@ -100,27 +94,16 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
                                      float* densify_accum, int32_t* densify_count, int32_t* densify_max_radius,
                                      const AdamStep* adam, cudaStream_t s);
 
-// Tile grids up to this many tiles are binned in a single pass (per-chunk tile
-// counts, their scan, then every instance written to its final place); larger
-// ones by the radix passes over the tile bits.
-constexpr int64_t kSinglePassTiles = 8192;
-
 struct SortWorkspace {
     unsigned long long* block_sums;  // [nb_emit]
     unsigned long long* total;       // [1]
     uint32_t* tkey[2];               // [max(capacity, n)] 32-bit keys, ping-pong
     uint32_t* tval[2];               // [max(capacity, n)] Gaussian indices, ping-pong
-    uint32_t* hist;                  // [256][max(nb_sort, nb_emit)]
+    uint32_t* hist;                  // [256][nb_sort]
     uint32_t* digit_totals;          // [256]
-    // single pass (tiles <= kSinglePassTiles): per chunk and tile the count, then its
-    // prefix within the chunk's segment; per segment and tile the count, then its
-    // prefix over segments; per tile the count, then its first position
-    uint16_t* thist;                 // [nb_emit][tiles]
-    uint32_t* segsum;                // [nseg][tiles]
-    uint32_t* tile_base;             // [tiles]
-    int64_t nb_emit, nb_sort, tiles, nseg;
+    int64_t nb_emit, nb_sort;
 };
-size_t sort_workspace_layout(int64_t n, int64_t capacity, int64_t tiles, void* base, SortWorkspace* ws);
+size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws);
 
 // Enqueues the whole binning and sort; the instance count stays on the device
 // (ws.total, and *count_out when given).  K > capacity: nothing emitted, ranges empty.
