@@ -273,11 +273,21 @@ struct Alpha {
 // -alpha at one pixel, 0 for a pixel that does not blend the entry (sigma < 0 or
 // alpha < 1/255); with kMayClamp alpha is clamped at 0.99 and (kGate) gate = 0 when
 // it was, else 1; without, alpha cannot reach the clamp and no gate is formed.
+// 1.0f where a >= b, else 0.0f: one compare that writes a float (the ALU pipe is
+// the busier one in these loops, and the mask's product runs on the FMA pipe)
+__device__ __forceinline__ float mask_ge(float a, float b) {
+    float m;
+    asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(m) : "f"(a), "f"(b));
+    return m;
+}
+
 template <bool kGate, bool kMayClamp>
 __device__ __forceinline__ void alpha_at(float e, bool sign_ok, float& nal, float& gate) {
     const float a = ex2_approx(e);
-    nal = kMayClamp ? fmaxf(-a, -kAlphaMax) : -a;  // -min(a, 0.99)
-    nal = (sign_ok && nal <= -kAlphaMin) ? nal : 0.f;
+    // min(a, 0.99) >= 1/255 exactly when a >= 1/255; a pixel that fails it (or the
+    // sign test) gets -alpha = -0, which leaves every sum as it was
+    const float m = sign_ok ? mask_ge(a, kAlphaMin) : 0.f;
+    nal = (kMayClamp ? fmaxf(-a, -kAlphaMax) : -a) * m;  // -min(a, 0.99), or 0
     if (kGate && kMayClamp) gate = a > kAlphaMax ? 0.f : 1.f;
 }
 
@@ -431,22 +441,21 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
             // pixel that blends, which stops there without taking the entry
 #pragma unroll
             for (int p = 0; p < kPairs; ++p) {
-                const f2 na = mul2(r.nal[p], on[p]);
+                f2 na = mul2(r.nal[p], on[p]);
                 const f2 Tn = mul2(T[p], add2(one, na));  // T (1 - alpha)
-                f2 nw = mul2(na, T[p]);                    // -alpha T
-                const bool low0 = Tn.x < kTMin, low1 = Tn.y < kTMin;
-                nw.x = low0 ? 0.f : nw.x;
-                nw.y = low1 ? 0.f : nw.y;
+                // 1 while T (1 - alpha) >= 1e-4; a pixel that reaches 0 stops there
+                // without the entry: its -alpha becomes 0, so T (1 - 0) = T exactly
+                const f2 keep = make_float2(mask_ge(Tn.x, kTMin), mask_ge(Tn.y, kTMin));
+                na = mul2(na, keep);
+                const f2 nw = mul2(na, T[p]);  // -alpha T
                 Cr[p] = fma2(ncr, nw, Cr[p]);
                 Cg[p] = fma2(ncg, nw, Cg[p]);
                 Cb[p] = fma2(ncb, nw, Cb[p]);
-                T[p].x = low0 ? T[p].x : Tn.x;
-                T[p].y = low1 ? T[p].y : Tn.y;
-                last[2 * p] = (na.x != 0.f && !low0) ? pos : last[2 * p];
-                last[2 * p + 1] = (na.y != 0.f && !low1) ? pos : last[2 * p + 1];
-                if (kCount) c_work += int(na.x != 0.f && !low0) + int(na.y != 0.f && !low1);
-                on[p].x = low0 ? 0.f : on[p].x;
-                on[p].y = low1 ? 0.f : on[p].y;
+                T[p] = mul2(T[p], add2(one, na));
+                on[p] = mul2(on[p], keep);
+                last[2 * p] = na.x != 0.f ? pos : last[2 * p];
+                last[2 * p + 1] = na.y != 0.f ? pos : last[2 * p + 1];
+                if (kCount) c_work += int(na.x != 0.f) + int(na.y != 0.f);
             }
         }
         __syncwarp();
