@@ -667,8 +667,9 @@ def narrow_views(views: int = 4, f: float = 3600.0):
 
 def measure_packed_narrow(torch, steps: int = 5):
     """The packed layout where a view keeps a small part of the scene (narrow_views):
-    training step time and peak device memory of Trainer(packed=True) against the same
-    step unpacked, both from the same scene."""
+    training step time and device memory (held after the warm-up steps, and the peak
+    over the timed steps, both above what was allocated before the Trainer) of
+    Trainer(packed=True) against the same step unpacked, both from the same scene."""
     from gaussian_splatting_differentiable_02_b200 import pipeline as pl
     from gaussian_splatting_differentiable_02_b200 import scenes
     scene, cams, targets_h = narrow_views()
@@ -679,13 +680,16 @@ def measure_packed_narrow(torch, steps: int = 5):
     for packed in (True, False):
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
-        torch.cuda.reset_peak_memory_stats()
         base = torch.cuda.memory_allocated()
         tr = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in cams], targets, dict(lrs),
                         densify=True, packed=packed)
-        for _ in range(3):
+        for _ in range(3):  # the packed Trainer sizes its slots to the views in these steps
             tr.step()
         torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        # memory held by the Trainer in the steady state, and its peak over the timed steps
+        res[f"resident_memory_gb_{'packed' if packed else 'unpacked'}"] = (torch.cuda.memory_allocated() - base) / 1e9
+        torch.cuda.reset_peak_memory_stats()
         s = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
