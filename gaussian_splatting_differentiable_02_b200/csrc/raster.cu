@@ -3,12 +3,13 @@
 // §2.1: shared-memory prefetch of the tile's Gaussians, SoA features, warp-level
 // synchronisation; §2.2: a standalone backward entry).
 //
-// Work decomposition: one warp per 16x16 tile (one tile per block, blocks
-// launched in the tile order of gs_tile_order when one is given); each lane owns
-// a column segment of 8 pixels (lane & 15 selects the column, lane >> 4 the
-// upper or lower half of the tile), so that the per-entry work of the warp (its
-// shared-memory reads, the gradient reduction, the branches) is spread over 256
-// pixels.  The warp walks its
+// Work decomposition: one warp per pixel box of a tile, one warp per block, blocks
+// launched in the tile order of gs_tile_order when one is given; each lane owns a
+// column segment of PX pixels (lane & 15 selects the column, lane >> 4 the upper
+// or lower half of the box).  Large tile grids take PX = 8, a box per tile, so
+// that the per-entry work of the warp (its shared-memory reads, the gradient
+// reduction, the branches) is spread over 256 pixels; small grids PX = 4, two
+// boxes per tile, for twice the warps (Layout below).  The warp walks its
 // tile's sorted list in batches of 32 entries: every lane gathers one entry's
 // 40 bytes (xy, conic + opacity, colour) by Gaussian index into shared memory
 // with cp.async, double-buffered so the next batch is in flight while the
@@ -18,7 +19,7 @@
 // and the constants of the others are compacted, so the warp's loop visits only
 // entries that can reach its box).  Every lane then reads each entry once
 // (broadcast loads) and
-// applies it to its 8 pixels, whose terms that depend only on dx are shared;
+// applies it to its PX pixels, whose terms that depend only on dx are shared;
 // the pixels go in pairs through the paired float32 instructions of sm_100
 // (fma/mul/add on two floats at once).  No block-wide barrier is used: warps
 // synchronise with __syncwarp and finish independently.
@@ -61,37 +62,31 @@ constexpr double kLog2eD = 1.4426950408889634;
 // trace^2 / det = kappa + 1/kappa + 2 for the eigenvalue ratio kappa; kappa = 8 -> 10.125
 constexpr float kCondMaxTraceSqOverDet = 10.125f;
 
-#ifndef GS_RASTER_PX
-#define GS_RASTER_PX 8
-#endif
-#ifndef GS_RASTER_BOXW
-#define GS_RASTER_BOXW 16
-#endif
-constexpr int kPx = GS_RASTER_PX;        // pixels per lane (a column segment)
-constexpr int kBoxW = GS_RASTER_BOXW;    // width of a warp's pixel box (16 or 8)
-constexpr int kLaneRows = 32 / kBoxW;    // lanes stacked vertically in the box
-constexpr int kBoxH = kLaneRows * kPx;   // height of a warp's pixel box
-constexpr int kSubX = kTile / kBoxW, kSubY = kTile / kBoxH;
-constexpr int kSub = kSubX * kSubY;      // warps per tile
-#ifndef GS_RASTER_WARPS
-#define GS_RASTER_WARPS 1
-#endif
-// warps per block: one tile per block, so that a block retires with its own tile.
-// Measured per 1080p view of the 1M mixture (forward / backward ms): 4 pixels per
-// lane in 16x8 boxes, two warps a block, 10 blocks an SM 0.622 / 1.144; 8 pixels
-// per lane, one warp a block, 12 / 14 / 16 / 20 blocks an SM 0.666 / 1.205,
-// 0.609 / 1.098, 0.618 / 1.069, 0.631 / 1.198; two warps a block, 8 blocks an
-// SM 0.639 / 1.208.
-constexpr int kWarps = GS_RASTER_WARPS;
-static_assert(kTile % kBoxW == 0 && kTile % kBoxH == 0, "warp boxes tile the 16x16 tile");
-// resident blocks per SM the register allocation is sized for (launch bounds; the
-// forward pass does best at 14, the reverse pass at 16)
-#ifndef GS_RASTER_FWD_MIN_BLOCKS
-#define GS_RASTER_FWD_MIN_BLOCKS 14
-#endif
-#ifndef GS_RASTER_BWD_MIN_BLOCKS
-#define GS_RASTER_BWD_MIN_BLOCKS 16
-#endif
+// Warp layouts: a warp composites a box 16 pixels wide and 2 PX tall, each lane a
+// column segment of PX pixels (lane & 15 selects the column, lane >> 4 the upper
+// or lower half of the box); one warp per block, so that a block retires with its
+// own box.  PX = 8: the box is the whole tile, and the warp's per-entry work (its
+// shared-memory reads, the gradient reduction, the branches) is spread over 256
+// pixels; PX = 4: two warps a tile, which culls entries against half tiles and
+// gives twice the warps.  Grids of at least kWideLayoutTiles tiles use PX = 8,
+// smaller ones PX = 4.  Measured (forward / backward ms per view): 16 1080p views
+// of the 1M mixture (8160 tiles) PX = 8 at 14 / 16 blocks an SM 0.589 / 1.067,
+// PX = 4 at 20 / 20 blocks 0.606 / 1.166; the 1296x840 view (4293 tiles) PX = 8
+// 0.454 / 0.856, PX = 4 0.404 / 0.806 (two warps a block, 10 blocks: 0.622 / 1.144
+// at 1080p; PX = 8 at 12 / 14 / 20 blocks slower).
+constexpr int kBoxW = 16;               // width of a warp's pixel box
+constexpr int kWarps = 1;               // warps per block
+constexpr int64_t kWideLayoutTiles = 6144;
+template <int PX>
+struct Layout {
+    static_assert(PX % 2 == 0 && kTile % (2 * PX) == 0, "pixel pairs; boxes tile the 16x16 tile");
+    static constexpr int kPairs = PX / 2;                // pixel pairs per lane
+    static constexpr int kBoxH = 2 * PX;                 // height of a warp's box
+    static constexpr int kSub = kTile / kBoxH;           // warps per tile
+    // resident blocks per SM the register allocation is sized for (launch bounds)
+    static constexpr int kFwdMinBlocks = PX == 8 ? 14 : 20;
+    static constexpr int kBwdMinBlocks = PX == 8 ? 16 : 20;
+};
 constexpr int kBatch = 32;  // list entries staged per warp per batch
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -185,8 +180,9 @@ __device__ __forceinline__ R box_min(R A, R B, R C, R u, R v, R bx0, R bx1, R by
 // in S.idx (bits 0-4) and kMayClamp (bit 5) when the entry's opacity is high
 // enough for its alpha to reach the 0.99 clamp; returns their number.  Called by
 // the whole warp.
-template <bool kNegRgb>
+template <bool kNegRgb, int PX>
 __device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, float bx0, float by0) {
+    constexpr int kBoxH = Layout<PX>::kBoxH;
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = make_float4(0.f, 0.f, 0.f, kSkip);
     float2 pc = make_float2(0.f, 0.f);
     bool may_clamp = false;
@@ -247,8 +243,6 @@ __device__ __forceinline__ int prep(WarpStage& S, int buf, int count, int lane, 
 
 // Pairs of pixels go through the paired float32 instructions of sm_100
 // (two IEEE operations per instruction, rounded as two scalar ones).
-constexpr int kPairs = kPx / 2;
-static_assert(kPx % 2 == 0, "pixels per lane come in pairs");
 using f2 = float2;
 __device__ __forceinline__ f2 splat(float v) { return make_float2(v, v); }
 __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
@@ -262,11 +256,12 @@ __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 // was clamped at 0.99 and 1 elsewhere.  The masks are floats rather than bits: a
 // pixel that does not take an entry runs the same paired instructions with alpha
 // 0, and a clamped pixel's dL/dsigma is multiplied by 0.
+template <int PX>
 struct Alpha {
-    f2 nal[kPairs];
-    f2 dy[kPairs];
-    f2 t[kPairs];
-    f2 gate[kPairs];  // 0 where alpha was clamped at 0.99, else 1 (backward pass)
+    f2 nal[PX / 2];
+    f2 dy[PX / 2];
+    f2 t[PX / 2];
+    f2 gate[PX / 2];  // 0 where alpha was clamped at 0.99, else 1 (backward pass)
     float dx;
 };
 
@@ -292,9 +287,10 @@ __device__ __forceinline__ void alpha_at(float e, bool sign_ok, float& nal, floa
 }
 
 // nyc[p]: minus the centres' y of the lane's pixels 2p and 2p + 1.
-template <bool kGate, bool kMayClamp>
+template <bool kGate, bool kMayClamp, int PX>
 __device__ __forceinline__ void eval_alpha(const float4& pa, const float4& pb, const float2& pc, const float4& con,
-                                           float px, const f2 (&nyc)[kPairs], Alpha& r) {
+                                           float px, const f2 (&nyc)[PX / 2], Alpha<PX>& r) {
+    constexpr int kPairs = PX / 2;
     const f2 vy = splat(pa.y);
     if (pb.w >= kFactored) {
         const bool indef = pb.w == kFactoredIndef;
@@ -348,19 +344,20 @@ struct FwdArgs {
 // the method's work (blended in the forward pass, took a gradient in the
 // reverse pass), list entries staged, and entries that reached the box.
 __device__ __forceinline__ void add_counts(unsigned long long* counts, int evaluated_entries, int work_pairs,
-                                           int staged, int lane) {
+                                           int staged, int lane, int box_pixels) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) work_pairs += __shfl_xor_sync(kFull, work_pairs, o);
     if (lane == 0) {
-        atomicAdd(counts + 0, (unsigned long long)evaluated_entries * (32 * kPx));
+        atomicAdd(counts + 0, (unsigned long long)evaluated_entries * box_pixels);
         atomicAdd(counts + 1, (unsigned long long)work_pairs);
         atomicAdd(counts + 2, (unsigned long long)staged);
         atomicAdd(counts + 3, (unsigned long long)evaluated_entries);
     }
 }
 
-template <bool kCount>
-__global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_fwd_kernel(const FwdArgs a) {
+template <int PX, bool kCount>
+__global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster_fwd_kernel(const FwdArgs a) {
+    constexpr int kPx = PX, kPairs = Layout<PX>::kPairs, kBoxH = Layout<PX>::kBoxH, kSub = Layout<PX>::kSub;
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
@@ -368,8 +365,8 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
     if (slot >= a.tiles) return;
     const int tile = a.order ? int(__ldg(a.order + slot)) : slot;  // longest lists first when ordered
     WarpStage& S = stage[warp];
-    const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
-    const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
+    const int xb = (tile % a.TX) * kTile;  // this warp's pixel box
+    const int yb = (tile / a.TX) * kTile + sub * kBoxH;
     const int x = xb + lane % kBoxW;
     const int y0 = yb + (lane / kBoxW) * kPx;
     const float px = float(x) + 0.5f;
@@ -410,7 +407,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (b + 1 < nb)
             gather<false>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t((b + 1) * kBatch),
                           min(n - (b + 1) * kBatch, kBatch), lane);
-        const int live = prep<true>(S, buf, cnt, lane, bx0, by0);
+        const int live = prep<true, PX>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         if (kCount) c_staged += cnt;
         bool finished = false;
@@ -428,13 +425,13 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
             const float4 pa = S.pa[e], pb = S.pb[e];
             const float4 con = S.con[buf][j];
             const float4 nc = S.rgb[buf][j];  // minus the colour
-            Alpha r;
+            Alpha<PX> r;
             const int pos = b * kBatch + j + 1;
             const f2 ncr = splat(nc.x), ncg = splat(nc.y), ncb = splat(nc.z);
             if (ij & kMayClampBit)
-                eval_alpha<false, true>(pa, pb, S.pc[e], con, px, nyc, r);
+                eval_alpha<false, true, PX>(pa, pb, S.pc[e], con, px, nyc, r);
             else
-                eval_alpha<false, false>(pa, pb, S.pc[e], con, px, nyc, r);
+                eval_alpha<false, false, PX>(pa, pb, S.pc[e], con, px, nyc, r);
             // branch-free with float masks: -alpha is 0 for a pixel that does not blend
             // the entry or has stopped (on 0), so T (1 - alpha) = T and -alpha T = 0
             // leave it exactly as it was; T (1 - alpha) < 1e-4 then only happens for a
@@ -462,7 +459,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_FWD_MIN_BLOCKS) raster_
         if (finished) break;
     }
     cp_async_wait_all();
-    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane);
+    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
     if (x < a.W) {
 #pragma unroll
         for (int i = 0; i < kPx; ++i) {
@@ -545,8 +542,9 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
     if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
-template <bool kAbs, bool kCount>
-__global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_bwd_kernel(const BwdArgs a) {
+template <int PX, bool kAbs, bool kCount>
+__global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster_bwd_kernel(const BwdArgs a) {
+    constexpr int kPx = PX, kPairs = Layout<PX>::kPairs, kBoxH = Layout<PX>::kBoxH, kSub = Layout<PX>::kSub;
     __shared__ WarpStage stage[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
@@ -554,8 +552,8 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
     if (slot >= a.tiles) return;
     const int tile = a.order ? int(__ldg(a.order + slot)) : slot;  // longest lists first when ordered
     WarpStage& S = stage[warp];
-    const int xb = (tile % a.TX) * kTile + (sub % kSubX) * kBoxW;  // this warp's pixel box
-    const int yb = (tile / a.TX) * kTile + (sub / kSubX) * kBoxH;
+    const int xb = (tile % a.TX) * kTile;  // this warp's pixel box
+    const int yb = (tile / a.TX) * kTile + sub * kBoxH;
     const int x = xb + lane % kBoxW;
     const int y0 = yb + (lane / kBoxW) * kPx;
     const float px = float(x) + 0.5f;
@@ -609,7 +607,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             const int nhi = hi - kBatch, ncnt = min(nhi, kBatch);
             gather<true>(S, buf ^ 1, a.vals, a.xy, a.con, a.rgb, range.x + uint32_t(nhi - ncnt), ncnt, lane);
         }
-        const int live = prep<false>(S, buf, cnt, lane, bx0, by0);
+        const int live = prep<false, PX>(S, buf, cnt, lane, bx0, by0);
         __syncwarp();
         if (kCount) {
             c_staged += cnt;
@@ -626,8 +624,8 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
             // whose gate then multiplies dL/dsigma (else the gate is 1 and not formed)
             const auto entry = [&](auto may_clamp) {
                 constexpr bool kMC = decltype(may_clamp)::value;
-                Alpha r;
-                eval_alpha<true, kMC>(pa, pb, S.pc[e], con, px, nyc, r);
+                Alpha<PX> r;
+                eval_alpha<true, kMC, PX>(pa, pb, S.pc[e], con, px, nyc, r);
                 const f2 cr = splat(c.x), cg = splat(c.y), cb = splat(c.z);
                 f2 ndr = zero, ndg = zero, ndb = zero, nmo = zero, s1 = zero, s2 = zero, nm[kPairs];
                 // branch-free: every pixel runs the same instructions, inactive ones
@@ -715,7 +713,7 @@ __global__ void __launch_bounds__(kWarps * 32, GS_RASTER_BWD_MIN_BLOCKS) raster_
         __syncwarp();
     }
     cp_async_wait_all();
-    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane);
+    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
 }
 
 // Tiles ordered by decreasing list length (bucketed by floor(sqrt(length)),
@@ -775,14 +773,39 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
     a.final_T = final_T;
     a.n_contrib = n_contrib;
     a.counts = counts;
-    const unsigned grid = unsigned((a.tiles * kSub + kWarps - 1) / kWarps);
-    if (counts)
-        raster_fwd_kernel<true><<<grid, kWarps * 32, 0, s>>>(a);
-    else
-        raster_fwd_kernel<false><<<grid, kWarps * 32, 0, s>>>(a);
+    if (a.tiles >= kWideLayoutTiles) {
+        const unsigned grid = unsigned(a.tiles * Layout<8>::kSub);
+        if (counts)
+            raster_fwd_kernel<8, true><<<grid, kWarps * 32, 0, s>>>(a);
+        else
+            raster_fwd_kernel<8, false><<<grid, kWarps * 32, 0, s>>>(a);
+    } else {
+        const unsigned grid = unsigned(a.tiles * Layout<4>::kSub);
+        if (counts)
+            raster_fwd_kernel<4, true><<<grid, kWarps * 32, 0, s>>>(a);
+        else
+            raster_fwd_kernel<4, false><<<grid, kWarps * 32, 0, s>>>(a);
+    }
     count_launches(1);
     return cudaGetLastError();
 }
+
+namespace {
+template <int PX>
+void launch_raster_bwd_layout(const BwdArgs& a, bool counted, cudaStream_t s) {
+    const unsigned grid = unsigned(a.tiles * Layout<PX>::kSub);
+    if (counted) {
+        if (a.g_xy_abs)
+            raster_bwd_kernel<PX, true, true><<<grid, kWarps * 32, 0, s>>>(a);
+        else
+            raster_bwd_kernel<PX, false, true><<<grid, kWarps * 32, 0, s>>>(a);
+    } else if (a.g_xy_abs) {
+        raster_bwd_kernel<PX, true, false><<<grid, kWarps * 32, 0, s>>>(a);
+    } else {
+        raster_bwd_kernel<PX, false, false><<<grid, kWarps * 32, 0, s>>>(a);
+    }
+}
+}  // namespace
 
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,
@@ -810,17 +833,10 @@ cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, co
     a.g_rgb = reinterpret_cast<float4*>(g2.rgb);
     a.g_xy_abs = reinterpret_cast<float2*>(g2.xy_abs);
     a.counts = counts;
-    const unsigned grid = unsigned((a.tiles * kSub + kWarps - 1) / kWarps);
-    if (counts) {
-        if (a.g_xy_abs)
-            raster_bwd_kernel<true, true><<<grid, kWarps * 32, 0, s>>>(a);
-        else
-            raster_bwd_kernel<false, true><<<grid, kWarps * 32, 0, s>>>(a);
-    } else if (a.g_xy_abs) {
-        raster_bwd_kernel<true, false><<<grid, kWarps * 32, 0, s>>>(a);
-    } else {
-        raster_bwd_kernel<false, false><<<grid, kWarps * 32, 0, s>>>(a);
-    }
+    if (a.tiles >= kWideLayoutTiles)
+        launch_raster_bwd_layout<8>(a, counts != nullptr, s);
+    else
+        launch_raster_bwd_layout<4>(a, counts != nullptr, s);
     count_launches(1);
     return cudaGetLastError();
 }
