@@ -25,14 +25,10 @@
 //                     block (warp votes + per-warp counters), reorder in shared
 //                     memory, coalesced scatter; the final tile pass writes
 //                     64-bit keys
-//   count_digits      per chunk of Gaussians in depth order: its instance count
-//                     and the histogram of the low 8 bits of its instances'
-//                     tile ids
-//   scan_blocks       one CTA: exclusive scan of the chunk counts, total K
-//   emit_ranked       every visible Gaussian, in depth order, emits its instances
-//                     (row-major over its tile rectangle), ranked stably by the
-//                     low tile digit and written to their place after the first
-//                     tile pass: emission and that pass in one kernel
+//   count_sorted      per-block sum of tiles_touched in depth order
+//   scan_blocks       one CTA: exclusive scan of the block sums, total K
+//   emit              every visible Gaussian, in depth order, writes its
+//                     instances (row-major over its tile rectangle)
 //   ranges            [begin, end) of each tile in the sorted keys
 #include "internal.cuh"
 
@@ -175,38 +171,6 @@ __global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t
 }
 
 // kFinal: write 64-bit keys (key32 << 32 | depth bits of the Gaussian) to keys_out64.
-// Writes the block's elements, reordered by digit in shared memory (sk, sv, n of
-// them), to their global places gbase[digit] + offset within the digit's run: a
-// thread's loads (and, for the final pass, its gathers of the Gaussians' depths)
-// are all issued before its stores, so their latencies overlap.
-template <bool kFinal>
-__device__ __forceinline__ void scatter_runs(const uint32_t* sk, const uint32_t* sv, int n, int shift,
-                                             const uint32_t* gbase, const uint32_t* lstart,
-                                             const float* __restrict__ depth, uint32_t* __restrict__ keys_out,
-                                             uint64_t* __restrict__ keys_out64, uint32_t* __restrict__ vals_out) {
-    uint32_t k[kSortPerThread], v[kSortPerThread], z[kSortPerThread];
-#pragma unroll
-    for (int r = 0; r < kSortPerThread; ++r) {
-        const int p = threadIdx.x + r * kSortBlock;
-        k[r] = p < n ? sk[p] : 0u;
-        v[r] = p < n ? sv[p] : 0u;
-        z[r] = (kFinal && p < n) ? __float_as_uint(__ldg(depth + v[r])) : 0u;
-    }
-#pragma unroll
-    for (int r = 0; r < kSortPerThread; ++r) {
-        const int p = threadIdx.x + r * kSortBlock;
-        if (p < n) {
-            const uint32_t digit = (k[r] >> shift) & 0xffu;
-            const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
-            if (kFinal)
-                keys_out64[g] = (uint64_t(k[r]) << 32) | z[r];
-            else
-                keys_out[g] = k[r];
-            vals_out[g] = v[r];
-        }
-    }
-}
-
 // digit_bits: how many of the digit's 8 bits can be set (the last pass over the
 // tile bits has fewer); the rank votes only on those.
 template <bool kFinal>
@@ -305,7 +269,31 @@ __global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* _
     }
     __syncthreads();
     const int in_block = int(min(int64_t(kSortTile), count - tile0));
-    scatter_runs<kFinal>(sk, sv, in_block, shift, gbase, lstart, depth, keys_out, keys_out64, vals_out);
+    for (int p = threadIdx.x; p < in_block; p += kSortBlock) {
+        const uint32_t k = sk[p], v = sv[p];
+        const uint32_t digit = (k >> shift) & 0xffu;
+        const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
+        if (kFinal) {
+            keys_out64[g] = (uint64_t(k) << 32) | __float_as_uint(__ldg(depth + v));
+        } else {
+            keys_out[g] = k;
+        }
+        vals_out[g] = v;
+    }
+}
+
+__global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const uint32_t* __restrict__ touched,
+                                                                  const uint32_t* __restrict__ order, int64_t n,
+                                                                  unsigned long long* block_sums) {
+    const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
+    unsigned long long s = 0;
+    for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
+        const int64_t i = base + k;
+        if (i < n) s += __ldg(touched + __ldg(order + i));
+    }
+    unsigned long long tot;
+    block_excl_scan(s, &tot);
+    if (threadIdx.x == 0) block_sums[blockIdx.x] = tot;
 }
 
 __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
@@ -326,13 +314,21 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* b
     }
 }
 
-// The Gaussians of emit block blockIdx.x (positions [b C, (b + 1) C) of the depth
-// order, C = kEmitChunk) into shared memory: each one's first instance slot
-// within the block (an exclusive scan of tiles_touched), index and tile
-// rectangle.  Returns the block's instance count.  Called by the whole block.
-__device__ __forceinline__ uint32_t load_chunk(const uint32_t* __restrict__ touched, const uint2* __restrict__ rect,
-                                               const uint32_t* __restrict__ order, int64_t n, uint32_t* s_start,
-                                               uint32_t* s_gid, uint2* s_rect) {
+// Instances of the block's Gaussians (depth order), load-balanced: the block's
+// output slots [0, total) are dealt to its threads round-robin, and each slot
+// finds its Gaussian by a binary search over the block's exclusive offsets in
+// shared memory, then its tile from its index inside the Gaussian's tile
+// rectangle (row-major).  Consecutive slots are written by consecutive threads.
+__global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
+                                                          const uint2* __restrict__ rect,
+                                                          const uint32_t* __restrict__ order, int64_t n, int tiles_x,
+                                                          const unsigned long long* __restrict__ block_offsets,
+                                                          const Count cnt, uint32_t* __restrict__ tkeys,
+                                                          uint32_t* __restrict__ tvals) {
+    __shared__ uint32_t s_start[kEmitChunk];
+    __shared__ uint32_t s_gid[kEmitChunk];
+    __shared__ uint2 s_rect[kEmitChunk];
+    if (cnt.get() == 0) return;  // nothing fits: emit nothing
     const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
     uint32_t gid[kEmitPerThread], tt[kEmitPerThread];
     unsigned long long mine = 0;
@@ -344,6 +340,7 @@ __device__ __forceinline__ uint32_t load_chunk(const uint32_t* __restrict__ touc
     }
     unsigned long long total;
     uint32_t run = uint32_t(block_excl_scan(mine, &total));
+    const unsigned long long base = block_offsets[blockIdx.x];
 #pragma unroll
     for (int k = 0; k < kEmitPerThread; ++k) {
         const int idx = threadIdx.x * kEmitPerThread + k;
@@ -353,150 +350,18 @@ __device__ __forceinline__ uint32_t load_chunk(const uint32_t* __restrict__ touc
         run += tt[k];
     }
     __syncthreads();
-    return uint32_t(total);
-}
-
-// Instance `slot` of the chunk in load_chunk's shared memory: its Gaussian (the
-// last one whose first slot is <= slot; it has at least one instance) by binary
-// search, and its tile from the index inside the Gaussian's rectangle (row-major).
-__device__ __forceinline__ void slot_instance(const uint32_t* s_start, const uint32_t* s_gid, const uint2* s_rect,
-                                              uint32_t slot, int tiles_x, uint32_t& tile, uint32_t& gid) {
-    int lo = 0;
+    for (uint32_t slot = threadIdx.x; slot < uint32_t(total); slot += kEmitBlock) {
+        // the last Gaussian whose first slot is <= slot (it has at least one instance)
+        int lo = 0;
 #pragma unroll
-    for (int step = kEmitChunk / 2; step > 0; step >>= 1)
-        if (s_start[lo + step] <= slot) lo += step;
-    const uint32_t j = slot - s_start[lo];
-    const uint2 r = s_rect[lo];
-    const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, w = (r.y & 0xffffu) - x0;
-    tile = (y0 + j / w) * uint32_t(tiles_x) + (x0 + j % w);
-    gid = s_gid[lo];
-}
-
-// Emission fused with the first radix pass over the tile id (its low 8 bits).
-// count_digits: per emit block, the histogram of that digit over the block's
-// instances (hist[digit][block]) and the block's instance count.
-__global__ void __launch_bounds__(kEmitBlock) count_digits_kernel(const uint32_t* __restrict__ touched,
-                                                                  const uint2* __restrict__ rect,
-                                                                  const uint32_t* __restrict__ order, int64_t n,
-                                                                  int tiles_x, uint32_t* __restrict__ hist, int64_t nb,
-                                                                  unsigned long long* __restrict__ block_sums) {
-    __shared__ uint32_t s_start[kEmitChunk];
-    __shared__ uint32_t s_gid[kEmitChunk];
-    __shared__ uint2 s_rect[kEmitChunk];
-    __shared__ uint32_t h[256];
-    for (int d = threadIdx.x; d < 256; d += kEmitBlock) h[d] = 0u;
-    const uint32_t total = load_chunk(touched, rect, order, n, s_start, s_gid, s_rect);  // synchronises
-    constexpr int kAtOnce = 8;  // independent binary searches in flight per thread
-    for (uint32_t first = threadIdx.x; first < total; first += kAtOnce * kEmitBlock) {
-        uint32_t tile[kAtOnce], gid;
-#pragma unroll
-        for (int r = 0; r < kAtOnce; ++r) {
-            const uint32_t slot = first + r * kEmitBlock;
-            tile[r] = 0u;
-            if (slot < total) slot_instance(s_start, s_gid, s_rect, slot, tiles_x, tile[r], gid);
-        }
-#pragma unroll
-        for (int r = 0; r < kAtOnce; ++r)
-            if (first + r * kEmitBlock < total) atomicAdd(&h[tile[r] & 0xffu], 1u);
-    }
-    __syncthreads();
-    for (int d = threadIdx.x; d < 256; d += kEmitBlock) hist[int64_t(d) * nb + blockIdx.x] = h[d];
-    if (threadIdx.x == 0) block_sums[blockIdx.x] = total;
-}
-
-// emit_ranked: the instances of the block in emission order, ranked stably by the
-// low 8 bits of the tile id (rounds of kSortTile slots: warp votes and per-warp
-// counters as in downsweep, a running count per digit across the rounds), then
-// written by digit runs to their place in the first pass's output, whose digit
-// offsets come from the scanned histograms.  kFinal (tile ids of at most 8 bits):
-// that is the last pass, and the 64-bit keys are written.
-template <bool kFinal>
-__global__ void __launch_bounds__(kSortBlock) emit_ranked_kernel(
-    const uint32_t* __restrict__ touched, const uint2* __restrict__ rect, const uint32_t* __restrict__ order,
-    int64_t n, int tiles_x, const uint32_t* __restrict__ hist, int64_t nb, const uint32_t* __restrict__ digit_totals,
-    int digit_bits, const Count cnt, uint32_t* __restrict__ keys_out, uint64_t* __restrict__ keys_out64,
-    uint32_t* __restrict__ vals_out, const float* __restrict__ depth) {
-    static_assert(kSortBlock == kEmitBlock, "the emission and sort blocks coincide");
-    __shared__ uint32_t s_start[kEmitChunk];
-    __shared__ uint32_t s_gid[kEmitChunk];
-    __shared__ uint2 s_rect[kEmitChunk];
-    __shared__ uint32_t wcount[kSortWarps][256];
-    __shared__ uint32_t gbase[256];    // global start of each digit's run from this block
-    __shared__ uint32_t lstart[256];   // start of each digit's run within the round
-    __shared__ uint32_t sk[kSortTile];
-    __shared__ uint32_t sv[kSortTile];
-    if (cnt.get() == 0) return;  // more instances than the capacity (or none): emit nothing
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    {
-        unsigned long long tot;
-        const unsigned long long ex = block_excl_scan(threadIdx.x < 256 ? digit_totals[threadIdx.x] : 0u, &tot);
-        if (threadIdx.x < 256) gbase[threadIdx.x] = uint32_t(ex) + hist[int64_t(threadIdx.x) * nb + blockIdx.x];
-    }
-    const uint32_t total = load_chunk(touched, rect, order, n, s_start, s_gid, s_rect);  // synchronises
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (uint32_t round = 0; round < total; round += kSortTile) {
-        for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&wcount[0][0])[k] = 0u;
-        __syncthreads();
-        const uint32_t base = round + uint32_t(warp) * kWarpSpan;
-        uint32_t key[kSortPerThread], val[kSortPerThread], rank[kSortPerThread];
-        // the thread's instances first (independent binary searches), then the votes
-#pragma unroll
-        for (int r = 0; r < kSortPerThread; ++r) {
-            const uint32_t slot = base + r * 32 + lane;
-            key[r] = 0u;
-            val[r] = 0u;
-            if (slot < total) slot_instance(s_start, s_gid, s_rect, slot, tiles_x, key[r], val[r]);
-        }
-#pragma unroll
-        for (int r = 0; r < kSortPerThread; ++r) {
-            const uint32_t slot = base + r * 32 + lane;
-            const bool in = slot < total;
-            const uint32_t digit = in ? (key[r] & 0xffu) : 256u;
-            uint32_t peers = __ballot_sync(0xffffffffu, in);
-            peers = in ? peers : ~peers;
-#pragma unroll
-            for (int bit = 0; bit < 8; ++bit) {
-                if (bit >= digit_bits) break;  // warp-uniform
-                const bool set = (digit >> bit) & 1u;
-                const uint32_t vb = __ballot_sync(0xffffffffu, set);
-                peers &= set ? vb : ~vb;
-            }
-            const uint32_t before = in ? wcount[warp][digit] : 0u;
-            __syncwarp();
-            if (in && (lane == __ffs(peers) - 1)) wcount[warp][digit] = before + __popc(peers);
-            __syncwarp();
-            rank[r] = before + __popc(peers & lt_mask);
-        }
-        __syncthreads();
-        uint32_t dtot = 0;
-        if (threadIdx.x < 256) {
-#pragma unroll
-            for (int w = 0; w < kSortWarps; ++w) {
-                const uint32_t c = wcount[w][threadIdx.x];
-                wcount[w][threadIdx.x] = dtot;
-                dtot += c;
-            }
-        }
-        {
-            unsigned long long tot;
-            const unsigned long long ex = block_excl_scan(dtot, &tot);  // synchronises
-            if (threadIdx.x < 256) lstart[threadIdx.x] = uint32_t(ex);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int r = 0; r < kSortPerThread; ++r) {
-            if (base + r * 32 + lane < total) {
-                const uint32_t digit = key[r] & 0xffu;
-                const uint32_t p = lstart[digit] + wcount[warp][digit] + rank[r];
-                sk[p] = key[r];
-                sv[p] = val[r];
-            }
-        }
-        __syncthreads();
-        const int in_round = int(min(uint32_t(kSortTile), total - round));
-        scatter_runs<kFinal>(sk, sv, in_round, 0, gbase, lstart, depth, keys_out, keys_out64, vals_out);
-        __syncthreads();
-        if (threadIdx.x < 256) gbase[threadIdx.x] += dtot;  // the next round continues every run
+        for (int step = kEmitChunk / 2; step > 0; step >>= 1)
+            if (s_start[lo + step] <= slot) lo += step;
+        const uint32_t j = slot - s_start[lo];
+        const uint2 r = s_rect[lo];
+        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, w = (r.y & 0xffffu) - x0;
+        const uint32_t ty = y0 + j / w, tx = x0 + j % w;
+        tkeys[base + slot] = ty * uint32_t(tiles_x) + tx;
+        tvals[base + slot] = s_gid[lo];
     }
 }
 
@@ -552,11 +417,8 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
         w.tval[r] = reinterpret_cast<uint32_t*>(b + off);
         off += align_up(sizeof(uint32_t) * size_t(slots > 0 ? slots : 1));
     }
-    // the histograms of the radix passes (nb_sort blocks) and of the fused first
-    // pass (one per emit block)
-    const int64_t nb_hist = nb_sort > nb_emit ? nb_sort : nb_emit;
     w.hist = reinterpret_cast<uint32_t*>(b + off);
-    off += align_up(sizeof(uint32_t) * 256 * size_t(nb_hist > 0 ? nb_hist : 1));
+    off += align_up(sizeof(uint32_t) * 256 * size_t(nb_sort > 0 ? nb_sort : 1));
     w.digit_totals = reinterpret_cast<uint32_t*>(b + off);
     off += align_up(sizeof(uint32_t) * 256);
     if (ws) *ws = w;
@@ -636,31 +498,19 @@ cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const u
         if (e == cudaSuccess && count_out) e = cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), s);
         return e;
     }
+    count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, order, n, ws.block_sums);
+    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total, count_out);
+    count_launches(2);
+    // instances: launched for the capacity, K read on the device
+    const Count inst{0, ws.total, capacity};
+    emit_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, reinterpret_cast<const uint2*>(proj.rect),
+                                                            order, n, cam.TX, ws.block_sums, inst, ws.tkey[0],
+                                                            ws.tval[0]);
+    count_launches(1);
     const int bits = tile_bits(T);
     const int passes = bits > 0 ? (bits + 7) / 8 : 1;
-    const uint2* rect = reinterpret_cast<const uint2*>(proj.rect);
-    // the first pass over the tile id (its low 8 bits) is fused into the emission:
-    // per-block digit histograms and instance counts, K, the scanned histograms,
-    // then the ranked emission into buffer 0 (or the final keys)
-    count_digits_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, rect, order, n, cam.TX,
-                                                                     ws.hist, ws.nb_emit, ws.block_sums);
-    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total, count_out);
-    scan_hist_kernel<<<dim3(256, 1), 1024, 0, s>>>(ws.hist, ws.nb_emit, ws.digit_totals);
-    count_launches(3);
-    const Count inst{0, ws.total, capacity};
-    const int first_bits = passes == 1 ? bits : 8;
-    if (passes == 1)
-        emit_ranked_kernel<true><<<unsigned(ws.nb_emit), kSortBlock, 0, s>>>(
-            proj.tiles_touched, rect, order, n, cam.TX, ws.hist, ws.nb_emit, ws.digit_totals, first_bits, inst,
-            nullptr, keys, vals, proj.depth);
-    else
-        emit_ranked_kernel<false><<<unsigned(ws.nb_emit), kSortBlock, 0, s>>>(
-            proj.tiles_touched, rect, order, n, cam.TX, ws.hist, ws.nb_emit, ws.digit_totals, first_bits, inst,
-            ws.tkey[0], nullptr, ws.tval[0], proj.depth);
-    count_launches(1);
-    // the remaining passes over the higher tile bits
     int cur = 0;
-    for (int p = 1; p < passes; ++p) {
+    for (int p = 0; p < passes; ++p) {
         const bool last = p == passes - 1;
         radix_pass(ws.tkey[cur], ws.tval[cur], last ? nullptr : ws.tkey[cur ^ 1], last ? keys : nullptr,
                    last ? vals : ws.tval[cur ^ 1], inst, capacity, 8 * p, ws.hist, ws.digit_totals, proj.depth, s,
