@@ -324,6 +324,8 @@ def gs_project_bwd(params: gs_params, cam: gs_camera, proj: gs_projected, grad2d
 
 
 GS_MAX_VIEWS = 16
+# views up to which the fused backward runs the chain and Adam in one kernel (grads optional)
+GS_ADAM_ONE_PASS_MAX_VIEWS = 2
 
 
 def _arr(ctype, items):

@@ -538,6 +538,9 @@ gs_status project_bwd_adam_common(const char* fn, const gs_params* params, int32
         a.lr[g] = lr_host[g];
     }
     if (!params_inout || !adam_m || !adam_v) return fail(GS_ERR_INVALID_ARG, "%s: Adam arrays are NULL", fn);
+    if (!grads && num_views > GS_ADAM_ONE_PASS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: grads is NULL (required for more than %d views: the gradient passes "
+                    "through it to the Adam step)", fn, GS_ADAM_ONE_PASS_MAX_VIEWS);
     if (params && (params_inout->means != params->means || params_inout->sh != params->sh))
         return fail(GS_ERR_INVALID_ARG, "%s: params_inout must be the arrays of params", fn);
     a.params = params_inout;

@@ -366,6 +366,20 @@ def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: d
                     lrs[name], betas[0], betas[1], eps, step, s)
 
 
+def _grad_buffer(g: Gaussians, grads: Gaussians, nviews: int):
+    """The gradient buffer of a backward + Adam call: the caller's; else, for more views than
+    the one-kernel form takes (the step then passes its gradient through the buffer), one kept
+    beside the Gaussians; else none."""
+    if grads is not None:
+        return grads.grads()
+    if nviews <= abi.GS_ADAM_ONE_PASS_MAX_VIEWS:
+        return None
+    buf = getattr(g, "_step_grads", None)
+    if buf is None or buf.n != g.n or buf.sh_degree != g.sh_degree or buf.means.device != g.means.device:
+        buf = g._step_grads = g.zeros_like()
+    return buf.grads()
+
+
 def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: torch.Tensor, grad2ds: list,
                            m: Gaussians, v: Gaussians, lrs: dict, step: int, grads: Gaussians = None,
                            densify_accum: torch.Tensor = None, densify_count: torch.Tensor = None,
@@ -377,7 +391,7 @@ def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: to
     abi.gs_project_bwd_views_adam(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES],
-        betas[0], betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum),
+        betas[0], betas[1], eps, step, _grad_buffer(g, grads, len(views)), _ptr(densify_accum),
         _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -391,7 +405,7 @@ def project_bwd_views_adam_sh16(g: Gaussians, sh_half: torch.Tensor, views: list
     abi.gs_project_bwd_views_adam_sh16(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], _ptr(sh_half), _ptr(sh_half), g.grads(), m.grads(), v.grads(),
-        [lrs[k] for k in PARAM_NAMES], betas[0], betas[1], eps, step, grads.grads() if grads is not None else None,
+        [lrs[k] for k in PARAM_NAMES], betas[0], betas[1], eps, step, _grad_buffer(g, grads, len(views)),
         _ptr(densify_accum), _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -403,7 +417,7 @@ def project_bwd_views_adam_packed(g: Gaussians, views: list, packs: list, grad2d
     abi.gs_project_bwd_views_adam_packed(
         g.params(), [vw.gcam for vw in views], [pk.proj.struct() for pk in packs], [_ptr(pk.slot_of) for pk in packs],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES], betas[0],
-        betas[1], eps, step, grads.grads() if grads is not None else None, _ptr(densify_accum), _ptr(densify_count),
+        betas[1], eps, step, _grad_buffer(g, grads, len(views)), _ptr(densify_accum), _ptr(densify_count),
         _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -521,7 +535,9 @@ class Trainer:
             self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
             self.grad2d = self.grad2ds[0]
             self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
-        self.grads = None if self.fused else self.gauss.zeros_like()
+        # the unfused path accumulates into it; the fused step with more views than the
+        # one-kernel form takes passes its gradient through it to the Adam launch
+        self.grads = self.gauss.zeros_like() if (not self.fused or nv > abi.GS_ADAM_ONE_PASS_MAX_VIEWS) else None
         self.sh_half = to_half(self.gauss.sh) if self.sh16 else None
         self.densify_accum = torch.zeros((max(n, 1),), device=dev, dtype=torch.float32) if self.densify else None
         self.densify_count = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None
@@ -750,7 +766,7 @@ class Trainer:
         self.step_count += 1
         if self.packed:
             project_bwd_views_adam_packed(self.gauss, self.views, self.packs, self.grad2ds, self.m, self.v, self.lrs,
-                                          self.step_count, None, self.densify_accum, self.densify_count,
+                                          self.step_count, self.grads, self.densify_accum, self.densify_count,
                                           densify_max_radius=self.densify_max_radius, sparse=self.sparse_grad)
             # far more slots than Gaussians kept (the first step starts with n): fewer slots from
             # the next step on
@@ -758,12 +774,12 @@ class Trainer:
                 self._alloc_packed(min(self.gauss.n, int(max(visible) * 1.25) + 1024))
         elif self.sh16:
             project_bwd_views_adam_sh16(self.gauss, self.sh_half, self.views, self.proj, self.radii, self.grad2ds,
-                                        self.m, self.v, self.lrs, self.step_count, None, self.densify_accum,
+                                        self.m, self.v, self.lrs, self.step_count, self.grads, self.densify_accum,
                                         self.densify_count, densify_max_radius=self.densify_max_radius,
                                         sparse=self.sparse_grad)
         elif self.fused:
             project_bwd_views_adam(self.gauss, self.views, self.proj, self.radii, self.grad2ds, self.m, self.v,
-                                   self.lrs, self.step_count, None, self.densify_accum, self.densify_count,
+                                   self.lrs, self.step_count, self.grads, self.densify_accum, self.densify_count,
                                    densify_max_radius=self.densify_max_radius, sparse=self.sparse_grad)
         else:
             adam_step(self.gauss, self.grads, self.m, self.v, self.lrs, self.step_count)

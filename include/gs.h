@@ -321,17 +321,27 @@ gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const
                                void* stream);
 
 /* gs_project_bwd_views_adam -- gs_project_bwd_views followed by the Adam step of
- * gs_adam for all five parameter groups in the same pass (gsplat guide §4.2:
- * lr_host[5] for means, quats, log_scales, opacity_logits, sh; shared betas,
- * eps and step).  params_inout holds the same arrays as params and is updated
- * in place; adam_m and adam_v are the first and second moments in the
- * parameter layout.  The summed gradient goes straight into Adam; grads, when
- * non-NULL, also receives it (+=).  With sparse_adam = 0 every Gaussian is
- * updated, visible or not, as gs_adam updates every element.  With
- * sparse_adam = 1 (the sparse_grad option of the gsplat guide §4.1) a Gaussian
- * visible in none of the views keeps its parameters and moments unchanged (no
- * decay of the moments), as a sparse Adam skips absent rows; the bias
- * correction still uses `step`. */
+ * gs_adam for all five parameter groups (gsplat guide §4.2: lr_host[5] for
+ * means, quats, log_scales, opacity_logits, sh; shared betas, eps and step).
+ * params_inout holds the same arrays as params and is updated in place; adam_m
+ * and adam_v are the first and second moments in the parameter layout.
+ *
+ * grads receives the step's summed gradient, written over (not added to): zero
+ * for a Gaussian visible in none of the views, and the w lane of each means
+ * entry holds the number of views in which the Gaussian is visible.  With up to
+ * GS_ADAM_ONE_PASS_MAX_VIEWS views the chain and the Adam step run as one kernel
+ * and grads may be NULL; with more views they are two launches (the chain, then
+ * one Adam launch over all five groups) that pass the gradient through grads,
+ * which is then required and must not overlap params, adam_m or adam_v.
+ *
+ * With sparse_adam = 0 every Gaussian is updated, visible or not, as gs_adam
+ * updates every element.  With sparse_adam = 1 (the sparse_grad option of the
+ * gsplat guide §4.1) a Gaussian visible in none of the views keeps its
+ * parameters and moments unchanged (no decay of the moments), as a sparse Adam
+ * skips absent rows; the bias correction still uses `step`.  Errors (nothing
+ * launched): those of gs_project_bwd_views, and GS_ERR_INVALID_ARG for grads
+ * NULL with more than GS_ADAM_ONE_PASS_MAX_VIEWS views. */
+#define GS_ADAM_ONE_PASS_MAX_VIEWS 2
 gs_status gs_project_bwd_views_adam(const gs_params* params, int32_t num_views, const gs_camera* cams,
                                     const gs_projected* projs, const gs_grad2d* grad2d, gs_param_grads* params_inout,
                                     gs_param_grads* adam_m, gs_param_grads* adam_v, const float* lr_host,

@@ -149,6 +149,11 @@ def test_invalid_arguments_rejected_before_launch(gs):
     assert L.gs_project_bwd_views_adam(C.byref(p), 1, C.byref(c), C.byref(proj), C.byref(g2), C.byref(gr),
                                        C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1, None, None, None, None, 2,
                                        None) == gs.GS_ERR_INVALID_ARG
+    # more views than the one-kernel form takes: the gradient buffer is required
+    assert L.gs_project_bwd_views_adam(C.byref(p), gs.GS_ADAM_ONE_PASS_MAX_VIEWS + 1, C.byref(c), C.byref(proj),
+                                       C.byref(g2), C.byref(gr), C.byref(gr), C.byref(gr), lr, 0.9, 0.99, 1e-15, 1,
+                                       None, None, None, None, 0, None) == gs.GS_ERR_INVALID_ARG
+    assert "grads" in gs.gs_last_error_detail()
     # packed projection: workspace size, capacity, the visible counter and the slot map
     wsp = gs.gs_project_packed_workspace_bytes(10)
     assert wsp >= 60 * 10
@@ -272,3 +277,11 @@ def test_counted_raster_calls_check_their_counter(gs):
     assert st == gs.GS_ERR_INVALID_ARG and "counts" in L.gs_last_error_detail().decode()
     st = L.gs_raster_bwd_counted(C.byref(proj), None, None, None, C.byref(c), bg, None, None, None, None, None, None)
     assert st == gs.GS_ERR_INVALID_ARG and "counts" in L.gs_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("name", ["GS_MAX_VIEWS", "GS_ADAM_ONE_PASS_MAX_VIEWS"])
+def test_view_limits_match_the_header(gs, name):
+    """The binding's view limits are the header's #defines, not stale copies."""
+    m = re.search(r"#define\s+%s\s+(\d+)\b" % name, open(HEADER).read())
+    assert m, f"{name} not found in gs.h"
+    assert int(m.group(1)) == getattr(gs, name)
