@@ -46,6 +46,12 @@ static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halv
 #ifndef GS_SORT_ITEMS
 #define GS_SORT_ITEMS 8
 #endif
+// downsweep blocks per SM the register budget is cut for (48 registers, no spill
+// to speak of: 80 registers held it to 3 blocks; 16 views of 10M instances at
+// 1080p 6.82 -> 5.83 ms of binning, 8 blocks with spills 6.72 ms)
+#ifndef GS_SORT_MIN_BLOCKS
+#define GS_SORT_MIN_BLOCKS 5
+#endif
 constexpr int kSortBlock = 256;
 constexpr int kSortWarps = kSortBlock / 32;
 constexpr int kSortPerThread = GS_SORT_ITEMS;
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t
 // digit_bits: how many of the digit's 8 bits can be set (the last pass over the
 // tile bits has fewer); the rank votes only on those.
 template <bool kFinal>
-__global__ void __launch_bounds__(kSortBlock) downsweep_kernel(const uint32_t* __restrict__ keys_in,
+__global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kernel(const uint32_t* __restrict__ keys_in,
                                                                const uint32_t* __restrict__ vals_in,
                                                                uint32_t* __restrict__ keys_out,
                                                                uint64_t* __restrict__ keys_out64,
