@@ -565,14 +565,14 @@ def measure_variants(tr, torch, reps: int = 10):
     res = {"raster_bwd_ms": timed(lambda: pl.raster_bwd(tr.proj, view, plain, tr.bg, radius=r)),
            "raster_bwd_absgrad_ms": timed(lambda: pl.raster_bwd(tr.proj, view, absg, tr.bg, radius=r))}
     # the fused backward with Adam on copies of the parameters and moments
-    g, m, v = (x.zeros_like() for x in (tr.gauss, tr.gauss, tr.gauss))
+    g, m, v, gbuf = (x.zeros_like() for x in (tr.gauss, tr.gauss, tr.gauss, tr.gauss))
     for dst, src in ((g, tr.gauss), (m, tr.m), (v, tr.v)):
         for a, b in zip(dst.tensors().values(), src.tensors().values()):
             a.copy_(b)
     for sparse in (False, True):
         res["project_bwd_adam_sparse_ms" if sparse else "project_bwd_adam_ms"] = timed(
             lambda: pl.project_bwd_views_adam(g, tr.views, tr.proj, tr.radii, tr.grad2ds, m, v, tr.lrs,
-                                              tr.step_count + 1, sparse=sparse))
+                                              tr.step_count + 1, gbuf, sparse=sparse))
     res["visible_fraction"] = float((tr.radii > 0).any(dim=0).float().mean().item())
     return res
 
@@ -985,7 +985,7 @@ def stage_breakdown(tr, pl, torch):
         timed("raster_bwd", pl.raster_bwd, proj, view, g2, tr.bg, None, r)
     tr.step_count += 1
     timed("project_bwd_adam", pl.project_bwd_views_adam, tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m,
-          tr.v, tr.lrs, tr.step_count, None, tr.densify_accum, tr.densify_count,
+          tr.v, tr.lrs, tr.step_count, tr.grads, tr.densify_accum, tr.densify_count,
           densify_max_radius=tr.densify_max_radius)
     torch.cuda.synchronize()
     return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in acc.items()}
@@ -1131,7 +1131,7 @@ def run_e2e(tr, targets_host, targets, args, world, torch):
             raise RuntimeError("instance buffers overflowed after the warm-up")
         tr.step_count += 1
         pl.project_bwd_views_adam(tr.gauss, tr.views, tr.proj, tr.radii, tr.grad2ds, tr.m, tr.v, tr.lrs,
-                                  tr.step_count, None, tr.densify_accum, tr.densify_count,
+                                  tr.step_count, tr.grads, tr.densify_accum, tr.densify_count,
                                   densify_max_radius=tr.densify_max_radius)
         loss_host.copy_(tr.loss, non_blocking=True)
 

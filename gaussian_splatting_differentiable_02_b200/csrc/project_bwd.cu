@@ -13,11 +13,13 @@
 //   * one or two views: one thread per Gaussian, the views in a loop, the 48 SH
 //     sums in a second pass over the visible views (their masked colour
 //     gradients kept in shared memory) so that they never share registers with
-//     the geometric chain; with Adam fused in, the gradients never reach memory;
+//     the geometric chain; with Adam and no gradient buffer, the step runs in the
+//     same thread and the gradients never reach memory (0.675 ms for 1M Gaussians
+//     seen by one view), with a buffer it is the second launch below (0.569 ms);
 //   * three to 16 views: one thread per Gaussian, the views in a loop, the 48 SH
 //     sums in shared memory; with Adam, the summed gradient is written to the
-//     caller's gradient buffer and the Adam step of all five groups follows as a
-//     second, streaming launch.  Fused into the chain, the step's 15 float4
+//     caller's gradient buffer (required here) and the Adam step of all five
+//     groups follows as a second, streaming launch.  Fused into the chain, the step's 15 float4
 //     read-modify-writes per Gaussian ran one memory round trip after another in
 //     a kernel held to 12 warps per SM by its registers (2.06 ms for 16 views of
 //     1M Gaussians); apart, the chain takes 1.2 ms and the step 0.3 ms at 82% of
@@ -887,7 +889,8 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
     const bool half = adam && adam->sh_half;
     // the Adam calls' gradient buffer receives the step's gradient (written over)
     a.overwrite = adam != nullptr;
-    if (V <= kSplitMaxViews) {
+    if (V <= kSplitMaxViews && !(adam && grads)) {
+        // no views loop to speak of, and (with Adam) no buffer: the step in the same kernel
         const unsigned grid = grid_for(p.n, kBwdBlock, 16);
         dispatch_flags(adam != nullptr, slots != nullptr, half, [&](auto ad, auto pk, auto hf) {
             project_bwd_split_kernel<decltype(ad)::value, decltype(pk)::value, decltype(hf)::value>
@@ -896,8 +899,16 @@ cudaError_t launch_project_bwd_views(const gs_params& p, int V, const CamArgs* c
         count_launches(1);
         return cudaGetLastError();
     }
+    // the gradient into the buffer, then the Adam launch
     const unsigned grid = grid_for(p.n, kBwdBlock, 16);
-    if (slots)
+    if (V <= kSplitMaxViews) {
+        if (slots)
+            project_bwd_split_kernel<false, true, false><<<grid, kBwdBlock, 0, s>>>(a);
+        else if (half)
+            project_bwd_split_kernel<false, false, true><<<grid, kBwdBlock, 0, s>>>(a);
+        else
+            project_bwd_split_kernel<false, false, false><<<grid, kBwdBlock, 0, s>>>(a);
+    } else if (slots)
         project_bwd_loop_kernel<true, false><<<grid, kBwdBlock, 0, s>>>(a);
     else if (half)
         project_bwd_loop_kernel<false, true><<<grid, kBwdBlock, 0, s>>>(a);

@@ -366,14 +366,11 @@ def adam_step(g: Gaussians, grads: Gaussians, m: Gaussians, v: Gaussians, lrs: d
                     lrs[name], betas[0], betas[1], eps, step, s)
 
 
-def _grad_buffer(g: Gaussians, grads: Gaussians, nviews: int):
-    """The gradient buffer of a backward + Adam call: the caller's; else, for more views than
-    the one-kernel form takes (the step then passes its gradient through the buffer), one kept
-    beside the Gaussians; else none."""
+def _grad_buffer(g: Gaussians, grads: Gaussians):
+    """The gradient buffer of a backward + Adam call (the chain passes the step's gradient
+    through it to the Adam launch): the caller's, else one kept beside the Gaussians."""
     if grads is not None:
         return grads.grads()
-    if nviews <= abi.GS_ADAM_ONE_PASS_MAX_VIEWS:
-        return None
     buf = getattr(g, "_step_grads", None)
     if buf is None or buf.n != g.n or buf.sh_degree != g.sh_degree or buf.means.device != g.means.device:
         buf = g._step_grads = g.zeros_like()
@@ -391,7 +388,7 @@ def project_bwd_views_adam(g: Gaussians, views: list, proj: Projected, radii: to
     abi.gs_project_bwd_views_adam(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES],
-        betas[0], betas[1], eps, step, _grad_buffer(g, grads, len(views)), _ptr(densify_accum),
+        betas[0], betas[1], eps, step, _grad_buffer(g, grads), _ptr(densify_accum),
         _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -405,7 +402,7 @@ def project_bwd_views_adam_sh16(g: Gaussians, sh_half: torch.Tensor, views: list
     abi.gs_project_bwd_views_adam_sh16(
         g.params(), [vw.gcam for vw in views], [proj.struct(radii[k]) for k in range(len(views))],
         [gd.struct() for gd in grad2ds], _ptr(sh_half), _ptr(sh_half), g.grads(), m.grads(), v.grads(),
-        [lrs[k] for k in PARAM_NAMES], betas[0], betas[1], eps, step, _grad_buffer(g, grads, len(views)),
+        [lrs[k] for k in PARAM_NAMES], betas[0], betas[1], eps, step, _grad_buffer(g, grads),
         _ptr(densify_accum), _ptr(densify_count), _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -417,7 +414,7 @@ def project_bwd_views_adam_packed(g: Gaussians, views: list, packs: list, grad2d
     abi.gs_project_bwd_views_adam_packed(
         g.params(), [vw.gcam for vw in views], [pk.proj.struct() for pk in packs], [_ptr(pk.slot_of) for pk in packs],
         [gd.struct() for gd in grad2ds], g.grads(), m.grads(), v.grads(), [lrs[k] for k in PARAM_NAMES], betas[0],
-        betas[1], eps, step, _grad_buffer(g, grads, len(views)), _ptr(densify_accum), _ptr(densify_count),
+        betas[1], eps, step, _grad_buffer(g, grads), _ptr(densify_accum), _ptr(densify_count),
         _ptr(densify_max_radius), int(sparse), _stream())
 
 
@@ -535,9 +532,9 @@ class Trainer:
             self.grad2ds = [Grad2D(n, dev, absgrad=self.absgrad) for _ in range(nv)]
             self.grad2d = self.grad2ds[0]
             self.radii = torch.zeros((nv, max(n, 1)), device=dev, dtype=torch.int32)
-        # the unfused path accumulates into it; the fused step with more views than the
-        # one-kernel form takes passes its gradient through it to the Adam launch
-        self.grads = self.gauss.zeros_like() if (not self.fused or nv > abi.GS_ADAM_ONE_PASS_MAX_VIEWS) else None
+        # the unfused path accumulates into it; the fused step passes its gradient through
+        # it to the Adam launch
+        self.grads = self.gauss.zeros_like()
         self.sh_half = to_half(self.gauss.sh) if self.sh16 else None
         self.densify_accum = torch.zeros((max(n, 1),), device=dev, dtype=torch.float32) if self.densify else None
         self.densify_count = torch.zeros((max(n, 1),), device=dev, dtype=torch.int32) if self.densify else None

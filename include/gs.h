@@ -24,7 +24,8 @@
  *     outside 1..16384 returns GS_ERR_UNSUPPORTED.  A CUDA launch or copy error
  *     returns GS_ERR_CUDA.  No kernel traps or asserts.
  *   - Gradient outputs are accumulated (+=): callers zero them, and several views
- *     can add into the same buffers.
+ *     can add into the same buffers.  (The backward calls with Adam are the
+ *     exception: their gradient buffer receives the step's gradient, written over.)
  *   - Arrays are structure-of-arrays, read with 128-bit loads: an array written
  *     "[n][4]" is n consecutive float4 records (16-byte aligned).
  *   - n (Gaussians) up to 2^31 - 1; instance counts up to 2^32 - 1; tiles up to 2^20.
@@ -328,11 +329,13 @@ gs_status gs_project_bwd_views(const gs_params* params, int32_t num_views, const
  *
  * grads receives the step's summed gradient, written over (not added to): zero
  * for a Gaussian visible in none of the views, and the w lane of each means
- * entry holds the number of views in which the Gaussian is visible.  With up to
- * GS_ADAM_ONE_PASS_MAX_VIEWS views the chain and the Adam step run as one kernel
- * and grads may be NULL; with more views they are two launches (the chain, then
- * one Adam launch over all five groups) that pass the gradient through grads,
- * which is then required and must not overlap params, adam_m or adam_v.
+ * entry holds the number of views in which the Gaussian is visible.  With grads
+ * the chain and the Adam step are two launches (the chain, then one Adam launch
+ * over all five groups) that pass the gradient through it; grads must not overlap
+ * params, adam_m or adam_v.  grads may be NULL with up to
+ * GS_ADAM_ONE_PASS_MAX_VIEWS views: the chain and the step then run as one
+ * kernel and the gradient never reaches memory (slower: the step's memory round
+ * trips wait on the chain's).
  *
  * With sparse_adam = 0 every Gaussian is updated, visible or not, as gs_adam
  * updates every element.  With sparse_adam = 1 (the sparse_grad option of the

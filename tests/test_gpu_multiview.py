@@ -303,3 +303,49 @@ def test_batched_depth_order_matches_the_per_view_sort(orc):
         z = projs[k].depth.cpu().numpy().view(np.uint32).astype(np.uint64)
         keyz = np.where(r > 0, z, 0xFFFFFFFF)
         assert np.array_equal(order, np.lexsort((np.arange(scene.n), keyz)).astype(np.uint32))
+
+
+@pytest.mark.parametrize("n_views,sparse", [(1, 0), (2, 1), (2, 0)])
+def test_one_kernel_step_equals_two_launches(orc, n_views, sparse):
+    """With one or two views and no gradient buffer the chain and the Adam step run in one
+    kernel; with a buffer, as two launches (the chain writes the gradient, one Adam launch
+    reads it).  Same inputs, same float32 gradient, same Adam arithmetic: parameters,
+    moments and densification statistics identical bit for bit, and the buffer holds the
+    gradient the multi-view chain gives (written over, not added to)."""
+    scene, cams, g0, proj, radii, views, g2s, want, acc, cnt = _setup(orc, n_views=n_views, deg=3, seed=21)
+    rng = np.random.default_rng(4)
+    init = {k: (0.01 * rng.random(tuple(getattr(g0, k).shape))).astype(np.float32) for k in NAMES}
+    lrs = [float(np.float32(LRS[k])) for k in NAMES]
+    out = []
+    for with_buffer in (False, True):
+        g = g0.zeros_like()
+        for k in NAMES:
+            getattr(g, k).copy_(getattr(g0, k))
+        m, v = g.zeros_like(), g.zeros_like()
+        for k in NAMES:
+            getattr(m, k).copy_(torch.from_numpy(init[k]))
+            getattr(v, k).copy_(torch.from_numpy(init[k] * 0.5))
+        grads = g.zeros_like()
+        for t in grads.tensors().values():
+            t.fill_(7.0)  # written over, so the fill must not survive
+        da = torch.zeros(scene.n, device="cuda")
+        dc = torch.zeros(scene.n, dtype=torch.int32, device="cuda")
+        abi.gs_project_bwd_views_adam(g.params(), [vw.gcam for vw in views],
+                                      [proj.struct(radii[k]) for k in range(n_views)], [x.struct() for x in g2s],
+                                      g.grads(), m.grads(), v.grads(), lrs, 0.9, 0.99, 1e-15, 2,
+                                      grads=grads.grads() if with_buffer else None, densify_accum=da.data_ptr(),
+                                      densify_count=dc.data_ptr(), sparse_adam=sparse,
+                                      stream=torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        out.append((g, m, v, grads, da.cpu().numpy(), dc.cpu().numpy()))
+    (ga, ma, va, _, daa, dca), (gb, mb, vb, grads, dab, dcb) = out
+    for k in NAMES:
+        for x, y in ((ga, gb), (ma, mb), (va, vb)):
+            assert torch.equal(getattr(x, k), getattr(y, k)), k
+    assert np.array_equal(daa, dab) and np.array_equal(dca, dcb)
+    # the buffer: the summed gradient, and the visible-view count in the means' w lane
+    got = grads.to_numpy()
+    vis = np.nonzero(cnt > 0)[0]
+    for k in NAMES:
+        check_grads(got[k].reshape(scene.n, -1), np.asarray(want[k]).reshape(scene.n, -1), k, rows=vis)
+    assert np.array_equal(grads.means[:, 3].cpu().numpy(), cnt.astype(np.float32))
