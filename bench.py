@@ -305,6 +305,29 @@ def cpu_oracle_render_sample(wl, fraction: float, seed: int = 0):
     return per_frame, threads, desc
 
 
+def measure_graph_frames(run_poses, poses, torch, stream, reps: int = 5):
+    """Every pose rendered once, eagerly and replayed from a CUDA graph captured from the
+    same calls (the poses' cameras are kernel arguments, fixed in the graph), ms per frame
+    with CUDA events over `reps` rounds each."""
+    def timed(fn):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * poses)
+    eager = timed(run_poses)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_poses()
+    graph.replay()
+    graphed = timed(graph.replay)
+    return {"ms_per_frame_eager": eager, "ms_per_frame_graph": graphed, "speedup": eager / graphed,
+            "frames_per_s_graph": 1e3 / graphed}
+
+
 def run_render(args, world, rank, local):
     """Forward-only workloads (the 100k box at 1080p over 100 poses, the 3M city at
     4K over 50 poses): one step renders every pose once (projection, binning,
@@ -379,6 +402,10 @@ def run_render(args, world, rank, local):
     last_ms = fwd_ev[-1][0].elapsed_time(fwd_ev[-1][1])
     roof = raster_roofline("raster_fwd", last_ms, work, alu)
     cam0 = cams[0]
+    graph_row = None
+    if not args.no_rows:
+        graph_row = measure_graph_frames(lambda: [frame(k, cam, False) for k, cam in enumerate(cams)], len(cams),
+                                         torch, stream)
     line = {"metric": RENDER_METRIC, "value": world * frames / (ms / 1e3), "unit": "frames/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -390,6 +417,8 @@ def run_render(args, world, rank, local):
             "roofline": roof, "raster_work_last_pose": work, "alu_peaks": alu,
             "gpu_launches": int(launches), "clocks": clk,
             "e2e": None, "hbm_peak_gbs": peaks["hbm_gbs"]}
+    if graph_row is not None:
+        line["rows"] = {"cuda_graph": graph_row}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cpu_oracle_render_sample, wl, args.cpu_fraction, "frames/s")
     if rank == 0:
@@ -521,7 +550,8 @@ def run_ours(args, world, rank, local):
     # rows outside the per-step path, measured after the step timing
     with_oracle = rank == 0 and not args.no_cpu_baseline and world == 1
     if not args.no_rows:
-        line["rows"] = {"densify": measure_densify(tr, wl, peaks, torch, with_oracle),
+        line["rows"] = {"cuda_graph": measure_graph_steps(tr, torch, abi),
+                        "densify": measure_densify(tr, wl, peaks, torch, with_oracle),
                         "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
                         "absgrad_and_sparse_adam": measure_variants(tr, torch),
                         "packed": measure_packed(tr, wl, peaks, torch),
@@ -536,6 +566,39 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_graph_steps(tr, torch, abi, steps: int = 10):
+    """The step with the views' part replayed from a CUDA graph (Trainer(graph=True)),
+    against the eager step, both timed with CUDA events over `steps` steps of the same
+    Trainer right after each other (the graph is captured in an untimed step first).
+    Kernel timing events cannot be captured into a graph, which is why the line's own
+    timing and roofline use the eager step."""
+    def timed():
+        torch.cuda.synchronize()
+        l0 = abi.gs_kernel_launches()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            tr.step()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps, (abi.gs_kernel_launches() - l0) / steps
+    tr.graph = False
+    tr.step()
+    eager_ms, eager_launches = timed()
+    tr.graph = True
+    l0 = abi.gs_kernel_launches()
+    tr.step()  # captures the views' part, then replays it
+    torch.cuda.synchronize()
+    captured = abi.gs_kernel_launches() - l0
+    graph_ms, host_launches = timed()
+    tr.graph = False
+    tr._graph = None
+    return {"step_ms_eager": eager_ms, "step_ms_graph": graph_ms, "speedup": eager_ms / graph_ms,
+            "library_launches_per_step": eager_launches,
+            "launches_per_step_from_the_graph": captured - host_launches,
+            "launches_per_step_from_the_host": host_launches}
 
 
 def measure_variants(tr, torch, reps: int = 10):

@@ -489,6 +489,11 @@ class Trainer:
                                # visible count seen
     sh16: bool = False         # fused unpacked path: the projections read a 16-bit (FP16) copy of the SH
                                # coefficients, which the fused Adam step refreshes from the float32 ones
+    graph: bool = False        # fused path: the views' part of a step (projections, sorts, compositing,
+                               # losses and their backward) is captured once into a CUDA graph and
+                               # replayed every step, so its few-microsecond launches cost no host time
+                               # and little device time between them; recaptured whenever a buffer it
+                               # uses is reallocated (instance or slot growth, densification)
 
     def __post_init__(self):
         n = self.gauss.n
@@ -512,6 +517,7 @@ class Trainer:
     def _alloc_per_gaussian(self, n: int):
         """Buffers sized by the Gaussian count (the projection, 2D gradients, visibility rows,
         gradients and densification statistics)."""
+        self._graph = None  # it holds the old buffers' addresses
         dev = self.gauss.means.device
         nv = len(self.views) if self.fused else 1
         if self.packed:
@@ -542,6 +548,7 @@ class Trainer:
 
     def _alloc_packed(self, capacity: int):
         """Packed views of `capacity` slots: features, 2D gradients, depth order and sort buffers."""
+        self._graph = None
         dev = self.gauss.means.device
         n, nv = self.gauss.n, len(self.views)
         self.pcap = int(capacity)
@@ -725,6 +732,21 @@ class Trainer:
             depth_order_views([self.projs[k] for k in ks], None if self.radii is None else [self.radii[k] for k in ks],
                               self.depth_orders[gi])
 
+    def _views_part(self) -> None:
+        abi.gs_zero(_ptr(self.loss), 8, _stream())
+        self._all_views()
+
+    def _replay_views(self) -> None:
+        """The views' part of the step from the CUDA graph, captured first when there is none."""
+        if getattr(self, "_graph", None) is None:
+            self.side_streams()  # the streams exist before the capture forks onto them
+            self.bin_stream()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                self._views_part()
+            self._graph = graph
+        self._graph.replay()
+
     def side_streams(self) -> list:
         """The streams the fused path runs views on."""
         if getattr(self, "_side", None) is None:
@@ -736,7 +758,10 @@ class Trainer:
         """forward + L1 + backward for every view, then one Adam step; loss stays on the device."""
         s = _stream()
         while True:
-            abi.gs_zero(_ptr(self.loss), 8, s)
+            if self.fused and self.graph:
+                self._replay_views()
+            else:
+                abi.gs_zero(_ptr(self.loss), 8, s)
             if not self.fused:
                 self.grads.zero_()
                 for k, tgt in enumerate(self.targets):
@@ -744,7 +769,8 @@ class Trainer:
                     project_bwd(self.gauss, self.views[k], self.proj, self.grad2d, self.grads, self.densify_accum,
                                 self.densify_count, radius=self.radii[0], densify_max_radius=self.densify_max_radius)
                 break
-            self._all_views()
+            if not self.graph:
+                self._all_views()
             # one wait per step: every view's instance count against its capacity (and in the
             # packed layout its visible count against the slot capacity)
             both = self.counts.cpu().tolist()
@@ -760,6 +786,7 @@ class Trainer:
                 break
             for k in over:  # grow and repeat the step's views (nothing was applied yet)
                 self.views[k]._alloc(int(counts[k] * 1.25) + 1024)
+                self._graph = None
         self.step_count += 1
         if self.packed:
             project_bwd_views_adam_packed(self.gauss, self.views, self.packs, self.grad2ds, self.m, self.v, self.lrs,

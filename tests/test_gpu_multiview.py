@@ -349,3 +349,43 @@ def test_one_kernel_step_equals_two_launches(orc, n_views, sparse):
     for k in NAMES:
         check_grads(got[k].reshape(scene.n, -1), np.asarray(want[k]).reshape(scene.n, -1), k, rows=vis)
     assert np.array_equal(grads.means[:, 3].cpu().numpy(), cnt.astype(np.float32))
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_graph_step_matches_eager(packed):
+    """Trainer(graph=True) replays the views' part of the step from a CUDA graph: the same
+    kernels on the same buffers as the eager step, so the same instance counts, the same
+    first loss up to the order of its double-precision atomic sums, and parameters equal
+    up to the order the gradient atomics happened to take.  The step is captured again
+    after the instance buffers grow (the first step starts with small ones) and after
+    densification reallocates everything."""
+    rng = np.random.default_rng(17)
+    scene = scenes.random_scene(rng, 600, 1, mean_box=1.0, log_scale=(-3.5, -2.0))
+    cams = _views(3, 6)
+    targets = [torch.from_numpy(rng.random((128, 128, 3)).astype(np.float32)).cuda() for _ in cams]
+    out = []
+    for graph in (False, True):
+        g = pl.Gaussians.from_scene(scene)
+        views = [pl.View(scene.n, c) for c in cams]
+        for vw in views:
+            vw._alloc(64)  # too small: the first step grows them
+        tr = pl.Trainer(g, views, targets, dict(LRS), densify=True, packed=packed, graph=graph)
+        losses, counts = [], []
+        for it in range(4):
+            tr.step()
+            torch.cuda.synchronize()
+            losses.append(tr.loss.item())
+            counts.append(tr.kcount.cpu().numpy().copy())
+            if it == 1:
+                tr.densify_and_prune(max_screen_size=0.0)  # no screen-size pruning: most Gaussians stay
+        out.append((tr.gauss.to_numpy(), losses, counts, tr.gauss.n))
+    (a, la, ca, na), (b, lb, cb, nb) = out
+    assert na == nb and na > 300
+    assert abs(la[0] - lb[0]) <= 1e-9 * max(1.0, abs(la[0]))
+    assert all(np.array_equal(x, y) for x, y in zip(ca[:2], cb[:2]))
+    np.testing.assert_allclose(la, lb, rtol=1e-5)
+    for k in NAMES:
+        d = np.abs(a[k] - b[k])
+        close = d <= 1e-6 + 1e-6 * np.abs(a[k])
+        assert close.mean() >= 0.999, (k, float(close.mean()))
+        assert d.max() <= 8 * LRS[k] + 1e-6, (k, float(d.max()))
