@@ -371,13 +371,25 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __rest
     }
 }
 
+// Four consecutive keys per thread: a tile starts at k when the key before k has
+// another tile, and ends after k when the key after k does.
 __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict__ keys, const Count cnt,
                                                      uint2* __restrict__ ranges) {
     const int64_t K = cnt.get();
-    for (int64_t k = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; k < K; k += int64_t(gridDim.x) * blockDim.x) {
-        const uint32_t t = uint32_t(__ldg(keys + k) >> 32);
-        if (k == 0 || uint32_t(__ldg(keys + k - 1) >> 32) != t) ranges[t].x = uint32_t(k);
-        if (k == K - 1 || uint32_t(__ldg(keys + k + 1) >> 32) != t) ranges[t].y = uint32_t(k + 1);
+    for (int64_t k0 = 4 * (blockIdx.x * int64_t(blockDim.x) + threadIdx.x); k0 < K;
+         k0 += 4 * int64_t(gridDim.x) * blockDim.x) {
+        uint32_t t[6];  // tiles of keys k0 - 1 .. k0 + 4 (0xffffffff past either end)
+#pragma unroll
+        for (int i = 0; i < 6; ++i) {
+            const int64_t k = k0 - 1 + i;
+            t[i] = k >= 0 && k < K ? uint32_t(__ldg(keys + k) >> 32) : 0xffffffffu;
+        }
+#pragma unroll
+        for (int i = 1; i < 5; ++i) {
+            if (k0 - 1 + i >= K) break;
+            if (t[i - 1] != t[i]) ranges[t[i]].x = uint32_t(k0 - 1 + i);
+            if (t[i + 1] != t[i]) ranges[t[i]].y = uint32_t(k0 + i);
+        }
     }
 }
 
