@@ -779,19 +779,36 @@ __global__ void __launch_bounds__(256) adam_groups_kernel(const __grid_constant_
         }
         return;
     }
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < count; i += stride) {
-        if (kSparse && __ldg(a.g[0] + (gr == 4 ? i % a.n : i)).w == 0.f) continue;
-        float4 pp = a.p[gr][i], mm = a.m[gr][i], vv = a.v[gr][i];
-        float4 gg = __ldg(a.g[gr] + i);
-        if (gr == 0) gg.w = 0.f;  // the means' w lane carries the visible-view count
-        pp.x = adam_scalar(pp.x, gg.x, mm.x, vv.x, lr_t, a);
-        pp.y = adam_scalar(pp.y, gg.y, mm.y, vv.y, lr_t, a);
-        pp.z = adam_scalar(pp.z, gg.z, mm.z, vv.z, lr_t, a);
-        pp.w = adam_scalar(pp.w, gg.w, mm.w, vv.w, lr_t, a);
-        a.p[gr][i] = pp;
-        a.m[gr][i] = mm;
-        a.v[gr][i] = vv;
-        if (kHalf && gr == 4) a.sh_half_out[i] = narrow(pp);
+    // two elements a thread per trip, every load before the first store: more bytes in
+    // flight per thread (one element a trip ran at 66-68% of the DRAM peak)
+    for (int64_t i0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i0 < count; i0 += 2 * stride) {
+        float4 pp[2], mm[2], vv[2], gg[2];
+        bool on[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t i = i0 + u * stride;
+            on[u] = i < count && !(kSparse && __ldg(a.g[0] + (gr == 4 ? i % a.n : i)).w == 0.f);
+            if (on[u]) {
+                pp[u] = a.p[gr][i];
+                mm[u] = a.m[gr][i];
+                vv[u] = a.v[gr][i];
+                gg[u] = __ldg(a.g[gr] + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (!on[u]) continue;
+            const int64_t i = i0 + u * stride;
+            if (gr == 0) gg[u].w = 0.f;  // the means' w lane carries the visible-view count
+            pp[u].x = adam_scalar(pp[u].x, gg[u].x, mm[u].x, vv[u].x, lr_t, a);
+            pp[u].y = adam_scalar(pp[u].y, gg[u].y, mm[u].y, vv[u].y, lr_t, a);
+            pp[u].z = adam_scalar(pp[u].z, gg[u].z, mm[u].z, vv[u].z, lr_t, a);
+            pp[u].w = adam_scalar(pp[u].w, gg[u].w, mm[u].w, vv[u].w, lr_t, a);
+            a.p[gr][i] = pp[u];
+            a.m[gr][i] = mm[u];
+            a.v[gr][i] = vv[u];
+            if (kHalf && gr == 4) a.sh_half_out[i] = narrow(pp[u]);
+        }
     }
 }
 
