@@ -446,7 +446,7 @@ def run_ours(args, world, rank, local):
     lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
                                                   "opacity_logits": 5e-2, "sh": 2.5e-3}
     tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams,
-                    batched_sort=not args.per_view_sort, groups=args.groups)
+                    batched_sort=not args.per_view_sort, groups=args.groups, bin_views=not args.per_view_bin)
     stream = torch.cuda.current_stream()
 
     # warm-up (also sizes every view's instance buffers)
@@ -529,6 +529,8 @@ def run_ours(args, world, rank, local):
             "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
                        "depth_sort": "per view" if args.per_view_sort else "batched over the views" + (
                            f", in {len(tr.view_groups())} pipelined view groups" if len(tr.view_groups()) > 1 else ""),
+                       "binning": "per view" if (args.per_view_bin or args.per_view_sort) else
+                                  "one launch per kernel for all the views of a group",
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -1033,11 +1035,14 @@ def stage_breakdown(tr, pl, torch):
             timed("project", pl.project_views, tr.gauss, [tr.views[k] for k in ks], [tr.projs[k] for k in ks],
                   [tr.radii[k] for k in ks])
             timed("bin_sort", pl.depth_order_views, [tr.projs[k] for k in ks], [tr.radii[k] for k in ks], d)
+            if tr.bin_views:
+                timed("bin_sort", pl.bin_sort_ordered_views_async, [tr.projs[k] for k in ks],
+                      [tr.views[k] for k in ks], d, tr.kcount[ks[0]:ks[-1] + 1], [tr.radii[k] for k in ks])
     for k, (view, tgt) in enumerate(zip(tr.views, tr.targets)):
         r = tr.radii[k]
         g2 = tr.grad2ds[k]
         proj = tr.projs[k] if batched else tr.proj
-        if batched:
+        if batched and not tr.bin_views:
             timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.order_row(k), tr.kcount[k:k + 1], r)
         else:
             timed("project", pl.project, tr.gauss, view, proj, r)
@@ -1233,6 +1238,8 @@ def main(argv=None):
     ap.add_argument("--groups", type=int, default=1,
                     help="view groups of the batched path (projection and depth sort of a group overlap "
                          "the compositing of the groups before it)")
+    ap.add_argument("--per-view-bin", action="store_true",
+                    help="bin each view with its own launches instead of one launch per kernel for a view group")
     ap.add_argument("--per-view-sort", action="store_true",
                     help="sort each view on its own stream instead of one batched depth sort of all views")
     ap.add_argument("--views", type=int, default=16,

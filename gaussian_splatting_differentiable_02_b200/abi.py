@@ -87,6 +87,10 @@ SIGNATURES = {
     "gs_depth_order_views": (C.c_int32, [C.POINTER(gs_projected), C.c_int32, C.c_int64, _P, C.c_size_t, _P, _P]),
     "gs_bin_sort_ordered_async": (C.c_int32, [C.POINTER(gs_projected), C.c_int64, _P, C.POINTER(gs_camera), _P,
                                               C.c_size_t, _P, _P, C.c_int64, _P, _P, _P]),
+    "gs_bin_sort_ordered_views_async": (C.c_int32, [C.POINTER(gs_projected), C.c_int32, C.c_int64, _P,
+                                                    C.POINTER(gs_camera), C.POINTER(_P), C.POINTER(C.c_size_t),
+                                                    C.POINTER(_P), C.POINTER(_P), C.POINTER(C.c_int64),
+                                                    C.POINTER(_P), C.POINTER(_P), _P]),
     "gs_tile_order": (C.c_int32, [_P, C.POINTER(gs_camera), _P, _P]),
     "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, _P]),
@@ -264,6 +268,18 @@ def gs_bin_sort_ordered_async(proj: gs_projected, n: int, order: int, cam: gs_ca
     return _check(lib().gs_bin_sort_ordered_async(C.byref(proj), n, order or None, C.byref(cam), workspace,
                                                   workspace_bytes, keys, vals, capacity, num_instances_dev,
                                                   tile_ranges, stream))
+
+
+def gs_bin_sort_ordered_views_async(projs, n: int, orders: int, cams, workspaces, workspace_bytes, keys, vals,
+                                    capacities, num_instances_dev, tile_ranges, stream: int = 0):
+    """projs, cams: sequences of gs_projected / gs_camera (one per view); orders: device
+    pointer of the [views][n] depth orders; the rest: per-view device pointers and sizes."""
+    V = len(projs)
+    ptrs = lambda xs: (_P * V)(*[x or None for x in xs])
+    return _check(lib().gs_bin_sort_ordered_views_async(
+        _arr(gs_projected, projs), V, n, orders or None, _arr(gs_camera, cams), ptrs(workspaces),
+        (C.c_size_t * V)(*workspace_bytes), ptrs(keys), ptrs(vals), (C.c_int64 * V)(*capacities),
+        ptrs(num_instances_dev), ptrs(tile_ranges), stream))
 
 
 def gs_tile_order(tile_ranges: int, cam: gs_camera, tile_order: int, stream: int = 0):

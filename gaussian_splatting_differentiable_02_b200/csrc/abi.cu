@@ -293,6 +293,58 @@ gs_status gs_bin_sort_ordered_async(const gs_projected* proj, int64_t n, const u
                          n > 0 ? order : nullptr);
 }
 
+gs_status gs_bin_sort_ordered_views_async(const gs_projected* projs, int32_t num_views, int64_t n,
+                                          const uint32_t* orders, const gs_camera* cams, void* const* workspaces,
+                                          const size_t* workspace_bytes, uint64_t* const* keys, uint32_t* const* vals,
+                                          const int64_t* capacities, uint64_t* const* num_instances_dev,
+                                          uint32_t* const* tile_ranges, void* stream) {
+    const char* fn = "gs_bin_sort_ordered_views_async";
+    if (num_views < 1 || num_views > GS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: num_views = %d (1..%d)", fn, int(num_views), GS_MAX_VIEWS);
+    if (!projs || !cams || !workspaces || !workspace_bytes || !keys || !vals || !capacities || !num_instances_dev ||
+        !tile_ranges)
+        return fail(GS_ERR_INVALID_ARG, "%s: a per-view array is NULL", fn);
+    if (n < 0 || n > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "%s: n out of range", fn);
+    if (n > 0) {
+        if (!orders) return fail(GS_ERR_INVALID_ARG, "%s: orders is NULL", fn);
+        CHECK_PTR(orders, 4);
+    }
+    gs_status st;
+    gsk::SortWorkspace ws[GS_MAX_VIEWS];
+    const uint32_t* ord[GS_MAX_VIEWS];
+    unsigned long long* cnt[GS_MAX_VIEWS];
+    for (int v = 0; v < num_views; ++v) {
+        const int64_t capacity = capacities[v];
+        if (capacity < 0 || capacity > 0xffffffffLL)
+            return fail(GS_ERR_INVALID_ARG, "%s: capacity of view %d out of range", fn, v);
+        if ((st = check_camera(fn, cams + v)) != GS_OK) return st;
+        if (cams[v].width != cams[0].width || cams[v].height != cams[0].height)
+            return fail(GS_ERR_INVALID_ARG, "%s: view %d has another image size than view 0", fn, v);
+        if ((st = check_projected(fn, projs + v, n, true)) != GS_OK) return st;
+        CHECK_PTR(num_instances_dev[v], 8);
+        CHECK_PTR(workspaces[v], 16);
+        CHECK_PTR(tile_ranges[v], 8);
+        if (capacity > 0) {
+            CHECK_PTR(keys[v], 8);
+            CHECK_PTR(vals[v], 4);
+        }
+        const size_t need = gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+        if (workspace_bytes[v] < need)
+            return fail(GS_ERR_INVALID_ARG, "%s: workspace of view %d has %zu bytes, %zu needed", fn, v,
+                        workspace_bytes[v], need);
+        gsk::sort_workspace_layout(n, capacity, workspaces[v], &ws[v]);
+        ord[v] = n > 0 ? orders + int64_t(v) * n : nullptr;
+        cnt[v] = reinterpret_cast<unsigned long long*>(num_instances_dev[v]);
+    }
+    const gs_camera* cam = cams;
+    const int64_t tiles = int64_t((cam->width + GS_TILE - 1) / GS_TILE) * ((cam->height + GS_TILE - 1) / GS_TILE);
+    if (tiles > (int64_t(1) << 20)) return fail(GS_ERR_UNSUPPORTED, "%s: more than 2^20 tiles", fn);
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_bin_sort_ordered_views(num_views, projs, n, ord, c, ws, keys, vals, capacities,
+                                                          tile_ranges, cnt, static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
 size_t gs_depth_order_workspace_bytes(int64_t n, int32_t num_views) {
     if (n < 0) n = 0;
     if (num_views < 1) num_views = 1;

@@ -101,15 +101,6 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, unsigned lon
     return before + inc - v;
 }
 
-__global__ void __launch_bounds__(256) depth_keys_kernel(const uint32_t* __restrict__ touched,
-                                                         const float* __restrict__ depth, int64_t n,
-                                                         uint32_t* __restrict__ keys, uint32_t* __restrict__ vals) {
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
-        keys[i] = __ldg(touched + i) > 0u ? __float_as_uint(__ldg(depth + i)) : 0xffffffffu;
-        vals[i] = uint32_t(i);
-    }
-}
-
 // The depth keys of several views at once: view blockIdx.y fills segment
 // blockIdx.y (n elements) of keys and vals.
 struct ViewDepths {
@@ -132,15 +123,31 @@ __global__ void __launch_bounds__(256) depth_keys_views_kernel(const ViewDepths 
 }
 
 // Radix passes over several independent segments at once (one per view): block
-// row blockIdx.y works on segment blockIdx.y, whose keys and values start
-// seg_stride elements further on and whose histograms start 256 nb further on.
-__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __restrict__ keys, const Count cnt,
-                                                             int shift, uint32_t* __restrict__ hist, int64_t nb,
-                                                             int64_t seg_stride) {
+// row blockIdx.y works on segment blockIdx.y, with its own keys, values, element
+// count, block histograms and digit totals.
+struct PassSeg {
+    const uint32_t* kin;
+    const uint32_t* vin;
+    uint32_t* kout;    // non-final passes
+    uint64_t* kout64;  // the final tile pass: key32 << 32 | depth bits of the Gaussian
+    uint32_t* vout;
+    uint32_t* hist;          // [256][nb]
+    uint32_t* digit_totals;  // [256]
+    const float* depth;      // final tile pass: the Gaussians' depths
+    Count cnt;
+    int64_t nb;  // blocks of this segment (the rest of the grid row returns)
+};
+struct PassArgs {
+    PassSeg seg[GS_MAX_VIEWS];
+    int shift;
+    int digit_bits;  // how many of the digit's 8 bits can be set (the last tile pass has fewer)
+};
+
+__global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const __grid_constant__ PassArgs a) {
     __shared__ uint32_t h[kSortWarps][256];
-    keys += int64_t(blockIdx.y) * seg_stride;
-    hist += int64_t(blockIdx.y) * 256 * nb;
-    const int64_t count = cnt.get();
+    const PassSeg& g = a.seg[blockIdx.y];
+    if (int64_t(blockIdx.x) >= g.nb) return;  // block-uniform
+    const int64_t count = g.cnt.get();
     const int warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&h[0][0])[k] = 0u;
     __syncthreads();
@@ -148,73 +155,52 @@ __global__ void __launch_bounds__(kSortBlock) upsweep_kernel(const uint32_t* __r
 #pragma unroll 4
     for (int k = 0; k < kSortPerThread; ++k) {
         const int64_t e = base + int64_t(k) * kSortBlock + threadIdx.x;
-        if (e < count) atomicAdd(&h[warp][(__ldg(keys + e) >> shift) & 0xffu], 1u);
+        if (e < count) atomicAdd(&h[warp][(__ldg(g.kin + e) >> a.shift) & 0xffu], 1u);
     }
     __syncthreads();
     for (int d = threadIdx.x; d < 256; d += kSortBlock) {
-        uint32_t s = 0;
+        uint32_t sum = 0;
 #pragma unroll
-        for (int w = 0; w < kSortWarps; ++w) s += h[w][d];
-        hist[int64_t(d) * nb + blockIdx.x] = s;
+        for (int w = 0; w < kSortWarps; ++w) sum += h[w][d];
+        g.hist[int64_t(d) * g.nb + blockIdx.x] = sum;
     }
 }
 
-// One CTA per digit: exclusive scan over the blocks' counts of that digit.
-__global__ void __launch_bounds__(1024) scan_hist_kernel(uint32_t* hist, int64_t nb, uint32_t* digit_totals) {
-    hist += int64_t(blockIdx.y) * 256 * nb;  // segment blockIdx.y
-    digit_totals += int64_t(blockIdx.y) * 256;
-    uint32_t* row = hist + int64_t(blockIdx.x) * nb;
+// One CTA per digit and segment: exclusive scan over the blocks' counts of that digit.
+__global__ void __launch_bounds__(1024) scan_hist_kernel(const __grid_constant__ PassArgs a) {
+    const PassSeg& g = a.seg[blockIdx.y];
+    uint32_t* row = g.hist + int64_t(blockIdx.x) * g.nb;
     unsigned long long carry = 0;
-    for (int64_t base = 0; base < nb; base += 1024) {
+    for (int64_t base = 0; base < g.nb; base += 1024) {
         const int64_t i = base + threadIdx.x;
-        const unsigned long long v = i < nb ? row[i] : 0ull;
+        const unsigned long long v = i < g.nb ? row[i] : 0ull;
         unsigned long long tot;
         const unsigned long long ex = block_excl_scan(v, &tot);
-        if (i < nb) row[i] = uint32_t(carry + ex);
+        if (i < g.nb) row[i] = uint32_t(carry + ex);
         carry += tot;
     }
-    if (threadIdx.x == 0) digit_totals[blockIdx.x] = uint32_t(carry);
+    if (threadIdx.x == 0) g.digit_totals[blockIdx.x] = uint32_t(carry);
 }
 
-// kFinal: write 64-bit keys (key32 << 32 | depth bits of the Gaussian) to keys_out64.
-// digit_bits: how many of the digit's 8 bits can be set (the last pass over the
-// tile bits has fewer); the rank votes only on those.
 template <bool kFinal>
-__global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kernel(const uint32_t* __restrict__ keys_in,
-                                                               const uint32_t* __restrict__ vals_in,
-                                                               uint32_t* __restrict__ keys_out,
-                                                               uint64_t* __restrict__ keys_out64,
-                                                               uint32_t* __restrict__ vals_out, const Count cnt,
-                                                               int shift, int digit_bits,
-                                                               const uint32_t* __restrict__ hist,
-                                                               int64_t nb, const uint32_t* __restrict__ digit_totals,
-                                                               const float* __restrict__ depth, int64_t seg_stride) {
+__global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kernel(const __grid_constant__ PassArgs a) {
     __shared__ uint32_t wcount[kSortWarps][256];
     __shared__ uint32_t gbase[256];   // global start of each digit's run from this block
     __shared__ uint32_t lstart[256];  // start of each digit's run within the block
     __shared__ uint32_t sk[kSortTile];
     __shared__ uint32_t sv[kSortTile];
-    {
-        const int64_t so = int64_t(blockIdx.y) * seg_stride;  // segment blockIdx.y
-        keys_in += so;
-        vals_in += so;
-        vals_out += so;
-        if (kFinal)
-            keys_out64 += so;
-        else
-            keys_out += so;
-        hist += int64_t(blockIdx.y) * 256 * nb;
-        digit_totals += int64_t(blockIdx.y) * 256;
-    }
-    const int64_t count = cnt.get();
+    const PassSeg& g = a.seg[blockIdx.y];
+    if (int64_t(blockIdx.x) >= g.nb) return;  // block-uniform
+    const int64_t count = g.cnt.get();
     const int64_t tile0 = int64_t(blockIdx.x) * kSortTile;
     if (tile0 >= count) return;  // block-uniform: launched for the capacity
+    const int shift = a.shift;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int k = threadIdx.x; k < kSortWarps * 256; k += kSortBlock) (&wcount[0][0])[k] = 0u;
     {
         unsigned long long tot;
-        const unsigned long long ex = block_excl_scan(threadIdx.x < 256 ? digit_totals[threadIdx.x] : 0u, &tot);
-        if (threadIdx.x < 256) gbase[threadIdx.x] = uint32_t(ex) + hist[int64_t(threadIdx.x) * nb + blockIdx.x];
+        const unsigned long long ex = block_excl_scan(threadIdx.x < 256 ? g.digit_totals[threadIdx.x] : 0u, &tot);
+        if (threadIdx.x < 256) gbase[threadIdx.x] = uint32_t(ex) + g.hist[int64_t(threadIdx.x) * g.nb + blockIdx.x];
     }
     __syncthreads();
 
@@ -225,8 +211,8 @@ __global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kern
     for (int r = 0; r < kSortPerThread; ++r) {
         const int64_t e = base + r * 32 + lane;
         const bool in = e < count;
-        key[r] = in ? __ldg(keys_in + e) : 0u;
-        val[r] = in ? __ldg(vals_in + e) : 0u;
+        key[r] = in ? __ldg(g.kin + e) : 0u;
+        val[r] = in ? __ldg(g.vin + e) : 0u;
         const uint32_t digit = in ? ((key[r] >> shift) & 0xffu) : 256u;
         // the lanes holding the same digit, from one vote per digit bit and one for
         // validity (cheaper than a match instruction here: 0.41 -> 0.38 ms per 1080p view)
@@ -234,7 +220,7 @@ __global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kern
         peers = in ? peers : ~peers;
 #pragma unroll
         for (int bit = 0; bit < 8; ++bit) {
-            if (bit >= digit_bits) break;  // warp-uniform
+            if (bit >= a.digit_bits) break;  // warp-uniform
             const bool set = (digit >> bit) & 1u;
             const uint32_t vb = __ballot_sync(0xffffffffu, set);
             peers &= set ? vb : ~vb;
@@ -278,45 +264,67 @@ __global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kern
     for (int p = threadIdx.x; p < in_block; p += kSortBlock) {
         const uint32_t k = sk[p], v = sv[p];
         const uint32_t digit = (k >> shift) & 0xffu;
-        const uint32_t g = gbase[digit] + (uint32_t(p) - lstart[digit]);
+        const uint32_t o = gbase[digit] + (uint32_t(p) - lstart[digit]);
         if (kFinal) {
-            keys_out64[g] = (uint64_t(k) << 32) | __float_as_uint(__ldg(depth + v));
+            g.kout64[o] = (uint64_t(k) << 32) | __float_as_uint(__ldg(g.depth + v));
         } else {
-            keys_out[g] = k;
+            g.kout[o] = k;
         }
-        vals_out[g] = v;
+        g.vout[o] = v;
     }
 }
 
-__global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const uint32_t* __restrict__ touched,
-                                                                  const uint32_t* __restrict__ order, int64_t n,
-                                                                  unsigned long long* block_sums) {
+// The emission of several views at once (one per block row): each view's
+// projection, depth order, workspace and outputs.
+struct EmitSeg {
+    const uint32_t* touched;
+    const uint2* rect;
+    const uint32_t* order;           // [n] the view's depth order
+    unsigned long long* block_sums;  // [nb_emit]
+    unsigned long long* total;       // the view's instance count K
+    unsigned long long* count_out;   // nullable: a copy of K for the caller
+    Count inst;                      // K, or 0 when it exceeds the view's capacity
+    uint32_t* tkey;                  // emitted (tile, gid) pairs
+    uint32_t* tval;
+    const uint64_t* keys;            // the sorted keys (ranges)
+    uint2* ranges;                   // [tiles]
+};
+struct EmitArgs {
+    EmitSeg seg[GS_MAX_VIEWS];
+    int64_t n;        // Gaussians, the same in every view
+    int64_t nb_emit;  // chunks of kEmitChunk Gaussians
+    int tiles_x;
+    int64_t tiles;
+};
+
+__global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const __grid_constant__ EmitArgs a) {
+    const EmitSeg& g = a.seg[blockIdx.y];
     const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
-    unsigned long long s = 0;
+    unsigned long long sum = 0;
     for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
         const int64_t i = base + k;
-        if (i < n) s += __ldg(touched + __ldg(order + i));
+        if (i < a.n) sum += __ldg(g.touched + __ldg(g.order + i));
     }
     unsigned long long tot;
-    block_excl_scan(s, &tot);
-    if (threadIdx.x == 0) block_sums[blockIdx.x] = tot;
+    block_excl_scan(sum, &tot);
+    if (threadIdx.x == 0) g.block_sums[blockIdx.x] = tot;
 }
 
-__global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* block_sums, int64_t nb,
-                                                           unsigned long long* total,
-                                                           unsigned long long* total_copy) {
+// One CTA per view: exclusive scan of the view's block sums, its total K.
+__global__ void __launch_bounds__(1024) scan_blocks_kernel(const __grid_constant__ EmitArgs a) {
+    const EmitSeg& g = a.seg[blockIdx.x];
     unsigned long long carry = 0;
-    for (int64_t base = 0; base < nb; base += 1024) {
+    for (int64_t base = 0; base < a.nb_emit; base += 1024) {
         const int64_t i = base + threadIdx.x;
-        const unsigned long long v = i < nb ? block_sums[i] : 0ull;
+        const unsigned long long v = i < a.nb_emit ? g.block_sums[i] : 0ull;
         unsigned long long tot;
         const unsigned long long ex = block_excl_scan(v, &tot);
-        if (i < nb) block_sums[i] = carry + ex;
+        if (i < a.nb_emit) g.block_sums[i] = carry + ex;
         carry += tot;
     }
     if (threadIdx.x == 0) {
-        *total = carry;
-        if (total_copy) *total_copy = carry;
+        *g.total = carry;
+        if (g.count_out) *g.count_out = carry;
     }
 }
 
@@ -325,34 +333,30 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(unsigned long long* b
 // finds its Gaussian by a binary search over the block's exclusive offsets in
 // shared memory, then its tile from its index inside the Gaussian's tile
 // rectangle (row-major).  Consecutive slots are written by consecutive threads.
-__global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __restrict__ touched,
-                                                          const uint2* __restrict__ rect,
-                                                          const uint32_t* __restrict__ order, int64_t n, int tiles_x,
-                                                          const unsigned long long* __restrict__ block_offsets,
-                                                          const Count cnt, uint32_t* __restrict__ tkeys,
-                                                          uint32_t* __restrict__ tvals) {
+__global__ void __launch_bounds__(kEmitBlock) emit_kernel(const __grid_constant__ EmitArgs a) {
     __shared__ uint32_t s_start[kEmitChunk];
     __shared__ uint32_t s_gid[kEmitChunk];
     __shared__ uint2 s_rect[kEmitChunk];
-    if (cnt.get() == 0) return;  // nothing fits: emit nothing
+    const EmitSeg& g = a.seg[blockIdx.y];
+    if (g.inst.get() == 0) return;  // nothing fits: emit nothing
     const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
     uint32_t gid[kEmitPerThread], tt[kEmitPerThread];
     unsigned long long mine = 0;
 #pragma unroll
     for (int k = 0; k < kEmitPerThread; ++k) {
-        gid[k] = first + k < n ? __ldg(order + first + k) : 0u;
-        tt[k] = first + k < n ? __ldg(touched + gid[k]) : 0u;
+        gid[k] = first + k < a.n ? __ldg(g.order + first + k) : 0u;
+        tt[k] = first + k < a.n ? __ldg(g.touched + gid[k]) : 0u;
         mine += tt[k];
     }
     unsigned long long total;
     uint32_t run = uint32_t(block_excl_scan(mine, &total));
-    const unsigned long long base = block_offsets[blockIdx.x];
+    const unsigned long long base = g.block_sums[blockIdx.x];
 #pragma unroll
     for (int k = 0; k < kEmitPerThread; ++k) {
         const int idx = threadIdx.x * kEmitPerThread + k;
         s_start[idx] = run;
         s_gid[idx] = gid[k];
-        s_rect[idx] = tt[k] ? __ldg(rect + gid[k]) : make_uint2(0u, 0u);
+        s_rect[idx] = tt[k] ? __ldg(g.rect + gid[k]) : make_uint2(0u, 0u);
         run += tt[k];
     }
     __syncthreads();
@@ -366,53 +370,59 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const uint32_t* __rest
         const uint2 r = s_rect[lo];
         const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, w = (r.y & 0xffffu) - x0;
         const uint32_t ty = y0 + j / w, tx = x0 + j % w;
-        tkeys[base + slot] = ty * uint32_t(tiles_x) + tx;
-        tvals[base + slot] = s_gid[lo];
+        g.tkey[base + slot] = ty * uint32_t(a.tiles_x) + tx;
+        g.tval[base + slot] = s_gid[lo];
     }
+}
+
+// Every view's tile ranges empty: [0, 0).
+__global__ void __launch_bounds__(256) zero_ranges_kernel(const __grid_constant__ EmitArgs a) {
+    const EmitSeg& g = a.seg[blockIdx.y];
+    for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < a.tiles; t += int64_t(gridDim.x) * blockDim.x)
+        g.ranges[t] = make_uint2(0u, 0u);
 }
 
 // Four consecutive keys per thread: a tile starts at k when the key before k has
 // another tile, and ends after k when the key after k does.
-__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* __restrict__ keys, const Count cnt,
-                                                     uint2* __restrict__ ranges) {
-    const int64_t K = cnt.get();
+__global__ void __launch_bounds__(256) ranges_kernel(const __grid_constant__ EmitArgs a) {
+    const EmitSeg& g = a.seg[blockIdx.y];
+    const int64_t K = g.inst.get();
     for (int64_t k0 = 4 * (blockIdx.x * int64_t(blockDim.x) + threadIdx.x); k0 < K;
          k0 += 4 * int64_t(gridDim.x) * blockDim.x) {
         uint32_t t[6];  // tiles of keys k0 - 1 .. k0 + 4 (0xffffffff past either end)
 #pragma unroll
         for (int i = 0; i < 6; ++i) {
             const int64_t k = k0 - 1 + i;
-            t[i] = k >= 0 && k < K ? uint32_t(__ldg(keys + k) >> 32) : 0xffffffffu;
+            t[i] = k >= 0 && k < K ? uint32_t(__ldg(g.keys + k) >> 32) : 0xffffffffu;
         }
 #pragma unroll
         for (int i = 1; i < 5; ++i) {
             if (k0 - 1 + i >= K) break;
-            if (t[i - 1] != t[i]) ranges[t[i]].x = uint32_t(k0 - 1 + i);
-            if (t[i + 1] != t[i]) ranges[t[i]].y = uint32_t(k0 + i);
+            if (t[i - 1] != t[i]) g.ranges[t[i]].x = uint32_t(k0 - 1 + i);
+            if (t[i + 1] != t[i]) g.ranges[t[i]].y = uint32_t(k0 + i);
         }
     }
 }
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
-// One LSD pass over up to `slots` (key, val) pairs (`cnt` of them when the pass
-// starts).  Final passes write 64-bit keys.
-void radix_pass(const uint32_t* kin, const uint32_t* vin, uint32_t* kout, uint64_t* kout64, uint32_t* vout,
-                Count cnt, int64_t slots, int shift, uint32_t* hist, uint32_t* digit_totals, const float* depth,
-                cudaStream_t s, int segments = 1, int64_t seg_stride = 0, int digit_bits = 8) {
-    const int64_t nb = (slots + kSortTile - 1) / kSortTile;
-    if (nb == 0) return;
+// One LSD pass over every segment of `a` (a.shift and a.digit_bits set for the
+// pass): the grid covers the segment with the most blocks.
+void radix_pass(const PassArgs& a, int segments, bool final, cudaStream_t s) {
+    int64_t nb = 0;
+    for (int v = 0; v < segments; ++v) nb = a.seg[v].nb > nb ? a.seg[v].nb : nb;
+    if (nb == 0 || segments == 0) return;
     const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>(segments));
-    upsweep_kernel<<<grid, kSortBlock, 0, s>>>(kin, cnt, shift, hist, nb, seg_stride);
-    scan_hist_kernel<<<dim3(256, unsigned(segments)), 1024, 0, s>>>(hist, nb, digit_totals);
-    if (kout64)
-        downsweep_kernel<true><<<grid, kSortBlock, 0, s>>>(kin, vin, nullptr, kout64, vout, cnt, shift, digit_bits,
-                                                           hist, nb, digit_totals, depth, seg_stride);
+    upsweep_kernel<<<grid, kSortBlock, 0, s>>>(a);
+    scan_hist_kernel<<<dim3(256, unsigned(segments)), 1024, 0, s>>>(a);
+    if (final)
+        downsweep_kernel<true><<<grid, kSortBlock, 0, s>>>(a);
     else
-        downsweep_kernel<false><<<grid, kSortBlock, 0, s>>>(kin, vin, kout, nullptr, vout, cnt, shift, digit_bits,
-                                                            hist, nb, digit_totals, depth, seg_stride);
+        downsweep_kernel<false><<<grid, kSortBlock, 0, s>>>(a);
     count_launches(3);
 }
+
+int64_t sort_blocks(int64_t slots) { return (slots + kSortTile - 1) / kSortTile; }
 
 }  // namespace
 
@@ -476,12 +486,26 @@ cudaError_t launch_depth_order(const gs_projected* projs, int views, int64_t n, 
     depth_keys_views_kernel<<<kgrid, 256, 0, s>>>(src, n, ws.key[0], ws.val[0]);
     count_launches(1);
     // four stable 8-bit passes A -> B -> A -> B -> (A, order), every view a segment
-    const Count all{n, nullptr, 0};
     for (int p = 0; p < 4; ++p) {
-        const int a = p & 1;
-        uint32_t* vout = p == 3 ? order : ws.val[a ^ 1];
-        radix_pass(ws.key[a], ws.val[a], ws.key[a ^ 1], nullptr, vout, all, n, 8 * p, ws.hist, ws.digit_totals,
-                   nullptr, s, views, n);
+        const int b = p & 1;
+        PassArgs a;
+        a.shift = 8 * p;
+        a.digit_bits = 8;
+        for (int v = 0; v < views; ++v) {
+            const int64_t o = int64_t(v) * n;
+            PassSeg& g = a.seg[v];
+            g.kin = ws.key[b] + o;
+            g.vin = ws.val[b] + o;
+            g.kout = ws.key[b ^ 1] + o;
+            g.kout64 = nullptr;
+            g.vout = (p == 3 ? order : ws.val[b ^ 1]) + o;
+            g.hist = ws.hist + int64_t(v) * 256 * ws.nb;
+            g.digit_totals = ws.digit_totals + int64_t(v) * 256;
+            g.depth = nullptr;
+            g.cnt = Count{n, nullptr, 0};
+            g.nb = ws.nb;
+        }
+        radix_pass(a, views, false, s);
     }
     return cudaGetLastError();
 }
@@ -492,51 +516,106 @@ cudaError_t launch_bin_sort(const gs_projected& proj, int64_t n, const CamArgs& 
     if (n > 0) {
         // depth order of the Gaussians: 4 passes from buffer 1 back into buffer 1, so
         // that tval[1] holds the order while the instances are emitted into buffer 0
-        depth_keys_kernel<<<grid_for(n, 256, 8), 256, 0, s>>>(proj.tiles_touched, proj.depth, n, ws.tkey[1],
-                                                               ws.tval[1]);
+        ViewDepths src;
+        src.touched[0] = proj.tiles_touched;
+        src.depth[0] = proj.depth;
+        depth_keys_views_kernel<<<dim3(grid_for(n, 256, 8), 1), 256, 0, s>>>(src, n, ws.tkey[1], ws.tval[1]);
         count_launches(1);
-        const Count all{n, nullptr, 0};
         for (int p = 0; p < 4; ++p) {
-            const int src = (p & 1) ? 0 : 1;
-            radix_pass(ws.tkey[src], ws.tval[src], ws.tkey[src ^ 1], nullptr, ws.tval[src ^ 1], all, n, 8 * p,
-                       ws.hist, ws.digit_totals, nullptr, s);
+            const int b = (p & 1) ? 0 : 1;
+            PassArgs a;
+            a.shift = 8 * p;
+            a.digit_bits = 8;
+            PassSeg& g = a.seg[0];
+            g.kin = ws.tkey[b];
+            g.vin = ws.tval[b];
+            g.kout = ws.tkey[b ^ 1];
+            g.kout64 = nullptr;
+            g.vout = ws.tval[b ^ 1];
+            g.hist = ws.hist;
+            g.digit_totals = ws.digit_totals;
+            g.depth = nullptr;
+            g.cnt = Count{n, nullptr, 0};
+            g.nb = sort_blocks(n);
+            radix_pass(a, 1, false, s);
         }
     }
-    return launch_bin_sort_ordered(proj, n, ws.tval[1], cam, ws, keys, vals, capacity, ranges, count_out, s);
+    return launch_bin_sort_ordered_views(1, &proj, n, &ws.tval[1], cam, &ws, &keys, &vals, &capacity, &ranges,
+                                         &count_out, s);
 }
 
 cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const uint32_t* order, const CamArgs& cam,
                                     const SortWorkspace& ws, uint64_t* keys, uint32_t* vals, int64_t capacity,
                                     uint32_t* ranges, unsigned long long* count_out, cudaStream_t s) {
+    return launch_bin_sort_ordered_views(1, &proj, n, &order, cam, &ws, &keys, &vals, &capacity, &ranges, &count_out,
+                                         s);
+}
+
+cudaError_t launch_bin_sort_ordered_views(int views, const gs_projected* projs, int64_t n,
+                                          const uint32_t* const* orders, const CamArgs& cam, const SortWorkspace* ws,
+                                          uint64_t* const* keys, uint32_t* const* vals, const int64_t* capacity,
+                                          uint32_t* const* ranges, unsigned long long* const* count_out,
+                                          cudaStream_t s) {
+    if (views == 0) return cudaSuccess;
     const int64_t T = int64_t(cam.TX) * cam.TY;
-    cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint32_t) * 2 * size_t(T), s);
-    if (e != cudaSuccess) return e;
-    if (n == 0) {
-        e = cudaMemsetAsync(ws.total, 0, sizeof(unsigned long long), s);
-        if (e == cudaSuccess && count_out) e = cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), s);
-        return e;
+    EmitArgs e;
+    e.n = n;
+    e.nb_emit = ws[0].nb_emit;  // n alone sets it: the same in every view
+    e.tiles_x = cam.TX;
+    e.tiles = T;
+    int64_t cap_max = 0;
+    for (int v = 0; v < views; ++v) {
+        EmitSeg& g = e.seg[v];
+        g.touched = projs[v].tiles_touched;
+        g.rect = reinterpret_cast<const uint2*>(projs[v].rect);
+        g.order = orders[v];
+        g.block_sums = ws[v].block_sums;
+        g.total = ws[v].total;
+        g.count_out = count_out[v];
+        g.inst = Count{0, ws[v].total, capacity[v]};
+        g.tkey = ws[v].tkey[0];
+        g.tval = ws[v].tval[0];
+        g.keys = keys[v];
+        g.ranges = reinterpret_cast<uint2*>(ranges[v]);
+        cap_max = capacity[v] > cap_max ? capacity[v] : cap_max;
     }
-    count_sorted_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, order, n, ws.block_sums);
-    scan_blocks_kernel<<<1, 1024, 0, s>>>(ws.block_sums, ws.nb_emit, ws.total, count_out);
-    count_launches(2);
-    // instances: launched for the capacity, K read on the device
-    const Count inst{0, ws.total, capacity};
-    emit_kernel<<<unsigned(ws.nb_emit), kEmitBlock, 0, s>>>(proj.tiles_touched, reinterpret_cast<const uint2*>(proj.rect),
-                                                            order, n, cam.TX, ws.block_sums, inst, ws.tkey[0],
-                                                            ws.tval[0]);
+    const unsigned V = static_cast<unsigned>(views);
+    zero_ranges_kernel<<<dim3(grid_for(T, 256, 2), V), 256, 0, s>>>(e);
+    count_launches(1);
+    if (e.nb_emit > 0)
+        count_sorted_kernel<<<dim3(unsigned(e.nb_emit), V), kEmitBlock, 0, s>>>(e);
+    scan_blocks_kernel<<<V, 1024, 0, s>>>(e);  // n = 0: every K is 0
+    count_launches(e.nb_emit > 0 ? 2 : 1);
+    if (n == 0) return cudaGetLastError();
+    // instances: launched for the capacities, K read on the device
+    emit_kernel<<<dim3(unsigned(e.nb_emit), V), kEmitBlock, 0, s>>>(e);
     count_launches(1);
     const int bits = tile_bits(T);
     const int passes = bits > 0 ? (bits + 7) / 8 : 1;
     int cur = 0;
     for (int p = 0; p < passes; ++p) {
         const bool last = p == passes - 1;
-        radix_pass(ws.tkey[cur], ws.tval[cur], last ? nullptr : ws.tkey[cur ^ 1], last ? keys : nullptr,
-                   last ? vals : ws.tval[cur ^ 1], inst, capacity, 8 * p, ws.hist, ws.digit_totals, proj.depth, s,
-                   1, 0, last ? bits - 8 * p : 8);
+        PassArgs a;
+        a.shift = 8 * p;
+        a.digit_bits = last ? bits - 8 * p : 8;
+        for (int v = 0; v < views; ++v) {
+            PassSeg& g = a.seg[v];
+            g.kin = ws[v].tkey[cur];
+            g.vin = ws[v].tval[cur];
+            g.kout = last ? nullptr : ws[v].tkey[cur ^ 1];
+            g.kout64 = last ? keys[v] : nullptr;
+            g.vout = last ? vals[v] : ws[v].tval[cur ^ 1];
+            g.hist = ws[v].hist;
+            g.digit_totals = ws[v].digit_totals;
+            g.depth = projs[v].depth;
+            g.cnt = e.seg[v].inst;
+            g.nb = sort_blocks(capacity[v]);
+        }
+        radix_pass(a, views, last, s);
         cur ^= 1;
     }
-    if (capacity > 0) {
-        ranges_kernel<<<grid_for(capacity, 256, 8), 256, 0, s>>>(keys, inst, reinterpret_cast<uint2*>(ranges));
+    if (cap_max > 0) {
+        ranges_kernel<<<dim3(grid_for((cap_max + 3) / 4, 256, 8), V), 256, 0, s>>>(e);
         count_launches(1);
     }
     return cudaGetLastError();

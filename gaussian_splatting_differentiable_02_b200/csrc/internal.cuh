@@ -117,6 +117,15 @@ cudaError_t launch_bin_sort_ordered(const gs_projected& proj, int64_t n, const u
                                     const SortWorkspace& ws, uint64_t* keys, uint32_t* vals, int64_t capacity,
                                     uint32_t* ranges, unsigned long long* count_out, cudaStream_t s);
 
+// launch_bin_sort_ordered for several views (at most GS_MAX_VIEWS) of the same n
+// Gaussians and tile grid in one launch per kernel: view v's projection, depth
+// order, workspace, outputs and capacity at index v.
+cudaError_t launch_bin_sort_ordered_views(int views, const gs_projected* projs, int64_t n,
+                                          const uint32_t* const* orders, const CamArgs& cam, const SortWorkspace* ws,
+                                          uint64_t* const* keys, uint32_t* const* vals, const int64_t* capacity,
+                                          uint32_t* const* ranges, unsigned long long* const* count_out,
+                                          cudaStream_t s);
+
 // Stable depth order of the Gaussians of several views (at most GS_MAX_VIEWS) in
 // one launch per radix pass: order [views][n].
 struct DepthOrderWorkspace {

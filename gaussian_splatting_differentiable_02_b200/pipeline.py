@@ -304,6 +304,20 @@ def bin_sort_ordered_async(proj: Projected, view: View, order_row: torch.Tensor,
     abi.gs_tile_order(_ptr(view.ranges), view.gcam, _ptr(view.order), _stream())
 
 
+def bin_sort_ordered_views_async(projs: list, views: list, d: DepthOrder, counters: torch.Tensor, radii=None):
+    """bin_sort_ordered_async for several views of the same image size at once (view k:
+    projs[k] with radius row radii[k], views[k], row k of d.order, counters[k]): every
+    binning kernel launched once for all of them; then each view's tile order."""
+    nv = len(views)
+    abi.gs_bin_sort_ordered_views_async(
+        [p.struct(None if radii is None else radii[k]) for k, p in enumerate(projs)], views[0].n, _ptr(d.order),
+        [vw.gcam for vw in views], [_ptr(vw.workspace) for vw in views], [vw.workspace.numel() for vw in views],
+        [_ptr(vw.keys) for vw in views], [_ptr(vw.vals) for vw in views], [vw.capacity for vw in views],
+        [counters.data_ptr() + 8 * k for k in range(nv)], [_ptr(vw.ranges) for vw in views], _stream())
+    for vw in views:
+        abi.gs_tile_order(_ptr(vw.ranges), vw.gcam, _ptr(vw.order), _stream())
+
+
 def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Tensor = None):
     abi.gs_raster_fwd(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam, bg,
                       _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _stream())
@@ -489,6 +503,8 @@ class Trainer:
                                # visible count seen
     sh16: bool = False         # fused unpacked path: the projections read a 16-bit (FP16) copy of the SH
                                # coefficients, which the fused Adam step refreshes from the float32 ones
+    bin_views: bool = True     # fused batched path: each view group's binning (emission, passes by tile,
+                               # ranges) launched once for all its views instead of once per view
     graph: bool = False        # fused path: the views' part of a step (projections, sorts, compositing,
                                # losses and their backward) is captured once into a CUDA graph and
                                # replayed every step, so its few-microsecond launches cost no host time
@@ -667,10 +683,18 @@ class Trainer:
                 bin_stream.wait_stream(main)
                 binned = {}
                 with torch.cuda.stream(bin_stream):
-                    for k in ks:
-                        bin_sort_ordered_async(self.projs[k], self.views[k], self.order_row(k),
-                                               self.kcount[k:k + 1], self._radius(k))
-                        binned[k] = bin_stream.record_event()
+                    sizes = {(self.views[k].cam["width"], self.views[k].cam["height"]) for k in ks}
+                    if self.bin_views and not self.packed and len(sizes) == 1:
+                        bin_sort_ordered_views_async([self.projs[k] for k in ks], [self.views[k] for k in ks],
+                                                     self.depth_orders[gi], self.kcount[ks[0]:ks[-1] + 1],
+                                                     [self._radius(k) for k in ks])
+                        done = bin_stream.record_event()
+                        binned = {k: done for k in ks}
+                    else:
+                        for k in ks:
+                            bin_sort_ordered_async(self.projs[k], self.views[k], self.order_row(k),
+                                                   self.kcount[k:k + 1], self._radius(k))
+                            binned[k] = bin_stream.record_event()
                 for k in ks:
                     st = side[k % len(side)]
                     st.wait_event(binned[k])

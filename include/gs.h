@@ -225,6 +225,25 @@ gs_status gs_bin_sort_ordered_async(const gs_projected* proj, int64_t n, const u
                                     int64_t capacity, uint64_t* num_instances_dev, uint32_t* tile_ranges,
                                     void* stream);
 
+/* gs_bin_sort_ordered_views_async -- gs_bin_sort_ordered_async for num_views
+ * (1..GS_MAX_VIEWS) views of the same n Gaussians and the same image size, every
+ * kernel launched once for all of them (grid rows = views): view v has
+ * projs[v], its depth order orders + v * n (the rows gs_depth_order_views
+ * writes), cams[v] (only the image size is read; all views must have the same),
+ * workspaces[v] of workspace_bytes[v] bytes, keys[v], vals[v], capacities[v],
+ * num_instances_dev[v] and tile_ranges[v] -- host arrays of device pointers and
+ * sizes.  Each view's results and capacity behaviour are gs_bin_sort_ordered_async's
+ * bit for bit; one launch per kernel instead of one per view and kernel removes
+ * the launch gaps and the partly filled last wave of every small launch.  The
+ * views' buffers must not overlap.  Errors (nothing launched): those of
+ * gs_bin_sort_ordered_async for any view, GS_ERR_INVALID_ARG for num_views
+ * outside 1..GS_MAX_VIEWS or image sizes that differ. */
+gs_status gs_bin_sort_ordered_views_async(const gs_projected* projs, int32_t num_views, int64_t n,
+                                          const uint32_t* orders, const gs_camera* cams, void* const* workspaces,
+                                          const size_t* workspace_bytes, uint64_t* const* keys, uint32_t* const* vals,
+                                          const int64_t* capacities, uint64_t* const* num_instances_dev,
+                                          uint32_t* const* tile_ranges, void* stream);
+
 /* Size of the device array gs_bin_sort_static uses as its workspace (32 MiB). */
 #define GS_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 

@@ -389,3 +389,55 @@ def test_graph_step_matches_eager(packed):
         close = d <= 1e-6 + 1e-6 * np.abs(a[k])
         assert close.mean() >= 0.999, (k, float(close.mean()))
         assert d.max() <= 8 * LRS[k] + 1e-6, (k, float(d.max()))
+
+
+@pytest.mark.parametrize("n_views", [1, 5, 16])
+def test_views_binning_matches_per_view_binning(orc, n_views):
+    """gs_bin_sort_ordered_views_async gives every view the keys, values, ranges, tile
+    order and instance count of gs_bin_sort_ordered_async, bit for bit, with views of
+    different capacities (one too small: its count is reported, nothing is emitted and
+    its ranges are empty); one view against the oracle."""
+    rng = np.random.default_rng(33)
+    scene = scenes.random_scene(rng, 2500, 1, mean_box=1.0, log_scale=(-4.0, -2.0))
+    scene.means[:50] += 30.0   # some Gaussians culled in every view
+    cams = _views(n_views, 12)
+    g = pl.Gaussians.from_scene(scene)
+    projs = [pl.Projected(scene.n) for _ in cams]
+    radii = torch.zeros((n_views, scene.n), dtype=torch.int32, device="cuda")
+    caps = [40 * scene.n + 1000 * k for k in range(n_views)]  # view 1 gets 64 slots below: too small
+    out = []
+    for batched in (False, True):
+        views = [pl.View(scene.n, c, capacity=caps[k]) for k, c in enumerate(cams)]
+        if n_views > 1:
+            views[1]._alloc(64)
+        for vw in views:
+            vw.keys.fill_(-3)
+        for k, vw in enumerate(views):
+            pl.project(g, vw, projs[k], radii[k])
+        d = pl.DepthOrder(scene.n, n_views)
+        pl.depth_order_views(projs, radii, d)
+        counts = torch.full((n_views,), -1, dtype=torch.int64, device="cuda")
+        if batched:
+            pl.bin_sort_ordered_views_async(projs, views, d, counts, radii)
+        else:
+            for k, vw in enumerate(views):
+                pl.bin_sort_ordered_async(projs[k], vw, d.order[k], counts[k:k + 1], radii[k])
+        torch.cuda.synchronize()
+        out.append(([vw.keys.cpu().numpy() for vw in views], [vw.vals.cpu().numpy() for vw in views],
+                    [vw.ranges.cpu().numpy() for vw in views], [vw.order.cpu().numpy() for vw in views],
+                    counts.cpu().numpy(), [vw.capacity for vw in views]))
+    (ka, va, ra, oa, ca, cap), (kb, vb, rb, ob, cb, _) = out
+    assert np.array_equal(ca, cb)
+    for k in range(n_views):
+        K = int(ca[k])
+        assert np.array_equal(ra[k], rb[k]) and np.array_equal(oa[k], ob[k])
+        if K <= cap[k]:
+            assert np.array_equal(ka[k][:K], kb[k][:K]) and np.array_equal(va[k][:K], vb[k][:K])
+        else:
+            assert not ra[k].any() and np.all(kb[k] == -3)
+    ref = orc.project(scene, cams[0])
+    keys, vals, ranges = orc.keys(ref, cams[0])
+    assert int(cb[0]) == len(keys)
+    assert np.array_equal(kb[0][:len(keys)].view(np.uint64), keys)
+    assert np.array_equal(vb[0][:len(keys)].view(np.uint32), vals)
+    assert np.array_equal(rb[0].view(np.uint32), ranges)
