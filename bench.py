@@ -1042,8 +1042,9 @@ def stage_breakdown(tr, pl, torch):
         r = tr.radii[k]
         g2 = tr.grad2ds[k]
         proj = tr.projs[k] if batched else tr.proj
-        if batched and not tr.bin_views:
-            timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.order_row(k), tr.kcount[k:k + 1], r)
+        if batched:
+            if not tr.bin_views:
+                timed("bin_sort", pl.bin_sort_ordered_async, proj, view, tr.order_row(k), tr.kcount[k:k + 1], r)
         else:
             timed("project", pl.project, tr.gauss, view, proj, r)
             timed("bin_sort", pl.bin_sort, proj, view, r)

@@ -92,6 +92,7 @@ SIGNATURES = {
                                                     C.POINTER(_P), C.POINTER(_P), C.POINTER(C.c_int64),
                                                     C.POINTER(_P), C.POINTER(_P), _P]),
     "gs_tile_order": (C.c_int32, [_P, C.POINTER(gs_camera), _P, _P]),
+    "gs_tile_order_views": (C.c_int32, [C.c_int32, C.POINTER(_P), C.POINTER(gs_camera), C.POINTER(_P), _P]),
     "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, _P]),
     "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
@@ -280,6 +281,12 @@ def gs_bin_sort_ordered_views_async(projs, n: int, orders: int, cams, workspaces
         _arr(gs_projected, projs), V, n, orders or None, _arr(gs_camera, cams), ptrs(workspaces),
         (C.c_size_t * V)(*workspace_bytes), ptrs(keys), ptrs(vals), (C.c_int64 * V)(*capacities),
         ptrs(num_instances_dev), ptrs(tile_ranges), stream))
+
+
+def gs_tile_order_views(tile_ranges, cam: gs_camera, tile_orders, stream: int = 0):
+    """tile_ranges, tile_orders: per-view device pointers."""
+    V = len(tile_ranges)
+    return _check(lib().gs_tile_order_views(V, (_P * V)(*tile_ranges), C.byref(cam), (_P * V)(*tile_orders), stream))
 
 
 def gs_tile_order(tile_ranges: int, cam: gs_camera, tile_order: int, stream: int = 0):

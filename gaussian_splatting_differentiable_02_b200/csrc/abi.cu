@@ -385,6 +385,24 @@ gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint3
                        fn);
 }
 
+gs_status gs_tile_order_views(int32_t num_views, const uint32_t* const* tile_ranges, const gs_camera* cam,
+                              uint32_t* const* tile_orders, void* stream) {
+    const char* fn = "gs_tile_order_views";
+    gs_status st;
+    if (num_views < 1 || num_views > GS_MAX_VIEWS)
+        return fail(GS_ERR_INVALID_ARG, "%s: num_views = %d (1..%d)", fn, int(num_views), GS_MAX_VIEWS);
+    if ((st = check_camera(fn, cam)) != GS_OK) return st;
+    if (!tile_ranges || !tile_orders) return fail(GS_ERR_INVALID_ARG, "%s: a per-view array is NULL", fn);
+    for (int v = 0; v < num_views; ++v) {
+        CHECK_PTR(tile_ranges[v], 8);
+        CHECK_PTR(tile_orders[v], 4);
+    }
+    const gsk::CamArgs c = gsk::make_cam(*cam);
+    return cuda_status(gsk::launch_tile_order_views(num_views, tile_ranges, c.TX * c.TY, tile_orders,
+                                                    static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
 }  // extern "C"
 
 namespace {

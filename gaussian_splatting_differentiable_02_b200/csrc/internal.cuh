@@ -140,6 +140,8 @@ cudaError_t launch_depth_order(const gs_projected* projs, int views, int64_t n, 
                                uint32_t* order, cudaStream_t s);
 
 cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s);
+cudaError_t launch_tile_order_views(int views, const uint32_t* const* ranges, int tiles, uint32_t* const* order,
+                                    cudaStream_t s);
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,

@@ -718,11 +718,18 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
 
 // Tiles ordered by decreasing list length (bucketed by floor(sqrt(length)),
 // 256 buckets; order inside a bucket unspecified), so that the longest tiles
-// start first and the kernel's tail holds short ones.  One CTA.
-__global__ void __launch_bounds__(1024) tile_order_kernel(const uint2* __restrict__ ranges, int tiles,
-                                                         uint32_t* __restrict__ order) {
+// start first and the kernel's tail holds short ones.  One CTA per view.
+struct TileOrderArgs {
+    const uint2* ranges[GS_MAX_VIEWS];
+    uint32_t* order[GS_MAX_VIEWS];
+    int tiles;
+};
+
+__global__ void __launch_bounds__(1024) tile_order_kernel(const __grid_constant__ TileOrderArgs a) {
     __shared__ uint32_t count[256];
     __shared__ uint32_t start[256];
+    const uint2* ranges = a.ranges[blockIdx.x];
+    uint32_t* order = a.order[blockIdx.x];
     for (int b = threadIdx.x; b < 256; b += blockDim.x) count[b] = 0u;
     __syncthreads();
     auto bucket = [&](int t) {
@@ -730,7 +737,7 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(const uint2* __restric
         const float len = float(r.y - r.x);
         return 255u - min(255u, uint32_t(sqrtf(len)));  // longest first
     };
-    for (int t = threadIdx.x; t < tiles; t += blockDim.x) atomicAdd(&count[bucket(t)], 1u);
+    for (int t = threadIdx.x; t < a.tiles; t += blockDim.x) atomicAdd(&count[bucket(t)], 1u);
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t run = 0;
@@ -740,16 +747,27 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(const uint2* __restric
         }
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < tiles; t += blockDim.x) order[atomicAdd(&start[bucket(t)], 1u)] = uint32_t(t);
+    for (int t = threadIdx.x; t < a.tiles; t += blockDim.x) order[atomicAdd(&start[bucket(t)], 1u)] = uint32_t(t);
 }
 
 }  // namespace
 
-cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s) {
-    if (tiles <= 0) return cudaSuccess;
-    tile_order_kernel<<<1, 1024, 0, s>>>(reinterpret_cast<const uint2*>(ranges), tiles, order);
+cudaError_t launch_tile_order_views(int views, const uint32_t* const* ranges, int tiles, uint32_t* const* order,
+                                    cudaStream_t s) {
+    if (tiles <= 0 || views <= 0) return cudaSuccess;
+    TileOrderArgs a;
+    for (int v = 0; v < views; ++v) {
+        a.ranges[v] = reinterpret_cast<const uint2*>(ranges[v]);
+        a.order[v] = order[v];
+    }
+    a.tiles = tiles;
+    tile_order_kernel<<<unsigned(views), 1024, 0, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
+}
+
+cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order, cudaStream_t s) {
+    return launch_tile_order_views(1, &ranges, tiles, &order, s);
 }
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,

@@ -307,15 +307,15 @@ def bin_sort_ordered_async(proj: Projected, view: View, order_row: torch.Tensor,
 def bin_sort_ordered_views_async(projs: list, views: list, d: DepthOrder, counters: torch.Tensor, radii=None):
     """bin_sort_ordered_async for several views of the same image size at once (view k:
     projs[k] with radius row radii[k], views[k], row k of d.order, counters[k]): every
-    binning kernel launched once for all of them; then each view's tile order."""
+    binning kernel launched once for all of them, then their tile orders in one launch."""
     nv = len(views)
     abi.gs_bin_sort_ordered_views_async(
         [p.struct(None if radii is None else radii[k]) for k, p in enumerate(projs)], views[0].n, _ptr(d.order),
         [vw.gcam for vw in views], [_ptr(vw.workspace) for vw in views], [vw.workspace.numel() for vw in views],
         [_ptr(vw.keys) for vw in views], [_ptr(vw.vals) for vw in views], [vw.capacity for vw in views],
         [counters.data_ptr() + 8 * k for k in range(nv)], [_ptr(vw.ranges) for vw in views], _stream())
-    for vw in views:
-        abi.gs_tile_order(_ptr(vw.ranges), vw.gcam, _ptr(vw.order), _stream())
+    abi.gs_tile_order_views([_ptr(vw.ranges) for vw in views], views[0].gcam, [_ptr(vw.order) for vw in views],
+                            _stream())
 
 
 def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Tensor = None):

@@ -277,6 +277,12 @@ gs_status gs_bin_sort_static(const gs_projected* proj, int64_t n, const gs_camer
  * depend on the order. */
 gs_status gs_tile_order(const uint32_t* tile_ranges, const gs_camera* cam, uint32_t* tile_order, void* stream);
 
+/* gs_tile_order_views -- gs_tile_order for num_views (1..GS_MAX_VIEWS) views of
+ * the same tile grid (cam's image size) in one launch: tile_ranges[v] and
+ * tile_orders[v] are view v's (host arrays of device pointers). */
+gs_status gs_tile_order_views(int32_t num_views, const uint32_t* const* tile_ranges, const gs_camera* cam,
+                              uint32_t* const* tile_orders, void* stream);
+
 /* gs_raster_fwd -- stage 3 (gsplat guide §2.1) over 16x16 tiles.  For each
  * pixel, front to back over its tile's sorted list: sigma as above with
  * d = (u, v) - pixel centre; entries with sigma < 0 are skipped;

@@ -393,10 +393,12 @@ def test_graph_step_matches_eager(packed):
 
 @pytest.mark.parametrize("n_views", [1, 5, 16])
 def test_views_binning_matches_per_view_binning(orc, n_views):
-    """gs_bin_sort_ordered_views_async gives every view the keys, values, ranges, tile
-    order and instance count of gs_bin_sort_ordered_async, bit for bit, with views of
-    different capacities (one too small: its count is reported, nothing is emitted and
-    its ranges are empty); one view against the oracle."""
+    """gs_bin_sort_ordered_views_async gives every view the keys, values, ranges and
+    instance count of gs_bin_sort_ordered_async, bit for bit, with views of different
+    capacities (one too small: its count is reported, nothing is emitted and its ranges
+    are empty); one view against the oracle.  The tile orders (one launch for the group)
+    are valid: a permutation of the tiles by non-increasing length bucket (the order
+    inside a bucket is not specified)."""
     rng = np.random.default_rng(33)
     scene = scenes.random_scene(rng, 2500, 1, mean_box=1.0, log_scale=(-4.0, -2.0))
     scene.means[:50] += 30.0   # some Gaussians culled in every view
@@ -430,7 +432,13 @@ def test_views_binning_matches_per_view_binning(orc, n_views):
     assert np.array_equal(ca, cb)
     for k in range(n_views):
         K = int(ca[k])
-        assert np.array_equal(ra[k], rb[k]) and np.array_equal(oa[k], ob[k])
+        assert np.array_equal(ra[k], rb[k])
+        r = rb[k].view(np.uint32).reshape(-1, 2)
+        bucket = 255 - np.minimum(255, np.floor(np.sqrt((r[:, 1] - r[:, 0]).astype(np.float32))).astype(np.int64))
+        for o in (oa[k], ob[k]):
+            o = o.view(np.uint32).astype(np.int64)
+            assert np.array_equal(np.sort(o), np.arange(len(r)))
+            assert np.all(np.diff(bucket[o]) >= 0)
         if K <= cap[k]:
             assert np.array_equal(ka[k][:K], kb[k][:K]) and np.array_equal(va[k][:K], vb[k][:K])
         else:
