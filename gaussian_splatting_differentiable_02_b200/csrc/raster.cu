@@ -77,6 +77,9 @@ constexpr float kCondMaxTraceSqOverDet = 10.125f;
 constexpr int kBoxW = 16;               // width of a warp's pixel box
 constexpr int kWarps = 1;               // warps per block
 constexpr int64_t kWideLayoutTiles = 6144;
+#ifndef GS_RASTER_BWD_BLOCKS8
+#define GS_RASTER_BWD_BLOCKS8 16
+#endif
 template <int PX>
 struct Layout {
     static_assert(PX % 2 == 0 && kTile % (2 * PX) == 0, "pixel pairs; boxes tile the 16x16 tile");
@@ -85,7 +88,7 @@ struct Layout {
     static constexpr int kSub = kTile / kBoxH;           // warps per tile
     // resident blocks per SM the register allocation is sized for (launch bounds)
     static constexpr int kFwdMinBlocks = PX == 8 ? 14 : 20;
-    static constexpr int kBwdMinBlocks = PX == 8 ? 16 : 20;
+    static constexpr int kBwdMinBlocks = PX == 8 ? GS_RASTER_BWD_BLOCKS8 : 20;
 };
 constexpr int kBatch = 32;  // list entries staged per warp per batch
 constexpr unsigned kFull = 0xffffffffu;
@@ -542,7 +545,10 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
     if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
-template <int PX, bool kAbs, bool kCount>
+// kBg: the background is not black.  With a black one (every workload here) the
+// background term of dL/dalpha is 0 and neither it nor its per-pixel factor is
+// formed, which saves a paired instruction per pixel pair and eight registers.
+template <int PX, bool kAbs, bool kCount, bool kBg>
 __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster_bwd_kernel(const BwdArgs a) {
     constexpr int kPx = PX, kPairs = Layout<PX>::kPairs, kBoxH = Layout<PX>::kBoxH, kSub = Layout<PX>::kSub;
     __shared__ WarpStage stage[kWarps];
@@ -562,7 +568,7 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
 
     // per pixel pair: transmittance, minus g . S (S the colour blended behind),
     // dL/dimage, -final_T (bg . g)
-    f2 nyc[kPairs], T[kPairs], nP[kPairs], gr[kPairs], gg[kPairs], gb[kPairs], ngb[kPairs];
+    f2 nyc[kPairs], T[kPairs], nP[kPairs], gr[kPairs], gg[kPairs], gb[kPairs], ngb[kBg ? kPairs : 1];
     int last[kPx];
     int lmax = 0;
 #pragma unroll
@@ -580,9 +586,11 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
         const float nb = -Ti * (a.bg0 * r + a.bg1 * g + a.bg2 * bb);
         const float ny = -(float(y0 + i) + 0.5f);
         if (i & 1) {
-            T[i / 2].y = Ti; gr[i / 2].y = r; gg[i / 2].y = g; gb[i / 2].y = bb; ngb[i / 2].y = nb; nyc[i / 2].y = ny;
+            T[i / 2].y = Ti; gr[i / 2].y = r; gg[i / 2].y = g; gb[i / 2].y = bb; nyc[i / 2].y = ny;
+            if (kBg) ngb[i / 2].y = nb;
         } else {
-            T[i / 2].x = Ti; gr[i / 2].x = r; gg[i / 2].x = g; gb[i / 2].x = bb; ngb[i / 2].x = nb; nyc[i / 2].x = ny;
+            T[i / 2].x = Ti; gr[i / 2].x = r; gg[i / 2].x = g; gb[i / 2].x = bb; nyc[i / 2].x = ny;
+            if (kBg) ngb[i / 2].x = nb;
         }
         lmax = max(lmax, last[i]);
     }
@@ -645,7 +653,7 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
                     ndb = fma2(nw, gb[p], ndb);
                     // only g . S enters the gradient: P = g . S with S <- c alpha + (1 - alpha) S
                     const f2 xg = add2(fma2(gr[p], cr, fma2(gg[p], cg, mul2(gb[p], cb))), nP[p]);  // g . c - P
-                    const f2 dLda = fma2(T[p], xg, mul2(ngb[p], rom));
+                    const f2 dLda = kBg ? fma2(T[p], xg, mul2(ngb[p], rom)) : mul2(T[p], xg);
                     nP[p] = fma2(nae, xg, nP[p]);
                     // -dL/dalpha alpha = dL/dsigma, zero where alpha was clamped (times a 0/1 gate)
                     f2 q = mul2(dLda, nae);
@@ -809,19 +817,27 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
 }
 
 namespace {
-template <int PX>
-void launch_raster_bwd_layout(const BwdArgs& a, bool counted, cudaStream_t s) {
+template <int PX, bool kBg>
+void launch_raster_bwd_bg(const BwdArgs& a, bool counted, cudaStream_t s) {
     const unsigned grid = unsigned(a.tiles * Layout<PX>::kSub);
     if (counted) {
         if (a.g_xy_abs)
-            raster_bwd_kernel<PX, true, true><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_bwd_kernel<PX, true, true, kBg><<<grid, kWarps * 32, 0, s>>>(a);
         else
-            raster_bwd_kernel<PX, false, true><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_bwd_kernel<PX, false, true, kBg><<<grid, kWarps * 32, 0, s>>>(a);
     } else if (a.g_xy_abs) {
-        raster_bwd_kernel<PX, true, false><<<grid, kWarps * 32, 0, s>>>(a);
+        raster_bwd_kernel<PX, true, false, kBg><<<grid, kWarps * 32, 0, s>>>(a);
     } else {
-        raster_bwd_kernel<PX, false, false><<<grid, kWarps * 32, 0, s>>>(a);
+        raster_bwd_kernel<PX, false, false, kBg><<<grid, kWarps * 32, 0, s>>>(a);
     }
+}
+
+template <int PX>
+void launch_raster_bwd_layout(const BwdArgs& a, bool counted, cudaStream_t s) {
+    if (a.bg0 != 0.f || a.bg1 != 0.f || a.bg2 != 0.f)
+        launch_raster_bwd_bg<PX, true>(a, counted, s);
+    else
+        launch_raster_bwd_bg<PX, false>(a, counted, s);
 }
 }  // namespace
 

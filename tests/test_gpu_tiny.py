@@ -300,3 +300,22 @@ def test_needle_and_indefinite_conics(orc):
     rows = np.nonzero(touched == 0)[0]
     for q, name in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
         check_grads(g2_gpu[:, q], g2[:, q], name, rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.002)
+
+
+@pytest.mark.parametrize("bg", [(0.2, 0.5, 0.8), (0.0, 0.0, 0.0)])
+def test_backward_grad2d_with_a_background(orc, bg):
+    """The reverse pass with a coloured background (its term of dL/dalpha, -T_final
+    bg . g / (1 - alpha), formed per pixel) and with a black one (where the kernel
+    leaves that term out), against the oracle's reverse pass with the same background."""
+    wl = scenes.tiny()
+    cam = wl.cameras[0]
+    run = CudaRun(wl.scene, cam, bg=bg)
+    ref = orc.project(wl.scene, cam)
+    g = wl.upstream[0]
+    g2_gpu = run.backward(g)
+    g2, g2a, touched = orc.render_bwd(ref, cam, g.reshape(-1, 3).astype(np.float64), bg=bg, band_alpha=BAND_ALPHA,
+                                      band_T=BAND_T)
+    rows = np.nonzero(touched == 0)[0]
+    assert len(rows) > 900
+    for q, name in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
+        check_grads(g2_gpu[:, q], g2[:, q], name, rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.002)
