@@ -1048,8 +1048,11 @@ def stage_breakdown(tr, pl, torch):
         else:
             timed("project", pl.project, tr.gauss, view, proj, r)
             timed("bin_sort", pl.bin_sort, proj, view, r)
-        timed("raster_fwd", pl.raster_fwd, proj, view, tr.bg, r)
-        timed("l1", pl.l1_loss_grad, view, tgt, tr.loss)
+        if tr.ssim_weight > 0.0:
+            timed("raster_fwd", pl.raster_fwd, proj, view, tr.bg, r)
+            timed("l1", pl.l1_dssim_loss_grad, view, tgt, tr.loss, 1.0, tr.ssim_weight)
+        else:   # the Trainer's L1 step: the loss and dL/dimage come out of the forward kernel
+            timed("raster_fwd", pl.raster_fwd_l1, proj, view, tgt, tr.loss, tr.bg, r)
         g2.zero_()
         timed("raster_bwd", pl.raster_bwd, proj, view, g2, tr.bg, None, r)
     tr.step_count += 1

@@ -95,6 +95,8 @@ SIGNATURES = {
     "gs_tile_order_views": (C.c_int32, [C.c_int32, C.POINTER(_P), C.POINTER(gs_camera), C.POINTER(_P), _P]),
     "gs_raster_fwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, _P]),
+    "gs_raster_fwd_l1": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera),
+                                     C.POINTER(C.c_float), _P, _P, _P, _P, _P, _P, _P]),
     "gs_raster_bwd": (C.c_int32, [C.POINTER(gs_projected), _P, _P, _P, C.POINTER(gs_camera), C.POINTER(C.c_float),
                                   _P, _P, _P, C.POINTER(gs_grad2d), _P]),
     "gs_project_bwd": (C.c_int32, [C.POINTER(gs_params), C.POINTER(gs_camera), C.POINTER(gs_projected),
@@ -299,6 +301,14 @@ def gs_raster_fwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: i
     b = (C.c_float * 3)(*[float(x) for x in bg])
     return _check(lib().gs_raster_fwd(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b, image,
                                       final_T, n_contrib, stream))
+
+
+def gs_raster_fwd_l1(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg, target: int,
+                     image: int, final_T: int, n_contrib: int, dL_dimage: int, loss_dev: int, stream: int = 0):
+    """gs_raster_fwd with the L1 term against target in the same kernel."""
+    b = (C.c_float * 3)(*[float(x) for x in bg])
+    return _check(lib().gs_raster_fwd_l1(C.byref(proj), vals, tile_ranges, tile_order or None, C.byref(cam), b, target,
+                                         image, final_T, n_contrib, dL_dimage, loss_dev, stream))
 
 
 def gs_raster_bwd(proj: gs_projected, vals: int, tile_ranges: int, tile_order: int, cam: gs_camera, bg, final_T: int,

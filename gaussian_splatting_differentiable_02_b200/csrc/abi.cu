@@ -410,7 +410,7 @@ namespace {
 gs_status raster_fwd_common(const char* fn, const gs_projected* proj, const uint32_t* vals,
                             const uint32_t* tile_ranges, const uint32_t* tile_order, const gs_camera* cam,
                             const float* bg_host, float* image, float* final_T, int32_t* n_contrib,
-                            unsigned long long* counts, void* stream) {
+                            unsigned long long* counts, void* stream, const gsk::L1Out* l1 = nullptr) {
     gs_status st;
     if ((st = check_camera(fn, cam)) != GS_OK) return st;
     if ((st = check_projected(fn, proj, 1, false)) != GS_OK) return st;
@@ -421,9 +421,14 @@ gs_status raster_fwd_common(const char* fn, const gs_projected* proj, const uint
     CHECK_PTR(image, 4);
     CHECK_PTR(final_T, 4);
     CHECK_PTR(n_contrib, 4);
+    if (l1) {
+        CHECK_PTR(l1->target, 4);
+        CHECK_PTR(l1->dL_dimage, 4);
+        CHECK_PTR(l1->loss, 8);
+    }
     const gsk::CamArgs c = gsk::make_cam(*cam);
     return cuda_status(gsk::launch_raster_fwd(*proj, vals, tile_ranges, tile_order, c, bg_host, image, final_T,
-                                              n_contrib, static_cast<cudaStream_t>(stream), counts),
+                                              n_contrib, static_cast<cudaStream_t>(stream), counts, l1),
                        fn);
 }
 
@@ -461,6 +466,15 @@ gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const ui
                         float* final_T, int32_t* n_contrib, void* stream) {
     return raster_fwd_common("gs_raster_fwd", proj, vals, tile_ranges, tile_order, cam, bg_host, image, final_T,
                              n_contrib, nullptr, stream);
+}
+
+gs_status gs_raster_fwd_l1(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                           const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* target,
+                           float* image, float* final_T, int32_t* n_contrib, float* dL_dimage, double* loss_dev,
+                           void* stream) {
+    const gsk::L1Out l1{target, dL_dimage, loss_dev};
+    return raster_fwd_common("gs_raster_fwd_l1", proj, vals, tile_ranges, tile_order, cam, bg_host, image, final_T,
+                             n_contrib, nullptr, stream, &l1);
 }
 
 gs_status gs_raster_bwd(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,

@@ -143,10 +143,17 @@ cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order
 cudaError_t launch_tile_order_views(int views, const uint32_t* const* ranges, int tiles, uint32_t* const* order,
                                     cudaStream_t s);
 
+// The L1 term fused into the forward pass (gs_raster_fwd_l1).
+struct L1Out {
+    const float* target;  // [H][W][3]
+    float* dL_dimage;     // [H][W][3]
+    double* loss;         // += mean |image - target|
+};
+
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
                               float* final_T, int32_t* n_contrib, cudaStream_t s,
-                              unsigned long long* counts = nullptr);
+                              unsigned long long* counts = nullptr, const L1Out* l1 = nullptr);
 
 cudaError_t launch_raster_bwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], const float* final_T,

@@ -340,6 +340,12 @@ struct FwdArgs {
     float* final_T;
     int32_t* n_contrib;
     unsigned long long* counts;  // kCount only: work counters (gs_raster_fwd_counted)
+    // kL1 only (gs_raster_fwd_l1): the L1 term of every rendered value against target
+    const float* target;
+    float* dL_dimage;
+    double* loss;
+    float inv_count;
+    double inv_count_d;
 };
 
 // Work counters of the counted variants (one atomic per warp at its end): pairs
@@ -358,7 +364,10 @@ __device__ __forceinline__ void add_counts(unsigned long long* counts, int evalu
     }
 }
 
-template <int PX, bool kCount>
+// kL1: the pixels' L1 terms against the target in the epilogue (gs_raster_fwd_l1):
+// dL/dimage = sign(image - target) / count, and the warp's sum of |image - target|
+// added to the loss with one double atomic, the arithmetic of gs_l1_loss_grad.
+template <int PX, bool kCount, bool kL1>
 __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster_fwd_kernel(const FwdArgs a) {
     constexpr int kPx = PX, kPairs = Layout<PX>::kPairs, kBoxH = Layout<PX>::kBoxH, kSub = Layout<PX>::kSub;
     __shared__ WarpStage stage[kWarps];
@@ -463,19 +472,36 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster
     }
     cp_async_wait_all();
     if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
+    double l1 = 0.0;  // kL1: this lane's sum of |image - target|
     if (x < a.W) {
 #pragma unroll
         for (int i = 0; i < kPx; ++i) {
             if (y0 + i < a.H) {
                 const int64_t pix = int64_t(y0 + i) * a.W + x;
                 const float Ti = i & 1 ? T[i / 2].y : T[i / 2].x;
-                a.image[3 * pix + 0] = __fmaf_rn(Ti, a.bg0, i & 1 ? Cr[i / 2].y : Cr[i / 2].x);
-                a.image[3 * pix + 1] = __fmaf_rn(Ti, a.bg1, i & 1 ? Cg[i / 2].y : Cg[i / 2].x);
-                a.image[3 * pix + 2] = __fmaf_rn(Ti, a.bg2, i & 1 ? Cb[i / 2].y : Cb[i / 2].x);
+                const float im[3] = {__fmaf_rn(Ti, a.bg0, i & 1 ? Cr[i / 2].y : Cr[i / 2].x),
+                                     __fmaf_rn(Ti, a.bg1, i & 1 ? Cg[i / 2].y : Cg[i / 2].x),
+                                     __fmaf_rn(Ti, a.bg2, i & 1 ? Cb[i / 2].y : Cb[i / 2].x)};
+#pragma unroll
+                for (int c = 0; c < 3; ++c) a.image[3 * pix + c] = im[c];
                 a.final_T[pix] = Ti;
                 a.n_contrib[pix] = last[i];
+                if (kL1) {
+#pragma unroll
+                    for (int c = 0; c < 3; ++c) {
+                        const float tg = __ldg(a.target + 3 * pix + c);
+                        const float d = im[c] - tg;
+                        l1 += fabs(double(im[c]) - double(tg));
+                        a.dL_dimage[3 * pix + c] = d > 0.f ? a.inv_count : (d < 0.f ? -a.inv_count : 0.f);
+                    }
+                }
             }
         }
+    }
+    if (kL1) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(kFull, l1, o);
+        if (lane == 0) atomicAdd(a.loss, l1 * a.inv_count_d);
     }
 }
 
@@ -780,7 +806,8 @@ cudaError_t launch_tile_order(const uint32_t* ranges, int tiles, uint32_t* order
 
 cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, const uint32_t* ranges,
                               const uint32_t* order, const CamArgs& cam, const float bg[3], float* image,
-                              float* final_T, int32_t* n_contrib, cudaStream_t s, unsigned long long* counts) {
+                              float* final_T, int32_t* n_contrib, cudaStream_t s, unsigned long long* counts,
+                              const L1Out* l1) {
     FwdArgs a;
     a.xy = reinterpret_cast<const float2*>(proj.xy);
     a.con = reinterpret_cast<const float4*>(proj.conic_opacity);
@@ -799,18 +826,28 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
     a.final_T = final_T;
     a.n_contrib = n_contrib;
     a.counts = counts;
+    a.target = l1 ? l1->target : nullptr;
+    a.dL_dimage = l1 ? l1->dL_dimage : nullptr;
+    a.loss = l1 ? l1->loss : nullptr;
+    const int64_t count = int64_t(3) * cam.W * cam.H;
+    a.inv_count = float(1.0 / double(count));
+    a.inv_count_d = 1.0 / double(count);
     if (a.tiles >= kWideLayoutTiles) {
         const unsigned grid = unsigned(a.tiles * Layout<8>::kSub);
         if (counts)
-            raster_fwd_kernel<8, true><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<8, true, false><<<grid, kWarps * 32, 0, s>>>(a);
+        else if (l1)
+            raster_fwd_kernel<8, false, true><<<grid, kWarps * 32, 0, s>>>(a);
         else
-            raster_fwd_kernel<8, false><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<8, false, false><<<grid, kWarps * 32, 0, s>>>(a);
     } else {
         const unsigned grid = unsigned(a.tiles * Layout<4>::kSub);
         if (counts)
-            raster_fwd_kernel<4, true><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<4, true, false><<<grid, kWarps * 32, 0, s>>>(a);
+        else if (l1)
+            raster_fwd_kernel<4, false, true><<<grid, kWarps * 32, 0, s>>>(a);
         else
-            raster_fwd_kernel<4, false><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<4, false, false><<<grid, kWarps * 32, 0, s>>>(a);
     }
     count_launches(1);
     return cudaGetLastError();

@@ -323,6 +323,15 @@ def raster_fwd(proj: Projected, view: View, bg=(0.0, 0.0, 0.0), radius: torch.Te
                       _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _stream())
 
 
+def raster_fwd_l1(proj: Projected, view: View, target: torch.Tensor, loss_dev: torch.Tensor, bg=(0.0, 0.0, 0.0),
+                  radius: torch.Tensor = None):
+    """raster_fwd and l1_loss_grad in one kernel: image, final_T, n_contrib, dL/dimage
+    into the view and loss_dev += mean |image - target|."""
+    abi.gs_raster_fwd_l1(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam, bg,
+                         _ptr(target), _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib),
+                         _ptr(view.dL_dimage), _ptr(loss_dev), _stream())
+
+
 def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), dL_dimage: torch.Tensor = None,
                radius: torch.Tensor = None):
     d = view.dL_dimage if dL_dimage is None else dL_dimage
@@ -645,11 +654,11 @@ class Trainer:
                 bin_sort_async(proj, view, self.kcount[k:k + 1], r)
             else:
                 bin_sort(proj, view, r)
-        raster_fwd(proj, view, self.bg, r)
         if self.ssim_weight > 0.0:
+            raster_fwd(proj, view, self.bg, r)
             l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
         else:
-            l1_loss_grad(view, target, self.loss)
+            raster_fwd_l1(proj, view, target, self.loss, self.bg, r)
         g2.zero_()
         raster_bwd(proj, view, g2, self.bg, radius=r)
 
@@ -725,11 +734,11 @@ class Trainer:
         """raster forward -> loss -> raster backward of an already binned view k."""
         view = self.views[k]
         r = self._radius(k)
-        raster_fwd(proj, view, self.bg, r)
         if self.ssim_weight > 0.0:
+            raster_fwd(proj, view, self.bg, r)
             l1_dssim_loss_grad(view, target, self.loss, 1.0, self.ssim_weight)
         else:
-            l1_loss_grad(view, target, self.loss)
+            raster_fwd_l1(proj, view, target, self.loss, self.bg, r)
         self.grad2ds[k].zero_()
         raster_bwd(proj, view, self.grad2ds[k], self.bg, radius=r)
 

@@ -301,6 +301,19 @@ gs_status gs_raster_fwd(const gs_projected* proj, const uint32_t* vals, const ui
                         const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,
                         float* final_T, int32_t* n_contrib, void* stream);
 
+/* gs_raster_fwd_l1 -- gs_raster_fwd followed by gs_l1_loss_grad on the image it
+ * renders, in one kernel: the compositing writes image, final_T and n_contrib as
+ * gs_raster_fwd does, and each pixel then takes its L1 term against target
+ * ([H][W][3] float, 4-byte aligned): dL_dimage ([H][W][3], 4-byte aligned) =
+ * sign(image - target) / (3 H W) (sign(0) = 0), and *loss_dev (one double, 8-byte
+ * aligned) += mean |image - target|.  Image, final_T, n_contrib and dL_dimage equal
+ * the two calls' bit for bit; the loss is their sum up to the order of its double
+ * additions.  Saves the image's second read, the L1 kernel and its launch. */
+gs_status gs_raster_fwd_l1(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
+                           const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, const float* target,
+                           float* image, float* final_T, int32_t* n_contrib, float* dL_dimage, double* loss_dev,
+                           void* stream);
+
 /* gs_raster_bwd -- the reverse of gs_raster_fwd for an upstream dL/dimage
  * [H][W][3]: per pixel, back to front from n_contrib, the transmittance in front
  * of each blended entry is recovered from final_T, and with S the colour blended

@@ -319,3 +319,41 @@ def test_backward_grad2d_with_a_background(orc, bg):
     assert len(rows) > 900
     for q, name in enumerate(["du", "dv", "dA", "dB", "dC", "do", "dr", "dg", "db"]):
         check_grads(g2_gpu[:, q], g2[:, q], name, rows=rows, ref_abs=g2a[:, q], max_bad_frac=0.002)
+
+
+@pytest.mark.parametrize("size", [(100, 37), (1920, 1080)])   # the narrow-tile layout with ragged edges; the wide one
+def test_forward_with_l1_equals_forward_then_l1(orc, size):
+    """gs_raster_fwd_l1 (the L1 term in the forward kernel's epilogue) against
+    gs_raster_fwd followed by gs_l1_loss_grad: image, final_T, n_contrib and
+    dL/dimage bit-exact, the loss equal up to the order of its double sums, and
+    both against the oracle's L1 of the rendered image."""
+    W, H = size
+    rng = np.random.default_rng(11)
+    scene = scenes.random_scene(rng, 1500, 1, log_scale=(-3.5, -1.5))
+    R, t = scenes.look_at((0.3, -0.2, -4.0))
+    f = 0.9 * W
+    cam = scenes.camera(R, t, f, f, 0.5 * W - 0.3, 0.5 * H + 0.2, W, H)
+    bg = (0.1, 0.3, 0.6)
+    run = CudaRun(scene, cam, bg=bg)     # runs gs_raster_fwd
+    v = run.view
+    img, T, nc = v.image.clone(), v.final_T.clone(), v.n_contrib.clone()
+    target = torch.from_numpy(rng.random((H, W, 3), dtype=np.float32)).cuda()
+    target.view(-1)[:64] = img.view(-1)[:64]      # sign(0) = 0
+    loss_a = torch.zeros(1, dtype=torch.float64, device="cuda")
+    pl.l1_loss_grad(v, target, loss_a)
+    torch.cuda.synchronize()
+    g_a = v.dL_dimage.clone()
+    v.image.fill_(-1.0)
+    v.final_T.fill_(-1.0)
+    v.n_contrib.fill_(-1)
+    v.dL_dimage.fill_(7.0)
+    loss_b = torch.full((1,), 0.25, dtype=torch.float64, device="cuda")    # accumulates onto what is there
+    pl.raster_fwd_l1(run.proj, v, target, loss_b, bg)
+    torch.cuda.synchronize()
+    assert torch.equal(v.image, img) and torch.equal(v.final_T, T) and torch.equal(v.n_contrib, nc)
+    assert torch.equal(v.dL_dimage, g_a)
+    assert abs((loss_b.item() - 0.25) - loss_a.item()) <= 1e-12 * loss_a.item()
+    want_loss, want_g = orc.l1(img.cpu().numpy(), target.cpu().numpy())
+    assert np.array_equal(g_a.cpu().numpy(), want_g)
+    assert abs(loss_a.item() - want_loss) <= 1e-12 * want_loss
+    assert (nc > 0).float().mean().item() > 0.05
