@@ -344,7 +344,7 @@ def run_render(args, world, rank, local):
     wl = make_workload(args.workload, args.views)
     scene, cams = wl.scene, wl.cameras
     g = pl.Gaussians.from_scene(scene)
-    view = pl.View(scene.n, cams[0])
+    view = pl.View(scene.n, cams[0], tile_cull=not args.no_tile_cull)
     proj = pl.Projected(scene.n)
     stream = torch.cuda.current_stream()
     # size the instance buffers for the largest pose
@@ -411,6 +411,7 @@ def run_render(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "gaussians": scene.n, "poses_per_step": len(cams),
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
+                       "tile_cull": not args.no_tile_cull,
                        "parallelism": f"replicas x{world}",
                        "l2": "a step renders every pose once; the instance lists of a pose exceed L2"},
             "stages_ms_per_frame": {"raster_fwd": fwd_ms, "frame": ms / frames},
@@ -446,7 +447,8 @@ def run_ours(args, world, rank, local):
     lrs = dict(wl.adam_lr) if wl.adam_lr else {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3,
                                                   "opacity_logits": 5e-2, "sh": 2.5e-3}
     tr = pl.Trainer(gauss, views, [targets[i] for i in range(nv)], lrs, densify=True, streams=args.streams,
-                    batched_sort=not args.per_view_sort, groups=args.groups, bin_views=not args.per_view_bin)
+                    batched_sort=not args.per_view_sort, groups=args.groups, bin_views=not args.per_view_bin,
+                    tile_cull=not args.no_tile_cull)
     stream = torch.cuda.current_stream()
 
     # warm-up (also sizes every view's instance buffers)
@@ -529,8 +531,11 @@ def run_ours(args, world, rank, local):
             "config": {"workload": wl.name, "gaussians": scene.n, "views_per_step": nv, "streams": args.streams,
                        "depth_sort": "per view" if args.per_view_sort else "batched over the views" + (
                            f", in {len(tr.view_groups())} pipelined view groups" if len(tr.view_groups()) > 1 else ""),
-                       "binning": "per view" if (args.per_view_bin or args.per_view_sort) else
-                                  "one launch per kernel for all the views of a group",
+                       "binning": ("per view" if (args.per_view_bin or args.per_view_sort) else
+                                   "one launch per kernel for all the views of a group") +
+                                  ("; each Gaussian in the tiles its footprint reaches" if tr.tile_cull else
+                                   "; each Gaussian in every tile of its 3-sigma rectangle"),
+                       "tile_cull": bool(tr.tile_cull),
                        "image": f"{cam0['width']}x{cam0['height']}", "sh_degree": scene.sh_degree,
                        "mean_instances_per_view": int(np.mean([s[0] for s in stats])),
                        "parallelism": f"replicas x{world}",
@@ -557,7 +562,8 @@ def run_ours(args, world, rank, local):
                         "l1_dssim": measure_dssim(tr, wl, peaks, torch, with_oracle),
                         "absgrad_and_sparse_adam": measure_variants(tr, torch),
                         "packed": measure_packed(tr, wl, peaks, torch),
-                        "sh16": measure_sh16(tr, wl, peaks, torch)}
+                        "sh16": measure_sh16(tr, wl, peaks, torch),
+                        "tile_cull": measure_tile_cull(tr, wl, torch)}
         # the two options where they are meant to pay: packed views that keep a small part
         # of the scene, FP16 SH on a single-view step
         torch.cuda.empty_cache()
@@ -674,12 +680,13 @@ def measure_packed(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     s = torch.cuda.current_stream()
     scene = wl.scene
     trp = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, packed=True)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, packed=True,
+                     tile_cull=tr.tile_cull)
 
     # the unpacked arm starts from the same scene (the benchmark's own Trainer has
     # trained for many steps by now, and its Gaussians have moved)
     tru = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, tile_cull=tr.tile_cull)
     ms_packed, ms_unpacked = paired_step_ms(trp, tru, steps, torch)
     del tru
     res = {"step_ms_packed": ms_packed, "step_ms_unpacked": ms_unpacked}
@@ -798,7 +805,8 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
     s = torch.cuda.current_stream()
     scene = wl.scene
     trh = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, sh16=True)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, sh16=True,
+                     tile_cull=tr.tile_cull)
 
     def timed(fn, count):
         for _ in range(3):
@@ -812,7 +820,7 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
         return e0.elapsed_time(e1) / count
 
     trf = pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
-                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups)
+                     dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, tile_cull=tr.tile_cull)
     ms_sh16, ms_f32 = paired_step_ms(trh, trf, steps, torch)
     del trf
     res = {"step_ms_sh16": ms_sh16, "step_ms_f32": ms_f32}
@@ -828,6 +836,29 @@ def measure_sh16(tr, wl, peaks, torch, steps: int = 5, reps: int = 10):
                                            "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes}
     del trh
     return res
+
+
+def measure_tile_cull(tr, wl, torch, steps: int = 5):
+    """Binning each Gaussian only into the tiles its footprint reaches (gs_camera.tile_cull)
+    against binning it into its whole 3-sigma rectangle: the training step of two Trainers
+    started from the same scene (paired_step_ms), the other settings those of the timed
+    Trainer, and the instances per view."""
+    from gaussian_splatting_differentiable_02_b200 import pipeline as pl
+    scene = wl.scene
+
+    def make(cull):
+        return pl.Trainer(pl.Gaussians.from_scene(scene), [pl.View(scene.n, c) for c in wl.cameras], tr.targets,
+                          dict(tr.lrs), densify=True, streams=tr.streams, groups=tr.groups, bin_views=tr.bin_views,
+                          tile_cull=cull)
+
+    on, off = make(True), make(False)
+    ms_on, ms_off = paired_step_ms(on, off, steps, torch)
+    k_on = float(on.kcount.double().mean().item())
+    k_off = float(off.kcount.double().mean().item())
+    del on, off
+    torch.cuda.empty_cache()
+    return {"step_ms_culled": ms_on, "step_ms_rectangles": ms_off, "instances_per_view_culled": k_on,
+            "instances_per_view_rectangles": k_off, "instances_kept": k_on / k_off}
 
 
 def measure_dssim(tr, wl, peaks, torch, with_oracle: bool, reps: int = 10):
@@ -1244,6 +1275,9 @@ def main(argv=None):
                          "the compositing of the groups before it)")
     ap.add_argument("--per-view-bin", action="store_true",
                     help="bin each view with its own launches instead of one launch per kernel for a view group")
+    ap.add_argument("--no-tile-cull", action="store_true",
+                    help="bin each Gaussian into every tile of its 3-sigma rectangle instead of only the tiles "
+                         "where its alpha can reach 1/255")
     ap.add_argument("--per-view-sort", action="store_true",
                     help="sort each view on its own stream instead of one batched depth sort of all views")
     ap.add_argument("--views", type=int, default=16,

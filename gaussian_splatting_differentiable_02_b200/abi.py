@@ -35,7 +35,7 @@ class GsError(RuntimeError):
 class gs_camera(C.Structure):
     _fields_ = [("R", C.c_float * 9), ("t", C.c_float * 3), ("fx", C.c_float), ("fy", C.c_float),
                 ("cx", C.c_float), ("cy", C.c_float), ("width", C.c_int32), ("height", C.c_int32),
-                ("near_plane", C.c_float), ("eps2d", C.c_float)]
+                ("near_plane", C.c_float), ("eps2d", C.c_float), ("tile_cull", C.c_int32)]
 
 
 class gs_params(C.Structure):
@@ -177,8 +177,9 @@ def _check(status: int):
     return status
 
 
-def make_camera(cam: dict) -> gs_camera:
-    """gs_camera from a scene camera dict (R 3x3 row-major, t, fx, fy, cx, cy, width, height, near, eps2d)."""
+def make_camera(cam: dict, tile_cull: bool = False) -> gs_camera:
+    """gs_camera from a scene camera dict (R 3x3 row-major, t, fx, fy, cx, cy, width, height, near, eps2d);
+    tile_cull bins each Gaussian only into the tiles its footprint reaches."""
     c = gs_camera()
     R = [float(v) for v in np.asarray(cam["R"], np.float32).reshape(9)]
     t = [float(v) for v in np.asarray(cam["t"], np.float32).reshape(3)]
@@ -190,6 +191,7 @@ def make_camera(cam: dict) -> gs_camera:
     c.width, c.height = int(cam["width"]), int(cam["height"])
     c.near_plane = cam.get("near", 0.2)
     c.eps2d = cam.get("eps2d", 0.3)
+    c.tile_cull = int(tile_cull)
     return c
 
 

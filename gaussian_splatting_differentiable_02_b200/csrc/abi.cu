@@ -30,6 +30,7 @@ CamArgs make_cam(const gs_camera& c) {
     k.H = c.height;
     k.TX = (c.width + kTile - 1) / kTile;
     k.TY = (c.height + kTile - 1) / kTile;
+    k.tile_cull = c.tile_cull;
     k.limx = 1.3 * (0.5 * double(c.width) / k.fx);
     k.limy = 1.3 * (0.5 * double(c.height) / k.fy);
     for (int j = 0; j < 3; ++j) k.cc[j] = -((k.R[0 + j] * k.t[0] + k.R[3 + j] * k.t[1]) + k.R[6 + j] * k.t[2]);
@@ -95,6 +96,8 @@ gs_status check_camera(const char* fn, const gs_camera* cam) {
     if (!(cam->fx > 0.f) || !(cam->fy > 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: focal lengths must be > 0", fn);
     if (!(cam->near_plane > 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: near_plane must be > 0", fn);
     if (!(cam->eps2d >= 0.f)) return fail(GS_ERR_INVALID_ARG, "%s: eps2d must be >= 0", fn);
+    if (cam->tile_cull != 0 && cam->tile_cull != 1)
+        return fail(GS_ERR_INVALID_ARG, "%s: tile_cull must be 0 or 1", fn);
     return GS_OK;
 }
 
@@ -207,10 +210,9 @@ gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_
 }
 
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam) {
-    (void)cam;
     if (n < 0) n = 0;
     if (capacity < 0) capacity = 0;
-    return gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+    return gsk::sort_workspace_layout(n, capacity, cam && cam->tile_cull == 1, nullptr, nullptr);
 }
 
 }  // extern "C"
@@ -236,14 +238,14 @@ gs_status bin_sort_impl(const char* fn, const gs_projected* proj, int64_t n, con
         CHECK_PTR(keys, 8);
         CHECK_PTR(vals, 4);
     }
-    const size_t need = gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+    const size_t need = gsk::sort_workspace_layout(n, capacity, cam->tile_cull == 1, nullptr, nullptr);
     if (workspace_bytes < need)
         return fail(GS_ERR_INVALID_ARG, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
     const int64_t tiles = int64_t((cam->width + GS_TILE - 1) / GS_TILE) * ((cam->height + GS_TILE - 1) / GS_TILE);
     if (tiles > (int64_t(1) << 20)) return fail(GS_ERR_UNSUPPORTED, "%s: more than 2^20 tiles", fn);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     gsk::SortWorkspace ws;
-    gsk::sort_workspace_layout(n, capacity, workspace, &ws);
+    gsk::sort_workspace_layout(n, capacity, cam->tile_cull == 1, workspace, &ws);
     const gsk::CamArgs c = gsk::make_cam(*cam);
     cudaError_t e = order ? gsk::launch_bin_sort_ordered(*proj, n, order, c, ws, keys, vals, capacity, tile_ranges,
                                                          count_dev, s)
@@ -328,11 +330,12 @@ gs_status gs_bin_sort_ordered_views_async(const gs_projected* projs, int32_t num
             CHECK_PTR(keys[v], 8);
             CHECK_PTR(vals[v], 4);
         }
-        const size_t need = gsk::sort_workspace_layout(n, capacity, nullptr, nullptr);
+        const bool cull = cams[v].tile_cull == 1;
+        const size_t need = gsk::sort_workspace_layout(n, capacity, cull, nullptr, nullptr);
         if (workspace_bytes[v] < need)
             return fail(GS_ERR_INVALID_ARG, "%s: workspace of view %d has %zu bytes, %zu needed", fn, v,
                         workspace_bytes[v], need);
-        gsk::sort_workspace_layout(n, capacity, workspaces[v], &ws[v]);
+        gsk::sort_workspace_layout(n, capacity, cull, workspaces[v], &ws[v]);
         ord[v] = n > 0 ? orders + int64_t(v) * n : nullptr;
         cnt[v] = reinterpret_cast<unsigned long long*>(num_instances_dev[v]);
     }

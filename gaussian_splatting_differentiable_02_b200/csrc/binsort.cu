@@ -25,12 +25,16 @@
 //                     block (warp votes + per-warp counters), reorder in shared
 //                     memory, coalesced scatter; the final tile pass writes
 //                     64-bit keys
-//   count_sorted      per-block sum of tiles_touched in depth order
+//   count_sorted      per-block sum of tiles_touched in depth order (culled
+//                     binning: of the tiles each footprint reaches, with the
+//                     runs of tiles of its first rows kept for emit)
 //   scan_blocks       one CTA: exclusive scan of the block sums, total K
 //   emit              every visible Gaussian, in depth order, writes its
-//                     instances (row-major over its tile rectangle)
+//                     instances (row-major over its tile rectangle, or its
+//                     runs of tiles)
 //   ranges            [begin, end) of each tile in the sorted keys
 #include "internal.cuh"
+#include "tile_reach.cuh"
 
 namespace gsk {
 namespace {
@@ -42,6 +46,11 @@ constexpr int kEmitBlock = 256;
 constexpr int kEmitPerThread = GS_EMIT_ITEMS;
 constexpr int kEmitChunk = kEmitBlock * kEmitPerThread;  // Gaussians per emit block
 static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halves a power of two");
+// rows of a culled Gaussian whose runs of tiles the count pass keeps for the
+// emission (32 bytes a Gaussian; 96% of the 1080p instances of the 1M mixture
+// belong to Gaussians of at most 8 rows)
+constexpr int kRunRows = 8;
+static_assert(kRunRows % 4 == 0, "runs move as uint4");
 
 #ifndef GS_SORT_ITEMS
 #define GS_SORT_ITEMS 8
@@ -279,6 +288,10 @@ __global__ void __launch_bounds__(kSortBlock, GS_SORT_MIN_BLOCKS) downsweep_kern
 struct EmitSeg {
     const uint32_t* touched;
     const uint2* rect;
+    const float2* xy;  // culled binning: the footprints (tile_reach.cuh)
+    const float4* con;
+    uint32_t* runs;    // culled binning (else null): [n][kRunRows] runs of the first rows, depth order
+    uint32_t* cnt;     // culled binning: [n] instances of each Gaussian, depth order
     const uint32_t* order;           // [n] the view's depth order
     unsigned long long* block_sums;  // [nb_emit]
     unsigned long long* total;       // the view's instance count K
@@ -297,13 +310,55 @@ struct EmitArgs {
     int64_t tiles;
 };
 
+// The culled binning's instances of the Gaussian at depth-order position i:
+// the runs of tiles its footprint reaches in each row of its rectangle
+// (tile_reach.cuh).  The first kRunRows rows' runs are kept for the emission as
+// (first column << 16 | length); returns the count over all rows.
+__device__ __forceinline__ uint32_t culled_runs(const EmitSeg& g, int64_t i, uint32_t gid) {
+    const uint2 r = __ldg(g.rect + gid);
+    const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu), y1 = int(r.y >> 16);
+    const TileReach R = tile_reach_setup(__ldg(g.xy + gid), __ldg(g.con + gid));
+    uint32_t w[kRunRows];
+    uint32_t c = 0;
+#pragma unroll
+    for (int k = 0; k < kRunRows; ++k) {
+        w[k] = 0u;
+        if (y0 + k < y1) {
+            int c0, c1;
+            tile_reach_row(R, y0 + k, x0, x1, &c0, &c1);
+            w[k] = (uint32_t(c0) << 16) | uint32_t(c1 - c0);
+            c += uint32_t(c1 - c0);
+        }
+    }
+    for (int y = y0 + kRunRows; y < y1; ++y) {
+        int c0, c1;
+        tile_reach_row(R, y, x0, x1, &c0, &c1);
+        c += uint32_t(c1 - c0);
+    }
+    uint4* out = reinterpret_cast<uint4*>(g.runs + i * kRunRows);
+    out[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    out[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    return c;
+}
+
+// Per block of kEmitChunk depth-ordered Gaussians, the sum of their instance
+// counts: tiles_touched, or in the culled binning the counts of culled_runs
+// (stored with the runs for the emission).
 __global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const __grid_constant__ EmitArgs a) {
     const EmitSeg& g = a.seg[blockIdx.y];
     const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
     unsigned long long sum = 0;
     for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
         const int64_t i = base + k;
-        if (i < a.n) sum += __ldg(g.touched + __ldg(g.order + i));
+        if (i < a.n) {
+            const uint32_t gid = __ldg(g.order + i);
+            uint32_t t = __ldg(g.touched + gid);
+            if (g.runs) {
+                if (t) t = culled_runs(g, i, gid);
+                g.cnt[i] = t;
+            }
+            sum += t;
+        }
     }
     unsigned long long tot;
     block_excl_scan(sum, &tot);
@@ -331,12 +386,17 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const __grid_constant
 // Instances of the block's Gaussians (depth order), load-balanced: the block's
 // output slots [0, total) are dealt to its threads round-robin, and each slot
 // finds its Gaussian by a binary search over the block's exclusive offsets in
-// shared memory, then its tile from its index inside the Gaussian's tile
-// rectangle (row-major).  Consecutive slots are written by consecutive threads.
+// shared memory, then its tile: from its index inside the Gaussian's tile
+// rectangle (row-major) when the Gaussian covers all of it, else (culled
+// binning) from the runs of tiles count_sorted kept for its first rows, and
+// past those rows from tile_reach_row again.  Consecutive slots are written by
+// consecutive threads.
 __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const __grid_constant__ EmitArgs a) {
     __shared__ uint32_t s_start[kEmitChunk];
     __shared__ uint32_t s_gid[kEmitChunk];
     __shared__ uint2 s_rect[kEmitChunk];
+    __shared__ unsigned char s_walk[kEmitChunk];
+    __shared__ uint4 s_runs[kEmitChunk][kRunRows / 4];
     const EmitSeg& g = a.seg[blockIdx.y];
     if (g.inst.get() == 0) return;  // nothing fits: emit nothing
     const int64_t first = int64_t(blockIdx.x) * kEmitChunk + int64_t(threadIdx.x) * kEmitPerThread;
@@ -345,7 +405,7 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const __grid_constant_
 #pragma unroll
     for (int k = 0; k < kEmitPerThread; ++k) {
         gid[k] = first + k < a.n ? __ldg(g.order + first + k) : 0u;
-        tt[k] = first + k < a.n ? __ldg(g.touched + gid[k]) : 0u;
+        tt[k] = first + k < a.n ? (g.runs ? __ldg(g.cnt + first + k) : __ldg(g.touched + gid[k])) : 0u;
         mine += tt[k];
     }
     unsigned long long total;
@@ -356,7 +416,16 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const __grid_constant_
         const int idx = threadIdx.x * kEmitPerThread + k;
         s_start[idx] = run;
         s_gid[idx] = gid[k];
-        s_rect[idx] = tt[k] ? __ldg(g.rect + gid[k]) : make_uint2(0u, 0u);
+        const uint2 r = tt[k] ? __ldg(g.rect + gid[k]) : make_uint2(0u, 0u);
+        s_rect[idx] = r;
+        const uint32_t area = ((r.y & 0xffffu) - (r.x & 0xffffu)) * ((r.y >> 16) - (r.x >> 16));
+        const bool walk = g.runs && tt[k] != 0u && tt[k] != area;
+        s_walk[idx] = walk;
+        if (walk) {
+            const uint4* src = reinterpret_cast<const uint4*>(g.runs + (first + k) * kRunRows);
+#pragma unroll
+            for (int q = 0; q < kRunRows / 4; ++q) s_runs[idx][q] = __ldg(src + q);
+        }
         run += tt[k];
     }
     __syncthreads();
@@ -368,8 +437,46 @@ __global__ void __launch_bounds__(kEmitBlock) emit_kernel(const __grid_constant_
             if (s_start[lo + step] <= slot) lo += step;
         const uint32_t j = slot - s_start[lo];
         const uint2 r = s_rect[lo];
-        const uint32_t x0 = r.x & 0xffffu, y0 = r.x >> 16, w = (r.y & 0xffffu) - x0;
-        const uint32_t ty = y0 + j / w, tx = x0 + j % w;
+        const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu), y1 = int(r.y >> 16);
+        uint32_t tx, ty;
+        if (!s_walk[lo]) {
+            const uint32_t w = uint32_t(x1 - x0);
+            ty = uint32_t(y0) + j / w;
+            tx = uint32_t(x0) + j % w;
+        } else {
+            // a count that matches no walk (tiles_touched written under another
+            // rule) leaves tile 0: a valid tile id, never a range written out of bounds
+            tx = 0u;
+            ty = 0u;
+            uint32_t rest = j;
+            bool found = false;
+            const uint32_t* rr = reinterpret_cast<const uint32_t*>(s_runs[lo]);
+#pragma unroll
+            for (int k = 0; k < kRunRows; ++k) {
+                const uint32_t m = rr[k] & 0xffffu;  // 0 past the rectangle's last row
+                if (!found && rest < m) {
+                    tx = (rr[k] >> 16) + rest;
+                    ty = uint32_t(y0 + k);
+                    found = true;
+                }
+                if (!found) rest -= m;
+            }
+            if (!found && y1 - y0 > kRunRows) {
+                const uint32_t gg = s_gid[lo];
+                const TileReach R = tile_reach_setup(__ldg(g.xy + gg), __ldg(g.con + gg));
+                for (int y = y0 + kRunRows; y < y1; ++y) {
+                    int c0, c1;
+                    tile_reach_row(R, y, x0, x1, &c0, &c1);
+                    const uint32_t m = uint32_t(c1 - c0);
+                    if (rest < m) {
+                        tx = uint32_t(c0) + rest;
+                        ty = uint32_t(y);
+                        break;
+                    }
+                    rest -= m;
+                }
+            }
+        }
         g.tkey[base + slot] = ty * uint32_t(a.tiles_x) + tx;
         g.tval[base + slot] = s_gid[lo];
     }
@@ -426,7 +533,7 @@ int64_t sort_blocks(int64_t slots) { return (slots + kSortTile - 1) / kSortTile;
 
 }  // namespace
 
-size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws) {
+size_t sort_workspace_layout(int64_t n, int64_t capacity, bool cull, void* base, SortWorkspace* ws) {
     const int64_t nb_emit = (n + kEmitChunk - 1) / kEmitChunk;
     const int64_t slots = capacity > n ? capacity : n;  // the depth sort borrows the tile buffers
     const int64_t nb_sort = (slots + kSortTile - 1) / kSortTile;
@@ -449,6 +556,14 @@ size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorksp
     off += align_up(sizeof(uint32_t) * 256 * size_t(nb_sort > 0 ? nb_sort : 1));
     w.digit_totals = reinterpret_cast<uint32_t*>(b + off);
     off += align_up(sizeof(uint32_t) * 256);
+    w.runs = nullptr;
+    w.cnt = nullptr;
+    if (cull) {
+        w.runs = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * kRunRows * size_t(n > 0 ? n : 1));
+        w.cnt = reinterpret_cast<uint32_t*>(b + off);
+        off += align_up(sizeof(uint32_t) * size_t(n > 0 ? n : 1));
+    }
     if (ws) *ws = w;
     return off;
 }
@@ -568,6 +683,10 @@ cudaError_t launch_bin_sort_ordered_views(int views, const gs_projected* projs, 
         EmitSeg& g = e.seg[v];
         g.touched = projs[v].tiles_touched;
         g.rect = reinterpret_cast<const uint2*>(projs[v].rect);
+        g.xy = reinterpret_cast<const float2*>(projs[v].xy);
+        g.con = reinterpret_cast<const float4*>(projs[v].conic_opacity);
+        g.runs = ws[v].runs;
+        g.cnt = ws[v].cnt;
         g.order = orders[v];
         g.block_sums = ws[v].block_sums;
         g.total = ws[v].total;

@@ -43,7 +43,8 @@ cudaError_t scratch_address(void** out) {
 extern "C" gs_status gs_bin_sort_static(const gs_projected* proj, int64_t n, const gs_camera* cam, uint64_t* keys,
                                         uint32_t* vals, int64_t capacity, int64_t* num_instances_host,
                                         uint32_t* tile_ranges, void* stream) {
-    const size_t need = gsk::sort_workspace_layout(n < 0 ? 0 : n, capacity < 0 ? 0 : capacity, nullptr, nullptr);
+    const size_t need = gsk::sort_workspace_layout(n < 0 ? 0 : n, capacity < 0 ? 0 : capacity,
+                                                   cam && cam->tile_cull == 1, nullptr, nullptr);
     if (n >= 0 && capacity >= 0 && need > size_t(GS_STATIC_SCRATCH_BYTES))
         return gsk::fail_detail(GS_ERR_UNSUPPORTED,
                                 "gs_bin_sort_static: n = %lld and capacity = %lld need %zu bytes of scratch; the "

@@ -20,6 +20,7 @@ struct CamArgs {
     double limx, limy;  // 1.3 x half field of view, in x/z and y/z
     double cc[3];       // camera centre -R^T t
     int W, H, TX, TY;
+    int tile_cull;  // the binning emits only the tiles each footprint reaches (tile_reach.cuh)
 };
 
 CamArgs make_cam(const gs_camera& c);
@@ -101,9 +102,11 @@ struct SortWorkspace {
     uint32_t* tval[2];               // [max(capacity, n)] Gaussian indices, ping-pong
     uint32_t* hist;                  // [256][nb_sort]
     uint32_t* digit_totals;          // [256]
+    uint32_t* runs;                  // culled binning (gs_camera.tile_cull), else null: [n][8] runs of tiles
+    uint32_t* cnt;                   // culled binning: [n] instances per Gaussian, depth order
     int64_t nb_emit, nb_sort;
 };
-size_t sort_workspace_layout(int64_t n, int64_t capacity, void* base, SortWorkspace* ws);
+size_t sort_workspace_layout(int64_t n, int64_t capacity, bool cull, void* base, SortWorkspace* ws);
 
 // Enqueues the whole binning and sort; the instance count stays on the device
 // (ws.total, and *count_out when given).  K > capacity: nothing emitted, ranges empty.

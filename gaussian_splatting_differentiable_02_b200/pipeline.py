@@ -182,9 +182,10 @@ def project_packed(g: Gaussians, view: View, packed: Packed, workspace: torch.Te
 class View:
     """Per-camera buffers: sorted instances, tile ranges, image and its gradient."""
 
-    def __init__(self, n: int, cam: dict, device="cuda", capacity: int = 0):
+    def __init__(self, n: int, cam: dict, device="cuda", capacity: int = 0, tile_cull: bool = False):
         self.cam = cam
-        self.gcam = abi.make_camera(cam)
+        self.tile_cull = bool(tile_cull)
+        self.gcam = abi.make_camera(cam, self.tile_cull)
         self.n = n
         self.device = device
         self.tiles_x, self.tiles_y = abi.gs_tile_grid(self.gcam)
@@ -205,7 +206,16 @@ class View:
         if (cam["width"], cam["height"]) != (self.cam["width"], self.cam["height"]):
             raise ValueError("set_camera keeps the image size")
         self.cam = cam
-        self.gcam = abi.make_camera(cam)
+        self.gcam = abi.make_camera(cam, self.tile_cull)
+
+    def set_tile_cull(self, on: bool):
+        """Bin each Gaussian only into the tiles of its rectangle that its footprint
+        reaches (gs_camera.tile_cull), or into the whole rectangle."""
+        self.tile_cull = bool(on)
+        self.gcam = abi.make_camera(self.cam, self.tile_cull)
+        nbytes = abi.gs_bin_sort_workspace_bytes(self.n, self.capacity, self.gcam)   # the culled binning's runs
+        if nbytes > self.workspace.numel():
+            self.workspace = torch.zeros((nbytes,), device=self.device, dtype=torch.uint8)
 
     def set_n(self, n: int):
         """Resize for a new Gaussian (or packed slot) count: the sort workspace depends on n.
@@ -514,6 +524,9 @@ class Trainer:
                                # coefficients, which the fused Adam step refreshes from the float32 ones
     bin_views: bool = True     # fused batched path: each view group's binning (emission, passes by tile,
                                # ranges) launched once for all its views instead of once per view
+    tile_cull: bool = True     # every view bins a Gaussian only into the tiles of its rectangle where its
+                               # alpha can reach 1/255 (gs_camera.tile_cull): the same images and gradients
+                               # from about half the instances of the 3-sigma rectangles
     graph: bool = False        # fused path: the views' part of a step (projections, sorts, compositing,
                                # losses and their backward) is captured once into a CUDA graph and
                                # replayed every step, so its few-microsecond launches cost no host time
@@ -524,6 +537,8 @@ class Trainer:
         n = self.gauss.n
         dev = self.gauss.means.device
         self.fused = self.fused and len(self.views) <= abi.GS_MAX_VIEWS
+        for vw in self.views:
+            vw.set_tile_cull(self.tile_cull)
         if self.packed and not (self.fused and self.batched_sort):
             raise ValueError("packed=True runs on the fused path with the batched sort")
         if self.sh16 and (self.packed or not self.fused):

@@ -53,7 +53,21 @@ typedef int32_t gs_status;
  * axes (x right, y down, z forward).  Pixel (x, y) samples the image plane at
  * (x + 0.5, y + 0.5).  Gaussians with camera depth <= near_plane are culled; eps2d
  * is added to both diagonal entries of every projected 2D covariance (the
- * screen-space low-pass of the original 3DGS rasterizer, 0.3). */
+ * screen-space low-pass of the original 3DGS rasterizer, 0.3).
+ *
+ * tile_cull (0 or 1; anything else is GS_ERR_INVALID_ARG) selects the tiles the
+ * binning calls put a visible Gaussian into:
+ *   0  every tile of its tile rectangle (tiles_touched of them);
+ *   1  only the tiles of the rectangle whose box of pixel centres, widened by
+ *      1/1024 px, meets the region where o e^-sigma >= 1/255 (alpha can pass
+ *      the compositing's skip test there), that bound taken with a margin of
+ *      1e-4 (|ln(255 o)| + 1): the culling stage of the MUSA co-design article
+ *      (qwbw.cn/news/278220 §1).  A conic that is not positive definite keeps
+ *      its whole rectangle; an opacity below about 1/255 gets no tile.
+ * The two give the same image, final_T and gradients (a dropped instance is
+ * skipped at every pixel of its tile); n_contrib counts positions in the
+ * lists actually binned.  The projection ignores the flag; a culled binning
+ * needs 36 bytes more workspace per Gaussian (gs_bin_sort_workspace_bytes). */
 typedef struct gs_camera {
     float R[9];
     float t[3];
@@ -61,6 +75,7 @@ typedef struct gs_camera {
     int32_t width, height;
     float near_plane;
     float eps2d;
+    int32_t tile_cull;
 } gs_camera;
 
 /* Gaussian parameters, stored pre-activation as the gsplat guide §3.3 sets
@@ -170,7 +185,8 @@ gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_
                            const uint16_t* sh_half, void* stream);
 
 /* Bytes of device workspace gs_bin_sort needs for n Gaussians and up to `capacity`
- * instances (16-byte aligned buffer, owned by the caller). */
+ * instances (16-byte aligned buffer, owned by the caller), with the camera's
+ * tile_cull (cam may be NULL: no culling). */
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam);
 
 /* gs_bin_sort -- tile binning.  Every visible Gaussian emits one instance per tile

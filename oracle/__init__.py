@@ -2,8 +2,10 @@
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 benchmark's CPU-baseline leg.  The product path (the CUDA library and its
-binding) never imports it.  The arithmetic lives in oracle.cpp; this module
-only marshals numpy arrays through ctypes.
+binding) never imports it.  The arithmetic lives in oracle.cpp, which this
+module calls through ctypes, except for a few short numpy formulas written
+out here (the L1 + D-SSIM combination, the tile-reach bound of the culled
+binning).
 
 Parity status: every function here is pinned by tests/test_oracle_*.py against
 closed forms, invariants, brute force, a library routine (scipy's spherical
@@ -308,3 +310,69 @@ def l1_dssim(image, target, l1_weight: float = 1.0, ssim_weight: float = 0.2):
     s, _, gs = ssim(img, tgt, want_grad=True)
     g = l1_weight * np.sign(img - tgt) / n - ssim_weight * gs
     return l1_weight * l1v + ssim_weight * (1.0 - s), g
+
+
+def tile_min_sigma(xy, conic, tx, ty, widen: float = 0.0):
+    """Smallest sigma = 1/2 (A dx^2 + C dy^2) + B dx dy (dx = x - u, dy = y - v) over the
+    box of pixel centres of tile (tx, ty), [16 tx + 0.5 - widen, 16 tx + 15.5 + widen] in x
+    and the same in y, for every row of xy [m, 2] and conic [m, 3] (A, B, C), in float64.
+
+    For a positive definite form the minimum over the box is 0 when the mean lies in
+    it; otherwise it lies on the box's boundary, and along an edge (one coordinate
+    fixed) sigma is a parabola in the other coordinate, smallest at its vertex
+    clamped to the edge.  Rows whose form is not positive definite get NaN."""
+    xy = np.asarray(xy, np.float64).reshape(-1, 2)
+    con = np.asarray(conic, np.float64).reshape(-1, 3)
+    u, v = xy[:, 0], xy[:, 1]
+    A, B, Cc = con[:, 0], con[:, 1], con[:, 2]
+    x0 = 16.0 * np.asarray(tx, np.float64) + 0.5 - widen
+    x1 = 16.0 * np.asarray(tx, np.float64) + 15.5 + widen
+    y0 = 16.0 * np.asarray(ty, np.float64) + 0.5 - widen
+    y1 = 16.0 * np.asarray(ty, np.float64) + 15.5 + widen
+    pd = (A > 0) & (Cc > 0) & (A * Cc - B * B > 0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        def sig(dx, dy):
+            return 0.5 * (A * dx * dx + Cc * dy * dy) + B * dx * dy
+        best = np.full(len(u), np.inf)
+        for xe in (x0, x1):   # x fixed: d sigma / d dy = B dx + C dy = 0
+            dx = xe - u
+            yc = np.clip(v - B * dx / Cc, y0, y1)
+            best = np.minimum(best, sig(dx, yc - v))
+        for ye in (y0, y1):   # y fixed: d sigma / d dx = A dx + B dy = 0
+            dy = ye - v
+            xc = np.clip(u - B * dy / A, x0, x1)
+            best = np.minimum(best, sig(xc - u, dy))
+    inside = (u >= x0) & (u <= x1) & (v >= y0) & (v <= y1)
+    best = np.where(inside, 0.0, best)
+    return np.where(pd, best, np.nan)
+
+
+def tile_reach_classes(proj: dict, keys, vals, tiles_x: int):
+    """For every instance (key, gid) of a rectangle binning (the list keys() returns):
+    (must_keep, must_drop) under the tile culling rule, "bin a Gaussian into a tile of
+    its rectangle only when its alpha = o e^-sigma can reach 1/255 somewhere in the
+    tile's box of pixel centres".  must_keep: the box meets the region sigma <= ln(255 o);
+    must_drop: even the box widened by 4/1024 px stays beyond sigma = ln(255 o) +
+    3e-4 (|ln(255 o)| + 1).  Between the two a culled binning may go either way (its
+    margins, and features 1 ulp apart).  A form that is clearly not positive definite
+    (det < -1e-6 A C, or A or C <= 0) must keep the tile; one within 1e-6 of
+    singular is left free."""
+    gid = np.asarray(vals).astype(np.int64)
+    tile = (np.asarray(keys).astype(np.uint64) >> np.uint64(32)).astype(np.int64)
+    tx, ty = tile % tiles_x, tile // tiles_x
+    xy = np.asarray(proj["xy"], np.float64)[gid]
+    con = np.asarray(proj["conic"], np.float64)[gid]
+    o = np.asarray(proj["opacity"], np.float64)[gid]
+    A, B, Cc = con[:, 0], con[:, 1], con[:, 2]
+    det = A * Cc - B * B
+    clearly_pd = (A > 0) & (Cc > 0) & (det > 1e-6 * A * Cc)
+    clearly_not = (A <= 0) | (Cc <= 0) | (det < -1e-6 * np.abs(A * Cc))
+    with np.errstate(divide="ignore"):
+        lnb = np.log(255.0 * o)
+    m0 = tile_min_sigma(xy, con, tx, ty, 0.0)
+    m1 = tile_min_sigma(xy, con, tx, ty, 4.0 / 1024.0)
+    with np.errstate(invalid="ignore"):
+        must_keep = clearly_not | (clearly_pd & (m0 <= lnb))
+        bound = np.where(np.isfinite(lnb), lnb + 3e-4 * (np.abs(lnb) + 1.0), lnb)   # o = 0: -inf
+        must_drop = clearly_pd & (m1 > bound)
+    return must_keep, must_drop

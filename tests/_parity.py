@@ -53,12 +53,12 @@ def ulp_diff(a, b):
 class CudaRun:
     """Forward (and optionally backward) of one view through the C ABI."""
 
-    def __init__(self, scene, cam, bg=(0.0, 0.0, 0.0), capacity=0):
+    def __init__(self, scene, cam, bg=(0.0, 0.0, 0.0), capacity=0, tile_cull=False):
         self.scene = scene
         self.cam = cam
         self.bg = bg
         self.g = pl.Gaussians.from_scene(scene)
-        self.view = pl.View(scene.n, cam, capacity=capacity)
+        self.view = pl.View(scene.n, cam, capacity=capacity, tile_cull=tile_cull)
         self.proj = pl.Projected(scene.n)
         pl.project(self.g, self.view, self.proj)
         self.K = pl.bin_sort(self.proj, self.view)
@@ -193,4 +193,75 @@ def chain_abs_bound(orc, scene, cam, delta2d):
         term = {k: np.abs(np.asarray(col[k], np.float64)).reshape(n, -1) * d[:, q:q + 1]
                 for k in ("means", "quats", "log_scales", "opacity_logits", "sh")}
         out = term if out is None else {k: out[k] + term[k] for k in out}
+    return out
+
+
+def _ranges_of(keys, tiles):
+    """[begin, end) of every tile in a list sorted by tile ([0, 0) for an empty tile)."""
+    t = (keys >> np.uint64(32)).astype(np.int64)
+    r = np.zeros((tiles, 2), np.int64)
+    if len(t):
+        first = np.r_[True, t[1:] != t[:-1]]
+        last = np.r_[t[1:] != t[:-1], True]
+        idx = np.arange(len(t))
+        r[t[first], 0] = idx[first]
+        r[t[last], 1] = idx[last] + 1
+    return r
+
+
+def check_culled_binning(gk, gv, granges, ref, ref_keys, ref_vals, tiles_x, tiles_y, counts=None):
+    """A culled binning (gs_camera.tile_cull) against the oracle's rectangle binning of
+    the same view: the GPU list is the oracle's list with some instances left out, in
+    the same order; it keeps every instance the oracle's tile-reach bound says must be
+    kept and none it says must go (oracle.tile_reach_classes); its ranges are its own
+    list's, bit for bit; and, when given, counts[g] is Gaussian g's number of instances.
+    Returns, for every instance of the oracle's list, its index in the GPU list (-1
+    when left out)."""
+    import oracle as orc
+    K = len(gk)
+    gk = np.asarray(gk, np.uint64)
+    gv = np.asarray(gv, np.uint32)
+    # (key, gid) strictly increasing: a sorted list without repeats
+    if K > 1:
+        inc = (gk[1:] > gk[:-1]) | ((gk[1:] == gk[:-1]) & (gv[1:] > gv[:-1]))
+        assert inc.all(), int((~inc).sum())
+    # every GPU instance is an instance of the oracle's list (equal keys: walk to the gid)
+    p = np.searchsorted(ref_keys, gk, side="left")
+    for _ in range(64):
+        pc = np.minimum(p, len(ref_keys) - 1)
+        off = (p < len(ref_keys)) & (ref_keys[pc] == gk) & (ref_vals[pc] != gv)
+        if not off.any():
+            break
+        p[off] += 1
+    pc = np.minimum(p, max(len(ref_keys) - 1, 0))
+    found = (p < len(ref_keys)) & (ref_keys[pc] == gk) & (ref_vals[pc] == gv) if len(ref_keys) else p < 0
+    assert found.all(), f"{int((~found).sum())} GPU instances are not in the rectangle binning"
+    pos = np.full(len(ref_keys), -1, np.int64)
+    pos[p] = np.arange(K)
+    must_keep, must_drop = orc.tile_reach_classes(ref, ref_keys, ref_vals, tiles_x)
+    kept = pos >= 0
+    assert kept[must_keep].all(), f"{int((~kept[must_keep]).sum())} instances that must stay were left out"
+    assert not kept[must_drop].any(), f"{int(kept[must_drop].sum())} instances that must go were kept"
+    assert np.array_equal(np.asarray(granges, np.int64).reshape(-1, 2), _ranges_of(gk, tiles_x * tiles_y))
+    if counts is not None:
+        per_gid = np.bincount(gv.astype(np.int64), minlength=len(counts))
+        assert np.array_equal(per_gid, np.asarray(counts, np.int64))
+    return pos
+
+
+def culled_n_contrib(ref_nc, pix, W, tiles_x, ref_ranges, pos, granges):
+    """The oracle's n_contrib (1 + the position of the last blended entry in its
+    rectangle list) moved into the culled GPU list: 1 + the GPU position of the same
+    instance; -1 where that instance is missing from the GPU list."""
+    ref_nc = np.asarray(ref_nc, np.int64)
+    pix = np.arange(len(ref_nc)) if pix is None else np.asarray(pix, np.int64)
+    x, y = pix % W, pix // W
+    t = (y // 16) * tiles_x + x // 16
+    rr = np.asarray(ref_ranges, np.int64).reshape(-1, 2)
+    gr = np.asarray(granges, np.int64).reshape(-1, 2)
+    out = np.zeros_like(ref_nc)
+    has = ref_nc > 0
+    e = rr[t[has], 0] + ref_nc[has] - 1
+    g = pos[e]
+    out[has] = np.where(g >= 0, g - gr[t[has], 0] + 1, -1)
     return out

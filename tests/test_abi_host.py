@@ -76,6 +76,19 @@ def test_tile_grid_and_camera_checks(gs):
     with pytest.raises(gs.GsError) as e:
         gs.gs_tile_grid(gs.make_camera(cam(near=0.0)))
     assert e.value.status == gs.GS_ERR_INVALID_ARG
+    assert gs.gs_tile_grid(gs.make_camera(cam(), tile_cull=True)) == (8, 8)
+    c = gs.make_camera(cam())
+    c.tile_cull = 2
+    with pytest.raises(gs.GsError) as e:
+        gs.gs_tile_grid(c)
+    assert e.value.status == gs.GS_ERR_INVALID_ARG
+
+
+def test_camera_struct_layout(gs):
+    import ctypes
+    # float R[9], t[3], fx, fy, cx, cy; int32 width, height; float near_plane, eps2d; int32 tile_cull
+    assert ctypes.sizeof(gs.gs_camera) == 4 * (9 + 3 + 4 + 2 + 2 + 1)
+    assert gs.gs_camera.tile_cull.offset == 4 * 20
 
 
 def test_invalid_arguments_rejected_before_launch(gs):

@@ -7,10 +7,13 @@ projection with the densification statistics and Adam on all five groups), again
 the oracle:
 
   * every view's projection (features <= 1 ulp, integers exact), and its complete
-    sorted instance list and tile ranges, bit-exact;
-  * per view, image, final T and n_contrib on every pixel of a set of tiles (the
-    heaviest, ragged edges, random tiles, and the tiles of the sampled Gaussians
-    below), and dL/dimage of the L1 loss there;
+    sorted instance list and tile ranges: the binning the benchmark runs is the
+    culled one (each Gaussian only in the tiles its footprint reaches), checked as
+    the oracle's rectangle list less instances the oracle's tile-reach bound lets
+    go, keeping all it must keep, in the same order, with its own ranges;
+  * per view, image, final T and n_contrib (moved into the culled lists) on every
+    pixel of a set of tiles (the heaviest, ragged edges, random tiles, and the tiles
+    of the sampled Gaussians below), and dL/dimage of the L1 loss there;
   * per view, the 2D gradients (full L1 upstream) of every Gaussian whose tile
     rectangle lies inside the rendered tiles, so the oracle sees all of its pixels;
   * for a sample of Gaussians covered that way in every view: the densification
@@ -29,8 +32,8 @@ import torch
 from gaussian_splatting_differentiable_02_b200 import pipeline as pl
 from gaussian_splatting_differentiable_02_b200 import scenes
 
-from _parity import (AMB_FRAC_LONG_LISTS, BAND_ALPHA, BAND_T, G_ATOL, G_RTOL, SUM_BOUND, check_grads,
-                     check_images, check_projection)
+from _parity import (AMB_FRAC_LONG_LISTS, BAND_ALPHA, BAND_T, G_ATOL, G_RTOL, SUM_BOUND, check_culled_binning,
+                     check_grads, check_images, check_projection, culled_n_contrib)
 
 pytestmark = pytest.mark.gpu
 
@@ -102,16 +105,26 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
 
     # ---- pass 1: projection and the complete sorted lists of every view, bit-exact
     rects, visible, lengths = [], [], []
+    moved = []   # culled binning: per view, the oracle's list index -> the GPU list index, and both ranges
     for k, cam in enumerate(cams):
         ref = orc.project(scene, cam)
         check_projection(_gpu_projection(tr, k), ref)
         keys, vals, ranges = orc.keys(ref, cam)
         K = int(counts[k])
-        assert K == len(keys), (k, K, len(keys))
         view = tr.views[k]
-        assert np.array_equal(view.keys[:K].cpu().numpy().view(np.uint64), keys), k
-        assert np.array_equal(view.vals[:K].cpu().numpy().view(np.uint32), vals), k
-        assert np.array_equal(view.ranges.cpu().numpy().view(np.uint32), ranges), k
+        gk = view.keys[:K].cpu().numpy().view(np.uint64)
+        gv = view.vals[:K].cpu().numpy().view(np.uint32)
+        gr = view.ranges.cpu().numpy().view(np.uint32)
+        if tr.tile_cull:
+            # the oracle's rectangle list less what the tile-reach bound lets go, in order
+            pos = check_culled_binning(gk, gv, gr, ref, keys, vals, tx, ty)
+            assert K < 0.6 * len(keys), (k, K, len(keys))
+            moved.append((pos.astype(np.int32), ranges.astype(np.int64), gr.astype(np.int64)))
+        else:
+            assert K == len(keys), (k, K, len(keys))
+            assert np.array_equal(gk, keys), k
+            assert np.array_equal(gv, vals), k
+            assert np.array_equal(gr, ranges), k
         rects.append(ref["rect"].copy())
         visible.append(ref["radius"] > 0)
         lengths.append((ranges[:, 1].astype(np.int64) - ranges[:, 0]))
@@ -150,6 +163,9 @@ def test_benchmarked_step_matches_oracle(orc, stepped):
         gi = view.image.cpu().numpy().reshape(-1, 3)[pix]
         gT = view.final_T.cpu().numpy().reshape(-1)[pix]
         gn = view.n_contrib.cpu().numpy().reshape(-1)[pix]
+        if tr.tile_cull:   # n_contrib counts positions in the culled lists
+            pos, rr, gr = moved[k]
+            nc = culled_n_contrib(nc, pix, W, tx, rr, pos, gr)
         err, namb = check_images(gi, gT, gn, img, T, nc, amb, max_amb_frac=AMB_FRAC_LONG_LISTS)
         n_amb_total += namb
         n_px_total += len(pix)
