@@ -28,7 +28,6 @@
 
 namespace gsk {
 
-// 64 bytes: what the emission keeps in shared memory per Gaussian.
 struct TileReach {
     float u, v;     // mean in pixels
     float A, B, C;  // conic
@@ -37,7 +36,8 @@ struct TileReach {
     double iA;      // 1 / A
     double s;       // the sigma bound, margin included
     double ym;      // half height of the region sigma <= s: sqrt(2 A s / det)
-    double dyr;     // dy of its rightmost point (dy of the leftmost: -dyr)
+    double xm;      // half width: sqrt(2 C s / det)
+    double dyr;     // dy of its rightmost point, where dx = xm (the leftmost: -dyr, -xm)
 };
 
 __device__ __forceinline__ float lg2_approx(float x) {
@@ -58,6 +58,7 @@ __device__ __forceinline__ TileReach tile_reach_setup(float2 xy, float4 conic_op
     r.iA = 0.0;
     r.s = 0.0;
     r.ym = 0.0;
+    r.xm = 0.0;
     r.dyr = 0.0;
     if (!(A > 0.0) || !(C > 0.0) || !(r.det > 0.0) || !(fabsf(r.u) < 1e30f) || !(fabsf(r.v) < 1e30f)) {
         r.mode = 2;
@@ -74,8 +75,8 @@ __device__ __forceinline__ TileReach tile_reach_setup(float2 xy, float4 conic_op
     r.iA = __drcp_rn(A);
     const double two_s = __dmul_rn(2.0, s);
     r.ym = __dsqrt_rn(__ddiv_rn(__dmul_rn(two_s, A), r.det));
-    const double xm = __dsqrt_rn(__ddiv_rn(__dmul_rn(two_s, C), r.det));  // half width
-    r.dyr = __ddiv_rn(__dmul_rn(-B, xm), C);
+    r.xm = __dsqrt_rn(__ddiv_rn(__dmul_rn(two_s, C), r.det));
+    r.dyr = __ddiv_rn(__dmul_rn(-B, r.xm), C);
     r.mode = 1;
     return r;
 }
@@ -99,16 +100,21 @@ __device__ __forceinline__ void tile_reach_row(const TileReach& r, int ty, int x
         return;
     }
     // x extent at dy: (-B dy +- sqrt(2 A s - det dy^2)) / A; the right end is
-    // concave in dy (largest at dyr clamped to the band), the left end convex
-    // (smallest at -dyr clamped)
+    // concave in dy (largest at dyr clamped to the band: xm when dyr lies in it),
+    // the left end convex (smallest at -dyr clamped: -xm when -dyr lies in it)
     const double A = r.A, B = r.B, u = r.u;
     const double two_as = __dmul_rn(__dmul_rn(2.0, A), r.s);
     const double dy_r = fmin(fmax(r.dyr, lo), hi);
     const double dy_l = fmin(fmax(-r.dyr, lo), hi);
-    const double q_r = fmax(__dsub_rn(two_as, __dmul_rn(r.det, __dmul_rn(dy_r, dy_r))), 0.0);
-    const double q_l = fmax(__dsub_rn(two_as, __dmul_rn(r.det, __dmul_rn(dy_l, dy_l))), 0.0);
-    const double xr = __dmul_rn(__dadd_rn(__dmul_rn(-B, dy_r), __dsqrt_rn(q_r)), r.iA);
-    const double xl = __dmul_rn(__dsub_rn(__dmul_rn(-B, dy_l), __dsqrt_rn(q_l)), r.iA);
+    double xr = r.xm, xl = -r.xm;
+    if (dy_r != r.dyr) {
+        const double q = fmax(__dsub_rn(two_as, __dmul_rn(r.det, __dmul_rn(dy_r, dy_r))), 0.0);
+        xr = __dmul_rn(__dadd_rn(__dmul_rn(-B, dy_r), __dsqrt_rn(q)), r.iA);
+    }
+    if (dy_l != -r.dyr) {
+        const double q = fmax(__dsub_rn(two_as, __dmul_rn(r.det, __dmul_rn(dy_l, dy_l))), 0.0);
+        xl = __dmul_rn(__dsub_rn(__dmul_rn(-B, dy_l), __dsqrt_rn(q)), r.iA);
+    }
     // tile tx reaches [u + xl, u + xr] when 16 tx + 0.5 - w <= u + xr and
     // 16 tx + 15.5 + w >= u + xl
     const double hi_t = floor(__dmul_rn(__dsub_rn(__dadd_rn(u, xr), 0.5 - kWiden), 0.0625));
