@@ -310,54 +310,86 @@ struct EmitArgs {
     int64_t tiles;
 };
 
-// The culled binning's instances of the Gaussian at depth-order position i:
-// the runs of tiles its footprint reaches in each row of its rectangle
-// (tile_reach.cuh).  The first kRunRows rows' runs are kept for the emission as
-// (first column << 16 | length); returns the count over all rows.
-__device__ __forceinline__ uint32_t culled_runs(const EmitSeg& g, int64_t i, uint32_t gid) {
-    const uint2 r = __ldg(g.rect + gid);
-    const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu), y1 = int(r.y >> 16);
-    const TileReach R = tile_reach_setup(__ldg(g.xy + gid), __ldg(g.con + gid));
-    uint32_t w[kRunRows];
-    uint32_t c = 0;
-#pragma unroll
-    for (int k = 0; k < kRunRows; ++k) {
-        w[k] = 0u;
-        if (y0 + k < y1) {
-            int c0, c1;
-            tile_reach_row(R, y0 + k, x0, x1, &c0, &c1);
-            w[k] = (uint32_t(c0) << 16) | uint32_t(c1 - c0);
-            c += uint32_t(c1 - c0);
+// The culled binning's counts for one chunk of kEmitChunk depth-ordered
+// Gaussians, in halves of one Gaussian per thread: each thread sets up its
+// Gaussian's footprint bound (tile_reach.cuh) in shared memory, a block scan
+// numbers the rows of all the half's rectangles, and the block's threads then
+// take those rows round-robin (a warp no longer waits for its tallest
+// Gaussian's rows), adding each row's run length to its Gaussian's count in
+// shared memory and writing the runs of the first kRunRows rows as (first
+// column << 16 | length) for the emission.  A Gaussian whose conic is not
+// positive definite counts its whole rectangle, one that reaches nothing 0.
+// Returns this thread's share of the chunk's instances.
+__device__ unsigned long long culled_counts(const EmitArgs& a, const EmitSeg& g, int64_t base) {
+    constexpr int kHalf = kEmitBlock;
+    __shared__ TileReach s_tr[kHalf];
+    __shared__ uint2 s_rect[kHalf];
+    __shared__ uint32_t s_roff[kHalf + 1];
+    __shared__ uint32_t s_cnt[kHalf];
+    unsigned long long sum = 0;
+    const int t = threadIdx.x;
+    for (int half = 0; half < kEmitChunk / kHalf; ++half) {
+        const int64_t i = base + int64_t(half) * kHalf + t;
+        uint32_t rows = 0, direct = 0;
+        if (i < a.n) {
+            const uint32_t gid = __ldg(g.order + i);
+            if (__ldg(g.touched + gid)) {
+                const uint2 r = __ldg(g.rect + gid);
+                const uint32_t w = (r.y & 0xffffu) - (r.x & 0xffffu), h = (r.y >> 16) - (r.x >> 16);
+                const TileReach R = tile_reach_setup(__ldg(g.xy + gid), __ldg(g.con + gid));
+                s_tr[t] = R;
+                s_rect[t] = r;
+                if (R.mode == 1) rows = h;
+                else if (R.mode == 2) direct = w * h;
+                // runs past the rectangle's last row read as empty
+                uint32_t* out = g.runs + i * kRunRows;
+                for (int k = int(rows); k < kRunRows; ++k) out[k] = 0u;
+            }
         }
+        s_cnt[t] = direct;
+        unsigned long long tot;
+        const uint32_t off = uint32_t(block_excl_scan(rows, &tot));
+        s_roff[t] = off;
+        if (t == 0) s_roff[kHalf] = uint32_t(tot);
+        __syncthreads();
+        for (uint32_t q = t; q < uint32_t(tot); q += kEmitBlock) {
+            // the last Gaussian whose first row is <= q (it has at least one row)
+            int lo = 0;
+#pragma unroll
+            for (int step = kHalf / 2; step > 0; step >>= 1)
+                if (s_roff[lo + step] <= q) lo += step;
+            const int k = int(q - s_roff[lo]);
+            const uint2 r = s_rect[lo];
+            const int x0 = int(r.x & 0xffffu), y0 = int(r.x >> 16), x1 = int(r.y & 0xffffu);
+            int c0, c1;
+            tile_reach_row(s_tr[lo], y0 + k, x0, x1, &c0, &c1);
+            if (c1 > c0) atomicAdd(&s_cnt[lo], uint32_t(c1 - c0));
+            if (k < kRunRows)
+                g.runs[(base + int64_t(half) * kHalf + lo) * kRunRows + k] = (uint32_t(c0) << 16) | uint32_t(c1 - c0);
+        }
+        __syncthreads();
+        if (i < a.n) {
+            g.cnt[i] = s_cnt[t];
+            sum += s_cnt[t];
+        }
+        __syncthreads();  // the shared arrays are reused by the next half
     }
-    for (int y = y0 + kRunRows; y < y1; ++y) {
-        int c0, c1;
-        tile_reach_row(R, y, x0, x1, &c0, &c1);
-        c += uint32_t(c1 - c0);
-    }
-    uint4* out = reinterpret_cast<uint4*>(g.runs + i * kRunRows);
-    out[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    out[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    return c;
+    return sum;
 }
 
 // Per block of kEmitChunk depth-ordered Gaussians, the sum of their instance
-// counts: tiles_touched, or in the culled binning the counts of culled_runs
+// counts: tiles_touched, or in the culled binning the counts of culled_counts
 // (stored with the runs for the emission).
 __global__ void __launch_bounds__(kEmitBlock) count_sorted_kernel(const __grid_constant__ EmitArgs a) {
     const EmitSeg& g = a.seg[blockIdx.y];
     const int64_t base = int64_t(blockIdx.x) * kEmitChunk;
     unsigned long long sum = 0;
-    for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
-        const int64_t i = base + k;
-        if (i < a.n) {
-            const uint32_t gid = __ldg(g.order + i);
-            uint32_t t = __ldg(g.touched + gid);
-            if (g.runs) {
-                if (t) t = culled_runs(g, i, gid);
-                g.cnt[i] = t;
-            }
-            sum += t;
+    if (g.runs) {
+        sum = culled_counts(a, g, base);
+    } else {
+        for (int k = threadIdx.x; k < kEmitChunk; k += kEmitBlock) {
+            const int64_t i = base + k;
+            if (i < a.n) sum += __ldg(g.touched + __ldg(g.order + i));
         }
     }
     unsigned long long tot;

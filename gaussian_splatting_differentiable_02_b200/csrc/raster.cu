@@ -68,15 +68,26 @@ constexpr float kCondMaxTraceSqOverDet = 10.125f;
 // own box.  PX = 8: the box is the whole tile, and the warp's per-entry work (its
 // shared-memory reads, the gradient reduction, the branches) is spread over 256
 // pixels; PX = 4: two warps a tile, which culls entries against half tiles and
-// gives twice the warps.  Grids of at least kWideLayoutTiles tiles use PX = 8,
-// smaller ones PX = 4.  Measured (forward / backward ms per view): 16 1080p views
-// of the 1M mixture (8160 tiles) PX = 8 at 14 / 16 blocks an SM 0.589 / 1.067,
-// PX = 4 at 20 / 20 blocks 0.606 / 1.166; the 1296x840 view (4293 tiles) PX = 8
-// 0.454 / 0.856, PX = 4 0.404 / 0.806 (two warps a block, 10 blocks: 0.622 / 1.144
-// at 1080p; PX = 8 at 12 / 14 / 20 blocks slower).
+// gives twice the warps.  The backward uses PX = 8 on grids of at least
+// kWideLayoutTiles tiles and PX = 4 on smaller ones; the forward uses PX = 4 on
+// grids below kWideLayoutTilesFwd (every grid by default).  Measured (forward /
+// backward ms per view) over the rectangle binning's lists: 16 1080p views of the
+// 1M mixture (8160 tiles) PX = 8 at 14 / 16 blocks an SM 0.589 / 1.067, PX = 4 at
+// 20 / 20 blocks 0.606 / 1.166; the 1296x840 view (4293 tiles) PX = 8 0.454 /
+// 0.856, PX = 4 0.404 / 0.806 (two warps a block, 10 blocks: 0.622 / 1.144 at
+// 1080p; PX = 8 at 12 / 14 / 20 blocks slower).  Over the culled binning's lists,
+// which hold about half the entries and so halve the staging PX = 4 pays twice,
+// at 1080p: PX = 8 0.504 / 0.970, PX = 4 0.463 / 1.012.
 constexpr int kBoxW = 16;               // width of a warp's pixel box
 constexpr int kWarps = 1;               // warps per block
-constexpr int64_t kWideLayoutTiles = 6144;
+#ifndef GS_WIDE_LAYOUT_TILES
+#define GS_WIDE_LAYOUT_TILES 6144
+#endif
+constexpr int64_t kWideLayoutTiles = GS_WIDE_LAYOUT_TILES;
+#ifndef GS_WIDE_LAYOUT_TILES_FWD
+#define GS_WIDE_LAYOUT_TILES_FWD (int64_t(1) << 40)
+#endif
+constexpr int64_t kWideLayoutTilesFwd = GS_WIDE_LAYOUT_TILES_FWD;
 #ifndef GS_RASTER_BWD_BLOCKS8
 #define GS_RASTER_BWD_BLOCKS8 16
 #endif
@@ -832,7 +843,7 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
     const int64_t count = int64_t(3) * cam.W * cam.H;
     a.inv_count = float(1.0 / double(count));
     a.inv_count_d = 1.0 / double(count);
-    if (a.tiles >= kWideLayoutTiles) {
+    if (a.tiles >= kWideLayoutTilesFwd) {
         const unsigned grid = unsigned(a.tiles * Layout<8>::kSub);
         if (counts)
             raster_fwd_kernel<8, true, false><<<grid, kWarps * 32, 0, s>>>(a);

@@ -10,7 +10,8 @@ against the rectangle binning on the GPU:
     the image tolerance; n_contrib equals the oracle's (and the rectangle run's)
     moved into the shorter lists;
   * the 2D gradients match the oracle's;
-  * at full size (a 1080p view of the 1M mixture) the whole list and every pixel;
+  * at full size (a 1080p view of the 1M mixture, a 4K view of the 3M city) the whole
+    list and every pixel;
   * the Trainer with and without culling gives the same losses and updates.
 """
 import numpy as np
@@ -128,6 +129,32 @@ def test_full_size_view_of_the_1m_mixture(orc):
     gk, gv, gr = b.sorted_instances()
     pos = check_culled_binning(gk, gv, gr, ref, keys, vals, tx, ty)
     assert len(gk) < 0.6 * len(keys)
+    ib, Tb, nb = b.images()
+    assert np.array_equal(ia, ib) and np.array_equal(Ta, Tb)
+    assert np.array_equal(culled_n_contrib(na, None, cam["width"], tx, ranges, pos, gr), nb)
+
+
+def test_full_size_4k_view_of_the_3m_city(orc):
+    """One 3840x2160 view of the 3M city (15 tile bits, two tile passes): the whole
+    culled list against the oracle's rectangle list and tile-reach bound, and every
+    pixel against the rectangle run."""
+    wl = scenes.city3m(poses=1)
+    cam = wl.cameras[0]
+    scene = wl.scene
+    a = CudaRun(scene, cam, capacity=40_000_000)
+    ia, Ta, na = a.images()
+    ak, av, ar = (x.copy() for x in a.sorted_instances())
+    del a
+    torch.cuda.empty_cache()
+    b = CudaRun(scene, cam, capacity=40_000_000, tile_cull=True)
+    ref = orc.project(scene, cam)
+    keys, vals, ranges = orc.keys(ref, cam)
+    assert np.array_equal(ak, keys) and np.array_equal(av, vals) and np.array_equal(ar, ranges)
+    del ak, av, ar
+    tx, ty = orc.tiles(cam)
+    gk, gv, gr = b.sorted_instances()
+    pos = check_culled_binning(gk, gv, gr, ref, keys, vals, tx, ty)
+    assert len(gk) < 0.8 * len(keys)
     ib, Tb, nb = b.images()
     assert np.array_equal(ia, ib) and np.array_equal(Ta, Tb)
     assert np.array_equal(culled_n_contrib(na, None, cam["width"], tx, ranges, pos, gr), nb)
