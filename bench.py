@@ -390,12 +390,12 @@ def run_render(args, world, rank, local):
     frames = args.steps * len(cams)
     # work counters of the last pose's compositing (counted variant, outside the timing) and
     # the measured float32 / special-function peaks, for the roofline of raster_fwd
-    counts = torch.zeros(4, device="cuda", dtype=torch.int64)
+    counts = torch.zeros(5, device="cuda", dtype=torch.int64)
     pl.raster_fwd_counted(proj, view, counts)
     torch.cuda.synchronize()
     c = counts.cpu().tolist()
     work = {"traversed_pairs": float(view.n_contrib.sum().item()), "fwd_evaluated_pairs": float(c[0]),
-            "fwd_blended_pairs": float(c[1]), "fwd_staged_entries": float(c[2])}
+            "fwd_blended_pairs": float(c[1]), "fwd_staged_entries": float(c[2]), "fwd_visited_pairs": float(c[4])}
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev[-len(cams):])
     peaks = measured_peaks()
     alu = measure_alu_peaks(torch, local)
@@ -1018,12 +1018,14 @@ def measure_alu_peaks(torch, local, target_ms: float = 60.0, reps: int = 5):
 def raster_work_counts(tr, torch):
     """Work counters of the compositing kernels over the step's views, from the
     counted variants run once on the last step's lists (outside any timing):
-    per view mean of the pairs a pixel traverses (sum of n_contrib), the pairs
-    it blends, the pairs the warps evaluate, and the list entries staged."""
+    per view mean of the pairs the reverse pass's per-pixel loop visits (sum of
+    n_contrib), of those the forward pass's loop visits (each pixel's list up to
+    the entry it stops at, or all of it), the pairs it blends, the pairs the
+    warps evaluate, and the list entries staged."""
     from gaussian_splatting_differentiable_02_b200 import pipeline as pl
     nv = len(tr.views)
-    cf = torch.zeros(4, device="cuda", dtype=torch.int64)
-    cb = torch.zeros(4, device="cuda", dtype=torch.int64)
+    cf = torch.zeros(5, device="cuda", dtype=torch.int64)
+    cb = torch.zeros(5, device="cuda", dtype=torch.int64)
     traversed = 0
     g2 = pl.Grad2D(tr.gauss.n)
     batched = getattr(tr, "depth_orders", None) is not None
@@ -1041,8 +1043,8 @@ def raster_work_counts(tr, torch):
     torch.cuda.synchronize()
     f, b = cf.cpu().tolist(), cb.cpu().tolist()
     return {"traversed_pairs": traversed / nv, "fwd_evaluated_pairs": f[0] / nv, "fwd_blended_pairs": f[1] / nv,
-            "fwd_staged_entries": f[2] / nv, "bwd_evaluated_pairs": b[0] / nv, "bwd_gradient_pairs": b[1] / nv,
-            "bwd_staged_entries": b[2] / nv}
+            "fwd_staged_entries": f[2] / nv, "fwd_visited_pairs": f[4] / nv, "bwd_evaluated_pairs": b[0] / nv,
+            "bwd_gradient_pairs": b[1] / nv, "bwd_staged_entries": b[2] / nv}
 
 
 def stage_breakdown(tr, pl, torch):
@@ -1146,26 +1148,29 @@ def profiled_traffic(stage, workload):
 
 def raster_roofline(stage, ms, work, alu, workload=""):
     """Roofline object of a compositing kernel against the measured float32 FMA
-    peak: achieved = the method's flops per launch (FLOPS_ALPHA per traversed
-    pair, plus the blend or gradient flops per blended pair) / the mean launch
-    time.  The special-function unit (ex2, rcp per evaluated pair) is reported
-    beside it against its own measured rate."""
+    peak: achieved = the method's flops per launch (FLOPS_ALPHA per pair its
+    per-pixel loop visits: in the forward pass each pixel's list up to the entry
+    at which it stops, in the reverse pass up to its n_contrib; plus the blend or
+    gradient flops per blended pair) / the mean launch time.  The
+    special-function unit (ex2, rcp per evaluated pair) is reported beside it
+    against its own measured rate."""
     fwd = stage == "raster_fwd"
     blended = work["fwd_blended_pairs"] if fwd else work["bwd_gradient_pairs"]
     evaluated = work["fwd_evaluated_pairs"] if fwd else work["bwd_evaluated_pairs"]
-    flops = FLOPS_ALPHA * work["traversed_pairs"] + (FLOPS_FWD_BLEND if fwd else FLOPS_BWD_GRAD) * blended
+    visited = work.get("fwd_visited_pairs", work["traversed_pairs"]) if fwd else work["traversed_pairs"]
+    flops = FLOPS_ALPHA * visited + (FLOPS_FWD_BLEND if fwd else FLOPS_BWD_GRAD) * blended
     achieved = flops / (ms * 1e-3) / 1e12
     peak = alu["fp32_tflops"]
     sfu_ops = evaluated * (SFU_FWD if fwd else SFU_BWD)
     sfu_rate = sfu_ops / (ms * 1e-3) / 1e12
     return {"kernel": stage, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": profiled_traffic(stage, workload),
-            "work": (f"{work['traversed_pairs']:.4g} traversed pairs x {FLOPS_ALPHA} + {blended:.4g} blended pairs x "
+            "work": (f"{visited:.4g} visited pairs x {FLOPS_ALPHA} + {blended:.4g} blended pairs x "
                      f"{FLOPS_FWD_BLEND if fwd else FLOPS_BWD_GRAD} flops per launch (mean over views)"),
             "peak_source": f"measured float32 FMA throughput ({alu['source']})",
             "sfu": {"achieved_tops": sfu_rate, "peak_tops": alu["ex2_tops"], "frac": sfu_rate / alu["ex2_tops"],
                     "ops": f"{evaluated:.4g} evaluated pairs x {SFU_FWD if fwd else SFU_BWD} (ex2{'' if fwd else ' + rcp'})"},
-            "evaluated_over_traversed": evaluated / max(work["traversed_pairs"], 1.0),
+            "evaluated_over_visited": evaluated / max(visited, 1.0),
             "nominal_fp32_tflops": NUM_SMS * FP32_LANES_PER_SM * 2 * 1965.0 * 1e6 / 1e12}
 
 

@@ -88,6 +88,12 @@ constexpr int64_t kWideLayoutTiles = GS_WIDE_LAYOUT_TILES;
 #define GS_WIDE_LAYOUT_TILES_FWD (int64_t(1) << 40)
 #endif
 constexpr int64_t kWideLayoutTilesFwd = GS_WIDE_LAYOUT_TILES_FWD;
+#ifndef GS_FWD_PX
+#define GS_FWD_PX 4  // the forward's layout below kWideLayoutTilesFwd
+#endif
+#ifndef GS_RASTER_FWD_BLOCKS2
+#define GS_RASTER_FWD_BLOCKS2 32
+#endif
 #ifndef GS_RASTER_BWD_BLOCKS8
 #define GS_RASTER_BWD_BLOCKS8 16
 #endif
@@ -98,7 +104,7 @@ struct Layout {
     static constexpr int kBoxH = 2 * PX;                 // height of a warp's box
     static constexpr int kSub = kTile / kBoxH;           // warps per tile
     // resident blocks per SM the register allocation is sized for (launch bounds)
-    static constexpr int kFwdMinBlocks = PX == 8 ? 14 : 20;
+    static constexpr int kFwdMinBlocks = PX == 8 ? 14 : (PX == 4 ? 20 : GS_RASTER_FWD_BLOCKS2);
     static constexpr int kBwdMinBlocks = PX == 8 ? GS_RASTER_BWD_BLOCKS8 : 20;
 };
 constexpr int kBatch = 32;  // list entries staged per warp per batch
@@ -362,16 +368,22 @@ struct FwdArgs {
 // Work counters of the counted variants (one atomic per warp at its end): pairs
 // the warp evaluated (entries that reach its box x its pixels), pairs that did
 // the method's work (blended in the forward pass, took a gradient in the
-// reverse pass), list entries staged, and entries that reached the box.
+// reverse pass), list entries staged, entries that reached the box, and (the
+// forward pass) the pairs the method's per-pixel loop visits: for each pixel of
+// the image, its tile's list up to the entry at which it stops, or all of it.
 __device__ __forceinline__ void add_counts(unsigned long long* counts, int evaluated_entries, int work_pairs,
-                                           int staged, int lane, int box_pixels) {
+                                           int staged, int lane, int box_pixels, int visited = 0) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) work_pairs += __shfl_xor_sync(kFull, work_pairs, o);
+    for (int o = 16; o > 0; o >>= 1) {
+        work_pairs += __shfl_xor_sync(kFull, work_pairs, o);
+        visited += __shfl_xor_sync(kFull, visited, o);
+    }
     if (lane == 0) {
         atomicAdd(counts + 0, (unsigned long long)evaluated_entries * box_pixels);
         atomicAdd(counts + 1, (unsigned long long)work_pairs);
         atomicAdd(counts + 2, (unsigned long long)staged);
         atomicAdd(counts + 3, (unsigned long long)evaluated_entries);
+        atomicAdd(counts + 4, (unsigned long long)visited);
     }
 }
 
@@ -419,6 +431,9 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster
     }
     const f2 one = splat(1.f);
     int c_eval = 0, c_work = 0, c_staged = 0;  // kCount only
+    int stop[kCount ? kPx : 1];                // kCount: 1-based position of the entry a pixel stopped at, or 0
+#pragma unroll
+    for (int i = 0; i < (kCount ? kPx : 1); ++i) stop[i] = 0;
 
     const int nb = (n + kBatch - 1) / kBatch;
     if (n > 0) gather<false>(S, 0, a.vals, a.xy, a.con, a.rgb, range.x, min(n, kBatch), lane);
@@ -472,6 +487,10 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster
                 Cg[p] = fma2(ncg, nw, Cg[p]);
                 Cb[p] = fma2(ncb, nw, Cb[p]);
                 T[p] = mul2(T[p], add2(one, na));
+                if (kCount) {
+                    if (on[p].x != 0.f && keep.x == 0.f) stop[2 * p] = pos;
+                    if (on[p].y != 0.f && keep.y == 0.f) stop[2 * p + 1] = pos;
+                }
                 on[p] = mul2(on[p], keep);
                 last[2 * p] = na.x != 0.f ? pos : last[2 * p];
                 last[2 * p + 1] = na.y != 0.f ? pos : last[2 * p + 1];
@@ -482,7 +501,13 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kFwdMinBlocks) raster
         if (finished) break;
     }
     cp_async_wait_all();
-    if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
+    if (kCount) {
+        int visited = 0;
+#pragma unroll
+        for (int i = 0; i < kPx; ++i)
+            if (x < a.W && y0 + i < a.H) visited += stop[i] ? stop[i] : n;
+        add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx, visited);
+    }
     double l1 = 0.0;  // kL1: this lane's sum of |image - target|
     if (x < a.W) {
 #pragma unroll
@@ -852,13 +877,14 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
         else
             raster_fwd_kernel<8, false, false><<<grid, kWarps * 32, 0, s>>>(a);
     } else {
-        const unsigned grid = unsigned(a.tiles * Layout<4>::kSub);
+        constexpr int P = GS_FWD_PX;
+        const unsigned grid = unsigned(a.tiles * Layout<P>::kSub);
         if (counts)
-            raster_fwd_kernel<4, true, false><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<P, true, false><<<grid, kWarps * 32, 0, s>>>(a);
         else if (l1)
-            raster_fwd_kernel<4, false, true><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<P, false, true><<<grid, kWarps * 32, 0, s>>>(a);
         else
-            raster_fwd_kernel<4, false, false><<<grid, kWarps * 32, 0, s>>>(a);
+            raster_fwd_kernel<P, false, false><<<grid, kWarps * 32, 0, s>>>(a);
     }
     count_launches(1);
     return cudaGetLastError();

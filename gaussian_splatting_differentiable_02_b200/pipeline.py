@@ -351,7 +351,9 @@ def raster_bwd(proj: Projected, view: View, grad2d: Grad2D, bg=(0.0, 0.0, 0.0), 
 
 def raster_fwd_counted(proj: Projected, view: View, counts: torch.Tensor, bg=(0.0, 0.0, 0.0),
                        radius: torch.Tensor = None):
-    """raster_fwd that also adds its work counters to counts (4 int64 on the device)."""
+    """raster_fwd that also adds its work counters to counts (5 int64 on the device, gs.h)."""
+    if counts.numel() < 5:
+        raise ValueError("the counted raster calls add to 5 counters")
     abi.gs_raster_fwd_counted(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam,
                               bg, _ptr(view.image), _ptr(view.final_T), _ptr(view.n_contrib), _ptr(counts),
                               _stream())
@@ -360,6 +362,8 @@ def raster_fwd_counted(proj: Projected, view: View, counts: torch.Tensor, bg=(0.
 def raster_bwd_counted(proj: Projected, view: View, grad2d: Grad2D, counts: torch.Tensor, bg=(0.0, 0.0, 0.0),
                        radius: torch.Tensor = None):
     """raster_bwd (upstream view.dL_dimage) that also adds its work counters to counts."""
+    if counts.numel() < 5:
+        raise ValueError("the counted raster calls add to 5 counters")
     abi.gs_raster_bwd_counted(proj.struct(radius), _ptr(view.vals), _ptr(view.ranges), _ptr(view.order), view.gcam,
                               bg, _ptr(view.final_T), _ptr(view.n_contrib), _ptr(view.dL_dimage), grad2d.struct(),
                               _ptr(counts), _stream())

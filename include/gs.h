@@ -595,15 +595,19 @@ gs_status gs_l1_dssim_loss_grad(const float* image, const float* target, int32_t
 
 /* gs_raster_fwd_counted / gs_raster_bwd_counted -- gs_raster_fwd / gs_raster_bwd
  * (same arguments, same results, bit for bit) that also add work counters to
- * counts[0..3] (uint64 on the device, 8-byte aligned, +=):
+ * counts[0..4] (uint64 on the device, 8-byte aligned, +=):
  *   counts[0]  (pixel, entry) pairs evaluated: entries that reached a warp's
- *              pixel box (its 16x16 tile) times the box's pixels (pixels
- *              outside the image included);
+ *              pixel box (its 16x16 tile, or a 16x8 half of it) times the box's
+ *              pixels (pixels outside the image included);
  *   counts[1]  pairs that did the method's work: in the forward pass the
  *              entries a pixel blended, in the reverse pass the entries a pixel
  *              takes a gradient from (the same blended set);
  *   counts[2]  list entries staged into shared memory, summed over warps;
- *   counts[3]  entries that reached a warp's box, summed over warps.
+ *   counts[3]  entries that reached a warp's box, summed over warps;
+ *   counts[4]  forward pass: the pairs the method's per-pixel loop visits, for
+ *              every pixel of the image its tile's list up to and including the
+ *              entry at which it stops, or the whole list; reverse pass: 0 (its
+ *              loop visits sum(n_contrib) pairs).
  * One atomic add per warp and counter at the warp's end. */
 gs_status gs_raster_fwd_counted(const gs_projected* proj, const uint32_t* vals, const uint32_t* tile_ranges,
                                 const uint32_t* tile_order, const gs_camera* cam, const float* bg_host, float* image,

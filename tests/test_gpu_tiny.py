@@ -357,3 +357,46 @@ def test_forward_with_l1_equals_forward_then_l1(orc, size):
     assert np.array_equal(g_a.cpu().numpy(), want_g)
     assert abs(loss_a.item() - want_loss) <= 1e-12 * want_loss
     assert (nc > 0).float().mean().item() > 0.05
+
+
+@pytest.mark.parametrize("opaque", [False, True])
+def test_counted_forward_visits(opaque):
+    """gs_raster_fwd_counted: the same image, final_T and n_contrib as gs_raster_fwd,
+    and its counters in their bounds: the pairs the per-pixel loop visits lie
+    between sum(n_contrib) (a pixel visits at least up to its last blended entry) and
+    the sum over pixels of their tile's list length (reached when no pixel stops);
+    blended pairs <= visited pairs.  The opaque stack stops the pixels it covers
+    after a few entries, so they visit less than their lists."""
+    if opaque:
+        n = 600
+        rng = np.random.default_rng(4)
+        means = np.zeros((n, 3), np.float32)
+        means[:, :2] = 0.02 * rng.standard_normal((n, 2))
+        means[:, 2] = np.linspace(-1.0, 1.0, n)
+        scene = scenes.Scene(means, np.tile(np.float32([1, 0, 0, 0]), (n, 1)),
+                             np.full((n, 3), -1.0, np.float32), np.full(n, 4.0, np.float32),
+                             rng.uniform(0, 1, (n, 1, 3)).astype(np.float32), 0)
+        cam = scenes.tiny().cameras[0]
+    else:
+        wl = scenes.tiny()
+        scene, cam = wl.scene, wl.cameras[0]
+    run = CudaRun(scene, cam)
+    img, T, nc = (x.clone() for x in (run.view.image, run.view.final_T, run.view.n_contrib))
+    counts = torch.zeros(5, device="cuda", dtype=torch.int64)
+    pl.raster_fwd_counted(run.proj, run.view, counts)
+    torch.cuda.synchronize()
+    assert torch.equal(run.view.image, img) and torch.equal(run.view.final_T, T) and torch.equal(run.view.n_contrib, nc)
+    evaluated, blended, staged, reached, visited = counts.cpu().tolist()
+    W, H = cam["width"], cam["height"]
+    r = run.view.ranges.cpu().numpy().astype(np.int64)
+    lens = r[:, 1] - r[:, 0]
+    ys, xs = np.mgrid[0:H, 0:W]
+    tile = (ys // 16) * ((W + 15) // 16) + xs // 16
+    list_pairs = int(lens[tile].sum())
+    assert int(nc.sum().item()) <= visited <= list_pairs
+    assert blended <= visited
+    assert reached <= staged and blended <= evaluated
+    if opaque:
+        assert visited < list_pairs
+    with pytest.raises(ValueError):
+        pl.raster_fwd_counted(run.proj, run.view, torch.zeros(4, device="cuda", dtype=torch.int64))
