@@ -222,6 +222,18 @@ def test_workspace_grows_with_capacity(gs):
     assert b >= 12 * 1_000_000          # the ping-pong key/value copy
 
 
+def test_culled_binning_workspace(gs):
+    """The culled binning keeps, per Gaussian, the runs of its first 8 rows (32 bytes)
+    and its count (4 bytes): exactly that much more workspace, each region aligned to
+    256 bytes; a NULL camera means no culling."""
+    for n in (1, 1000, 1_000_000):
+        plain = gs.gs_bin_sort_workspace_bytes(n, 10 * n, gs.make_camera(cam()))
+        culled = gs.gs_bin_sort_workspace_bytes(n, 10 * n, gs.make_camera(cam(), tile_cull=True))
+        up = lambda x: (x + 255) // 256 * 256
+        assert culled - plain == up(32 * n) + up(4 * n), n
+        assert gs.lib().gs_bin_sort_workspace_bytes(n, 10 * n, None) == plain
+
+
 def test_binding_argument_counts_match_the_header(gs):
     """Every prototype of include/gs.h takes as many parameters as the ctypes binding
     passes (a missing or extra argument would be undefined behaviour at the call)."""
