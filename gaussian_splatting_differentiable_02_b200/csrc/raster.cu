@@ -607,19 +607,82 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
     if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
 }
 
+// The reverse pass's per-entry sums, taken in batches: each lane stashes its
+// kVals partial values of an entry in shared memory (slot s, column lane ^ swz(s)),
+// and once kSlots entries are stashed the warp sums them transposed: lanes
+// s * kL .. s * kL + kL - 1 (kL = 32 / kSlots) each add kSlots of the slot's 32
+// columns with float4 loads, two shuffle-add levels (kSlots = 8) finish the sums,
+// and the first of them adds the Gaussian's gradient records with one vector
+// atomic each.  Per entry that costs kVals shared stores and about two loads a
+// value, against a five-level shuffle reduce-scatter.  swz(s) = 4 (s & 1) keeps
+// the float4 loads of the two slots a wavefront serves on different banks.
+template <int kSlots, int kVals>
+struct EntrySums {
+    static constexpr int kL = 32 / kSlots;  // lanes that sum one slot
+    float v[kVals][kSlots * 32];
+    uint32_t gid[kSlots];
+};
+
+template <int kSlots, int kVals>
+__device__ __forceinline__ void stash_entry(EntrySums<kSlots, kVals>& R, int slot, int lane, uint32_t gid,
+                                            const float (&v)[kVals]) {
+    const int col = slot * 32 + (lane ^ (4 * (slot & 1)));
+#pragma unroll
+    for (int q = 0; q < kVals; ++q) R.v[q][col] = v[q];
+    if (lane == 0) R.gid[slot] = gid;
+}
+
+template <int kSlots, int kVals>
+__device__ __forceinline__ void flush_entries(const EntrySums<kSlots, kVals>& R, int count, int lane,
+                                              const BwdArgs& a) {
+    constexpr int kL = EntrySums<kSlots, kVals>::kL;
+    const int sl = lane / kL, part = lane % kL;
+    const int swz = 4 * (sl & 1);
+    float sum[kVals];
+#pragma unroll
+    for (int q = 0; q < kVals; ++q) {
+        float acc = 0.f;
+#pragma unroll
+        for (int g = 0; g < kSlots / 4; ++g) {
+            const float4 f =
+                *reinterpret_cast<const float4*>(&R.v[q][sl * 32 + ((part * kSlots + 4 * g) ^ swz)]);
+            acc += (f.x + f.y) + (f.z + f.w);
+        }
+        sum[q] = acc;
+    }
+#pragma unroll
+    for (int o = 1; o < kL; o <<= 1)
+#pragma unroll
+        for (int q = 0; q < kVals; ++q) sum[q] += __shfl_xor_sync(kFull, sum[q], o);
+    if (part == 0 && sl < count) {
+        const uint32_t gid = R.gid[sl];
+        atomicAdd(a.g_xy + gid, make_float2(sum[0], sum[1]));
+        atomicAdd(a.g_con + gid, make_float4(sum[2], sum[3], sum[4], sum[5]));
+        atomicAdd(a.g_rgb + gid, make_float4(sum[6], sum[7], sum[8], 0.f));
+        if (kVals > 9) atomicAdd(a.g_xy_abs + gid, make_float2(sum[9], sum[kVals > 9 ? 10 : 0]));
+    }
+}
+
 // kBg: the background is not black.  With a black one (every workload here) the
 // background term of dL/dalpha is 0 and neither it nor its per-pixel factor is
 // formed, which saves a paired instruction per pixel pair and eight registers.
 template <int PX, bool kAbs, bool kCount, bool kBg>
 __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster_bwd_kernel(const BwdArgs a) {
     constexpr int kPx = PX, kPairs = Layout<PX>::kPairs, kBoxH = Layout<PX>::kBoxH, kSub = Layout<PX>::kSub;
+    // entries summed per batch: 8 with one warp per tile, 4 with two (whose 20 blocks
+    // an SM the larger stash would not let fit in shared memory)
+    constexpr int kSlots = PX == 8 ? 8 : 4;
+    constexpr int kVals = kAbs ? 11 : 9;
     __shared__ WarpStage stage[kWarps];
+    __shared__ __align__(16) EntrySums<kSlots, kVals> sums[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + warp;
     const int slot = gw / kSub, sub = gw % kSub;
     if (slot >= a.tiles) return;
     const int tile = a.order ? int(__ldg(a.order + slot)) : slot;  // longest lists first when ordered
     WarpStage& S = stage[warp];
+    EntrySums<kSlots, kVals>& R = sums[warp];
+    int stashed = 0;  // entries in R not yet added (the same in every lane)
     const int xb = (tile % a.TX) * kTile;  // this warp's pixel box
     const int yb = (tile / a.TX) * kTile + sub * kBoxH;
     const int x = xb + lane % kBoxW;
@@ -763,16 +826,26 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
                         }
                     }
                 }
-                float v[8] = {du, dv, 0.5f * r.dx * r.dx * s0, r.dx * m1, 0.5f * (s2.x + s2.y), mo * pa.w,
-                              -(ndr.x + ndr.y), -(ndg.x + ndg.y)};
-                warp_reduce_and_add(v, -(ndb.x + ndb.y), lane, S.gid[buf][j], a);
+                float v[kVals];
+                v[0] = du;
+                v[1] = dv;
+                v[2] = 0.5f * r.dx * r.dx * s0;
+                v[3] = r.dx * m1;
+                v[4] = 0.5f * (s2.x + s2.y);
+                v[5] = mo * pa.w;
+                v[6] = -(ndr.x + ndr.y);
+                v[7] = -(ndg.x + ndg.y);
+                v[8] = -(ndb.x + ndb.y);
                 if (kAbs) {
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        au += __shfl_xor_sync(kFull, au, o);
-                        av += __shfl_xor_sync(kFull, av, o);
-                    }
-                    if (lane == 3) atomicAdd(a.g_xy_abs + S.gid[buf][j], make_float2(au, av));
+                    v[kAbs ? 9 : 0] = au;
+                    v[kAbs ? 10 : 0] = av;
+                }
+                stash_entry(R, stashed, lane, S.gid[buf][j], v);
+                if (++stashed == kSlots) {
+                    __syncwarp();
+                    flush_entries(R, kSlots, lane, a);
+                    __syncwarp();
+                    stashed = 0;
                 }
             };
             if (ij & kMayClampBit)
@@ -783,6 +856,10 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
         __syncwarp();
     }
     cp_async_wait_all();
+    if (stashed) {
+        __syncwarp();
+        flush_entries(R, stashed, lane, a);
+    }
     if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
 }
 
@@ -893,6 +970,19 @@ cudaError_t launch_raster_fwd(const gs_projected& proj, const uint32_t* vals, co
 namespace {
 template <int PX, bool kBg>
 void launch_raster_bwd_bg(const BwdArgs& a, bool counted, cudaStream_t s) {
+    // the reverse pass keeps its entry sums in shared memory: ask for the largest
+    // shared-memory carveout, so that its blocks an SM are set by registers alone
+    static const bool carveout = [] {
+        const int c = cudaSharedmemCarveoutMaxShared;
+        const cudaFuncAttribute at = cudaFuncAttributePreferredSharedMemoryCarveout;
+        bool ok = cudaFuncSetAttribute(raster_bwd_kernel<PX, false, false, kBg>, at, c) == cudaSuccess;
+        ok = cudaFuncSetAttribute(raster_bwd_kernel<PX, true, false, kBg>, at, c) == cudaSuccess && ok;
+        ok = cudaFuncSetAttribute(raster_bwd_kernel<PX, false, true, kBg>, at, c) == cudaSuccess && ok;
+        ok = cudaFuncSetAttribute(raster_bwd_kernel<PX, true, true, kBg>, at, c) == cudaSuccess && ok;
+        if (!ok) cudaGetLastError();  // a hint only: a refusal leaves the default carveout
+        return ok;
+    }();
+    (void)carveout;
     const unsigned grid = unsigned(a.tiles * Layout<PX>::kSub);
     if (counted) {
         if (a.g_xy_abs)
