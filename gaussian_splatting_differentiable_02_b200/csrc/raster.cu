@@ -608,33 +608,43 @@ __device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int
 }
 
 // The reverse pass's per-entry sums, taken in batches: each lane stashes its
-// kVals partial values of an entry in shared memory (slot s, column lane ^ swz(s)),
-// and once kSlots entries are stashed the warp sums them transposed: lanes
-// s * kL .. s * kL + kL - 1 (kL = 32 / kSlots) each add kSlots of the slot's 32
-// columns with float4 loads, two shuffle-add levels (kSlots = 8) finish the sums,
-// and the first of them adds the Gaussian's gradient records with one vector
-// atomic each.  Per entry that costs kVals shared stores and about two loads a
-// value, against a five-level shuffle reduce-scatter.  swz(s) = 4 (s & 1) keeps
-// the float4 loads of the two slots a wavefront serves on different banks.
+// kVals partial moments of an entry in shared memory (slot s, column
+// lane ^ swz(s)), and once kSlots entries are stashed the warp sums them
+// transposed: lanes s * kL .. s * kL + kL - 1 (kL = 32 / kSlots) each add kSlots
+// of the slot's 32 columns with float4 loads, two shuffle-add levels (kSlots = 8)
+// finish the sums, and the first of them turns the slot's moments into the
+// Gaussian's gradients (with the entry's conic, read from the batch's staging)
+// and adds them with one vector atomic per record.  The slots are emptied at the
+// end of every batch, while its staged entries are still in place.  Per entry that costs kVals shared stores
+// and about two loads a value, against a five-level shuffle reduce-scatter, and
+// the conic algebra runs once per entry instead of in every lane.
+// swz(s) = 4 (s & 1) keeps the float4 loads of the two slots a wavefront serves
+// on different banks.
+//
+// The moments, per lane (sums over its pixels of q = dL/dsigma times): X = dx s0
+// (or, for an entry evaluated in the factored form, sum q t), s1 = sum q dy,
+// dx^2 s0, dx s1, sum q dy^2, s0 = sum q, and the colour sums; with them
+// dL/du = A X + B s1 (factored: A X), dL/dv = B X + C s1 (factored: B X + D s1),
+// dL/dA = dx^2 s0 / 2, dL/dB = dx s1, dL/dC = sum q dy^2 / 2, dL/do = -s0 / o.
 template <int kSlots, int kVals>
 struct EntrySums {
     static constexpr int kL = 32 / kSlots;  // lanes that sum one slot
     float v[kVals][kSlots * 32];
-    uint32_t gid[kSlots];
+    int e[kSlots];  // the slot's entry: its index among the batch's compacted entries
 };
 
 template <int kSlots, int kVals>
-__device__ __forceinline__ void stash_entry(EntrySums<kSlots, kVals>& R, int slot, int lane, uint32_t gid,
+__device__ __forceinline__ void stash_entry(EntrySums<kSlots, kVals>& R, int slot, int lane, int e,
                                             const float (&v)[kVals]) {
     const int col = slot * 32 + (lane ^ (4 * (slot & 1)));
 #pragma unroll
     for (int q = 0; q < kVals; ++q) R.v[q][col] = v[q];
-    if (lane == 0) R.gid[slot] = gid;
+    if (lane == 0) R.e[slot] = e;
 }
 
 template <int kSlots, int kVals>
-__device__ __forceinline__ void flush_entries(const EntrySums<kSlots, kVals>& R, int count, int lane,
-                                              const BwdArgs& a) {
+__device__ __forceinline__ void flush_entries(const EntrySums<kSlots, kVals>& R, const WarpStage& S, int buf,
+                                              int count, int lane, const BwdArgs& a) {
     constexpr int kL = EntrySums<kSlots, kVals>::kL;
     const int sl = lane / kL, part = lane % kL;
     const int swz = 4 * (sl & 1);
@@ -655,10 +665,18 @@ __device__ __forceinline__ void flush_entries(const EntrySums<kSlots, kVals>& R,
 #pragma unroll
         for (int q = 0; q < kVals; ++q) sum[q] += __shfl_xor_sync(kFull, sum[q], o);
     if (part == 0 && sl < count) {
-        const uint32_t gid = R.gid[sl];
-        atomicAdd(a.g_xy + gid, make_float2(sum[0], sum[1]));
-        atomicAdd(a.g_con + gid, make_float4(sum[2], sum[3], sum[4], sum[5]));
-        atomicAdd(a.g_rgb + gid, make_float4(sum[6], sum[7], sum[8], 0.f));
+        const int e = R.e[sl];
+        const int j = S.idx[e] & (kBatch - 1);
+        const uint32_t gid = S.gid[buf][j];
+        const float4 con = S.con[buf][j];
+        const float4 pb = S.pb[e];
+        // plain: dL/du = A X + B s1, dL/dv = B X + C s1; factored: A X, B X + D s1
+        const bool factored = pb.w >= kFactored;
+        const float du = fmaf(con.x, sum[0], factored ? 0.f : con.y * sum[1]);
+        const float dv = fmaf(con.y, sum[0], (factored ? pb.z : con.z) * sum[1]);
+        atomicAdd(a.g_xy + gid, make_float2(du, dv));
+        atomicAdd(a.g_con + gid, make_float4(0.5f * sum[2], sum[3], 0.5f * sum[4], -sum[5] * S.pa[e].w));
+        atomicAdd(a.g_rgb + gid, make_float4(-sum[6], -sum[7], -sum[8], 0.f));
         if (kVals > 9) atomicAdd(a.g_xy_abs + gid, make_float2(sum[9], sum[kVals > 9 ? 10 : 0]));
     }
 }
@@ -791,17 +809,16 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
                 // no vote on whether any pixel took the entry: 9 in 10 entries that reach
                 // the box take a gradient somewhere in it, and the test costs more than the
                 // reductions of zeros it would save
-                const float s0 = nmo.x + nmo.y, mo = -s0, m1 = s1.x + s1.y;
-                float du, dv;
+                const float s0 = nmo.x + nmo.y, m1 = s1.x + s1.y;
+                const float dxs0 = r.dx * s0;
+                float X;  // dx s0, or sum q t in the factored form
                 float au = 0.f, av = 0.f;  // absgrad: sums of |per-pixel dL/du|, |per-pixel dL/dv|
                 if (pb.w >= kFactored) {
                     // dsigma/du = A t, dsigma/dv = B t + D dy
                     f2 st = zero;
 #pragma unroll
                     for (int p = 0; p < kPairs; ++p) st = fma2(nm[p], r.t[p], st);
-                    const float stt = st.x + st.y;
-                    du = con.x * stt;
-                    dv = fmaf(con.y, stt, pb.z * m1);
+                    X = st.x + st.y;
                     if (kAbs) {
 #pragma unroll
                         for (int p = 0; p < kPairs; ++p) {
@@ -812,8 +829,7 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
                         }
                     }
                 } else {
-                    du = fmaf(con.x * r.dx, s0, con.y * m1);
-                    dv = fmaf(con.y * r.dx, s0, con.z * m1);
+                    X = dxs0;
                     if (kAbs) {
                         // per pixel dsigma/du = A dx + B dy, dsigma/dv = B dx + C dy
                         const f2 adx = splat(con.x * r.dx), bdx = splat(con.y * r.dx);
@@ -827,23 +843,23 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
                     }
                 }
                 float v[kVals];
-                v[0] = du;
-                v[1] = dv;
-                v[2] = 0.5f * r.dx * r.dx * s0;
+                v[0] = X;
+                v[1] = m1;
+                v[2] = r.dx * dxs0;
                 v[3] = r.dx * m1;
-                v[4] = 0.5f * (s2.x + s2.y);
-                v[5] = mo * pa.w;
-                v[6] = -(ndr.x + ndr.y);
-                v[7] = -(ndg.x + ndg.y);
-                v[8] = -(ndb.x + ndb.y);
+                v[4] = s2.x + s2.y;
+                v[5] = s0;
+                v[6] = ndr.x + ndr.y;
+                v[7] = ndg.x + ndg.y;
+                v[8] = ndb.x + ndb.y;
                 if (kAbs) {
                     v[kAbs ? 9 : 0] = au;
                     v[kAbs ? 10 : 0] = av;
                 }
-                stash_entry(R, stashed, lane, S.gid[buf][j], v);
+                stash_entry(R, stashed, lane, e, v);
                 if (++stashed == kSlots) {
                     __syncwarp();
-                    flush_entries(R, kSlots, lane, a);
+                    flush_entries(R, S, buf, kSlots, lane, a);
                     __syncwarp();
                     stashed = 0;
                 }
@@ -853,13 +869,14 @@ __global__ void __launch_bounds__(kWarps * 32, Layout<PX>::kBwdMinBlocks) raster
             else
                 entry(std::false_type{});
         }
+        if (stashed) {  // the batch's last entries, while its staging is in place
+            __syncwarp();
+            flush_entries(R, S, buf, stashed, lane, a);
+            stashed = 0;
+        }
         __syncwarp();
     }
     cp_async_wait_all();
-    if (stashed) {
-        __syncwarp();
-        flush_entries(R, stashed, lane, a);
-    }
     if (kCount) add_counts(a.counts, c_eval, c_work, c_staged, lane, 32 * kPx);
 }
 
