@@ -190,7 +190,8 @@ gs_status gs_project_views(const gs_params* params, int32_t num_views, const gs_
 size_t gs_bin_sort_workspace_bytes(int64_t n, int64_t capacity, const gs_camera* cam);
 
 /* gs_bin_sort -- tile binning.  Every visible Gaussian emits one instance per tile
- * of its rectangle, key = (ty * tiles_x + tx) << 32 | float32 bits of its depth,
+ * of its rectangle (with the camera's tile_cull, per tile of the rectangle that its
+ * footprint reaches: gs_camera), key = (ty * tiles_x + tx) << 32 | float32 bits of its depth,
  * value = Gaussian index; the instances are sorted by key, equal keys keeping
  * ascending Gaussian index, and tile_ranges[2t], [2t+1] receive the [begin, end)
  * of tile t in the sorted list ([0, 0) when empty).  Method: a stable LSD radix
