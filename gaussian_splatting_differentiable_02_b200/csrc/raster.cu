@@ -560,53 +560,6 @@ struct BwdArgs {
     unsigned long long* counts;  // kCount only: work counters (gs_raster_bwd_counted)
 };
 
-// Sum 9 per-lane values over the warp and add them to the Gaussian's three
-// gradient records with one vector atomic each (lanes 0, 1, 2).
-__device__ __forceinline__ void warp_reduce_and_add(float (&v)[8], float v8, int lane, uint32_t gid,
-                                                    const BwdArgs& a) {
-    // reduce-scatter of 8 values: after it, lanes 4k..4k+3 hold the total of value k
-    {
-        const bool hi = (lane >> 4) & 1;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float send = hi ? v[k] : v[k + 4];
-            const float keep = hi ? v[k + 4] : v[k];
-            v[k] = keep + __shfl_xor_sync(kFull, send, 16);
-        }
-    }
-    {
-        const bool hi = (lane >> 3) & 1;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const float send = hi ? v[k] : v[k + 2];
-            const float keep = hi ? v[k + 2] : v[k];
-            v[k] = keep + __shfl_xor_sync(kFull, send, 8);
-        }
-    }
-    {
-        const bool hi = (lane >> 2) & 1;
-        const float send = hi ? v[0] : v[1];
-        const float keep = hi ? v[1] : v[0];
-        v[0] = keep + __shfl_xor_sync(kFull, send, 4);
-    }
-    v[0] += __shfl_xor_sync(kFull, v[0], 2);
-    v[0] += __shfl_xor_sync(kFull, v[0], 1);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v8 += __shfl_xor_sync(kFull, v8, o);
-    // gather: lane 0 <- values 0,1 (du, dv); lane 1 <- 2..5 (dA, dB, dC, do); lane 2 <- 6,7 (dr, dg) + v8 (db)
-    const int i0 = lane == 0 ? 0 : (lane == 1 ? 2 : 6);
-    const int i1 = i0 + 1;
-    const int i2 = lane == 1 ? 4 : 0;
-    const int i3 = lane == 1 ? 5 : 0;
-    const float f0 = __shfl_sync(kFull, v[0], 4 * i0);
-    const float f1 = __shfl_sync(kFull, v[0], 4 * i1);
-    const float f2 = __shfl_sync(kFull, v[0], 4 * i2);
-    const float f3 = __shfl_sync(kFull, v[0], 4 * i3);
-    if (lane == 0) atomicAdd(a.g_xy + gid, make_float2(f0, f1));
-    if (lane == 1) atomicAdd(a.g_con + gid, make_float4(f0, f1, f2, f3));
-    if (lane == 2) atomicAdd(a.g_rgb + gid, make_float4(f0, f1, v8, 0.f));
-}
-
 // The reverse pass's per-entry sums, taken in batches: each lane stashes its
 // kVals partial moments of an entry in shared memory (slot s, column
 // lane ^ swz(s)), and once kSlots entries are stashed the warp sums them
