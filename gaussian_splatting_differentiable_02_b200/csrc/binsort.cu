@@ -50,7 +50,7 @@ static_assert((kEmitChunk & (kEmitChunk - 1)) == 0, "the emit binary search halv
 // emission (32 bytes a Gaussian; 96% of the 1080p instances of the 1M mixture
 // belong to Gaussians of at most 8 rows)
 constexpr int kRunRows = 8;
-static_assert(kRunRows % 4 == 0, "runs move as uint4");
+static_assert(kRunRows % 4 == 0, "the emission loads runs as uint4");
 
 #ifndef GS_SORT_ITEMS
 #define GS_SORT_ITEMS 8
@@ -314,7 +314,7 @@ struct EmitArgs {
 // Gaussians, in halves of one Gaussian per thread: each thread sets up its
 // Gaussian's footprint bound (tile_reach.cuh) in shared memory, a block scan
 // numbers the rows of all the half's rectangles, and the block's threads then
-// take those rows round-robin (a warp no longer waits for its tallest
+// take those rows round-robin (so that no warp waits on its tallest
 // Gaussian's rows), adding each row's run length to its Gaussian's count in
 // shared memory and writing the runs of the first kRunRows rows as (first
 // column << 16 | length) for the emission.  A Gaussian whose conic is not
