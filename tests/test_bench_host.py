@@ -105,6 +105,14 @@ def test_raster_roofline_counts_the_method_work():
     f = bench.raster_roofline("raster_fwd", 1.0, work, alu)
     assert abs(f["achieved"] - (14 * 1e9 + 8 * 4e8) / 1e-3 / 1e12) < 1e-9
     assert abs(f["sfu"]["achieved_tops"] - 2e9 / 1e-3 / 1e12) < 1e-9
+    # with the counted forward's fifth counter the forward charges the pairs its
+    # per-pixel loop visits (up to each pixel's stop); the reverse pass keeps sum(n_contrib)
+    work["fwd_visited_pairs"] = 1.25e9
+    f = bench.raster_roofline("raster_fwd", 1.0, work, alu)
+    assert abs(f["achieved"] - (14 * 1.25e9 + 8 * 4e8) / 1e-3 / 1e12) < 1e-9
+    assert abs(f["evaluated_over_visited"] - 2e9 / 1.25e9) < 1e-12
+    r = bench.raster_roofline("raster_bwd", 2.0, work, alu)
+    assert abs(r["achieved"] - (14 * 1e9 + 46 * 4e8) / 2e-3 / 1e12) < 1e-9
 
 
 def test_cpu_baseline_times_all_cores_and_one_thread():
