@@ -6,10 +6,11 @@
 // Work decomposition: one warp per pixel box of a tile, one warp per block, blocks
 // launched in the tile order of gs_tile_order when one is given; each lane owns a
 // column segment of PX pixels (lane & 15 selects the column, lane >> 4 the upper
-// or lower half of the box).  Large tile grids take PX = 8, a box per tile, so
-// that the per-entry work of the warp (its shared-memory reads, the gradient
-// reduction, the branches) is spread over 256 pixels; small grids PX = 4, two
-// boxes per tile, for twice the warps (Layout below).  The warp walks its
+// or lower half of the box).  The backward on large tile grids takes PX = 8, a
+// box per tile, so that the per-entry work of the warp (its shared-memory reads,
+// the gradient sums, the branches) is spread over 256 pixels, on small grids
+// PX = 4, two boxes per tile, for twice the warps; the forward takes PX = 4 on
+// every grid (Layout below).  The warp walks its
 // tile's sorted list in batches of 32 entries: every lane gathers one entry's
 // 40 bytes (xy, conic + opacity, colour) by Gaussian index into shared memory
 // with cp.async, double-buffered so the next batch is in flight while the
@@ -28,12 +29,12 @@
 // per entry).  Backward: back to front from the largest n_contrib of the box,
 // the transmittance in front of each entry recovered with rcp(1 - alpha) and
 // g . S (S the colour blended behind) tracked per pixel; each lane sums its
-// pixels' contributions, the 9 per-Gaussian sums are reduce-scattered across
-// the warp (18 shuffles) and three lanes issue one float2 / float4 atomic add
-// each (batched atomics, MUSA co-design article qwbw.cn/news/278220 §2.2).  The
-// gradient with respect to (u, v, A, B, C) is accumulated as moments of
-// dL/dsigma over the lane's pixels, then combined with dx and the conic once
-// per entry.
+// pixels' contributions as 9 moments of the entry (dL/dsigma against 1, dx,
+// dy, ... and the colour terms), stashes them in shared memory, and every 8
+// entries the warp adds the stashed moments up across its lanes, turns each
+// entry's sums into its Gaussian's gradients with the entry's conic, and one
+// lane per entry issues a float2 and two float4 atomic adds (batched atomics,
+// MUSA co-design article qwbw.cn/news/278220 §2.2; EntrySums below).
 //
 // Both passes evaluate alpha with the same inline code built from explicit
 // rounding intrinsics, so the backward pass repeats the forward pass's skip and
