@@ -88,3 +88,25 @@ def test_view_set_n_keeps_or_grows_the_instance_buffers():
     assert view.workspace.numel() >= ws
     from gaussian_splatting_differentiable_02_b200 import abi
     assert view.workspace.numel() >= abi.gs_bin_sort_workspace_bytes(3000, 12000, view.gcam)
+
+
+@pytest.mark.parametrize("cull", [True, False])
+def test_tile_cull_reaches_every_view_and_its_workspace(cull):
+    """Trainer(tile_cull=...) sets the flag in every view's camera and grows each view's
+    sort workspace to what the culled binning needs (its runs and counts); set_n after
+    densification keeps sizing it for the flag."""
+    from gaussian_splatting_differentiable_02_b200 import abi
+    tr = _trainer(3, n=400, tile_cull=cull)
+    for vw in tr.views:
+        assert vw.tile_cull is cull and vw.gcam.tile_cull == int(cull)
+        need = abi.gs_bin_sort_workspace_bytes(vw.n, vw.capacity, vw.gcam)
+        assert vw.workspace.numel() >= need
+    plain = abi.gs_bin_sort_workspace_bytes(400, tr.views[0].capacity, abi.make_camera(tr.views[0].cam))
+    culled = abi.gs_bin_sort_workspace_bytes(400, tr.views[0].capacity, abi.make_camera(tr.views[0].cam, True))
+    assert culled > plain
+    vw = tr.views[0]
+    vw.set_n(900)
+    assert vw.workspace.numel() >= abi.gs_bin_sort_workspace_bytes(900, vw.capacity, vw.gcam)
+    # set_camera keeps the flag
+    vw.set_camera(dict(vw.cam))
+    assert vw.gcam.tile_cull == int(cull)
