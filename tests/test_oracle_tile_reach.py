@@ -167,3 +167,34 @@ def test_culled_list_checks_accept_valid_and_reject_broken_lists():
     swapped_v[[3, 4]] = swapped_v[[4, 3]]
     with pytest.raises(AssertionError):
         check_culled_binning(swapped_k, swapped_v, _ranges_of(gk, tx * ty), ref, keys, vals, tx, ty)
+
+
+def test_every_blending_pixel_lies_in_a_must_keep_instance():
+    """Against the compositing rule itself: for every instance of the tiny workload's
+    rectangle binning and every pixel centre of its tile, alpha = o e^-sigma >= 1/255
+    there implies the instance is one the culled binning must keep; and an instance the
+    rule lets go has alpha below 1/255 at all of its tile's pixel centres."""
+    from gaussian_splatting_differentiable_02_b200 import scenes
+    wl = scenes.tiny()
+    cam = wl.cameras[0]
+    ref = orc.project(wl.scene, cam)
+    keys, vals, _ = orc.keys(ref, cam)
+    tx, _ = orc.tiles(cam)
+    keep, drop = orc.tile_reach_classes(ref, keys, vals, tx)
+    gid = vals.astype(np.int64)
+    tile = (keys >> np.uint64(32)).astype(np.int64)
+    u, v = ref["xy"][gid].T
+    A, B, C = ref["conic"][gid].T
+    o = ref["opacity"][gid]
+    px = 16.0 * (tile % tx)[:, None] + np.arange(16)[None, :] + 0.5        # [K, 16]
+    py = 16.0 * (tile // tx)[:, None] + np.arange(16)[None, :] + 0.5
+    dx = px[:, None, :] - u[:, None, None]                                  # [K, 16 rows, 16 cols]
+    dy = py[:, :, None] - v[:, None, None]
+    sig = 0.5 * (A[:, None, None] * dx * dx + C[:, None, None] * dy * dy) + B[:, None, None] * dx * dy
+    alpha_max = (o[:, None, None] * np.exp(-sig)).reshape(len(gid), -1).max(axis=1)
+    blends = alpha_max >= 1.0 / 255.0
+    assert blends.sum() > 1000
+    assert keep[blends].all()
+    assert (alpha_max[drop] < 1.0 / 255.0).all()
+    # the culling is worth having: many instances reach no pixel
+    assert (~blends).sum() > 0.2 * len(gid)
