@@ -210,7 +210,9 @@ class View:
 
     def set_tile_cull(self, on: bool):
         """Bin each Gaussian only into the tiles of its rectangle that its footprint
-        reaches (gs_camera.tile_cull), or into the whole rectangle."""
+        reaches (gs_camera.tile_cull), or into the whole rectangle.  The workspace may
+        be reallocated: for the views of a Trainer use Trainer.set_tile_cull, which
+        also drops a captured CUDA graph."""
         self.tile_cull = bool(on)
         self.gcam = abi.make_camera(self.cam, self.tile_cull)
         nbytes = abi.gs_bin_sort_workspace_bytes(self.n, self.capacity, self.gcam)   # the culled binning's runs
@@ -604,6 +606,15 @@ class Trainer:
         self.grad2d = self.grad2ds[0]
         for view in self.views:
             view.set_n(self.pcap)
+
+    def set_tile_cull(self, on: bool):
+        """Switch every view between the culled binning and the rectangles; a captured
+        CUDA graph holds the old camera flags and workspace addresses, so it is dropped
+        and the next step captures again."""
+        self.tile_cull = bool(on)
+        for vw in self.views:
+            vw.set_tile_cull(self.tile_cull)
+        self._graph = None
 
     def view_groups(self) -> list:
         """The consecutive groups of view indices the batched path projects, sorts and bins together."""

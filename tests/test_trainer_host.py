@@ -110,3 +110,11 @@ def test_tile_cull_reaches_every_view_and_its_workspace(cull):
     # set_camera keeps the flag
     vw.set_camera(dict(vw.cam))
     assert vw.gcam.tile_cull == int(cull)
+
+
+def test_trainer_set_tile_cull_switches_views_and_drops_the_graph():
+    tr = _trainer(3, n=300, tile_cull=True)
+    tr._graph = object()   # stands for a captured graph
+    tr.set_tile_cull(False)
+    assert tr._graph is None and tr.tile_cull is False
+    assert all(not vw.tile_cull and vw.gcam.tile_cull == 0 for vw in tr.views)
