@@ -537,7 +537,9 @@ class Trainer:
                                # losses and their backward) is captured once into a CUDA graph and
                                # replayed every step, so its few-microsecond launches cost no host time
                                # and little device time between them; recaptured whenever a buffer it
-                               # uses is reallocated (instance or slot growth, densification)
+                               # uses is reallocated (instance or slot growth, densification); the
+                               # cameras and target tensors are those seen at capture, so after
+                               # View.set_camera or new targets call drop_graph()
 
     def __post_init__(self):
         n = self.gauss.n
@@ -614,6 +616,11 @@ class Trainer:
         self.tile_cull = bool(on)
         for vw in self.views:
             vw.set_tile_cull(self.tile_cull)
+        self.drop_graph()
+
+    def drop_graph(self):
+        """Forget the captured CUDA graph (graph=True): the next step captures the views'
+        part again with the current cameras, targets and buffers."""
         self._graph = None
 
     def view_groups(self) -> list:
